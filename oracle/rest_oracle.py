@@ -1,0 +1,282 @@
+"""fp64 CPU oracle of the ReST encode-once / decode-many ranking forward.
+
+TEST INFRASTRUCTURE ONLY. This module is the slow, plain statement of what
+the CUDA path must compute. Only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may import it; the library never does, and the
+library shares no code with it.
+
+Every function follows the ReST paper as read on the page "From Language to
+Behavior" (paper-archivist close reading of arXiv 2609.01240); the section
+and equation numbers below are that page's. Where the page leaves a detail
+open the reading taken is stated in the docstring (the same readings are
+fixed in the repository's written specification).
+
+Everything is float64; inputs (bf16 or fp32 values) are upcast exactly.
+Matrix products use numpy's matmul as a library primitive; there is no
+fusion or reordering beyond the definitions.
+
+Pins (tests/test_oracle_pins.py): every public function is checked against
+something other than itself -- a literal loop implementation with explicit
+rotation matrices (oracle/brute.py) on tiny inputs, torch's fp64
+scaled_dot_product_attention and layer_norm, closed forms (first causal row,
+cutoff 1, alpha 0), and the invariants the page states (relative position and
+relative time, eq. 14; causality; candidate permutation; shared-prefix
+reuse, §3.5).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+LN_EPS = 1e-5
+
+
+class UnsortedTimestamps(ValueError):
+    pass
+
+
+# --------------------------------------------------------------------------
+# §3.2.2: rotation index (RoPE position or RoTE time bucket) and angles
+# --------------------------------------------------------------------------
+
+def rotation_index(ts: np.ndarray, cu_seqlens: np.ndarray, taus: np.ndarray,
+                   time_origin: Optional[Sequence[int]] = None,
+                   pos_offset: int = 0) -> np.ndarray:
+    """Per (token, head) rotation index, int64 [T, n_heads].
+
+    §3.2.2: RoPE heads (tau_h = 0) use the ordinal position; RoTE heads use
+    the bucket b_i = floor((t_i - t_1) / tau_h), t_1 the first timestamp of
+    the user's sequence. Reading: positions are 0-based within each user.
+
+    ``time_origin`` (per user) replaces t_1 and ``pos_offset`` shifts every
+    position; both exist only so the tests can check the invariances of
+    eq. 14 and are not part of the method.
+    """
+    ts = np.asarray(ts, dtype=np.int64)
+    T = ts.shape[0]
+    H = len(taus)
+    idx = np.zeros((T, H), dtype=np.int64)
+    for u in range(len(cu_seqlens) - 1):
+        s, e = int(cu_seqlens[u]), int(cu_seqlens[u + 1])
+        if e <= s:
+            continue
+        t = ts[s:e]
+        if np.any(t[1:] < t[:-1]):
+            raise UnsortedTimestamps(f"user {u}: timestamps decrease")
+        origin = t[0] if time_origin is None else np.int64(time_origin[u])
+        rel = t - origin                                    # exact int64
+        for h, tau in enumerate(taus):
+            if tau == 0:
+                idx[s:e, h] = np.arange(e - s, dtype=np.int64) + pos_offset
+            else:
+                idx[s:e, h] = np.floor_divide(rel, np.int64(tau))
+    return idx
+
+
+def frequencies(head_dim: int, rope_base: float) -> np.ndarray:
+    """theta_j = base^(-2j/d_h), j = 0..d_h/2-1 (RoPE's schedule; §3.2.2 says
+    RoPE and RoTE share one rotation mechanism, so RoTE heads use it too)."""
+    j = np.arange(head_dim // 2, dtype=np.float64)
+    return np.power(np.float64(rope_base), -2.0 * j / head_dim)
+
+
+def rotation_angles(idx: np.ndarray, head_dim: int, rope_base: float,
+                    angle_scale: float = 1.0) -> np.ndarray:
+    """phi[i, h, j] = idx[i, h] * theta_j in fp64 (eq. 5's R_Theta(idx)).
+
+    ``angle_scale`` = 0 turns every rotation into the identity (test knob).
+    """
+    return idx.astype(np.float64)[:, :, None] * frequencies(head_dim, rope_base)[None, None, :] * angle_scale
+
+
+def rotate(v: np.ndarray, phi: np.ndarray) -> np.ndarray:
+    """Apply the block-diagonal R_Theta per head to rows of v [T, H*d_h].
+
+    Reading: 2x2 blocks on the column pairs (2j, 2j+1) of each head,
+    (a, b) -> (a cos phi - b sin phi, a sin phi + b cos phi).
+    """
+    T, H, half = phi.shape
+    x = v.reshape(T, H, half, 2)
+    a, b = x[..., 0], x[..., 1]
+    c, s = np.cos(phi), np.sin(phi)
+    out = np.empty_like(x)
+    out[..., 0] = a * c - b * s
+    out[..., 1] = a * s + b * c
+    return out.reshape(T, H * half * 2)
+
+
+# --------------------------------------------------------------------------
+# elementwise pieces
+# --------------------------------------------------------------------------
+
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    """Bounded sigmoid gate (§3.2.1: sigmoid instead of HSTU's SiLU gate)."""
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def silu(z: np.ndarray) -> np.ndarray:
+    """SiLU(z) = z * sigmoid(z), the SwiGLU activation of the LLaMA block (§3.2)."""
+    return z * sigmoid(z)
+
+
+def layer_norm(v: np.ndarray, g: np.ndarray, b: np.ndarray, eps: float = LN_EPS) -> np.ndarray:
+    """LN over the last axis with the biased variance (eq. 6's LN)."""
+    mu = v.mean(axis=-1, keepdims=True)
+    var = ((v - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (v - mu) / np.sqrt(var + eps) * g.astype(np.float64) + b.astype(np.float64)
+
+
+def softmax_rows(S: np.ndarray) -> np.ndarray:
+    """Row softmax with the row maximum subtracted; -inf entries give 0."""
+    m = S.max(axis=-1, keepdims=True)
+    E = np.exp(S - m)
+    return E / E.sum(axis=-1, keepdims=True)
+
+
+# --------------------------------------------------------------------------
+# §3.2.1: Dual-Gated Attention
+# --------------------------------------------------------------------------
+
+def causal_attention_probs(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
+    """P = softmax(q k^T * scale + M_causal) for one sequence and one head (eq. 3)."""
+    L = q.shape[0]
+    S = (q @ k.T) * scale
+    S[np.triu_indices(L, 1)] = -np.inf
+    return softmax_rows(S)
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def dga_sublayer(y: np.ndarray, phi: np.ndarray, cu_seqlens: np.ndarray, layer: dict,
+                 n_heads: int, gates: bool = True, row_chunk: int = 2048) -> np.ndarray:
+    """Eqs. 3-5: (Attention(R q, R k, sigmoid(y W_gv) * y W_V) * sigmoid(y W_go)) W_o.
+
+    Readings: no biases; the gates are full d x d projections applied
+    elementwise; head h owns columns h*d_h..(h+1)*d_h-1; the score scale is
+    1/sqrt(d_h) (eq. 7's multi-head form; eq. 3 is written single-head).
+    ``gates=False`` replaces both sigmoids by 1 (test knob).
+    """
+    T, d = y.shape
+    hd = d // n_heads
+    W = _f64(layer["w_qkvgg"])
+    P5 = y @ W
+    Q, Kx, V, Gv, Go = (P5[:, i * d:(i + 1) * d] for i in range(5))
+    Vg = V * sigmoid(Gv) if gates else V
+    Qr, Kr = rotate(Q, phi), rotate(Kx, phi)
+    O = np.zeros((T, d))
+    scale = 1.0 / math.sqrt(hd)
+    for u in range(len(cu_seqlens) - 1):
+        s, e = int(cu_seqlens[u]), int(cu_seqlens[u + 1])
+        L = e - s
+        for h in range(n_heads):
+            cols = slice(h * hd, (h + 1) * hd)
+            q, k, v = Qr[s:e, cols], Kr[s:e, cols], Vg[s:e, cols]
+            for r0 in range(0, L, row_chunk):
+                r1 = min(L, r0 + row_chunk)
+                # rows r0..r1-1 see keys 0..r1-1 at most (j <= i)
+                S = (q[r0:r1] @ k[:r1].T) * scale
+                ii = np.arange(r0, r1)[:, None]
+                jj = np.arange(r1)[None, :]
+                S[jj > ii] = -np.inf
+                O[s + r0:s + r1, cols] = softmax_rows(S) @ v[:r1]
+    G = sigmoid(Go) if gates else 1.0
+    return (O * G) @ _f64(layer["w_o"])
+
+
+def ffn_sublayer(y: np.ndarray, layer: dict) -> np.ndarray:
+    """SwiGLU FFN of the LLaMA-style block (§3.2): (SiLU(y W_1) * y W_3) W_2."""
+    W13 = _f64(layer["w_ffn13"])
+    dff = W13.shape[1] // 2
+    A = y @ W13
+    return (silu(A[:, :dff]) * A[:, dff:]) @ _f64(layer["w_ffn2"])
+
+
+def srn(x: np.ndarray, sub, alpha: float, post: bool, g: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Eq. 6 (Stabilized Residual Normalization) around one sublayer.
+
+    post:  LN(x + alpha * Sub(x));   pre:  x + alpha * Sub(LN(x)).
+    """
+    if post:
+        return layer_norm(x + alpha * sub(x), g, b)
+    return x + alpha * sub(layer_norm(x, g, b))
+
+
+# --------------------------------------------------------------------------
+# encoder T, cross decoder C, rank_request
+# --------------------------------------------------------------------------
+
+def encoder(inp: dict, gates: bool = True, angle_scale: float = 1.0,
+            time_origin=None, pos_offset: int = 0, n_layers: Optional[int] = None) -> np.ndarray:
+    """Encoder T (§3.2, Fig. 1 left): n_layers blocks of [DGA, SwiGLU FFN],
+    each sublayer wrapped by eq. 6 with post-LN for l <= l_switch (1-based).
+
+    Readings: one layer = attention sublayer then FFN sublayer (the LLaMA
+    block the page starts from); no final norm; separate alpha per sublayer.
+    """
+    x = _f64(inp["x"]).copy()
+    taus = np.asarray(inp["taus"], dtype=np.int64)
+    H = len(taus)
+    d = x.shape[1]
+    hd = d // H
+    idx = rotation_index(inp["ts"], inp["cu_seqlens"], taus, time_origin, pos_offset)
+    phi = rotation_angles(idx, hd, inp["rope_base"], angle_scale)
+    layers = inp["layers"] if n_layers is None else inp["layers"][:n_layers]
+    for l, lay in enumerate(layers, start=1):
+        post = l <= inp["l_switch"]
+        x = srn(x, lambda y: dga_sublayer(y, phi, inp["cu_seqlens"], lay, H, gates),
+                lay["alpha_attn"], post, lay["ln_attn_g"], lay["ln_attn_b"])
+        if lay.get("w_ffn13") is not None:
+            x = srn(x, lambda y: ffn_sublayer(y, lay),
+                    lay["alpha_ffn"], post, lay["ln_ffn_g"], lay["ln_ffn_b"])
+    return x
+
+
+def cross_decode(Hmem: np.ndarray, cu_seqlens: np.ndarray, req_user, req_cutoff, cu_cands,
+                 z: np.ndarray, dec: dict, n_heads: int, gates: bool = True,
+                 row_chunk: int = 1024) -> np.ndarray:
+    """Cross decoder C (§3.3, eqs. 7-8) -> y [N_total, K, d].
+
+    Projection-free keys and values: the first c_r rows of the user's H are
+    used directly as K and V. Token-specific W_Q^(k), W_go^(k) (eq. 8); a
+    shared W_o. Readings: one decoder layer exactly as eq. 7 (no residual,
+    no rotation); scale 1/sqrt(d_h).
+    """
+    Hm = _f64(Hmem)
+    z = _f64(z)
+    N, K, d = z.shape
+    hd = d // n_heads
+    Wq, Wg, Wo = _f64(dec["w_q"]), _f64(dec["w_go"]), _f64(dec["w_o"])
+    q = np.einsum("nkd,kde->nke", z, Wq)
+    g = sigmoid(np.einsum("nkd,kde->nke", z, Wg)) if gates else np.ones_like(q)
+    o = np.zeros_like(q)
+    scale = 1.0 / math.sqrt(hd)
+    for r in range(len(req_user)):
+        u, c = int(req_user[r]), int(req_cutoff[r])
+        n0, n1 = int(cu_cands[r]), int(cu_cands[r + 1])
+        if n1 <= n0:
+            continue
+        s = int(cu_seqlens[u])
+        mem = Hm[s:s + c]
+        qr = q[n0:n1].reshape(-1, d)
+        orows = np.zeros_like(qr)
+        for h in range(n_heads):
+            cols = slice(h * hd, (h + 1) * hd)
+            for r0 in range(0, qr.shape[0], row_chunk):
+                r1 = min(qr.shape[0], r0 + row_chunk)
+                S = (qr[r0:r1, cols] @ mem[:, cols].T) * scale
+                orows[r0:r1, cols] = softmax_rows(S) @ mem[:, cols]
+        o[n0:n1] = orows.reshape(n1 - n0, K, d)
+    return (o * g) @ Wo
+
+
+def rank_request(inp: dict, **kw):
+    """Shared-prefix serving (§3.5): H = T(S_u) once, then C for every
+    candidate of every request against it. Returns (H, y)."""
+    Hm = encoder(inp, **kw)
+    y = cross_decode(Hm, inp["cu_seqlens"], inp["req_user"], inp["req_cutoff"], inp["cu_cands"],
+                     inp["z"], inp["dec"], len(inp["taus"]))
+    return Hm, y
