@@ -1,0 +1,365 @@
+"""Benchmark of the ReST encode-once / decode-many ranking forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl reference]
+
+One step = one ``rank_request`` over a batch of the named workload (default:
+32 users x 1024 tokens, d=256, 8 heads of 32 (4 RoPE + 4 RoTE), 4 encoder
+layers, 128 candidates x 3 query tokens per user, bf16): the encoder over
+every history, then every candidate of every request against its user's
+encoder output. Multi-GPU runs shard users across ranks (weak scaling: every
+rank runs its own batch), with no collective on the data path.
+
+Rank 0 prints one JSON line. ``value`` is candidate scores/s over all ranks
+with inputs resident in HBM, timed with CUDA events (max over ranks);
+``e2e`` is the same metric with the step's inputs copied from pinned host
+memory and the scores copied back inside the timed region. ``roofline`` is
+for the kernel with the largest share of device time, from a second pass of
+the same steps with per-kernel CUDA events. ``cpu_baseline`` times the fp64
+oracle on the host cores on a bounded sample. ``--impl reference`` times that
+oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "candidate scores/s & encoder tokens/s on 1 B200; % bf16 tensor peak / HBM roofline"
+UNIT = "candidate scores/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TENSOR_KERNELS = ("gemm", "enc_attn", "dec_attn")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w: W.Workload, n: int) -> dict:
+    n_rope = int(np.sum(w.taus == 0))
+    return {
+        "workload": w.name,
+        "users_per_gpu": w.n_users,
+        "history_len": w.lengths[0] if len(set(w.lengths)) == 1 else "ragged",
+        "tokens_per_gpu": w.total_tokens,
+        "d": w.d,
+        "heads": f"{w.n_heads}x{w.head_dim} ({n_rope} RoPE + {w.n_heads - n_rope} RoTE)",
+        "encoder_layers": w.n_layers,
+        "candidates_per_gpu": w.total_cands,
+        "query_tokens": w.K,
+        "parallelism": f"dp{n}: users sharded across ranks, no collective",
+        "l2": "not flushed: one step writes and reads ~0.5 GB of activations, above the 126 MB L2",
+    }
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- oracle (CPU baseline / reference arm)
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(w: W.Workload, inp: dict, users):
+    """Time the fp64 oracle on a subset of users: returns (seconds, candidates, tokens)."""
+    from oracle import rest_oracle as O
+    from tests.parity import subset_users
+    sub = subset_users(inp, users)
+    t0 = time.perf_counter()
+    O.rank_request(sub)
+    dt = time.perf_counter() - t0
+    return dt, int(sub["cu_cands"][-1]), int(sub["cu_seqlens"][-1])
+
+
+def cpu_baseline(w: W.Workload, inp: dict, budget_s: float) -> dict:
+    t_tot, c_tot, tok_tot, users = 0.0, 0, 0, []
+    for u in range(w.n_users):
+        dt, c, tok = oracle_sample(w, inp, [u])
+        t_tot += dt
+        c_tot += c
+        tok_tot += tok
+        users.append(u)
+        if t_tot >= budget_s:
+            break
+    return {"value": c_tot / t_tot, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(users)} of {w.n_users} users of {w.name} (encoder + all their candidates), "
+                      f"fp64 numpy, {t_tot:.1f} s", "encoder_tokens_per_s": tok_tot / t_tot}
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    w = W.workload(args.workload)
+    inp = W.make_inputs(w, 1000 + args.workload)
+    for i in range(args.warmup):
+        oracle_sample(w, inp, [i % w.n_users])
+    t_tot, c_tot, tok_tot = 0.0, 0, 0
+    for i in range(args.steps):
+        dt, c, tok = oracle_sample(w, inp, [(args.warmup + i) % w.n_users])
+        t_tot += dt
+        c_tot += c
+        tok_tot += tok
+    value = c_tot / t_tot
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: 1 of {w.n_users} users of {w.name} (encoder + its candidates)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "encoder_tokens_per_s": tok_tot / t_tot,
+    }
+    print(json.dumps(out), flush=True)
+
+
+# --------------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import shared_prefix_behavior_b200 as R
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = W.workload(args.workload)
+    inp = W.make_inputs(w, 1000 + args.workload + 7919 * rank)
+    t = R.to_device(inp, dev)
+    dt_name = "bf16" if w.dtype == "bf16" else "f32"
+    args_rank = (t["x"], t["ts"], t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"], t["z"],
+                 t["dec"], t["rope_base"])
+    nbytes = R.workspace_size(R.REST_BF16 if w.dtype == "bf16" else R.REST_F32, t["taus"], w.d, t["cu_seqlens"],
+                              t["layers"], t["reqs"], w.K, t["rope_base"])
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    H = torch.empty_like(t["x"])
+    Y = torch.empty(t["z"].shape, dtype=torch.float32, device=dev)
+
+    def step():
+        R.rank_request(*args_rank, h_out=H, y_out=Y, ws=ws, check=False)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # correctness guard: the device status word must stay clear
+    R.rank_request(*args_rank, h_out=H, y_out=Y, ws=ws, check=True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    R.launch_count(reset=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    launches = R.launch_count(reset=True)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        tm = torch.tensor([ms], device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ms = float(tm.item())
+    ms_step = ms / args.steps
+    cands = w.total_cands * world
+    tokens = w.total_tokens * world
+    value = cands / (ms_step * 1e-3)
+
+    # per-kernel pass: the same steps with CUDA events around every launch
+    R.profile_begin()
+    for _ in range(args.steps):
+        step()
+    stats = R.profile_end()
+    torch.cuda.synchronize()
+
+    # end to end through the public API: pinned host inputs in, scores out
+    x_h = t["x"].cpu().pin_memory()
+    ts_h = t["ts"].cpu().pin_memory()
+    z_h = t["z"].cpu().pin_memory()
+    y_h = torch.empty(Y.shape, dtype=torch.float32).pin_memory()
+    x_d, ts_d, z_d = torch.empty_like(t["x"]), torch.empty_like(t["ts"]), torch.empty_like(t["z"])
+    e_args = (x_d, ts_d, t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"], z_d, t["dec"],
+              t["rope_base"])
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        ts_d.copy_(ts_h, non_blocking=True)
+        z_d.copy_(z_h, non_blocking=True)
+        R.rank_request(*e_args, h_out=H, y_out=Y, ws=ws, check=False)
+        y_h.copy_(Y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tm = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tm.item())
+    e2e_value = cands / (e2e_ms / args.steps * 1e-3)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    total_ms = sum(s["ms"] for s in stats)
+    top = max(stats, key=lambda s: s["ms"])
+    per_launch_s = top["ms"] / top["launches"] * 1e-3
+    if top["name"].startswith(TENSOR_KERNELS):
+        bound, unit = "tensor", "TFLOP/s"
+        achieved = top["flops"] / top["launches"] / per_launch_s / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        peak_note = f"bf16 dense, sustained ({peak_src})"
+    else:
+        bound, unit = "hbm", "GB/s"
+        achieved = top["bytes"] / top["launches"] / per_launch_s / 1e9
+        peak = float(peaks["hbm_gbs"])
+        peak_note = f"HBM copy ({peak_src})"
+    kernels = []
+    for s in sorted(stats, key=lambda s: -s["ms"]):
+        sec = s["ms"] * 1e-3
+        kernels.append({"name": s["name"], "launches_per_step": s["launches"] / args.steps,
+                        "ms_per_step": s["ms"] / args.steps, "share": s["ms"] / total_ms,
+                        "tflops": s["flops"] / sec / 1e12 if sec > 0 else None,
+                        "gbs": s["bytes"] / sec / 1e9 if sec > 0 else None})
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": dt_name, "data": "synthetic (seeded; shapes of the named workload)",
+        "config": workload_config(w, world),
+        "encoder_tokens_per_s": tokens / (ms_step * 1e-3),
+        "roofline": {"kernel": top["name"], "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "peak_source": peak_note, "traffic": None,
+                     "share_of_step": top["ms"] / total_ms},
+        "kernels": kernels,
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": int(x_h.numel() * x_h.element_size() + ts_h.numel() * 8 +
+                                          z_h.numel() * z_h.element_size()),
+                "d2h_bytes_per_step": int(y_h.numel() * 4)},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_budget)
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * rest.h -- C ABI of the ReST encode-once / decode-many ranking forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the one described in "From Language to Behavior" (a close
+ * reading of the ReST paper, arXiv 2609.01240): a causal Dual-Gated-Attention
+ * encoder T run once per user history (§3.2, eqs. 3-6) and a projection-free,
+ * token-specific cross decoder C run for every candidate against T's output
+ * (§3.3, eqs. 7-8), served with a shared prefix (§3.5).
+ *
+ * Conventions for every entry point
+ *   - Matrices are row-major; a projection is x . W with W stored [d_in, d_out].
+ *   - "dev" pointers are CUDA device memory owned by the caller (for example
+ *     allocated by PyTorch); "host" pointers are ordinary host memory read
+ *     before the call returns. The library never frees or keeps any pointer,
+ *     and allocates no device memory: all scratch lives in the caller's
+ *     workspace `ws` of at least rest_workspace_size() bytes.
+ *   - Every dev pointer must be 16-byte aligned.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream). Host-detectable errors are returned
+ *     synchronously before anything is enqueued. Errors found on the device
+ *     (decreasing timestamps, a bounded wait that ran out) are written to the
+ *     int32 word `*dev_err` (dev, may be NULL to ignore them); the caller
+ *     zeroes it beforehand and reads it after synchronizing.
+ *   - An empty batch (no tokens, or no candidates) is a successful no-op.
+ *   - No C++ exception crosses this boundary.
+ *   - REST_F32 computes with fp32 storage throughout. REST_BF16 takes bf16
+ *     inputs and weights, multiplies bf16 operands with fp32 accumulation,
+ *     keeps the residual stream, softmax statistics and gates in fp32, and
+ *     stores the activations that feed a matrix product in bf16.
+ */
+#ifndef REST_H_
+#define REST_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  REST_OK = 0,
+  REST_ERR_INVALID_ARG = 1,   /* a shape, pointer, alignment or index argument is invalid */
+  REST_ERR_UNSORTED_TIME = 2, /* (device) a user's timestamps decrease */
+  REST_ERR_UNSUPPORTED = 3,   /* valid but not supported (e.g. head_dim outside the built set) */
+  REST_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, copy, device query) */
+  REST_ERR_TIMEOUT = 5,       /* (device) a bounded wait inside a kernel ran out */
+  REST_ERR_WORKSPACE = 6,     /* ws is NULL or smaller than rest_workspace_size() */
+  REST_ERR_NO_DEVICE = 7      /* no CUDA device of compute capability 10.0 is current */
+} rest_status;
+
+typedef enum { REST_F32 = 0, REST_BF16 = 1 } rest_dtype;
+
+/* Attention-head split (§3.2.2, eq. 5). Head h owns columns
+ * h*head_dim .. (h+1)*head_dim-1 of every d-wide activation. */
+typedef struct {
+  int d;               /* model width, == n_heads * head_dim */
+  int n_heads;
+  int head_dim;        /* even; REST_BF16 supports 32 and 64, REST_F32 16, 32 and 64 */
+  const int64_t* tau;  /* host [n_heads]: 0 = RoPE head (ordinal position),
+                          > 0 = RoTE head with time buckets of tau seconds */
+  double rope_base;    /* theta_j = rope_base^(-2j/head_dim), normally 10000 */
+} rest_heads;
+
+/* Packed, padding-free histories: user u owns rows cu_seqlens[u] ..
+ * cu_seqlens[u+1]-1 of every [T, *] array, T = cu_seqlens[n_users]. */
+typedef struct {
+  int n_users;
+  const int32_t* cu_seqlens;  /* host [n_users+1]; cu_seqlens[0] == 0, non-decreasing */
+} rest_batch;
+
+/* One encoder layer (Fig. 1 left): a DGA sublayer and an optional SwiGLU FFN
+ * sublayer, each wrapped by SRN (eq. 6). Weights have the dtype of the call. */
+typedef struct {
+  const void* w_qkvgg;   /* dev [d, 5d]: column blocks W_Q | W_K | W_V | W_gv | W_go (eqs. 3-4) */
+  const void* w_o;       /* dev [d, d] */
+  const void* w_ffn13;   /* dev [d, 2*d_ff]: W_1 | W_3, or NULL for an attention-only layer */
+  const void* w_ffn2;    /* dev [d_ff, d] (ignored when w_ffn13 is NULL) */
+  const float* ln_attn_g; /* dev [d] fp32 LayerNorm gain/bias of the attention sublayer */
+  const float* ln_attn_b;
+  const float* ln_ffn_g;  /* dev [d] fp32, of the FFN sublayer (ignored without FFN) */
+  const float* ln_ffn_b;
+  float alpha_attn;      /* SRN residual scale of each sublayer */
+  float alpha_ffn;
+  int d_ff;              /* FFN width, a multiple of 64 (0 without FFN) */
+} rest_enc_layer;
+
+/* Cross-decoder parameters (§3.3): token-specific W_Q and W_go (eq. 8), a
+ * shared W_o. Weights have the dtype of the call. */
+typedef struct {
+  int K;              /* query tokens per candidate, 1..8 ([CLS], ad, user: K = 3) */
+  const void* w_q;    /* dev [K, d, d] */
+  const void* w_go;   /* dev [K, d, d] */
+  const void* w_o;    /* dev [d, d] */
+} rest_dec_params;
+
+/* Ranking requests sharing encoded prefixes (§3.5). Request r belongs to user
+ * req_user[r], reads the first req_cutoff[r] rows of that user's encoder
+ * output, and scores candidates cu_cands[r] .. cu_cands[r+1]-1. */
+typedef struct {
+  int n_req;
+  const int32_t* req_user;    /* host [n_req], 0 .. n_users-1 */
+  const int32_t* req_cutoff;  /* host [n_req], 1 .. L_user */
+  const int32_t* cu_cands;    /* host [n_req+1]; cu_cands[0] == 0, non-decreasing */
+} rest_requests;
+
+/* Bytes of workspace that rest_rank_request (and therefore each of the
+ * entry points below) needs for this batch. `reqs` may be NULL (encoder
+ * only); `n_layers`/`layers` may be 0/NULL (decoder only). Returns
+ * REST_ERR_INVALID_ARG for invalid shapes. */
+rest_status rest_workspace_size(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                const rest_enc_layer* layers, int n_layers,
+                                const rest_requests* reqs, int K, size_t* bytes);
+
+/* Rotation index and table of §3.2.2 / eq. 5, the first step of the encoder.
+ * For row i of user u (position p = i - cu_seqlens[u]) and head h:
+ *   idx[i,h] = p                                   if tau_h == 0 (RoPE)
+ *   idx[i,h] = floor((ts[i] - ts[cu_seqlens[u]]) / tau_h)   otherwise (RoTE)
+ * and for j < head_dim/2, with phi = idx * rope_base^(-2j/head_dim) in fp64:
+ *   cos_out[i,h,j] = cos(phi), sin_out[i,h,j] = sin(phi)   (stored fp32).
+ *   ts:      dev [T] int64 seconds, non-decreasing within each user
+ *            (a decrease sets *dev_err = REST_ERR_UNSORTED_TIME)
+ *   idx_out: dev [T, n_heads] int64 (may be NULL)
+ *   cos_out, sin_out: dev [T, n_heads, head_dim/2] fp32 (both or neither NULL)
+ * Needs no workspace beyond the batch index copy: ws as for the encoder. */
+rest_status rest_rotation_table(const rest_heads* heads, const rest_batch* batch, const int64_t* ts,
+                                int64_t* idx_out, float* cos_out, float* sin_out,
+                                void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Encoder T (§3.2, eqs. 3-6; Fig. 1 left): n_layers layers over the packed
+ * histories. Layer l (1-based) uses post-LN when l <= l_switch and pre-LN
+ * otherwise (eq. 6). Each DGA sublayer computes, per head and per user,
+ * causal softmax(q k^T / sqrt(head_dim)) over rotated q, k (eq. 5) against the
+ * value-gated V' = sigmoid(x W_gv) * (x W_V), then the output gate
+ * sigmoid(x W_go) and W_o (eqs. 3-4).
+ *   x:     dev [T, d] (dtype of the call)  history features s_i
+ *   ts:    dev [T] int64 timestamps t_i in seconds
+ *   layers: host [n_layers]
+ *   h_out: dev [T, d] (dtype of the call)  the encoder memory H
+ */
+rest_status rest_encoder_attn(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                              const void* x, const int64_t* ts,
+                              const rest_enc_layer* layers, int n_layers, int l_switch,
+                              void* h_out, void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Cross decoder C (§3.3, eq. 7 with the token-specific weights of eq. 8).
+ * For every request r, candidate n, query token k:
+ *   q = z[n,k] W_Q^(k),  g = sigmoid(z[n,k] W_go^(k)),
+ *   per head: o_h = softmax(q_h H_h^T / sqrt(head_dim)) H_h over the first
+ *   req_cutoff[r] rows of the user's H (keys and values are H itself),
+ *   y[n,k] = (o * g) W_o.
+ * Every H tile is staged once per request and head and read by all of the
+ * request's candidate query rows (the shared prefix).
+ *   h:     dev [T, d] (dtype of the call)  encoder memory
+ *   z:     dev [N_total, K, d] (dtype of the call)  candidate query tokens
+ *   y_out: dev [N_total, K, d] fp32
+ */
+rest_status rest_cross_decode(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                              const void* h, const rest_requests* reqs, const void* z,
+                              const rest_dec_params* dec, float* y_out,
+                              void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Shared-prefix serving (§3.5): the encoder runs once over the packed
+ * histories and the decoder scores every candidate of every request against
+ * its output: FLOPs(T) + N * FLOPs(C) instead of N * (FLOPs(T) + FLOPs(C)).
+ * Arguments as in rest_encoder_attn and rest_cross_decode; h_out receives H. */
+rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                              const void* x, const int64_t* ts,
+                              const rest_enc_layer* layers, int n_layers, int l_switch,
+                              const rest_requests* reqs, const void* z, const rest_dec_params* dec,
+                              void* h_out, float* y_out,
+                              void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Static description of a status code. */
+const char* rest_status_string(rest_status s);
+
+/* Number of kernel launches the library enqueued on this host thread since
+ * the last call with reset != 0 (instrumentation for benchmarks). */
+long long rest_launch_count(int reset);
+
+/* Per-kernel timing (instrumentation for benchmarks; not part of the method).
+ * Between rest_profile_begin() and rest_profile_end(), every kernel the
+ * library launches from this host thread is bracketed by two CUDA events on
+ * its own stream. rest_profile_end() waits for those events, aggregates them
+ * by kernel name and writes up to max_out records to `out` (host), returning
+ * the number of distinct kernels. `flops` and `bytes` are the algorithmic
+ * work of the launches (the FLOPs and the bytes that must cross HBM once),
+ * computed from the shapes; `name` points to a static string. */
+typedef struct {
+  const char* name;
+  int launches;
+  double ms;
+  double flops;
+  double bytes;
+} rest_kernel_stat;
+void rest_profile_begin(void);
+int rest_profile_end(rest_kernel_stat* out, int max_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REST_H_ */

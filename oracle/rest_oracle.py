@@ -235,6 +235,59 @@ def encoder(inp: dict, gates: bool = True, angle_scale: float = 1.0,
     return x
 
 
+def encoder_rows(inp: dict, rows: Sequence[int]) -> np.ndarray:
+    """Selected rows of H for a one-layer encoder, each computed on its own.
+
+    Same definition as ``encoder`` (§3.2, eqs. 3-6); a query row of a single
+    layer only needs its own row and the keys/values of the rows before it,
+    so a handful of rows of a 16k-token history can be checked without the
+    full L x L computation.
+    """
+    assert len(inp["layers"]) == 1, "row sampling is exact only for one layer"
+    lay = inp["layers"][0]
+    post = 1 <= inp["l_switch"]
+    x = _f64(inp["x"])
+    taus = np.asarray(inp["taus"], dtype=np.int64)
+    H = len(taus)
+    d = x.shape[1]
+    hd = d // H
+    cu = np.asarray(inp["cu_seqlens"])
+    idx = rotation_index(inp["ts"], cu, taus)
+    phi = rotation_angles(idx, hd, inp["rope_base"])
+    W = _f64(lay["w_qkvgg"])
+    scale = 1.0 / math.sqrt(hd)
+    out = np.zeros((len(rows), d))
+    cache = {}
+    for n, i in enumerate(rows):
+        u = int(np.searchsorted(cu, i, side="right") - 1)
+        s = int(cu[u])
+        if u not in cache:   # projections of the user's rows 0..L-1
+            e = int(cu[u + 1])
+            y = x[s:e] if post else layer_norm(x[s:e], lay["ln_attn_g"], lay["ln_attn_b"])
+            P5 = y @ W
+            Q, Kx, V, Gv, Go = (P5[:, j * d:(j + 1) * d] for j in range(5))
+            cache = {u: (rotate(Q, phi[s:e]), rotate(Kx, phi[s:e]), V * sigmoid(Gv), sigmoid(Go))}
+        Qr, Kr, Vg, G = cache[u]
+        p = i - s
+        o = np.zeros(d)
+        for h in range(H):
+            c = slice(h * hd, (h + 1) * hd)
+            sc = (Kr[:p + 1, c] @ Qr[p, c]) * scale
+            w = np.exp(sc - sc.max())
+            o[c] = (w / w.sum()) @ Vg[:p + 1, c]
+        a = (o * G[p]) @ _f64(lay["w_o"])
+        xi = x[i]
+        x1 = layer_norm(xi + lay["alpha_attn"] * a, lay["ln_attn_g"], lay["ln_attn_b"]) if post \
+            else xi + lay["alpha_attn"] * a
+        if lay.get("w_ffn13") is not None:
+            y2 = x1 if post else layer_norm(x1, lay["ln_ffn_g"], lay["ln_ffn_b"])
+            f = ffn_sublayer(y2[None, :], lay)[0]
+            x1 = layer_norm(x1 + lay["alpha_ffn"] * f, lay["ln_ffn_g"], lay["ln_ffn_b"]) if post \
+                else x1 + lay["alpha_ffn"] * f
+        out[n] = x1
+    return out
+
+
 def cross_decode(Hmem: np.ndarray, cu_seqlens: np.ndarray, req_user, req_cutoff, cu_cands,
                  z: np.ndarray, dec: dict, n_heads: int, gates: bool = True,
                  row_chunk: int = 1024) -> np.ndarray:

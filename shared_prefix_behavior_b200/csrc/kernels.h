@@ -1,0 +1,81 @@
+// Internal launcher interface between the C-ABI layer (rest_api.cu) and the
+// kernel translation units. Host-side C++ only; not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rest {
+
+// ---------------------------------------------------------------- table
+struct TableParams {
+  int n_heads, half;            // half = head_dim / 2
+  long long tau[32];            // per head, 0 = RoPE
+  double theta[64];             // theta_j = base^(-2j/head_dim)
+};
+cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users,
+                                  int T, const TableParams& p, int64_t* idx_out, float* cos_out,
+                                  float* sin_out, int32_t* err, cudaStream_t s);
+
+// ---------------------------------------------------------------- casts / norms
+// mode 0: y = dt(LN(x))  (pre-LN input of a sublayer)
+// mode 1: x = LN(x); y = dt(x)  (post-LN after the residual add)
+// mode 2: y = dt(x)  (post-LN sublayer input, no norm)
+// mode 3: x = LN(x)  (post-LN, y not written)
+cudaError_t launch_layernorm(bool bf16, float* x, void* y, const float* g, const float* b, int T, int d,
+                             int mode, cudaStream_t s);
+// x_res = float(x_in)
+cudaError_t launch_to_f32(bool bf16, const void* x_in, float* x_res, long long n, cudaStream_t s);
+
+// ---------------------------------------------------------------- GEMM
+enum Epilogue {
+  EPI_F32 = 0,      // out0[m, n] = acc (fp32)
+  EPI_DT = 1,       // out0[m, n] = dt(acc)
+  EPI_SIGMOID = 2,  // out0[m, n] = sigmoid(acc) (fp32)
+  EPI_RESID = 3,    // out0[m, n] += alpha * acc (fp32 residual stream)
+  EPI_QKVG = 4,     // the DGA projection epilogue (rotation, value gate, output gate)
+  EPI_SWIGLU = 5    // out0[m, j] = dt(SiLU(acc_1) * acc_3)
+};
+struct GemmArgs {
+  const void* A; long long lda;   // [M, K], row stride lda elements
+  const void* B; long long ldb;   // [K, N] row-major, row stride ldb elements
+  int M, N, K;
+  int epi;
+  void* out0; void* out1; void* out2; void* out3;
+  long long ldo;                  // row stride of the outputs (elements)
+  const float* cos_t; const float* sin_t;  // [M, d/2] rotation table (EPI_QKVG)
+  float alpha;
+  int d;                          // model width (EPI_QKVG) or d_ff (EPI_SWIGLU)
+  int a_f32;                      // A is fp32 even when the call's dtype is bf16
+};
+// Logical output columns of EPI_QKVG are [Q | K | V,Gv interleaved | Go] and of
+// EPI_SWIGLU [W1,W3 interleaved]: every group of 4 logical columns holds
+// columns (2p, 2p+1) of the first block then of the second.
+cudaError_t launch_gemm_simt(bool bf16, const GemmArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+struct EncTile { int user; int q0; };          // q0: first query position within the user
+struct DecTile { int row0; int nrows; int key0; int nkeys; };  // query rows, memory rows of H
+struct EncAttnArgs {
+  const void* q; const void* k; const void* v;  // [T, d] rotated Q, K and gated V'
+  const float* gate;                            // [T, d] sigmoid(Go)
+  void* out;                                    // [T, d] dt(O * gate)
+  const int32_t* cu;                            // [n_users+1]
+  const EncTile* tiles; int n_tiles;
+  int n_heads, d;
+  float scale_log2;                             // log2(e) / sqrt(head_dim)
+};
+cudaError_t launch_enc_attn_simt(bool bf16, int hd, const EncAttnArgs& a, cudaStream_t s);
+
+struct DecAttnArgs {
+  const float* q;      // [NK, d] decoder queries (fp32)
+  const float* g;      // [NK, d] sigmoid output gate
+  const void* h;       // [T, d] encoder memory: keys and values
+  float* out;          // [NK, d] o * g (fp32)
+  const DecTile* tiles; int n_tiles;
+  int n_heads, d;
+  float scale_log2;
+};
+cudaError_t launch_dec_attn_simt(bool bf16, int hd, const DecAttnArgs& a, cudaStream_t s);
+
+}  // namespace rest

@@ -1,0 +1,620 @@
+// C-ABI entry points of the ReST ranking forward: argument validation,
+// workspace layout, work lists, and the launch sequence of the encoder
+// (ReST §3.2) and the shared-prefix cross decoder (§3.3, §3.5).
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "rest.h"
+#include "sm100.h"
+
+namespace rest {
+
+static thread_local long long g_launches = 0;
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+static inline size_t dt_size(rest_dtype dt) { return dt == REST_BF16 ? 2 : 4; }
+
+// ---------------------------------------------------------------- validation
+
+static rest_status check_heads(rest_dtype dt, const rest_heads* hs) {
+  if (dt != REST_F32 && dt != REST_BF16) return REST_ERR_INVALID_ARG;
+  if (!hs || !hs->tau) return REST_ERR_INVALID_ARG;
+  if (hs->n_heads < 1 || hs->n_heads > 32 || hs->head_dim < 2 || (hs->head_dim & 1)) return REST_ERR_INVALID_ARG;
+  if (hs->d != hs->n_heads * hs->head_dim) return REST_ERR_INVALID_ARG;
+  if (!(hs->rope_base > 0.0) || !isfinite(hs->rope_base)) return REST_ERR_INVALID_ARG;
+  for (int h = 0; h < hs->n_heads; ++h)
+    if (hs->tau[h] < 0) return REST_ERR_INVALID_ARG;
+  if (hs->head_dim != 16 && hs->head_dim != 32 && hs->head_dim != 64) return REST_ERR_UNSUPPORTED;
+  if (hs->d % 32 != 0 || hs->d > 1024) return REST_ERR_UNSUPPORTED;
+  return REST_OK;
+}
+
+static rest_status check_batch(const rest_batch* b, long long* total) {
+  if (!b || b->n_users < 0) return REST_ERR_INVALID_ARG;
+  *total = 0;
+  if (b->n_users == 0) return REST_OK;
+  if (!b->cu_seqlens || b->cu_seqlens[0] != 0) return REST_ERR_INVALID_ARG;
+  for (int u = 0; u < b->n_users; ++u)
+    if (b->cu_seqlens[u + 1] < b->cu_seqlens[u]) return REST_ERR_INVALID_ARG;
+  *total = b->cu_seqlens[b->n_users];
+  return REST_OK;
+}
+
+static rest_status check_layers(const rest_enc_layer* layers, int n_layers, int l_switch, int* max_dff) {
+  *max_dff = 0;
+  if (n_layers < 0 || (n_layers > 0 && !layers)) return REST_ERR_INVALID_ARG;
+  if (l_switch < 0 || l_switch > n_layers) return REST_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    const rest_enc_layer& L = layers[l];
+    if (!L.w_qkvgg || !L.w_o || !L.ln_attn_g || !L.ln_attn_b) return REST_ERR_INVALID_ARG;
+    if (!aligned16(L.w_qkvgg) || !aligned16(L.w_o) || !aligned16(L.ln_attn_g) || !aligned16(L.ln_attn_b))
+      return REST_ERR_INVALID_ARG;
+    if (!isfinite(L.alpha_attn) || !isfinite(L.alpha_ffn)) return REST_ERR_INVALID_ARG;
+    if (L.w_ffn13) {
+      if (!L.w_ffn2 || !L.ln_ffn_g || !L.ln_ffn_b || L.d_ff <= 0 || L.d_ff % 64 != 0 || L.d_ff > 16384)
+        return REST_ERR_INVALID_ARG;
+      if (!aligned16(L.w_ffn13) || !aligned16(L.w_ffn2) || !aligned16(L.ln_ffn_g) || !aligned16(L.ln_ffn_b))
+        return REST_ERR_INVALID_ARG;
+      *max_dff = std::max(*max_dff, L.d_ff);
+    }
+  }
+  return REST_OK;
+}
+
+static rest_status check_requests(const rest_requests* r, const rest_batch* b, long long* n_cands) {
+  if (!r || r->n_req < 0) return REST_ERR_INVALID_ARG;
+  *n_cands = 0;
+  if (r->n_req == 0) return REST_OK;
+  if (!r->req_user || !r->req_cutoff || !r->cu_cands || r->cu_cands[0] != 0) return REST_ERR_INVALID_ARG;
+  for (int i = 0; i < r->n_req; ++i) {
+    int u = r->req_user[i];
+    if (u < 0 || u >= b->n_users) return REST_ERR_INVALID_ARG;
+    int L = b->cu_seqlens[u + 1] - b->cu_seqlens[u];
+    if (r->req_cutoff[i] < 1 || r->req_cutoff[i] > L) return REST_ERR_INVALID_ARG;
+    if (r->cu_cands[i + 1] < r->cu_cands[i]) return REST_ERR_INVALID_ARG;
+  }
+  *n_cands = r->cu_cands[r->n_req];
+  return REST_OK;
+}
+
+static rest_status check_dec(const rest_dec_params* dec) {
+  if (!dec || dec->K < 1 || dec->K > 8) return REST_ERR_INVALID_ARG;
+  if (!dec->w_q || !dec->w_go || !dec->w_o) return REST_ERR_INVALID_ARG;
+  if (!aligned16(dec->w_q) || !aligned16(dec->w_go) || !aligned16(dec->w_o)) return REST_ERR_INVALID_ARG;
+  return REST_OK;
+}
+
+// ---------------------------------------------------------------- work lists
+
+constexpr int ENC_TILE_ROWS = 128;
+constexpr int DEC_TILE_ROWS = 128;
+
+static void build_enc_tiles(const rest_batch* b, std::vector<EncTile>& t) {
+  t.clear();
+  for (int u = 0; u < b->n_users; ++u) {
+    int L = b->cu_seqlens[u + 1] - b->cu_seqlens[u];
+    for (int q0 = 0; q0 < L; q0 += ENC_TILE_ROWS) t.push_back(EncTile{u, q0});
+  }
+  // longest causal rows first, so the tail of the grid holds the short tiles
+  std::stable_sort(t.begin(), t.end(), [](const EncTile& a, const EncTile& c) { return a.q0 > c.q0; });
+}
+
+static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, std::vector<DecTile>& t) {
+  t.clear();
+  if (!r) return;
+  for (int i = 0; i < r->n_req; ++i) {
+    long long rows0 = (long long)r->cu_cands[i] * K, rows1 = (long long)r->cu_cands[i + 1] * K;
+    int key0 = b->cu_seqlens[r->req_user[i]];
+    for (long long p = rows0; p < rows1; p += DEC_TILE_ROWS)
+      t.push_back(DecTile{(int)p, (int)std::min<long long>(DEC_TILE_ROWS, rows1 - p), key0, r->req_cutoff[i]});
+  }
+  std::stable_sort(t.begin(), t.end(), [](const DecTile& a, const DecTile& c) { return a.nkeys > c.nkeys; });
+}
+
+// ---------------------------------------------------------------- workspace
+
+struct Layout {
+  size_t cu, enc_tiles, dec_tiles, meta_end;
+  size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
+  size_t dq, dg, dout;
+  size_t total;
+  int n_enc_tiles, n_dec_tiles;
+};
+
+static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
+                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles) {
+  Layout L;
+  const size_t A = 256, e = dt_size(dt);
+  const size_t d = (size_t)hs->d;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, A); return o; };
+  L.n_enc_tiles = n_enc_tiles;
+  L.n_dec_tiles = n_dec_tiles;
+  L.cu = take(sizeof(int32_t) * (size_t)(b->n_users + 1));
+  L.enc_tiles = take(sizeof(EncTile) * (size_t)n_enc_tiles);
+  L.dec_tiles = take(sizeof(DecTile) * (size_t)n_dec_tiles);
+  L.meta_end = off;
+  L.cos_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
+  L.sin_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
+  L.xres = take(enc ? 4 * (size_t)T * d : 0);
+  L.y = take(enc ? e * (size_t)T * d : 0);
+  L.q = take(enc ? e * (size_t)T * d : 0);
+  L.k = take(enc ? e * (size_t)T * d : 0);
+  L.v = take(enc ? e * (size_t)T * d : 0);
+  L.g = take(enc ? 4 * (size_t)T * d : 0);
+  L.o = take(enc ? e * (size_t)T * d : 0);
+  L.hid = take(enc ? e * (size_t)T * (size_t)max_dff : 0);
+  L.dq = take(4 * (size_t)NK * d);
+  L.dg = take(4 * (size_t)NK * d);
+  L.dout = take(4 * (size_t)NK * d);
+  L.total = off;
+  return L;
+}
+
+struct Plan {
+  rest_dtype dt;
+  const rest_heads* hs;
+  const rest_batch* b;
+  long long T, n_cands, NK;
+  int max_dff, K;
+  std::vector<EncTile> enc_tiles;
+  std::vector<DecTile> dec_tiles;
+  Layout L;
+  int32_t* err;
+};
+
+static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const rest_batch* b,
+                             const rest_enc_layer* layers, int n_layers, int l_switch, const rest_requests* reqs,
+                             int K, bool encoder_runs) {
+  rest_status st = check_heads(dt, hs);
+  if (st != REST_OK) return st;
+  if ((st = check_batch(b, &p.T)) != REST_OK) return st;
+  if ((st = check_layers(layers, n_layers, l_switch, &p.max_dff)) != REST_OK) return st;
+  p.n_cands = 0;
+  if (reqs) {
+    if ((st = check_requests(reqs, b, &p.n_cands)) != REST_OK) return st;
+    if (K < 1 || K > 8) return REST_ERR_INVALID_ARG;
+  }
+  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr;
+  p.NK = p.n_cands * (reqs ? K : 0);
+  if (p.T * (long long)hs->d >= (1LL << 40) || p.NK >= (1LL << 31)) return REST_ERR_UNSUPPORTED;
+  if (encoder_runs) build_enc_tiles(b, p.enc_tiles);
+  build_dec_tiles(b, reqs, K, p.dec_tiles);
+  p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),
+                    (int)p.dec_tiles.size());
+  return REST_OK;
+}
+
+static rest_status check_device() {
+  static int checked[64] = {0};  // 0 unknown, 1 ok, 2 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return REST_ERR_NO_DEVICE; }
+  if (dev < 0 || dev >= 64) return REST_ERR_NO_DEVICE;
+  if (checked[dev] == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return REST_ERR_NO_DEVICE;
+    }
+    checked[dev] = (major == 10) ? 1 : 2;
+  }
+  return checked[dev] == 1 ? REST_OK : REST_ERR_NO_DEVICE;
+}
+
+// ---------------------------------------------------------------- instrumentation
+// When profiling is on, every launch is bracketed by a pair of CUDA events on
+// its own stream and tagged with its algorithmic FLOPs and bytes.
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+static thread_local bool g_prof = false;
+static thread_local std::vector<ProfRec>* g_recs = nullptr;
+static thread_local std::vector<cudaEvent_t>* g_event_pool = nullptr;
+
+static cudaEvent_t prof_event() {
+  if (!g_event_pool) g_event_pool = new std::vector<cudaEvent_t>();
+  if (!g_event_pool->empty()) {
+    cudaEvent_t e = g_event_pool->back();
+    g_event_pool->pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct LaunchScope {
+  ProfRec rec;
+  cudaStream_t s;
+  bool on;
+  LaunchScope(cudaStream_t s_, const char* name, double flops, double bytes) : s(s_), on(g_prof) {
+    ++g_launches;
+    if (on) {
+      rec = ProfRec{name, prof_event(), prof_event(), flops, bytes};
+      cudaEventRecord(rec.a, s);
+    }
+  }
+  void done() {
+    if (on) {
+      cudaEventRecord(rec.b, s);
+      if (!g_recs) g_recs = new std::vector<ProfRec>();
+      g_recs->push_back(rec);
+    }
+  }
+};
+
+#define REST_KLAUNCH(stream, name, flops, bytes, call)        \
+  do {                                                        \
+    LaunchScope sc_((stream), (name), (flops), (bytes));      \
+    cudaError_t e_ = (call);                                  \
+    sc_.done();                                               \
+    if (e_ != cudaSuccess) return REST_ERR_CUDA;              \
+  } while (0)
+
+template <typename P> static inline P* at(void* ws, size_t off) { return reinterpret_cast<P*>((char*)ws + off); }
+
+static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
+  std::vector<char> host(p.L.meta_end, 0);
+  memcpy(host.data() + p.L.cu, p.b->cu_seqlens ? p.b->cu_seqlens : (const int32_t*)"\0\0\0\0",
+         sizeof(int32_t) * (size_t)(p.b->n_users + 1));
+  if (!p.enc_tiles.empty())
+    memcpy(host.data() + p.L.enc_tiles, p.enc_tiles.data(), sizeof(EncTile) * p.enc_tiles.size());
+  if (!p.dec_tiles.empty())
+    memcpy(host.data() + p.L.dec_tiles, p.dec_tiles.data(), sizeof(DecTile) * p.dec_tiles.size());
+  if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) return REST_ERR_CUDA;
+  return REST_OK;
+}
+
+static TableParams table_params(const rest_heads* hs) {
+  TableParams tp;
+  memset(&tp, 0, sizeof(tp));
+  tp.n_heads = hs->n_heads;
+  tp.half = hs->head_dim / 2;
+  for (int h = 0; h < hs->n_heads; ++h) tp.tau[h] = hs->tau[h];
+  for (int j = 0; j < tp.half; ++j) tp.theta[j] = pow(hs->rope_base, -2.0 * j / hs->head_dim);
+  return tp;
+}
+
+static GemmArgs gemm(const void* A, long long lda, const void* B, long long ldb, long long M, int N, int K, int epi,
+                     void* out0, long long ldo) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.A = A; a.lda = lda; a.B = B; a.ldb = ldb; a.M = (int)M; a.N = N; a.K = K; a.epi = epi;
+  a.out0 = out0; a.ldo = ldo;
+  return a;
+}
+
+static double gemm_out_bytes(const GemmArgs& a, size_t e) {
+  double MN = (double)a.M * a.N;
+  switch (a.epi) {
+    case EPI_F32: case EPI_SIGMOID: return 4 * MN;
+    case EPI_DT: return e * MN;
+    case EPI_RESID: return 8 * MN;
+    case EPI_QKVG: return (double)a.M * a.d * (3 * e + 4) + 4.0 * a.M * a.d;  // + cos/sin reads
+    case EPI_SWIGLU: return e * MN / 2;
+  }
+  return 0;
+}
+
+static rest_status run_gemm(const Plan& p, const GemmArgs& a, const char* name, cudaStream_t s) {
+  const bool bf = p.dt == REST_BF16;
+  const size_t e = dt_size(p.dt);
+  const double flops = 2.0 * a.M * a.N * a.K;
+  const double bytes = (a.a_f32 ? 4 : e) * (double)a.M * a.K + e * (double)a.K * a.N + gemm_out_bytes(a, e);
+  if (bf && sm100_gemm_supported(a)) {
+    REST_KLAUNCH(s, name, flops, bytes, launch_gemm_sm100(a, s, p.err));
+  } else {
+    REST_KLAUNCH(s, name, flops, bytes, launch_gemm_simt(bf, a, s));
+  }
+  return REST_OK;
+}
+
+// ---------------------------------------------------------------- encoder
+
+static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, const rest_enc_layer* layers,
+                               int n_layers, int l_switch, void* h_out, void* ws, int32_t* err, cudaStream_t s) {
+  const bool bf = p.dt == REST_BF16;
+  const int d = p.hs->d, hd = p.hs->head_dim, H = p.hs->n_heads;
+  const long long T = p.T;
+  const size_t e = dt_size(p.dt);
+  const double Td = (double)T * d;
+  const Layout& L = p.L;
+  const int32_t* cu = at<int32_t>(ws, L.cu);
+  float* cos_t = at<float>(ws, L.cos_t);
+  float* sin_t = at<float>(ws, L.sin_t);
+  float* xres = at<float>(ws, L.xres);
+  void* y = at<void>(ws, L.y);
+  void *q = at<void>(ws, L.q), *k = at<void>(ws, L.k), *v = at<void>(ws, L.v), *o = at<void>(ws, L.o);
+  float* g = at<float>(ws, L.g);
+  void* hid = at<void>(ws, L.hid);
+
+  double causal_pairs = 0;  // sum over users of L(L+1)/2
+  for (int u = 0; u < p.b->n_users; ++u) {
+    double Lu = p.b->cu_seqlens[u + 1] - p.b->cu_seqlens[u];
+    causal_pairs += Lu * (Lu + 1) / 2;
+  }
+  const double attn_flops = 4.0 * d * causal_pairs;  // QK^T and PV over every head
+  const double attn_bytes = Td * (3 * e + 4 + e);
+
+  TableParams tp = table_params(p.hs);
+  REST_KLAUNCH(s, "rotation_table", 0, 8.0 * T + 4 * Td,
+               launch_rotation_table(ts, cu, p.b->n_users, (int)T, tp, nullptr, cos_t, sin_t, err, s));
+  REST_KLAUNCH(s, "to_f32", 0, Td * (e + 4), launch_to_f32(bf, x, xres, T * d, s));
+
+  EncAttnArgs ea;
+  ea.q = q; ea.k = k; ea.v = v; ea.gate = g; ea.out = o; ea.cu = cu;
+  ea.tiles = at<EncTile>(ws, L.enc_tiles); ea.n_tiles = L.n_enc_tiles;
+  ea.n_heads = H; ea.d = d;
+  ea.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
+
+  for (int l = 0; l < n_layers; ++l) {
+    const rest_enc_layer& Ly = layers[l];
+    const bool post = (l + 1) <= l_switch;  // eq. 6: post-LN for the first l_switch layers
+    // ---- DGA sublayer (eqs. 3-5)
+    REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
+                 launch_layernorm(bf, xres, y, Ly.ln_attn_g, Ly.ln_attn_b, (int)T, d, post ? 2 : 0, s));
+    GemmArgs a = gemm(y, d, Ly.w_qkvgg, 5LL * d, T, 5 * d, d, EPI_QKVG, q, d);
+    a.out1 = k; a.out2 = v; a.out3 = g; a.cos_t = cos_t; a.sin_t = sin_t; a.d = d;
+    if (rest_status st = run_gemm(p, a, "gemm_qkvg", s)) return st;
+    if (bf && sm100_attn_supported(hd)) {
+      REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_sm100(hd, ea, s, err));
+    } else {
+      REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_simt(bf, hd, ea, s));
+    }
+    a = gemm(o, d, Ly.w_o, d, T, d, d, EPI_RESID, xres, d);
+    a.alpha = Ly.alpha_attn;
+    if (rest_status st = run_gemm(p, a, "gemm_attn_out", s)) return st;
+    if (post)
+      REST_KLAUNCH(s, "layernorm", 0, 8 * Td,
+                   launch_layernorm(bf, xres, y, Ly.ln_attn_g, Ly.ln_attn_b, (int)T, d, 3, s));
+    // ---- SwiGLU FFN sublayer
+    if (Ly.w_ffn13) {
+      const int dff = Ly.d_ff;
+      REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
+                   launch_layernorm(bf, xres, y, Ly.ln_ffn_g, Ly.ln_ffn_b, (int)T, d, post ? 2 : 0, s));
+      a = gemm(y, d, Ly.w_ffn13, 2LL * dff, T, 2 * dff, d, EPI_SWIGLU, hid, dff);
+      a.d = dff;
+      if (rest_status st = run_gemm(p, a, "gemm_ffn13", s)) return st;
+      a = gemm(hid, dff, Ly.w_ffn2, d, T, d, dff, EPI_RESID, xres, d);
+      a.alpha = Ly.alpha_ffn;
+      if (rest_status st = run_gemm(p, a, "gemm_ffn2", s)) return st;
+      if (post)
+        REST_KLAUNCH(s, "layernorm", 0, 8 * Td,
+                     launch_layernorm(bf, xres, y, Ly.ln_ffn_g, Ly.ln_ffn_b, (int)T, d, 3, s));
+    }
+  }
+  // H: the residual stream after the last layer, in the call's dtype (no final norm)
+  REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
+               launch_layernorm(bf, xres, h_out, nullptr, nullptr, (int)T, d, 2, s));
+  return REST_OK;
+}
+
+// ---------------------------------------------------------------- decoder
+
+static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const void* h, const void* z,
+                               const rest_dec_params* dec, float* y_out, void* ws, int32_t* err, cudaStream_t s) {
+  const bool bf = p.dt == REST_BF16;
+  const int d = p.hs->d, hd = p.hs->head_dim, K = dec->K;
+  const size_t e = dt_size(p.dt);
+  const Layout& L = p.L;
+  float* dq = at<float>(ws, L.dq);
+  float* dg = at<float>(ws, L.dg);
+  float* dout = at<float>(ws, L.dout);
+  const long long N = p.n_cands;
+  // token-specific projections (eq. 8): rows n*K + k use W_Q^(k), W_go^(k)
+  for (int kk = 0; kk < K; ++kk) {
+    const char* zk = (const char*)z + e * (size_t)kk * d;
+    GemmArgs a = gemm(zk, (long long)K * d, (const char*)dec->w_q + e * (size_t)kk * d * d, d, N, d, d, EPI_F32,
+                      dq + (size_t)kk * d, (long long)K * d);
+    if (rest_status st = run_gemm(p, a, "gemm_dec_q", s)) return st;
+    a = gemm(zk, (long long)K * d, (const char*)dec->w_go + e * (size_t)kk * d * d, d, N, d, d, EPI_SIGMOID,
+             dg + (size_t)kk * d, (long long)K * d);
+    if (rest_status st = run_gemm(p, a, "gemm_dec_g", s)) return st;
+  }
+  // every H prefix is read once per request; each candidate row reads q, g and writes o
+  double flops = 0, hbytes = 0;
+  for (int r = 0; r < reqs->n_req; ++r) {
+    double rows = (double)(reqs->cu_cands[r + 1] - reqs->cu_cands[r]) * K;
+    if (rows == 0) continue;
+    flops += 4.0 * d * rows * reqs->req_cutoff[r];
+    hbytes += (double)e * reqs->req_cutoff[r] * d;
+  }
+  const double bytes = hbytes + (double)p.NK * d * 12;
+  DecAttnArgs da;
+  da.q = dq; da.g = dg; da.h = h; da.out = dout;
+  da.tiles = at<DecTile>(ws, L.dec_tiles); da.n_tiles = L.n_dec_tiles;
+  da.n_heads = p.hs->n_heads; da.d = d;
+  da.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
+  if (bf && sm100_attn_supported(hd)) {
+    REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_sm100(hd, da, s, err));
+  } else {
+    REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_simt(bf, hd, da, s));
+  }
+  GemmArgs a = gemm(dout, d, dec->w_o, d, p.NK, d, d, EPI_F32, y_out, d);
+  a.a_f32 = 1;
+  if (rest_status st = run_gemm(p, a, "gemm_dec_out", s)) return st;
+  return REST_OK;
+}
+
+}  // namespace rest
+
+using namespace rest;
+
+extern "C" {
+
+const char* rest_status_string(rest_status s) {
+  switch (s) {
+    case REST_OK: return "ok";
+    case REST_ERR_INVALID_ARG: return "invalid argument";
+    case REST_ERR_UNSORTED_TIME: return "timestamps decrease within a user";
+    case REST_ERR_UNSUPPORTED: return "unsupported shape";
+    case REST_ERR_CUDA: return "CUDA runtime error";
+    case REST_ERR_TIMEOUT: return "bounded device wait ran out";
+    case REST_ERR_WORKSPACE: return "workspace missing or too small";
+    case REST_ERR_NO_DEVICE: return "no sm_100 CUDA device is current";
+  }
+  return "unknown status";
+}
+
+void rest_profile_begin(void) {
+  g_prof = true;
+  if (!g_recs) g_recs = new std::vector<ProfRec>();
+  g_recs->clear();
+}
+
+int rest_profile_end(rest_kernel_stat* out, int max_out) {
+  g_prof = false;
+  if (!g_recs) return 0;
+  std::vector<rest_kernel_stat> agg;
+  for (ProfRec& r : *g_recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+      cudaGetLastError();
+      ms = 0.f;
+    }
+    size_t i = 0;
+    while (i < agg.size() && strcmp(agg[i].name, r.name) != 0) ++i;
+    if (i == agg.size()) agg.push_back(rest_kernel_stat{r.name, 0, 0.0, 0.0, 0.0});
+    agg[i].launches += 1;
+    agg[i].ms += ms;
+    agg[i].flops += r.flops;
+    agg[i].bytes += r.bytes;
+    if (!g_event_pool) g_event_pool = new std::vector<cudaEvent_t>();
+    g_event_pool->push_back(r.a);
+    g_event_pool->push_back(r.b);
+  }
+  g_recs->clear();
+  int n = (int)agg.size();
+  for (int i = 0; i < n && i < max_out; ++i) out[i] = agg[i];
+  return n;
+}
+
+long long rest_launch_count(int reset) {
+  long long v = g_launches;
+  if (reset) g_launches = 0;
+  return v;
+}
+
+rest_status rest_workspace_size(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                const rest_enc_layer* layers, int n_layers, const rest_requests* reqs, int K,
+                                size_t* bytes) {
+  if (!bytes) return REST_ERR_INVALID_ARG;
+  try {
+    Plan p;
+    rest_status st = make_plan(p, dt, heads, batch, layers, n_layers, n_layers, reqs, K,
+                               n_layers > 0 || !reqs);
+    if (st != REST_OK) return st;
+    *bytes = p.L.total;
+    return REST_OK;
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_rotation_table(const rest_heads* heads, const rest_batch* batch, const int64_t* ts,
+                                int64_t* idx_out, float* cos_out, float* sin_out, void* ws, size_t ws_bytes,
+                                int32_t* dev_err, void* stream) {
+  try {
+    Plan p;
+    rest_status st = make_plan(p, REST_F32, heads, batch, nullptr, 0, 0, nullptr, 1, true);
+    if (st != REST_OK) return st;
+    if ((cos_out == nullptr) != (sin_out == nullptr)) return REST_ERR_INVALID_ARG;
+    if (p.T > 0 && !ts) return REST_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < p.L.total) return REST_ERR_WORKSPACE;
+    if (p.T == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    TableParams tp = table_params(heads);
+    REST_KLAUNCH(s, "rotation_table", 0, 8.0 * p.T + 4.0 * p.T * heads->d,
+                 launch_rotation_table(ts, at<int32_t>(ws, p.L.cu), batch->n_users, (int)p.T, tp, idx_out, cos_out,
+                                       sin_out, dev_err, s));
+    return REST_OK;
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_encoder_attn(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, const void* x,
+                              const int64_t* ts, const rest_enc_layer* layers, int n_layers, int l_switch,
+                              void* h_out, void* ws, size_t ws_bytes, int32_t* dev_err, void* stream) {
+  try {
+    Plan p;
+    rest_status st = make_plan(p, dt, heads, batch, layers, n_layers, l_switch, nullptr, 1, true);
+    if (st != REST_OK) return st;
+    if (p.T > 0 && (!x || !ts || !h_out || !aligned16(x) || !aligned16(ts) || !aligned16(h_out)))
+      return REST_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < p.L.total || !aligned16(ws)) return REST_ERR_WORKSPACE;
+    if (p.T == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    return run_encoder(p, x, ts, layers, n_layers, l_switch, h_out, ws, dev_err, s);
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_cross_decode(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, const void* h,
+                              const rest_requests* reqs, const void* z, const rest_dec_params* dec, float* y_out,
+                              void* ws, size_t ws_bytes, int32_t* dev_err, void* stream) {
+  try {
+    rest_status st = check_dec(dec);
+    if (st != REST_OK) return st;
+    if (!reqs) return REST_ERR_INVALID_ARG;
+    Plan p;
+    if ((st = make_plan(p, dt, heads, batch, nullptr, 0, 0, reqs, dec->K, false)) != REST_OK) return st;
+    if (p.NK > 0 && (!h || !z || !y_out || !aligned16(h) || !aligned16(z) || !aligned16(y_out)))
+      return REST_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < p.L.total || !aligned16(ws)) return REST_ERR_WORKSPACE;
+    if (p.NK == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    return run_decoder(p, reqs, h, z, dec, y_out, ws, dev_err, s);
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, const void* x,
+                              const int64_t* ts, const rest_enc_layer* layers, int n_layers, int l_switch,
+                              const rest_requests* reqs, const void* z, const rest_dec_params* dec, void* h_out,
+                              float* y_out, void* ws, size_t ws_bytes, int32_t* dev_err, void* stream) {
+  try {
+    rest_status st = check_dec(dec);
+    if (st != REST_OK) return st;
+    if (!reqs) return REST_ERR_INVALID_ARG;
+    Plan p;
+    if ((st = make_plan(p, dt, heads, batch, layers, n_layers, l_switch, reqs, dec->K, true)) != REST_OK) return st;
+    if (p.T > 0 && (!x || !ts || !h_out || !aligned16(x) || !aligned16(ts) || !aligned16(h_out)))
+      return REST_ERR_INVALID_ARG;
+    if (p.NK > 0 && (!z || !y_out || !aligned16(z) || !aligned16(y_out))) return REST_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < p.L.total || !aligned16(ws)) return REST_ERR_WORKSPACE;
+    if (p.T == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    if ((st = run_encoder(p, x, ts, layers, n_layers, l_switch, h_out, ws, dev_err, s)) != REST_OK) return st;
+    if (p.NK == 0) return REST_OK;
+    return run_decoder(p, reqs, h_out, z, dec, y_out, ws, dev_err, s);
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+}  // extern "C"

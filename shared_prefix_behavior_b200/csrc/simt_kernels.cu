@@ -1,0 +1,471 @@
+// Plain CUDA-core kernels of the ReST forward: the rotation table, LayerNorm,
+// a tiled fp32-accumulating GEMM with the fused epilogues of the encoder and
+// decoder, and a thread-per-query-row flash attention for the causal
+// encoder and the shared-prefix decoder. These carry the fp32 path (the
+// tolerance there, 1e-4, rules out tf32/bf16 tensor cores) and every shape
+// the tensor-core kernels do not cover.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rest {
+
+// ============================================================================
+// Rotation index and cos/sin table (ReST §3.2.2, bucket definition and eq. 5)
+// ============================================================================
+
+__device__ __forceinline__ int find_user(const int32_t* cu, int n_users, int i) {
+  // largest u with cu[u] <= i (empty users share their start with the next one)
+  int lo = 0, hi = n_users;  // invariant: cu[lo] <= i < cu[hi]
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (cu[mid] <= i) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu,
+                                      int n_users, int T, TableParams p, int64_t* idx_out,
+                                      float* cos_out, float* sin_out, int32_t* err) {
+  long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)T * p.n_heads) return;
+  int i = (int)(gid / p.n_heads), h = (int)(gid % p.n_heads);
+  int s = cu[find_user(cu, n_users, i)];
+  long long t = ts[i];
+  if (h == 0 && i > s && ts[i - 1] > t) set_error(err, REST_ERR_UNSORTED_TIME);
+  long long tau = p.tau[h];
+  long long idx;
+  if (tau == 0) {
+    idx = i - s;
+  } else {
+    long long rel = t - ts[s];           // exact int64
+    long long q = rel / tau;             // floor division (rel < 0 only on invalid input)
+    if ((rel % tau != 0) && (rel < 0)) q -= 1;
+    idx = q;
+  }
+  if (idx_out) idx_out[gid] = idx;
+  if (cos_out) {
+    float* cp = cos_out + gid * p.half;
+    float* sp = sin_out + gid * p.half;
+    for (int j = 0; j < p.half; ++j) {
+      double phi = (double)idx * p.theta[j];
+      double sv, cv;
+      sincos(phi, &sv, &cv);
+      cp[j] = (float)cv;
+      sp[j] = (float)sv;
+    }
+  }
+}
+
+cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users, int T,
+                                    const TableParams& p, int64_t* idx_out, float* cos_out,
+                                    float* sin_out, int32_t* err, cudaStream_t s) {
+  long long n = (long long)T * p.n_heads;
+  if (n == 0) return cudaSuccess;
+  int threads = 256;
+  long long blocks = (n + threads - 1) / threads;
+  rotation_table_kernel<<<(unsigned)blocks, threads, 0, s>>>(ts, cu, n_users, T, p, idx_out, cos_out,
+                                                             sin_out, err);
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// LayerNorm / casts (ReST §3.2.3, eq. 6)
+// ============================================================================
+
+template <typename T>
+__global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
+                                 const float* __restrict__ b, int rows, int d, int mode) {
+  constexpr int VMAX = 32;  // d <= 1024
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  float* xr = x + (long long)warp * d;
+  float v[VMAX];
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < VMAX; ++k) {
+    int c = k * 32 + lane;
+    v[k] = (c < d) ? xr[c] : 0.f;
+    sum += v[k];
+  }
+  if (mode == 2) {
+    T* yr = y + (long long)warp * d;
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k) {
+      int c = k * 32 + lane;
+      if (c < d) yr[c] = from_f<T>(v[k]);
+    }
+    return;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  float mean = sum / d;
+  float sq = 0.f;
+#pragma unroll
+  for (int k = 0; k < VMAX; ++k) {
+    int c = k * 32 + lane;
+    float t = (c < d) ? v[k] - mean : 0.f;
+    sq += t * t;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  float rstd = 1.0f / sqrtf(sq / d + 1e-5f);
+#pragma unroll
+  for (int k = 0; k < VMAX; ++k) {
+    int c = k * 32 + lane;
+    if (c < d) {
+      float n = (v[k] - mean) * rstd * g[c] + b[c];
+      if (mode == 1 || mode == 3) xr[c] = n;
+      if (mode != 3) y[(long long)warp * d + c] = from_f<T>(n);
+    }
+  }
+}
+
+cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, const float* b, int T, int d,
+                             int mode, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  int threads = 256;
+  int blocks = (T * 32 + threads - 1) / threads;
+  if (bf16m)
+    layernorm_kernel<bf16><<<blocks, threads, 0, s>>>(x, (bf16*)y, g, b, T, d, mode);
+  else
+    layernorm_kernel<float><<<blocks, threads, 0, s>>>(x, (float*)y, g, b, T, d, mode);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, long long n) {
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = to_f<T>(in[i]);
+}
+
+cudaError_t launch_to_f32(bool bf16m, const void* x_in, float* x_res, long long n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  int threads = 256;
+  long long blocks = (n + threads - 1) / threads;
+  if (bf16m)
+    to_f32_kernel<bf16><<<(unsigned)blocks, threads, 0, s>>>((const bf16*)x_in, x_res, n);
+  else
+    to_f32_kernel<float><<<(unsigned)blocks, threads, 0, s>>>((const float*)x_in, x_res, n);
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// Tiled GEMM with the fused epilogues
+// ============================================================================
+
+// Physical column of logical column n for the interleaved epilogues: every
+// group of 4 logical columns is (2p, 2p+1) of block one and (2p, 2p+1) of
+// block two, the blocks `width` columns apart starting at `base`.
+__device__ __forceinline__ int interleave_col(int n, int base, int width) {
+  int r = n - base, p = r >> 2, w = r & 3;
+  return base + (w < 2 ? 2 * p + w : width + 2 * p + w - 2);
+}
+
+__device__ __forceinline__ int physical_col(const GemmArgs& a, int n) {
+  if (a.epi == EPI_QKVG) {
+    if (n >= 2 * a.d && n < 4 * a.d) return interleave_col(n, 2 * a.d, a.d);
+    return n;
+  }
+  if (a.epi == EPI_SWIGLU) return interleave_col(n, 0, a.d);
+  return n;
+}
+
+// TA: type of A; T: the call's dtype (B and the dtype outputs).
+template <typename TA, typename T>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
+  constexpr int BM = 64, BN = 64, BK = 16;
+  __shared__ __align__(16) float As[BK][BM + 4];
+  __shared__ __align__(16) float Bs[BK][BN];
+  const TA* A = (const TA*)a.A;
+  const T* B = (const T*)a.B;
+  int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  int ar = tid >> 2, ak = (tid & 3) * 4;
+  int bk = tid >> 4, bn = (tid & 15) * 4;
+  int bcol[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int ln = n0 + bn + i;
+    bcol[i] = (ln < a.N) ? physical_col(a, ln) : -1;
+  }
+  for (int k0 = 0; k0 < a.K; k0 += BK) {
+    float av[4] = {0.f, 0.f, 0.f, 0.f};
+    int gm = m0 + ar;
+    if (gm < a.M) load4(A + (long long)gm * a.lda + k0 + ak, av);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) As[ak + i][ar] = av[i];
+    const T* brow = B + (long long)(k0 + bk) * a.ldb;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) Bs[bk][bn + i] = (bcol[i] >= 0) ? to_f<T>(brow[bcol[i]]) : 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float4 a4 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      float4 b4 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      float av2[4] = {a4.x, a4.y, a4.z, a4.w}, bv2[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av2[i], bv2[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+
+  int n = n0 + tx * 4;
+  if (n >= a.N) return;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int m = m0 + ty * 4 + i;
+    if (m >= a.M) break;
+    float* c = acc[i];
+    long long ro = (long long)m * a.ldo;
+    switch (a.epi) {
+      case EPI_F32: store4((float*)a.out0 + ro + n, c); break;
+      case EPI_DT: store4((T*)a.out0 + ro + n, c); break;
+      case EPI_SIGMOID: {
+        float v[4] = {sigmoid_f(c[0]), sigmoid_f(c[1]), sigmoid_f(c[2]), sigmoid_f(c[3])};
+        store4((float*)a.out0 + ro + n, v);
+        break;
+      }
+      case EPI_RESID: {
+        float* p = (float*)a.out0 + ro + n;
+        float v[4];
+        load4(p, v);
+        for (int j = 0; j < 4; ++j) v[j] = fmaf(a.alpha, c[j], v[j]);
+        store4(p, v);
+        break;
+      }
+      case EPI_QKVG: {
+        int d = a.d;
+        if (n < 2 * d) {  // Q or K: rotate the pairs (eq. 5)
+          int col = n < d ? n : n - d;
+          const float* ct = a.cos_t + (long long)m * (d / 2) + col / 2;
+          const float* st = a.sin_t + (long long)m * (d / 2) + col / 2;
+          float v[4];
+          v[0] = c[0] * ct[0] - c[1] * st[0];
+          v[1] = c[0] * st[0] + c[1] * ct[0];
+          v[2] = c[2] * ct[1] - c[3] * st[1];
+          v[3] = c[2] * st[1] + c[3] * ct[1];
+          store4((T*)(n < d ? a.out0 : a.out1) + ro + col, v);
+        } else if (n < 4 * d) {  // value gate: V' = sigmoid(Gv) * V (eq. 3)
+          int col = ((n - 2 * d) >> 2) * 2;
+          store2((T*)a.out2 + ro + col, c[0] * sigmoid_f(c[2]), c[1] * sigmoid_f(c[3]));
+        } else {  // output gate sigmoid(Go) (eq. 4), kept in fp32
+          float v[4] = {sigmoid_f(c[0]), sigmoid_f(c[1]), sigmoid_f(c[2]), sigmoid_f(c[3])};
+          store4((float*)a.out3 + ro + (n - 4 * d), v);
+        }
+        break;
+      }
+      case EPI_SWIGLU: {
+        int col = (n >> 2) * 2;
+        store2((T*)a.out0 + ro + col, c[0] * sigmoid_f(c[0]) * c[2], c[1] * sigmoid_f(c[1]) * c[3]);
+        break;
+      }
+    }
+  }
+}
+
+cudaError_t launch_gemm_simt(bool bf16m, const GemmArgs& a, cudaStream_t s) {
+  if (a.M == 0 || a.N == 0) return cudaSuccess;
+  dim3 grid((a.N + 63) / 64, (a.M + 63) / 64);
+  if (bf16m && a.a_f32)
+    gemm_simt_kernel<float, bf16><<<grid, 256, 0, s>>>(a);
+  else if (bf16m)
+    gemm_simt_kernel<bf16, bf16><<<grid, 256, 0, s>>>(a);
+  else
+    gemm_simt_kernel<float, float><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// Attention: one thread per query row, K/V tiles staged in shared memory.
+// Online softmax in base 2 (scores pre-scaled by log2(e)/sqrt(head_dim)).
+// ============================================================================
+
+template <int HD>
+struct RowState {
+  float q[HD];
+  float o[HD];
+  float m, l;
+};
+
+template <typename T, int HD, int BK>
+__device__ __forceinline__ void stage_kv(float (*Ks)[HD], float (*Vs)[HD], const T* kbase, const T* vbase,
+                                         long long ld, int nvalid) {
+  for (int e = threadIdx.x * 4; e < BK * HD; e += blockDim.x * 4) {
+    int r = e / HD, c = e % HD;
+    float kv[4] = {0.f, 0.f, 0.f, 0.f}, vv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (r < nvalid) {
+      load4(kbase + r * ld + c, kv);
+      load4(vbase + r * ld + c, vv);
+    }
+    *reinterpret_cast<float4*>(&Ks[r][c]) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+    *reinterpret_cast<float4*>(&Vs[r][c]) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+  }
+}
+
+// Process one staged tile for one row: keys j < jmax are visible.
+template <int HD, int BK>
+__device__ __forceinline__ void row_tile(RowState<HD>& st, const float (*Ks)[HD], const float (*Vs)[HD], int jmax) {
+  float sc[BK];
+  float mt = st.m;
+#pragma unroll
+  for (int j = 0; j < BK; ++j) {
+    float dot = 0.f;
+#pragma unroll
+    for (int c = 0; c < HD; c += 4) {
+      float4 k4 = *reinterpret_cast<const float4*>(&Ks[j][c]);
+      dot = fmaf(st.q[c], k4.x, dot);
+      dot = fmaf(st.q[c + 1], k4.y, dot);
+      dot = fmaf(st.q[c + 2], k4.z, dot);
+      dot = fmaf(st.q[c + 3], k4.w, dot);
+    }
+    sc[j] = (j < jmax) ? dot : -INFINITY;
+    mt = fmaxf(mt, sc[j]);
+  }
+  float alpha = exp2_approx(st.m - mt);
+  st.l *= alpha;
+#pragma unroll
+  for (int c = 0; c < HD; ++c) st.o[c] *= alpha;
+  st.m = mt;
+#pragma unroll
+  for (int j = 0; j < BK; ++j) {
+    float p = exp2_approx(sc[j] - mt);
+    st.l += p;
+#pragma unroll
+    for (int c = 0; c < HD; c += 4) {
+      float4 v4 = *reinterpret_cast<const float4*>(&Vs[j][c]);
+      st.o[c] = fmaf(p, v4.x, st.o[c]);
+      st.o[c + 1] = fmaf(p, v4.y, st.o[c + 1]);
+      st.o[c + 2] = fmaf(p, v4.z, st.o[c + 2]);
+      st.o[c + 3] = fmaf(p, v4.w, st.o[c + 3]);
+    }
+  }
+}
+
+template <typename T, int HD>
+__device__ __forceinline__ void load_q(RowState<HD>& st, const T* q, float scale) {
+#pragma unroll
+  for (int c = 0; c < HD; c += 4) {
+    float v[4];
+    load4(q + c, v);
+    st.q[c] = v[0] * scale; st.q[c + 1] = v[1] * scale; st.q[c + 2] = v[2] * scale; st.q[c + 3] = v[3] * scale;
+  }
+#pragma unroll
+  for (int c = 0; c < HD; ++c) st.o[c] = 0.f;
+  st.m = -INFINITY;
+  st.l = 0.f;
+}
+
+template <typename T, int HD>
+__device__ __forceinline__ void store_row(const RowState<HD>& st, const float* gate, T* out) {
+  float inv = 1.0f / st.l;
+#pragma unroll
+  for (int c = 0; c < HD; c += 4) {
+    float g[4];
+    load4(gate + c, g);
+    float v[4] = {st.o[c] * inv * g[0], st.o[c + 1] * inv * g[1], st.o[c + 2] * inv * g[2], st.o[c + 3] * inv * g[3]};
+    store4(out + c, v);
+  }
+}
+
+constexpr int ATT_ROWS = 128;  // query rows per block (one per thread)
+constexpr int ATT_BK = 16;     // keys per staged tile
+
+template <typename T, int HD>
+__global__ void __launch_bounds__(ATT_ROWS) enc_attn_simt_kernel(EncAttnArgs a) {
+  __shared__ __align__(16) float Ks[ATT_BK][HD];
+  __shared__ __align__(16) float Vs[ATT_BK][HD];
+  EncTile tile = a.tiles[blockIdx.x];
+  int h = blockIdx.y;
+  int s = a.cu[tile.user];
+  int L = a.cu[tile.user + 1] - s;
+  int i = tile.q0 + threadIdx.x;
+  bool valid = i < L;
+  long long hoff = (long long)h * HD;
+  RowState<HD> st;
+  load_q<T, HD>(st, (const T*)a.q + (long long)(s + (valid ? i : 0)) * a.d + hoff, a.scale_log2);
+  int kv_end = min(L, tile.q0 + ATT_ROWS);
+  const T* K = (const T*)a.k + (long long)s * a.d + hoff;
+  const T* V = (const T*)a.v + (long long)s * a.d + hoff;
+  for (int kb = 0; kb < kv_end; kb += ATT_BK) {
+    __syncthreads();
+    stage_kv<T, HD, ATT_BK>(Ks, Vs, K + (long long)kb * a.d, V + (long long)kb * a.d, a.d, kv_end - kb);
+    __syncthreads();
+    if (valid && kb <= i) row_tile<HD, ATT_BK>(st, Ks, Vs, i - kb + 1);  // causal: key <= i
+  }
+  if (valid) {
+    long long ro = (long long)(s + i) * a.d + hoff;
+    store_row<T, HD>(st, a.gate + ro, (T*)a.out + ro);
+  }
+}
+
+template <typename T, int HD>
+__global__ void __launch_bounds__(ATT_ROWS) dec_attn_simt_kernel(DecAttnArgs a) {
+  __shared__ __align__(16) float Ks[ATT_BK][HD];
+  __shared__ __align__(16) float Vs[ATT_BK][HD];
+  DecTile tile = a.tiles[blockIdx.x];
+  int h = blockIdx.y;
+  long long hoff = (long long)h * HD;
+  bool valid = threadIdx.x < tile.nrows;
+  long long row = tile.row0 + (valid ? threadIdx.x : 0);
+  RowState<HD> st;
+  load_q<float, HD>(st, a.q + row * a.d + hoff, a.scale_log2);
+  const T* Hm = (const T*)a.h + (long long)tile.key0 * a.d + hoff;
+  for (int kb = 0; kb < tile.nkeys; kb += ATT_BK) {
+    __syncthreads();
+    // keys and values are the same rows of H (projection-free, ReST eq. 7)
+    stage_kv<T, HD, ATT_BK>(Ks, Vs, Hm + (long long)kb * a.d, Hm + (long long)kb * a.d, a.d, tile.nkeys - kb);
+    __syncthreads();
+    if (valid) row_tile<HD, ATT_BK>(st, Ks, Vs, tile.nkeys - kb);
+  }
+  if (valid) {
+    long long ro = row * a.d + hoff;
+    store_row<float, HD>(st, a.g + ro, a.out + ro);
+  }
+}
+
+template <typename T>
+static cudaError_t enc_dispatch(int hd, const EncAttnArgs& a, cudaStream_t s) {
+  dim3 grid(a.n_tiles, a.n_heads);
+  switch (hd) {
+    case 16: enc_attn_simt_kernel<T, 16><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    case 32: enc_attn_simt_kernel<T, 32><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    case 64: enc_attn_simt_kernel<T, 64><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t dec_dispatch(int hd, const DecAttnArgs& a, cudaStream_t s) {
+  dim3 grid(a.n_tiles, a.n_heads);
+  switch (hd) {
+    case 16: dec_attn_simt_kernel<T, 16><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    case 32: dec_attn_simt_kernel<T, 32><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    case 64: dec_attn_simt_kernel<T, 64><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_enc_attn_simt(bool bf16m, int hd, const EncAttnArgs& a, cudaStream_t s) {
+  if (a.n_tiles == 0) return cudaSuccess;
+  return bf16m ? enc_dispatch<bf16>(hd, a, s) : enc_dispatch<float>(hd, a, s);
+}
+
+cudaError_t launch_dec_attn_simt(bool bf16m, int hd, const DecAttnArgs& a, cudaStream_t s) {
+  if (a.n_tiles == 0) return cudaSuccess;
+  return bf16m ? dec_dispatch<bf16>(hd, a, s) : dec_dispatch<float>(hd, a, s);
+}
+
+}  // namespace rest

@@ -1,0 +1,152 @@
+"""The C-ABI library loads, exports what include/rest.h declares, and rejects
+invalid arguments on the host before touching a GPU (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import shared_prefix_behavior_b200 as R
+import workloads as W
+from tests.conftest import gpu_available
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "rest.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rest_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "rest_encoder_attn" in names and "rest_cross_decode" in names and "rest_rank_request" in names
+    lib = ctypes.CDLL(R.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(R.EXPORTS) <= set(names)
+
+
+def test_status_strings():
+    for code in range(8):
+        assert R.library().rest_status_string(code)
+    assert R.library().rest_status_string(0) == b"ok"
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced on the host
+
+
+def _heads(taus, d, base=10000.0):
+    taus = np.asarray(taus, dtype=np.int64)
+    return taus, R.Heads(d, len(taus), d // len(taus), taus.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), base)
+
+
+def _batch(cu):
+    cu = np.asarray(cu, dtype=np.int32)
+    return cu, R.Batch(len(cu) - 1, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+
+
+def _layer(d, dff=0):
+    return R.EncLayer(FAKE, FAKE, FAKE if dff else None, FAKE if dff else None, FAKE, FAKE, FAKE, FAKE, 0.1, 0.1, dff)
+
+
+def _enc(dt=R.REST_BF16, taus=(0, 0, 1, 64), d=64, cu=(0, 10, 30), layers=None, l_switch=0, x=FAKE, ts=FAKE,
+         out=FAKE, ws=FAKE, ws_bytes=1 << 40, base=10000.0):
+    t, hs = _heads(taus, d, base)
+    c, b = _batch(cu)
+    if layers is None:
+        layers = [_layer(d, 192)]
+    arr = (R.EncLayer * max(1, len(layers)))(*layers)
+    return R.library().rest_encoder_attn(dt, ctypes.byref(hs), ctypes.byref(b), x, ts, arr, len(layers), l_switch,
+                                         out, ws, ws_bytes, None, None)
+
+
+def _reqs(u, c, cc):
+    u, c, cc = (np.asarray(a, dtype=np.int32) for a in (u, c, cc))
+    P = ctypes.POINTER(ctypes.c_int32)
+    return (u, c, cc), R.Requests(len(u), u.ctypes.data_as(P), c.ctypes.data_as(P), cc.ctypes.data_as(P))
+
+
+def _dec_call(dt=R.REST_BF16, cu=(0, 10, 30), req=((0, 1), (10, 5), (0, 4, 6)), K=3, d=64, ws_bytes=1 << 40,
+              wq=FAKE):
+    t, hs = _heads((0, 0, 1, 64), d)
+    c, b = _batch(cu)
+    keep, rq = _reqs(*req)
+    dp = R.DecParams(K, wq, FAKE, FAKE)
+    return R.library().rest_cross_decode(dt, ctypes.byref(hs), ctypes.byref(b), FAKE, ctypes.byref(rq), FAKE,
+                                         ctypes.byref(dp), FAKE, FAKE, ws_bytes, None, None)
+
+
+INVALID, UNSUPPORTED, WORKSPACE, NO_DEVICE = 1, 3, 6, 7
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=60), INVALID),                       # d != n_heads * head_dim
+    (dict(taus=(0, 0, -1, 64)), INVALID),        # negative granularity
+    (dict(taus=(0, 0, 0)), INVALID),             # 64 / 3 heads
+    (dict(dt=7), INVALID),
+    (dict(cu=(1, 10)), INVALID),                 # cu_seqlens[0] != 0
+    (dict(cu=(0, 10, 5)), INVALID),              # decreasing
+    (dict(l_switch=2), INVALID),                 # l_switch > n_layers
+    (dict(x=FAKE + 4), INVALID),                 # misaligned
+    (dict(ts=None), INVALID),
+    (dict(layers=[_layer(64, 100)]), INVALID),   # d_ff not a multiple of 64
+    (dict(base=-1.0), INVALID),
+    (dict(d=4 * 24, taus=(0, 0, 1, 64)), UNSUPPORTED),  # head_dim 24
+    (dict(ws_bytes=1000), WORKSPACE),
+    (dict(ws=None), WORKSPACE),
+])
+def test_encoder_rejects_invalid_arguments(kw, code):
+    assert _enc(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(req=((0, 2), (10, 5), (0, 4, 6))), INVALID),   # user out of range
+    (dict(req=((0, 1), (11, 5), (0, 4, 6))), INVALID),   # cutoff > L_u
+    (dict(req=((0, 1), (0, 5), (0, 4, 6))), INVALID),    # cutoff 0
+    (dict(req=((0, 1), (10, 5), (0, 4, 3))), INVALID),   # cu_cands decreasing
+    (dict(req=((0, 1), (10, 5), (1, 4, 6))), INVALID),   # cu_cands[0] != 0
+    (dict(K=0), INVALID),
+    (dict(K=9), INVALID),
+    (dict(wq=None), INVALID),
+    (dict(ws_bytes=16), WORKSPACE),
+])
+def test_decoder_rejects_invalid_arguments(kw, code):
+    assert _dec_call(**kw) == code
+
+
+def test_empty_work_is_a_successful_noop():
+    assert _enc(cu=(0,)) == 0                           # no users
+    assert _enc(cu=(0, 0, 0)) == 0                      # users without tokens
+    assert _dec_call(req=((0, 1), (10, 5), (0, 0, 0))) == 0   # no candidates
+    assert _dec_call(req=((), (), (0,))) == 0            # no requests
+
+
+@pytest.mark.skipif(gpu_available(), reason="checks the no-GPU status")
+def test_valid_call_without_gpu_reports_no_device():
+    assert _enc() == NO_DEVICE
+    assert _dec_call() == NO_DEVICE
+
+
+def test_workspace_size_grows_with_the_batch():
+    for i in (0, 1, 4):
+        w = W.workload(i)
+        cu = np.concatenate([[0], np.cumsum(w.lengths)]).astype(np.int32)
+        cc = np.concatenate([[0], np.cumsum(w.req_ncand)]).astype(np.int32)
+        nb = R.workspace_size(R.REST_BF16 if w.dtype == "bf16" else R.REST_F32, w.taus, w.d, cu, (),
+                              (w.req_user, w.req_cutoff, cc), 3)
+        e = 2 if w.dtype == "bf16" else 4
+        assert nb >= w.total_cands * 3 * w.d * (2 * e + 4)
+
+
+def test_rank_request_host_validation():
+    t, hs = _heads((0, 0, 1, 64), 64)
+    c, b = _batch((0, 10, 30))
+    keep, rq = _reqs((0, 1), (10, 21), (0, 4, 6))   # cutoff 21 > 20
+    arr = (R.EncLayer * 1)(_layer(64, 192))
+    dp = R.DecParams(3, FAKE, FAKE, FAKE)
+    st = R.library().rest_rank_request(R.REST_BF16, ctypes.byref(hs), ctypes.byref(b), FAKE, FAKE, arr, 1, 0,
+                                       ctypes.byref(rq), FAKE, ctypes.byref(dp), FAKE, FAKE, FAKE, 1 << 40, None, None)
+    assert st == INVALID

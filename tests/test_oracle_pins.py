@@ -338,3 +338,11 @@ def test_named_workloads_are_well_formed():
     assert list(W.workload(1).taus) == [0, 0, 0, 0, 1, 4096, 524288, 33554432]
     assert list(W.workload(0).taus) == [0, 0, 64, 65536]
     assert [W.ffn_width(d) for d in (64, 256, 512)] == [192, 704, 1408]
+
+
+@pytest.mark.parametrize("l_switch,ffn", [(0, True), (1, True), (0, False)])
+def test_row_sampled_encoder_equals_full_encoder(l_switch, ffn):
+    w, inp = tiny_inputs(seed=21, lengths=(40, 23), d=32, n_heads=4, n_layers=1, l_switch=l_switch, ffn=ffn)
+    full = O.encoder(inp)
+    rows = [0, 5, 39, 40, 41, 62]
+    assert rel_err(O.encoder_rows(inp, rows), full[rows]) < 1e-13
