@@ -1,6 +1,6 @@
 """Build the in-tree CUDA library librest_b200.so for sm_100a.
 
-    python -m shared_prefix_behavior_b200.build [--verbose]
+    python shared_prefix_behavior_b200/build.py [--verbose] [--ptxas]
 
 Each .cu under csrc/ compiles to an object under _build/ (rebuilt when it or
 any header is newer), then all link into one shared library next to this
