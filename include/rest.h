@@ -161,6 +161,38 @@ rest_status rest_cross_decode(rest_dtype dt, const rest_heads* heads, const rest
                               const rest_dec_params* dec, float* y_out,
                               void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
+/* Size in bytes of the scratch array that rest_cross_decode_static_ws uses. */
+#define REST_STATIC_WS_BYTES (32u * 1024u * 1024u)
+
+/* rest_cross_decode without a workspace argument. The paper has no
+ * counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory themselves. Examples: a plain-C host program
+ * linking only this library (it has no device allocator of its own), and a
+ * serving process whose device memory is all handed to a fixed arena at
+ * start-up, after which nothing may call cudaMalloc.
+ *
+ * The decoder's scratch (index/tile lists and the per-row q, g and o
+ * buffers) lives in one REST_STATIC_WS_BYTES array in the library's device
+ * image instead. Every GPU that loads the library holds this array until the
+ * process exits. The caller still passes inputs and outputs exactly as for
+ * rest_cross_decode, with the same meaning, and the same results.
+ *   - A batch whose scratch would exceed the array returns
+ *     REST_ERR_WORKSPACE; rest_workspace_size() with n_layers = 0 tells the
+ *     bytes a batch needs.
+ *   - This entry point calls no cudaMalloc, cudaFree or other allocating
+ *     routine.
+ *   - The first call on a device looks up the array's device address
+ *     (once per device, with that device current). Make that first call
+ *     before any CUDA stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero. Calls whose work overlaps on the
+ *     GPU (different streams, or different host threads without ordering)
+ *     race on it: order them on one stream. */
+rest_status rest_cross_decode_static_ws(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                        const void* h, const rest_requests* reqs, const void* z,
+                                        const rest_dec_params* dec, float* y_out, int32_t* dev_err,
+                                        void* stream);
+
 /* Shared-prefix serving (§3.5): the encoder runs once over the packed
  * histories and the decoder scores every candidate of every request against
  * its output: FLOPs(T) + N * FLOPs(C) instead of N * (FLOPs(T) + FLOPs(C)).

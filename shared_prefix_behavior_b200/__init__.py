@@ -28,7 +28,8 @@ STATUS = {0: "REST_OK", 1: "REST_ERR_INVALID_ARG", 2: "REST_ERR_UNSORTED_TIME", 
           4: "REST_ERR_CUDA", 5: "REST_ERR_TIMEOUT", 6: "REST_ERR_WORKSPACE", 7: "REST_ERR_NO_DEVICE"}
 EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
            "rest_rank_request", "rest_status_string", "rest_launch_count", "rest_profile_begin",
-           "rest_profile_end")
+           "rest_profile_end", "rest_cross_decode_static_ws")
+STATIC_WS_BYTES = 32 * 1024 * 1024  # REST_STATIC_WS_BYTES
 
 
 class RestError(RuntimeError):
@@ -68,7 +69,7 @@ class KernelStat(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m shared_prefix_behavior_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python shared_prefix_behavior_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P = c_void_p
     lib.rest_workspace_size.argtypes = [c_int, POINTER(Heads), POINTER(Batch), POINTER(EncLayer), c_int,
@@ -78,10 +79,12 @@ def _load() -> ctypes.CDLL:
                                       P, P, c_size_t, P, P]
     lib.rest_cross_decode.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, POINTER(Requests), P,
                                       POINTER(DecParams), P, P, c_size_t, P, P]
+    lib.rest_cross_decode_static_ws.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, POINTER(Requests), P,
+                                                POINTER(DecParams), P, P, P]
     lib.rest_rank_request.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, POINTER(EncLayer), c_int, c_int,
                                       POINTER(Requests), P, POINTER(DecParams), P, P, P, c_size_t, P, P]
     for name in ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
-                 "rest_rank_request"):
+                 "rest_rank_request", "rest_cross_decode_static_ws"):
         getattr(lib, name).restype = c_int
     lib.rest_status_string.argtypes = [c_int]
     lib.rest_status_string.restype = ctypes.c_char_p
@@ -247,6 +250,33 @@ def cross_decode(hmem, cu_seqlens, taus, reqs, z, dec: dict, rope_base: float = 
     _check(_lib.rest_cross_decode(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(hmem), ctypes.byref(h.reqs),
                                   _ptr(z), ctypes.byref(dp), _ptr(y_out), _ptr(ws), ws.numel(), _ptr(err),
                                   _stream(stream)), "rest_cross_decode")
+    if check:
+        check_device_error(err)
+    return y_out
+
+
+def cross_decode_static_ws(hmem, cu_seqlens, taus, reqs, z, dec: dict, rope_base: float = 10000.0, y_out=None,
+                           stream=None, check=True):
+    """``cross_decode`` for callers that cannot allocate device memory.
+
+    The decoder's scratch lives in the library's own fixed device array of
+    STATIC_WS_BYTES bytes instead of a caller workspace; batches that need
+    more raise RestError(REST_ERR_WORKSPACE). Calls share that array, so
+    calls that overlap on the GPU race; order them on one stream. (This
+    wrapper itself allocates y_out and the status word with torch when they
+    are not given; a caller that cannot allocate passes its own.)
+    """
+    import torch
+    dev, d = hmem.device, hmem.shape[1]
+    dt = _dtype_code(hmem)
+    h = _Host(taus, d, rope_base, cu_seqlens, reqs)
+    dp = _dec(dec)
+    if y_out is None:
+        y_out = torch.empty(z.shape, dtype=torch.float32, device=dev)
+    err = _err_word(dev)
+    _check(_lib.rest_cross_decode_static_ws(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(hmem),
+                                            ctypes.byref(h.reqs), _ptr(z), ctypes.byref(dp), _ptr(y_out), _ptr(err),
+                                            _stream(stream)), "rest_cross_decode_static_ws")
     if check:
         check_device_error(err)
     return y_out

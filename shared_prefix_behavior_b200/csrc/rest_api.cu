@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -618,3 +619,68 @@ rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- decoder without a caller workspace
+//
+// For callers that cannot allocate device memory (see rest.h): the decoder's
+// scratch lives in a fixed array in the library's own device image instead of
+// a caller-provided workspace. Every call on a device shares this one array.
+
+namespace rest {
+
+static __device__ __align__(256) unsigned char g_static_ws[REST_STATIC_WS_BYTES];
+
+static std::mutex g_static_ws_mu;
+static void* g_static_ws_ptr[64];
+
+// Device address of g_static_ws on the current device, looked up once per
+// device (host code may not use the symbol itself as an address).
+static rest_status static_ws_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return REST_ERR_NO_DEVICE;
+  }
+  if (dev < 0 || dev >= 64) return REST_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(g_static_ws_mu);
+  if (!g_static_ws_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return REST_ERR_CUDA;
+    }
+    g_static_ws_ptr[dev] = p;
+  }
+  *out = g_static_ws_ptr[dev];
+  return REST_OK;
+}
+
+}  // namespace rest
+
+extern "C" rest_status rest_cross_decode_static_ws(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                                   const void* h, const rest_requests* reqs, const void* z,
+                                                   const rest_dec_params* dec, float* y_out, int32_t* dev_err,
+                                                   void* stream) {
+  try {
+    rest_status st = check_dec(dec);
+    if (st != REST_OK) return st;
+    if (!reqs) return REST_ERR_INVALID_ARG;
+    Plan p;
+    if ((st = make_plan(p, dt, heads, batch, nullptr, 0, 0, reqs, dec->K, false)) != REST_OK) return st;
+    if (p.NK > 0 && (!h || !z || !y_out || !aligned16(h) || !aligned16(z) || !aligned16(y_out)))
+      return REST_ERR_INVALID_ARG;
+    if (p.L.total > (size_t)REST_STATIC_WS_BYTES) return REST_ERR_WORKSPACE;  // batch too large for the array
+    if (p.NK == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    void* ws = nullptr;
+    if ((st = static_ws_address(&ws)) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    // Nothing in the scratch needs to start at zero: the index/tile lists are
+    // uploaded and q, g, o are written in full before they are read.
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    return run_decoder(p, reqs, h, z, dec, y_out, ws, dev_err, s);
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
