@@ -1,12 +1,18 @@
 // Launchers of the tcgen05 / TMEM / TMA kernels for sm_100a (bf16 path).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "kernels.h"
 
 namespace rest {
+
+// 2-D bf16 TMA descriptor over a row-major [rows, cols] array with a row stride
+// of `stride` elements; box of box_cols x box_rows; swizzle 128 or 64 bytes.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, long long stride,
+                    int box_cols, int box_rows, int swizzle_bytes);
 
 // True when the tensor-core GEMM handles this shape and epilogue.
 bool sm100_gemm_supported(const GemmArgs& a);

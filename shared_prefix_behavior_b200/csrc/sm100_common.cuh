@@ -53,6 +53,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
+    if (err && *reinterpret_cast<volatile int32_t*>(err) != 0) {  // another CTA already failed
+      *abort = 1;
+      return false;
+    }
     if (clock64() - t0 > kWaitCycles) {
       set_error(err, REST_ERR_TIMEOUT);
       *abort = 1;

@@ -1,0 +1,334 @@
+// tcgen05 GEMM for sm_100a with the fused epilogues of the ReST encoder and
+// decoder (bf16 operands, fp32 accumulation in TMEM).
+//
+// One CTA computes a 128 x BN tile of C = A . B:
+//   warp 0       TMA producer: A box [128 rows x 64 K] (K-major, 128B swizzle)
+//                and BN/64 boxes of B [64 K rows x 64 N] (N-major, 128B swizzle)
+//                per stage, into a STAGES-deep ring;
+//   warp 1       allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
+//                K=16) over the ring and commits each stage back to the producer;
+//   warps 2..5   epilogue: tcgen05.ld of the accumulator rows (warp w owns TMEM
+//                lanes 32*(w%4)..), the fused epilogue, and the global stores.
+// B is read directly from the weight as stored ([K, N] row-major, x . W
+// layout), so no transposed copy of any weight is made. The column blocks an
+// epilogue must pair (V with its gate Gv; W_1 with W_3) are brought into the
+// same tile by choosing which 64-column box of B each slot of the tile loads.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "sm100.h"
+#include "sm100_common.cuh"
+
+namespace rest {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int NUM_THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int BOX_B_BYTES = 64 * BK * 2;  // one 64-column box of B: 8 KB
+
+// Global column of B loaded into box b of N-tile t.
+__device__ __forceinline__ int b_box_col(const GemmArgs& a, int BN, int t, int b) {
+  const int nbh = BN / 128;  // boxes per half tile (paired epilogues)
+  const int half = BN / 2;
+  if (a.epi == EPI_QKVG) {
+    const int d = a.d, nQ = d / BN, nV = d / half;
+    if (t < 2 * nQ) return t * BN + 64 * b;
+    if (t < 2 * nQ + nV) {
+      int u = t - 2 * nQ;
+      return b < nbh ? 2 * d + u * half + 64 * b : 3 * d + u * half + 64 * (b - nbh);
+    }
+    return 4 * d + (t - 2 * nQ - nV) * BN + 64 * b;
+  }
+  if (a.epi == EPI_SWIGLU) return b < nbh ? t * half + 64 * b : a.d + t * half + 64 * (b - nbh);
+  return t * BN + 64 * b;
+}
+
+template <typename T>
+__device__ __forceinline__ void store32(T* p, const float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) store4(p + i, &v[i]);
+}
+
+// Every lane executes the (warp-collective) TMEM loads; only rows < M touch
+// global memory.
+template <int BN>
+__device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, int m, int t, bool valid) {
+  float v[32];
+  const long long ro = (long long)m * a.ldo;
+  if (a.epi == EPI_QKVG || a.epi == EPI_SWIGLU) {
+    const int half = BN / 2;
+    const int d = a.d;
+    if (a.epi == EPI_QKVG) {
+      const int nQ = d / BN, nV = d / half;
+      if (t < 2 * nQ) {  // Q or K: rotate the pairs (ReST eq. 5)
+        const bool isq = t < nQ;
+        const int col0 = (isq ? t : t - nQ) * BN;
+        bf16* out = (bf16*)(isq ? a.out0 : a.out1) + ro + col0;
+        const float* ct = a.cos_t + (long long)m * (d / 2) + col0 / 2;
+        const float* st = a.sin_t + (long long)m * (d / 2) + col0 / 2;
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          tmem_ld32(tmem_row + c0, v);
+          if (!valid) continue;
+          float w[32];
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) {
+            float c[4], sn[4];
+            load4(ct + c0 / 2 + j, c);
+            load4(st + c0 / 2 + j, sn);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int jj = j + i;
+              w[2 * jj] = v[2 * jj] * c[i] - v[2 * jj + 1] * sn[i];
+              w[2 * jj + 1] = v[2 * jj] * sn[i] + v[2 * jj + 1] * c[i];
+            }
+          }
+          store32(out + c0, w);
+        }
+        return;
+      }
+      if (t < 2 * nQ + nV) {  // value gate: V' = sigmoid(Gv) * V (eq. 3)
+        const int col0 = (t - 2 * nQ) * half;
+        bf16* out = (bf16*)a.out2 + ro + col0;
+        for (int c0 = 0; c0 < half; c0 += 32) {
+          float g[32];
+          tmem_ld32(tmem_row + c0, v);
+          tmem_ld32(tmem_row + half + c0, g);
+          if (!valid) continue;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= sigmoid_f(g[j]);
+          store32(out + c0, v);
+        }
+        return;
+      }
+      // output gate sigmoid(Go) (eq. 4), fp32
+      float* out = (float*)a.out3 + ro + (t - 2 * nQ - nV) * BN;
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        tmem_ld32(tmem_row + c0, v);
+        if (!valid) continue;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = sigmoid_f(v[j]);
+        store32(out + c0, v);
+      }
+      return;
+    }
+    // SwiGLU: SiLU(x W_1) * (x W_3)
+    bf16* out = (bf16*)a.out0 + ro + t * half;
+    for (int c0 = 0; c0 < half; c0 += 32) {
+      float u[32];
+      tmem_ld32(tmem_row + c0, v);
+      tmem_ld32(tmem_row + half + c0, u);
+      if (!valid) continue;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = v[j] * sigmoid_f(v[j]) * u[j];
+      store32(out + c0, v);
+    }
+    return;
+  }
+  const int n0 = t * BN;
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    tmem_ld32(tmem_row + c0, v);
+    if (!valid) continue;
+    switch (a.epi) {
+      case EPI_F32: store32((float*)a.out0 + ro + n0 + c0, v); break;
+      case EPI_DT: store32((bf16*)a.out0 + ro + n0 + c0, v); break;
+      case EPI_SIGMOID: {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = sigmoid_f(v[j]);
+        store32((float*)a.out0 + ro + n0 + c0, v);
+        break;
+      }
+      case EPI_RESID: {
+        float* p = (float*)a.out0 + ro + n0 + c0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          float x[4];
+          load4(p + j, x);
+          x[0] = fmaf(a.alpha, v[j], x[0]);
+          x[1] = fmaf(a.alpha, v[j + 1], x[1]);
+          x[2] = fmaf(a.alpha, v[j + 2], x[2]);
+          x[3] = fmaf(a.alpha, v[j + 3], x[3]);
+          store4(p + j, x);
+        }
+        break;
+      }
+    }
+  }
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs a, int num_kb, int32_t* err) {
+  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t full[STAGES], empty[STAGES], accf, drain;
+  __shared__ uint32_t tslot;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x, mt = blockIdx.y;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&accf, 1);
+    mbar_init(&drain, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&tslot, BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tslot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    int issued = 0;
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % STAGES;
+      if (!mbar_wait(&empty[s], ((kb / STAGES) & 1) ^ 1, err, &abort_flag)) break;
+      uint8_t* st = smem + s * STAGE_BYTES;
+      mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+      tma_load_2d(st, &tmA, kb * BK, mt * BM, &full[s]);
+#pragma unroll
+      for (int b = 0; b < BN / 64; ++b)
+        tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &tmB, b_box_col(a, BN, t, b), kb * BK, &full[s]);
+      issued = kb + 1;
+    }
+    if (abort_flag) {  // let the copies already in flight land before the CTA exits
+      for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb) {
+        volatile int no_abort = 0;
+        mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, &no_abort);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_bf16(BN, 1);
+    bool ok = true;
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % STAGES;
+      if (!mbar_wait(&full[s], (kb / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
+      const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+      for (int k = 0; k < BK / 16; ++k) {
+        // A: K-major, 128B swizzle; a K step of 16 is 32 bytes inside the swizzle row
+        const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
+        // B: N-major, 128B swizzle; 8-row K groups 1024 B apart, 64-column boxes 8 KB apart
+        const uint64_t bd = smem_desc(b_base + k * 2048, BOX_B_BYTES, 1024, 2);
+        mma_bf16(tmem, ad, bd, idesc, (kb | k) != 0);
+      }
+      mma_commit(&empty[s]);
+    }
+    mma_commit(ok ? &accf : &drain);
+    if (!ok) {
+      volatile int no_abort = 0;
+      mbar_wait(&drain, 0, nullptr, &no_abort);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------ epilogue
+    if (mbar_wait(&accf, 0, err, &abort_flag)) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int m = mt * BM + q * 32 + lane;
+      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+      epilogue<BN>(a, trow, m, t, m < a.M);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// 2-D bf16 tensor map over rows x cols (row stride in elements), box of
+// box_cols x box_rows, swizzle of 128 or 64 bytes; out-of-range elements
+// read as zero.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, long long stride,
+                    int box_cols, int box_rows, int swizzle_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)stride * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+constexpr int TC_BN = 128;
+constexpr int TC_STAGES = 6;
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
+  CUtensorMap ma, mb;
+  if (!make_tmap_bf16(&ma, a.A, a.M, a.K, a.lda, BK, BM, 128)) return cudaErrorInvalidValue;
+  // B is [K, Ncols] with Ncols = ldb (the full weight width)
+  if (!make_tmap_bf16(&mb, a.B, a.K, a.ldb, a.ldb, 64, BK, 128)) return cudaErrorInvalidValue;
+  constexpr int smem = STAGES * (A_BYTES + BN * BK * 2) + 1024;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int n_tiles = a.N / BN;
+  if (a.epi == EPI_QKVG) n_tiles = 5 * a.d / BN;
+  dim3 grid(n_tiles, (a.M + BM - 1) / BM);
+  gemm_tc_kernel<BN, STAGES><<<grid, NUM_THREADS, smem, s>>>(ma, mb, a, a.K / BK, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sm100_gemm_supported(const GemmArgs& a) {
+  if (a.a_f32) return false;
+  if (a.M <= 0 || a.K % BK != 0 || a.K <= 0) return false;
+  if ((a.lda % 8) || (a.ldb % 8) || (a.ldo % 8)) return false;
+  switch (a.epi) {
+    case EPI_QKVG: return a.d % TC_BN == 0 && a.N == 5 * a.d && a.ldb == 5LL * a.d;
+    case EPI_SWIGLU: return a.d % (TC_BN / 2) == 0 && a.N == 2 * a.d && a.ldb == 2LL * a.d;
+    default: return a.N % TC_BN == 0 && a.ldb == a.N;
+  }
+}
+
+cudaError_t launch_gemm_sm100(const GemmArgs& a, cudaStream_t s, int32_t* err) {
+  return launch_bn<TC_BN, TC_STAGES>(a, s, err);
+}
+
+}  // namespace rest

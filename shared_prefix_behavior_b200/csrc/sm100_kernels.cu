@@ -8,8 +8,3 @@ cudaError_t launch_enc_attn_sm100(int, const EncAttnArgs&, cudaStream_t, int32_t
 cudaError_t launch_dec_attn_sm100(int, const DecAttnArgs&, cudaStream_t, int32_t*) { return cudaErrorNotSupported; }
 
 }  // namespace rest
-
-namespace rest {
-bool sm100_gemm_supported(const GemmArgs&) { return false; }
-cudaError_t launch_gemm_sm100(const GemmArgs&, cudaStream_t, int32_t*) { return cudaErrorNotSupported; }
-}  // namespace rest
