@@ -26,6 +26,8 @@ cudaError_t launch_layernorm(bool bf16, float* x, void* y, const float* g, const
                              int mode, cudaStream_t s);
 // x_res = float(x_in)
 cudaError_t launch_to_f32(bool bf16, const void* x_in, float* x_res, long long n, cudaStream_t s);
+// hi = bf16(x), lo = bf16(x - hi): x as an unevaluated sum of two bf16 numbers
+cudaError_t launch_split_bf16(const float* x, void* hi, void* lo, long long n, cudaStream_t s);
 
 // ---------------------------------------------------------------- GEMM
 enum Epilogue {
@@ -64,6 +66,7 @@ struct EncAttnArgs {
   const EncTile* tiles; int n_tiles;
   int n_heads, d;
   float scale_log2;                             // log2(e) / sqrt(head_dim)
+  long long rows;                               // T, rows of the packed arrays
 };
 cudaError_t launch_enc_attn_simt(bool bf16, int hd, const EncAttnArgs& a, cudaStream_t s);
 
@@ -71,10 +74,12 @@ struct DecAttnArgs {
   const float* q;      // [NK, d] decoder queries (fp32)
   const float* g;      // [NK, d] sigmoid output gate
   const void* h;       // [T, d] encoder memory: keys and values
+  const void* h_lo;    // [T, d] bf16 low part of H (H = h + h_lo), or null
   float* out;          // [NK, d] o * g (fp32)
   const DecTile* tiles; int n_tiles;
   int n_heads, d;
   float scale_log2;
+  long long key_rows;  // T, rows of h
 };
 cudaError_t launch_dec_attn_simt(bool bf16, int hd, const DecAttnArgs& a, cudaStream_t s);
 

@@ -125,13 +125,13 @@ static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, 
 struct Layout {
   size_t cu, enc_tiles, dec_tiles, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
-  size_t dq, dg, dout;
+  size_t dq, dg, dout, hlo;
   size_t total;
   int n_enc_tiles, n_dec_tiles;
 };
 
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
-                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles) {
+                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -156,6 +156,7 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dq = take(4 * (size_t)NK * d);
   L.dg = take(4 * (size_t)NK * d);
   L.dout = take(4 * (size_t)NK * d);
+  L.hlo = take(hsplit ? 2 * (size_t)T * d : 0);
   L.total = off;
   return L;
 }
@@ -170,6 +171,7 @@ struct Plan {
   std::vector<DecTile> dec_tiles;
   Layout L;
   int32_t* err;
+  bool hsplit;
 };
 
 static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const rest_batch* b,
@@ -184,13 +186,15 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
     if ((st = check_requests(reqs, b, &p.n_cands)) != REST_OK) return st;
     if (K < 1 || K > 8) return REST_ERR_INVALID_ARG;
   }
-  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr;
+  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false;
   p.NK = p.n_cands * (reqs ? K : 0);
   if (p.T * (long long)hs->d >= (1LL << 40) || p.NK >= (1LL << 31)) return REST_ERR_UNSUPPORTED;
   if (encoder_runs) build_enc_tiles(b, p.enc_tiles);
   build_dec_tiles(b, reqs, K, p.dec_tiles);
+  // encoder followed by the decoder in bf16: the decoder reads H as hi + lo
+  p.hsplit = encoder_runs && reqs != nullptr && dt == REST_BF16;
   p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),
-                    (int)p.dec_tiles.size());
+                    (int)p.dec_tiles.size(), p.hsplit);
   return REST_OK;
 }
 
@@ -357,6 +361,7 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   ea.tiles = at<EncTile>(ws, L.enc_tiles); ea.n_tiles = L.n_enc_tiles;
   ea.n_heads = H; ea.d = d;
   ea.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
+  ea.rows = T;
 
   for (int l = 0; l < n_layers; ++l) {
     const rest_enc_layer& Ly = layers[l];
@@ -394,16 +399,22 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
                      launch_layernorm(bf, xres, y, Ly.ln_ffn_g, Ly.ln_ffn_b, (int)T, d, 3, s));
     }
   }
-  // H: the residual stream after the last layer, in the call's dtype (no final norm)
-  REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
-               launch_layernorm(bf, xres, h_out, nullptr, nullptr, (int)T, d, 2, s));
+  // H: the residual stream after the last layer, in the call's dtype (no final norm).
+  // When the decoder follows in bf16 it also gets H's low part: H = h_out + h_lo.
+  if (p.hsplit) {
+    REST_KLAUNCH(s, "split_h", 0, Td * 8, launch_split_bf16(xres, h_out, at<void>(ws, L.hlo), T * d, s));
+  } else {
+    REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
+                 launch_layernorm(bf, xres, h_out, nullptr, nullptr, (int)T, d, 2, s));
+  }
   return REST_OK;
 }
 
 // ---------------------------------------------------------------- decoder
 
-static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const void* h, const void* z,
-                               const rest_dec_params* dec, float* y_out, void* ws, int32_t* err, cudaStream_t s) {
+static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const void* h, const void* h_lo,
+                               const void* z, const rest_dec_params* dec, float* y_out, void* ws, int32_t* err,
+                               cudaStream_t s) {
   const bool bf = p.dt == REST_BF16;
   const int d = p.hs->d, hd = p.hs->head_dim, K = dec->K;
   const size_t e = dt_size(p.dt);
@@ -428,14 +439,15 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
     double rows = (double)(reqs->cu_cands[r + 1] - reqs->cu_cands[r]) * K;
     if (rows == 0) continue;
     flops += 4.0 * d * rows * reqs->req_cutoff[r];
-    hbytes += (double)e * reqs->req_cutoff[r] * d;
+    hbytes += (double)e * reqs->req_cutoff[r] * d * (h_lo ? 2 : 1);
   }
   const double bytes = hbytes + (double)p.NK * d * 12;
   DecAttnArgs da;
-  da.q = dq; da.g = dg; da.h = h; da.out = dout;
+  da.q = dq; da.g = dg; da.h = h; da.h_lo = h_lo; da.out = dout;
   da.tiles = at<DecTile>(ws, L.dec_tiles); da.n_tiles = L.n_dec_tiles;
   da.n_heads = p.hs->n_heads; da.d = d;
   da.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
+  da.key_rows = p.T;
   if (bf && sm100_attn_supported(hd)) {
     REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_sm100(hd, da, s, err));
   } else {
@@ -585,7 +597,7 @@ rest_status rest_cross_decode(rest_dtype dt, const rest_heads* heads, const rest
     cudaStream_t s = (cudaStream_t)stream;
     p.err = dev_err;
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
-    return run_decoder(p, reqs, h, z, dec, y_out, ws, dev_err, s);
+    return run_decoder(p, reqs, h, nullptr, z, dec, y_out, ws, dev_err, s);
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }
@@ -612,7 +624,7 @@ rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
     if ((st = run_encoder(p, x, ts, layers, n_layers, l_switch, h_out, ws, dev_err, s)) != REST_OK) return st;
     if (p.NK == 0) return REST_OK;
-    return run_decoder(p, reqs, h_out, z, dec, y_out, ws, dev_err, s);
+    return run_decoder(p, reqs, h_out, p.hsplit ? at<void>(ws, p.L.hlo) : nullptr, z, dec, y_out, ws, dev_err, s);
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }
@@ -679,7 +691,7 @@ extern "C" rest_status rest_cross_decode_static_ws(rest_dtype dt, const rest_hea
     // Nothing in the scratch needs to start at zero: the index/tile lists are
     // uploaded and q, g, o are written in full before they are read.
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
-    return run_decoder(p, reqs, h, z, dec, y_out, ws, dev_err, s);
+    return run_decoder(p, reqs, h, nullptr, z, dec, y_out, ws, dev_err, s);
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }

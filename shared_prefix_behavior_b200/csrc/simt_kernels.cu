@@ -152,6 +152,25 @@ cudaError_t launch_to_f32(bool bf16m, const void* x_in, float* x_res, long long 
   return cudaGetLastError();
 }
 
+__global__ void split_bf16_kernel(const float* __restrict__ x, bf16* __restrict__ hi, bf16* __restrict__ lo,
+                                  long long n) {
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    float v = x[i];
+    bf16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+cudaError_t launch_split_bf16(const float* x, void* hi, void* lo, long long n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  int threads = 256;
+  long long blocks = (n + threads - 1) / threads;
+  split_bf16_kernel<<<(unsigned)blocks, threads, 0, s>>>(x, (bf16*)hi, (bf16*)lo, n);
+  return cudaGetLastError();
+}
+
 // ============================================================================
 // Tiled GEMM with the fused epilogues
 // ============================================================================
@@ -298,6 +317,26 @@ struct RowState {
   float m, l;
 };
 
+// Decoder: keys and values are both the rows of H (+ its low part when given).
+template <typename T, int HD, int BK>
+__device__ __forceinline__ void stage_h(float (*Ks)[HD], float (*Vs)[HD], const T* hbase, const T* lobase,
+                                        long long ld, int nvalid) {
+  for (int e = threadIdx.x * 4; e < BK * HD; e += blockDim.x * 4) {
+    int r = e / HD, c = e % HD;
+    float hv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (r < nvalid) {
+      load4(hbase + r * ld + c, hv);
+      if (lobase) {
+        float lv[4];
+        load4(lobase + r * ld + c, lv);
+        for (int i = 0; i < 4; ++i) hv[i] += lv[i];
+      }
+    }
+    *reinterpret_cast<float4*>(&Ks[r][c]) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<float4*>(&Vs[r][c]) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+  }
+}
+
 template <typename T, int HD, int BK>
 __device__ __forceinline__ void stage_kv(float (*Ks)[HD], float (*Vs)[HD], const T* kbase, const T* vbase,
                                          long long ld, int nvalid) {
@@ -421,10 +460,12 @@ __global__ void __launch_bounds__(ATT_ROWS) dec_attn_simt_kernel(DecAttnArgs a) 
   RowState<HD> st;
   load_q<float, HD>(st, a.q + row * a.d + hoff, a.scale_log2);
   const T* Hm = (const T*)a.h + (long long)tile.key0 * a.d + hoff;
+  const T* Hlo = a.h_lo ? (const T*)a.h_lo + (long long)tile.key0 * a.d + hoff : nullptr;
   for (int kb = 0; kb < tile.nkeys; kb += ATT_BK) {
     __syncthreads();
     // keys and values are the same rows of H (projection-free, ReST eq. 7)
-    stage_kv<T, HD, ATT_BK>(Ks, Vs, Hm + (long long)kb * a.d, Hm + (long long)kb * a.d, a.d, tile.nkeys - kb);
+    stage_h<T, HD, ATT_BK>(Ks, Vs, Hm + (long long)kb * a.d, Hlo ? Hlo + (long long)kb * a.d : nullptr, a.d,
+                           tile.nkeys - kb);
     __syncthreads();
     if (valid) row_tile<HD, ATT_BK>(st, Ks, Vs, tile.nkeys - kb);
   }

@@ -284,3 +284,26 @@ def make_memory(w: Workload, seed: int) -> np.ndarray:
     """A synthetic encoder output H ~ N(0,1) [T, d], for testing the decoder alone."""
     rng = np.random.default_rng(seed + 7919)
     return _store(rng.standard_normal((w.total_tokens, w.d)), w.dtype)
+
+
+def subset_users(inp: dict, users, with_requests=True) -> dict:
+    """The inputs of a subset of users (and their requests), re-packed."""
+    users = list(users)
+    cu = inp["cu_seqlens"]
+    rows = np.concatenate([np.arange(cu[u], cu[u + 1]) for u in users])
+    new_cu = np.zeros(len(users) + 1, dtype=np.int32)
+    new_cu[1:] = np.cumsum([cu[u + 1] - cu[u] for u in users])
+    out = dict(inp, x=inp["x"][rows], ts=inp["ts"][rows], cu_seqlens=new_cu)
+    if with_requests:
+        ru, rc, cc = inp["req_user"], inp["req_cutoff"], inp["cu_cands"]
+        keep = [r for r in range(len(ru)) if ru[r] in users]
+        remap = {u: i for i, u in enumerate(users)}
+        cand_rows = np.concatenate([np.arange(cc[r], cc[r + 1]) for r in keep]) if keep else np.zeros(0, int)
+        ncs = [cc[r + 1] - cc[r] for r in keep]
+        new_cc = np.zeros(len(keep) + 1, dtype=np.int32)
+        new_cc[1:] = np.cumsum(ncs)
+        out.update(req_user=np.array([remap[ru[r]] for r in keep], dtype=np.int32),
+                   req_cutoff=np.array([rc[r] for r in keep], dtype=np.int32), cu_cands=new_cc,
+                   z=inp["z"][cand_rows], _cand_rows=cand_rows)
+    out["_rows"] = rows
+    return out
