@@ -74,9 +74,78 @@ cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_us
 // LayerNorm / casts (ReST §3.2.3, eq. 6)
 // ============================================================================
 
-template <typename T>
+// One warp per row; lane l holds columns 4l + 128k (k < d/128) as float4s.
+template <typename T, int NV>
 __global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
                                  const float* __restrict__ b, int rows, int d, int mode) {
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  float* xr = x + (long long)warp * d;
+  float v[NV][4];
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    load4(xr + 128 * k + 4 * lane, v[k]);
+    sum += v[k][0] + v[k][1] + v[k][2] + v[k][3];
+  }
+  T* yr = y ? y + (long long)warp * d : nullptr;
+  if (mode == 2) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) store4(yr + 128 * k + 4 * lane, v[k]);
+    return;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum / d;
+  float sq = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float t = v[k][i] - mean;
+      sq += t * t;
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  const float rstd = 1.0f / sqrtf(sq / d + 1e-5f);
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int c = 128 * k + 4 * lane;
+    float gg[4], bb[4], n[4];
+    load4(g + c, gg);
+    load4(b + c, bb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) n[i] = (v[k][i] - mean) * rstd * gg[i] + bb[i];
+    if (mode == 1 || mode == 3) store4(xr + c, n);
+    if (mode != 3) store4(yr + c, n);
+  }
+}
+
+template <typename T>
+static cudaError_t layernorm_dispatch(float* x, T* y, const float* g, const float* b, int rows, int d, int mode,
+                                      cudaStream_t s) {
+  int threads = 256;
+  int blocks = (rows * 32 + threads - 1) / threads;
+  switch (d / 128) {
+    case 1: layernorm_kernel<T, 1><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 2: layernorm_kernel<T, 2><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 3: layernorm_kernel<T, 3><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 4: layernorm_kernel<T, 4><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 5: layernorm_kernel<T, 5><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 6: layernorm_kernel<T, 6><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 7: layernorm_kernel<T, 7><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 8: layernorm_kernel<T, 8><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// Rows whose width is not a multiple of 128 (d = 32, 64, 96, ...): one warp
+// per row, one column per lane and step.
+template <typename T>
+__global__ void layernorm_narrow_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
+                                        const float* __restrict__ b, int rows, int d, int mode) {
   constexpr int VMAX = 32;  // d <= 1024
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
@@ -126,12 +195,15 @@ __global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const
 cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, const float* b, int T, int d,
                              int mode, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
+  if (d % 128 == 0 && d <= 1024)
+    return bf16m ? layernorm_dispatch<bf16>(x, (bf16*)y, g, b, T, d, mode, s)
+                 : layernorm_dispatch<float>(x, (float*)y, g, b, T, d, mode, s);
   int threads = 256;
   int blocks = (T * 32 + threads - 1) / threads;
   if (bf16m)
-    layernorm_kernel<bf16><<<blocks, threads, 0, s>>>(x, (bf16*)y, g, b, T, d, mode);
+    layernorm_narrow_kernel<bf16><<<blocks, threads, 0, s>>>(x, (bf16*)y, g, b, T, d, mode);
   else
-    layernorm_kernel<float><<<blocks, threads, 0, s>>>(x, (float*)y, g, b, T, d, mode);
+    layernorm_narrow_kernel<float><<<blocks, threads, 0, s>>>(x, (float*)y, g, b, T, d, mode);
   return cudaGetLastError();
 }
 

@@ -291,7 +291,7 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long 
 namespace {
 
 constexpr int TC_BN = 128;
-constexpr int TC_STAGES = 6;
+constexpr int TC_STAGES = 3;  // 97 KB of shared memory: two CTAs per SM, so one's epilogue overlaps the other's loads
 
 template <int BN, int STAGES>
 cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
