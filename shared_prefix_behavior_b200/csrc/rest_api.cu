@@ -95,27 +95,31 @@ static rest_status check_dec(const rest_dec_params* dec) {
 
 // ---------------------------------------------------------------- work lists
 
-constexpr int ENC_TILE_ROWS = 128;
-constexpr int DEC_TILE_ROWS = 128;
+// Query rows per work item: 128 for the CUDA-core attention, the
+// tensor-core kernel's own size (two 128-row tiles) otherwise.
+static int attn_tile_rows(rest_dtype dt, int head_dim) {
+  return (dt == REST_BF16 && sm100_attn_supported(head_dim)) ? sm100_attn_tile_rows() : 128;
+}
 
-static void build_enc_tiles(const rest_batch* b, std::vector<EncTile>& t) {
+static void build_enc_tiles(const rest_batch* b, int rows, std::vector<EncTile>& t) {
   t.clear();
   for (int u = 0; u < b->n_users; ++u) {
     int L = b->cu_seqlens[u + 1] - b->cu_seqlens[u];
-    for (int q0 = 0; q0 < L; q0 += ENC_TILE_ROWS) t.push_back(EncTile{u, q0});
+    for (int q0 = 0; q0 < L; q0 += rows) t.push_back(EncTile{u, q0});
   }
   // longest causal rows first, so the tail of the grid holds the short tiles
   std::stable_sort(t.begin(), t.end(), [](const EncTile& a, const EncTile& c) { return a.q0 > c.q0; });
 }
 
-static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, std::vector<DecTile>& t) {
+static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, int rows,
+                            std::vector<DecTile>& t) {
   t.clear();
   if (!r) return;
   for (int i = 0; i < r->n_req; ++i) {
     long long rows0 = (long long)r->cu_cands[i] * K, rows1 = (long long)r->cu_cands[i + 1] * K;
     int key0 = b->cu_seqlens[r->req_user[i]];
-    for (long long p = rows0; p < rows1; p += DEC_TILE_ROWS)
-      t.push_back(DecTile{(int)p, (int)std::min<long long>(DEC_TILE_ROWS, rows1 - p), key0, r->req_cutoff[i]});
+    for (long long p = rows0; p < rows1; p += rows)
+      t.push_back(DecTile{(int)p, (int)std::min<long long>(rows, rows1 - p), key0, r->req_cutoff[i]});
   }
   std::stable_sort(t.begin(), t.end(), [](const DecTile& a, const DecTile& c) { return a.nkeys > c.nkeys; });
 }
@@ -189,8 +193,9 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false;
   p.NK = p.n_cands * (reqs ? K : 0);
   if (p.T * (long long)hs->d >= (1LL << 40) || p.NK >= (1LL << 31)) return REST_ERR_UNSUPPORTED;
-  if (encoder_runs) build_enc_tiles(b, p.enc_tiles);
-  build_dec_tiles(b, reqs, K, p.dec_tiles);
+  const int tile_rows = attn_tile_rows(dt, hs->head_dim);
+  if (encoder_runs) build_enc_tiles(b, tile_rows, p.enc_tiles);
+  build_dec_tiles(b, reqs, K, tile_rows, p.dec_tiles);
   // encoder followed by the decoder in bf16: the decoder reads H as hi + lo
   p.hsplit = encoder_runs && reqs != nullptr && dt == REST_BF16;
   p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),

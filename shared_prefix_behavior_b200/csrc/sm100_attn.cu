@@ -2,24 +2,29 @@
 // Attention of the ReST encoder (§3.2.1 eqs. 3-4) and the shared-prefix,
 // projection-free cross attention of the decoder (§3.3.1 eq. 7, §3.5).
 //
-// One CTA owns 128 query rows of one head (one thread per row in the
-// softmax warpgroup) and streams 128-key blocks:
-//   warp 0       TMA producer. Encoder: Q once, then K and V' tiles per
-//                block. Decoder: one H tile per block, which serves as both
-//                the keys (K-major operand of S = q H^T) and the values
-//                (N-major operand of O = P H): H crosses HBM once per
-//                (request, head) and is staged once per block.
-//   warp 1       TMEM owner and MMA issuer: S_j = Q K_j^T into one of two
-//                128-column TMEM buffers, O_j = P_j V_j into one of two
-//                head_dim-column buffers; commits release smem stages.
-//   warps 2..5   softmax: a thread reads its row of S_j from TMEM, masks,
-//                takes the running max, exponentiates in base 2, writes P_j
-//                (bf16) to shared memory in the 128B-swizzled K-major layout
-//                the MMA reads, and folds O_{j-1} into fp32 registers.
-// The decoder's query comes in fp32; it is staged as a hi + lo pair of bf16
-// tiles and S accumulates q_hi H^T + q_lo H^T. When the encoder ran in the
-// same call, the decoder also reads H's low part (H = H_hi + H_lo, from the
-// encoder's fp32 residual stream): S adds q_hi H_lo^T and O adds P H_lo.
+// One CTA owns 256 query rows of one head as two 128-row tiles that share
+// every staged key block (so each K/V (or H) tile crosses to shared memory
+// once per 256 query rows), with one softmax warpgroup per tile:
+//   warp 0       TMA producer. Encoder: Q tiles once, then K and V' per
+//                128-key block. Decoder: H (and H_lo) per block; one H tile
+//                is both the keys (K-major operand of S = q H^T) and the
+//                values (N-major operand of O = P H).
+//   warp 1       TMEM owner and MMA issuer. Per block j and tile t: S_t(j) =
+//                Q_t K_j^T into the tile's 128-column TMEM buffer, then
+//                O_t += P_t(j-1) V_{j-1} into the tile's head_dim-column
+//                accumulator. The two tiles alternate, so one warpgroup's
+//                softmax overlaps the other's MMAs.
+//   warps 4..7   softmax of tile 0, warps 8..11 of tile 1: a thread owns a
+//                query row; it reads its row of S from TMEM, masks, keeps the
+//                running max, exponentiates in base 2, and writes P (bf16) to
+//                shared memory in the 128B-swizzled K-major layout the MMA
+//                reads. O stays in TMEM: when a row's max grows by more than
+//                2^8 the thread rescales its O row in TMEM (after the previous
+//                P V has completed); otherwise P is taken relative to the old
+//                max (values up to 2^8, exact in fp32 accumulation).
+// The decoder's query comes in fp32 and is staged as a hi + lo pair of bf16
+// tiles (S = q_hi H^T + q_lo H^T); when the encoder ran in the same call the
+// decoder also reads H_lo (H = H_hi + H_lo): S adds q_hi H_lo^T, O adds P H_lo.
 //
 // MODE 0: encoder; 1: decoder over H; 2: decoder over H_hi + H_lo.
 #include <cudaTypedefs.h>
@@ -33,47 +38,47 @@ namespace {
 
 using namespace sm100;
 
-constexpr int ROWS = 128;      // query rows per CTA
-constexpr int KB = 128;        // keys per block
-constexpr int NTHREADS = 192;
-constexpr int KV_STAGES = 3;
+constexpr int ROWS = 128;  // query rows per tile
+constexpr int NT = 2;      // tiles per CTA
+constexpr int KB = 128;    // keys per block
+constexpr int NTHREADS = 384;
+constexpr float RESCALE_LOG2 = 8.0f;  // rescale O when the row max grows by more than 2^8
 
 template <int HD>
 struct Cfg {
-  static constexpr int ROW_BYTES = HD * 2;                   // one bf16 row of a head slice
-  static constexpr int TILE_BYTES = ROWS * ROW_BYTES;        // 128 rows
-  static constexpr int SWZ = HD == 64 ? 2 : 4;               // descriptor code: 128B / 64B swizzle
-  static constexpr int ATOM = 8 * ROW_BYTES;                 // bytes of 8 swizzled rows
-  static constexpr int P_BYTES = ROWS * KB * 2;              // 32 KB
-  static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + HD;
+  static constexpr int ROW_BYTES = HD * 2;             // one bf16 row of a head slice
+  static constexpr int TILE_BYTES = ROWS * ROW_BYTES;  // 128 rows
+  static constexpr int SWZ = HD == 64 ? 2 : 4;         // descriptor code: 128B / 64B swizzle
+  static constexpr int ATOM = 8 * ROW_BYTES;           // bytes of 8 swizzled rows
+  static constexpr int P_BYTES = ROWS * KB * 2;        // 32 KB
 };
+// TMEM columns: S_0 | S_1 | O_0 | O_1
+__device__ __forceinline__ uint32_t s_col(int t) { return (uint32_t)(t * 128); }
+template <int HD>
+__device__ __forceinline__ uint32_t o_col(int t) { return (uint32_t)(256 + t * HD); }
 
-// byte offset of 16-byte chunk u (0..ROW_BYTES/16-1) of row r in a swizzled tile
+// byte offset of 16-byte chunk u of row r in a swizzled [128 x HD] bf16 tile
 template <int HD>
 __device__ __forceinline__ uint32_t swz_off(int r, int u) {
-  constexpr int CH = Cfg<HD>::ROW_BYTES / 16;  // chunks per row: 8 (128B) or 4 (64B)
+  constexpr int CH = Cfg<HD>::ROW_BYTES / 16;  // 16B chunks per row: 8 (128B rows) or 4 (64B rows)
   return r * Cfg<HD>::ROW_BYTES + ((u ^ ((r >> (HD == 64 ? 0 : 1)) & (CH - 1))) * 16);
 }
 
 template <int HD, int MODE>
 struct SmemLayout {
-  // [Q (hi) | Q lo (decoder) | KV stages | P x2], every block 1024-aligned.
-  // A stage holds K and V' (encoder), H (decoder), or H_hi and H_lo.
+  // [Q_0 | Q_1 | (decoder) Qlo_0 | Qlo_1 | KV stages | P_0 | P_1], 1024-aligned blocks
+  static constexpr int STAGES = MODE == 2 ? 2 : 3;
   static constexpr int Q = 0;
-  static constexpr int QLO = Cfg<HD>::TILE_BYTES;
-  static constexpr int KV = (MODE >= 1 ? 2 : 1) * Cfg<HD>::TILE_BYTES;
+  static constexpr int QLO = NT * Cfg<HD>::TILE_BYTES;
+  static constexpr int KV = (MODE >= 1 ? 2 : 1) * NT * Cfg<HD>::TILE_BYTES;
+  // a stage holds K and V' (encoder), H (decoder), or H_hi and H_lo
   static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
-  static constexpr int P = KV + KV_STAGES * STAGE;
-  static constexpr int TOTAL = P + 2 * Cfg<HD>::P_BYTES;
+  static constexpr int P = KV + STAGES * STAGE;
+  static constexpr int TOTAL = P + NT * Cfg<HD>::P_BYTES;
 };
 
-struct AttnWork {
-  int q_row0;     // first query row (packed row index: encoder token / decoder q row)
-  int nrows;      // valid query rows (<= 128)
-  int key_row0;   // first key row in the packed [T, d] array
-  int nkeys;      // keys visible to the last query row (encoder: causal bound)
-  int causal_off; // encoder: position of query row 0 minus position of key row 0
-};
+__device__ __forceinline__ void setmaxnreg_dec72() { asm volatile("setmaxnreg.dec.sync.aligned.u32 72;"); }
+__device__ __forceinline__ void setmaxnreg_inc216() { asm volatile("setmaxnreg.inc.sync.aligned.u32 216;"); }
 
 template <int HD, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -82,10 +87,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr bool DEC = MODE >= 1, HLO = MODE == 2;
   using C = Cfg<HD>;
   using L = SmemLayout<HD, MODE>;
+  constexpr int STAGES = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t q_full, kv_full[KV_STAGES], kv_empty[KV_STAGES], s_full[2], p_full[2], p_free[2], o_full[2],
-      o_free[2], drain;
+  __shared__ uint64_t q_full[NT], kv_full[STAGES], kv_empty[STAGES], s_full[NT], p_full[NT], p_free[NT], drain;
   __shared__ uint32_t tslot;
   __shared__ volatile int abort_flag;
 
@@ -95,29 +100,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int tile = blockIdx.x / n_heads, h = blockIdx.x % n_heads;
 
   // ---------------------------------------------------------------- work item
-  AttnWork w;
+  // rows: first packed query row of tile 0; nrow[t]: valid rows of tile t;
+  // nblk[t]: key blocks tile t reads; key_row0: packed row of key 0.
+  int q_row0, key_row0, nrow[NT], nblk[NT], user_len = 0, q_pos0 = 0, nkeys = 0;
   if (DEC) {
     DecTile t = da.tiles[tile];
-    w = AttnWork{t.row0, t.nrows, t.key0, t.nkeys, 0};
+    q_row0 = t.row0;
+    key_row0 = t.key0;
+    nkeys = t.nkeys;
+    for (int i = 0; i < NT; ++i) {
+      nrow[i] = max(0, min(ROWS, t.nrows - i * ROWS));
+      nblk[i] = nrow[i] > 0 ? (t.nkeys + KB - 1) / KB : 0;
+    }
   } else {
     EncTile t = ea.tiles[tile];
-    int s = ea.cu[t.user], Lu = ea.cu[t.user + 1] - s;
-    w = AttnWork{s + t.q0, min(ROWS, Lu - t.q0), s, min(Lu, t.q0 + ROWS), t.q0};
+    key_row0 = ea.cu[t.user];
+    user_len = ea.cu[t.user + 1] - key_row0;
+    q_pos0 = t.q0;
+    q_row0 = key_row0 + t.q0;
+    for (int i = 0; i < NT; ++i) {
+      const int r0 = t.q0 + i * ROWS;
+      nrow[i] = max(0, min(ROWS, user_len - r0));
+      nblk[i] = nrow[i] > 0 ? (min(user_len, r0 + ROWS) + KB - 1) / KB : 0;
+    }
   }
-  const int nblk = (w.nkeys + KB - 1) / KB;
+  const int nblk_all = max(nblk[0], nblk[1]);
 
   if (threadIdx.x == 0) {
-    mbar_init(&q_full, DEC ? 128 : 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
+    for (int t = 0; t < NT; ++t) {
+      mbar_init(&q_full[t], DEC ? 128 : 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&p_free[t], 1);
+    }
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
-      mbar_init(&p_free[b], 1);
-      mbar_init(&o_full[b], 1);
-      mbar_init(&o_free[b], 128);
     }
     mbar_init(&drain, 1);
     abort_flag = 0;
@@ -129,111 +147,119 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = tslot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- TMA producer
+  if (warp < 4) {
+    setmaxnreg_dec72();
+    if (warp == 0 && lane == 0) {
+      // -------------------------------------------------------- TMA producer
       if (!DEC) {
-        mbar_arrive_expect_tx(&q_full, C::TILE_BYTES);
-        tma_load_2d(smem + L::Q, &tmQ, h * HD, w.q_row0, &q_full);
+        for (int t = 0; t < NT; ++t) {
+          if (nrow[t] == 0) continue;
+          mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
+          tma_load_2d(smem + L::Q + t * C::TILE_BYTES, &tmQ, h * HD, q_row0 + t * ROWS, &q_full[t]);
+        }
       }
       int issued = 0;
-      for (int j = 0; j < nblk; ++j) {
-        const int st = j % KV_STAGES;
-        if (!mbar_wait(&kv_empty[st], ((j / KV_STAGES) & 1) ^ 1, err, &abort_flag)) break;
+      for (int j = 0; j < nblk_all; ++j) {
+        const int st = j % STAGES;
+        if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1, err, &abort_flag)) break;
         uint8_t* base = smem + L::KV + st * L::STAGE;
         mbar_arrive_expect_tx(&kv_full[st], L::STAGE);
-        tma_load_2d(base, &tmK, h * HD, w.key_row0 + j * KB, &kv_full[st]);
-        if (MODE != 1) tma_load_2d(base + C::TILE_BYTES, &tmV, h * HD, w.key_row0 + j * KB, &kv_full[st]);
+        tma_load_2d(base, &tmK, h * HD, key_row0 + j * KB, &kv_full[st]);
+        if (MODE != 1) tma_load_2d(base + C::TILE_BYTES, &tmV, h * HD, key_row0 + j * KB, &kv_full[st]);
         issued = j + 1;
       }
-      if (abort_flag) {
+      if (abort_flag) {  // let the copies in flight land before the CTA exits
         volatile int no_abort = 0;
-        if (!DEC) mbar_wait(&q_full, 0, nullptr, &no_abort);
-        for (int j = (issued > KV_STAGES ? issued - KV_STAGES : 0); j < issued; ++j)
-          mbar_wait(&kv_full[j % KV_STAGES], (j / KV_STAGES) & 1, nullptr, &no_abort);
+        if (!DEC)
+          for (int t = 0; t < NT; ++t)
+            if (nrow[t] > 0) mbar_wait(&q_full[t], 0, nullptr, &no_abort);
+        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+          mbar_wait(&kv_full[j % STAGES], (j / STAGES) & 1, nullptr, &no_abort);
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idS = idesc_bf16(KB, 0);   // N = 128 keys, B (keys) K-major
-      constexpr uint32_t idO = idesc_bf16(HD, 1);   // N = head_dim, B (values) N-major
-      bool ok = mbar_wait(&q_full, 0, err, &abort_flag);
+    } else if (warp == 1 && lane == 0) {
+      // -------------------------------------------------------- MMA issuer
+      constexpr uint32_t idS = idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
+      constexpr uint32_t idO = idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
+      bool ok = true;
+      for (int t = 0; t < NT && ok; ++t)
+        if (nrow[t] > 0) ok = mbar_wait(&q_full[t], 0, err, &abort_flag);
       tc_fence_after();
-      const uint32_t q_base = smem_u32(smem + L::Q);
-      const uint32_t qlo_base = smem_u32(smem + L::QLO);
-      for (int j = 0; ok && j <= nblk; ++j) {
-        if (j < nblk) {
-          const int st = j % KV_STAGES;
-          if (!mbar_wait(&kv_full[st], (j / KV_STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+      for (int j = 0; ok && j <= nblk_all; ++j) {
+        const int st = j % STAGES;
+        if (j < nblk_all) {
+          if (!mbar_wait(&kv_full[st], (j / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t k_base = smem_u32(smem + L::KV + st * L::STAGE);
-          const uint32_t tS = tmem + ((j & 1) ? C::TMEM_S1 : C::TMEM_S0);
-#pragma unroll
-          for (int k = 0; k < HD / 16; ++k) {
-            const uint64_t ad = smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ);
-            const uint64_t bd = smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ);
-            mma_bf16(tS, ad, bd, idS, k != 0);
-          }
-          if (DEC) {  // + q_lo . H^T
-#pragma unroll
-            for (int k = 0; k < HD / 16; ++k) {
-              const uint64_t ad = smem_desc(qlo_base + k * 32, 16, C::ATOM, C::SWZ);
-              const uint64_t bd = smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ);
-              mma_bf16(tS, ad, bd, idS, 1);
-            }
-          }
-          if (HLO) {  // + q_hi . H_lo^T
-#pragma unroll
-            for (int k = 0; k < HD / 16; ++k) {
-              const uint64_t ad = smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ);
-              const uint64_t bd = smem_desc(k_base + C::TILE_BYTES + k * 32, 16, C::ATOM, C::SWZ);
-              mma_bf16(tS, ad, bd, idS, 1);
-            }
-          }
-          mma_commit(&s_full[j & 1]);
         }
-        if (j >= 1) {
-          const int i = j - 1, b = i & 1, st = i % KV_STAGES;
-          if (!mbar_wait(&p_full[b], (i >> 1) & 1, err, &abort_flag)) { ok = false; break; }
-          if (i >= 2 && !mbar_wait(&o_free[b], ((i - 2) >> 1) & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t p_base = smem_u32(smem + L::P + b * C::P_BYTES);
-          const uint32_t v_base = smem_u32(smem + L::KV + st * L::STAGE + (DEC ? 0 : C::TILE_BYTES));
-          const uint32_t tO = tmem + (b ? C::TMEM_O1 : C::TMEM_O0);
-#pragma unroll
-          for (int k = 0; k < KB / 16; ++k) {
-            const uint64_t ad = smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(v_base + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ);
-            mma_bf16(tO, ad, bd, idO, k != 0);
+        for (int t = 0; t < NT; ++t) {
+          // S_t(j) overwrites the tile's S buffer: the softmax has taken S_t(j-1)
+          // (and written P_t(j-1)) once p_full[t] completes its phase j-1.
+          if (j >= 1 && j - 1 < nblk[t]) {
+            if (!mbar_wait(&p_full[t], (j - 1) & 1, err, &abort_flag)) { ok = false; break; }
+            tc_fence_after();
           }
-          if (HLO) {  // + P . H_lo
+          if (j < nblk[t]) {
+            const uint32_t k_base = smem_u32(smem + L::KV + st * L::STAGE);
+            const uint32_t q_base = smem_u32(smem + L::Q + t * C::TILE_BYTES);
+            const uint32_t tS = tmem + s_col(t);
 #pragma unroll
-            for (int k = 0; k < KB / 16; ++k) {
-              const uint64_t ad = smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2);
-              const uint64_t bd = smem_desc(v_base + C::TILE_BYTES + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ);
-              mma_bf16(tO, ad, bd, idO, 1);
+            for (int k = 0; k < HD / 16; ++k)
+              mma_bf16(tS, smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ),
+                       smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, k != 0);
+            if (DEC) {  // + q_lo . H^T
+              const uint32_t qlo_base = smem_u32(smem + L::QLO + t * C::TILE_BYTES);
+#pragma unroll
+              for (int k = 0; k < HD / 16; ++k)
+                mma_bf16(tS, smem_desc(qlo_base + k * 32, 16, C::ATOM, C::SWZ),
+                         smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
             }
+            if (HLO) {  // + q_hi . H_lo^T
+#pragma unroll
+              for (int k = 0; k < HD / 16; ++k)
+                mma_bf16(tS, smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ),
+                         smem_desc(k_base + C::TILE_BYTES + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
+            }
+            mma_commit(&s_full[t]);
           }
-          mma_commit(&o_full[b]);
-          mma_commit(&p_free[b]);
-          mma_commit(&kv_empty[st]);
+          if (j >= 1 && j - 1 < nblk[t]) {  // O_t += P_t(j-1) V_{j-1}
+            const int i = j - 1, sti = i % STAGES;
+            const uint32_t p_base = smem_u32(smem + L::P + t * C::P_BYTES);
+            const uint32_t v_base = smem_u32(smem + L::KV + sti * L::STAGE + (DEC ? 0 : C::TILE_BYTES));
+            const uint32_t tO = tmem + o_col<HD>(t);
+#pragma unroll
+            for (int k = 0; k < KB / 16; ++k)
+              mma_bf16(tO, smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2),
+                       smem_desc(v_base + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO, (i | k) != 0);
+            if (HLO) {  // + P H_lo
+#pragma unroll
+              for (int k = 0; k < KB / 16; ++k)
+                mma_bf16(tO, smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2),
+                         smem_desc(v_base + C::TILE_BYTES + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO,
+                         1);
+            }
+            mma_commit(&p_free[t]);
+          }
         }
+        if (j >= 1 && ok) mma_commit(&kv_empty[(j - 1) % STAGES]);  // block j-1 fully consumed
       }
       mma_commit(&drain);
       volatile int no_abort = 0;
       mbar_wait(&drain, 0, nullptr, &no_abort);
     }
   } else {
+    setmaxnreg_inc216();
     // -------------------------------------------------------------- softmax
-    const int q = warp & 3;
-    const int r = q * 32 + lane;                  // row within the tile
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const bool valid = r < w.nrows;
+    const int t = (warp - 4) >> 2;               // tile of this warpgroup
+    const int q4 = warp & 3;                     // TMEM lane quarter
+    const int r = q4 * 32 + lane;                // row within the tile
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const bool valid = r < nrow[t];
     const float sl2 = DEC ? da.scale_log2 : ea.scale_log2;
+    const int nb = nblk[t];
 
-    if (DEC) {  // stage q (fp32) as hi + lo bf16 tiles in the swizzled K-major layout
-      const float* qrow = da.q + (long long)(w.q_row0 + (valid ? r : 0)) * d + h * HD;
+    if (DEC && nb > 0) {  // stage q (fp32) as hi + lo bf16 tiles in the swizzled K-major layout
+      const float* qrow = da.q + (long long)(q_row0 + t * ROWS + (valid ? r : 0)) * d + h * HD;
+      uint8_t* qh = smem + L::Q + t * C::TILE_BYTES;
+      uint8_t* ql = smem + L::QLO + t * C::TILE_BYTES;
 #pragma unroll
       for (int u = 0; u < HD / 8; ++u) {
         float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -251,106 +277,123 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           lo[e] = *reinterpret_cast<uint32_t*>(&l2);
         }
         const uint32_t off = swz_off<HD>(r, u);
-        *reinterpret_cast<uint4*>(smem + L::Q + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(smem + L::QLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(qh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(ql + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       fence_async_smem();
-      mbar_arrive(&q_full);
+      mbar_arrive(&q_full[t]);
     }
 
-    float acc[HD];
-#pragma unroll
-    for (int c = 0; c < HD; ++c) acc[c] = 0.f;
-    float m_run = -INFINITY;  // running max after the last block (log2 domain)
-    float l_run = 0.f;        // running sum of exponentials, relative to m_run
-    float m_acc = -INFINITY;  // max that acc is expressed relative to
+    const uint32_t tS = tmem + lane_off + s_col(t);
+    const uint32_t tO = tmem + lane_off + o_col<HD>(t);
+    uint8_t* pb = smem + L::P + t * C::P_BYTES;
+    // visible keys: index < row_lim - 128 j (the causal bound and the user end / cutoff)
+    const int row_lim = DEC ? nkeys : min(q_pos0 + t * ROWS + r + 1, user_len);
+    float m_ref = -INFINITY;  // reference max (scaled, log2 domain) of P and O
+    float l_run = 0.f;        // sum of exponentials relative to m_ref
     bool ok = true;
-    // O_i (relative to m_i) folded into acc: acc = acc * 2^(m_acc - m_i) + O_i
-    auto fold = [&](int i, float m_i) -> bool {
-      const int bo = i & 1;
-      if (!mbar_wait(&o_full[bo], (i >> 1) & 1, err, &abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t tO = tmem + lane_off + (bo ? C::TMEM_O1 : C::TMEM_O0);
-      const float f = exp2_approx(m_acc - m_i);
-#pragma unroll
-      for (int c0 = 0; c0 < HD; c0 += 32) {
-        float t32[32];
-        tmem_ld32(tO + c0, t32);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) acc[c0 + e] = fmaf(acc[c0 + e], f, t32[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(&o_free[bo]);
-      m_acc = m_i;
-      return true;
-    };
-    for (int j = 0; j < nblk; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(&s_full[b], (j >> 1) & 1, err, &abort_flag)) { ok = false; break; }
+    for (int j = 0; j < nb; ++j) {
+      if (!mbar_wait(&s_full[t], j & 1, err, &abort_flag)) { ok = false; break; }
       tc_fence_after();
       float s[KB];
-      const uint32_t tS = tmem + lane_off + (b ? C::TMEM_S1 : C::TMEM_S0);
+      {
+        uint32_t raw[4][32];
 #pragma unroll
-      for (int c0 = 0; c0 < KB; c0 += 32) {
-        float t32[32];
-        tmem_ld32(tS + c0, t32);
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, raw[c]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c0 + i] = t32[i];
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[c][i]);
       }
-      // keys visible to this row in block j: index < lim (the tail; and causality in the encoder)
-      int lim = w.nkeys - j * KB;
-      if (!DEC) lim = min(lim, w.causal_off + r + 1 - j * KB);
-      float mx = -INFINITY;
+      const int lim = row_lim - j * KB;
+      if (lim < KB) {
 #pragma unroll
-      for (int c = 0; c < KB; ++c) {
-        s[c] = (c < lim) ? s[c] * sl2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < KB; ++c)
+          if (c >= lim) s[c] = -INFINITY;
       }
-      const float m_old = m_run;
-      const float m_new = fmaxf(m_run, mx);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      float sum = 0.f;
+      // row max of the raw scores (tree, for ILP)
+      float mx[8];
 #pragma unroll
-      for (int c = 0; c < KB; ++c) {
-        s[c] = exp2_approx(s[c] - m_use);
-        sum += s[c];
+      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < KB; c += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
+      const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      // P_t(j) replaces P_t(j-1): wait until O += P_t(j-1) V has completed
+      if (j >= 1) {
+        if (!mbar_wait(&p_free[t], (j - 1) & 1, err, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
       }
-      l_run = l_run * exp2_approx(m_old - m_use) + sum;
-      m_run = m_use;
-      // P_j -> shared memory, once PV_{j-2} has finished reading this buffer
-      if (j >= 2 && !mbar_wait(&p_free[b], ((j - 2) >> 1) & 1, err, &abort_flag)) { ok = false; break; }
-      uint8_t* pb = smem + L::P + b * C::P_BYTES;
+      if (j == 0) {
+        m_ref = m_blk;
+      } else if (m_blk > m_ref + RESCALE_LOG2) {  // rescale the O row and l to the new max
+        const float f = exp2_approx(m_ref - m_blk);
+#pragma unroll
+        for (int c0 = 0; c0 < HD; c0 += 32) {
+          float o[32];
+          tmem_ld32(tO + c0, o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= f;
+          tmem_st32(tO + c0, o);
+        }
+        l_run *= f;
+        m_ref = m_blk;
+      }
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int u = 0; u < KB / 8; ++u) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[e] = exp2_approx(fmaf(s[8 * u + e], sl2, -m_ref));
+          sum[e & 3] += p[e];
+        }
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 t2 = __floats2bfloat162_rn(s[8 * u + 2 * e], s[8 * u + 2 * e + 1]);
+          __nv_bfloat162 t2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
           pk[e] = *reinterpret_cast<uint32_t*>(&t2);
         }
         const int chunk = u >> 3, uu = u & 7;
         *reinterpret_cast<uint4*>(pb + chunk * (ROWS * 128) + r * 128 + ((uu ^ (r & 7)) * 16)) =
             make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+      l_run += (sum[0] + sum[1]) + (sum[2] + sum[3]);
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[b]);
-      if (j >= 1 && !fold(j - 1, m_old)) { ok = false; break; }
+      mbar_arrive(&p_full[t]);
     }
-    if (ok && nblk > 0) ok = fold(nblk - 1, m_run);
-    if (ok && valid) {
-      const float inv = 1.0f / l_run;
-      const long long ro = (long long)(w.q_row0 + r) * d + h * HD;
-      const float* gate = (DEC ? da.g : ea.gate) + ro;
+    if (ok && nb > 0) {
+      ok = mbar_wait(&p_free[t], (nb - 1) & 1, err, &abort_flag);  // the last P V has completed
+      tc_fence_after();
+    }
+    if (nb > 0) {
+      // every lane takes part in the (warp-collective) TMEM loads
+      float o[HD];
 #pragma unroll
-      for (int c = 0; c < HD; c += 4) {
-        float g[4];
-        load4(gate + c, g);
-        float v[4] = {acc[c] * inv * g[0], acc[c + 1] * inv * g[1], acc[c + 2] * inv * g[2], acc[c + 3] * inv * g[3]};
-        if (DEC)
-          store4(da.out + ro + c, v);
-        else
-          store4((bf16*)ea.out + ro + c, v);
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        float v32[32];
+        tmem_ld32(tO + c0, v32);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[c0 + e] = v32[e];
+      }
+      if (ok && valid) {
+        const float inv = 1.0f / l_run;
+        const long long ro = (long long)(q_row0 + t * ROWS + r) * d + h * HD;
+        const float* gate = (DEC ? da.g : ea.gate) + ro;
+#pragma unroll
+        for (int c = 0; c < HD; c += 4) {
+          float g[4];
+          load4(gate + c, g);
+          float v[4] = {o[c] * inv * g[0], o[c + 1] * inv * g[1], o[c + 2] * inv * g[2], o[c + 3] * inv * g[3]};
+          if (DEC)
+            store4(da.out + ro + c, v);
+          else
+            store4((bf16*)ea.out + ro + c, v);
+        }
       }
     }
   }
@@ -371,7 +414,6 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
   const int n_heads = DEC ? da->n_heads : ea->n_heads;
   const int d = DEC ? da->d : ea->d;
   if (n_tiles == 0) return cudaSuccess;
-  // the packed [T, d] arrays: T is not needed by the kernel; the maps cover every row the tiles name
   const long long rows = DEC ? da->key_rows : ea->rows;
   if (DEC) {
     if (!make_tmap_bf16(&mk, da->h, rows, d, d, HD, ROWS, swz)) return cudaErrorInvalidValue;
@@ -384,7 +426,7 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
         !make_tmap_bf16(&mv, ea->v, rows, d, d, HD, ROWS, swz))
       return cudaErrorInvalidValue;
   }
-  // at least 120 KB so that one CTA (which takes all 512 TMEM columns) runs per SM
+  // at least 120 KB so that exactly one CTA (which takes all 512 TMEM columns) runs per SM
   constexpr int smem_need = SmemLayout<HD, MODE>::TOTAL + 1024;
   constexpr int smem = smem_need > 120 * 1024 ? smem_need : 120 * 1024;
   static bool attr_set = false;
@@ -402,6 +444,7 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
 }  // namespace
 
 bool sm100_attn_supported(int head_dim) { return head_dim == 32 || head_dim == 64; }
+int sm100_attn_tile_rows() { return NT * ROWS; }
 
 cudaError_t launch_enc_attn_sm100(int hd, const EncAttnArgs& a, cudaStream_t s, int32_t* err) {
   return hd == 64 ? launch_attn<64, 0>(&a, nullptr, s, err) : launch_attn<32, 0>(&a, nullptr, s, err);
