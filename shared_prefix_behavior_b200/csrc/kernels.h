@@ -57,7 +57,10 @@ cudaError_t launch_gemm_simt(bool bf16, const GemmArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 struct EncTile { int user; int q0; };          // q0: first query position within the user
-struct DecTile { int row0; int nrows; int key0; int nkeys; };  // query rows, memory rows of H
+// Decoder work item: query rows [row0, row0 + nrows) against the first nkeys
+// rows of H starting at key0; it covers the 128-key blocks [kb0, kb1) and, when
+// the launch splits keys, writes partial results as split number `split`.
+struct DecTile { int row0; int nrows; int key0; int nkeys; int kb0; int kb1; int split; int pad; };
 struct EncAttnArgs {
   const void* q; const void* k; const void* v;  // [T, d] rotated Q, K and gated V'
   const float* gate;                            // [T, d] sigmoid(Go)
@@ -80,7 +83,15 @@ struct DecAttnArgs {
   int n_heads, d;
   float scale_log2;
   long long key_rows;  // T, rows of h
+  // split keys (n_split > 1): per split, the unnormalized O [NK, d] and the
+  // reference max m (log2 domain) and sum l [NK, n_heads, 2]; combined by
+  // launch_dec_combine into out.
+  int n_split;
+  long long nk_rows;   // NK
+  float* part_o;
+  float* part_ml;
 };
 cudaError_t launch_dec_attn_simt(bool bf16, int hd, const DecAttnArgs& a, cudaStream_t s);
+cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s);
 
 }  // namespace rest

@@ -111,17 +111,28 @@ static void build_enc_tiles(const rest_batch* b, int rows, std::vector<EncTile>&
   std::stable_sort(t.begin(), t.end(), [](const EncTile& a, const EncTile& c) { return a.q0 > c.q0; });
 }
 
-static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, int rows,
+constexpr int KEY_BLOCK = 128;   // keys per block of the attention kernels
+constexpr int TARGET_CTAS = 296;  // two waves of the B200's 148 SMs
+
+// Decoder work items. With n_split > 1 every (request, row chunk) is split
+// into n_split ranges of whole key blocks (some may be empty) whose partial
+// results a combine kernel merges.
+static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, int rows, int n_split,
                             std::vector<DecTile>& t) {
   t.clear();
   if (!r) return;
   for (int i = 0; i < r->n_req; ++i) {
     long long rows0 = (long long)r->cu_cands[i] * K, rows1 = (long long)r->cu_cands[i + 1] * K;
     int key0 = b->cu_seqlens[r->req_user[i]];
+    int c = r->req_cutoff[i];
+    int nb = (c + KEY_BLOCK - 1) / KEY_BLOCK;
     for (long long p = rows0; p < rows1; p += rows)
-      t.push_back(DecTile{(int)p, (int)std::min<long long>(rows, rows1 - p), key0, r->req_cutoff[i]});
+      for (int sp = 0; sp < n_split; ++sp)
+        t.push_back(DecTile{(int)p, (int)std::min<long long>(rows, rows1 - p), key0, c,
+                            (int)((long long)nb * sp / n_split), (int)((long long)nb * (sp + 1) / n_split), sp, 0});
   }
-  std::stable_sort(t.begin(), t.end(), [](const DecTile& a, const DecTile& c) { return a.nkeys > c.nkeys; });
+  std::stable_sort(t.begin(), t.end(),
+                   [](const DecTile& a, const DecTile& c) { return a.kb1 - a.kb0 > c.kb1 - c.kb0; });
 }
 
 // ---------------------------------------------------------------- workspace
@@ -129,13 +140,13 @@ static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, 
 struct Layout {
   size_t cu, enc_tiles, dec_tiles, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
-  size_t dq, dg, dout, hlo;
+  size_t dq, dg, dout, hlo, part_o, part_ml;
   size_t total;
   int n_enc_tiles, n_dec_tiles;
 };
 
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
-                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit) {
+                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -161,6 +172,8 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dg = take(4 * (size_t)NK * d);
   L.dout = take(4 * (size_t)NK * d);
   L.hlo = take(hsplit ? 2 * (size_t)T * d : 0);
+  L.part_o = take(n_split > 1 ? 4 * (size_t)n_split * NK * d : 0);
+  L.part_ml = take(n_split > 1 ? 8 * (size_t)n_split * NK * hs->n_heads : 0);
   L.total = off;
   return L;
 }
@@ -176,6 +189,7 @@ struct Plan {
   Layout L;
   int32_t* err;
   bool hsplit;
+  int n_split;  // decoder key splits (tensor-core path)
 };
 
 static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const rest_batch* b,
@@ -190,16 +204,28 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
     if ((st = check_requests(reqs, b, &p.n_cands)) != REST_OK) return st;
     if (K < 1 || K > 8) return REST_ERR_INVALID_ARG;
   }
-  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false;
+  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false; p.n_split = 1;
   p.NK = p.n_cands * (reqs ? K : 0);
   if (p.T * (long long)hs->d >= (1LL << 40) || p.NK >= (1LL << 31)) return REST_ERR_UNSUPPORTED;
   const int tile_rows = attn_tile_rows(dt, hs->head_dim);
   if (encoder_runs) build_enc_tiles(b, tile_rows, p.enc_tiles);
-  build_dec_tiles(b, reqs, K, tile_rows, p.dec_tiles);
+  // split the decoder's keys when its work items alone would leave SMs idle
+  p.n_split = 1;
+  if (reqs && tile_rows != 128) {
+    build_dec_tiles(b, reqs, K, tile_rows, 1, p.dec_tiles);
+    long long base = (long long)p.dec_tiles.size() * hs->n_heads, blocks = 0;
+    for (const DecTile& t : p.dec_tiles) blocks += t.kb1 - t.kb0;
+    if (base > 0 && base < TARGET_CTAS) {
+      long long want = (TARGET_CTAS + base - 1) / base;
+      long long most = std::max(1LL, blocks / (long long)p.dec_tiles.size() / 4);  // >= ~4 blocks per split
+      p.n_split = (int)std::min<long long>(8, std::min(want, most));
+    }
+  }
+  build_dec_tiles(b, reqs, K, tile_rows, p.n_split, p.dec_tiles);
   // encoder followed by the decoder in bf16: the decoder reads H as hi + lo
   p.hsplit = encoder_runs && reqs != nullptr && dt == REST_BF16;
   p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),
-                    (int)p.dec_tiles.size(), p.hsplit);
+                    (int)p.dec_tiles.size(), p.hsplit, p.n_split);
   return REST_OK;
 }
 
@@ -453,8 +479,15 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   da.n_heads = p.hs->n_heads; da.d = d;
   da.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
   da.key_rows = p.T;
+  da.n_split = p.n_split;
+  da.nk_rows = p.NK;
+  da.part_o = at<float>(ws, L.part_o);
+  da.part_ml = at<float>(ws, L.part_ml);
   if (bf && sm100_attn_supported(hd)) {
     REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_sm100(hd, da, s, err));
+    if (p.n_split > 1)
+      REST_KLAUNCH(s, "dec_combine", 0, (double)p.NK * d * 4 * (p.n_split + 2),
+                   launch_dec_combine(hd, da, s));
   } else {
     REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_simt(bf, hd, da, s));
   }

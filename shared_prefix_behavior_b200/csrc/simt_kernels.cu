@@ -25,46 +25,47 @@ __device__ __forceinline__ int find_user(const int32_t* cu, int n_users, int i) 
   return lo;
 }
 
+// One thread per (token, head, frequency j): consecutive threads write
+// consecutive table entries.
 __global__ void rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu,
                                       int n_users, int T, TableParams p, int64_t* idx_out,
                                       float* cos_out, float* sin_out, int32_t* err) {
-  long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= (long long)T * p.n_heads) return;
-  int i = (int)(gid / p.n_heads), h = (int)(gid % p.n_heads);
-  int s = cu[find_user(cu, n_users, i)];
-  long long t = ts[i];
-  if (h == 0 && i > s && ts[i - 1] > t) set_error(err, REST_ERR_UNSORTED_TIME);
-  long long tau = p.tau[h];
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long per_tok = (long long)p.n_heads * p.half;
+  if (gid >= (long long)T * per_tok) return;
+  const int i = (int)(gid / per_tok);
+  const int rem = (int)(gid % per_tok);
+  const int h = rem / p.half, j = rem % p.half;
+  const int s = cu[find_user(cu, n_users, i)];
+  const long long t = ts[i];
+  if (rem == 0 && i > s && ts[i - 1] > t) set_error(err, REST_ERR_UNSORTED_TIME);
+  const long long tau = p.tau[h];
   long long idx;
   if (tau == 0) {
     idx = i - s;
   } else {
-    long long rel = t - ts[s];           // exact int64
-    long long q = rel / tau;             // floor division (rel < 0 only on invalid input)
+    const long long rel = t - ts[s];  // exact int64
+    long long q = rel / tau;          // floor division (rel < 0 only on invalid input)
     if ((rel % tau != 0) && (rel < 0)) q -= 1;
     idx = q;
   }
-  if (idx_out) idx_out[gid] = idx;
+  if (idx_out && j == 0) idx_out[(long long)i * p.n_heads + h] = idx;
   if (cos_out) {
-    float* cp = cos_out + gid * p.half;
-    float* sp = sin_out + gid * p.half;
-    for (int j = 0; j < p.half; ++j) {
-      double phi = (double)idx * p.theta[j];
-      double sv, cv;
-      sincos(phi, &sv, &cv);
-      cp[j] = (float)cv;
-      sp[j] = (float)sv;
-    }
+    const double phi = (double)idx * p.theta[j];
+    double sv, cv;
+    sincos(phi, &sv, &cv);
+    cos_out[gid] = (float)cv;
+    sin_out[gid] = (float)sv;
   }
 }
 
 cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users, int T,
                                     const TableParams& p, int64_t* idx_out, float* cos_out,
                                     float* sin_out, int32_t* err, cudaStream_t s) {
-  long long n = (long long)T * p.n_heads;
+  const long long n = (long long)T * p.n_heads * p.half;
   if (n == 0) return cudaSuccess;
-  int threads = 256;
-  long long blocks = (n + threads - 1) / threads;
+  const int threads = 256;
+  const long long blocks = (n + threads - 1) / threads;
   rotation_table_kernel<<<(unsigned)blocks, threads, 0, s>>>(ts, cu, n_users, T, p, idx_out, cos_out,
                                                              sin_out, err);
   return cudaGetLastError();
@@ -568,6 +569,42 @@ static cudaError_t dec_dispatch(int hd, const DecAttnArgs& a, cudaStream_t s) {
     case 64: dec_attn_simt_kernel<T, 64><<<grid, ATT_ROWS, 0, s>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
+}
+
+// Split-key decoder: out = (sum_s 2^(m_s - M) O_s) / (sum_s 2^(m_s - M) l_s) * g,
+// M = max_s m_s; one thread per 4 output columns of a row.
+__global__ void dec_combine_kernel(DecAttnArgs a, int hd) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int cols4 = a.d / 4;
+  if (gid >= a.nk_rows * cols4) return;
+  const long long row = gid / cols4;
+  const int c = (int)(gid % cols4) * 4;
+  const int h = c / hd;
+  float M = -INFINITY;
+  for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, a.part_ml[((s * a.nk_rows + row) * a.n_heads + h) * 2]);
+  float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < a.n_split; ++s) {
+    const float* ml = a.part_ml + ((s * a.nk_rows + row) * a.n_heads + h) * 2;
+    if (ml[0] == -INFINITY) continue;  // a split with no keys
+    const float w = exp2f(ml[0] - M);
+    L = fmaf(w, ml[1], L);
+    float v[4];
+    load4(a.part_o + (s * a.nk_rows + row) * a.d + c, v);
+    for (int i = 0; i < 4; ++i) o[i] = fmaf(w, v[i], o[i]);
+  }
+  float g[4];
+  load4(a.g + row * a.d + c, g);
+  const float inv = 1.0f / L;
+  float r[4] = {o[0] * inv * g[0], o[1] * inv * g[1], o[2] * inv * g[2], o[3] * inv * g[3]};
+  store4(a.out + row * a.d + c, r);
+}
+
+cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s) {
+  const long long n = a.nk_rows * (a.d / 4);
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  dec_combine_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(a, hd);
   return cudaGetLastError();
 }
 

@@ -106,11 +106,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (DEC) {
     DecTile t = da.tiles[tile];
     q_row0 = t.row0;
-    key_row0 = t.key0;
-    nkeys = t.nkeys;
+    key_row0 = t.key0 + t.kb0 * KB;  // this work item's keys: blocks kb0 .. kb1-1
+    nkeys = t.nkeys - t.kb0 * KB;
     for (int i = 0; i < NT; ++i) {
       nrow[i] = max(0, min(ROWS, t.nrows - i * ROWS));
-      nblk[i] = nrow[i] > 0 ? (t.nkeys + KB - 1) / KB : 0;
+      nblk[i] = nrow[i] > 0 ? t.kb1 - t.kb0 : 0;
     }
   } else {
     EncTile t = ea.tiles[tile];
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idO = idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
       bool ok = true;
       for (int t = 0; t < NT && ok; ++t)
-        if (nrow[t] > 0) ok = mbar_wait(&q_full[t], 0, err, &abort_flag);
+        if (nblk[t] > 0) ok = mbar_wait(&q_full[t], 0, err, &abort_flag);  // staged only when the tile has keys
       tc_fence_after();
       for (int j = 0; ok && j <= nblk_all; ++j) {
         const int st = j % STAGES;
@@ -370,6 +370,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = mbar_wait(&p_free[t], (nb - 1) & 1, err, &abort_flag);  // the last P V has completed
       tc_fence_after();
     }
+    const bool split = DEC && da.n_split > 1;
+    const long long row_g = (long long)(q_row0 + t * ROWS + r);
     if (nb > 0) {
       // every lane takes part in the (warp-collective) TMEM loads
       float o[HD];
@@ -380,9 +382,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[c0 + e] = v32[e];
       }
-      if (ok && valid) {
+      if (ok && valid && split) {  // partial result of this key range, combined later
+        const int sp = da.tiles[tile].split;
+        float* po = da.part_o + ((long long)sp * da.nk_rows + row_g) * d + h * HD;
+#pragma unroll
+        for (int c = 0; c < HD; c += 4) store4(po + c, &o[c]);
+        float* pml = da.part_ml + (((long long)sp * da.nk_rows + row_g) * n_heads + h) * 2;
+        pml[0] = m_ref;
+        pml[1] = l_run;
+      } else if (ok && valid) {
         const float inv = 1.0f / l_run;
-        const long long ro = (long long)(q_row0 + t * ROWS + r) * d + h * HD;
+        const long long ro = row_g * d + h * HD;
         const float* gate = (DEC ? da.g : ea.gate) + ro;
 #pragma unroll
         for (int c = 0; c < HD; c += 4) {
@@ -395,6 +405,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             store4((bf16*)ea.out + ro + c, v);
         }
       }
+    } else if (split && valid) {  // an empty key range: a partial that carries no weight
+      const int sp = da.tiles[tile].split;
+      float* po = da.part_o + ((long long)sp * da.nk_rows + row_g) * d + h * HD;
+      const float z4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < HD; c += 4) store4(po + c, z4);
+      float* pml = da.part_ml + (((long long)sp * da.nk_rows + row_g) * n_heads + h) * 2;
+      pml[0] = -INFINITY;
+      pml[1] = 0.f;
     }
   }
   tc_fence_before();

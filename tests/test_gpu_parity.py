@@ -120,6 +120,29 @@ def test_bf16_decoder_with_synthetic_memory(cuda):
     assert_parity(y, oracle_decode(inp, Hm), "bf16", "y")
 
 
+@pytest.mark.parametrize("hd", [32, 64])
+def test_bf16_decoder_split_keys(cuda, hd):
+    """Few query rows against long prefixes: the tensor-core decoder splits the
+    keys across CTAs (one split of the 300-key request is empty) and combines
+    the partial results."""
+    w = W.small_workload("bf16", lengths=(2000, 300), d=4 * hd, n_heads=4,
+                         requests=[(0, 2000, 20), (1, 300, 7), (0, 1, 3), (0, 1500, 2)])
+    inp = W.make_inputs(w, 47)
+    Hm = W.make_memory(w, 47)
+    y = run_decoder(inp, Hm, cuda)
+    assert_parity(y, oracle_decode(inp, Hm), "bf16", "y")
+
+
+def test_bf16_rank_request_split_keys(cuda):
+    w = W.small_workload("bf16", lengths=(1800, 300), d=128, n_heads=4, n_layers=1, l_switch=0,
+                         requests=[(0, 1800, 12), (1, 300, 5), (0, 400, 3)])
+    inp = W.make_inputs(w, 48)
+    H, y = run_rank(inp, cuda)
+    Hr, yr = O.rank_request(inp)
+    assert_parity(H, Hr, "bf16", "H")
+    assert_parity(y, yr, "bf16", "y")
+
+
 # ------------------------------------------------------------- properties on the GPU
 
 def test_causality_on_gpu(cuda):
