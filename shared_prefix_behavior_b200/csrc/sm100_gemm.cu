@@ -26,7 +26,7 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int BOX_B_BYTES = 64 * BK * 2;  // one 64-column box of B: 8 KB
 
@@ -55,8 +55,11 @@ __device__ __forceinline__ void store32(T* p, const float (&v)[32]) {
 
 // Every lane executes the (warp-collective) TMEM loads; only rows < M touch
 // global memory.
+// Columns [part * span, (part + 1) * span) of the tile, span = BN / nparts
+// (paired epilogues: of each half).
 template <int BN>
-__device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, int m, int t, bool valid) {
+__device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, int m, int t, bool valid, int part,
+                                         int nparts) {
   float v[32];
   const long long ro = (long long)m * a.ldo;
   if (a.epi == EPI_QKVG || a.epi == EPI_SWIGLU) {
@@ -70,7 +73,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
         bf16* out = (bf16*)(isq ? a.out0 : a.out1) + ro + col0;
         const float* ct = a.cos_t + (long long)m * (d / 2) + col0 / 2;
         const float* st = a.sin_t + (long long)m * (d / 2) + col0 / 2;
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        for (int c0 = part * BN / nparts; c0 < (part + 1) * BN / nparts; c0 += 32) {
           tmem_ld32(tmem_row + c0, v);
           if (!valid) continue;
           float w[32];
@@ -93,7 +96,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
       if (t < 2 * nQ + nV) {  // value gate: V' = sigmoid(Gv) * V (eq. 3)
         const int col0 = (t - 2 * nQ) * half;
         bf16* out = (bf16*)a.out2 + ro + col0;
-        for (int c0 = 0; c0 < half; c0 += 32) {
+        for (int c0 = part * half / nparts; c0 < (part + 1) * half / nparts; c0 += 32) {
           float g[32];
           tmem_ld32(tmem_row + c0, v);
           tmem_ld32(tmem_row + half + c0, g);
@@ -106,7 +109,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
       }
       // output gate sigmoid(Go) (eq. 4), fp32
       float* out = (float*)a.out3 + ro + (t - 2 * nQ - nV) * BN;
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = part * BN / nparts; c0 < (part + 1) * BN / nparts; c0 += 32) {
         tmem_ld32(tmem_row + c0, v);
         if (!valid) continue;
 #pragma unroll
@@ -117,7 +120,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
     }
     // SwiGLU: SiLU(x W_1) * (x W_3)
     bf16* out = (bf16*)a.out0 + ro + t * half;
-    for (int c0 = 0; c0 < half; c0 += 32) {
+    for (int c0 = part * half / nparts; c0 < (part + 1) * half / nparts; c0 += 32) {
       float u[32];
       tmem_ld32(tmem_row + c0, v);
       tmem_ld32(tmem_row + half + c0, u);
@@ -129,7 +132,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
     return;
   }
   const int n0 = t * BN;
-  for (int c0 = 0; c0 < BN; c0 += 32) {
+  for (int c0 = part * BN / nparts; c0 < (part + 1) * BN / nparts; c0 += 32) {
     tmem_ld32(tmem_row + c0, v);
     if (!valid) continue;
     switch (a.epi) {
@@ -159,31 +162,38 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
   }
 }
 
+// Persistent kernel: one CTA per SM walks the tiles t = blockIdx.x, +gridDim.x,
+// ... (N-tiles of one 128-row block adjacent, so concurrent CTAs share A and
+// B in L2). The accumulator is double-buffered in TMEM: the epilogue of tile
+// i runs while the MMAs of tile i+1 proceed.
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs a, int num_kb, int32_t* err) {
+                   const GemmArgs a, int num_kb, int n_tiles_n, int n_tiles, int32_t* err) {
   constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+  constexpr int EPI_THREADS = NUM_THREADS - 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[STAGES], empty[STAGES], accf, drain;
+  __shared__ uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tslot;
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x, mt = blockIdx.y;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], EPI_THREADS);
+    }
     mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(&tslot, BN);
+  if (warp == 1) tmem_alloc(&tslot, 2 * BN);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -193,68 +203,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------ TMA producer
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    int issued = 0;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % STAGES;
-      if (!mbar_wait(&empty[s], ((kb / STAGES) & 1) ^ 1, err, &abort_flag)) break;
-      uint8_t* st = smem + s * STAGE_BYTES;
-      mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-      tma_load_2d(st, &tmA, kb * BK, mt * BM, &full[s]);
+    int it = 0, issued = 0;
+    for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
+      const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err, &abort_flag)) break;
+        uint8_t* st = smem + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+        tma_load_2d(st, &tmA, kb * BK, mt * BM, &full[s]);
 #pragma unroll
-      for (int b = 0; b < BN / 64; ++b)
-        tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &tmB, b_box_col(a, BN, t, b), kb * BK, &full[s]);
-      issued = kb + 1;
+        for (int b = 0; b < BN / 64; ++b)
+          tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &tmB, b_box_col(a, BN, t, b), kb * BK, &full[s]);
+        issued = it + 1;
+      }
     }
     if (abort_flag) {  // let the copies already in flight land before the CTA exits
-      for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb) {
-        volatile int no_abort = 0;
-        mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, &no_abort);
-      }
+      volatile int no_abort = 0;
+      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr, &no_abort);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = idesc_bf16(BN, 1);
+    int it = 0, i = 0;
     bool ok = true;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % STAGES;
-      if (!mbar_wait(&full[s], (kb / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++i) {
+      const int b = i & 1;
+      // the epilogue has drained this accumulator (tile i-2)
+      if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, err, &abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
-      const uint32_t b_base = a_base + A_BYTES;
+      const uint32_t acc = tmem + b * BN;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&full[s], (it / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
-      for (int k = 0; k < BK / 16; ++k) {
-        // A: K-major, 128B swizzle; a K step of 16 is 32 bytes inside the swizzle row
-        const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
-        // B: N-major, 128B swizzle; 8-row K groups 1024 B apart, 64-column boxes 8 KB apart
-        const uint64_t bd = smem_desc(b_base + k * 2048, BOX_B_BYTES, 1024, 2);
-        mma_bf16(tmem, ad, bd, idesc, (kb | k) != 0);
+        for (int k = 0; k < BK / 16; ++k) {
+          // A: K-major, 128B swizzle; a K step of 16 is 32 bytes inside the swizzle row
+          const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
+          // B: N-major, 128B swizzle; 8-row K groups 1024 B apart, 64-column boxes 8 KB apart
+          const uint64_t bd = smem_desc(b_base + k * 2048, BOX_B_BYTES, 1024, 2);
+          mma_bf16(acc, ad, bd, idesc, (kb | k) != 0);
+        }
+        mma_commit(&empty[s]);
       }
-      mma_commit(&empty[s]);
+      if (ok) mma_commit(&acc_full[b]);
     }
-    mma_commit(ok ? &accf : &drain);
-    if (!ok) {
-      volatile int no_abort = 0;
-      mbar_wait(&drain, 0, nullptr, &no_abort);
-    }
+    mma_commit(&drain);
+    volatile int no_abort = 0;
+    mbar_wait(&drain, 0, nullptr, &no_abort);
   } else if (warp >= 2) {
-    // ------------------------------------------------ epilogue
-    if (mbar_wait(&accf, 0, err, &abort_flag)) {
+    // ------------------------------------------------ epilogue (two warps per TMEM lane quarter)
+    const int q = warp & 3;
+    const int part = (warp - 2) >> 2;  // warps 2..5: first half of the columns, 6..9: second half
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    int i = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+      const int b = i & 1;
+      if (!mbar_wait(&acc_full[b], (i >> 1) & 1, err, &abort_flag)) break;
       tc_fence_after();
-      const int q = warp & 3;
+      const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
       const int m = mt * BM + q * 32 + lane;
-      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-      epilogue<BN>(a, trow, m, t, m < a.M);
+      epilogue<BN>(a, tmem + b * BN + lane_off, m, t, m < a.M, part, 2);
+      tc_fence_before();
+      mbar_arrive(&acc_empty[b]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
-
-// ------------------------------------------------------------------ host side
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -291,7 +315,7 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long 
 namespace {
 
 constexpr int TC_BN = 128;
-constexpr int TC_STAGES = 3;  // 97 KB of shared memory: two CTAs per SM, so one's epilogue overlaps the other's loads
+constexpr int TC_STAGES = 6;  // 192 KB of shared memory, one persistent CTA per SM
 
 template <int BN, int STAGES>
 cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
@@ -307,10 +331,17 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  int n_tiles = a.N / BN;
-  if (a.epi == EPI_QKVG) n_tiles = 5 * a.d / BN;
-  dim3 grid(n_tiles, (a.M + BM - 1) / BM);
-  gemm_tc_kernel<BN, STAGES><<<grid, NUM_THREADS, smem, s>>>(ma, mb, a, a.K / BK, err);
+  int n_tiles_n = a.N / BN;
+  if (a.epi == EPI_QKVG) n_tiles_n = 5 * a.d / BN;
+  const int n_tiles = n_tiles_n * ((a.M + BM - 1) / BM);
+  static int n_sm = 0;
+  if (n_sm == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n_sm = 148;
+  }
+  const int grid = n_tiles < n_sm ? n_tiles : n_sm;
+  gemm_tc_kernel<BN, STAGES><<<grid, NUM_THREADS, smem, s>>>(ma, mb, a, a.K / BK, n_tiles_n, n_tiles, err);
   return cudaGetLastError();
 }
 
