@@ -77,6 +77,31 @@ struct SmemLayout {
   static constexpr int TOTAL = P + NT * Cfg<HD>::P_BYTES;
 };
 
+// Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ void setmaxnreg_dec72() { asm volatile("setmaxnreg.dec.sync.aligned.u32 72;"); }
 __device__ __forceinline__ void setmaxnreg_inc216() { asm volatile("setmaxnreg.inc.sync.aligned.u32 216;"); }
 
@@ -312,14 +337,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int c = 0; c < KB; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      // row max of the raw scores (tree, for ILP)
+      // row max of the raw scores: 8 chains of three-input maxima
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[i], s[8 + i]);
 #pragma unroll
-      for (int c = 8; c < KB; c += 8)
+      for (int c = 16; c < KB; c += 16)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
+        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
       const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
       // P_t(j) replaces P_t(j-1): wait until O += P_t(j-1) V has completed
@@ -342,14 +367,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         l_run *= f;
         m_ref = m_blk;
       }
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
       for (int u = 0; u < KB / 8; ++u) {
         float p[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = exp2_approx(fmaf(s[8 * u + e], sl2, -m_ref));
-          sum[e & 3] += p[e];
+        for (int e = 0; e < 8; e += 2) {
+          const float2 x = ffma2(make_float2(s[8 * u + e], s[8 * u + e + 1]), scale2, neg_m2);
+          p[e] = exp2_approx(x.x);
+          p[e + 1] = exp2_approx(x.y);
+          sum2[(e >> 1) & 1] = fadd2(sum2[(e >> 1) & 1], make_float2(p[e], p[e + 1]));
         }
         uint32_t pk[4];
 #pragma unroll
@@ -361,7 +389,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         *reinterpret_cast<uint4*>(pb + chunk * (ROWS * 128) + r * 128 + ((uu ^ (r & 7)) * 16)) =
             make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      l_run += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      l_run += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
