@@ -47,115 +47,157 @@ __device__ __forceinline__ int b_box_col(const GemmArgs& a, int BN, int t, int b
   return t * BN + 64 * b;
 }
 
-template <typename T>
-__device__ __forceinline__ void store32(T* p, const float (&v)[32]) {
+__device__ __forceinline__ void store32(float* p, const float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; i += 4) store4(p + i, &v[i]);
+}
+// 32 bf16 values as four 16-byte stores
+__device__ __forceinline__ void store32(bf16* p, const float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    uint4 u;
+    __nv_bfloat162 t0 = __floats2bfloat162_rn(v[i], v[i + 1]), t1 = __floats2bfloat162_rn(v[i + 2], v[i + 3]);
+    __nv_bfloat162 t2 = __floats2bfloat162_rn(v[i + 4], v[i + 5]), t3 = __floats2bfloat162_rn(v[i + 6], v[i + 7]);
+    u.x = *reinterpret_cast<uint32_t*>(&t0);
+    u.y = *reinterpret_cast<uint32_t*>(&t1);
+    u.z = *reinterpret_cast<uint32_t*>(&t2);
+    u.w = *reinterpret_cast<uint32_t*>(&t3);
+    *reinterpret_cast<uint4*>(p + i) = u;
+  }
+}
+// sigmoid from the hardware base-2 exponential and reciprocal (relative
+// error about 3e-7; every consumer of these gates rounds to bf16 or feeds a
+// bf16 product)
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  const float e = exp2_approx(-1.4426950408889634f * x);
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+  return r;
 }
 
 // Every lane executes the (warp-collective) TMEM loads; only rows < M touch
 // global memory.
-// Columns [part * span, (part + 1) * span) of the tile, span = BN / nparts
-// (paired epilogues: of each half).
+// The epilogue of one 128 x BN tile, split between two warps per TMEM lane
+// quarter (part 0: the first half of the columns, part 1: the second half;
+// for the paired epilogues, of each half). Inputs that do not depend on the
+// accumulator (the residual row, the rotation table) are loaded by
+// epi_prefetch before the accumulator is waited for, so their latency hides
+// behind the tile's MMAs. Every lane executes the (warp-collective) TMEM
+// loads; only rows < M touch global memory.
+template <int BN>
+struct EpiIn {
+  float v[BN / 2];
+};
+
+template <int BN>
+__device__ __forceinline__ void epi_prefetch(const GemmArgs& a, int m, int t, bool valid, int part, EpiIn<BN>& in) {
+  if (!valid) return;
+  const long long ro = (long long)m * a.ldo;
+  if (a.epi == EPI_RESID) {
+    const float* p = (const float*)a.out0 + ro + t * BN + part * (BN / 2);
+#pragma unroll
+    for (int j = 0; j < BN / 2; j += 4) load4(p + j, &in.v[j]);
+  } else if (a.epi == EPI_QKVG) {
+    const int d = a.d, nQ = d / BN;
+    if (t < 2 * nQ) {  // cos and sin of the BN/4 column pairs of this part
+      const int col0 = (t < nQ ? t : t - nQ) * BN + part * (BN / 2);
+      const float* ct = a.cos_t + (long long)m * (d / 2) + col0 / 2;
+      const float* st = a.sin_t + (long long)m * (d / 2) + col0 / 2;
+#pragma unroll
+      for (int j = 0; j < BN / 4; j += 4) {
+        load4(ct + j, &in.v[j]);
+        load4(st + j, &in.v[BN / 4 + j]);
+      }
+    }
+  }
+}
+
 template <int BN>
 __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, int m, int t, bool valid, int part,
-                                         int nparts) {
+                                         const EpiIn<BN>& in) {
   float v[32];
   const long long ro = (long long)m * a.ldo;
-  if (a.epi == EPI_QKVG || a.epi == EPI_SWIGLU) {
-    const int half = BN / 2;
-    const int d = a.d;
-    if (a.epi == EPI_QKVG) {
-      const int nQ = d / BN, nV = d / half;
-      if (t < 2 * nQ) {  // Q or K: rotate the pairs (ReST eq. 5)
-        const bool isq = t < nQ;
-        const int col0 = (isq ? t : t - nQ) * BN;
-        bf16* out = (bf16*)(isq ? a.out0 : a.out1) + ro + col0;
-        const float* ct = a.cos_t + (long long)m * (d / 2) + col0 / 2;
-        const float* st = a.sin_t + (long long)m * (d / 2) + col0 / 2;
-        for (int c0 = part * BN / nparts; c0 < (part + 1) * BN / nparts; c0 += 32) {
-          tmem_ld32(tmem_row + c0, v);
-          if (!valid) continue;
-          float w[32];
+  const int half = BN / 2;
+  if (a.epi == EPI_QKVG) {
+    const int d = a.d, nQ = d / BN, nV = d / half;
+    if (t < 2 * nQ) {  // Q or K: rotate the pairs (ReST eq. 5)
+      const bool isq = t < nQ;
+      const int col0 = (isq ? t : t - nQ) * BN + part * half;
+      bf16* out = (bf16*)(isq ? a.out0 : a.out1) + ro + col0;
 #pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            float c[4], sn[4];
-            load4(ct + c0 / 2 + j, c);
-            load4(st + c0 / 2 + j, sn);
+      for (int c0 = 0; c0 < half; c0 += 32) {
+        tmem_ld32(tmem_row + part * half + c0, v);
+        if (!valid) continue;
+        float w[32];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int jj = j + i;
-              w[2 * jj] = v[2 * jj] * c[i] - v[2 * jj + 1] * sn[i];
-              w[2 * jj + 1] = v[2 * jj] * sn[i] + v[2 * jj + 1] * c[i];
-            }
-          }
-          store32(out + c0, w);
+        for (int jj = 0; jj < 16; ++jj) {
+          const float c = in.v[c0 / 2 + jj], sn = in.v[BN / 4 + c0 / 2 + jj];
+          w[2 * jj] = v[2 * jj] * c - v[2 * jj + 1] * sn;
+          w[2 * jj + 1] = v[2 * jj] * sn + v[2 * jj + 1] * c;
         }
-        return;
+        store32(out + c0, w);
       }
-      if (t < 2 * nQ + nV) {  // value gate: V' = sigmoid(Gv) * V (eq. 3)
-        const int col0 = (t - 2 * nQ) * half;
-        bf16* out = (bf16*)a.out2 + ro + col0;
-        for (int c0 = part * half / nparts; c0 < (part + 1) * half / nparts; c0 += 32) {
-          float g[32];
-          tmem_ld32(tmem_row + c0, v);
-          tmem_ld32(tmem_row + half + c0, g);
-          if (!valid) continue;
+      return;
+    }
+    if (t < 2 * nQ + nV) {  // value gate: V' = sigmoid(Gv) * V (eq. 3)
+      const int col0 = (t - 2 * nQ) * half + part * (half / 2);
+      bf16* out = (bf16*)a.out2 + ro + col0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= sigmoid_f(g[j]);
-          store32(out + c0, v);
-        }
-        return;
-      }
-      // output gate sigmoid(Go) (eq. 4), fp32
-      float* out = (float*)a.out3 + ro + (t - 2 * nQ - nV) * BN;
-      for (int c0 = part * BN / nparts; c0 < (part + 1) * BN / nparts; c0 += 32) {
-        tmem_ld32(tmem_row + c0, v);
+      for (int c0 = 0; c0 < half / 2; c0 += 32) {
+        float g[32];
+        tmem_ld32(tmem_row + part * (half / 2) + c0, v);
+        tmem_ld32(tmem_row + half + part * (half / 2) + c0, g);
         if (!valid) continue;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = sigmoid_f(v[j]);
+        for (int j = 0; j < 32; ++j) v[j] *= sigmoid_fast(g[j]);
         store32(out + c0, v);
       }
       return;
     }
-    // SwiGLU: SiLU(x W_1) * (x W_3)
-    bf16* out = (bf16*)a.out0 + ro + t * half;
-    for (int c0 = part * half / nparts; c0 < (part + 1) * half / nparts; c0 += 32) {
-      float u[32];
-      tmem_ld32(tmem_row + c0, v);
-      tmem_ld32(tmem_row + half + c0, u);
+    // output gate sigmoid(Go) (eq. 4), fp32
+    float* out = (float*)a.out3 + ro + (t - 2 * nQ - nV) * BN + part * half;
+#pragma unroll
+    for (int c0 = 0; c0 < half; c0 += 32) {
+      tmem_ld32(tmem_row + part * half + c0, v);
       if (!valid) continue;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = v[j] * sigmoid_f(v[j]) * u[j];
+      for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
       store32(out + c0, v);
     }
     return;
   }
-  const int n0 = t * BN;
-  for (int c0 = part * BN / nparts; c0 < (part + 1) * BN / nparts; c0 += 32) {
-    tmem_ld32(tmem_row + c0, v);
+  if (a.epi == EPI_SWIGLU) {  // SiLU(x W_1) * (x W_3)
+    bf16* out = (bf16*)a.out0 + ro + t * half + part * (half / 2);
+#pragma unroll
+    for (int c0 = 0; c0 < half / 2; c0 += 32) {
+      float u[32];
+      tmem_ld32(tmem_row + part * (half / 2) + c0, v);
+      tmem_ld32(tmem_row + half + part * (half / 2) + c0, u);
+      if (!valid) continue;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = v[j] * sigmoid_fast(v[j]) * u[j];
+      store32(out + c0, v);
+    }
+    return;
+  }
+  const int n0 = t * BN + part * half;
+#pragma unroll
+  for (int c0 = 0; c0 < half; c0 += 32) {
+    tmem_ld32(tmem_row + part * half + c0, v);
     if (!valid) continue;
     switch (a.epi) {
       case EPI_F32: store32((float*)a.out0 + ro + n0 + c0, v); break;
       case EPI_DT: store32((bf16*)a.out0 + ro + n0 + c0, v); break;
       case EPI_SIGMOID: {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = sigmoid_f(v[j]);
+        for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
         store32((float*)a.out0 + ro + n0 + c0, v);
         break;
       }
       case EPI_RESID: {
-        float* p = (float*)a.out0 + ro + n0 + c0;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          float x[4];
-          load4(p + j, x);
-          x[0] = fmaf(a.alpha, v[j], x[0]);
-          x[1] = fmaf(a.alpha, v[j + 1], x[1]);
-          x[2] = fmaf(a.alpha, v[j + 2], x[2]);
-          x[3] = fmaf(a.alpha, v[j + 3], x[3]);
-          store4(p + j, x);
-        }
+        for (int j = 0; j < 32; ++j) v[j] = fmaf(a.alpha, v[j], in.v[c0 + j]);
+        store32((float*)a.out0 + ro + n0 + c0, v);
         break;
       }
     }
@@ -263,11 +305,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int i = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
       const int b = i & 1;
-      if (!mbar_wait(&acc_full[b], (i >> 1) & 1, err, &abort_flag)) break;
-      tc_fence_after();
       const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
       const int m = mt * BM + q * 32 + lane;
-      epilogue<BN>(a, tmem + b * BN + lane_off, m, t, m < a.M, part, 2);
+      EpiIn<BN> in;
+      epi_prefetch<BN>(a, m, t, m < a.M, part, in);
+      if (!mbar_wait(&acc_full[b], (i >> 1) & 1, err, &abort_flag)) break;
+      tc_fence_after();
+      epilogue<BN>(a, tmem + b * BN + lane_off, m, t, m < a.M, part, in);
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
     }
