@@ -21,6 +21,7 @@ oracle alone as the reference arm.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -77,7 +78,7 @@ def workload_config(w: W.Workload, n: int) -> dict:
         "encoder_layers": w.n_layers,
         "candidates_per_gpu": w.total_cands,
         "query_tokens": w.K,
-        "parallelism": f"dp{n}: users sharded across ranks, no collective",
+        "parallelism": f"dp{n}: users LPT-sharded across ranks, no collective",
         "l2": "not flushed: one step writes and reads ~0.5 GB of activations, above the 126 MB L2",
     }
 
@@ -225,7 +226,22 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     w = W.workload(args.workload)
-    inp = W.make_inputs(w, 1000 + args.workload + 7919 * rank)
+    if world == 1:
+        inp = W.make_inputs(w, 1000 + args.workload)
+    else:
+        # one global batch of world x the workload's users (one model); this
+        # rank runs its LPT shard of the users (weak scaling, no collective)
+        from shared_prefix_behavior_b200 import shard as S
+        gw = W.tile_workload(w, world)
+        g = W.make_inputs(gw, 1000 + args.workload)
+        plan = S.partition_users(S.user_costs(g["cu_seqlens"], g["req_user"], g["req_cutoff"], g["cu_cands"],
+                                              gw.d, gw.n_layers, gw.d_ff, gw.K), world)
+        rows, cu, ru, rc, cc, cand_rows, _ = S.shard_arrays(g["cu_seqlens"], g["req_user"], g["req_cutoff"],
+                                                            g["cu_cands"], plan[rank])
+        inp = dict(g, x=g["x"][rows], ts=g["ts"][rows], cu_seqlens=cu, req_user=ru, req_cutoff=rc, cu_cands=cc,
+                   z=g["z"][cand_rows])
+        w = dataclasses.replace(w, lengths=[int(cu[i + 1] - cu[i]) for i in range(len(cu) - 1)],
+                                req_user=list(ru), req_cutoff=list(rc), req_ncand=list(np.diff(cc)))
     t = R.to_device(inp, dev)
     dt_name = "bf16" if w.dtype == "bf16" else "f32"
     args_rank = (t["x"], t["ts"], t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"], t["z"],
@@ -268,8 +284,12 @@ def main():
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
         ms = float(tm.item())
     ms_step = ms / args.steps
-    cands = w.total_cands * world
-    tokens = w.total_tokens * world
+    cands = w.total_cands
+    tokens = w.total_tokens
+    if world > 1:  # whole-job totals: every rank's shard
+        tot = torch.tensor([float(cands), float(tokens)], device=dev)
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+        cands, tokens = int(tot[0].item()), int(tot[1].item())
     value = cands / (ms_step * 1e-3)
 
     # per-kernel pass: the same steps with CUDA events around every launch
@@ -290,34 +310,47 @@ def main():
              torch.empty(Y.shape, dtype=torch.float32, device=dev)) for _ in range(2)]
     s_copy, s_comp = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     copied = [torch.cuda.Event() for _ in range(2)]
-    done = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(i):
-        k = i % 2
-        x_d, ts_d, z_d, y_d = bufs[k]
+    # copy stream: H2D(i), D2H(i-1), H2D(i+1), D2H(i), ...; compute stream: step i.
+    # D2H(i) waits for step i's compute; H2D(i+2) follows D2H(i) on the copy
+    # stream, so buffer set i%2 is free again when it is overwritten.
+    def h2d(i):
+        x_d, ts_d, z_d, _ = bufs[i % 2]
         with torch.cuda.stream(s_copy):
-            if i >= 2:
-                s_copy.wait_event(done[k])       # buffer k's previous step has finished
             x_d.copy_(x_h, non_blocking=True)
             ts_d.copy_(ts_h, non_blocking=True)
             z_d.copy_(z_h, non_blocking=True)
-            copied[k].record(s_copy)
+            copied[i % 2].record(s_copy)
+
+    def compute(i):
+        x_d, ts_d, z_d, y_d = bufs[i % 2]
         with torch.cuda.stream(s_comp):
-            s_comp.wait_event(copied[k])
+            s_comp.wait_event(copied[i % 2])
             R.rank_request(x_d, ts_d, t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"], z_d,
                            t["dec"], t["rope_base"], h_out=H, y_out=y_d, ws=ws, stream=s_comp, check=False)
-            y_h[k].copy_(y_d, non_blocking=True)
-            done[k].record(s_comp)
+            computed[i % 2].record(s_comp)
 
-    for i in range(2):
-        e2e_step(i)
+    def d2h(i):
+        with torch.cuda.stream(s_copy):
+            s_copy.wait_event(computed[i % 2])
+            y_h[i % 2].copy_(bufs[i % 2][3], non_blocking=True)
+
+    def e2e_run(n):
+        h2d(0)
+        for i in range(n):
+            compute(i)
+            if i + 1 < n:
+                h2d(i + 1)
+            d2h(i)
+
+    e2e_run(2)
     torch.cuda.synchronize()
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(s_copy)
     s_comp.wait_stream(s_copy)
-    for i in range(args.steps):
-        e2e_step(i)
+    e2e_run(args.steps)
     s_comp.wait_stream(s_copy)
     t1.record(s_comp)
     torch.cuda.synchronize()
@@ -369,7 +402,8 @@ def main():
                 "h2d_bytes_per_step": int(x_h.numel() * x_h.element_size() + ts_h.numel() * 8 +
                                           z_h.numel() * z_h.element_size()),
                 "d2h_bytes_per_step": int(y_h[0].numel() * 4),
-                "overlap": "inputs double-buffered: step i+1's copies overlap step i's compute"},
+                "overlap": "double-buffered: step i+1's input copies and step i-1's score copy-back run on a "
+                           "copy stream while step i computes"},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }

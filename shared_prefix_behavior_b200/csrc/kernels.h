@@ -36,7 +36,9 @@ enum Epilogue {
   EPI_SIGMOID = 2,  // out0[m, n] = sigmoid(acc) (fp32)
   EPI_RESID = 3,    // out0[m, n] += alpha * acc (fp32 residual stream)
   EPI_QKVG = 4,     // the DGA projection epilogue (rotation, value gate, output gate)
-  EPI_SWIGLU = 5    // out0[m, j] = dt(SiLU(acc_1) * acc_3)
+  EPI_SWIGLU = 5,   // out0[m, j] = dt(SiLU(acc_1) * acc_3)
+  EPI_DECQG = 6     // decoder token-specific projections, all token types in one launch:
+                    // q[n, k] = z[n, k] W_Q^(k) -> out0, sigmoid(z[n, k] W_go^(k)) -> out1
 };
 struct GemmArgs {
   const void* A; long long lda;   // [M, K], row stride lda elements
@@ -49,6 +51,9 @@ struct GemmArgs {
   float alpha;
   int d;                          // model width (EPI_QKVG) or d_ff (EPI_SWIGLU)
   int a_f32;                      // A is fp32 even when the call's dtype is bf16
+  const void* A2;                 // bf16 low part of A (A = A + A2, same layout), or null
+  const void* B2;                 // EPI_DECQG: the stacked W_go [K_tok * K, N] (B is W_Q)
+  int k_tok;                      // EPI_DECQG: number of token types
 };
 // Logical output columns of EPI_QKVG are [Q | K | V,Gv interleaved | Go] and of
 // EPI_SWIGLU [W1,W3 interleaved]: every group of 4 logical columns holds
@@ -78,7 +83,8 @@ struct DecAttnArgs {
   const float* g;      // [NK, d] sigmoid output gate
   const void* h;       // [T, d] encoder memory: keys and values
   const void* h_lo;    // [T, d] bf16 low part of H (H = h + h_lo), or null
-  float* out;          // [NK, d] o * g (fp32)
+  void* out;           // [NK, d] o * g: fp32, or its bf16 high part when out_lo is set
+  void* out_lo;        // [NK, d] bf16 low part of o * g, or null
   const DecTile* tiles; int n_tiles;
   int n_heads, d;
   float scale_log2;

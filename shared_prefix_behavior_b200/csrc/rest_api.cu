@@ -338,6 +338,7 @@ static double gemm_out_bytes(const GemmArgs& a, size_t e) {
     case EPI_RESID: return 8 * MN;
     case EPI_QKVG: return (double)a.M * a.d * (3 * e + 4) + 4.0 * a.M * a.d;  // + cos/sin reads
     case EPI_SWIGLU: return e * MN / 2;
+    case EPI_DECQG: return 8.0 * a.k_tok * MN;  // q and g, fp32, for every token type
   }
   return 0;
 }
@@ -345,8 +346,10 @@ static double gemm_out_bytes(const GemmArgs& a, size_t e) {
 static rest_status run_gemm(const Plan& p, const GemmArgs& a, const char* name, cudaStream_t s) {
   const bool bf = p.dt == REST_BF16;
   const size_t e = dt_size(p.dt);
-  const double flops = 2.0 * a.M * a.N * a.K;
-  const double bytes = (a.a_f32 ? 4 : e) * (double)a.M * a.K + e * (double)a.K * a.N + gemm_out_bytes(a, e);
+  const double groups = a.epi == EPI_DECQG ? 2.0 * a.k_tok : 1.0;  // (q, g) x token types
+  const double flops = 2.0 * a.M * a.N * a.K * groups;
+  const double bytes = (a.a_f32 || a.A2 ? 4 : e) * (double)a.M * a.K * (a.epi == EPI_DECQG ? a.k_tok : 1) +
+                       e * (double)a.K * a.N * groups + gemm_out_bytes(a, e);
   if (bf && sm100_gemm_supported(a)) {
     REST_KLAUNCH(s, name, flops, bytes, launch_gemm_sm100(a, s, p.err));
   } else {
@@ -454,7 +457,15 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   float* dg = at<float>(ws, L.dg);
   float* dout = at<float>(ws, L.dout);
   const long long N = p.n_cands;
-  // token-specific projections (eq. 8): rows n*K + k use W_Q^(k), W_go^(k)
+  // token-specific projections (eq. 8): rows n*K + k use W_Q^(k), W_go^(k);
+  // the tensor-core GEMM does all token types and both weights in one launch
+  GemmArgs qg = gemm(z, (long long)K * d, dec->w_q, d, N, d, d, EPI_DECQG, dq, (long long)K * d);
+  qg.out1 = dg;
+  qg.B2 = dec->w_go;
+  qg.k_tok = K;
+  if (bf && sm100_gemm_supported(qg)) {
+    if (rest_status st = run_gemm(p, qg, "gemm_dec_qg", s)) return st;
+  } else
   for (int kk = 0; kk < K; ++kk) {
     const char* zk = (const char*)z + e * (size_t)kk * d;
     GemmArgs a = gemm(zk, (long long)K * d, (const char*)dec->w_q + e * (size_t)kk * d * d, d, N, d, d, EPI_F32,
@@ -473,8 +484,12 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
     hbytes += (double)e * reqs->req_cutoff[r] * d * (h_lo ? 2 : 1);
   }
   const double bytes = hbytes + (double)p.NK * d * 12;
+  // The tensor-core decoder hands o * g to the output projection as a hi + lo
+  // pair of bf16 arrays (in the same workspace bytes); the CUDA-core one as fp32.
+  const bool tc = bf && sm100_attn_supported(hd);
   DecAttnArgs da;
   da.q = dq; da.g = dg; da.h = h; da.h_lo = h_lo; da.out = dout;
+  da.out_lo = tc ? (void*)((bf16*)dout + (size_t)p.NK * d) : nullptr;
   da.tiles = at<DecTile>(ws, L.dec_tiles); da.n_tiles = L.n_dec_tiles;
   da.n_heads = p.hs->n_heads; da.d = d;
   da.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
@@ -492,7 +507,10 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
     REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_simt(bf, hd, da, s));
   }
   GemmArgs a = gemm(dout, d, dec->w_o, d, p.NK, d, d, EPI_F32, y_out, d);
-  a.a_f32 = 1;
+  if (tc)
+    a.A2 = da.out_lo;
+  else
+    a.a_f32 = 1;
   if (rest_status st = run_gemm(p, a, "gemm_dec_out", s)) return st;
   return REST_OK;
 }

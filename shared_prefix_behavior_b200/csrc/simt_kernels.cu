@@ -292,7 +292,14 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
   for (int k0 = 0; k0 < a.K; k0 += BK) {
     float av[4] = {0.f, 0.f, 0.f, 0.f};
     int gm = m0 + ar;
-    if (gm < a.M) load4(A + (long long)gm * a.lda + k0 + ak, av);
+    if (gm < a.M) {
+      load4(A + (long long)gm * a.lda + k0 + ak, av);
+      if (a.A2) {  // A = A + A2 (a bf16 hi + lo pair)
+        float lv[4];
+        load4((const TA*)a.A2 + (long long)gm * a.lda + k0 + ak, lv);
+        for (int i = 0; i < 4; ++i) av[i] += lv[i];
+      }
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) As[ak + i][ar] = av[i];
     const T* brow = B + (long long)(k0 + bk) * a.ldb;
@@ -544,7 +551,7 @@ __global__ void __launch_bounds__(ATT_ROWS) dec_attn_simt_kernel(DecAttnArgs a) 
   }
   if (valid) {
     long long ro = row * a.d + hoff;
-    store_row<float, HD>(st, a.g + ro, a.out + ro);
+    store_row<float, HD>(st, a.g + ro, (float*)a.out + ro);
   }
 }
 
@@ -597,7 +604,14 @@ __global__ void dec_combine_kernel(DecAttnArgs a, int hd) {
   load4(a.g + row * a.d + c, g);
   const float inv = 1.0f / L;
   float r[4] = {o[0] * inv * g[0], o[1] * inv * g[1], o[2] * inv * g[2], o[3] * inv * g[3]};
-  store4(a.out + row * a.d + c, r);
+  if (a.out_lo) {  // as a hi + lo pair of bf16 values
+    float lo[4];
+    for (int i = 0; i < 4; ++i) lo[i] = r[i] - __bfloat162float(__float2bfloat16_rn(r[i]));
+    store4((bf16*)a.out + row * a.d + c, r);
+    store4((bf16*)a.out_lo + row * a.d + c, lo);
+  } else {
+    store4((float*)a.out + row * a.d + c, r);
+  }
 }
 
 cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s) {

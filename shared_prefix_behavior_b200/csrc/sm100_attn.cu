@@ -427,10 +427,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float g[4];
           load4(gate + c, g);
           float v[4] = {o[c] * inv * g[0], o[c + 1] * inv * g[1], o[c + 2] * inv * g[2], o[c + 3] * inv * g[3]};
-          if (DEC)
-            store4(da.out + ro + c, v);
-          else
+          if (DEC && da.out_lo) {  // o * g as a hi + lo pair of bf16 values
+            float lo[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
+            store4((bf16*)da.out + ro + c, v);
+            store4((bf16*)da.out_lo + ro + c, lo);
+          } else if (DEC) {
+            store4((float*)da.out + ro + c, v);
+          } else {
             store4((bf16*)ea.out + ro + c, v);
+          }
         }
       }
     } else if (split && valid) {  // an empty key range: a partial that carries no weight

@@ -180,6 +180,21 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
     }
     return;
   }
+  if (a.epi == EPI_DECQG) {  // q (fp32) or the sigmoid gate (fp32) of token k
+    const int per = a.N / BN, g = t / per, nt = t % per, k = g % a.k_tok;
+    float* out = (float*)(g < a.k_tok ? a.out0 : a.out1) + ro + (long long)k * a.N + nt * BN + part * half;
+#pragma unroll
+    for (int c0 = 0; c0 < half; c0 += 32) {
+      tmem_ld32(tmem_row + part * half + c0, v);
+      if (!valid) continue;
+      if (g >= a.k_tok) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
+      }
+      store32(out + c0, v);
+    }
+    return;
+  }
   const int n0 = t * BN + part * half;
 #pragma unroll
   for (int c0 = 0; c0 < half; c0 += 32) {
@@ -210,8 +225,11 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, i
 // i runs while the MMAs of tile i+1 proceed.
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs a, int num_kb, int n_tiles_n, int n_tiles, int32_t* err) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2, const GemmArgs a,
+                   int num_kb, int n_tiles_n, int n_tiles, int32_t* err) {
+  // with a low part A2, the K loop runs twice: A . B, then A2 . B
+  const int nkb = a.A2 ? 2 * num_kb : num_kb;
   constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
   constexpr int EPI_THREADS = NUM_THREADS - 64;
   extern __shared__ uint8_t smem_raw[];
@@ -244,19 +262,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA producer
     prefetch_tmap(&tmA);
+    if (a.A2) prefetch_tmap(&tmA2);
     prefetch_tmap(&tmB);
+    if (a.B2) prefetch_tmap(&tmB2);
     int it = 0, issued = 0;
     for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
       const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % STAGES;
+        const int kk = kb < num_kb ? kb : kb - num_kb;
         if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err, &abort_flag)) break;
         uint8_t* st = smem + s * STAGE_BYTES;
         mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-        tma_load_2d(st, &tmA, kb * BK, mt * BM, &full[s]);
+        if (a.epi == EPI_DECQG) {
+          // tile t: group g (q of token k = g, or the gate of token k = g - k_tok), N-tile nt
+          const int per = a.N / BN, g = t / per, nt = t % per, k = g % a.k_tok;
+          tma_load_2d(st, &tmA, k * a.K + kk * BK, mt * BM, &full[s]);
 #pragma unroll
-        for (int b = 0; b < BN / 64; ++b)
-          tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &tmB, b_box_col(a, BN, t, b), kb * BK, &full[s]);
+          for (int b = 0; b < BN / 64; ++b)
+            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, g < a.k_tok ? &tmB : &tmB2, nt * BN + 64 * b,
+                        k * a.K + kk * BK, &full[s]);
+        } else {
+          tma_load_2d(st, kb < num_kb ? &tmA : &tmA2, kk * BK, mt * BM, &full[s]);
+#pragma unroll
+          for (int b = 0; b < BN / 64; ++b)
+            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &tmB, b_box_col(a, BN, t, b), kk * BK, &full[s]);
+        }
         issued = it + 1;
       }
     }
@@ -276,7 +307,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, err, &abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t acc = tmem + b * BN;
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % STAGES;
         if (!mbar_wait(&full[s], (it / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -363,10 +394,22 @@ constexpr int TC_STAGES = 6;  // 192 KB of shared memory, one persistent CTA per
 
 template <int BN, int STAGES>
 cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
-  CUtensorMap ma, mb;
-  if (!make_tmap_bf16(&ma, a.A, a.M, a.K, a.lda, BK, BM, 128)) return cudaErrorInvalidValue;
-  // B is [K, Ncols] with Ncols = ldb (the full weight width)
-  if (!make_tmap_bf16(&mb, a.B, a.K, a.ldb, a.ldb, 64, BK, 128)) return cudaErrorInvalidValue;
+  CUtensorMap ma, ma2, mb, mb2;
+  if (a.epi == EPI_DECQG) {
+    // A: z as [M, k_tok * K]; B, B2: the stacked [k_tok * K, N] weights
+    if (!make_tmap_bf16(&ma, a.A, a.M, (long long)a.k_tok * a.K, a.lda, BK, BM, 128) ||
+        !make_tmap_bf16(&mb, a.B, (long long)a.k_tok * a.K, a.N, a.ldb, 64, BK, 128) ||
+        !make_tmap_bf16(&mb2, a.B2, (long long)a.k_tok * a.K, a.N, a.ldb, 64, BK, 128))
+      return cudaErrorInvalidValue;
+    ma2 = ma;
+  } else {
+    if (!make_tmap_bf16(&ma, a.A, a.M, a.K, a.lda, BK, BM, 128)) return cudaErrorInvalidValue;
+    ma2 = ma;
+    if (a.A2 && !make_tmap_bf16(&ma2, a.A2, a.M, a.K, a.lda, BK, BM, 128)) return cudaErrorInvalidValue;
+    // B is [K, Ncols] with Ncols = ldb (the full weight width)
+    if (!make_tmap_bf16(&mb, a.B, a.K, a.ldb, a.ldb, 64, BK, 128)) return cudaErrorInvalidValue;
+    mb2 = mb;
+  }
   constexpr int smem = STAGES * (A_BYTES + BN * BK * 2) + 1024;
   static bool attr_set = false;
   if (!attr_set) {
@@ -377,6 +420,7 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   }
   int n_tiles_n = a.N / BN;
   if (a.epi == EPI_QKVG) n_tiles_n = 5 * a.d / BN;
+  if (a.epi == EPI_DECQG) n_tiles_n = 2 * a.k_tok * (a.N / BN);
   const int n_tiles = n_tiles_n * ((a.M + BM - 1) / BM);
   static int n_sm = 0;
   if (n_sm == 0) {
@@ -385,7 +429,7 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
       n_sm = 148;
   }
   const int grid = n_tiles < n_sm ? n_tiles : n_sm;
-  gemm_tc_kernel<BN, STAGES><<<grid, NUM_THREADS, smem, s>>>(ma, mb, a, a.K / BK, n_tiles_n, n_tiles, err);
+  gemm_tc_kernel<BN, STAGES><<<grid, NUM_THREADS, smem, s>>>(ma, ma2, mb, mb2, a, a.K / BK, n_tiles_n, n_tiles, err);
   return cudaGetLastError();
 }
 
@@ -398,6 +442,7 @@ bool sm100_gemm_supported(const GemmArgs& a) {
   switch (a.epi) {
     case EPI_QKVG: return a.d % TC_BN == 0 && a.N == 5 * a.d && a.ldb == 5LL * a.d;
     case EPI_SWIGLU: return a.d % (TC_BN / 2) == 0 && a.N == 2 * a.d && a.ldb == 2LL * a.d;
+    case EPI_DECQG: return a.N % TC_BN == 0 && a.ldb == a.N && a.B2 != nullptr && a.k_tok >= 1;
     default: return a.N % TC_BN == 0 && a.ldb == a.N;
   }
 }

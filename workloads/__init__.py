@@ -307,3 +307,14 @@ def subset_users(inp: dict, users, with_requests=True) -> dict:
                    z=inp["z"][cand_rows], _cand_rows=cand_rows)
     out["_rows"] = rows
     return out
+
+
+def tile_workload(w: Workload, n: int) -> Workload:
+    """The workload's users and requests repeated n times (one global batch)."""
+    if n == 1:
+        return w
+    U = w.n_users
+    return dataclasses.replace(
+        w, name=f"{w.name}x{n}", lengths=list(w.lengths) * n,
+        req_user=[u + i * U for i in range(n) for u in w.req_user],
+        req_cutoff=list(w.req_cutoff) * n, req_ncand=list(w.req_ncand) * n)
