@@ -75,6 +75,9 @@ struct EncAttnArgs {
   int n_heads, d;
   float scale_log2;                             // log2(e) / sqrt(head_dim)
   long long rows;                               // T, rows of the packed arrays
+  // tensor-core kernel: CTA c runs the work items (tile * n_heads + head)
+  // sched[n_cta + 1 + k] for k in [sched[c], sched[c + 1])
+  const int* sched; int n_cta;
 };
 cudaError_t launch_enc_attn_simt(bool bf16, int hd, const EncAttnArgs& a, cudaStream_t s);
 
@@ -96,6 +99,7 @@ struct DecAttnArgs {
   long long nk_rows;   // NK
   float* part_o;
   float* part_ml;
+  const int* sched; int n_cta;  // as in EncAttnArgs
 };
 cudaError_t launch_dec_attn_simt(bool bf16, int hd, const DecAttnArgs& a, cudaStream_t s);
 cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s);

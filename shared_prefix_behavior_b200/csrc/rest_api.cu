@@ -135,10 +135,64 @@ static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, 
                    [](const DecTile& a, const DecTile& c) { return a.kb1 - a.kb0 > c.kb1 - c.kb0; });
 }
 
+// Longest-processing-time assignment of attention work items to the
+// tensor-core kernel's persistent CTAs: items by decreasing cost (key blocks
+// times active query tiles), each to the least-loaded CTA. Returned as
+// [n_cta + 1 offsets | item ids], each CTA's items in decreasing cost.
+constexpr int SCHED_CTAS = 148;  // one persistent CTA per B200 SM
+
+static std::vector<int> lpt_schedule(const std::vector<long long>& cost) {
+  const int n = (int)cost.size();
+  const int n_cta = std::min(n, SCHED_CTAS);
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  std::vector<std::vector<int>> lists(n_cta);
+  std::vector<std::pair<long long, int>> heap;  // (load, cta), min-heap
+  for (int c = 0; c < n_cta; ++c) heap.push_back({0, c});
+  auto cmp = [](const std::pair<long long, int>& a, const std::pair<long long, int>& b) { return a > b; };
+  std::make_heap(heap.begin(), heap.end(), cmp);
+  for (int i : order) {
+    std::pop_heap(heap.begin(), heap.end(), cmp);
+    auto& top = heap.back();
+    lists[top.second].push_back(i);
+    top.first += std::max(1LL, cost[i]);
+    std::push_heap(heap.begin(), heap.end(), cmp);
+  }
+  std::vector<int> out(n_cta + 1 + n);
+  out[0] = 0;
+  int k = n_cta + 1;
+  for (int c = 0; c < n_cta; ++c) {
+    for (int i : lists[c]) out[k++] = i;
+    out[c + 1] = out[c] + (int)lists[c].size();
+  }
+  return out;
+}
+
+static std::vector<int> enc_schedule(const rest_batch* b, const std::vector<EncTile>& tiles, int n_heads, int rows) {
+  std::vector<long long> cost;
+  for (const EncTile& t : tiles) {
+    const int L = b->cu_seqlens[t.user + 1] - b->cu_seqlens[t.user];
+    long long c = 0;
+    for (int r0 = t.q0; r0 < std::min(L, t.q0 + rows); r0 += 128) c += (std::min(L, r0 + 128) + 127) / 128;
+    for (int h = 0; h < n_heads; ++h) cost.push_back(c);
+  }
+  return lpt_schedule(cost);
+}
+
+static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_heads) {
+  std::vector<long long> cost;
+  for (const DecTile& t : tiles) {
+    const long long c = (long long)(t.kb1 - t.kb0) * ((t.nrows + 127) / 128);
+    for (int h = 0; h < n_heads; ++h) cost.push_back(c);
+  }
+  return lpt_schedule(cost);
+}
+
 // ---------------------------------------------------------------- workspace
 
 struct Layout {
-  size_t cu, enc_tiles, dec_tiles, meta_end;
+  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
   size_t dq, dg, dout, hlo, part_o, part_ml;
   size_t total;
@@ -146,7 +200,8 @@ struct Layout {
 };
 
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
-                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split) {
+                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split,
+                          size_t n_enc_sched, size_t n_dec_sched) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -157,6 +212,8 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.cu = take(sizeof(int32_t) * (size_t)(b->n_users + 1));
   L.enc_tiles = take(sizeof(EncTile) * (size_t)n_enc_tiles);
   L.dec_tiles = take(sizeof(DecTile) * (size_t)n_dec_tiles);
+  L.enc_sched = take(sizeof(int) * n_enc_sched);
+  L.dec_sched = take(sizeof(int) * n_dec_sched);
   L.meta_end = off;
   L.cos_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
   L.sin_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
@@ -186,6 +243,7 @@ struct Plan {
   int max_dff, K;
   std::vector<EncTile> enc_tiles;
   std::vector<DecTile> dec_tiles;
+  std::vector<int> enc_sched, dec_sched;  // tensor-core attention: per-CTA item lists
   Layout L;
   int32_t* err;
   bool hsplit;
@@ -224,8 +282,12 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   build_dec_tiles(b, reqs, K, tile_rows, p.n_split, p.dec_tiles);
   // encoder followed by the decoder in bf16: the decoder reads H as hi + lo
   p.hsplit = encoder_runs && reqs != nullptr && dt == REST_BF16;
+  if (tile_rows != 128) {  // the tensor-core attention runs: schedule its persistent CTAs
+    if (!p.enc_tiles.empty()) p.enc_sched = enc_schedule(b, p.enc_tiles, hs->n_heads, tile_rows);
+    if (!p.dec_tiles.empty()) p.dec_sched = dec_schedule(p.dec_tiles, hs->n_heads);
+  }
   p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),
-                    (int)p.dec_tiles.size(), p.hsplit, p.n_split);
+                    (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size());
   return REST_OK;
 }
 
@@ -307,6 +369,10 @@ static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
     memcpy(host.data() + p.L.enc_tiles, p.enc_tiles.data(), sizeof(EncTile) * p.enc_tiles.size());
   if (!p.dec_tiles.empty())
     memcpy(host.data() + p.L.dec_tiles, p.dec_tiles.data(), sizeof(DecTile) * p.dec_tiles.size());
+  if (!p.enc_sched.empty())
+    memcpy(host.data() + p.L.enc_sched, p.enc_sched.data(), sizeof(int) * p.enc_sched.size());
+  if (!p.dec_sched.empty())
+    memcpy(host.data() + p.L.dec_sched, p.dec_sched.data(), sizeof(int) * p.dec_sched.size());
   if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) return REST_ERR_CUDA;
   return REST_OK;
 }
@@ -393,6 +459,8 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   EncAttnArgs ea;
   ea.q = q; ea.k = k; ea.v = v; ea.gate = g; ea.out = o; ea.cu = cu;
   ea.tiles = at<EncTile>(ws, L.enc_tiles); ea.n_tiles = L.n_enc_tiles;
+  ea.sched = at<int>(ws, L.enc_sched);
+  ea.n_cta = p.enc_sched.empty() ? 0 : std::min((int)p.enc_tiles.size() * H, SCHED_CTAS);
   ea.n_heads = H; ea.d = d;
   ea.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
   ea.rows = T;
@@ -491,6 +559,8 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   da.q = dq; da.g = dg; da.h = h; da.h_lo = h_lo; da.out = dout;
   da.out_lo = tc ? (void*)((bf16*)dout + (size_t)p.NK * d) : nullptr;
   da.tiles = at<DecTile>(ws, L.dec_tiles); da.n_tiles = L.n_dec_tiles;
+  da.sched = at<int>(ws, L.dec_sched);
+  da.n_cta = p.dec_sched.empty() ? 0 : std::min((int)p.dec_tiles.size() * p.hs->n_heads, SCHED_CTAS);
   da.n_heads = p.hs->n_heads; da.d = d;
   da.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
   da.key_rows = p.T;

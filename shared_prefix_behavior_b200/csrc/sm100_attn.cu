@@ -105,6 +105,59 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ void setmaxnreg_dec72() { asm volatile("setmaxnreg.dec.sync.aligned.u32 72;"); }
 __device__ __forceinline__ void setmaxnreg_inc216() { asm volatile("setmaxnreg.inc.sync.aligned.u32 216;"); }
 
+// One work item: 256 query rows (two 128-row tiles) of one head.
+struct AttnItem {
+  int q_row0;     // packed row of query row 0 of tile 0
+  int key_row0;   // packed row of the item's first key
+  int nrow[NT];   // valid query rows of each tile
+  int nblk[NT];   // key blocks each tile reads
+  int user_len;   // encoder: the user's history length
+  int q_pos0;     // encoder: position of query row 0 within the user
+  int nkeys;      // keys from key_row0 visible to the item (decoder: cutoff minus the split start)
+  int split;      // decoder: split index of the partial result
+  int h;          // head
+};
+
+template <bool DEC>
+__device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const DecAttnArgs& da, int item) {
+  AttnItem w;
+  const int n_heads = DEC ? da.n_heads : ea.n_heads;
+  const int tile = item / n_heads;
+  w.h = item % n_heads;
+  if (DEC) {
+    const DecTile t = da.tiles[tile];
+    w.q_row0 = t.row0;
+    w.key_row0 = t.key0 + t.kb0 * KB;  // this item's keys: blocks kb0 .. kb1-1
+    w.nkeys = t.nkeys - t.kb0 * KB;
+    w.user_len = 0;
+    w.q_pos0 = 0;
+    w.split = t.split;
+    for (int i = 0; i < NT; ++i) {
+      w.nrow[i] = max(0, min(ROWS, t.nrows - i * ROWS));
+      w.nblk[i] = w.nrow[i] > 0 ? t.kb1 - t.kb0 : 0;
+    }
+  } else {
+    const EncTile t = ea.tiles[tile];
+    w.key_row0 = ea.cu[t.user];
+    w.user_len = ea.cu[t.user + 1] - w.key_row0;
+    w.q_pos0 = t.q0;
+    w.q_row0 = w.key_row0 + t.q0;
+    w.nkeys = 0;
+    w.split = 0;
+    for (int i = 0; i < NT; ++i) {
+      const int r0 = t.q0 + i * ROWS;
+      w.nrow[i] = max(0, min(ROWS, w.user_len - r0));
+      w.nblk[i] = w.nrow[i] > 0 ? (min(w.user_len, r0 + ROWS) + KB - 1) / KB : 0;
+    }
+  }
+  return w;
+}
+
+// Persistent: one CTA per SM walks its own list of work items (a
+// longest-processing-time schedule built on the host: sched[n_cta + 1 + k] for
+// k in [sched[c], sched[c + 1])). TMEM, barriers and the pipelines persist
+// across items; every role keeps, per tile, the count of key blocks (cb) and of
+// items with work (qn) processed so far, from which all barrier parities follow.
 template <int HD, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -115,48 +168,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr int STAGES = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t q_full[NT], kv_full[STAGES], kv_empty[STAGES], s_full[NT], p_full[NT], p_free[NT], drain;
+  // q_full: Q_t staged; q_empty: the item's last S_t has read Q_t; s_full / p_full /
+  // p_free: S_t(j) ready / P_t(j) written / O_t += P_t(j) V done; o_empty: the
+  // item's O_t has been read out of TMEM.
+  __shared__ uint64_t q_full[NT], q_empty[NT], kv_full[STAGES], kv_empty[STAGES], s_full[NT], p_full[NT], p_free[NT],
+      o_empty[NT], drain;
   __shared__ uint32_t tslot;
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_heads = DEC ? da.n_heads : ea.n_heads;
   const int d = DEC ? da.d : ea.d;
-  const int tile = blockIdx.x / n_heads, h = blockIdx.x % n_heads;
-
-  // ---------------------------------------------------------------- work item
-  // rows: first packed query row of tile 0; nrow[t]: valid rows of tile t;
-  // nblk[t]: key blocks tile t reads; key_row0: packed row of key 0.
-  int q_row0, key_row0, nrow[NT], nblk[NT], user_len = 0, q_pos0 = 0, nkeys = 0;
-  if (DEC) {
-    DecTile t = da.tiles[tile];
-    q_row0 = t.row0;
-    key_row0 = t.key0 + t.kb0 * KB;  // this work item's keys: blocks kb0 .. kb1-1
-    nkeys = t.nkeys - t.kb0 * KB;
-    for (int i = 0; i < NT; ++i) {
-      nrow[i] = max(0, min(ROWS, t.nrows - i * ROWS));
-      nblk[i] = nrow[i] > 0 ? t.kb1 - t.kb0 : 0;
-    }
-  } else {
-    EncTile t = ea.tiles[tile];
-    key_row0 = ea.cu[t.user];
-    user_len = ea.cu[t.user + 1] - key_row0;
-    q_pos0 = t.q0;
-    q_row0 = key_row0 + t.q0;
-    for (int i = 0; i < NT; ++i) {
-      const int r0 = t.q0 + i * ROWS;
-      nrow[i] = max(0, min(ROWS, user_len - r0));
-      nblk[i] = nrow[i] > 0 ? (min(user_len, r0 + ROWS) + KB - 1) / KB : 0;
-    }
-  }
-  const int nblk_all = max(nblk[0], nblk[1]);
+  const int* sched = DEC ? da.sched : ea.sched;
+  const int* items = sched + (DEC ? da.n_cta : ea.n_cta) + 1;
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < NT; ++t) {
       mbar_init(&q_full[t], DEC ? 128 : 1);
+      mbar_init(&q_empty[t], 1);
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
       mbar_init(&p_free[t], 1);
+      mbar_init(&o_empty[t], 128);
     }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -176,95 +209,117 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     setmaxnreg_dec72();
     if (warp == 0 && lane == 0) {
       // -------------------------------------------------------- TMA producer
-      if (!DEC) {
-        for (int t = 0; t < NT; ++t) {
-          if (nrow[t] == 0) continue;
-          mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
-          tma_load_2d(smem + L::Q + t * C::TILE_BYTES, &tmQ, h * HD, q_row0 + t * ROWS, &q_full[t]);
+      int g = 0, issued = 0, qn[NT] = {0, 0};
+      bool ok = true;
+      for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
+        const AttnItem w = decode_item<DEC>(ea, da, items[k]);
+        if (!DEC) {
+          for (int t = 0; t < NT && ok; ++t) {
+            if (w.nblk[t] == 0) continue;
+            if (qn[t] >= 1 && !mbar_wait(&q_empty[t], (qn[t] - 1) & 1, err, &abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
+            tma_load_2d(smem + L::Q + t * C::TILE_BYTES, &tmQ, w.h * HD, w.q_row0 + t * ROWS, &q_full[t]);
+            ++qn[t];
+          }
+        }
+        const int nblk_all = max(w.nblk[0], w.nblk[1]);
+        for (int j = 0; j < nblk_all && ok; ++j, ++g) {
+          const int st = g % STAGES;
+          if (!mbar_wait(&kv_empty[st], ((g / STAGES) & 1) ^ 1, err, &abort_flag)) { ok = false; break; }
+          uint8_t* base = smem + L::KV + st * L::STAGE;
+          mbar_arrive_expect_tx(&kv_full[st], L::STAGE);
+          tma_load_2d(base, &tmK, w.h * HD, w.key_row0 + j * KB, &kv_full[st]);
+          if (MODE != 1) tma_load_2d(base + C::TILE_BYTES, &tmV, w.h * HD, w.key_row0 + j * KB, &kv_full[st]);
+          issued = g + 1;
         }
       }
-      int issued = 0;
-      for (int j = 0; j < nblk_all; ++j) {
-        const int st = j % STAGES;
-        if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1, err, &abort_flag)) break;
-        uint8_t* base = smem + L::KV + st * L::STAGE;
-        mbar_arrive_expect_tx(&kv_full[st], L::STAGE);
-        tma_load_2d(base, &tmK, h * HD, key_row0 + j * KB, &kv_full[st]);
-        if (MODE != 1) tma_load_2d(base + C::TILE_BYTES, &tmV, h * HD, key_row0 + j * KB, &kv_full[st]);
-        issued = j + 1;
-      }
-      if (abort_flag) {  // let the copies in flight land before the CTA exits
+      if (!ok) {  // let the copies in flight land before the CTA exits
         volatile int no_abort = 0;
         if (!DEC)
           for (int t = 0; t < NT; ++t)
-            if (nrow[t] > 0) mbar_wait(&q_full[t], 0, nullptr, &no_abort);
-        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-          mbar_wait(&kv_full[j % STAGES], (j / STAGES) & 1, nullptr, &no_abort);
+            if (qn[t] >= 1) mbar_wait(&q_full[t], (qn[t] - 1) & 1, nullptr, &no_abort);
+        for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+          mbar_wait(&kv_full[i % STAGES], (i / STAGES) & 1, nullptr, &no_abort);
       }
     } else if (warp == 1 && lane == 0) {
       // -------------------------------------------------------- MMA issuer
       constexpr uint32_t idS = idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
       constexpr uint32_t idO = idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
+      int g = 0, cb[NT] = {0, 0}, qn[NT] = {0, 0};
       bool ok = true;
-      for (int t = 0; t < NT && ok; ++t)
-        if (nblk[t] > 0) ok = mbar_wait(&q_full[t], 0, err, &abort_flag);  // staged only when the tile has keys
-      tc_fence_after();
-      for (int j = 0; ok && j <= nblk_all; ++j) {
-        const int st = j % STAGES;
-        if (j < nblk_all) {
-          if (!mbar_wait(&kv_full[st], (j / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-        }
-        for (int t = 0; t < NT; ++t) {
-          // S_t(j) overwrites the tile's S buffer: the softmax has taken S_t(j-1)
-          // (and written P_t(j-1)) once p_full[t] completes its phase j-1.
-          if (j >= 1 && j - 1 < nblk[t]) {
-            if (!mbar_wait(&p_full[t], (j - 1) & 1, err, &abort_flag)) { ok = false; break; }
+      for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
+        const AttnItem w = decode_item<DEC>(ea, da, items[k]);
+        const int nblk_all = max(w.nblk[0], w.nblk[1]);
+        for (int t = 0; t < NT && ok; ++t)
+          if (w.nblk[t] > 0) ok = mbar_wait(&q_full[t], qn[t] & 1, err, &abort_flag);
+        tc_fence_after();
+        for (int j = 0; ok && j <= nblk_all; ++j) {
+          const int st = (g + j) % STAGES;
+          if (j < nblk_all) {
+            if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
             tc_fence_after();
           }
-          if (j < nblk[t]) {
-            const uint32_t k_base = smem_u32(smem + L::KV + st * L::STAGE);
-            const uint32_t q_base = smem_u32(smem + L::Q + t * C::TILE_BYTES);
-            const uint32_t tS = tmem + s_col(t);
-#pragma unroll
-            for (int k = 0; k < HD / 16; ++k)
-              mma_bf16(tS, smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ),
-                       smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, k != 0);
-            if (DEC) {  // + q_lo . H^T
-              const uint32_t qlo_base = smem_u32(smem + L::QLO + t * C::TILE_BYTES);
-#pragma unroll
-              for (int k = 0; k < HD / 16; ++k)
-                mma_bf16(tS, smem_desc(qlo_base + k * 32, 16, C::ATOM, C::SWZ),
-                         smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
+          for (int t = 0; t < NT; ++t) {
+            // S_t(j) overwrites the tile's S buffer: the softmax has taken S_t(j-1)
+            // (and written P_t(j-1)) once p_full[t] completes that block's phase.
+            if (j >= 1 && j - 1 < w.nblk[t]) {
+              if (!mbar_wait(&p_full[t], (cb[t] + j - 1) & 1, err, &abort_flag)) { ok = false; break; }
+              tc_fence_after();
             }
-            if (HLO) {  // + q_hi . H_lo^T
+            if (j < w.nblk[t]) {
+              const uint32_t k_base = smem_u32(smem + L::KV + st * L::STAGE);
+              const uint32_t q_base = smem_u32(smem + L::Q + t * C::TILE_BYTES);
+              const uint32_t tS = tmem + s_col(t);
 #pragma unroll
               for (int k = 0; k < HD / 16; ++k)
                 mma_bf16(tS, smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ),
-                         smem_desc(k_base + C::TILE_BYTES + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
-            }
-            mma_commit(&s_full[t]);
-          }
-          if (j >= 1 && j - 1 < nblk[t]) {  // O_t += P_t(j-1) V_{j-1}
-            const int i = j - 1, sti = i % STAGES;
-            const uint32_t p_base = smem_u32(smem + L::P + t * C::P_BYTES);
-            const uint32_t v_base = smem_u32(smem + L::KV + sti * L::STAGE + (DEC ? 0 : C::TILE_BYTES));
-            const uint32_t tO = tmem + o_col<HD>(t);
+                         smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, k != 0);
+              if (DEC) {  // + q_lo . H^T
+                const uint32_t qlo_base = smem_u32(smem + L::QLO + t * C::TILE_BYTES);
 #pragma unroll
-            for (int k = 0; k < KB / 16; ++k)
-              mma_bf16(tO, smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2),
-                       smem_desc(v_base + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO, (i | k) != 0);
-            if (HLO) {  // + P H_lo
+                for (int k = 0; k < HD / 16; ++k)
+                  mma_bf16(tS, smem_desc(qlo_base + k * 32, 16, C::ATOM, C::SWZ),
+                           smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
+              }
+              if (HLO) {  // + q_hi . H_lo^T
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                  mma_bf16(tS, smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ),
+                           smem_desc(k_base + C::TILE_BYTES + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
+              }
+              if (j == w.nblk[t] - 1) mma_commit(&q_empty[t]);  // the item's last read of Q_t
+              mma_commit(&s_full[t]);
+            }
+            if (j >= 1 && j - 1 < w.nblk[t]) {  // O_t += P_t(j-1) V_{j-1}
+              const int i = j - 1, sti = (g + i) % STAGES;
+              if (i == 0 && qn[t] >= 1 &&  // the previous item's O_t has been read out
+                  !mbar_wait(&o_empty[t], (qn[t] - 1) & 1, err, &abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t p_base = smem_u32(smem + L::P + t * C::P_BYTES);
+              const uint32_t v_base = smem_u32(smem + L::KV + sti * L::STAGE + (DEC ? 0 : C::TILE_BYTES));
+              const uint32_t tO = tmem + o_col<HD>(t);
 #pragma unroll
               for (int k = 0; k < KB / 16; ++k)
                 mma_bf16(tO, smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2),
-                         smem_desc(v_base + C::TILE_BYTES + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO,
-                         1);
+                         smem_desc(v_base + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO, (i | k) != 0);
+              if (HLO) {  // + P H_lo
+#pragma unroll
+                for (int k = 0; k < KB / 16; ++k)
+                  mma_bf16(tO, smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2),
+                           smem_desc(v_base + C::TILE_BYTES + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ),
+                           idO, 1);
+              }
+              mma_commit(&p_free[t]);
             }
-            mma_commit(&p_free[t]);
           }
+          if (j >= 1 && ok) mma_commit(&kv_empty[(g + j - 1) % STAGES]);  // block j-1 fully consumed
         }
-        if (j >= 1 && ok) mma_commit(&kv_empty[(j - 1) % STAGES]);  // block j-1 fully consumed
+        g += nblk_all;
+        for (int t = 0; t < NT; ++t)
+          if (w.nblk[t] > 0) {
+            cb[t] += w.nblk[t];
+            ++qn[t];
+          }
       }
       mma_commit(&drain);
       volatile int no_abort = 0;
@@ -277,130 +332,144 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q4 = warp & 3;                     // TMEM lane quarter
     const int r = q4 * 32 + lane;                // row within the tile
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const bool valid = r < nrow[t];
     const float sl2 = DEC ? da.scale_log2 : ea.scale_log2;
-    const int nb = nblk[t];
-
-    if (DEC && nb > 0) {  // stage q (fp32) as hi + lo bf16 tiles in the swizzled K-major layout
-      const float* qrow = da.q + (long long)(q_row0 + t * ROWS + (valid ? r : 0)) * d + h * HD;
-      uint8_t* qh = smem + L::Q + t * C::TILE_BYTES;
-      uint8_t* ql = smem + L::QLO + t * C::TILE_BYTES;
-#pragma unroll
-      for (int u = 0; u < HD / 8; ++u) {
-        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (valid) {
-          load4(qrow + 8 * u, v);
-          load4(qrow + 8 * u + 4, v + 4);
-        }
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-          float2 hf = __bfloat1622float2(h2);
-          __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
-          hi[e] = *reinterpret_cast<uint32_t*>(&h2);
-          lo[e] = *reinterpret_cast<uint32_t*>(&l2);
-        }
-        const uint32_t off = swz_off<HD>(r, u);
-        *reinterpret_cast<uint4*>(qh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(ql + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-      fence_async_smem();
-      mbar_arrive(&q_full[t]);
-    }
-
     const uint32_t tS = tmem + lane_off + s_col(t);
     const uint32_t tO = tmem + lane_off + o_col<HD>(t);
     uint8_t* pb = smem + L::P + t * C::P_BYTES;
-    // visible keys: index < row_lim - 128 j (the causal bound and the user end / cutoff)
-    const int row_lim = DEC ? nkeys : min(q_pos0 + t * ROWS + r + 1, user_len);
-    float m_ref = -INFINITY;  // reference max (scaled, log2 domain) of P and O
-    float l_run = 0.f;        // sum of exponentials relative to m_ref
-    bool ok = true;
-    for (int j = 0; j < nb; ++j) {
-      if (!mbar_wait(&s_full[t], j & 1, err, &abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      float s[KB];
-      {
-        uint32_t raw[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, raw[c]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[c][i]);
-      }
-      const int lim = row_lim - j * KB;
-      if (lim < KB) {
-#pragma unroll
-        for (int c = 0; c < KB; ++c)
-          if (c >= lim) s[c] = -INFINITY;
-      }
-      // row max of the raw scores: 8 chains of three-input maxima
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[i], s[8 + i]);
-#pragma unroll
-      for (int c = 16; c < KB; c += 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
-      const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-      // P_t(j) replaces P_t(j-1): wait until O += P_t(j-1) V has completed
-      if (j >= 1) {
-        if (!mbar_wait(&p_free[t], (j - 1) & 1, err, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
-      }
-      if (j == 0) {
-        m_ref = m_blk;
-      } else if (m_blk > m_ref + RESCALE_LOG2) {  // rescale the O row and l to the new max
-        const float f = exp2_approx(m_ref - m_blk);
-#pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += 32) {
-          float o[32];
-          tmem_ld32(tO + c0, o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= f;
-          tmem_st32(tO + c0, o);
-        }
-        l_run *= f;
-        m_ref = m_blk;
-      }
-      float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m_ref, -m_ref);
-#pragma unroll
-      for (int u = 0; u < KB / 8; ++u) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const float2 x = ffma2(make_float2(s[8 * u + e], s[8 * u + e + 1]), scale2, neg_m2);
-          p[e] = exp2_approx(x.x);
-          p[e + 1] = exp2_approx(x.y);
-          sum2[(e >> 1) & 1] = fadd2(sum2[(e >> 1) & 1], make_float2(p[e], p[e + 1]));
-        }
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 t2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
-          pk[e] = *reinterpret_cast<uint32_t*>(&t2);
-        }
-        const int chunk = u >> 3, uu = u & 7;
-        *reinterpret_cast<uint4*>(pb + chunk * (ROWS * 128) + r * 128 + ((uu ^ (r & 7)) * 16)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-      l_run += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-    }
-    if (ok && nb > 0) {
-      ok = mbar_wait(&p_free[t], (nb - 1) & 1, err, &abort_flag);  // the last P V has completed
-      tc_fence_after();
-    }
     const bool split = DEC && da.n_split > 1;
-    const long long row_g = (long long)(q_row0 + t * ROWS + r);
-    if (nb > 0) {
+    int cb = 0, qn = 0;
+    bool ok = true;
+    for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
+      const AttnItem w = decode_item<DEC>(ea, da, items[k]);
+      const int nb = w.nblk[t];
+      const bool valid = r < w.nrow[t];
+      const long long row_g = (long long)(w.q_row0 + t * ROWS + r);
+      const int h = w.h;
+      if (nb == 0) {
+        if (split && valid) {  // an empty key range: a partial that carries no weight
+          float* po = da.part_o + ((long long)w.split * da.nk_rows + row_g) * d + h * HD;
+          const float z4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < HD; c += 4) store4(po + c, z4);
+          float* pml = da.part_ml + (((long long)w.split * da.nk_rows + row_g) * n_heads + h) * 2;
+          pml[0] = -INFINITY;
+          pml[1] = 0.f;
+        }
+        continue;
+      }
+      if (DEC) {  // stage q (fp32) as hi + lo bf16 tiles in the swizzled K-major layout
+        if (qn >= 1 && !mbar_wait(&q_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
+        const float* qrow = da.q + (long long)(w.q_row0 + t * ROWS + (valid ? r : 0)) * d + h * HD;
+        uint8_t* qh = smem + L::Q + t * C::TILE_BYTES;
+        uint8_t* ql = smem + L::QLO + t * C::TILE_BYTES;
+#pragma unroll
+        for (int u = 0; u < HD / 8; ++u) {
+          float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+          if (valid) {
+            load4(qrow + 8 * u, v);
+            load4(qrow + 8 * u + 4, v + 4);
+          }
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+            float2 hf = __bfloat1622float2(h2);
+            __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+            hi[e] = *reinterpret_cast<uint32_t*>(&h2);
+            lo[e] = *reinterpret_cast<uint32_t*>(&l2);
+          }
+          const uint32_t off = swz_off<HD>(r, u);
+          *reinterpret_cast<uint4*>(qh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(ql + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_async_smem();
+        mbar_arrive(&q_full[t]);
+      }
+      // visible keys: index < row_lim - 128 j (the causal bound and the user end / cutoff)
+      const int row_lim = DEC ? w.nkeys : min(w.q_pos0 + t * ROWS + r + 1, w.user_len);
+      float m_ref = -INFINITY;  // reference max (scaled, log2 domain) of P and O
+      float l_run = 0.f;        // sum of exponentials relative to m_ref
+      for (int j = 0; j < nb; ++j) {
+        const int gj = cb + j;
+        if (!mbar_wait(&s_full[t], gj & 1, err, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        float s[KB];
+        {
+          uint32_t raw[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, raw[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[c][i]);
+        }
+        const int lim = row_lim - j * KB;
+        if (lim < KB) {
+#pragma unroll
+          for (int c = 0; c < KB; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        // row max of the raw scores: 8 chains of three-input maxima
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+        for (int c = 16; c < KB; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
+        const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        // P_t replaces the previous block's: wait until its O += P V has completed
+        if (gj >= 1) {
+          if (!mbar_wait(&p_free[t], (gj - 1) & 1, err, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+        }
+        if (j == 0) {
+          m_ref = m_blk;
+        } else if (m_blk > m_ref + RESCALE_LOG2) {  // rescale the O row and l to the new max
+          const float f = exp2_approx(m_ref - m_blk);
+#pragma unroll
+          for (int c0 = 0; c0 < HD; c0 += 32) {
+            float o[32];
+            tmem_ld32(tO + c0, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= f;
+            tmem_st32(tO + c0, o);
+          }
+          l_run *= f;
+          m_ref = m_blk;
+        }
+        float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m_ref, -m_ref);
+#pragma unroll
+        for (int u = 0; u < KB / 8; ++u) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const float2 x = ffma2(make_float2(s[8 * u + e], s[8 * u + e + 1]), scale2, neg_m2);
+            p[e] = exp2_approx(x.x);
+            p[e + 1] = exp2_approx(x.y);
+            sum2[(e >> 1) & 1] = fadd2(sum2[(e >> 1) & 1], make_float2(p[e], p[e + 1]));
+          }
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
+            pk[e] = *reinterpret_cast<uint32_t*>(&t2);
+          }
+          const int chunk = u >> 3, uu = u & 7;
+          *reinterpret_cast<uint4*>(pb + chunk * (ROWS * 128) + r * 128 + ((uu ^ (r & 7)) * 16)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        l_run += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      if (!mbar_wait(&p_free[t], (cb + nb - 1) & 1, err, &abort_flag)) { ok = false; break; }  // the last P V
+      tc_fence_after();
       // every lane takes part in the (warp-collective) TMEM loads
       float o[HD];
 #pragma unroll
@@ -410,23 +479,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[c0 + e] = v32[e];
       }
-      if (ok && valid && split) {  // partial result of this key range, combined later
-        const int sp = da.tiles[tile].split;
-        float* po = da.part_o + ((long long)sp * da.nk_rows + row_g) * d + h * HD;
+      tc_fence_before();
+      mbar_arrive(&o_empty[t]);  // O_t may now be overwritten by the next item
+      if (valid && split) {  // partial result of this key range, combined later
+        float* po = da.part_o + ((long long)w.split * da.nk_rows + row_g) * d + h * HD;
 #pragma unroll
         for (int c = 0; c < HD; c += 4) store4(po + c, &o[c]);
-        float* pml = da.part_ml + (((long long)sp * da.nk_rows + row_g) * n_heads + h) * 2;
+        float* pml = da.part_ml + (((long long)w.split * da.nk_rows + row_g) * n_heads + h) * 2;
         pml[0] = m_ref;
         pml[1] = l_run;
-      } else if (ok && valid) {
+      } else if (valid) {
         const float inv = 1.0f / l_run;
         const long long ro = row_g * d + h * HD;
         const float* gate = (DEC ? da.g : ea.gate) + ro;
 #pragma unroll
         for (int c = 0; c < HD; c += 4) {
-          float g[4];
-          load4(gate + c, g);
-          float v[4] = {o[c] * inv * g[0], o[c + 1] * inv * g[1], o[c + 2] * inv * g[2], o[c + 3] * inv * g[3]};
+          float gg[4];
+          load4(gate + c, gg);
+          float v[4] = {o[c] * inv * gg[0], o[c + 1] * inv * gg[1], o[c + 2] * inv * gg[2], o[c + 3] * inv * gg[3]};
           if (DEC && da.out_lo) {  // o * g as a hi + lo pair of bf16 values
             float lo[4];
 #pragma unroll
@@ -440,15 +510,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-    } else if (split && valid) {  // an empty key range: a partial that carries no weight
-      const int sp = da.tiles[tile].split;
-      float* po = da.part_o + ((long long)sp * da.nk_rows + row_g) * d + h * HD;
-      const float z4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < HD; c += 4) store4(po + c, z4);
-      float* pml = da.part_ml + (((long long)sp * da.nk_rows + row_g) * n_heads + h) * 2;
-      pml[0] = -INFINITY;
-      pml[1] = 0.f;
+      cb += nb;
+      ++qn;
     }
   }
   tc_fence_before();
@@ -465,7 +528,6 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
   const int swz = HD == 64 ? 128 : 64;
   CUtensorMap mq, mk, mv;
   const int n_tiles = DEC ? da->n_tiles : ea->n_tiles;
-  const int n_heads = DEC ? da->n_heads : ea->n_heads;
   const int d = DEC ? da->d : ea->d;
   if (n_tiles == 0) return cudaSuccess;
   const long long rows = DEC ? da->key_rows : ea->rows;
@@ -491,7 +553,9 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
   }
   EncAttnArgs e0 = ea ? *ea : EncAttnArgs{};
   DecAttnArgs d0 = da ? *da : DecAttnArgs{};
-  attn_tc_kernel<HD, MODE><<<n_tiles * n_heads, NTHREADS, smem, s>>>(mq, mk, mv, e0, d0, err);
+  const int n_cta = DEC ? da->n_cta : ea->n_cta;
+  if (n_cta <= 0) return cudaErrorInvalidValue;
+  attn_tc_kernel<HD, MODE><<<n_cta, NTHREADS, smem, s>>>(mq, mk, mv, e0, d0, err);
   return cudaGetLastError();
 }
 
