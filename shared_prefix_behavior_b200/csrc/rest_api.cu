@@ -112,6 +112,12 @@ static void build_enc_tiles(const rest_batch* b, int rows, std::vector<EncTile>&
 }
 
 constexpr int KEY_BLOCK = 128;   // keys per block of the attention kernels
+// In rank_request the decoder reads H_lo (H = H_hi + H_lo) only for requests
+// with fewer keys than this: H's bf16 rounding reaches y through per-key
+// perturbations that the attention average shrinks about as 1/sqrt(keys), so
+// long prefixes do not need the extra MMA passes, while a cutoff of 1 key
+// passes H's rounding straight into y.
+constexpr int HLO_MAX_CUTOFF = 1024;
 constexpr int TARGET_CTAS = 296;  // two waves of the B200's 148 SMs
 
 // Decoder work items. With n_split > 1 every (request, row chunk) is split
@@ -129,10 +135,14 @@ static void build_dec_tiles(const rest_batch* b, const rest_requests* r, int K, 
     for (long long p = rows0; p < rows1; p += rows)
       for (int sp = 0; sp < n_split; ++sp)
         t.push_back(DecTile{(int)p, (int)std::min<long long>(rows, rows1 - p), key0, c,
-                            (int)((long long)nb * sp / n_split), (int)((long long)nb * (sp + 1) / n_split), sp, 0});
+                            (int)((long long)nb * sp / n_split), (int)((long long)nb * (sp + 1) / n_split), sp,
+                            c < HLO_MAX_CUTOFF ? 1 : 0});
   }
-  std::stable_sort(t.begin(), t.end(),
-                   [](const DecTile& a, const DecTile& c) { return a.kb1 - a.kb0 > c.kb1 - c.kb0; });
+  // the tiles that read H_lo first (they run as a launch of their own), each group longest first
+  std::stable_sort(t.begin(), t.end(), [](const DecTile& a, const DecTile& c) {
+    if (a.pad != c.pad) return a.pad > c.pad;
+    return a.kb1 - a.kb0 > c.kb1 - c.kb0;
+  });
 }
 
 // Longest-processing-time assignment of attention work items to the
@@ -192,7 +202,7 @@ static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_he
 // ---------------------------------------------------------------- workspace
 
 struct Layout {
-  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, meta_end;
+  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
   size_t dq, dg, dout, hlo, part_o, part_ml;
   size_t total;
@@ -201,7 +211,7 @@ struct Layout {
 
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
                           int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split,
-                          size_t n_enc_sched, size_t n_dec_sched) {
+                          size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -214,6 +224,7 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dec_tiles = take(sizeof(DecTile) * (size_t)n_dec_tiles);
   L.enc_sched = take(sizeof(int) * n_enc_sched);
   L.dec_sched = take(sizeof(int) * n_dec_sched);
+  L.dec_sched2 = take(sizeof(int) * n_dec_sched2);
   L.meta_end = off;
   L.cos_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
   L.sin_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
@@ -243,7 +254,8 @@ struct Plan {
   int max_dff, K;
   std::vector<EncTile> enc_tiles;
   std::vector<DecTile> dec_tiles;
-  std::vector<int> enc_sched, dec_sched;  // tensor-core attention: per-CTA item lists
+  std::vector<int> enc_sched, dec_sched, dec_sched2;  // tensor-core attention: per-CTA item lists
+  int n_dec_hlo;  // leading decoder tiles that read H_lo (rank_request, bf16)
   Layout L;
   int32_t* err;
   bool hsplit;
@@ -262,7 +274,7 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
     if ((st = check_requests(reqs, b, &p.n_cands)) != REST_OK) return st;
     if (K < 1 || K > 8) return REST_ERR_INVALID_ARG;
   }
-  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false; p.n_split = 1;
+  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false; p.n_split = 1; p.n_dec_hlo = 0;
   p.NK = p.n_cands * (reqs ? K : 0);
   if (p.T * (long long)hs->d >= (1LL << 40) || p.NK >= (1LL << 31)) return REST_ERR_UNSUPPORTED;
   const int tile_rows = attn_tile_rows(dt, hs->head_dim);
@@ -281,13 +293,28 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   }
   build_dec_tiles(b, reqs, K, tile_rows, p.n_split, p.dec_tiles);
   // encoder followed by the decoder in bf16: the decoder reads H as hi + lo
-  p.hsplit = encoder_runs && reqs != nullptr && dt == REST_BF16;
+  p.n_dec_hlo = 0;
+  if (encoder_runs && reqs != nullptr && dt == REST_BF16)
+    for (const DecTile& t : p.dec_tiles) p.n_dec_hlo += t.pad;
+  p.hsplit = p.n_dec_hlo > 0;
+  if (!p.hsplit)
+    for (DecTile& t : p.dec_tiles) t.pad = 0;
   if (tile_rows != 128) {  // the tensor-core attention runs: schedule its persistent CTAs
     if (!p.enc_tiles.empty()) p.enc_sched = enc_schedule(b, p.enc_tiles, hs->n_heads, tile_rows);
-    if (!p.dec_tiles.empty()) p.dec_sched = dec_schedule(p.dec_tiles, hs->n_heads);
+    if (!p.dec_tiles.empty()) {  // [tiles that read H_lo | the others], scheduled separately
+      std::vector<DecTile> a(p.dec_tiles.begin(), p.dec_tiles.begin() + p.n_dec_hlo);
+      std::vector<DecTile> c(p.dec_tiles.begin() + p.n_dec_hlo, p.dec_tiles.end());
+      if (a.empty()) {
+        p.dec_sched = dec_schedule(c, hs->n_heads);
+      } else {
+        p.dec_sched = dec_schedule(a, hs->n_heads);
+        if (!c.empty()) p.dec_sched2 = dec_schedule(c, hs->n_heads);
+      }
+    }
   }
   p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),
-                    (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size());
+                    (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size(),
+                    p.dec_sched2.size());
   return REST_OK;
 }
 
@@ -373,6 +400,8 @@ static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
     memcpy(host.data() + p.L.enc_sched, p.enc_sched.data(), sizeof(int) * p.enc_sched.size());
   if (!p.dec_sched.empty())
     memcpy(host.data() + p.L.dec_sched, p.dec_sched.data(), sizeof(int) * p.dec_sched.size());
+  if (!p.dec_sched2.empty())
+    memcpy(host.data() + p.L.dec_sched2, p.dec_sched2.data(), sizeof(int) * p.dec_sched2.size());
   if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) return REST_ERR_CUDA;
   return REST_OK;
 }
@@ -559,8 +588,7 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   da.q = dq; da.g = dg; da.h = h; da.h_lo = h_lo; da.out = dout;
   da.out_lo = tc ? (void*)((bf16*)dout + (size_t)p.NK * d) : nullptr;
   da.tiles = at<DecTile>(ws, L.dec_tiles); da.n_tiles = L.n_dec_tiles;
-  da.sched = at<int>(ws, L.dec_sched);
-  da.n_cta = p.dec_sched.empty() ? 0 : std::min((int)p.dec_tiles.size() * p.hs->n_heads, SCHED_CTAS);
+
   da.n_heads = p.hs->n_heads; da.d = d;
   da.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
   da.key_rows = p.T;
@@ -569,7 +597,28 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   da.part_o = at<float>(ws, L.part_o);
   da.part_ml = at<float>(ws, L.part_ml);
   if (bf && sm100_attn_supported(hd)) {
-    REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_sm100(hd, da, s, err));
+    // tiles that read H_lo (short cutoffs, within rank_request) and the others
+    const int n_hlo = h_lo ? p.n_dec_hlo : 0;
+    const int n_rest = L.n_dec_tiles - n_hlo;
+    const int H = p.hs->n_heads;
+    if (n_hlo > 0) {
+      DecAttnArgs a1 = da;
+      a1.n_tiles = n_hlo;
+      a1.sched = at<int>(ws, L.dec_sched);
+      a1.n_cta = std::min(n_hlo * H, SCHED_CTAS);
+      REST_KLAUNCH(s, "dec_attn", flops * n_hlo / L.n_dec_tiles, bytes * n_hlo / L.n_dec_tiles,
+                   launch_dec_attn_sm100(hd, a1, s, err));
+    }
+    if (n_rest > 0) {
+      DecAttnArgs a2 = da;
+      a2.h_lo = nullptr;
+      a2.tiles = da.tiles + n_hlo;
+      a2.n_tiles = n_rest;
+      a2.sched = at<int>(ws, n_hlo > 0 ? L.dec_sched2 : L.dec_sched);
+      a2.n_cta = std::min(n_rest * H, SCHED_CTAS);
+      REST_KLAUNCH(s, "dec_attn", flops * n_rest / L.n_dec_tiles, bytes * n_rest / L.n_dec_tiles,
+                   launch_dec_attn_sm100(hd, a2, s, err));
+    }
     if (p.n_split > 1)
       REST_KLAUNCH(s, "dec_combine", 0, (double)p.NK * d * 4 * (p.n_split + 2),
                    launch_dec_combine(hd, da, s));
