@@ -76,10 +76,39 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// Make generic-proxy shared-memory writes visible to the async proxy (MMA reads).
+// Make generic-proxy shared-memory writes visible to the async proxy (MMA
+// reads, TMA stores).
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// TMA tile store shared -> global (rows past the tensor's extent are not
+// written), and the same with an fp32 add into the global values.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed store groups are still
+// reading their shared-memory source (.read), or still in flight at all.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// Byte offset of 16-byte chunk k of row r in a TMA box whose rows are 128
+// bytes (128B swizzle) or 64 bytes (64B swizzle); the box must start on a
+// 1024-byte (resp. 512-byte) boundary of shared memory.
+__device__ __forceinline__ uint32_t sw128_off(int r, int k) { return r * 128 + ((k ^ (r & 7)) << 4); }
+__device__ __forceinline__ uint32_t sw64_off(int r, int k) { return r * 64 + ((k ^ ((r >> 1) & 3)) << 4); }
 
 // ------------------------------------------------------------------ TMEM
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

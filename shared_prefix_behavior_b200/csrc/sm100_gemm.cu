@@ -1,19 +1,27 @@
 // tcgen05 GEMM for sm_100a with the fused epilogues of the ReST encoder and
 // decoder (bf16 operands, fp32 accumulation in TMEM).
 //
-// One CTA computes a 128 x BN tile of C = A . B:
-//   warp 0       TMA producer: A box [128 rows x 64 K] (K-major, 128B swizzle)
-//                and BN/64 boxes of B [64 K rows x 64 N] (N-major, 128B swizzle)
-//                per stage, into a STAGES-deep ring;
-//   warp 1       allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
-//                K=16) over the ring and commits each stage back to the producer;
-//   warps 2..5   epilogue: tcgen05.ld of the accumulator rows (warp w owns TMEM
-//                lanes 32*(w%4)..), the fused epilogue, and the global stores.
+// A persistent CTA per SM walks 128 x 128 tiles of C = A . B:
+//   warp 0       TMA producer: per stage an A box [128 rows x 64 K] (K-major,
+//                128B swizzle) and two 64-column boxes of B [64 K x 64 N]
+//                (N-major, 128B swizzle); for the DGA projection also the
+//                tile's rows of the rotation table (cos, sin) into a side
+//                slot, one tile ahead of the epilogue that uses them;
+//   warp 1       allocates TMEM (two accumulators); one thread issues
+//                tcgen05.mma (M=128, N=128, K=16) and commits each stage back;
+//   warps 2..9   epilogue, two warps per TMEM lane quarter (each takes half of
+//                the columns): tcgen05.ld of its rows, the fused epilogue, the
+//                result written into a swizzled shared-memory box and sent to
+//                global memory by a TMA store; the residual sublayers add into
+//                the fp32 residual stream with a TMA reduce-add, so the
+//                residual is never loaded by the SM.
 // B is read directly from the weight as stored ([K, N] row-major, x . W
 // layout), so no transposed copy of any weight is made. The column blocks an
 // epilogue must pair (V with its gate Gv; W_1 with W_3) are brought into the
 // same tile by choosing which 64-column box of B each slot of the tile loads.
 #include <cudaTypedefs.h>
+
+#include <cstring>
 
 #include "kernels.h"
 #include "sm100.h"
@@ -25,46 +33,35 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128;
+constexpr int BN = 128;
 constexpr int BK = 64;
 constexpr int NUM_THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
-constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int EPI_WARPS = 8;
+constexpr int A_BYTES = BM * BK * 2;      // 16 KB
 constexpr int BOX_B_BYTES = 64 * BK * 2;  // one 64-column box of B: 8 KB
+constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+constexpr int BOX128 = BM * 128;  // a [128 rows x 128 bytes] staging box: 16 KB
 
-// Global column of B loaded into box b of N-tile t.
-__device__ __forceinline__ int b_box_col(const GemmArgs& a, int BN, int t, int b) {
-  const int nbh = BN / 128;  // boxes per half tile (paired epilogues)
-  const int half = BN / 2;
+// The tensor maps of one launch: operands, side inputs (rotation table) and
+// up to four outputs.
+struct GemmMaps {
+  CUtensorMap a, a2, b, b2;
+  CUtensorMap s0, s1;  // EPI_QKVG: cos, sin [M, d/2] fp32, boxes of 32 columns x 128 rows
+  CUtensorMap o[4];    // outputs, boxes of 32 rows (see setup_maps)
+};
+
+// Global column of B loaded into box b (0 or 1) of N-tile t.
+__device__ __forceinline__ int b_box_col(const GemmArgs& a, int t, int b) {
   if (a.epi == EPI_QKVG) {
-    const int d = a.d, nQ = d / BN, nV = d / half;
+    const int d = a.d, nQ = d / BN, nV = d / (BN / 2);
     if (t < 2 * nQ) return t * BN + 64 * b;
-    if (t < 2 * nQ + nV) {
-      int u = t - 2 * nQ;
-      return b < nbh ? 2 * d + u * half + 64 * b : 3 * d + u * half + 64 * (b - nbh);
-    }
+    if (t < 2 * nQ + nV) return (b == 0 ? 2 * d : 3 * d) + (t - 2 * nQ) * 64;  // V and its gate Gv
     return 4 * d + (t - 2 * nQ - nV) * BN + 64 * b;
   }
-  if (a.epi == EPI_SWIGLU) return b < nbh ? t * half + 64 * b : a.d + t * half + 64 * (b - nbh);
+  if (a.epi == EPI_SWIGLU) return (b == 0 ? 0 : a.d) + t * 64;  // W_1 and W_3
   return t * BN + 64 * b;
 }
 
-__device__ __forceinline__ void store32(float* p, const float (&v)[32]) {
-#pragma unroll
-  for (int i = 0; i < 32; i += 4) store4(p + i, &v[i]);
-}
-// 32 bf16 values as four 16-byte stores
-__device__ __forceinline__ void store32(bf16* p, const float (&v)[32]) {
-#pragma unroll
-  for (int i = 0; i < 32; i += 8) {
-    uint4 u;
-    __nv_bfloat162 t0 = __floats2bfloat162_rn(v[i], v[i + 1]), t1 = __floats2bfloat162_rn(v[i + 2], v[i + 3]);
-    __nv_bfloat162 t2 = __floats2bfloat162_rn(v[i + 4], v[i + 5]), t3 = __floats2bfloat162_rn(v[i + 6], v[i + 7]);
-    u.x = *reinterpret_cast<uint32_t*>(&t0);
-    u.y = *reinterpret_cast<uint32_t*>(&t1);
-    u.z = *reinterpret_cast<uint32_t*>(&t2);
-    u.w = *reinterpret_cast<uint32_t*>(&t3);
-    *reinterpret_cast<uint4*>(p + i) = u;
-  }
-}
 // sigmoid from the hardware base-2 exponential and reciprocal (relative
 // error about 3e-7; every consumer of these gates rounds to bf16 or feeds a
 // bf16 product)
@@ -75,166 +72,220 @@ __device__ __forceinline__ float sigmoid_fast(float x) {
   return r;
 }
 
-// Every lane executes the (warp-collective) TMEM loads; only rows < M touch
-// global memory.
-// The epilogue of one 128 x BN tile, split between two warps per TMEM lane
-// quarter (part 0: the first half of the columns, part 1: the second half;
-// for the paired epilogues, of each half). Inputs that do not depend on the
-// accumulator (the residual row, the rotation table) are loaded by
-// epi_prefetch before the accumulator is waited for, so their latency hides
-// behind the tile's MMAs. Every lane executes the (warp-collective) TMEM
-// loads; only rows < M touch global memory.
-template <int BN>
-struct EpiIn {
-  float v[BN / 2];
-};
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
 
-template <int BN>
-__device__ __forceinline__ void epi_prefetch(const GemmArgs& a, int m, int t, bool valid, int part, EpiIn<BN>& in) {
-  if (!valid) return;
-  const long long ro = (long long)m * a.ldo;
-  if (a.epi == EPI_RESID) {
-    const float* p = (const float*)a.out0 + ro + t * BN + part * (BN / 2);
+// 32 fp32 values: one 128-byte row (row r) of a 128B-swizzled box
+__device__ __forceinline__ void stage_f32(uint8_t* box, int r, const float (&v)[32]) {
 #pragma unroll
-    for (int j = 0; j < BN / 2; j += 4) load4(p + j, &in.v[j]);
-  } else if (a.epi == EPI_QKVG) {
-    const int d = a.d, nQ = d / BN;
-    if (t < 2 * nQ) {  // cos and sin of the BN/4 column pairs of this part
-      const int col0 = (t < nQ ? t : t - nQ) * BN + part * (BN / 2);
-      const float* ct = a.cos_t + (long long)m * (d / 2) + col0 / 2;
-      const float* st = a.sin_t + (long long)m * (d / 2) + col0 / 2;
+  for (int k = 0; k < 8; ++k)
+    *reinterpret_cast<float4*>(box + sw128_off(r, k)) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+// 32 values as bf16: one 64-byte row (row r) of a 64B-swizzled box
+__device__ __forceinline__ void stage_bf16_sw64(uint8_t* box, int r, const float (&v)[32]) {
 #pragma unroll
-      for (int j = 0; j < BN / 4; j += 4) {
-        load4(ct + j, &in.v[j]);
-        load4(st + j, &in.v[BN / 4 + j]);
-      }
-    }
+  for (int k = 0; k < 4; ++k) {
+    uint4 u;
+    u.x = pack_bf16(v[8 * k], v[8 * k + 1]);
+    u.y = pack_bf16(v[8 * k + 2], v[8 * k + 3]);
+    u.z = pack_bf16(v[8 * k + 4], v[8 * k + 5]);
+    u.w = pack_bf16(v[8 * k + 6], v[8 * k + 7]);
+    *reinterpret_cast<uint4*>(box + sw64_off(r, k)) = u;
+  }
+}
+// 32 values as bf16 into half (chunks k0..k0+3) of a 128-byte row of a 128B-swizzled box
+__device__ __forceinline__ void stage_bf16_sw128(uint8_t* box, int r, int k0, const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint4 u;
+    u.x = pack_bf16(v[8 * k], v[8 * k + 1]);
+    u.y = pack_bf16(v[8 * k + 2], v[8 * k + 3]);
+    u.z = pack_bf16(v[8 * k + 4], v[8 * k + 5]);
+    u.w = pack_bf16(v[8 * k + 6], v[8 * k + 7]);
+    *reinterpret_cast<uint4*>(box + sw128_off(r, k0 + k)) = u;
   }
 }
 
-template <int BN>
-__device__ __forceinline__ void epilogue(const GemmArgs& a, uint32_t tmem_row, int m, int t, bool valid, int part,
-                                         const EpiIn<BN>& in) {
+// The epilogue of one tile for one epilogue warp: rows r = 32 q + lane of the
+// tile, accumulator columns [64 part, 64 part + 64). The result is written
+// into the tile's shared-memory slot as 32-row TMA boxes and lane 0 issues
+// their stores. With SIDE (the DGA projection) the slot already holds this
+// tile's rotation table rows and is known to be free; otherwise the warp
+// first waits until its own stores of the previous tile have left the slot.
+template <bool SIDE>
+__device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, uint32_t trow, uint8_t* slot, int t,
+                                         int mt, int q, int lane, int part) {
+  const int r = q * 32 + lane;
+  const int y0 = mt * BM + q * 32;
   float v[32];
-  const long long ro = (long long)m * a.ldo;
-  const int half = BN / 2;
+  auto slot_ready = [&]() {
+    if (!SIDE) {
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+    }
+  };
+  auto issue = [&]() {
+    fence_async_smem();
+    __syncwarp();
+  };
   if (a.epi == EPI_QKVG) {
-    const int d = a.d, nQ = d / BN, nV = d / half;
-    if (t < 2 * nQ) {  // Q or K: rotate the pairs (ReST eq. 5)
+    const int d = a.d, nQ = d / BN, nV = d / (BN / 2);
+    if (t < 2 * nQ) {  // Q or K: rotate the pairs (ReST eq. 5) with the staged cos / sin rows
       const bool isq = t < nQ;
-      const int col0 = (isq ? t : t - nQ) * BN + part * half;
-      bf16* out = (bf16*)(isq ? a.out0 : a.out1) + ro + col0;
+      uint8_t* cb = slot + part * BOX128;             // cos of pairs [32 part, 32 part + 32)
+      const uint8_t* sb = slot + (2 + part) * BOX128;  // sin of the same pairs
 #pragma unroll
-      for (int c0 = 0; c0 < half; c0 += 32) {
-        tmem_ld32(tmem_row + part * half + c0, v);
-        if (!valid) continue;
-        float w[32];
+      for (int j = 0; j < 2; ++j) {
+        tmem_ld32(trow + part * 64 + 32 * j, v);
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const float c = in.v[c0 / 2 + jj], sn = in.v[BN / 4 + c0 / 2 + jj];
-          w[2 * jj] = v[2 * jj] * c - v[2 * jj + 1] * sn;
-          w[2 * jj + 1] = v[2 * jj] * sn + v[2 * jj + 1] * c;
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t off = sw128_off(r, 4 * j + kk);
+          const float4 c = *reinterpret_cast<const float4*>(cb + off);
+          const float4 s = *reinterpret_cast<const float4*>(sb + off);
+          const float* p = v + 8 * kk;
+          uint4 u;
+          u.x = pack_bf16(p[0] * c.x - p[1] * s.x, p[0] * s.x + p[1] * c.x);
+          u.y = pack_bf16(p[2] * c.y - p[3] * s.y, p[2] * s.y + p[3] * c.y);
+          u.z = pack_bf16(p[4] * c.z - p[5] * s.z, p[4] * s.z + p[5] * c.z);
+          u.w = pack_bf16(p[6] * c.w - p[7] * s.w, p[6] * s.w + p[7] * c.w);
+          // the 8 outputs of these 4 pairs take the bytes of their cos values
+          *reinterpret_cast<uint4*>(cb + off) = u;
         }
-        store32(out + c0, w);
+      }
+      issue();
+      if (lane == 0) {
+        tma_store_2d(&mp.o[isq ? 0 : 1], cb + q * 32 * 128, (isq ? t : t - nQ) * BN + 64 * part, y0);
+        bulk_commit();
       }
       return;
     }
-    if (t < 2 * nQ + nV) {  // value gate: V' = sigmoid(Gv) * V (eq. 3)
-      const int col0 = (t - 2 * nQ) * half + part * (half / 2);
-      bf16* out = (bf16*)a.out2 + ro + col0;
+    if (t < 2 * nQ + nV) {  // value gate: V' = sigmoid(Gv) * V (eq. 3), 64 output columns
+      uint8_t* box = slot + part * (BM * 64);
+      float g[32];
+      tmem_ld32(trow + 32 * part, v);
+      tmem_ld32(trow + 64 + 32 * part, g);
 #pragma unroll
-      for (int c0 = 0; c0 < half / 2; c0 += 32) {
-        float g[32];
-        tmem_ld32(tmem_row + part * (half / 2) + c0, v);
-        tmem_ld32(tmem_row + half + part * (half / 2) + c0, g);
-        if (!valid) continue;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= sigmoid_fast(g[j]);
-        store32(out + c0, v);
+      for (int j = 0; j < 32; ++j) v[j] *= sigmoid_fast(g[j]);
+      slot_ready();
+      stage_bf16_sw64(box, r, v);
+      issue();
+      if (lane == 0) {
+        tma_store_2d(&mp.o[2], box + q * 32 * 64, (t - 2 * nQ) * 64 + 32 * part, y0);
+        bulk_commit();
       }
       return;
     }
     // output gate sigmoid(Go) (eq. 4), fp32
-    float* out = (float*)a.out3 + ro + (t - 2 * nQ - nV) * BN + part * half;
 #pragma unroll
-    for (int c0 = 0; c0 < half; c0 += 32) {
-      tmem_ld32(tmem_row + part * half + c0, v);
-      if (!valid) continue;
+    for (int j = 0; j < 2; ++j) {
+      tmem_ld32(trow + part * 64 + 32 * j, v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
-      store32(out + c0, v);
+      for (int i = 0; i < 32; ++i) v[i] = sigmoid_fast(v[i]);
+      if (j == 0) slot_ready();
+      stage_f32(slot + (2 * part + j) * BOX128, r, v);
+    }
+    issue();
+    if (lane == 0) {
+      const int x0 = (t - 2 * nQ - nV) * BN;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int c = 2 * part + j;
+        tma_store_2d(&mp.o[3], slot + c * BOX128 + q * 32 * 128, x0 + 32 * c, y0);
+      }
+      bulk_commit();
     }
     return;
   }
-  if (a.epi == EPI_SWIGLU) {  // SiLU(x W_1) * (x W_3)
-    bf16* out = (bf16*)a.out0 + ro + t * half + part * (half / 2);
+  if (a.epi == EPI_SWIGLU) {  // SiLU(x W_1) * (x W_3), 64 output columns
+    uint8_t* box = slot + part * (BM * 64);
+    float u[32];
+    tmem_ld32(trow + 32 * part, v);
+    tmem_ld32(trow + 64 + 32 * part, u);
 #pragma unroll
-    for (int c0 = 0; c0 < half / 2; c0 += 32) {
-      float u[32];
-      tmem_ld32(tmem_row + part * (half / 2) + c0, v);
-      tmem_ld32(tmem_row + half + part * (half / 2) + c0, u);
-      if (!valid) continue;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = v[j] * sigmoid_fast(v[j]) * u[j];
-      store32(out + c0, v);
+    for (int j = 0; j < 32; ++j) v[j] = v[j] * sigmoid_fast(v[j]) * u[j];
+    slot_ready();
+    stage_bf16_sw64(box, r, v);
+    issue();
+    if (lane == 0) {
+      tma_store_2d(&mp.o[0], box + q * 32 * 64, t * 64 + 32 * part, y0);
+      bulk_commit();
     }
     return;
   }
-  if (a.epi == EPI_DECQG) {  // q (fp32) or the sigmoid gate (fp32) of token k
+  if (a.epi == EPI_DT) {  // bf16 copy of the accumulator
+    uint8_t* box = slot + part * BOX128;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      tmem_ld32(trow + part * 64 + 32 * j, v);
+      if (j == 0) slot_ready();
+      stage_bf16_sw128(box, r, 4 * j, v);
+    }
+    issue();
+    if (lane == 0) {
+      tma_store_2d(&mp.o[0], box + q * 32 * 128, t * BN + 64 * part, y0);
+      bulk_commit();
+    }
+    return;
+  }
+  // fp32 outputs: plain, sigmoid, the decoder's q / gate, or the residual add
+  const CUtensorMap* om = &mp.o[0];
+  int x0 = t * BN;
+  bool sig = a.epi == EPI_SIGMOID;
+  if (a.epi == EPI_DECQG) {  // tile t: group g (q of token k = g, or the gate of token k = g - k_tok), N-tile nt
     const int per = a.N / BN, g = t / per, nt = t % per, k = g % a.k_tok;
-    float* out = (float*)(g < a.k_tok ? a.out0 : a.out1) + ro + (long long)k * a.N + nt * BN + part * half;
-#pragma unroll
-    for (int c0 = 0; c0 < half; c0 += 32) {
-      tmem_ld32(tmem_row + part * half + c0, v);
-      if (!valid) continue;
-      if (g >= a.k_tok) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
-      }
-      store32(out + c0, v);
-    }
-    return;
+    om = g < a.k_tok ? &mp.o[0] : &mp.o[1];
+    x0 = k * a.N + nt * BN;
+    sig = g >= a.k_tok;
   }
-  const int n0 = t * BN + part * half;
+  const bool resid = a.epi == EPI_RESID;
 #pragma unroll
-  for (int c0 = 0; c0 < half; c0 += 32) {
-    tmem_ld32(tmem_row + part * half + c0, v);
-    if (!valid) continue;
-    switch (a.epi) {
-      case EPI_F32: store32((float*)a.out0 + ro + n0 + c0, v); break;
-      case EPI_DT: store32((bf16*)a.out0 + ro + n0 + c0, v); break;
-      case EPI_SIGMOID: {
+  for (int j = 0; j < 2; ++j) {
+    tmem_ld32(trow + part * 64 + 32 * j, v);
+    if (resid) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
-        store32((float*)a.out0 + ro + n0 + c0, v);
-        break;
-      }
-      case EPI_RESID: {
+      for (int i = 0; i < 32; ++i) v[i] *= a.alpha;
+    } else if (sig) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = fmaf(a.alpha, v[j], in.v[c0 + j]);
-        store32((float*)a.out0 + ro + n0 + c0, v);
-        break;
-      }
+      for (int i = 0; i < 32; ++i) v[i] = sigmoid_fast(v[i]);
     }
+    if (j == 0) slot_ready();
+    stage_f32(slot + (2 * part + j) * BOX128, r, v);
+  }
+  issue();
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int c = 2 * part + j;
+      const uint8_t* src = slot + c * BOX128 + q * 32 * 128;
+      // x_res += alpha * acc: the add happens at the residual's home in memory
+      if (resid) tma_reduce_add_2d(om, src, x0 + 32 * c, y0);
+      else tma_store_2d(om, src, x0 + 32 * c, y0);
+    }
+    bulk_commit();
   }
 }
 
 // Persistent kernel: one CTA per SM walks the tiles t = blockIdx.x, +gridDim.x,
 // ... (N-tiles of one 128-row block adjacent, so concurrent CTAs share A and
 // B in L2). The accumulator is double-buffered in TMEM: the epilogue of tile
-// i runs while the MMAs of tile i+1 proceed.
-template <int BN, int STAGES>
+// i runs while the MMAs of tile i+1 proceed. NSLOT shared-memory slots of
+// SLOT bytes hold the epilogue's side inputs and staged outputs; with SIDE the
+// producer fills slot i % 2 for tile i once every epilogue warp has released
+// it (after the stores of tile i - 2 have read it out).
+template <int STAGES, int NSLOT, int SLOT, bool SIDE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
-                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2, const GemmArgs a,
-                   int num_kb, int n_tiles_n, int n_tiles, int32_t* err) {
+    gemm_tc_kernel(const __grid_constant__ GemmMaps mp, const GemmArgs a, int num_kb, int n_tiles_n, int n_tiles,
+                   int32_t* err) {
+  static_assert(!SIDE || NSLOT == 2, "side inputs are double-buffered");
   // with a low part A2, the K loop runs twice: A . B, then A2 . B
   const int nkb = a.A2 ? 2 * num_kb : num_kb;
-  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
-  constexpr int EPI_THREADS = NUM_THREADS - 64;
+  constexpr int EPI_THREADS = EPI_WARPS * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain;
+  uint8_t* slots = smem + STAGES * STAGE_BYTES;
+  __shared__ uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], side_full[2], side_empty[2], drain;
   __shared__ uint32_t tslot;
   __shared__ volatile int abort_flag;
 
@@ -248,6 +299,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_THREADS);
+      mbar_init(&side_full[b], 1);
+      mbar_init(&side_empty[b], EPI_WARPS);
     }
     mbar_init(&drain, 1);
     abort_flag = 0;
@@ -261,12 +314,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA producer
-    prefetch_tmap(&tmA);
-    if (a.A2) prefetch_tmap(&tmA2);
-    prefetch_tmap(&tmB);
-    if (a.B2) prefetch_tmap(&tmB2);
-    int it = 0, issued = 0;
-    for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x) {
+    prefetch_tmap(&mp.a);
+    if (a.A2) prefetch_tmap(&mp.a2);
+    prefetch_tmap(&mp.b);
+    if (a.B2) prefetch_tmap(&mp.b2);
+    if (SIDE) {
+      prefetch_tmap(&mp.s0);
+      prefetch_tmap(&mp.s1);
+    }
+    int it = 0, issued = 0, i = 0, side_issued = 0;
+    for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x, ++i) {
       const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % STAGES;
@@ -275,26 +332,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint8_t* st = smem + s * STAGE_BYTES;
         mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
         if (a.epi == EPI_DECQG) {
-          // tile t: group g (q of token k = g, or the gate of token k = g - k_tok), N-tile nt
           const int per = a.N / BN, g = t / per, nt = t % per, k = g % a.k_tok;
-          tma_load_2d(st, &tmA, k * a.K + kk * BK, mt * BM, &full[s]);
+          tma_load_2d(st, &mp.a, k * a.K + kk * BK, mt * BM, &full[s]);
 #pragma unroll
-          for (int b = 0; b < BN / 64; ++b)
-            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, g < a.k_tok ? &tmB : &tmB2, nt * BN + 64 * b,
+          for (int b = 0; b < 2; ++b)
+            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, g < a.k_tok ? &mp.b : &mp.b2, nt * BN + 64 * b,
                         k * a.K + kk * BK, &full[s]);
         } else {
-          tma_load_2d(st, kb < num_kb ? &tmA : &tmA2, kk * BK, mt * BM, &full[s]);
+          tma_load_2d(st, kb < num_kb ? &mp.a : &mp.a2, kk * BK, mt * BM, &full[s]);
 #pragma unroll
-          for (int b = 0; b < BN / 64; ++b)
-            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &tmB, b_box_col(a, BN, t, b), kk * BK, &full[s]);
+          for (int b = 0; b < 2; ++b)
+            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &mp.b, b_box_col(a, t, b), kk * BK, &full[s]);
         }
         issued = it + 1;
+      }
+      if (SIDE && !abort_flag) {
+        // the rotation table rows of a Q or K tile; other tiles only pass the slot on
+        const int s = i & 1;
+        if (!mbar_wait(&side_empty[s], ((i >> 1) & 1) ^ 1, err, &abort_flag)) break;
+        const int nQ = a.d / BN;
+        if (t < 2 * nQ) {
+          const int pair0 = (t < nQ ? t : t - nQ) * (BN / 2);
+          uint8_t* sl = slots + s * SLOT;
+          mbar_arrive_expect_tx(&side_full[s], 4 * BOX128);
+#pragma unroll
+          for (int p = 0; p < 2; ++p) {
+            tma_load_2d(sl + p * BOX128, &mp.s0, pair0 + 32 * p, mt * BM, &side_full[s]);
+            tma_load_2d(sl + (2 + p) * BOX128, &mp.s1, pair0 + 32 * p, mt * BM, &side_full[s]);
+          }
+          side_issued = i + 1;
+        } else {
+          mbar_arrive(&side_full[s]);
+        }
       }
     }
     if (abort_flag) {  // let the copies already in flight land before the CTA exits
       volatile int no_abort = 0;
-      for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr, &no_abort);
+      for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+        mbar_wait(&full[j % STAGES], (j / STAGES) & 1, nullptr, &no_abort);
+      for (int j = (side_issued > 2 ? side_issued - 2 : 0); SIDE && j < side_issued; ++j)
+        mbar_wait(&side_full[j & 1], (j >> 1) & 1, nullptr, &no_abort);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ MMA issuer
@@ -337,15 +414,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
       const int b = i & 1;
       const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
-      const int m = mt * BM + q * 32 + lane;
-      EpiIn<BN> in;
-      epi_prefetch<BN>(a, m, t, m < a.M, part, in);
+      if (SIDE) {
+        // release the previous tile's slot once this warp's stores have read it out
+        if (i > 0 && lane == 0) {
+          bulk_wait_read<0>();
+          mbar_arrive(&side_empty[(i - 1) & 1]);
+        }
+        if (!mbar_wait(&side_full[i & 1], (i >> 1) & 1, err, &abort_flag)) break;
+      }
       if (!mbar_wait(&acc_full[b], (i >> 1) & 1, err, &abort_flag)) break;
       tc_fence_after();
-      epilogue<BN>(a, tmem + b * BN + lane_off, m, t, m < a.M, part, in);
+      epilogue<SIDE>(a, mp, tmem + b * BN + lane_off, slots + (i % NSLOT) * SLOT, t, mt, q, lane, part);
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
     }
+    if (lane == 0) bulk_wait<0>();  // every store has completed before the CTA's shared memory goes away
   }
   tc_fence_before();
   __syncthreads();
@@ -367,54 +450,77 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-}  // namespace
-
-// 2-D bf16 tensor map over rows x cols (row stride in elements), box of
-// box_cols x box_rows, swizzle of 128 or 64 bytes; out-of-range elements
-// read as zero.
-bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, long long stride,
-                    int box_cols, int box_rows, int swizzle_bytes) {
+// 2-D tensor map over a row-major [rows, cols] array of 2- or 4-byte
+// elements (row stride in elements), box of box_cols x box_rows, swizzle of
+// 128, 64 or 0 bytes; out-of-range elements read as zero and are not written.
+bool make_tmap(CUtensorMap* m, bool f32, const void* base, long long rows, long long cols, long long stride,
+               int box_cols, int box_rows, int swizzle_bytes) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const int es = f32 ? 4 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)stride * 2};
+  cuuint64_t strides[1] = {(cuuint64_t)stride * es};
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-namespace {
-
-constexpr int TC_BN = 128;
-constexpr int TC_STAGES = 6;  // 192 KB of shared memory, one persistent CTA per SM
-
-template <int BN, int STAGES>
-cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
-  CUtensorMap ma, ma2, mb, mb2;
+// Operand, side-input and output maps of one launch (unused maps stay zero).
+bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
+  memset(&mp, 0, sizeof(mp));
+  bool ok = true;
   if (a.epi == EPI_DECQG) {
     // A: z as [M, k_tok * K]; B, B2: the stacked [k_tok * K, N] weights
-    if (!make_tmap_bf16(&ma, a.A, a.M, (long long)a.k_tok * a.K, a.lda, BK, BM, 128) ||
-        !make_tmap_bf16(&mb, a.B, (long long)a.k_tok * a.K, a.N, a.ldb, 64, BK, 128) ||
-        !make_tmap_bf16(&mb2, a.B2, (long long)a.k_tok * a.K, a.N, a.ldb, 64, BK, 128))
-      return cudaErrorInvalidValue;
-    ma2 = ma;
+    const long long kk = (long long)a.k_tok * a.K;
+    ok = make_tmap(&mp.a, false, a.A, a.M, kk, a.lda, BK, BM, 128) &&
+         make_tmap(&mp.b, false, a.B, kk, a.N, a.ldb, 64, BK, 128) &&
+         make_tmap(&mp.b2, false, a.B2, kk, a.N, a.ldb, 64, BK, 128);
+    mp.a2 = mp.a;
   } else {
-    if (!make_tmap_bf16(&ma, a.A, a.M, a.K, a.lda, BK, BM, 128)) return cudaErrorInvalidValue;
-    ma2 = ma;
-    if (a.A2 && !make_tmap_bf16(&ma2, a.A2, a.M, a.K, a.lda, BK, BM, 128)) return cudaErrorInvalidValue;
+    ok = make_tmap(&mp.a, false, a.A, a.M, a.K, a.lda, BK, BM, 128);
+    mp.a2 = mp.a;
+    if (ok && a.A2) ok = make_tmap(&mp.a2, false, a.A2, a.M, a.K, a.lda, BK, BM, 128);
     // B is [K, Ncols] with Ncols = ldb (the full weight width)
-    if (!make_tmap_bf16(&mb, a.B, a.K, a.ldb, a.ldb, 64, BK, 128)) return cudaErrorInvalidValue;
-    mb2 = mb;
+    ok = ok && make_tmap(&mp.b, false, a.B, a.K, a.ldb, a.ldb, 64, BK, 128);
+    mp.b2 = mp.b;
   }
-  constexpr int smem = STAGES * (A_BYTES + BN * BK * 2) + 1024;
+  if (!ok) return false;
+  switch (a.epi) {
+    case EPI_QKVG: {
+      const int d = a.d;
+      return make_tmap(&mp.s0, true, a.cos_t, a.M, d / 2, d / 2, 32, BM, 128) &&
+             make_tmap(&mp.s1, true, a.sin_t, a.M, d / 2, d / 2, 32, BM, 128) &&
+             make_tmap(&mp.o[0], false, a.out0, a.M, d, a.ldo, 64, 32, 128) &&
+             make_tmap(&mp.o[1], false, a.out1, a.M, d, a.ldo, 64, 32, 128) &&
+             make_tmap(&mp.o[2], false, a.out2, a.M, d, a.ldo, 32, 32, 64) &&
+             make_tmap(&mp.o[3], true, a.out3, a.M, d, a.ldo, 32, 32, 128);
+    }
+    case EPI_SWIGLU: return make_tmap(&mp.o[0], false, a.out0, a.M, a.d, a.ldo, 32, 32, 64);
+    case EPI_DT: return make_tmap(&mp.o[0], false, a.out0, a.M, a.N, a.ldo, 64, 32, 128);
+    case EPI_DECQG: {
+      const long long w = (long long)a.k_tok * a.N;
+      return make_tmap(&mp.o[0], true, a.out0, a.M, w, a.ldo, 32, 32, 128) &&
+             make_tmap(&mp.o[1], true, a.out1, a.M, w, a.ldo, 32, 32, 128);
+    }
+    default: return make_tmap(&mp.o[0], true, a.out0, a.M, a.N, a.ldo, 32, 32, 128);
+  }
+}
+
+template <int STAGES, int NSLOT, int SLOT, bool SIDE>
+cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t s, int32_t* err) {
+  GemmMaps mp;
+  if (!setup_maps(a, mp)) return cudaErrorInvalidValue;
+  constexpr int smem = STAGES * STAGE_BYTES + NSLOT * SLOT + 1024;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<STAGES, NSLOT, SLOT, SIDE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -429,26 +535,37 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t s, int32_t* err) {
       n_sm = 148;
   }
   const int grid = n_tiles < n_sm ? n_tiles : n_sm;
-  gemm_tc_kernel<BN, STAGES><<<grid, NUM_THREADS, smem, s>>>(ma, ma2, mb, mb2, a, a.K / BK, n_tiles_n, n_tiles, err);
+  gemm_tc_kernel<STAGES, NSLOT, SLOT, SIDE><<<grid, NUM_THREADS, smem, s>>>(mp, a, a.K / BK, n_tiles_n, n_tiles, err);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, long long stride,
+                    int box_cols, int box_rows, int swizzle_bytes) {
+  return make_tmap(m, false, base, rows, cols, stride, box_cols, box_rows, swizzle_bytes);
+}
 
 bool sm100_gemm_supported(const GemmArgs& a) {
   if (a.a_f32) return false;
   if (a.M <= 0 || a.K % BK != 0 || a.K <= 0) return false;
   if ((a.lda % 8) || (a.ldb % 8) || (a.ldo % 8)) return false;
   switch (a.epi) {
-    case EPI_QKVG: return a.d % TC_BN == 0 && a.N == 5 * a.d && a.ldb == 5LL * a.d;
-    case EPI_SWIGLU: return a.d % (TC_BN / 2) == 0 && a.N == 2 * a.d && a.ldb == 2LL * a.d;
-    case EPI_DECQG: return a.N % TC_BN == 0 && a.ldb == a.N && a.B2 != nullptr && a.k_tok >= 1;
-    default: return a.N % TC_BN == 0 && a.ldb == a.N;
+    case EPI_QKVG: return a.d % BN == 0 && a.N == 5 * a.d && a.ldb == 5LL * a.d;
+    case EPI_SWIGLU: return a.d % (BN / 2) == 0 && a.N == 2 * a.d && a.ldb == 2LL * a.d;
+    case EPI_DECQG: return a.N % BN == 0 && a.ldb == a.N && a.B2 != nullptr && a.k_tok >= 1;
+    default: return a.N % BN == 0 && a.ldb == a.N;
   }
 }
 
+// Shared memory per configuration: stages of 32 KB plus the epilogue slots
+// (224 KB in each case, one CTA per SM).
 cudaError_t launch_gemm_sm100(const GemmArgs& a, cudaStream_t s, int32_t* err) {
-  return launch_bn<TC_BN, TC_STAGES>(a, s, err);
+  switch (a.epi) {
+    case EPI_QKVG: return launch_cfg<3, 2, 65536, true>(a, s, err);    // cos + sin in, double-buffered
+    case EPI_SWIGLU: case EPI_DT: return launch_cfg<6, 1, 32768, false>(a, s, err);  // bf16 out
+    default: return launch_cfg<5, 1, 65536, false>(a, s, err);        // fp32 out (store or residual add)
+  }
 }
 
 }  // namespace rest
