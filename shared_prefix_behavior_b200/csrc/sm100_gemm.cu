@@ -1,24 +1,33 @@
 // tcgen05 GEMM for sm_100a with the fused epilogues of the ReST encoder and
 // decoder (bf16 operands, fp32 accumulation in TMEM).
 //
-// A persistent CTA per SM walks 128 x 128 tiles of C = A . B:
-//   warp 0       TMA producer: per stage an A box [128 rows x 64 K] (K-major,
-//                128B swizzle) and two 64-column boxes of B [64 K x 64 N]
-//                (N-major, 128B swizzle); for the DGA projection also the
-//                tile's rows of the rotation table (cos, sin) into a side
-//                slot, one tile ahead of the epilogue that uses them;
-//   warp 1       allocates TMEM (two accumulators); one thread issues
-//                tcgen05.mma (M=128, N=128, K=16) and commits each stage back;
-//   warps 2..9   epilogue, two warps per TMEM lane quarter (each takes half of
-//                the columns): tcgen05.ld of its rows, the fused epilogue, the
-//                result written into a swizzled shared-memory box and sent to
-//                global memory by a TMA store; the residual sublayers add into
-//                the fp32 residual stream with a TMA reduce-add, so the
-//                residual is never loaded by the SM.
-// B is read directly from the weight as stored ([K, N] row-major, x . W
-// layout), so no transposed copy of any weight is made. The column blocks an
-// epilogue must pair (V with its gate Gv; W_1 with W_3) are brought into the
-// same tile by choosing which 64-column box of B each slot of the tile loads.
+// CTA pairs (clusters of two CTAs on two SMs) walk tiles of 256 rows of C =
+// A . B; each pair tile is one M=256 tcgen05 MMA chain issued by rank 0, with
+// rank r holding rows [128 r, 128 r + 128) of A and half of the tile's B
+// columns in its own shared memory, and receiving its 128 accumulator rows
+// in its own TMEM. Per CTA and K block that is 16 KB of A and 8 or 16 KB of
+// B for a 128 x 128 or 128 x 256 output block, half the L2 traffic of a
+// single-CTA tile of the same output. In each CTA:
+//   warp 0       TMA producer: the CTA's A box [128 rows x 64 K] (K-major,
+//                128B swizzle) and its 64-column boxes of B [64 K x 64 N]
+//                (N-major, 128B swizzle) into a STAGES-deep ring, completing
+//                on rank 0's barriers;
+//   warp 1       allocates the pair's TMEM (two accumulators of 256 columns);
+//                on rank 0 one thread issues the pair MMAs (M=256, K=16) and
+//                commits each stage back to both producers;
+//   warps 2..9   epilogue, two warps per TMEM lane quarter: tcgen05.ld of the
+//                CTA's rows, the fused epilogue, the result written into a
+//                swizzled shared-memory box and sent to global memory by a
+//                TMA store; the residual sublayers add into the fp32 residual
+//                stream with a TMA reduce-add, so the residual is never loaded;
+//   warp 10      for the DGA projection, the tile's rows of the rotation table
+//                (cos, sin) into a side slot by TMA, one tile ahead of the
+//                epilogue that uses them.
+// Tiles are 256 columns wide for the epilogues that pair two column blocks
+// (rotated Q with K of the same heads, V with its gate Gv, W_1 with W_3) and
+// 128 wide for the fp32 outputs. B is read directly from the weight as stored
+// ([K, N] row-major, x . W layout), so no transposed copy of any weight is
+// made.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -32,14 +41,14 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;
-constexpr int BN = 128;
+constexpr int BM = 128;  // rows per CTA; a pair tile has 256
 constexpr int BK = 64;
-constexpr int NUM_THREADS = 320;  // TMA warp, MMA warp, 8 epilogue warps
+constexpr int NUM_THREADS = 352;  // TMA warp, MMA warp, 8 epilogue warps, side-input TMA warp
 constexpr int EPI_WARPS = 8;
 constexpr int A_BYTES = BM * BK * 2;      // 16 KB
 constexpr int BOX_B_BYTES = 64 * BK * 2;  // one 64-column box of B: 8 KB
-constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + 2 * BOX_B_BYTES;
+constexpr int ACC_COLS = 256;     // TMEM columns of one accumulator
 constexpr int BOX128 = BM * 128;  // a [128 rows x 128 bytes] staging box: 16 KB
 
 // The tensor maps of one launch: operands, side inputs (rotation table) and
@@ -50,16 +59,36 @@ struct GemmMaps {
   CUtensorMap o[4];    // outputs, boxes of 32 rows (see setup_maps)
 };
 
-// Global column of B loaded into box b (0 or 1) of N-tile t.
-__device__ __forceinline__ int b_box_col(const GemmArgs& a, int t, int b) {
+// Width (MMA N) of the tiles: 256 columns (128 per CTA of the pair), 128 for
+// the plain bf16 copy. EPI_QKVG tiles: [0, nH) rotated Q and K of head group
+// t (128 columns each), [nH, 2 nH) V and Gv, then Go in 256-column tiles,
+// with nH = d / 128.
+__host__ __device__ __forceinline__ int tile_n(const GemmArgs& a) { return a.epi == EPI_DT ? 128 : 256; }
+// Output columns of a 256-column tile of an fp32 output; the last tile may end past the width.
+__host__ __device__ __forceinline__ int f32_tiles(int width) { return (width + 255) / 256; }
+
+// Global column (in the B map that box_map selects) of the 64-column box b
+// that CTA `rank` loads for N-tile t.
+__device__ __forceinline__ int b_box_col(const GemmArgs& a, int t, int rank, int b, bool* second_map) {
+  *second_map = false;
   if (a.epi == EPI_QKVG) {
-    const int d = a.d, nQ = d / BN, nV = d / (BN / 2);
-    if (t < 2 * nQ) return t * BN + 64 * b;
-    if (t < 2 * nQ + nV) return (b == 0 ? 2 * d : 3 * d) + (t - 2 * nQ) * 64;  // V and its gate Gv
-    return 4 * d + (t - 2 * nQ - nV) * BN + 64 * b;
+    const int d = a.d, nH = d / 128;
+    if (t < nH) return (rank ? d : 0) + t * 128 + 64 * b;                   // Q | K
+    if (t < 2 * nH) return (rank ? 3 * d : 2 * d) + (t - nH) * 128 + 64 * b;  // V | Gv
+    *second_map = true;                                                     // Go, through its [K, d] view
+    return (t - 2 * nH) * 256 + 128 * rank + 64 * b;
   }
-  if (a.epi == EPI_SWIGLU) return (b == 0 ? 0 : a.d) + t * 64;  // W_1 and W_3
-  return t * BN + 64 * b;
+  if (a.epi == EPI_SWIGLU) {  // W_1 | W_3, each through its own [K, d_ff] view
+    *second_map = rank != 0;
+    return t * 128 + 64 * b;
+  }
+  if (a.epi == EPI_DECQG) {
+    const int per = f32_tiles(a.N), g = t / per, nt = t % per;
+    *second_map = g >= a.k_tok;
+    return nt * 256 + 128 * rank + 64 * b;
+  }
+  if (a.epi == EPI_DT) return t * 128 + 64 * rank;
+  return t * 256 + 128 * rank + 64 * b;
 }
 
 // sigmoid from the hardware base-2 exponential and reciprocal (relative
@@ -83,18 +112,6 @@ __device__ __forceinline__ void stage_f32(uint8_t* box, int r, const float (&v)[
   for (int k = 0; k < 8; ++k)
     *reinterpret_cast<float4*>(box + sw128_off(r, k)) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
 }
-// 32 values as bf16: one 64-byte row (row r) of a 64B-swizzled box
-__device__ __forceinline__ void stage_bf16_sw64(uint8_t* box, int r, const float (&v)[32]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    uint4 u;
-    u.x = pack_bf16(v[8 * k], v[8 * k + 1]);
-    u.y = pack_bf16(v[8 * k + 2], v[8 * k + 3]);
-    u.z = pack_bf16(v[8 * k + 4], v[8 * k + 5]);
-    u.w = pack_bf16(v[8 * k + 6], v[8 * k + 7]);
-    *reinterpret_cast<uint4*>(box + sw64_off(r, k)) = u;
-  }
-}
 // 32 values as bf16 into half (chunks k0..k0+3) of a 128-byte row of a 128B-swizzled box
 __device__ __forceinline__ void stage_bf16_sw128(uint8_t* box, int r, int k0, const float (&v)[32]) {
 #pragma unroll
@@ -108,21 +125,32 @@ __device__ __forceinline__ void stage_bf16_sw128(uint8_t* box, int r, int k0, co
   }
 }
 
-// The epilogue of one tile for one epilogue warp: rows r = 32 q + lane of the
-// tile, accumulator columns [64 part, 64 part + 64). The result is written
-// into the tile's shared-memory slot as 32-row TMA boxes and lane 0 issues
-// their stores. With SIDE (the DGA projection) the slot already holds this
-// tile's rotation table rows and is known to be free; otherwise the warp
-// first waits until its own stores of the previous tile have left the slot.
-template <bool SIDE>
+// Q and K columns of four rotation pairs (ReST eq. 5): outputs 8 bf16 each.
+__device__ __forceinline__ uint4 rotate4(const float* p, float4 c, float4 s) {
+  uint4 u;
+  u.x = pack_bf16(p[0] * c.x - p[1] * s.x, p[0] * s.x + p[1] * c.x);
+  u.y = pack_bf16(p[2] * c.y - p[3] * s.y, p[2] * s.y + p[3] * c.y);
+  u.z = pack_bf16(p[4] * c.z - p[5] * s.z, p[4] * s.z + p[5] * c.z);
+  u.w = pack_bf16(p[6] * c.w - p[7] * s.w, p[6] * s.w + p[7] * c.w);
+  return u;
+}
+
+// The epilogue of one tile for one epilogue warp: rows r = 32 q + lane of
+// the CTA's 128 rows (global rows from y0), a part of the accumulator's
+// columns. The result is written into the tile's shared-memory slot as
+// 32-row TMA boxes and lane 0 issues their stores. With SIDE (the DGA
+// projection) the slot already holds this tile's rotation table rows and is
+// known to be free; otherwise the warp first waits until its own stores of
+// the previous tile have left the slot.
+template <bool SIDE, int NSLOT>
 __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, uint32_t trow, uint8_t* slot, int t,
-                                         int mt, int q, int lane, int part) {
+                                         int m0, int q, int lane, int part, uint32_t acc_empty_addr) {
   const int r = q * 32 + lane;
-  const int y0 = mt * BM + q * 32;
-  float v[32];
+  const int y0 = m0 + q * 32;
+  float v[32], w[32];
   auto slot_ready = [&]() {
     if (!SIDE) {
-      if (lane == 0) bulk_wait_read<0>();
+      if (lane == 0) bulk_wait_read<NSLOT - 1>();  // the stores of this slot's previous tile
       __syncwarp();
     }
   };
@@ -130,86 +158,64 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     fence_async_smem();
     __syncwarp();
   };
-  if (a.epi == EPI_QKVG) {
-    const int d = a.d, nQ = d / BN, nV = d / (BN / 2);
-    if (t < 2 * nQ) {  // Q or K: rotate the pairs (ReST eq. 5) with the staged cos / sin rows
-      const bool isq = t < nQ;
-      uint8_t* cb = slot + part * BOX128;             // cos of pairs [32 part, 32 part + 32)
-      const uint8_t* sb = slot + (2 + part) * BOX128;  // sin of the same pairs
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        tmem_ld32(trow + part * 64 + 32 * j, v);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t off = sw128_off(r, 4 * j + kk);
-          const float4 c = *reinterpret_cast<const float4*>(cb + off);
-          const float4 s = *reinterpret_cast<const float4*>(sb + off);
-          const float* p = v + 8 * kk;
-          uint4 u;
-          u.x = pack_bf16(p[0] * c.x - p[1] * s.x, p[0] * s.x + p[1] * c.x);
-          u.y = pack_bf16(p[2] * c.y - p[3] * s.y, p[2] * s.y + p[3] * c.y);
-          u.z = pack_bf16(p[4] * c.z - p[5] * s.z, p[4] * s.z + p[5] * c.z);
-          u.w = pack_bf16(p[6] * c.w - p[7] * s.w, p[6] * s.w + p[7] * c.w);
-          // the 8 outputs of these 4 pairs take the bytes of their cos values
-          *reinterpret_cast<uint4*>(cb + off) = u;
-        }
-      }
-      issue();
-      if (lane == 0) {
-        tma_store_2d(&mp.o[isq ? 0 : 1], cb + q * 32 * 128, (isq ? t : t - nQ) * BN + 64 * part, y0);
-        bulk_commit();
-      }
-      return;
-    }
-    if (t < 2 * nQ + nV) {  // value gate: V' = sigmoid(Gv) * V (eq. 3), 64 output columns
-      uint8_t* box = slot + part * (BM * 64);
-      float g[32];
-      tmem_ld32(trow + 32 * part, v);
-      tmem_ld32(trow + 64 + 32 * part, g);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= sigmoid_fast(g[j]);
-      slot_ready();
-      stage_bf16_sw64(box, r, v);
-      issue();
-      if (lane == 0) {
-        tma_store_2d(&mp.o[2], box + q * 32 * 64, (t - 2 * nQ) * 64 + 32 * part, y0);
-        bulk_commit();
-      }
-      return;
-    }
-    // output gate sigmoid(Go) (eq. 4), fp32
+  // the accumulator is free for the next MMAs as soon as its last columns are in registers
+  auto release = [&]() {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(acc_empty_addr);
+  };
+  const int nH = a.d / 128;
+  if (a.epi == EPI_QKVG && t < nH) {
+    // rotated Q and K of head group t; this warp takes pairs [32 part, 32 part + 32) of both,
+    // and the outputs take the bytes of the cos (Q) and sin (K) values they were made from
+    uint8_t* cb = slot + part * BOX128;
+    uint8_t* sb = slot + (2 + part) * BOX128;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      tmem_ld32(trow + part * 64 + 32 * j, v);
+      tmem_ld32x2(trow + part * 64 + 32 * j, v, trow + 128 + part * 64 + 32 * j, w);  // Q and K columns
+      if (j == 1) release();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = sigmoid_fast(v[i]);
-      if (j == 0) slot_ready();
-      stage_f32(slot + (2 * part + j) * BOX128, r, v);
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t off = sw128_off(r, 4 * j + kk);
+        const float4 c = *reinterpret_cast<const float4*>(cb + off);
+        const float4 s = *reinterpret_cast<const float4*>(sb + off);
+        const uint4 uq = rotate4(v + 8 * kk, c, s);
+        const uint4 uk = rotate4(w + 8 * kk, c, s);
+        *reinterpret_cast<uint4*>(cb + off) = uq;
+        *reinterpret_cast<uint4*>(sb + off) = uk;
+      }
     }
     issue();
     if (lane == 0) {
-      const int x0 = (t - 2 * nQ - nV) * BN;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int c = 2 * part + j;
-        tma_store_2d(&mp.o[3], slot + c * BOX128 + q * 32 * 128, x0 + 32 * c, y0);
-      }
+      tma_store_2d(&mp.o[0], cb + q * 32 * 128, t * 128 + 64 * part, y0);
+      tma_store_2d(&mp.o[1], sb + q * 32 * 128, t * 128 + 64 * part, y0);
       bulk_commit();
     }
     return;
   }
-  if (a.epi == EPI_SWIGLU) {  // SiLU(x W_1) * (x W_3), 64 output columns
-    uint8_t* box = slot + part * (BM * 64);
-    float u[32];
-    tmem_ld32(trow + 32 * part, v);
-    tmem_ld32(trow + 64 + 32 * part, u);
+  if ((a.epi == EPI_QKVG && t < 2 * nH) || a.epi == EPI_SWIGLU) {
+    // V' = sigmoid(Gv) * V (eq. 3) or SiLU(x W_1) * (x W_3): accumulator columns
+    // [0, 128) and [128, 256) pair up; this warp makes output columns [64 part, 64 part + 64)
+    const bool gate = a.epi == EPI_QKVG;
+    uint8_t* box = slot + part * BOX128;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = v[j] * sigmoid_fast(v[j]) * u[j];
-    slot_ready();
-    stage_bf16_sw64(box, r, v);
+    for (int j = 0; j < 2; ++j) {
+      tmem_ld32x2(trow + part * 64 + 32 * j, v, trow + 128 + part * 64 + 32 * j, w);
+      if (j == 1) release();
+      if (gate) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= sigmoid_fast(w[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = v[i] * sigmoid_fast(v[i]) * w[i];
+      }
+      if (j == 0) slot_ready();
+      stage_bf16_sw128(box, r, 4 * j, v);
+    }
     issue();
-    if (lane == 0) {
-      tma_store_2d(&mp.o[0], box + q * 32 * 64, t * 64 + 32 * part, y0);
+    const int x = (gate ? t - nH : t) * 128 + 64 * part;
+    if (lane == 0 && x < a.d) {  // the last SwiGLU tile may end past d_ff
+      tma_store_2d(&mp.o[gate ? 2 : 0], box + q * 32 * 128, x, y0);
       bulk_commit();
     }
     return;
@@ -219,30 +225,40 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       tmem_ld32(trow + part * 64 + 32 * j, v);
+      if (j == 1) release();
       if (j == 0) slot_ready();
       stage_bf16_sw128(box, r, 4 * j, v);
     }
     issue();
     if (lane == 0) {
-      tma_store_2d(&mp.o[0], box + q * 32 * 128, t * BN + 64 * part, y0);
+      tma_store_2d(&mp.o[0], box + q * 32 * 128, t * 128 + 64 * part, y0);
       bulk_commit();
     }
     return;
   }
-  // fp32 outputs: plain, sigmoid, the decoder's q / gate, or the residual add
+  // fp32 outputs (256-column tiles, this warp's 128 columns in four 32-column
+  // chunks through two staging boxes): the output gate sigmoid(Go) (eq. 4),
+  // plain, sigmoid, the decoder's q / gate, or the residual add
   const CUtensorMap* om = &mp.o[0];
-  int x0 = t * BN;
+  int x0 = t * 256, width = a.N;
   bool sig = a.epi == EPI_SIGMOID;
-  if (a.epi == EPI_DECQG) {  // tile t: group g (q of token k = g, or the gate of token k = g - k_tok), N-tile nt
-    const int per = a.N / BN, g = t / per, nt = t % per, k = g % a.k_tok;
+  if (a.epi == EPI_QKVG) {
+    om = &mp.o[3];
+    x0 = (t - 2 * nH) * 256;
+    width = a.d;
+    sig = true;
+  } else if (a.epi == EPI_DECQG) {  // tile t: group g (q of token k = g, or the gate of token k = g - k_tok), N-tile nt
+    const int per = f32_tiles(a.N), g = t / per, nt = t % per, k = g % a.k_tok;
     om = g < a.k_tok ? &mp.o[0] : &mp.o[1];
-    x0 = k * a.N + nt * BN;
+    x0 = k * a.N + nt * 256;
+    width = k * a.N + a.N;
     sig = g >= a.k_tok;
   }
   const bool resid = a.epi == EPI_RESID;
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    tmem_ld32(trow + part * 64 + 32 * j, v);
+  for (int c = 0; c < 4; ++c) {
+    tmem_ld32(trow + part * 128 + 32 * c, v);
+    if (c == 3) release();
     if (resid) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] *= a.alpha;
@@ -250,30 +266,34 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = sigmoid_fast(v[i]);
     }
-    if (j == 0) slot_ready();
-    stage_f32(slot + (2 * part + j) * BOX128, r, v);
-  }
-  issue();
-  if (lane == 0) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int c = 2 * part + j;
-      const uint8_t* src = slot + c * BOX128 + q * 32 * 128;
-      // x_res += alpha * acc: the add happens at the residual's home in memory
-      if (resid) tma_reduce_add_2d(om, src, x0 + 32 * c, y0);
-      else tma_store_2d(om, src, x0 + 32 * c, y0);
+    uint8_t* box = slot + (2 * part + (c & 1)) * BOX128;
+    if (c >= 2 || !SIDE) {  // the store that last read this box (two chunks back) is done
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
     }
-    bulk_commit();
+    stage_f32(box, r, v);
+    issue();
+    const int x = x0 + part * 128 + 32 * c;
+    if (lane == 0 && x < width) {
+      const uint8_t* src = box + q * 32 * 128;
+      // x_res += alpha * acc: the add happens at the residual's home in memory
+      if (resid) tma_reduce_add_2d(om, src, x, y0);
+      else tma_store_2d(om, src, x, y0);
+    }
+    if (lane == 0) bulk_commit();
   }
 }
 
-// Persistent kernel: one CTA per SM walks the tiles t = blockIdx.x, +gridDim.x,
-// ... (N-tiles of one 128-row block adjacent, so concurrent CTAs share A and
-// B in L2). The accumulator is double-buffered in TMEM: the epilogue of tile
-// i runs while the MMAs of tile i+1 proceed. NSLOT shared-memory slots of
-// SLOT bytes hold the epilogue's side inputs and staged outputs; with SIDE the
-// producer fills slot i % 2 for tile i once every epilogue warp has released
-// it (after the stores of tile i - 2 have read it out).
+// Persistent kernel: pair c walks the pair tiles c, c + n_pairs, ... (N-tiles
+// of one 256-row block adjacent, so concurrent pairs share A and B in L2).
+// The accumulator is double-buffered in TMEM: the epilogue of tile i runs
+// while the MMAs of tile i+1 proceed. NSLOT shared-memory slots of SLOT
+// bytes hold the epilogue's side inputs and staged outputs; with SIDE the
+// producer fills slot i % 2 for tile i once every epilogue warp of its CTA
+// has released it (after the stores of tile i - 2 have read it out).
+// Barriers: full[s] and acc_empty[b] of rank 0 collect both CTAs (the TMA
+// bytes of both, the epilogue warps of both); empty[s], acc_full[b] and the
+// side barriers are per CTA, the MMA commits arriving on both CTAs' copies.
 template <int STAGES, int NSLOT, int SLOT, bool SIDE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ GemmMaps mp, const GemmArgs a, int num_kb, int n_tiles_n, int n_tiles,
@@ -281,7 +301,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   static_assert(!SIDE || NSLOT == 2, "side inputs are double-buffered");
   // with a low part A2, the K loop runs twice: A . B, then A2 . B
   const int nkb = a.A2 ? 2 * num_kb : num_kb;
-  constexpr int EPI_THREADS = EPI_WARPS * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* slots = smem + STAGES * STAGE_BYTES;
@@ -290,6 +309,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = (int)cluster_rank();
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int nH = a.d / 128;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -298,7 +320,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], EPI_THREADS);
+      mbar_init(&acc_empty[b], 2 * EPI_WARPS);
       mbar_init(&side_full[b], 1);
       mbar_init(&side_empty[b], EPI_WARPS);
     }
@@ -306,84 +328,89 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(&tslot, 2 * BN);
+  if (warp == 1) tmem_alloc_pair(&tslot, 2 * ACC_COLS);
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or complete_tx
   tc_fence_after();
   const uint32_t tmem = tslot;
 
   if (warp == 0 && lane == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA producer (both CTAs)
     prefetch_tmap(&mp.a);
     if (a.A2) prefetch_tmap(&mp.a2);
     prefetch_tmap(&mp.b);
-    if (a.B2) prefetch_tmap(&mp.b2);
-    if (SIDE) {
-      prefetch_tmap(&mp.s0);
-      prefetch_tmap(&mp.s1);
-    }
-    int it = 0, issued = 0, i = 0, side_issued = 0;
-    for (int tile = blockIdx.x; tile < n_tiles && !abort_flag; tile += gridDim.x, ++i) {
-      const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
+    if (a.B2 || a.epi == EPI_SWIGLU || a.epi == EPI_QKVG) prefetch_tmap(&mp.b2);
+    int it = 0, issued = 0;
+    for (int tile = pair; tile < n_tiles && !abort_flag; tile += n_pairs) {
+      const int t = tile % n_tiles_n;
+      const int m0 = (tile / n_tiles_n) * 2 * BM + rank * BM;
+      const int nb = tile_n(a) / 128;  // 64-column boxes of B per CTA
+      const uint32_t tx = 2 * (A_BYTES + nb * BOX_B_BYTES);
+      // decoder projections: token type k selects the column block of z and the row block of the weights
+      const int kofs = a.epi == EPI_DECQG ? ((t / f32_tiles(a.N)) % a.k_tok) * a.K : 0;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % STAGES;
         const int kk = kb < num_kb ? kb : kb - num_kb;
         if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, err, &abort_flag)) break;
         uint8_t* st = smem + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-        if (a.epi == EPI_DECQG) {
-          const int per = a.N / BN, g = t / per, nt = t % per, k = g % a.k_tok;
-          tma_load_2d(st, &mp.a, k * a.K + kk * BK, mt * BM, &full[s]);
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, g < a.k_tok ? &mp.b : &mp.b2, nt * BN + 64 * b,
-                        k * a.K + kk * BK, &full[s]);
-        } else {
-          tma_load_2d(st, kb < num_kb ? &mp.a : &mp.a2, kk * BK, mt * BM, &full[s]);
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-            tma_load_2d(st + A_BYTES + b * BOX_B_BYTES, &mp.b, b_box_col(a, t, b), kk * BK, &full[s]);
+        if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
+        const uint32_t fb = peer_addr(&full[s], 0);
+        tma_load_2d_pair(st, kb < num_kb ? &mp.a : &mp.a2, kofs + kk * BK, m0, fb);
+        for (int b = 0; b < nb; ++b) {
+          bool second;
+          const int col = b_box_col(a, t, rank, b, &second);
+          tma_load_2d_pair(st + A_BYTES + b * BOX_B_BYTES, second ? &mp.b2 : &mp.b, col, kofs + kk * BK, fb);
         }
         issued = it + 1;
-      }
-      if (SIDE && !abort_flag) {
-        // the rotation table rows of a Q or K tile; other tiles only pass the slot on
-        const int s = i & 1;
-        if (!mbar_wait(&side_empty[s], ((i >> 1) & 1) ^ 1, err, &abort_flag)) break;
-        const int nQ = a.d / BN;
-        if (t < 2 * nQ) {
-          const int pair0 = (t < nQ ? t : t - nQ) * (BN / 2);
-          uint8_t* sl = slots + s * SLOT;
-          mbar_arrive_expect_tx(&side_full[s], 4 * BOX128);
-#pragma unroll
-          for (int p = 0; p < 2; ++p) {
-            tma_load_2d(sl + p * BOX128, &mp.s0, pair0 + 32 * p, mt * BM, &side_full[s]);
-            tma_load_2d(sl + (2 + p) * BOX128, &mp.s1, pair0 + 32 * p, mt * BM, &side_full[s]);
-          }
-          side_issued = i + 1;
-        } else {
-          mbar_arrive(&side_full[s]);
-        }
       }
     }
     if (abort_flag) {  // let the copies already in flight land before the CTA exits
       volatile int no_abort = 0;
-      for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+      for (int j = (issued > STAGES ? issued - STAGES : 0); rank == 0 && j < issued; ++j)
         mbar_wait(&full[j % STAGES], (j / STAGES) & 1, nullptr, &no_abort);
-      for (int j = (side_issued > 2 ? side_issued - 2 : 0); SIDE && j < side_issued; ++j)
+    }
+  } else if (SIDE && warp == 10 && lane == 0) {
+    // ------------------------------------------------ side-input TMA (DGA projection)
+    // the rotation table rows of a Q/K tile into slot i % 2 once every epilogue
+    // warp has released it; other tiles only pass the slot on
+    prefetch_tmap(&mp.s0);
+    prefetch_tmap(&mp.s1);
+    int i = 0, side_issued = 0;
+    for (int tile = pair; tile < n_tiles && !abort_flag; tile += n_pairs, ++i) {
+      const int t = tile % n_tiles_n;
+      const int m0 = (tile / n_tiles_n) * 2 * BM + rank * BM;
+      const int s = i & 1;
+      if (!mbar_wait(&side_empty[s], ((i >> 1) & 1) ^ 1, err, &abort_flag)) break;
+      if (t < nH) {
+        uint8_t* sl = slots + s * SLOT;
+        mbar_arrive_expect_tx(&side_full[s], 4 * BOX128);
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          tma_load_2d(sl + p * BOX128, &mp.s0, t * 64 + 32 * p, m0, &side_full[s]);
+          tma_load_2d(sl + (2 + p) * BOX128, &mp.s1, t * 64 + 32 * p, m0, &side_full[s]);
+        }
+        side_issued = i + 1;
+      } else {
+        mbar_arrive(&side_full[s]);
+      }
+    }
+    if (abort_flag) {  // let the copies already in flight land before the CTA exits
+      volatile int no_abort = 0;
+      for (int j = (side_issued > 2 ? side_issued - 2 : 0); j < side_issued; ++j)
         mbar_wait(&side_full[j & 1], (j >> 1) & 1, nullptr, &no_abort);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc = idesc_bf16(BN, 1);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------ MMA issuer (rank 0 only)
     int it = 0, i = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++i) {
+    for (int tile = pair; tile < n_tiles && ok; tile += n_pairs, ++i) {
+      const uint32_t idesc = idesc_bf16_pair(tile_n(a));
       const int b = i & 1;
-      // the epilogue has drained this accumulator (tile i-2)
+      // both CTAs' epilogues have drained this accumulator (tile i-2)
       if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, err, &abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t acc = tmem + b * BN;
+      const uint32_t acc = tmem + b * ACC_COLS;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % STAGES;
         if (!mbar_wait(&full[s], (it / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
@@ -396,24 +423,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
           // B: N-major, 128B swizzle; 8-row K groups 1024 B apart, 64-column boxes 8 KB apart
           const uint64_t bd = smem_desc(b_base + k * 2048, BOX_B_BYTES, 1024, 2);
-          mma_bf16(acc, ad, bd, idesc, (kb | k) != 0);
+          mma_bf16_pair(acc, ad, bd, idesc, (kb | k) != 0);
         }
-        mma_commit(&empty[s]);
+        mma_commit_pair(&empty[s]);
       }
-      if (ok) mma_commit(&acc_full[b]);
+      if (ok) mma_commit_pair(&acc_full[b]);
     }
-    mma_commit(&drain);
+    mma_commit_pair(&drain);
     volatile int no_abort = 0;
     mbar_wait(&drain, 0, nullptr, &no_abort);
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp < 10) {
     // ------------------------------------------------ epilogue (two warps per TMEM lane quarter)
     const int q = warp & 3;
     const int part = (warp - 2) >> 2;  // warps 2..5: first half of the columns, 6..9: second half
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t acc_empty0[2] = {peer_addr(&acc_empty[0], 0), peer_addr(&acc_empty[1], 0)};
     int i = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++i) {
+    for (int tile = pair; tile < n_tiles; tile += n_pairs, ++i) {
       const int b = i & 1;
-      const int t = tile % n_tiles_n, mt = tile / n_tiles_n;
+      const int t = tile % n_tiles_n;
+      const int m0 = (tile / n_tiles_n) * 2 * BM + rank * BM;
       if (SIDE) {
         // release the previous tile's slot once this warp's stores have read it out
         if (i > 0 && lane == 0) {
@@ -424,17 +453,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!mbar_wait(&acc_full[b], (i >> 1) & 1, err, &abort_flag)) break;
       tc_fence_after();
-      epilogue<SIDE>(a, mp, tmem + b * BN + lane_off, slots + (i % NSLOT) * SLOT, t, mt, q, lane, part);
-      tc_fence_before();
-      mbar_arrive(&acc_empty[b]);
+      epilogue<SIDE, NSLOT>(a, mp, tmem + b * ACC_COLS + lane_off, slots + (i % NSLOT) * SLOT, t, m0, q, lane, part,
+                            acc_empty0[b]);
     }
     if (lane == 0) bulk_wait<0>();  // every store has completed before the CTA's shared memory goes away
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the pair's MMAs, remote arrivals and TMEM reads are all done
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    tmem_dealloc_pair(tmem, 2 * ACC_COLS);
   }
 }
 
@@ -486,9 +515,20 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
     ok = make_tmap(&mp.a, false, a.A, a.M, a.K, a.lda, BK, BM, 128);
     mp.a2 = mp.a;
     if (ok && a.A2) ok = make_tmap(&mp.a2, false, a.A2, a.M, a.K, a.lda, BK, BM, 128);
-    // B is [K, Ncols] with Ncols = ldb (the full weight width)
-    ok = ok && make_tmap(&mp.b, false, a.B, a.K, a.ldb, a.ldb, 64, BK, 128);
-    mp.b2 = mp.b;
+    if (a.epi == EPI_SWIGLU) {
+      // W_1 and W_3 as two [K, d_ff] views of the [K, 2 d_ff] weight, so that a
+      // ragged last tile reads zeros past d_ff rather than the other block
+      const bf16* w = static_cast<const bf16*>(a.B);
+      ok = ok && make_tmap(&mp.b, false, w, a.K, a.d, a.ldb, 64, BK, 128) &&
+           make_tmap(&mp.b2, false, w + a.d, a.K, a.d, a.ldb, 64, BK, 128);
+    } else {
+      // B is [K, Ncols] with Ncols = ldb (the full weight width)
+      ok = ok && make_tmap(&mp.b, false, a.B, a.K, a.ldb, a.ldb, 64, BK, 128);
+      mp.b2 = mp.b;
+      // the output-gate block W_go as its own [K, d] view (a ragged last Go tile reads zeros)
+      if (ok && a.epi == EPI_QKVG)
+        ok = make_tmap(&mp.b2, false, static_cast<const bf16*>(a.B) + 4LL * a.d, a.K, a.d, a.ldb, 64, BK, 128);
+    }
   }
   if (!ok) return false;
   switch (a.epi) {
@@ -498,10 +538,10 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
              make_tmap(&mp.s1, true, a.sin_t, a.M, d / 2, d / 2, 32, BM, 128) &&
              make_tmap(&mp.o[0], false, a.out0, a.M, d, a.ldo, 64, 32, 128) &&
              make_tmap(&mp.o[1], false, a.out1, a.M, d, a.ldo, 64, 32, 128) &&
-             make_tmap(&mp.o[2], false, a.out2, a.M, d, a.ldo, 32, 32, 64) &&
+             make_tmap(&mp.o[2], false, a.out2, a.M, d, a.ldo, 64, 32, 128) &&
              make_tmap(&mp.o[3], true, a.out3, a.M, d, a.ldo, 32, 32, 128);
     }
-    case EPI_SWIGLU: return make_tmap(&mp.o[0], false, a.out0, a.M, a.d, a.ldo, 32, 32, 64);
+    case EPI_SWIGLU: return make_tmap(&mp.o[0], false, a.out0, a.M, a.d, a.ldo, 64, 32, 128);
     case EPI_DT: return make_tmap(&mp.o[0], false, a.out0, a.M, a.N, a.ldo, 64, 32, 128);
     case EPI_DECQG: {
       const long long w = (long long)a.k_tok * a.N;
@@ -516,27 +556,40 @@ template <int STAGES, int NSLOT, int SLOT, bool SIDE>
 cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   GemmMaps mp;
   if (!setup_maps(a, mp)) return cudaErrorInvalidValue;
+  auto kern = gemm_tc_kernel<STAGES, NSLOT, SLOT, SIDE>;
   constexpr int smem = STAGES * STAGE_BYTES + NSLOT * SLOT + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<STAGES, NSLOT, SLOT, SIDE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // pairs that can be resident at once (one CTA per SM)
+  static int max_pairs = 0;
+  if (max_pairs == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    cfg.gridDim = dim3(2 * 74);
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    max_pairs = n;
   }
-  int n_tiles_n = a.N / BN;
-  if (a.epi == EPI_QKVG) n_tiles_n = 5 * a.d / BN;
-  if (a.epi == EPI_DECQG) n_tiles_n = 2 * a.k_tok * (a.N / BN);
-  const int n_tiles = n_tiles_n * ((a.M + BM - 1) / BM);
-  static int n_sm = 0;
-  if (n_sm == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      n_sm = 148;
-  }
-  const int grid = n_tiles < n_sm ? n_tiles : n_sm;
-  gemm_tc_kernel<STAGES, NSLOT, SLOT, SIDE><<<grid, NUM_THREADS, smem, s>>>(mp, a, a.K / BK, n_tiles_n, n_tiles, err);
-  return cudaGetLastError();
+  int n_tiles_n = f32_tiles(a.N);
+  if (a.epi == EPI_DT) n_tiles_n = a.N / 128;
+  if (a.epi == EPI_QKVG) n_tiles_n = 2 * (a.d / 128) + f32_tiles(a.d);
+  if (a.epi == EPI_SWIGLU) n_tiles_n = (a.d + 127) / 128;
+  if (a.epi == EPI_DECQG) n_tiles_n = 2 * a.k_tok * f32_tiles(a.N);
+  const int n_tiles = n_tiles_n * ((a.M + 2 * BM - 1) / (2 * BM));
+  cfg.gridDim = dim3(2 * (n_tiles < max_pairs ? n_tiles : max_pairs));
+  return cudaLaunchKernelEx(&cfg, kern, mp, a, a.K / BK, n_tiles_n, n_tiles, err);
 }
 
 }  // namespace
@@ -551,10 +604,10 @@ bool sm100_gemm_supported(const GemmArgs& a) {
   if (a.M <= 0 || a.K % BK != 0 || a.K <= 0) return false;
   if ((a.lda % 8) || (a.ldb % 8) || (a.ldo % 8)) return false;
   switch (a.epi) {
-    case EPI_QKVG: return a.d % BN == 0 && a.N == 5 * a.d && a.ldb == 5LL * a.d;
-    case EPI_SWIGLU: return a.d % (BN / 2) == 0 && a.N == 2 * a.d && a.ldb == 2LL * a.d;
-    case EPI_DECQG: return a.N % BN == 0 && a.ldb == a.N && a.B2 != nullptr && a.k_tok >= 1;
-    default: return a.N % BN == 0 && a.ldb == a.N;
+    case EPI_QKVG: return a.d % 128 == 0 && a.N == 5 * a.d && a.ldb == 5LL * a.d;
+    case EPI_SWIGLU: return a.d % 64 == 0 && a.N == 2 * a.d && a.ldb == 2LL * a.d;
+    case EPI_DECQG: return a.N % 128 == 0 && a.ldb == a.N && a.B2 != nullptr && a.k_tok >= 1;
+    default: return a.N % 128 == 0 && a.ldb == a.N;
   }
 }
 
@@ -562,9 +615,9 @@ bool sm100_gemm_supported(const GemmArgs& a) {
 // (224 KB in each case, one CTA per SM).
 cudaError_t launch_gemm_sm100(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   switch (a.epi) {
-    case EPI_QKVG: return launch_cfg<3, 2, 65536, true>(a, s, err);    // cos + sin in, double-buffered
-    case EPI_SWIGLU: case EPI_DT: return launch_cfg<6, 1, 32768, false>(a, s, err);  // bf16 out
-    default: return launch_cfg<5, 1, 65536, false>(a, s, err);        // fp32 out (store or residual add)
+    case EPI_QKVG: return launch_cfg<3, 2, 65536, true>(a, s, err);                  // cos + sin in, double-buffered
+    case EPI_SWIGLU: case EPI_DT: return launch_cfg<5, 2, 32768, false>(a, s, err);  // bf16 out, double-buffered
+    default: return launch_cfg<5, 1, 65536, false>(a, s, err);                       // fp32 out (store or residual add)
   }
 }
 
