@@ -48,10 +48,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase of `parity` to complete. Returns false (and records
 // REST_ERR_TIMEOUT) if it has not after kWaitCycles; `*abort` is then set so
 // that the caller's loops stop issuing work.
+// The abort flag, the global error word and the clock are looked at only
+// every 128 unsuccessful polls, so that a phase that completes is seen at the
+// next poll rather than after a round trip to global memory.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  const long long t0 = clock64();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 127) != 0) continue;
     if (*abort) return false;
     if (err && *reinterpret_cast<volatile int32_t*>(err) != 0) {  // another CTA already failed
       *abort = 1;
@@ -63,7 +68,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
       return false;
     }
   }
-  return true;
 }
 
 // ------------------------------------------------------------------ TMA
