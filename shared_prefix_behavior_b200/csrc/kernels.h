@@ -22,8 +22,9 @@ cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_us
 // mode 1: x = LN(x); y = dt(x)  (post-LN after the residual add)
 // mode 2: y = dt(x)  (post-LN sublayer input, no norm)
 // mode 3: x = LN(x)  (post-LN, y not written)
+// mode 4: x = LN(x); y = dt(LN2(x))  (post-LN, then the next sublayer's pre-LN with g2, b2)
 cudaError_t launch_layernorm(bool bf16, float* x, void* y, const float* g, const float* b, int T, int d,
-                             int mode, cudaStream_t s);
+                             int mode, cudaStream_t s, const float* g2 = nullptr, const float* b2 = nullptr);
 // x_res = float(x_in)
 cudaError_t launch_to_f32(bool bf16, const void* x_in, float* x_res, long long n, cudaStream_t s);
 // hi = bf16(x), lo = bf16(x - hi): x as an unevaluated sum of two bf16 numbers

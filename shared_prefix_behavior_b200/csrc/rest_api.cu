@@ -494,49 +494,86 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   ea.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
   ea.rows = T;
 
+  // The sublayers in order (attention, then the FFN, per layer), each wrapped
+  // by eq. 6: post-LN in the first l_switch layers, pre-LN after. One
+  // normalisation launch follows each residual add: the post-LN of the
+  // sublayer just finished (if any) merged with the next sublayer's input
+  // (its pre-LN, or a plain cast), or with the cast of H.
+  struct Sub {
+    bool attn;
+    int layer;
+    bool post;
+    const float* g;
+    const float* b;
+  };
+  std::vector<Sub> subs;
   for (int l = 0; l < n_layers; ++l) {
-    const rest_enc_layer& Ly = layers[l];
-    const bool post = (l + 1) <= l_switch;  // eq. 6: post-LN for the first l_switch layers
-    // ---- DGA sublayer (eqs. 3-5)
-    REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
-                 launch_layernorm(bf, xres, y, Ly.ln_attn_g, Ly.ln_attn_b, (int)T, d, post ? 2 : 0, s));
-    GemmArgs a = gemm(y, d, Ly.w_qkvgg, 5LL * d, T, 5 * d, d, EPI_QKVG, q, d);
-    a.out1 = k; a.out2 = v; a.out3 = g; a.cos_t = cos_t; a.sin_t = sin_t; a.d = d;
-    if (rest_status st = run_gemm(p, a, "gemm_qkvg", s)) return st;
-    if (bf && sm100_attn_supported(hd)) {
-      REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_sm100(hd, ea, s, err));
-    } else {
-      REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_simt(bf, hd, ea, s));
-    }
-    a = gemm(o, d, Ly.w_o, d, T, d, d, EPI_RESID, xres, d);
-    a.alpha = Ly.alpha_attn;
-    if (rest_status st = run_gemm(p, a, "gemm_attn_out", s)) return st;
-    if (post)
-      REST_KLAUNCH(s, "layernorm", 0, 8 * Td,
-                   launch_layernorm(bf, xres, y, Ly.ln_attn_g, Ly.ln_attn_b, (int)T, d, 3, s));
-    // ---- SwiGLU FFN sublayer
-    if (Ly.w_ffn13) {
+    const bool post = (l + 1) <= l_switch;
+    subs.push_back({true, l, post, layers[l].ln_attn_g, layers[l].ln_attn_b});
+    if (layers[l].w_ffn13) subs.push_back({false, l, post, layers[l].ln_ffn_g, layers[l].ln_ffn_b});
+  }
+  auto norm = [&](void* out, const float* g, const float* b, int mode, const float* g2, const float* b2) -> rest_status {
+    const double bytes = Td * (mode == 2 ? 4 + e : mode == 3 ? 8 : mode == 0 ? 4 + e : 8 + e);
+    REST_KLAUNCH(s, "layernorm", 0, bytes, launch_layernorm(bf, xres, out, g, b, (int)T, d, mode, s, g2, b2));
+    return REST_OK;
+  };
+  // input of the first sublayer: with post-LN it reads x itself, which in bf16
+  // is the call's input as it stands
+  const void* a_in = y;
+  if (subs[0].post) {
+    if (bf) a_in = x;
+    else if (rest_status st = norm(y, nullptr, nullptr, 2, nullptr, nullptr)) return st;
+  } else if (rest_status st = norm(y, subs[0].g, subs[0].b, 0, nullptr, nullptr)) {
+    return st;
+  }
+  bool h_written = false;
+  for (size_t i = 0; i < subs.size(); ++i) {
+    const Sub& S = subs[i];
+    const rest_enc_layer& Ly = layers[S.layer];
+    if (S.attn) {  // DGA sublayer (eqs. 3-5)
+      GemmArgs a = gemm(a_in, d, Ly.w_qkvgg, 5LL * d, T, 5 * d, d, EPI_QKVG, q, d);
+      a.out1 = k; a.out2 = v; a.out3 = g; a.cos_t = cos_t; a.sin_t = sin_t; a.d = d;
+      if (rest_status st = run_gemm(p, a, "gemm_qkvg", s)) return st;
+      if (bf && sm100_attn_supported(hd)) {
+        REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_sm100(hd, ea, s, err));
+      } else {
+        REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_simt(bf, hd, ea, s));
+      }
+      a = gemm(o, d, Ly.w_o, d, T, d, d, EPI_RESID, xres, d);
+      a.alpha = Ly.alpha_attn;
+      if (rest_status st = run_gemm(p, a, "gemm_attn_out", s)) return st;
+    } else {  // SwiGLU FFN sublayer
       const int dff = Ly.d_ff;
-      REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
-                   launch_layernorm(bf, xres, y, Ly.ln_ffn_g, Ly.ln_ffn_b, (int)T, d, post ? 2 : 0, s));
-      a = gemm(y, d, Ly.w_ffn13, 2LL * dff, T, 2 * dff, d, EPI_SWIGLU, hid, dff);
+      GemmArgs a = gemm(a_in, d, Ly.w_ffn13, 2LL * dff, T, 2 * dff, d, EPI_SWIGLU, hid, dff);
       a.d = dff;
       if (rest_status st = run_gemm(p, a, "gemm_ffn13", s)) return st;
       a = gemm(hid, dff, Ly.w_ffn2, d, T, d, dff, EPI_RESID, xres, d);
       a.alpha = Ly.alpha_ffn;
       if (rest_status st = run_gemm(p, a, "gemm_ffn2", s)) return st;
-      if (post)
-        REST_KLAUNCH(s, "layernorm", 0, 8 * Td,
-                     launch_layernorm(bf, xres, y, Ly.ln_ffn_g, Ly.ln_ffn_b, (int)T, d, 3, s));
     }
+    a_in = y;
+    rest_status st = REST_OK;
+    if (i + 1 < subs.size()) {
+      const Sub& N = subs[i + 1];  // post-LN sublayers come first, so a pre-LN one is followed by pre-LN
+      if (S.post && N.post) st = norm(y, S.g, S.b, 1, nullptr, nullptr);        // x = LN(x), y = x
+      else if (S.post) st = norm(y, S.g, S.b, 4, N.g, N.b);                     // x = LN(x), y = LN'(x)
+      else st = norm(y, N.g, N.b, 0, nullptr, nullptr);                         // y = LN'(x)
+    } else if (S.post) {
+      if (p.hsplit) {
+        st = norm(nullptr, S.g, S.b, 3, nullptr, nullptr);  // x = LN(x)
+      } else {
+        st = norm(h_out, S.g, S.b, 1, nullptr, nullptr);    // x = LN(x), H = x
+        h_written = true;
+      }
+    }
+    if (st != REST_OK) return st;
   }
   // H: the residual stream after the last layer, in the call's dtype (no final norm).
   // When the decoder follows in bf16 it also gets H's low part: H = h_out + h_lo.
   if (p.hsplit) {
     REST_KLAUNCH(s, "split_h", 0, Td * 8, launch_split_bf16(xres, h_out, at<void>(ws, L.hlo), T * d, s));
-  } else {
-    REST_KLAUNCH(s, "layernorm", 0, Td * (4 + e),
-                 launch_layernorm(bf, xres, h_out, nullptr, nullptr, (int)T, d, 2, s));
+  } else if (!h_written) {
+    if (rest_status st = norm(h_out, nullptr, nullptr, 2, nullptr, nullptr)) return st;
   }
   return REST_OK;
 }

@@ -78,7 +78,8 @@ cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_us
 // One warp per row; lane l holds columns 4l + 128k (k < d/128) as float4s.
 template <typename T, int NV>
 __global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
-                                 const float* __restrict__ b, int rows, int d, int mode) {
+                                 const float* __restrict__ b, const float* __restrict__ g2,
+                                 const float* __restrict__ b2, int rows, int d, int mode) {
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
   if (warp >= rows) return;
@@ -118,25 +119,58 @@ __global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const
     load4(b + c, bb);
 #pragma unroll
     for (int i = 0; i < 4; ++i) n[i] = (v[k][i] - mean) * rstd * gg[i] + bb[i];
-    if (mode == 1 || mode == 3) store4(xr + c, n);
-    if (mode != 3) store4(yr + c, n);
+    if (mode == 1 || mode == 3 || mode == 4) store4(xr + c, n);
+    if (mode == 0 || mode == 1) store4(yr + c, n);
+    if (mode == 4) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = n[i];
+    }
+  }
+  if (mode != 4) return;
+  // mode 4: the next sublayer's pre-LN of the row just normalized
+  float sum2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) sum2 += v[k][0] + v[k][1] + v[k][2] + v[k][3];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum2 += __shfl_xor_sync(0xffffffffu, sum2, o);
+  const float mean2 = sum2 / d;
+  float sq2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float t = v[k][i] - mean2;
+      sq2 += t * t;
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq2 += __shfl_xor_sync(0xffffffffu, sq2, o);
+  const float rstd2 = 1.0f / sqrtf(sq2 / d + 1e-5f);
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int c = 128 * k + 4 * lane;
+    float gg[4], bb[4], n[4];
+    load4(g2 + c, gg);
+    load4(b2 + c, bb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) n[i] = (v[k][i] - mean2) * rstd2 * gg[i] + bb[i];
+    store4(yr + c, n);
   }
 }
 
 template <typename T>
-static cudaError_t layernorm_dispatch(float* x, T* y, const float* g, const float* b, int rows, int d, int mode,
-                                      cudaStream_t s) {
+static cudaError_t layernorm_dispatch(float* x, T* y, const float* g, const float* b, const float* g2,
+                                      const float* b2, int rows, int d, int mode, cudaStream_t s) {
   int threads = 256;
   int blocks = (rows * 32 + threads - 1) / threads;
   switch (d / 128) {
-    case 1: layernorm_kernel<T, 1><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
-    case 2: layernorm_kernel<T, 2><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
-    case 3: layernorm_kernel<T, 3><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
-    case 4: layernorm_kernel<T, 4><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
-    case 5: layernorm_kernel<T, 5><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
-    case 6: layernorm_kernel<T, 6><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
-    case 7: layernorm_kernel<T, 7><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
-    case 8: layernorm_kernel<T, 8><<<blocks, threads, 0, s>>>(x, y, g, b, rows, d, mode); break;
+    case 1: layernorm_kernel<T, 1><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 2: layernorm_kernel<T, 2><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 3: layernorm_kernel<T, 3><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 4: layernorm_kernel<T, 4><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 5: layernorm_kernel<T, 5><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 6: layernorm_kernel<T, 6><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 7: layernorm_kernel<T, 7><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 8: layernorm_kernel<T, 8><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -146,7 +180,8 @@ static cudaError_t layernorm_dispatch(float* x, T* y, const float* g, const floa
 // per row, one column per lane and step.
 template <typename T>
 __global__ void layernorm_narrow_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
-                                        const float* __restrict__ b, int rows, int d, int mode) {
+                                        const float* __restrict__ b, const float* __restrict__ g2,
+                                        const float* __restrict__ b2, int rows, int d, int mode) {
   constexpr int VMAX = 32;  // d <= 1024
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
@@ -187,24 +222,48 @@ __global__ void layernorm_narrow_kernel(float* __restrict__ x, T* __restrict__ y
     int c = k * 32 + lane;
     if (c < d) {
       float n = (v[k] - mean) * rstd * g[c] + b[c];
-      if (mode == 1 || mode == 3) xr[c] = n;
-      if (mode != 3) y[(long long)warp * d + c] = from_f<T>(n);
+      if (mode == 1 || mode == 3 || mode == 4) xr[c] = n;
+      if (mode == 0 || mode == 1) y[(long long)warp * d + c] = from_f<T>(n);
+      v[k] = n;
     }
+  }
+  if (mode != 4) return;
+  // mode 4: the next sublayer's pre-LN of the row just normalized
+  float sum2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < VMAX; ++k) sum2 += (k * 32 + lane < d) ? v[k] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum2 += __shfl_xor_sync(0xffffffffu, sum2, o);
+  const float mean2 = sum2 / d;
+  float sq2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < VMAX; ++k) {
+    float t = (k * 32 + lane < d) ? v[k] - mean2 : 0.f;
+    sq2 += t * t;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq2 += __shfl_xor_sync(0xffffffffu, sq2, o);
+  const float rstd2 = 1.0f / sqrtf(sq2 / d + 1e-5f);
+#pragma unroll
+  for (int k = 0; k < VMAX; ++k) {
+    int c = k * 32 + lane;
+    if (c < d) y[(long long)warp * d + c] = from_f<T>((v[k] - mean2) * rstd2 * g2[c] + b2[c]);
   }
 }
 
 cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, const float* b, int T, int d,
-                             int mode, cudaStream_t s) {
+                             int mode, cudaStream_t s, const float* g2, const float* b2) {
   if (T == 0) return cudaSuccess;
+  if (mode == 4 && (!g2 || !b2)) return cudaErrorInvalidValue;
   if (d % 128 == 0 && d <= 1024)
-    return bf16m ? layernorm_dispatch<bf16>(x, (bf16*)y, g, b, T, d, mode, s)
-                 : layernorm_dispatch<float>(x, (float*)y, g, b, T, d, mode, s);
+    return bf16m ? layernorm_dispatch<bf16>(x, (bf16*)y, g, b, g2, b2, T, d, mode, s)
+                 : layernorm_dispatch<float>(x, (float*)y, g, b, g2, b2, T, d, mode, s);
   int threads = 256;
   int blocks = (T * 32 + threads - 1) / threads;
   if (bf16m)
-    layernorm_narrow_kernel<bf16><<<blocks, threads, 0, s>>>(x, (bf16*)y, g, b, T, d, mode);
+    layernorm_narrow_kernel<bf16><<<blocks, threads, 0, s>>>(x, (bf16*)y, g, b, g2, b2, T, d, mode);
   else
-    layernorm_narrow_kernel<float><<<blocks, threads, 0, s>>>(x, (float*)y, g, b, T, d, mode);
+    layernorm_narrow_kernel<float><<<blocks, threads, 0, s>>>(x, (float*)y, g, b, g2, b2, T, d, mode);
   return cudaGetLastError();
 }
 
@@ -213,10 +272,32 @@ __global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ out,
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = to_f<T>(in[i]);
 }
+// 8 bf16 values (16 bytes) per thread in, 32 bytes out
+__global__ void bf16_to_f32_x8_kernel(const uint4* __restrict__ in, float4* __restrict__ out, long long n8) {
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 u = in[i];
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  float f[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f[2 * k] = __uint_as_float(w[k] << 16);
+    f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+  }
+  out[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
+  out[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
+}
 
 cudaError_t launch_to_f32(bool bf16m, const void* x_in, float* x_res, long long n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   int threads = 256;
+  if (bf16m && n % 8 == 0 && (reinterpret_cast<uintptr_t>(x_in) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(x_res) & 15) == 0) {
+    const long long n8 = n / 8;
+    bf16_to_f32_x8_kernel<<<(unsigned)((n8 + threads - 1) / threads), threads, 0, s>>>(
+        static_cast<const uint4*>(x_in), reinterpret_cast<float4*>(x_res), n8);
+    return cudaGetLastError();
+  }
   long long blocks = (n + threads - 1) / threads;
   if (bf16m)
     to_f32_kernel<bf16><<<(unsigned)blocks, threads, 0, s>>>((const bf16*)x_in, x_res, n);

@@ -468,6 +468,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
+      // the output gate of this row, loaded while the last P V completes (head_dim 32;
+      // at 64 the row would not fit the softmax warps' registers next to O)
+      constexpr bool GATE_EARLY = HD <= 32;
+      const long long ro = row_g * d + h * HD;
+      float gate_row[GATE_EARLY ? HD : 4];
+      if (GATE_EARLY && valid && !split) {
+        const float* gate = (DEC ? da.g : ea.gate) + ro;
+#pragma unroll
+        for (int c = 0; c < HD; c += 4) load4(gate + c, &gate_row[c]);
+      }
       if (!mbar_wait(&p_free[t], (cb + nb - 1) & 1, err, &abort_flag)) { ok = false; break; }  // the last P V
       tc_fence_after();
       // every lane takes part in the (warp-collective) TMEM loads
@@ -490,23 +500,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         pml[1] = l_run;
       } else if (valid) {
         const float inv = 1.0f / l_run;
-        const long long ro = row_g * d + h * HD;
-        const float* gate = (DEC ? da.g : ea.gate) + ro;
 #pragma unroll
-        for (int c = 0; c < HD; c += 4) {
-          float gg[4];
-          load4(gate + c, gg);
-          float v[4] = {o[c] * inv * gg[0], o[c + 1] * inv * gg[1], o[c + 2] * inv * gg[2], o[c + 3] * inv * gg[3]};
-          if (DEC && da.out_lo) {  // o * g as a hi + lo pair of bf16 values
-            float lo[4];
+        for (int c0 = 0; c0 < HD; c0 += 32) {  // 32 columns at a time, their gate loads in flight together
+          float gh[32];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
-            store4((bf16*)da.out + ro + c, v);
-            store4((bf16*)da.out_lo + ro + c, lo);
-          } else if (DEC) {
-            store4((float*)da.out + ro + c, v);
-          } else {
-            store4((bf16*)ea.out + ro + c, v);
+          for (int c = 0; c < 32; c += 4) {
+            if (GATE_EARLY) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) gh[c + i] = gate_row[(c0 + c + i) % (GATE_EARLY ? HD : 4)];
+            } else {
+              load4((DEC ? da.g : ea.gate) + ro + c0 + c, &gh[c]);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const int cc = c0 + c;
+            float v[4] = {o[cc] * inv * gh[c], o[cc + 1] * inv * gh[c + 1], o[cc + 2] * inv * gh[c + 2],
+                          o[cc + 3] * inv * gh[c + 3]};
+            if (DEC && da.out_lo) {  // o * g as a hi + lo pair of bf16 values
+              float lo[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
+              store4((bf16*)da.out + ro + cc, v);
+              store4((bf16*)da.out_lo + ro + cc, lo);
+            } else if (DEC) {
+              store4((float*)da.out + ro + cc, v);
+            } else {
+              store4((bf16*)ea.out + ro + cc, v);
+            }
           }
         }
       }
