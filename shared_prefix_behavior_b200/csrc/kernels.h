@@ -12,6 +12,9 @@ struct TableParams {
   int n_heads, half;            // half = head_dim / 2
   long long tau[32];            // per head, 0 = RoPE
   double theta[64];             // theta_j = base^(-2j/head_dim)
+  // fractional turns of 2^(16 k) theta_j / (2 pi), k = 0, 1, 2 (extended precision
+  // on the host): idx theta_j mod 2 pi from the 16-bit pieces of idx
+  double turn[3][64];
 };
 cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users,
                                   int T, const TableParams& p, int64_t* idx_out, float* cos_out,

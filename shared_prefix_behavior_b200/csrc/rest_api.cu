@@ -412,7 +412,14 @@ static TableParams table_params(const rest_heads* hs) {
   tp.n_heads = hs->n_heads;
   tp.half = hs->head_dim / 2;
   for (int h = 0; h < hs->n_heads; ++h) tp.tau[h] = hs->tau[h];
-  for (int j = 0; j < tp.half; ++j) tp.theta[j] = pow(hs->rope_base, -2.0 * j / hs->head_dim);
+  const long double two_pi = 2.0L * 3.141592653589793238462643383279502884L;
+  for (int j = 0; j < tp.half; ++j) {
+    tp.theta[j] = pow(hs->rope_base, -2.0 * j / hs->head_dim);
+    for (int k = 0; k < 3; ++k) {
+      const long double t = (long double)tp.theta[j] * ldexpl(1.0L, 16 * k) / two_pi;
+      tp.turn[k][j] = (double)(t - floorl(t));
+    }
+  }
   return tp;
 }
 

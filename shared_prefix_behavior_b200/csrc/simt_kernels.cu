@@ -25,44 +25,55 @@ __device__ __forceinline__ int find_user(const int32_t* cu, int n_users, int i) 
   return lo;
 }
 
-// One thread per (token, head, frequency j): consecutive threads write
-// consecutive table entries.
+// floor(rel / tau) for tau > 0, exact: a double quotient corrected by integer steps
+__device__ __forceinline__ long long floor_div(long long rel, long long tau) {
+  long long q = (long long)floor((double)rel / (double)tau);
+  while (q * tau > rel) --q;
+  while ((q + 1) * tau <= rel) ++q;
+  return q;
+}
+
+// sin and cos of idx * theta_j: the angle in turns is reduced modulo 1 from the
+// three 16-bit pieces of idx and the host's fractional turns of 2^(16 k) theta_j,
+// so the library routine only ever sees an argument in [-1, 1] half-turns.
+__device__ __forceinline__ void rotation(long long idx, const TableParams& p, int j, double* sv, double* cv) {
+  const double h2 = (double)(idx >> 32), h1 = (double)((idx >> 16) & 0xffff), h0 = (double)(idx & 0xffff);
+  double tr = fma(h2, p.turn[2][j], fma(h1, p.turn[1][j], h0 * p.turn[0][j]));
+  tr -= rint(tr);
+  sincospi(2.0 * tr, sv, cv);
+}
+
+// One thread per (token, frequency j), looping over the heads: the user lookup
+// happens once per token, and consecutive threads write consecutive entries.
 __global__ void rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu,
                                       int n_users, int T, TableParams p, int64_t* idx_out,
                                       float* cos_out, float* sin_out, int32_t* err) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long per_tok = (long long)p.n_heads * p.half;
-  if (gid >= (long long)T * per_tok) return;
-  const int i = (int)(gid / per_tok);
-  const int rem = (int)(gid % per_tok);
-  const int h = rem / p.half, j = rem % p.half;
+  if (gid >= (long long)T * p.half) return;
+  const int i = (int)(gid / p.half);
+  const int j = (int)(gid % p.half);
   const int s = cu[find_user(cu, n_users, i)];
   const long long t = ts[i];
-  if (rem == 0 && i > s && ts[i - 1] > t) set_error(err, REST_ERR_UNSORTED_TIME);
-  const long long tau = p.tau[h];
-  long long idx;
-  if (tau == 0) {
-    idx = i - s;
-  } else {
-    const long long rel = t - ts[s];  // exact int64
-    long long q = rel / tau;          // floor division (rel < 0 only on invalid input)
-    if ((rel % tau != 0) && (rel < 0)) q -= 1;
-    idx = q;
-  }
-  if (idx_out && j == 0) idx_out[(long long)i * p.n_heads + h] = idx;
-  if (cos_out) {
-    const double phi = (double)idx * p.theta[j];
-    double sv, cv;
-    sincos(phi, &sv, &cv);
-    cos_out[gid] = (float)cv;
-    sin_out[gid] = (float)sv;
+  if (j == 0 && i > s && ts[i - 1] > t) set_error(err, REST_ERR_UNSORTED_TIME);
+  const long long rel = t - ts[s];  // exact int64
+  for (int h = 0; h < p.n_heads; ++h) {
+    const long long tau = p.tau[h];
+    const long long idx = tau == 0 ? (long long)(i - s) : floor_div(rel, tau);
+    if (idx_out && j == 0) idx_out[(long long)i * p.n_heads + h] = idx;
+    if (cos_out) {
+      double sv, cv;
+      rotation(idx, p, j, &sv, &cv);
+      const long long o = ((long long)i * p.n_heads + h) * p.half + j;
+      cos_out[o] = (float)cv;
+      sin_out[o] = (float)sv;
+    }
   }
 }
 
 cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users, int T,
                                     const TableParams& p, int64_t* idx_out, float* cos_out,
                                     float* sin_out, int32_t* err, cudaStream_t s) {
-  const long long n = (long long)T * p.n_heads * p.half;
+  const long long n = (long long)T * p.half;
   if (n == 0) return cudaSuccess;
   const int threads = 256;
   const long long blocks = (n + threads - 1) / threads;
@@ -76,22 +87,15 @@ cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_us
 // ============================================================================
 
 // One warp per row; lane l holds columns 4l + 128k (k < d/128) as float4s.
+// One row per warp at a time: the normalisation of a row already in registers
+// (lane holds columns 128 k + 4 lane .. + 3).
 template <typename T, int NV>
-__global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
-                                 const float* __restrict__ b, const float* __restrict__ g2,
-                                 const float* __restrict__ b2, int rows, int d, int mode) {
-  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  float* xr = x + (long long)warp * d;
-  float v[NV][4];
+__device__ __forceinline__ void ln_row(float* __restrict__ xr, T* __restrict__ yr, const float* __restrict__ g,
+                                       const float* __restrict__ b, const float* __restrict__ g2,
+                                       const float* __restrict__ b2, int d, int mode, int lane, float (&v)[NV][4]) {
   float sum = 0.f;
 #pragma unroll
-  for (int k = 0; k < NV; ++k) {
-    load4(xr + 128 * k + 4 * lane, v[k]);
-    sum += v[k][0] + v[k][1] + v[k][2] + v[k][3];
-  }
-  T* yr = y ? y + (long long)warp * d : nullptr;
+  for (int k = 0; k < NV; ++k) sum += v[k][0] + v[k][1] + v[k][2] + v[k][3];
   if (mode == 2) {
 #pragma unroll
     for (int k = 0; k < NV; ++k) store4(yr + 128 * k + 4 * lane, v[k]);
@@ -157,11 +161,49 @@ __global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const
   }
 }
 
+
+// Grid-stride over rows; each warp loads its next row before normalising the
+// current one, so the load latency of one row hides behind the work of another.
+template <typename T, int NV>
+__global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
+                                 const float* __restrict__ b, const float* __restrict__ g2,
+                                 const float* __restrict__ b2, int rows, int d, int mode) {
+  const int lane = threadIdx.x & 31;
+  const int n_warps = gridDim.x * (blockDim.x >> 5);
+  int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  float v[NV][4], nx[NV][4];
+  if (row < rows) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) load4(x + (long long)row * d + 128 * k + 4 * lane, v[k]);
+  }
+  for (; row < rows; row += n_warps) {
+    const int next = row + n_warps;
+    if (next < rows) {
+#pragma unroll
+      for (int k = 0; k < NV; ++k) load4(x + (long long)next * d + 128 * k + 4 * lane, nx[k]);
+    }
+    ln_row<T, NV>(x + (long long)row * d, y ? y + (long long)row * d : nullptr, g, b, g2, b2, d, mode, lane, v);
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = nx[k][i];
+  }
+}
+
 template <typename T>
 static cudaError_t layernorm_dispatch(float* x, T* y, const float* g, const float* b, const float* g2,
                                       const float* b2, int rows, int d, int mode, cudaStream_t s) {
   int threads = 256;
   int blocks = (rows * 32 + threads - 1) / threads;
+  static int cap = 0;
+  if (cap == 0) {
+    int dev = 0, n_sm = 0;
+    cap = (cudaGetDevice(&dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n_sm > 0)
+              ? 8 * n_sm
+              : 1184;
+  }
+  if (blocks > cap) blocks = cap;
   switch (d / 128) {
     case 1: layernorm_kernel<T, 1><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
     case 2: layernorm_kernel<T, 2><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
