@@ -16,9 +16,9 @@
 //                softmax overlaps the other's MMAs.
 //   warps 4..7   softmax of tile 0, warps 8..11 of tile 1: a thread owns a
 //                query row; it reads its row of S from TMEM, masks, keeps the
-//                running max, exponentiates in base 2, and writes P (bf16) to
-//                shared memory in the 128B-swizzled K-major layout the MMA
-//                reads. O stays in TMEM: when a row's max grows by more than
+//                running max, exponentiates in base 2, and writes P (bf16
+//                pairs) back to the tile's P columns of TMEM, from where the
+//                P V MMA takes its A operand. O stays in TMEM: when a row's max grows by more than
 //                2^8 the thread rescales its O row in TMEM (after the previous
 //                P V has completed); otherwise P is taken relative to the old
 //                max (values up to 2^8, exact in fp32 accumulation).
@@ -50,12 +50,13 @@ struct Cfg {
   static constexpr int TILE_BYTES = ROWS * ROW_BYTES;  // 128 rows
   static constexpr int SWZ = HD == 64 ? 2 : 4;         // descriptor code: 128B / 64B swizzle
   static constexpr int ATOM = 8 * ROW_BYTES;           // bytes of 8 swizzled rows
-  static constexpr int P_BYTES = ROWS * KB * 2;        // 32 KB
 };
-// TMEM columns: S_0 | S_1 | O_0 | O_1
+// TMEM columns: S_0 | S_1 | O_0 | O_1 | P_0 | P_1 (P: 128 bf16 keys packed in 64 columns)
 __device__ __forceinline__ uint32_t s_col(int t) { return (uint32_t)(t * 128); }
 template <int HD>
 __device__ __forceinline__ uint32_t o_col(int t) { return (uint32_t)(256 + t * HD); }
+template <int HD>
+__device__ __forceinline__ uint32_t p_col(int t) { return (uint32_t)(256 + NT * HD + t * 64); }
 
 // byte offset of 16-byte chunk u of row r in a swizzled [128 x HD] bf16 tile
 template <int HD>
@@ -66,15 +67,14 @@ __device__ __forceinline__ uint32_t swz_off(int r, int u) {
 
 template <int HD, int MODE>
 struct SmemLayout {
-  // [Q_0 | Q_1 | (decoder) Qlo_0 | Qlo_1 | KV stages | P_0 | P_1], 1024-aligned blocks
+  // [Q_0 | Q_1 | (decoder) Qlo_0 | Qlo_1 | KV stages], 1024-aligned blocks
   static constexpr int STAGES = MODE == 2 ? 2 : 3;
   static constexpr int Q = 0;
   static constexpr int QLO = NT * Cfg<HD>::TILE_BYTES;
   static constexpr int KV = (MODE >= 1 ? 2 : 1) * NT * Cfg<HD>::TILE_BYTES;
   // a stage holds K and V' (encoder), H (decoder), or H_hi and H_lo
   static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
-  static constexpr int P = KV + STAGES * STAGE;
-  static constexpr int TOTAL = P + NT * Cfg<HD>::P_BYTES;
+  static constexpr int TOTAL = KV + STAGES * STAGE;
 };
 
 // Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
@@ -295,19 +295,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               if (i == 0 && qn[t] >= 1 &&  // the previous item's O_t has been read out
                   !mbar_wait(&o_empty[t], (qn[t] - 1) & 1, err, &abort_flag)) { ok = false; break; }
               tc_fence_after();
-              const uint32_t p_base = smem_u32(smem + L::P + t * C::P_BYTES);
+              const uint32_t tP = tmem + p_col<HD>(t);  // A = P_t from TMEM, 8 columns per K step of 16
               const uint32_t v_base = smem_u32(smem + L::KV + sti * L::STAGE + (DEC ? 0 : C::TILE_BYTES));
               const uint32_t tO = tmem + o_col<HD>(t);
 #pragma unroll
               for (int k = 0; k < KB / 16; ++k)
-                mma_bf16(tO, smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2),
-                         smem_desc(v_base + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO, (i | k) != 0);
+                mma_bf16_ts(tO, tP + k * 8, smem_desc(v_base + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO,
+                            (i | k) != 0);
               if (HLO) {  // + P H_lo
 #pragma unroll
                 for (int k = 0; k < KB / 16; ++k)
-                  mma_bf16(tO, smem_desc(p_base + (k >> 2) * (ROWS * 128) + (k & 3) * 32, 16, 1024, 2),
-                           smem_desc(v_base + C::TILE_BYTES + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ),
-                           idO, 1);
+                  mma_bf16_ts(tO, tP + k * 8,
+                              smem_desc(v_base + C::TILE_BYTES + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO,
+                              1);
               }
               mma_commit(&p_free[t]);
             }
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float sl2 = DEC ? da.scale_log2 : ea.scale_log2;
     const uint32_t tS = tmem + lane_off + s_col(t);
     const uint32_t tO = tmem + lane_off + o_col<HD>(t);
-    uint8_t* pb = smem + L::P + t * C::P_BYTES;
+    const uint32_t tP = tmem + lane_off + p_col<HD>(t);
     const bool split = DEC && da.n_split > 1;
     int cb = 0, qn = 0;
     bool ok = true;
@@ -442,28 +442,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m_ref, -m_ref);
+        // P as bf16 pairs (keys 2c, 2c+1 in column c) into the tile's P columns of TMEM
 #pragma unroll
-        for (int u = 0; u < KB / 8; ++u) {
-          float p[8];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const float2 x = ffma2(make_float2(s[8 * u + e], s[8 * u + e + 1]), scale2, neg_m2);
-            p[e] = exp2_approx(x.x);
-            p[e + 1] = exp2_approx(x.y);
-            sum2[(e >> 1) & 1] = fadd2(sum2[(e >> 1) & 1], make_float2(p[e], p[e + 1]));
+          for (int c = 0; c < 32; ++c) {
+            const int e = 64 * half + 2 * c;
+            const float2 x = ffma2(make_float2(s[e], s[e + 1]), scale2, neg_m2);
+            const float p0 = exp2_approx(x.x), p1 = exp2_approx(x.y);
+            sum2[c & 1] = fadd2(sum2[c & 1], make_float2(p0, p1));
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
+            pk[c] = *reinterpret_cast<uint32_t*>(&t2);
           }
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 t2 = __floats2bfloat162_rn(p[2 * e], p[2 * e + 1]);
-            pk[e] = *reinterpret_cast<uint32_t*>(&t2);
-          }
-          const int chunk = u >> 3, uu = u & 7;
-          *reinterpret_cast<uint4*>(pb + chunk * (ROWS * 128) + r * 128 + ((uu ^ (r & 7)) * 16)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          tmem_st32_async(tP + 32 * half, pk);
         }
         l_run += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
-        fence_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[t]);
       }
