@@ -21,6 +21,7 @@ oracle alone as the reference arm.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import dataclasses
 import json
 import math
@@ -43,11 +44,50 @@ UNIT = "candidate scores/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TENSOR_KERNELS = ("gemm", "enc_attn", "dec_attn")
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# workload's dominant kernel from one ncu capture, with a digest of the kernel
+# sources it was taken on: reported only while those sources are unchanged.
+CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "shared_prefix_behavior_b200", "csrc")
+KERNEL_SOURCES = {
+    "attn": ("sm100_attn.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
+    "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
+}
+TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
+    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (91858432, "attn", "3b4e606152946af1",
+                                                "profiles/attn_tc_kernel_bf16-32x1024-d256.md"),
+    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (260766464, "attn", "3b4e606152946af1",
+                                                    "profiles/attn_tc_kernel_bf16-8x4096-d512.md"),
+    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (291689728, "attn", "3b4e606152946af1",
+                                                   "profiles/attn_tc_kernel_bf16-2x16384-d512.md"),
+}
+
+
+def source_digest(kind: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kind]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """(bytes per launch or None, note)."""
+    t = TRAFFIC.get((kernel, workload))
+    if t is None:
+        return None, "no ncu capture of this kernel on this workload"
+    nbytes, kind, digest, src = t
+    try:
+        if source_digest(kind) != digest:
+            return None, "kernel sources changed since the capture in " + src
+    except OSError:
+        return None, "kernel sources not found"
+    return nbytes, "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch (" + src + ")"
+
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -88,7 +128,7 @@ def workload_config(w: W.Workload, n: int) -> dict:
 class ClockSampler:
     """nvidia-smi clock and throttle-reason samples during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -108,7 +148,12 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def mark(self):
+        """Call when the timed region starts: earlier samples are not counted."""
+        self.t_mark = time.time()
+
     def __exit__(self, *a):
+        self.t_end = time.time()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -122,17 +167,22 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        t0 = getattr(self, "t_mark", 0.0)
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
+                    whole, _, frac = parts[0].partition(".")
+                    ts = time.mktime(time.strptime(whole, "%Y/%m/%d %H:%M:%S")) + float("0." + (frac or "0"))
+                    if ts < t0:  # taken before the timed region
+                        continue
+                    sm.append(float(parts[2]))
+                    smax.append(float(parts[3]))
                 except ValueError:
                     continue
-                for nm, v in zip(names, parts[5:9]):
+                for nm, v in zip(names, parts[6:10]):
                     if v.lower() == "active":
                         reasons.add(nm)
         os.unlink(self.path)
@@ -271,6 +321,7 @@ def main():
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize()
+        clk.mark()
         e0.record(stream)
         for _ in range(args.steps):
             step()
@@ -381,6 +432,7 @@ def main():
         achieved = top["bytes"] / top["launches"] / per_launch_s / 1e9
         peak = float(peaks["hbm_gbs"])
         peak_note = f"HBM copy ({peak_src})"
+    traffic, traffic_note = traffic_for(top["name"], w.name)
     kernels = []
     for s in sorted(stats, key=lambda s: -s["ms"]):
         sec = s["ms"] * 1e-3
@@ -395,7 +447,9 @@ def main():
         "config": workload_config(w, world),
         "encoder_tokens_per_s": tokens / (ms_step * 1e-3),
         "roofline": {"kernel": top["name"], "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "peak_source": peak_note, "traffic": None,
+                     "frac": achieved / peak, "peak_source": peak_note, "traffic": traffic,
+                     "traffic_note": traffic_note,
+                     "algorithmic_bytes_per_launch": top["bytes"] / top["launches"],
                      "share_of_step": top["ms"] / total_ms},
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": UNIT,

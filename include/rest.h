@@ -20,8 +20,9 @@
  *     the legacy default stream). Host-detectable errors are returned
  *     synchronously before anything is enqueued. Errors found on the device
  *     (decreasing timestamps, a bounded wait that ran out) are written to the
- *     int32 word `*dev_err` (dev, may be NULL to ignore them); the caller
- *     zeroes it beforehand and reads it after synchronizing.
+ *     int32 word `*dev_err` (dev, may be NULL to ignore them). Each call
+ *     clears the word on `stream` before its first kernel, so after
+ *     synchronizing it holds this call's status (0 = no device error).
  *   - An empty batch (no tokens, or no candidates) is a successful no-op.
  *   - No C++ exception crosses this boundary.
  *   - REST_F32 computes with fp32 storage throughout. REST_BF16 takes bf16

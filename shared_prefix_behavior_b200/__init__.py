@@ -175,15 +175,29 @@ def _workspace(nbytes: int, device):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def _err_word(device):
+_ERR_WORDS = {}
+
+
+def _err_word(device, stream=None):
+    """The device status word for calls on (device, stream): one per pair, kept
+    for the process; every library call clears it on its stream before its
+    first kernel, so concurrent calls on different streams never share one."""
     import torch
-    return torch.zeros(1, dtype=torch.int32, device=device)
+    dev = torch.device(device)
+    if dev.index is None:
+        dev = torch.device(dev.type, torch.cuda.current_device())
+    key = (dev, _stream(stream))
+    w = _ERR_WORDS.get(key)
+    if w is None:
+        w = _ERR_WORDS[key] = torch.zeros(1, dtype=torch.int32, device=dev)
+    return w
 
 
 def check_device_error(err) -> None:
     """Synchronize and raise if a kernel reported an error in the status word."""
     code = int(err.item())
     if code != 0:
+        err.zero_()  # the word is kept for later calls: leave it clear even for one that enqueues nothing
         raise RestError(code, "device")
 
 
@@ -198,7 +212,7 @@ def rotation_table(ts, cu_seqlens, taus, head_dim: int, rope_base: float = 10000
     cos = torch.empty((T, H, head_dim // 2), dtype=torch.float32, device=dev)
     sin = torch.empty_like(cos)
     nb = workspace_size(REST_F32, taus, H * head_dim, cu_seqlens, rope_base=rope_base)
-    ws, err = _workspace(nb, dev), _err_word(dev)
+    ws, err = _workspace(nb, dev), _err_word(dev, stream)
     _check(_lib.rest_rotation_table(ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(ts), _ptr(idx), _ptr(cos),
                                     _ptr(sin), _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "rest_rotation_table")
     if check:
@@ -218,7 +232,7 @@ def encoder_attn(x, ts, cu_seqlens, taus, layers: Sequence[dict], l_switch: int,
         h_out = torch.empty_like(x)
     if ws is None:
         ws = _workspace(workspace_size(dt, taus, d, cu_seqlens, layers, rope_base=rope_base), dev)
-    err = _err_word(dev)
+    err = _err_word(dev, stream)
     _check(_lib.rest_encoder_attn(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(x), _ptr(ts), arr,
                                   len(layers), l_switch, _ptr(h_out), _ptr(ws), ws.numel(), _ptr(err),
                                   _stream(stream)), "rest_encoder_attn")
@@ -246,7 +260,7 @@ def cross_decode(hmem, cu_seqlens, taus, reqs, z, dec: dict, rope_base: float = 
         y_out = torch.empty(z.shape, dtype=torch.float32, device=dev)
     if ws is None:
         ws = _workspace(workspace_size(dt, taus, d, cu_seqlens, (), reqs, dp.K, rope_base), dev)
-    err = _err_word(dev)
+    err = _err_word(dev, stream)
     _check(_lib.rest_cross_decode(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(hmem), ctypes.byref(h.reqs),
                                   _ptr(z), ctypes.byref(dp), _ptr(y_out), _ptr(ws), ws.numel(), _ptr(err),
                                   _stream(stream)), "rest_cross_decode")
@@ -273,7 +287,7 @@ def cross_decode_static_ws(hmem, cu_seqlens, taus, reqs, z, dec: dict, rope_base
     dp = _dec(dec)
     if y_out is None:
         y_out = torch.empty(z.shape, dtype=torch.float32, device=dev)
-    err = _err_word(dev)
+    err = _err_word(dev, stream)
     _check(_lib.rest_cross_decode_static_ws(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(hmem),
                                             ctypes.byref(h.reqs), _ptr(z), ctypes.byref(dp), _ptr(y_out), _ptr(err),
                                             _stream(stream)), "rest_cross_decode_static_ws")
@@ -297,7 +311,7 @@ def rank_request(x, ts, cu_seqlens, taus, layers: Sequence[dict], l_switch: int,
         y_out = torch.empty(z.shape, dtype=torch.float32, device=dev)
     if ws is None:
         ws = _workspace(workspace_size(dt, taus, d, cu_seqlens, layers, reqs, dp.K, rope_base), dev)
-    err = _err_word(dev)
+    err = _err_word(dev, stream)
     _check(_lib.rest_rank_request(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(x), _ptr(ts), arr,
                                   len(layers), l_switch, ctypes.byref(h.reqs), _ptr(z), ctypes.byref(dp), _ptr(h_out),
                                   _ptr(y_out), _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "rest_rank_request")

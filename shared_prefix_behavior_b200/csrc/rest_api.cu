@@ -403,6 +403,8 @@ static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
   if (!p.dec_sched2.empty())
     memcpy(host.data() + p.L.dec_sched2, p.dec_sched2.data(), sizeof(int) * p.dec_sched2.size());
   if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) return REST_ERR_CUDA;
+  // the status word reports this call only
+  if (p.err && cudaMemsetAsync(p.err, 0, sizeof(int32_t), s) != cudaSuccess) return REST_ERR_CUDA;
   return REST_OK;
 }
 
