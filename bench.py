@@ -93,6 +93,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sharing", action="store_true",
+                    help="also run the no-sharing variant (every candidate re-encodes its own history)")
     return ap.parse_args()
 
 
@@ -126,68 +128,219 @@ def workload_config(w: W.Workload, n: int) -> dict:
 # --------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clock and throttle-reason samples during the timed region."""
+    """SM clock and clock-event reasons during the timed region: NVML read every
+    10 ms from a host thread (read-only queries), or nvidia-smi every 200 ms when
+    NVML is not available. Only samples taken after mark() count."""
 
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ((0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x20, "sw_thermal_slowdown"),
+               (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"))
 
     def __init__(self, gpu_index: int):
-        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
         self.gpu = gpu_index
-        self.proc = None
-
-    def __enter__(self):
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except Exception:
-            self.proc = None
-        return self
+        self.samples = []
+        self.t_mark = 0.0
+        self.source = None
 
     def mark(self):
         """Call when the timed region starts: earlier samples are not counted."""
         self.t_mark = time.time()
 
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, h):
+        import pynvml
+        while not self.stop.is_set():
+            try:
+                clk = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.time(), float(clk), float(mx), int(rs)))
+            except Exception:
+                pass
+            self.stop.wait(0.01)
+
+    def __enter__(self):
+        import threading
+        self.stop = threading.Event()
+        try:
+            h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll, args=(h,), daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+        except Exception:
+            self.thread = None
+            self._smi_start()
+        return self
+
+    def _smi_start(self):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=timestamp,clocks.sm,"
+                                          "clocks.max.sm,clocks_event_reasons.active", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 200 ms"
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
     def __exit__(self, *a):
         self.t_end = time.time()
-        if self.proc is not None:
+        self.stop.set()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        elif getattr(self, "proc", None) is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
             self.f.close()
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    try:
+                        whole, _, frac = parts[0].partition(".")
+                        ts = time.mktime(time.strptime(whole, "%Y/%m/%d %H:%M:%S")) + float("0." + (frac or "0"))
+                        self.samples.append((ts, float(parts[1]), float(parts[2]), int(parts[3], 16)))
+                    except (ValueError, IndexError):
+                        continue
+            os.unlink(self.path)
 
     def summary(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        t0 = getattr(self, "t_mark", 0.0)
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 10:
-                    continue
-                try:
-                    whole, _, frac = parts[0].partition(".")
-                    ts = time.mktime(time.strptime(whole, "%Y/%m/%d %H:%M:%S")) + float("0." + (frac or "0"))
-                    if ts < t0:  # taken before the timed region
-                        continue
-                    sm.append(float(parts[2]))
-                    smax.append(float(parts[3]))
-                except ValueError:
-                    continue
-                for nm, v in zip(names, parts[6:10]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [s for s in self.samples if self.t_mark <= s[0] <= getattr(self, "t_end", float("inf"))]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = sorted({nm for s in inside for bit, nm in self.REASONS if s[3] & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": max(s[2] for s in inside),
+                "sm_mhz_min": min(s[1] for s in inside), "reasons": reasons, "samples": len(inside),
+                "source": self.source}
+
+
+# --------------------------------------------------------------------- the two halves on their own
+
+def peaks_for_parts():
+    peaks, src = load_peaks()
+    return float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))), float(peaks["hbm_gbs"]), src
+
+
+def component_timings(args, w, t, H, Y, ws, dev, peaks):
+    """Encoder alone (rest_encoder_attn) and the decoder alone (rest_cross_decode),
+    the latter with L2 flushed before every call (a 256 MB write), so that the
+    shared prefix H is read from HBM as it would be when it is not resident."""
+    import torch
+    import shared_prefix_behavior_b200 as R
+    tensor_peak, hbm_peak, src = peaks
+    n = max(3, min(args.steps, 50))
+
+    def enc():
+        R.encoder_attn(t["x"], t["ts"], t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"],
+                       rope_base=t["rope_base"], h_out=H, ws=ws, check=False)
+
+    def dec():
+        R.cross_decode(H, t["cu_seqlens"], t["taus"], t["reqs"], t["z"], t["dec"], t["rope_base"], y_out=Y, ws=ws,
+                       check=False)
+
+    for _ in range(3):
+        enc()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        enc()
+    b.record()
+    torch.cuda.synchronize()
+    enc_ms = a.elapsed_time(b) / n
+    enc_part = {"tokens_per_s": w.total_tokens / (enc_ms * 1e-3), "ms": enc_ms, "calls": n, "l2": "not flushed"}
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for _ in range(3):
+        dec()
+    R.profile_begin()
+    for i in range(n):
+        flush.fill_(i & 0xff)
+        evs[i][0].record()
+        dec()
+        evs[i][1].record()
+    stats = R.profile_end()
+    torch.cuda.synchronize()
+    dec_ms = sum(x.elapsed_time(y) for x, y in evs) / n
+    attn = [s_ for s_ in stats if s_["name"] == "dec_attn"]
+    d, K = w.d, w.K
+    flops = sum(4.0 * d * K * nr * c for nr, c in zip(w.req_ncand, w.req_cutoff))
+    # algorithmic bytes of the attention: every H prefix once per request, q and g in (fp32), o * g out (4 B)
+    nk = K * w.total_cands
+    h_bytes = sum(2.0 * c * d for c in w.req_cutoff)
+    abytes = h_bytes + 12.0 * nk * d
+    dec_part = {"candidate_scores_per_s": w.total_cands / (dec_ms * 1e-3), "ms": dec_ms, "calls": n,
+                "l2": "flushed before every call (256 MB write)"}
+    if attn:
+        t_attn = attn[0]["ms"] / n * 1e-3  # seconds of decoder attention per call (all its launches)
+        t_roof = max(flops / (tensor_peak * 1e12), abytes / (hbm_peak * 1e9))
+        dec_part["attention"] = {
+            "ms": t_attn * 1e3, "tflops": flops / t_attn / 1e12, "algorithmic_flops": flops,
+            "algorithmic_bytes": abytes, "roofline_ms": t_roof * 1e3, "roofline_frac": t_roof / t_attn,
+            "roofline": f"max(FLOPs / sustained bf16 peak, bytes / HBM copy bandwidth), measured peaks ({src})"}
+    return {"encoder_only": enc_part, "decoder_only": dec_part}
+
+
+def sharing_comparison(w, inp, dev, ms_shared):
+    """The same candidates without the shared prefix: every candidate becomes a
+    user of its own whose history is its request's prefix, encoded and decoded
+    alone (what the decoder's sharing avoids). Run on whole users of the batch,
+    as many as keep the re-encoded tokens near 1M, and compared per candidate."""
+    import torch
+    import shared_prefix_behavior_b200 as R
+    cu = np.asarray(inp["cu_seqlens"])
+    ru, rc, cc = (np.asarray(inp[k]) for k in ("req_user", "req_cutoff", "cu_cands"))
+    users, tok = [], 0
+    for u in range(len(cu) - 1):
+        need = sum(int(rc[r]) * int(cc[r + 1] - cc[r]) for r in range(len(ru)) if ru[r] == u)
+        if users and tok + need > (1 << 20):
+            break
+        users.append(u)
+        tok += need
+    rows, ts_rows, z_rows, lens = [], [], [], []
+    for r in range(len(ru)):
+        if ru[r] not in users:
+            continue
+        s0 = int(cu[ru[r]])
+        for c in range(int(cc[r]), int(cc[r + 1])):
+            rows.append(np.arange(s0, s0 + int(rc[r])))
+            z_rows.append(c)
+            lens.append(int(rc[r]))
+    rows = np.concatenate(rows)
+    n = len(lens)
+    ns = dict(inp, x=inp["x"][rows], ts=inp["ts"][rows],
+              cu_seqlens=np.concatenate([[0], np.cumsum(lens)]).astype(np.int32),
+              req_user=np.arange(n, dtype=np.int32), req_cutoff=np.asarray(lens, dtype=np.int32),
+              cu_cands=np.arange(n + 1, dtype=np.int32), z=inp["z"][np.asarray(z_rows)])
+    t = R.to_device(ns, dev)
+    args_rank = (t["x"], t["ts"], t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"], t["z"],
+                 t["dec"], t["rope_base"])
+    R.rank_request(*args_rank, check=True)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(3):
+        R.rank_request(*args_rank, check=False)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / 3
+    shared_per_cand = ms_shared / w.total_cands
+    alone_per_cand = ms / n
+    return {"users": len(users), "candidates": n, "reencoded_tokens": int(len(rows)), "ms": ms,
+            "ms_per_candidate_alone": alone_per_cand, "ms_per_candidate_shared": shared_per_cand,
+            "speedup_of_sharing": alone_per_cand / shared_per_cand}
 
 
 # --------------------------------------------------------------------- oracle (CPU baseline / reference arm)
@@ -412,6 +565,10 @@ def main():
         e2e_ms = float(tm.item())
     e2e_value = cands / (e2e_ms / args.steps * 1e-3)
 
+    parts = component_timings(args, w, t, H, Y, ws, dev, peaks_for_parts())
+    if args.sharing and world == 1:
+        parts["sharing"] = sharing_comparison(w, inp, dev, ms_step)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -460,7 +617,11 @@ def main():
                            "copy stream while step i computes"},
         "gpu_launches": launches,
         "clocks": clk.summary(),
+        "encoder_only": parts["encoder_only"],
+        "decoder_only": parts["decoder_only"],
     }
+    if "sharing" in parts:
+        out["sharing"] = parts["sharing"]
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_budget)
     print(json.dumps(out), flush=True)
