@@ -160,3 +160,22 @@ def cross_decode(Hmem, cu_seqlens, req_user, req_cutoff, cu_cands, z, dec, n_hea
                         o[sl] += p[j] * Hm[s + j, sl]
                 y[n, k] = matvec([o[i] * g[i] for i in range(d)], dec["w_o"])
     return y
+
+
+def score_head(z, y, sp):
+    """Decoder block and score, candidate by candidate and token by token:
+    a = z + y; u = LN_k(a); f = a + SwiGLU_k(u); score = f[token 0] . w_s + b_s."""
+    z = np.asarray(z, dtype=np.float64)
+    y = np.asarray(y, dtype=np.float64)
+    N, K, d = z.shape
+    f = np.zeros((N, K, d))
+    score = np.zeros(N)
+    for n in range(N):
+        for k in range(K):
+            a = [z[n, k, i] + y[n, k, i] for i in range(d)]
+            u = ln_row(a, sp["ln_g"][k], sp["ln_b"][k])
+            hid = ffn([u], {"w_ffn13": sp["w_ffn13"][k], "w_ffn2": sp["w_ffn2"][k]})[0]
+            for i in range(d):
+                f[n, k, i] = a[i] + hid[i]
+        score[n] = sum(f[n, 0, i] * float(sp["w_s"][i]) for i in range(d)) + float(sp["b_s"])
+    return f, score

@@ -326,6 +326,26 @@ def cross_decode(Hmem: np.ndarray, cu_seqlens: np.ndarray, req_user, req_cutoff,
     return (o * g) @ Wo
 
 
+def score_head(z: np.ndarray, y: np.ndarray, sp: dict):
+    """Decoder block and candidate score (§3.3.2 eq. 8, Fig. 1 right) -> (f, score).
+
+    Readings: the query token plus eq. 7's output, a = z + y; then a pre-LN
+    FFN sublayer whose LN and SwiGLU weights are specific to the token type
+    (eq. 8), f = a + SwiGLU_k(LN_k(a)); the score is a linear logit on token 0
+    ([CLS]): f[:, 0] . w_s + b_s.
+    """
+    z = _f64(z)
+    a = z + _f64(y)
+    N, K, d = a.shape
+    f = np.empty_like(a)
+    for k in range(K):
+        layer = {"w_ffn13": sp["w_ffn13"][k], "w_ffn2": sp["w_ffn2"][k]}
+        u = layer_norm(a[:, k], _f64(sp["ln_g"][k]), _f64(sp["ln_b"][k]))
+        f[:, k] = a[:, k] + ffn_sublayer(u, layer)
+    score = f[:, 0] @ _f64(sp["w_s"]) + float(sp["b_s"])
+    return f, score
+
+
 def rank_request(inp: dict, **kw):
     """Shared-prefix serving (§3.5): H = T(S_u) once, then C for every
     candidate of every request against it. Returns (H, y)."""

@@ -346,3 +346,57 @@ def test_row_sampled_encoder_equals_full_encoder(l_switch, ffn):
     full = O.encoder(inp)
     rows = [0, 5, 39, 40, 41, 62]
     assert rel_err(O.encoder_rows(inp, rows), full[rows]) < 1e-13
+
+
+# ------------------------------------------------------------ decoder block and score (eq. 8, R23-R25)
+
+def _score_case(seed=31, n=4, K=3, d=16, ln_affine=True):
+    w, inp = tiny_inputs(seed=seed, lengths=(9,), d=d, n_heads=4, n_layers=1, requests=[(0, 9, n)],
+                         ln_affine=ln_affine)
+    rng = np.random.default_rng(seed + 1)
+    y = rng.standard_normal(inp["z"].shape)
+    return inp["z"], y, inp["score"]
+
+
+def test_score_head_matches_brute_force():
+    z, y, sp = _score_case()
+    f, s = O.score_head(z, y, sp)
+    fb, sb = brute.score_head(z, y, sp)
+    assert rel_err(f, fb) < 1e-13 and rel_err(s, sb) < 1e-13
+
+
+def test_score_head_without_ffn_is_the_residual_sum():
+    """W_2 = 0 removes the FFN: f = z + y exactly and the score is its [CLS] logit."""
+    z, y, sp = _score_case(seed=32)
+    sp0 = dict(sp, w_ffn2=np.zeros_like(sp["w_ffn2"]))
+    f, s = O.score_head(z, y, sp0)
+    a = z.astype(np.float64) + y
+    assert np.array_equal(f, a)
+    assert rel_err(s, a[:, 0] @ sp["w_s"].astype(np.float64) + sp["b_s"]) < 1e-14
+
+
+def test_score_head_single_token_type_is_the_encoder_pre_ln_ffn_sublayer():
+    """With one token type the block's FFN is eq. 6's pre-LN sublayer with alpha = 1."""
+    z, y, sp = _score_case(seed=33)
+    sp1 = {k: (v[:1] if isinstance(v, np.ndarray) and v.ndim >= 2 else v) for k, v in sp.items()}
+    f, _ = O.score_head(z[:, :1], y[:, :1], sp1)
+    a = z[:, 0].astype(np.float64) + y[:, 0]
+    layer = {"w_ffn13": sp["w_ffn13"][0], "w_ffn2": sp["w_ffn2"][0]}
+    want = O.srn(a, lambda u: O.ffn_sublayer(u, layer), 1.0, False, sp["ln_g"][0], sp["ln_b"][0])
+    assert rel_err(f[:, 0], want) < 1e-14
+
+
+def test_score_head_token_types_use_only_their_own_parameters():
+    """Eq. 8: swapping the parameters of token types 1 and 2 together with their
+    input rows swaps their outputs; changing type 2's weights leaves types 0 and 1."""
+    z, y, sp = _score_case(seed=34)
+    f, s = O.score_head(z, y, sp)
+    perm = [0, 2, 1]
+    spp = {k: (v[perm] if isinstance(v, np.ndarray) and v.ndim >= 2 else v) for k, v in sp.items()}
+    fp, sp_score = O.score_head(z[:, perm], y[:, perm], spp)
+    assert rel_err(fp, f[:, perm]) < 1e-14 and rel_err(sp_score, s) < 1e-14
+    sp2 = dict(sp, w_ffn2=sp["w_ffn2"].copy())
+    sp2["w_ffn2"][2] *= -3.0
+    f2, s2 = O.score_head(z, y, sp2)
+    assert np.array_equal(f2[:, :2], f[:, :2]) and np.array_equal(s2, s)
+    assert not np.allclose(f2[:, 2], f[:, 2])

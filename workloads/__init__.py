@@ -263,6 +263,19 @@ def make_inputs(w: Workload, seed: int, ln_affine: bool = False) -> dict:
     cu_c = np.zeros(w.n_req + 1, dtype=np.int32)
     cu_c[1:] = np.cumsum(w.req_ncand)
     z = _store(rng.standard_normal((w.total_cands, w.K, d)), w.dtype)
+    # decoder block FFN and score readout: drawn after every array above, which stay as they were
+    dff = ffn_width(d)
+    score = {
+        "w_ffn13": _store(rng.standard_normal((w.K, d, 2 * dff)) * sd, w.dtype),
+        "w_ffn2": _store(rng.standard_normal((w.K, dff, d)) * sd, w.dtype),
+        "ln_g": np.ones((w.K, d), dtype=np.float32),
+        "ln_b": np.zeros((w.K, d), dtype=np.float32),
+        "w_s": (rng.standard_normal(d) * sd).astype(np.float32),
+        "b_s": 0.25,
+    }
+    if ln_affine:
+        score["ln_g"] = (1.0 + 0.2 * rng.standard_normal((w.K, d))).astype(np.float32)
+        score["ln_b"] = (0.1 * rng.standard_normal((w.K, d))).astype(np.float32)
     return {
         "x": _store(x, w.dtype),
         "ts": ts,
@@ -271,6 +284,7 @@ def make_inputs(w: Workload, seed: int, ln_affine: bool = False) -> dict:
         "layers": layers,
         "l_switch": w.l_switch,
         "dec": dec,
+        "score": score,
         "z": z,
         "req_user": np.asarray(w.req_user, dtype=np.int32),
         "req_cutoff": np.asarray(w.req_cutoff, dtype=np.int32),
