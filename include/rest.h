@@ -205,6 +205,40 @@ rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest
                               void* h_out, float* y_out,
                               void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
+/* Decoder block and candidate score ("From Language to Behavior", §3.3.2
+ * eq. 8 and Fig. 1 right; the wiring the page leaves open is fixed as: a
+ * residual on the query token, a pre-LN feed-forward sublayer whose LN and
+ * SwiGLU weights are specific to the token type, and a linear logit on
+ * token 0, [CLS]). For candidate n and token k:
+ *   a = z[n,k] + y[n,k];  u = LN_k(a);
+ *   f[n,k] = a + (SiLU(u W_1^(k)) * (u W_3^(k))) W_2^(k);
+ *   score[n] = f[n,0] . w_s + b_s.
+ * All weights are device memory: w_ffn13 [K, d, 2 d_ff] in the call's dtype
+ * (W_1^(k) in the first d_ff columns of block k, W_3^(k) after), w_ffn2
+ * [K, d_ff, d] in the call's dtype, ln_g and ln_b fp32 [K, d], w_s fp32 [d]. */
+typedef struct {
+  const void* w_ffn13;
+  const void* w_ffn2;
+  const float* ln_g;
+  const float* ln_b;
+  const float* w_s;
+  float b_s;
+  int d_ff;            /* > 0, a multiple of 8 */
+} rest_score_params;
+
+/* Workspace bytes rest_score_head needs for n_cands candidates of K tokens. */
+rest_status rest_score_workspace_size(rest_dtype dt, int d, int K, long long n_cands, int d_ff, size_t* bytes);
+
+/* z: dev [n_cands, K, d] in the call's dtype (the decoder's query tokens);
+ * y: dev fp32 [n_cands, K, d] (rest_cross_decode's or rest_rank_request's
+ * y_out); f_out: dev fp32 [n_cands, K, d] receives f (it also holds a while
+ * the block runs); score_out: dev fp32 [n_cands]. d is a multiple of 8 and at
+ * most 1024, 1 <= K <= 8. Errors as for the other calls; an empty batch is a
+ * no-op. */
+rest_status rest_score_head(rest_dtype dt, int d, int K, long long n_cands, const void* z, const float* y,
+                            const rest_score_params* sp, float* f_out, float* score_out,
+                            void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
 /* Static description of a status code. */
 const char* rest_status_string(rest_status s);
 

@@ -28,7 +28,7 @@ STATUS = {0: "REST_OK", 1: "REST_ERR_INVALID_ARG", 2: "REST_ERR_UNSORTED_TIME", 
           4: "REST_ERR_CUDA", 5: "REST_ERR_TIMEOUT", 6: "REST_ERR_WORKSPACE", 7: "REST_ERR_NO_DEVICE"}
 EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
            "rest_rank_request", "rest_status_string", "rest_launch_count", "rest_profile_begin",
-           "rest_profile_end", "rest_cross_decode_static_ws")
+           "rest_profile_end", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head")
 STATIC_WS_BYTES = 32 * 1024 * 1024  # REST_STATIC_WS_BYTES
 
 
@@ -57,6 +57,11 @@ class DecParams(ctypes.Structure):
     _fields_ = [("K", c_int), ("w_q", c_void_p), ("w_go", c_void_p), ("w_o", c_void_p)]
 
 
+class ScoreParams(ctypes.Structure):
+    _fields_ = [("w_ffn13", c_void_p), ("w_ffn2", c_void_p), ("ln_g", c_void_p), ("ln_b", c_void_p),
+                ("w_s", c_void_p), ("b_s", c_float), ("d_ff", c_int)]
+
+
 class Requests(ctypes.Structure):
     _fields_ = [("n_req", c_int), ("req_user", POINTER(c_int32)), ("req_cutoff", POINTER(c_int32)),
                 ("cu_cands", POINTER(c_int32))]
@@ -83,8 +88,11 @@ def _load() -> ctypes.CDLL:
                                                 POINTER(DecParams), P, P, P]
     lib.rest_rank_request.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, POINTER(EncLayer), c_int, c_int,
                                       POINTER(Requests), P, POINTER(DecParams), P, P, P, c_size_t, P, P]
+    lib.rest_score_workspace_size.argtypes = [c_int, c_int, c_int, c_longlong, c_int, POINTER(c_size_t)]
+    lib.rest_score_head.argtypes = [c_int, c_int, c_int, c_longlong, P, P, POINTER(ScoreParams), P, P, P, c_size_t,
+                                    P, P]
     for name in ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
-                 "rest_rank_request", "rest_cross_decode_static_ws"):
+                 "rest_rank_request", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head"):
         getattr(lib, name).restype = c_int
     lib.rest_status_string.argtypes = [c_int]
     lib.rest_status_string.restype = ctypes.c_char_p
@@ -338,6 +346,36 @@ def profile_end() -> List[dict]:
              "bytes": buf[i].bytes} for i in range(min(n, 64))]
 
 
+def score_workspace_size(dtype: int, d: int, K: int, n_cands: int, d_ff: int) -> int:
+    out = c_size_t(0)
+    _check(_lib.rest_score_workspace_size(dtype, d, K, n_cands, d_ff, ctypes.byref(out)), "rest_score_workspace_size")
+    return out.value
+
+
+def score_head(z, y, sp: dict, f_out=None, score_out=None, ws=None, stream=None, check=True):
+    """Decoder block and candidate score (ReST §3.3.2 eq. 8): returns (f [N, K, d]
+    fp32, score [N] fp32) from the query tokens z and the decoder output y."""
+    import torch
+    dev = z.device
+    N, K, d = z.shape
+    dt = _dtype_code(z)
+    d_ff = int(sp["w_ffn2"].shape[1])
+    if f_out is None:
+        f_out = torch.empty((N, K, d), dtype=torch.float32, device=dev)
+    if score_out is None:
+        score_out = torch.empty((N,), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(score_workspace_size(dt, d, K, N, d_ff), dev)
+    params = ScoreParams(_ptr(sp["w_ffn13"]), _ptr(sp["w_ffn2"]), _ptr(sp["ln_g"]), _ptr(sp["ln_b"]),
+                         _ptr(sp["w_s"]), float(sp["b_s"]), d_ff)
+    err = _err_word(dev, stream)
+    _check(_lib.rest_score_head(dt, d, K, N, _ptr(z), _ptr(y), ctypes.byref(params), _ptr(f_out), _ptr(score_out),
+                                _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "rest_score_head")
+    if check:
+        check_device_error(err)
+    return f_out, score_out
+
+
 def to_device(inp: dict, device) -> dict:
     """Move one batch of host inputs (numpy) to device tensors of the batch's dtype."""
     import torch
@@ -356,6 +394,9 @@ def to_device(inp: dict, device) -> dict:
     return {
         "x": dev(inp["x"]), "ts": dev(inp["ts"], torch.int64), "z": dev(inp["z"]),
         "dec": {k: dev(v) for k, v in inp["dec"].items()}, "layers": layers,
+        "score": ({"w_ffn13": dev(inp["score"]["w_ffn13"]), "w_ffn2": dev(inp["score"]["w_ffn2"]),
+                   **{k: dev(inp["score"][k], torch.float32) for k in ("ln_g", "ln_b", "w_s")},
+                   "b_s": float(inp["score"]["b_s"])} if "score" in inp else None),
         "cu_seqlens": np.asarray(inp["cu_seqlens"], dtype=np.int32), "taus": np.asarray(inp["taus"]),
         "l_switch": int(inp["l_switch"]), "rope_base": float(inp["rope_base"]),
         "reqs": (np.asarray(inp["req_user"], np.int32), np.asarray(inp["req_cutoff"], np.int32),

@@ -28,6 +28,14 @@ cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_us
 // mode 4: x = LN(x); y = dt(LN2(x))  (post-LN, then the next sublayer's pre-LN with g2, b2)
 cudaError_t launch_layernorm(bool bf16, float* x, void* y, const float* g, const float* b, int T, int d,
                              int mode, cudaStream_t s, const float* g2 = nullptr, const float* b2 = nullptr);
+// Decoder block input: a = z + y (fp32, into f) and u = dt(LN_k(a)) with the
+// parameters of token type k = row % K (ln_g, ln_b are [K, d]); in bf16 with
+// u_lo also the low part, u_lo = bf16(LN_k(a) - u). One warp per row.
+cudaError_t launch_score_ln(bool bf16, const void* z, const float* y, float* f, void* u, void* u_lo,
+                            const float* ln_g, const float* ln_b, long long rows, int d, int K, cudaStream_t s);
+// score[n] = f[n, 0, :] . w_s + b_s; one warp per candidate.
+cudaError_t launch_score_readout(const float* f, const float* w_s, float b_s, float* score, long long n, int d, int K,
+                                 cudaStream_t s);
 // x_res = float(x_in)
 cudaError_t launch_to_f32(bool bf16, const void* x_in, float* x_res, long long n, cudaStream_t s);
 // hi = bf16(x), lo = bf16(x - hi): x as an unevaluated sum of two bf16 numbers
@@ -40,7 +48,8 @@ enum Epilogue {
   EPI_SIGMOID = 2,  // out0[m, n] = sigmoid(acc) (fp32)
   EPI_RESID = 3,    // out0[m, n] += alpha * acc (fp32 residual stream)
   EPI_QKVG = 4,     // the DGA projection epilogue (rotation, value gate, output gate)
-  EPI_SWIGLU = 5,   // out0[m, j] = dt(SiLU(acc_1) * acc_3)
+  EPI_SWIGLU = 5,   // out0[m, j] = dt(SiLU(acc_1) * acc_3); with out1 (bf16) also its low part,
+                    // out1 = bf16(value - out0)
   EPI_DECQG = 6     // decoder token-specific projections, all token types in one launch:
                     // q[n, k] = z[n, k] W_Q^(k) -> out0, sigmoid(z[n, k] W_go^(k)) -> out1
 };

@@ -851,6 +851,99 @@ rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest
   }
 }
 
+// ---------------------------------------------------------------- decoder block and score
+
+// Workspace of the score head: the LN output u and the SwiGLU hidden state,
+// each with a low part in bf16 (u = u + u_lo, hid = hid + hid_lo feed the
+// tensor-core products at fp32-level precision: the block has no residual
+// scale to damp their rounding).
+struct ScoreLayout {
+  size_t u, u_lo, hid, hid_lo, total;
+};
+
+static rest_status score_layout(rest_dtype dt, int d, int K, long long n, int d_ff, ScoreLayout* L) {
+  if ((dt != REST_F32 && dt != REST_BF16) || d <= 0 || d > 1024 || d % 8 || K < 1 || K > 8 || n < 0 ||
+      d_ff <= 0 || d_ff % 8)
+    return REST_ERR_INVALID_ARG;
+  const size_t e = dt_size(dt), rows = (size_t)n * K;
+  const size_t ub = align_up(rows * d * e, 256), hb = align_up(rows * (size_t)d_ff * e, 256);
+  const bool lo = dt == REST_BF16;
+  L->u = 0;
+  L->u_lo = ub;
+  L->hid = L->u_lo + (lo ? ub : 0);
+  L->hid_lo = L->hid + hb;
+  L->total = L->hid_lo + (lo ? hb : 0);
+  if (L->total == 0) L->total = 256;
+  return REST_OK;
+}
+
+rest_status rest_score_workspace_size(rest_dtype dt, int d, int K, long long n_cands, int d_ff, size_t* bytes) {
+  if (!bytes) return REST_ERR_INVALID_ARG;
+  ScoreLayout L;
+  rest_status st = score_layout(dt, d, K, n_cands, d_ff, &L);
+  if (st == REST_OK) *bytes = L.total;
+  return st;
+}
+
+rest_status rest_score_head(rest_dtype dt, int d, int K, long long n_cands, const void* z, const float* y,
+                            const rest_score_params* sp, float* f_out, float* score_out, void* ws, size_t ws_bytes,
+                            int32_t* dev_err, void* stream) {
+  try {
+    if (!sp) return REST_ERR_INVALID_ARG;
+    ScoreLayout SL;
+    rest_status st = score_layout(dt, d, K, n_cands, sp->d_ff, &SL);
+    const size_t total = SL.total;
+    if (st != REST_OK) return st;
+    if (n_cands == 0) return REST_OK;
+    if (!z || !y || !f_out || !score_out || !sp->w_ffn13 || !sp->w_ffn2 || !sp->ln_g || !sp->ln_b || !sp->w_s ||
+        !aligned16(z) || !aligned16(y) || !aligned16(f_out) || !aligned16(sp->w_ffn13) || !aligned16(sp->w_ffn2))
+      return REST_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < total || !aligned16(ws)) return REST_ERR_WORKSPACE;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dev_err && cudaMemsetAsync(dev_err, 0, sizeof(int32_t), s) != cudaSuccess) return REST_ERR_CUDA;
+    Plan p;
+    p.dt = dt;
+    p.err = dev_err;
+    const bool bf = dt == REST_BF16;
+    const size_t e = dt_size(dt);
+    const long long rows = n_cands * K;
+    const int dff = sp->d_ff;
+    char* u = at<char>(ws, SL.u);
+    char* u_lo = bf ? at<char>(ws, SL.u_lo) : nullptr;
+    char* hid = at<char>(ws, SL.hid);
+    char* hid_lo = bf ? at<char>(ws, SL.hid_lo) : nullptr;
+    // a = z + y (the query token's residual, fp32 in f_out) and u = LN_k(a)
+    REST_KLAUNCH(s, "score_ln", 0, (double)rows * d * (e + 4 + 4 + 2 * e),
+                 launch_score_ln(bf, z, y, f_out, u, u_lo, sp->ln_g, sp->ln_b, rows, d, K, s));
+    // token type k: rows n K + k of u, f_out and the hidden state, with that type's weights (eq. 8)
+    for (int k = 0; k < K; ++k) {
+      GemmArgs a = gemm(u + e * (size_t)k * d, (long long)K * d,
+                        (const char*)sp->w_ffn13 + e * (size_t)k * d * 2 * dff, 2LL * dff, n_cands, 2 * dff, d,
+                        EPI_SWIGLU, hid + e * (size_t)k * dff, (long long)K * dff);
+      a.d = dff;
+      if (bf) {
+        a.A2 = u_lo + e * (size_t)k * d;
+        a.out1 = hid_lo + e * (size_t)k * dff;
+      }
+      if ((st = run_gemm(p, a, "gemm_score_ffn13", s)) != REST_OK) return st;
+    }
+    for (int k = 0; k < K; ++k) {
+      GemmArgs a = gemm(hid + e * (size_t)k * dff, (long long)K * dff,
+                        (const char*)sp->w_ffn2 + e * (size_t)k * dff * d, d, n_cands, d, dff, EPI_RESID,
+                        f_out + (size_t)k * d, (long long)K * d);
+      a.alpha = 1.0f;
+      if (bf) a.A2 = hid_lo + e * (size_t)k * dff;
+      if ((st = run_gemm(p, a, "gemm_score_ffn2", s)) != REST_OK) return st;
+    }
+    REST_KLAUNCH(s, "score_readout", 2.0 * n_cands * d, (double)n_cands * d * 4,
+                 launch_score_readout(f_out, sp->w_s, sp->b_s, score_out, n_cands, d, K, s));
+    return REST_OK;
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------- decoder without a caller workspace

@@ -309,6 +309,95 @@ cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, cons
   return cudaGetLastError();
 }
 
+// ============================================================================
+// Decoder block and candidate score (ReST §3.3.2 eq. 8, Fig. 1 right)
+// ============================================================================
+
+// a = z + y into f; u = dt(LN_k(a)) with token type k = row % K. One warp per
+// row of d <= 1024 columns (lane holds columns lane, lane + 32, ...).
+template <typename T>
+__global__ void score_ln_kernel(const T* __restrict__ z, const float* __restrict__ y, float* __restrict__ f,
+                                T* __restrict__ u, T* __restrict__ u_lo, const float* __restrict__ ln_g,
+                                const float* __restrict__ ln_b, long long rows, int d, int K) {
+  constexpr int VMAX = 32;
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int k = (int)(row % K);
+  const long long o = row * d;
+  float v[VMAX];
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < VMAX; ++i) {
+    const int c = i * 32 + lane;
+    v[i] = c < d ? to_f<T>(z[o + c]) + y[o + c] : 0.f;
+    if (c < d) f[o + c] = v[i];
+    sum += v[i];
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+  const float mean = sum / d;
+  float sq = 0.f;
+#pragma unroll
+  for (int i = 0; i < VMAX; ++i) {
+    const float t = i * 32 + lane < d ? v[i] - mean : 0.f;
+    sq += t * t;
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, m);
+  const float rstd = 1.0f / sqrtf(sq / d + 1e-5f);
+  const float* g = ln_g + (long long)k * d;
+  const float* b = ln_b + (long long)k * d;
+#pragma unroll
+  for (int i = 0; i < VMAX; ++i) {
+    const int c = i * 32 + lane;
+    if (c < d) {
+      const float n = (v[i] - mean) * rstd * g[c] + b[c];
+      const T hi = from_f<T>(n);
+      u[o + c] = hi;
+      if (u_lo) u_lo[o + c] = from_f<T>(n - to_f<T>(hi));
+    }
+  }
+}
+
+cudaError_t launch_score_ln(bool bf16m, const void* z, const float* y, float* f, void* u, void* u_lo,
+                            const float* ln_g, const float* ln_b, long long rows, int d, int K, cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  if (d > 1024 || K < 1) return cudaErrorInvalidValue;
+  const int threads = 256;
+  const long long blocks = (rows * 32 + threads - 1) / threads;
+  if (bf16m)
+    score_ln_kernel<bf16><<<(unsigned)blocks, threads, 0, s>>>((const bf16*)z, y, f, (bf16*)u, (bf16*)u_lo, ln_g,
+                                                                ln_b, rows, d, K);
+  else
+    score_ln_kernel<float><<<(unsigned)blocks, threads, 0, s>>>((const float*)z, y, f, (float*)u, nullptr, ln_g,
+                                                                 ln_b, rows, d, K);
+  return cudaGetLastError();
+}
+
+// score[n] = f[n, 0, :] . w_s + b_s (token 0 is [CLS]); one warp per candidate.
+__global__ void score_readout_kernel(const float* __restrict__ f, const float* __restrict__ w_s, float b_s,
+                                     float* __restrict__ score, long long n, int d, int K) {
+  const long long c = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (c >= n) return;
+  const float* row = f + c * K * d;
+  float acc = 0.f;
+  for (int i = lane; i < d; i += 32) acc = fmaf(row[i], w_s[i], acc);
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (lane == 0) score[c] = acc + b_s;
+}
+
+cudaError_t launch_score_readout(const float* f, const float* w_s, float b_s, float* score, long long n, int d, int K,
+                                 cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  const long long blocks = (n * 32 + threads - 1) / threads;
+  score_readout_kernel<<<(unsigned)blocks, threads, 0, s>>>(f, w_s, b_s, score, n, d, K);
+  return cudaGetLastError();
+}
+
 template <typename T>
 __global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, long long n) {
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -489,7 +578,10 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
       }
       case EPI_SWIGLU: {
         int col = (n >> 2) * 2;
-        store2((T*)a.out0 + ro + col, c[0] * sigmoid_f(c[0]) * c[2], c[1] * sigmoid_f(c[1]) * c[3]);
+        const float h0 = c[0] * sigmoid_f(c[0]) * c[2], h1 = c[1] * sigmoid_f(c[1]) * c[3];
+        store2((T*)a.out0 + ro + col, h0, h1);
+        if (a.out1)  // the low part of a bf16 hi + lo pair
+          store2((T*)a.out1 + ro + col, h0 - to_f<T>(from_f<T>(h0)), h1 - to_f<T>(from_f<T>(h1)));
         break;
       }
     }

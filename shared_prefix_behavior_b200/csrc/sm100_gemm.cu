@@ -197,7 +197,9 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     // V' = sigmoid(Gv) * V (eq. 3) or SiLU(x W_1) * (x W_3): accumulator columns
     // [0, 128) and [128, 256) pair up; this warp makes output columns [64 part, 64 part + 64)
     const bool gate = a.epi == EPI_QKVG;
+    const bool lo = !gate && a.out1 != nullptr;  // SwiGLU output as a bf16 hi + lo pair (out0, out1)
     uint8_t* box = slot + part * BOX128;
+    uint8_t* box_lo = slot + (2 + part) * BOX128;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       tmem_ld32x2(trow + part * 64 + 32 * j, v, trow + 128 + part * 64 + 32 * j, w);
@@ -211,11 +213,17 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
       }
       if (j == 0) slot_ready();
       stage_bf16_sw128(box, r, 4 * j, v);
+      if (lo) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
+        stage_bf16_sw128(box_lo, r, 4 * j, w);
+      }
     }
     issue();
     const int x = (gate ? t - nH : t) * 128 + 64 * part;
     if (lane == 0 && x < a.d) {  // the last SwiGLU tile may end past d_ff
       tma_store_2d(&mp.o[gate ? 2 : 0], box + q * 32 * 128, x, y0);
+      if (lo) tma_store_2d(&mp.o[1], box_lo + q * 32 * 128, x, y0);
       bulk_commit();
     }
     return;
@@ -541,7 +549,9 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
              make_tmap(&mp.o[2], false, a.out2, a.M, d, a.ldo, 64, 32, 128) &&
              make_tmap(&mp.o[3], true, a.out3, a.M, d, a.ldo, 32, 32, 128);
     }
-    case EPI_SWIGLU: return make_tmap(&mp.o[0], false, a.out0, a.M, a.d, a.ldo, 64, 32, 128);
+    case EPI_SWIGLU:
+      return make_tmap(&mp.o[0], false, a.out0, a.M, a.d, a.ldo, 64, 32, 128) &&
+             (!a.out1 || make_tmap(&mp.o[1], false, a.out1, a.M, a.d, a.ldo, 64, 32, 128));
     case EPI_DT: return make_tmap(&mp.o[0], false, a.out0, a.M, a.N, a.ldo, 64, 32, 128);
     case EPI_DECQG: {
       const long long w = (long long)a.k_tok * a.N;
@@ -616,7 +626,10 @@ bool sm100_gemm_supported(const GemmArgs& a) {
 cudaError_t launch_gemm_sm100(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   switch (a.epi) {
     case EPI_QKVG: return launch_cfg<3, 2, 65536, true>(a, s, err);                  // cos + sin in, double-buffered
-    case EPI_SWIGLU: case EPI_DT: return launch_cfg<5, 2, 32768, false>(a, s, err);  // bf16 out, double-buffered
+    case EPI_SWIGLU:
+      if (a.out1) return launch_cfg<5, 1, 65536, false>(a, s, err);  // bf16 hi + lo out
+      return launch_cfg<5, 2, 32768, false>(a, s, err);               // bf16 out, double-buffered
+    case EPI_DT: return launch_cfg<5, 2, 32768, false>(a, s, err);
     default: return launch_cfg<5, 1, 65536, false>(a, s, err);                       // fp32 out (store or residual add)
   }
 }

@@ -150,3 +150,32 @@ def test_rank_request_host_validation():
     st = R.library().rest_rank_request(R.REST_BF16, ctypes.byref(hs), ctypes.byref(b), FAKE, FAKE, arr, 1, 0,
                                        ctypes.byref(rq), FAKE, ctypes.byref(dp), FAKE, FAKE, FAKE, 1 << 40, None, None)
     assert st == INVALID
+
+
+def _score_call(dt=R.REST_BF16, d=256, K=3, n=5, d_ff=704, z=FAKE, y=FAKE, f=FAKE, score=FAKE, ws=FAKE,
+                ws_bytes=1 << 30, null_params=False, w13=FAKE):
+    sp = R.ScoreParams(w13, FAKE, FAKE, FAKE, FAKE, 0.5, d_ff)
+    return R.library().rest_score_head(dt, d, K, n, z, y, None if null_params else ctypes.byref(sp), f, score, ws,
+                                       ws_bytes, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=0), 1), (dict(d=2048), 1), (dict(d=100), 1), (dict(K=0), 1), (dict(K=9), 1), (dict(n=-1), 1),
+    (dict(d_ff=0), 1), (dict(d_ff=100), 1), (dict(dt=7), 1), (dict(null_params=True), 1), (dict(z=None), 1),
+    (dict(y=FAKE + 4), 1), (dict(f=None), 1), (dict(score=None), 1), (dict(w13=None), 1),
+    (dict(ws=None), 6), (dict(ws_bytes=100), 6),
+])
+def test_score_head_rejects_invalid_arguments(kw, code):
+    assert _score_call(**kw) == code
+
+
+def test_score_head_workspace_and_empty_batch():
+    out = ctypes.c_size_t(0)
+    assert R.library().rest_score_workspace_size(R.REST_BF16, 256, 3, 1000, 704, ctypes.byref(out)) == 0
+    assert out.value >= 1000 * 3 * (256 + 704) * 2
+    assert _score_call(n=0, z=None, y=None, f=None, score=None, ws=None) == 0  # nothing to do
+
+
+@pytest.mark.skipif(gpu_available(), reason="the no-device status needs a host without a GPU")
+def test_score_head_without_gpu_reports_no_device():
+    assert _score_call() == 7

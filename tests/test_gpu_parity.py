@@ -236,3 +236,40 @@ def test_full_workload_decoder_sampled_requests(cuda, cfg, n_req):
         one = dict(inp, req_user=inp["req_user"][r:r + 1], req_cutoff=inp["req_cutoff"][r:r + 1],
                    cu_cands=np.array([0, cc[r + 1] - cc[r]], dtype=np.int32), z=inp["z"][cc[r]:cc[r + 1]])
         assert_parity(y[cc[r]:cc[r + 1]], oracle_decode(one, Hm), "bf16", f"request {r}")
+
+
+# ------------------------------------------------------------- decoder block and candidate score
+
+@pytest.mark.parametrize("dtype,hd", [("f32", 16), ("bf16", 32), ("bf16", 64)])
+def test_score_head_small_ragged(cuda, dtype, hd):
+    """Encoder, decoder and the score head end to end (eq. 8 FFN sublayer, [CLS] logit)."""
+    w = W.small_workload(dtype, lengths=(300, 129, 1, 64), d=4 * hd, n_heads=4, n_layers=1, l_switch=0,
+                         requests=[(0, 300, 50), (0, 77, 3), (1, 129, 1), (2, 1, 5), (3, 64, 44)])
+    inp = W.make_inputs(w, 51, ln_affine=True)
+    t = R.to_device(inp, cuda)
+    _, y = R.rank_request(t["x"], t["ts"], t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"],
+                          t["z"], t["dec"], t["rope_base"])
+    f, s = R.score_head(t["z"], y, t["score"])
+    torch.cuda.synchronize()
+    _, yr = O.rank_request(inp)
+    fr, sr = O.score_head(inp["z"], yr, inp["score"])
+    assert_parity(f.cpu().numpy(), fr, dtype, "f")
+    assert_parity(s.cpu().numpy(), sr, dtype, "score")
+
+
+@pytest.mark.parametrize("cfg", [1, 4])
+def test_score_head_full_size_sampled_candidates(cuda, cfg):
+    """The score head over every candidate of a full workload with a synthetic
+    decoder output; a sample of candidates (first, last, random) in the oracle."""
+    w = W.workload(cfg)
+    inp = W.make_inputs(w, 1000 + cfg)
+    t = R.to_device(inp, cuda)
+    rng = np.random.default_rng(cfg)
+    y_h = (0.5 * rng.standard_normal(inp["z"].shape)).astype(np.float32)
+    f, s = R.score_head(t["z"], torch.from_numpy(y_h).to(cuda), t["score"])
+    torch.cuda.synchronize()
+    n = w.total_cands
+    pick = np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, 62)]))
+    fr, sr = O.score_head(inp["z"][pick], y_h[pick], inp["score"])
+    assert_parity(f.cpu().numpy()[pick], fr, "bf16", "f")
+    assert_parity(s.cpu().numpy()[pick], sr, "bf16", "score")
