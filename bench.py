@@ -454,9 +454,16 @@ def main():
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     H = torch.empty_like(t["x"])
     Y = torch.empty(t["z"].shape, dtype=torch.float32, device=dev)
+    # the decoder block and [CLS] logit turn y into the candidate scores
+    dt_code = R.REST_BF16 if w.dtype == "bf16" else R.REST_F32
+    ws_s = torch.empty(R.score_workspace_size(dt_code, w.d, w.K, w.total_cands, int(t["score"]["w_ffn2"].shape[1])),
+                       dtype=torch.uint8, device=dev)
+    F = torch.empty_like(Y)
+    S = torch.empty((w.total_cands,), dtype=torch.float32, device=dev)
 
     def step():
         R.rank_request(*args_rank, h_out=H, y_out=Y, ws=ws, check=False)
+        R.score_head(t["z"], Y, t["score"], f_out=F, score_out=S, ws=ws_s, check=False)
 
     def barrier():
         if world > 1:
@@ -464,6 +471,7 @@ def main():
 
     # correctness guard: the device status word must stay clear
     R.rank_request(*args_rank, h_out=H, y_out=Y, ws=ws, check=True)
+    R.score_head(t["z"], Y, t["score"], f_out=F, score_out=S, ws=ws_s, check=True)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -509,9 +517,9 @@ def main():
     x_h = t["x"].cpu().pin_memory()
     ts_h = t["ts"].cpu().pin_memory()
     z_h = t["z"].cpu().pin_memory()
-    y_h = [torch.empty(Y.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_h = [torch.empty(S.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
     bufs = [(torch.empty_like(t["x"]), torch.empty_like(t["ts"]), torch.empty_like(t["z"]),
-             torch.empty(Y.shape, dtype=torch.float32, device=dev)) for _ in range(2)]
+             torch.empty_like(S)) for _ in range(2)]
     s_copy, s_comp = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     copied = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
@@ -528,17 +536,18 @@ def main():
             copied[i % 2].record(s_copy)
 
     def compute(i):
-        x_d, ts_d, z_d, y_d = bufs[i % 2]
+        x_d, ts_d, z_d, s_d = bufs[i % 2]
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(copied[i % 2])
             R.rank_request(x_d, ts_d, t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"], z_d,
-                           t["dec"], t["rope_base"], h_out=H, y_out=y_d, ws=ws, stream=s_comp, check=False)
+                           t["dec"], t["rope_base"], h_out=H, y_out=Y, ws=ws, stream=s_comp, check=False)
+            R.score_head(z_d, Y, t["score"], f_out=F, score_out=s_d, ws=ws_s, stream=s_comp, check=False)
             computed[i % 2].record(s_comp)
 
     def d2h(i):
         with torch.cuda.stream(s_copy):
             s_copy.wait_event(computed[i % 2])
-            y_h[i % 2].copy_(bufs[i % 2][3], non_blocking=True)
+            s_h[i % 2].copy_(bufs[i % 2][3], non_blocking=True)
 
     def e2e_run(n):
         h2d(0)
@@ -612,7 +621,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": int(x_h.numel() * x_h.element_size() + ts_h.numel() * 8 +
                                           z_h.numel() * z_h.element_size()),
-                "d2h_bytes_per_step": int(y_h[0].numel() * 4),
+                "d2h_bytes_per_step": int(s_h[0].numel() * 4),
                 "overlap": "double-buffered: step i+1's input copies and step i-1's score copy-back run on a "
                            "copy stream while step i computes"},
         "gpu_launches": launches,

@@ -67,6 +67,11 @@ struct GemmArgs {
   const void* A2;                 // bf16 low part of A (A = A + A2, same layout), or null
   const void* B2;                 // EPI_DECQG: the stacked W_go [K_tok * K, N] (B is W_Q)
   int k_tok;                      // EPI_DECQG: number of token types
+  // EPI_SWIGLU / EPI_RESID / EPI_F32: `groups` independent products in one
+  // launch; group g reads A columns [g K, g K + K), B rows [g K, g K + K) (the
+  // groups' weights stacked) and writes output columns [g W, g W + W), W the
+  // output width (d_ff, resp. N). 0 or 1: one product.
+  int groups;
 };
 // Logical output columns of EPI_QKVG are [Q | K | V,Gv interleaved | Go] and of
 // EPI_SWIGLU [W1,W3 interleaved]: every group of 4 logical columns holds

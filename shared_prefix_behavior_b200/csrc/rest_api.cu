@@ -450,10 +450,12 @@ static double gemm_out_bytes(const GemmArgs& a, size_t e) {
 static rest_status run_gemm(const Plan& p, const GemmArgs& a, const char* name, cudaStream_t s) {
   const bool bf = p.dt == REST_BF16;
   const size_t e = dt_size(p.dt);
-  const double groups = a.epi == EPI_DECQG ? 2.0 * a.k_tok : 1.0;  // (q, g) x token types
+  const double groups = a.epi == EPI_DECQG ? 2.0 * a.k_tok : a.groups > 1 ? (double)a.groups : 1.0;
   const double flops = 2.0 * a.M * a.N * a.K * groups;
-  const double bytes = (a.a_f32 || a.A2 ? 4 : e) * (double)a.M * a.K * (a.epi == EPI_DECQG ? a.k_tok : 1) +
-                       e * (double)a.K * a.N * groups + gemm_out_bytes(a, e);
+  const double a_sets = a.epi == EPI_DECQG ? a.k_tok : a.groups > 1 ? a.groups : 1;  // distinct A column blocks
+  const double out_sets = a.epi != EPI_DECQG && a.groups > 1 ? a.groups : 1;
+  const double bytes = (a.a_f32 || a.A2 ? 4 : e) * (double)a.M * a.K * a_sets + e * (double)a.K * a.N * groups +
+                       gemm_out_bytes(a, e) * out_sets;
   if (bf && sm100_gemm_supported(a)) {
     REST_KLAUNCH(s, name, flops, bytes, launch_gemm_sm100(a, s, p.err));
   } else {
@@ -916,8 +918,10 @@ rest_status rest_score_head(rest_dtype dt, int d, int K, long long n_cands, cons
     // a = z + y (the query token's residual, fp32 in f_out) and u = LN_k(a)
     REST_KLAUNCH(s, "score_ln", 0, (double)rows * d * (e + 4 + 4 + 2 * e),
                  launch_score_ln(bf, z, y, f_out, u, u_lo, sp->ln_g, sp->ln_b, rows, d, K, s));
-    // token type k: rows n K + k of u, f_out and the hidden state, with that type's weights (eq. 8)
-    for (int k = 0; k < K; ++k) {
+    // token type k: columns [k d, k d + d) of u and f_out and [k d_ff, k d_ff + d_ff) of the
+    // hidden state (rows n K + k of the [n K, d] views), with that type's weights (eq. 8). The
+    // tensor-core GEMM takes all token types in one grouped launch; otherwise one launch each.
+    auto ffn13 = [&](int k) {
       GemmArgs a = gemm(u + e * (size_t)k * d, (long long)K * d,
                         (const char*)sp->w_ffn13 + e * (size_t)k * d * 2 * dff, 2LL * dff, n_cands, 2 * dff, d,
                         EPI_SWIGLU, hid + e * (size_t)k * dff, (long long)K * dff);
@@ -926,15 +930,29 @@ rest_status rest_score_head(rest_dtype dt, int d, int K, long long n_cands, cons
         a.A2 = u_lo + e * (size_t)k * d;
         a.out1 = hid_lo + e * (size_t)k * dff;
       }
-      if ((st = run_gemm(p, a, "gemm_score_ffn13", s)) != REST_OK) return st;
-    }
-    for (int k = 0; k < K; ++k) {
+      return a;
+    };
+    auto ffn2 = [&](int k) {
       GemmArgs a = gemm(hid + e * (size_t)k * dff, (long long)K * dff,
                         (const char*)sp->w_ffn2 + e * (size_t)k * dff * d, d, n_cands, d, dff, EPI_RESID,
                         f_out + (size_t)k * d, (long long)K * d);
       a.alpha = 1.0f;
       if (bf) a.A2 = hid_lo + e * (size_t)k * dff;
-      if ((st = run_gemm(p, a, "gemm_score_ffn2", s)) != REST_OK) return st;
+      return a;
+    };
+    for (int stage = 0; stage < 2; ++stage) {
+      const char* name = stage == 0 ? "gemm_score_ffn13" : "gemm_score_ffn2";
+      GemmArgs all = stage == 0 ? ffn13(0) : ffn2(0);
+      all.groups = K;
+      // one launch per token type already fills the GPU when it has a few hundred
+      // 256-row x 256-column tiles; below that the grouped launch avoids idle SMs
+      const long long tiles = (n_cands + 255) / 256 * (stage == 0 ? (dff + 127) / 128 : (d + 255) / 256);
+      if (bf && K > 1 && tiles < 2 * SCHED_CTAS && sm100_gemm_supported(all)) {
+        if ((st = run_gemm(p, all, name, s)) != REST_OK) return st;
+      } else {
+        for (int k = 0; k < K; ++k)
+          if ((st = run_gemm(p, stage == 0 ? ffn13(k) : ffn2(k), name, s)) != REST_OK) return st;
+      }
     }
     REST_KLAUNCH(s, "score_readout", 2.0 * n_cands * d, (double)n_cands * d * 4,
                  launch_score_readout(f_out, sp->w_s, sp->b_s, score_out, n_cands, d, K, s));

@@ -314,33 +314,49 @@ cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, cons
 // ============================================================================
 
 // a = z + y into f; u = dt(LN_k(a)) with token type k = row % K. One warp per
-// row of d <= 1024 columns (lane holds columns lane, lane + 32, ...).
-template <typename T>
+// row; lane holds columns 128 i + 4 lane .. + 3 (d a multiple of 128, NV = d / 128)
+// or, for other widths, columns lane, lane + 32, ... (NV = 0).
+template <typename T, int NV>
 __global__ void score_ln_kernel(const T* __restrict__ z, const float* __restrict__ y, float* __restrict__ f,
                                 T* __restrict__ u, T* __restrict__ u_lo, const float* __restrict__ ln_g,
                                 const float* __restrict__ ln_b, long long rows, int d, int K) {
-  constexpr int VMAX = 32;
+  constexpr int VN = NV > 0 ? 4 * NV : 32;  // values per lane
   const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   const int k = (int)(row % K);
   const long long o = row * d;
-  float v[VMAX];
+  auto col = [&](int i) { return NV > 0 ? 128 * (i >> 2) + 4 * lane + (i & 3) : 32 * i + lane; };
+  float v[VN];
   float sum = 0.f;
+  if (NV > 0) {
 #pragma unroll
-  for (int i = 0; i < VMAX; ++i) {
-    const int c = i * 32 + lane;
-    v[i] = c < d ? to_f<T>(z[o + c]) + y[o + c] : 0.f;
-    if (c < d) f[o + c] = v[i];
-    sum += v[i];
+    for (int i = 0; i < NV; ++i) {
+      float zz[4], yy[4];
+      load4(z + o + 128 * i + 4 * lane, zz);
+      load4(y + o + 128 * i + 4 * lane, yy);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[4 * i + e] = zz[e] + yy[e];
+      store4(f + o + 128 * i + 4 * lane, &v[4 * i]);
+    }
+#pragma unroll
+    for (int i = 0; i < VN; ++i) sum += v[i];
+  } else {
+#pragma unroll
+    for (int i = 0; i < VN; ++i) {
+      const int c = col(i);
+      v[i] = c < d ? to_f<T>(z[o + c]) + y[o + c] : 0.f;
+      if (c < d) f[o + c] = v[i];
+      sum += v[i];
+    }
   }
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
   const float mean = sum / d;
   float sq = 0.f;
 #pragma unroll
-  for (int i = 0; i < VMAX; ++i) {
-    const float t = i * 32 + lane < d ? v[i] - mean : 0.f;
+  for (int i = 0; i < VN; ++i) {
+    const float t = col(i) < d ? v[i] - mean : 0.f;
     sq += t * t;
   }
 #pragma unroll
@@ -348,31 +364,59 @@ __global__ void score_ln_kernel(const T* __restrict__ z, const float* __restrict
   const float rstd = 1.0f / sqrtf(sq / d + 1e-5f);
   const float* g = ln_g + (long long)k * d;
   const float* b = ln_b + (long long)k * d;
+  if (NV > 0) {
 #pragma unroll
-  for (int i = 0; i < VMAX; ++i) {
-    const int c = i * 32 + lane;
-    if (c < d) {
-      const float n = (v[i] - mean) * rstd * g[c] + b[c];
-      const T hi = from_f<T>(n);
-      u[o + c] = hi;
-      if (u_lo) u_lo[o + c] = from_f<T>(n - to_f<T>(hi));
+    for (int i = 0; i < NV; ++i) {
+      const int c = 128 * i + 4 * lane;
+      float gg[4], bb[4], hi[4], lo[4];
+      load4(g + c, gg);
+      load4(b + c, bb);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float n = (v[4 * i + e] - mean) * rstd * gg[e] + bb[e];
+        hi[e] = to_f<T>(from_f<T>(n));
+        lo[e] = n - hi[e];
+      }
+      store4(u + o + c, hi);
+      if (u_lo) store4(u_lo + o + c, lo);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VN; ++i) {
+      const int c = col(i);
+      if (c < d) {
+        const float n = (v[i] - mean) * rstd * g[c] + b[c];
+        const T hi = from_f<T>(n);
+        u[o + c] = hi;
+        if (u_lo) u_lo[o + c] = from_f<T>(n - to_f<T>(hi));
+      }
     }
   }
+}
+
+template <typename T>
+static cudaError_t score_ln_dispatch(const T* z, const float* y, float* f, T* u, T* u_lo, const float* ln_g,
+                                    const float* ln_b, long long rows, int d, int K, cudaStream_t s) {
+  const int threads = 256;
+  const long long blocks = (rows * 32 + threads - 1) / threads;
+  const unsigned nb = (unsigned)blocks;
+  switch (d % 128 == 0 ? d / 128 : 0) {
+    case 1: score_ln_kernel<T, 1><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
+    case 2: score_ln_kernel<T, 2><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
+    case 4: score_ln_kernel<T, 4><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
+    case 8: score_ln_kernel<T, 8><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
+    default: score_ln_kernel<T, 0><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_score_ln(bool bf16m, const void* z, const float* y, float* f, void* u, void* u_lo,
                             const float* ln_g, const float* ln_b, long long rows, int d, int K, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
   if (d > 1024 || K < 1) return cudaErrorInvalidValue;
-  const int threads = 256;
-  const long long blocks = (rows * 32 + threads - 1) / threads;
   if (bf16m)
-    score_ln_kernel<bf16><<<(unsigned)blocks, threads, 0, s>>>((const bf16*)z, y, f, (bf16*)u, (bf16*)u_lo, ln_g,
-                                                                ln_b, rows, d, K);
-  else
-    score_ln_kernel<float><<<(unsigned)blocks, threads, 0, s>>>((const float*)z, y, f, (float*)u, nullptr, ln_g,
-                                                                 ln_b, rows, d, K);
-  return cudaGetLastError();
+    return score_ln_dispatch<bf16>((const bf16*)z, y, f, (bf16*)u, (bf16*)u_lo, ln_g, ln_b, rows, d, K, s);
+  return score_ln_dispatch<float>((const float*)z, y, f, (float*)u, nullptr, ln_g, ln_b, rows, d, K, s);
 }
 
 // score[n] = f[n, 0, :] . w_s + b_s (token 0 is [CLS]); one warp per candidate.

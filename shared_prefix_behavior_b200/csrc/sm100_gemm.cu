@@ -67,6 +67,14 @@ __host__ __device__ __forceinline__ int tile_n(const GemmArgs& a) { return a.epi
 // Output columns of a 256-column tile of an fp32 output; the last tile may end past the width.
 __host__ __device__ __forceinline__ int f32_tiles(int width) { return (width + 255) / 256; }
 
+// Grouped products: N-tiles per group and the group of N-tile t.
+__host__ __device__ __forceinline__ int tiles_per_group(const GemmArgs& a) {
+  return a.epi == EPI_SWIGLU ? (a.d + 127) / 128 : f32_tiles(a.N);
+}
+__host__ __device__ __forceinline__ bool grouped(const GemmArgs& a) {
+  return a.groups > 1 && (a.epi == EPI_SWIGLU || a.epi == EPI_RESID || a.epi == EPI_F32);
+}
+
 // Global column (in the B map that box_map selects) of the 64-column box b
 // that CTA `rank` loads for N-tile t.
 __device__ __forceinline__ int b_box_col(const GemmArgs& a, int t, int rank, int b, bool* second_map) {
@@ -78,6 +86,7 @@ __device__ __forceinline__ int b_box_col(const GemmArgs& a, int t, int rank, int
     *second_map = true;                                                     // Go, through its [K, d] view
     return (t - 2 * nH) * 256 + 128 * rank + 64 * b;
   }
+  if (grouped(a)) t %= tiles_per_group(a);  // the group's rows of B come from the K offset
   if (a.epi == EPI_SWIGLU) {  // W_1 | W_3, each through its own [K, d_ff] view
     *second_map = rank != 0;
     return t * 128 + 64 * b;
@@ -220,10 +229,12 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
       }
     }
     issue();
-    const int x = (gate ? t - nH : t) * 128 + 64 * part;
+    const int tl = gate ? t - nH : grouped(a) ? t % tiles_per_group(a) : t;
+    const int gofs = gate || !grouped(a) ? 0 : (t / tiles_per_group(a)) * a.d;
+    const int x = tl * 128 + 64 * part;
     if (lane == 0 && x < a.d) {  // the last SwiGLU tile may end past d_ff
-      tma_store_2d(&mp.o[gate ? 2 : 0], box + q * 32 * 128, x, y0);
-      if (lo) tma_store_2d(&mp.o[1], box_lo + q * 32 * 128, x, y0);
+      tma_store_2d(&mp.o[gate ? 2 : 0], box + q * 32 * 128, gofs + x, y0);
+      if (lo) tma_store_2d(&mp.o[1], box_lo + q * 32 * 128, gofs + x, y0);
       bulk_commit();
     }
     return;
@@ -249,6 +260,11 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
   // plain, sigmoid, the decoder's q / gate, or the residual add
   const CUtensorMap* om = &mp.o[0];
   int x0 = t * 256, width = a.N;
+  if (grouped(a)) {  // group g writes columns [g N, g N + N)
+    const int g = t / tiles_per_group(a);
+    x0 = g * a.N + (t % tiles_per_group(a)) * 256;
+    width = g * a.N + a.N;
+  }
   bool sig = a.epi == EPI_SIGMOID;
   if (a.epi == EPI_QKVG) {
     om = &mp.o[3];
@@ -356,7 +372,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int nb = tile_n(a) / 128;  // 64-column boxes of B per CTA
       const uint32_t tx = 2 * (A_BYTES + nb * BOX_B_BYTES);
       // decoder projections: token type k selects the column block of z and the row block of the weights
-      const int kofs = a.epi == EPI_DECQG ? ((t / f32_tiles(a.N)) % a.k_tok) * a.K : 0;
+      const int kofs = a.epi == EPI_DECQG ? ((t / f32_tiles(a.N)) % a.k_tok) * a.K
+                       : grouped(a)       ? (t / tiles_per_group(a)) * a.K
+                                          : 0;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % STAGES;
         const int kk = kb < num_kb ? kb : kb - num_kb;
@@ -520,18 +538,19 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
          make_tmap(&mp.b2, false, a.B2, kk, a.N, a.ldb, 64, BK, 128);
     mp.a2 = mp.a;
   } else {
-    ok = make_tmap(&mp.a, false, a.A, a.M, a.K, a.lda, BK, BM, 128);
+    const long long G = grouped(a) ? a.groups : 1, KG = G * a.K;  // grouped: the groups' K blocks side by side
+    ok = make_tmap(&mp.a, false, a.A, a.M, KG, a.lda, BK, BM, 128);
     mp.a2 = mp.a;
-    if (ok && a.A2) ok = make_tmap(&mp.a2, false, a.A2, a.M, a.K, a.lda, BK, BM, 128);
+    if (ok && a.A2) ok = make_tmap(&mp.a2, false, a.A2, a.M, KG, a.lda, BK, BM, 128);
     if (a.epi == EPI_SWIGLU) {
       // W_1 and W_3 as two [K, d_ff] views of the [K, 2 d_ff] weight, so that a
       // ragged last tile reads zeros past d_ff rather than the other block
       const bf16* w = static_cast<const bf16*>(a.B);
-      ok = ok && make_tmap(&mp.b, false, w, a.K, a.d, a.ldb, 64, BK, 128) &&
-           make_tmap(&mp.b2, false, w + a.d, a.K, a.d, a.ldb, 64, BK, 128);
+      ok = ok && make_tmap(&mp.b, false, w, KG, a.d, a.ldb, 64, BK, 128) &&
+           make_tmap(&mp.b2, false, w + a.d, KG, a.d, a.ldb, 64, BK, 128);
     } else {
       // B is [K, Ncols] with Ncols = ldb (the full weight width)
-      ok = ok && make_tmap(&mp.b, false, a.B, a.K, a.ldb, a.ldb, 64, BK, 128);
+      ok = ok && make_tmap(&mp.b, false, a.B, KG, a.ldb, a.ldb, 64, BK, 128);
       mp.b2 = mp.b;
       // the output-gate block W_go as its own [K, d] view (a ragged last Go tile reads zeros)
       if (ok && a.epi == EPI_QKVG)
@@ -549,16 +568,19 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
              make_tmap(&mp.o[2], false, a.out2, a.M, d, a.ldo, 64, 32, 128) &&
              make_tmap(&mp.o[3], true, a.out3, a.M, d, a.ldo, 32, 32, 128);
     }
-    case EPI_SWIGLU:
-      return make_tmap(&mp.o[0], false, a.out0, a.M, a.d, a.ldo, 64, 32, 128) &&
-             (!a.out1 || make_tmap(&mp.o[1], false, a.out1, a.M, a.d, a.ldo, 64, 32, 128));
+    case EPI_SWIGLU: {
+      const long long wd = (grouped(a) ? a.groups : 1) * (long long)a.d;
+      return make_tmap(&mp.o[0], false, a.out0, a.M, wd, a.ldo, 64, 32, 128) &&
+             (!a.out1 || make_tmap(&mp.o[1], false, a.out1, a.M, wd, a.ldo, 64, 32, 128));
+    }
     case EPI_DT: return make_tmap(&mp.o[0], false, a.out0, a.M, a.N, a.ldo, 64, 32, 128);
     case EPI_DECQG: {
       const long long w = (long long)a.k_tok * a.N;
       return make_tmap(&mp.o[0], true, a.out0, a.M, w, a.ldo, 32, 32, 128) &&
              make_tmap(&mp.o[1], true, a.out1, a.M, w, a.ldo, 32, 32, 128);
     }
-    default: return make_tmap(&mp.o[0], true, a.out0, a.M, a.N, a.ldo, 32, 32, 128);
+    default: return make_tmap(&mp.o[0], true, a.out0, a.M, (grouped(a) ? a.groups : 1) * (long long)a.N, a.ldo, 32,
+                              32, 128);
   }
 }
 
@@ -597,6 +619,7 @@ cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   if (a.epi == EPI_QKVG) n_tiles_n = 2 * (a.d / 128) + f32_tiles(a.d);
   if (a.epi == EPI_SWIGLU) n_tiles_n = (a.d + 127) / 128;
   if (a.epi == EPI_DECQG) n_tiles_n = 2 * a.k_tok * f32_tiles(a.N);
+  if (grouped(a)) n_tiles_n = a.groups * tiles_per_group(a);
   const int n_tiles = n_tiles_n * ((a.M + 2 * BM - 1) / (2 * BM));
   cfg.gridDim = dim3(2 * (n_tiles < max_pairs ? n_tiles : max_pairs));
   return cudaLaunchKernelEx(&cfg, kern, mp, a, a.K / BK, n_tiles_n, n_tiles, err);
