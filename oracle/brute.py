@@ -138,6 +138,73 @@ def encoder(inp, gates_on: bool = True):
     return np.array(x)
 
 
+def encoder_stream(inp, cached):
+    """The encoder as a server with a per-layer cache runs it: each user's
+    tokens arrive one at a time, in order, and pass through all layers; at
+    every layer the token appends its rotated key (explicit R_Theta per head)
+    and gated value to that layer's cache and attends to the cache as it then
+    stands (every earlier token and itself). No full-sequence score matrix is
+    ever formed. Returns the H rows and each layer's cache rows of the tokens
+    at positions >= cached[u], packed in user order."""
+    X = np.asarray(inp["x"], dtype=np.float64)
+    ts = [int(t) for t in inp["ts"]]
+    taus = [int(t) for t in inp["taus"]]
+    H = len(taus)
+    d = X.shape[1]
+    hd = d // H
+    base = float(inp["rope_base"])
+    layers = inp["layers"]
+    cu = [int(c) for c in inp["cu_seqlens"]]
+    h_rows, k_rows, v_rows = [], [[] for _ in layers], [[] for _ in layers]
+    for u in range(len(cu) - 1):
+        s, e = cu[u], cu[u + 1]
+        kc = [[] for _ in layers]  # per layer: rotated keys of the tokens seen so far
+        vc = [[] for _ in layers]  # per layer: gated values
+        for i in range(s, e):
+            pos = i - s
+            idx = [pos if tau == 0 else bucket(ts[i], ts[s], tau) for tau in taus]
+            x = [float(c) for c in X[i]]
+            for l, lay in enumerate(layers, start=1):
+                post = l <= inp["l_switch"]
+                g, b, a = lay["ln_attn_g"], lay["ln_attn_b"], float(lay["alpha_attn"])
+                y = x if post else ln_row(x, g, b)
+                W = np.asarray(lay["w_qkvgg"], dtype=np.float64)
+                q, k, v, gv, go = (matvec(y, W[:, c * d:(c + 1) * d]) for c in range(5))
+                qr, kr = np.zeros(d), np.zeros(d)
+                for h in range(H):
+                    sl = slice(h * hd, (h + 1) * hd)
+                    R = R_matrix(idx[h], hd, base)
+                    qr[sl] = R @ q[sl]
+                    kr[sl] = R @ k[sl]
+                kc[l - 1].append(kr)
+                vc[l - 1].append(np.array([v[c] * sig(gv[c]) for c in range(d)]))
+                o = np.zeros(d)
+                for h in range(H):
+                    sl = slice(h * hd, (h + 1) * hd)
+                    p = softmax_list([float(qr[sl] @ km[sl]) / math.sqrt(hd) for km in kc[l - 1]])
+                    for m, pm in enumerate(p):
+                        o[sl] += pm * vc[l - 1][m][sl]
+                upd = matvec([o[c] * sig(go[c]) for c in range(d)], lay["w_o"])
+                x = [x[c] + a * upd[c] for c in range(d)]
+                if post:
+                    x = ln_row(x, g, b)
+                if lay.get("w_ffn13") is not None:
+                    g, b, a = lay["ln_ffn_g"], lay["ln_ffn_b"], float(lay["alpha_ffn"])
+                    y = x if post else ln_row(x, g, b)
+                    upd = ffn([y], lay)[0]
+                    x = [x[c] + a * upd[c] for c in range(d)]
+                    if post:
+                        x = ln_row(x, g, b)
+            if pos >= int(cached[u]):
+                h_rows.append(x)
+                for l in range(len(layers)):
+                    k_rows[l].append(kc[l][-1])
+                    v_rows[l].append(vc[l][-1])
+    shape = (-1, d)
+    return (np.array(h_rows, dtype=np.float64).reshape(shape),
+            [(np.array(k_rows[l]).reshape(shape), np.array(v_rows[l]).reshape(shape)) for l in range(len(layers))])
+
+
 def cross_decode(Hmem, cu_seqlens, req_user, req_cutoff, cu_cands, z, dec, n_heads):
     Hm = np.asarray(Hmem, dtype=np.float64)
     z = np.asarray(z, dtype=np.float64)

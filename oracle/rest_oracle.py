@@ -152,13 +152,16 @@ def _f64(a):
 
 
 def dga_sublayer(y: np.ndarray, phi: np.ndarray, cu_seqlens: np.ndarray, layer: dict,
-                 n_heads: int, gates: bool = True, row_chunk: int = 2048) -> np.ndarray:
+                 n_heads: int, gates: bool = True, row_chunk: int = 2048,
+                 kv_out: Optional[list] = None) -> np.ndarray:
     """Eqs. 3-5: (Attention(R q, R k, sigmoid(y W_gv) * y W_V) * sigmoid(y W_go)) W_o.
 
     Readings: no biases; the gates are full d x d projections applied
     elementwise; head h owns columns h*d_h..(h+1)*d_h-1; the score scale is
     1/sqrt(d_h) (eq. 7's multi-head form; eq. 3 is written single-head).
-    ``gates=False`` replaces both sigmoids by 1 (test knob).
+    ``gates=False`` replaces both sigmoids by 1 (test knob). When ``kv_out``
+    is a list, the rotated keys R k and the gated values V' of every row (the
+    operands later queries attend to) are appended to it as a pair.
     """
     T, d = y.shape
     hd = d // n_heads
@@ -167,6 +170,8 @@ def dga_sublayer(y: np.ndarray, phi: np.ndarray, cu_seqlens: np.ndarray, layer: 
     Q, Kx, V, Gv, Go = (P5[:, i * d:(i + 1) * d] for i in range(5))
     Vg = V * sigmoid(Gv) if gates else V
     Qr, Kr = rotate(Q, phi), rotate(Kx, phi)
+    if kv_out is not None:
+        kv_out.append((Kr, Vg))
     O = np.zeros((T, d))
     scale = 1.0 / math.sqrt(hd)
     for u in range(len(cu_seqlens) - 1):
@@ -210,12 +215,14 @@ def srn(x: np.ndarray, sub, alpha: float, post: bool, g: np.ndarray, b: np.ndarr
 # --------------------------------------------------------------------------
 
 def encoder(inp: dict, gates: bool = True, angle_scale: float = 1.0,
-            time_origin=None, pos_offset: int = 0, n_layers: Optional[int] = None) -> np.ndarray:
+            time_origin=None, pos_offset: int = 0, n_layers: Optional[int] = None,
+            kv_out: Optional[list] = None) -> np.ndarray:
     """Encoder T (§3.2, Fig. 1 left): n_layers blocks of [DGA, SwiGLU FFN],
     each sublayer wrapped by eq. 6 with post-LN for l <= l_switch (1-based).
 
     Readings: one layer = attention sublayer then FFN sublayer (the LLaMA
     block the page starts from); no final norm; separate alpha per sublayer.
+    ``kv_out`` (a list) receives each layer's (R k, V') pair, layer by layer.
     """
     x = _f64(inp["x"]).copy()
     taus = np.asarray(inp["taus"], dtype=np.int64)
@@ -227,12 +234,48 @@ def encoder(inp: dict, gates: bool = True, angle_scale: float = 1.0,
     layers = inp["layers"] if n_layers is None else inp["layers"][:n_layers]
     for l, lay in enumerate(layers, start=1):
         post = l <= inp["l_switch"]
-        x = srn(x, lambda y: dga_sublayer(y, phi, inp["cu_seqlens"], lay, H, gates),
+        x = srn(x, lambda y: dga_sublayer(y, phi, inp["cu_seqlens"], lay, H, gates, kv_out=kv_out),
                 lay["alpha_attn"], post, lay["ln_attn_g"], lay["ln_attn_b"])
         if lay.get("w_ffn13") is not None:
             x = srn(x, lambda y: ffn_sublayer(y, lay),
                     lay["alpha_ffn"], post, lay["ln_ffn_g"], lay["ln_ffn_b"])
     return x
+
+
+def encoder_append(hist: dict, cached: Sequence[int]):
+    """Append-only encoding of the tokens that follow a cached prefix.
+
+    Why a prefix can be cached: the encoder's attention is causal (eqs. 3-5:
+    row i reads rows j <= i only), every other step acts on one row at a time,
+    and RoTE counts time from the history's first timestamp t_1 (§3.2.2),
+    which appending does not move. So H and every layer's rotated keys R k and
+    gated values V' on a history's first c rows stay the same when tokens are
+    appended after them (the same argument §3.5 makes for the prefix a request
+    reads). An append therefore computes only the new rows, attending to the
+    cached keys and values of the old ones.
+
+    Definition: ``hist`` is each user's whole history (the cached tokens, then
+    the new ones) in the encoder's input form; user u has cached[u] tokens in
+    the cache. The result holds rows cached[u] .. L_u - 1 of every user, packed
+    in user order:
+        H_new  [T_new, d]      those rows of encoder(hist)
+        kv     [(K_l, V_l)]    those rows of layer l's R k and V'
+        cu_new [n_users + 1]   prefix sums of L_u - cached[u]
+    """
+    cu = np.asarray(hist["cu_seqlens"], dtype=np.int64)
+    n_users = len(cu) - 1
+    if len(cached) != n_users:
+        raise ValueError("one cached length per user")
+    for u in range(n_users):
+        if not 0 <= int(cached[u]) <= cu[u + 1] - cu[u]:
+            raise ValueError(f"user {u}: cached length outside 0..L_u")
+    kv = []
+    H = encoder(hist, kv_out=kv)
+    rows = [np.arange(cu[u] + int(cached[u]), cu[u + 1], dtype=np.int64) for u in range(n_users)]
+    rows = np.concatenate(rows) if rows else np.zeros(0, dtype=np.int64)
+    cu_new = np.zeros(n_users + 1, dtype=np.int64)
+    cu_new[1:] = np.cumsum([cu[u + 1] - cu[u] - int(cached[u]) for u in range(n_users)])
+    return H[rows], [(k[rows], v[rows]) for k, v in kv], cu_new
 
 
 def encoder_rows(inp: dict, rows: Sequence[int]) -> np.ndarray:

@@ -318,6 +318,62 @@ def test_union_encoding_equals_encoding_each_prefix_alone():
     assert rel_err(yc, y[3:6]) < 1e-12
 
 
+# ------------------------------------------------- append-only encoder cache
+
+def truncate(inp, lengths):
+    """Each user's first lengths[u] tokens, in the encoder's input form."""
+    cu = inp["cu_seqlens"]
+    rows = np.concatenate([np.arange(cu[u], cu[u] + lengths[u]) for u in range(len(lengths))])
+    cu2 = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cu2[1:] = np.cumsum(lengths)
+    return dict(inp, x=inp["x"][rows], ts=inp["ts"][rows], cu_seqlens=cu2)
+
+
+@pytest.mark.parametrize("l_switch,ffn", [(1, True), (0, False), (2, True)])
+def test_encoder_append_matches_token_by_token_stream(l_switch, ffn):
+    """The append's definition (rows of the full-history encoder) against a
+    server loop that sees one token at a time and only a per-layer cache of
+    rotated keys and gated values."""
+    w, inp = tiny_inputs(seed=21, lengths=(7, 5, 3), n_layers=2, l_switch=l_switch, ffn=ffn, n_rope=1)
+    cached = [3, 0, 3]
+    Hn, kv, cu_new = O.encoder_append(inp, cached)
+    Hb, kvb = brute.encoder_stream(inp, cached)
+    assert list(cu_new) == [0, 4, 9, 9]
+    assert Hn.shape == (9, 16) and len(kv) == 2
+    assert rel_err(Hn, Hb) < 1e-12
+    for (k, v), (kb, vb) in zip(kv, kvb):
+        assert rel_err(k, kb) < 1e-12 and rel_err(v, vb) < 1e-12
+
+
+def test_cache_of_a_prefix_is_unchanged_by_later_tokens():
+    """Keys, values and H cached while the history was shorter stay valid:
+    the prefix alone gives the prefix rows of the longer history (causality,
+    and RoTE's origin is the first timestamp, which appending keeps)."""
+    w, inp = tiny_inputs(seed=22, lengths=(9, 6), n_layers=2, l_switch=1, n_rope=1)
+    cut = [4, 2]
+    H_pre, kv_pre, _ = O.encoder_append(truncate(inp, cut), [0, 0])
+    H_all, kv_all, _ = O.encoder_append(inp, [0, 0])
+    rows = np.r_[0:4, 9:11]
+    assert rel_err(H_pre, H_all[rows]) < 1e-13
+    for (kp, vp), (ka, va) in zip(kv_pre, kv_all):
+        assert rel_err(kp, ka[rows]) < 1e-13 and rel_err(vp, va[rows]) < 1e-13
+    # the rest of the history, appended to that cache, gives the remaining rows
+    H_new, kv_new, cu_new = O.encoder_append(inp, cut)
+    rest = np.r_[4:9, 11:15]
+    assert list(cu_new) == [0, 5, 9]
+    assert rel_err(H_new, H_all[rest]) < 1e-13
+
+
+def test_encoder_append_of_nothing_and_of_everything():
+    w, inp = tiny_inputs(seed=23, lengths=(5, 4), n_layers=1, l_switch=0)
+    H_new, kv, cu_new = O.encoder_append(inp, [5, 4])
+    assert H_new.shape == (0, 16) and list(cu_new) == [0, 0, 0] and kv[0][0].shape == (0, 16)
+    H_all, _, _ = O.encoder_append(inp, [0, 0])
+    assert np.array_equal(H_all, O.encoder(inp))
+    with pytest.raises(ValueError):
+        O.encoder_append(inp, [6, 0])
+
+
 # ------------------------------------------------------------ input module
 
 def test_bf16_rounding_matches_torch():
