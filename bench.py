@@ -343,6 +343,89 @@ def sharing_comparison(w, inp, dev, ms_shared):
             "speedup_of_sharing": alone_per_cand / shared_per_cand}
 
 
+def append_comparison(w, inp, dev, full_ms, n_new=64):
+    """Append-only encoding: every user's history minus its last n_new tokens
+    sits in the key/value cache, and the call encodes those n_new tokens
+    against it; compared with re-encoding the whole history (the encoder-only
+    time above). L2 is flushed (a 256 MB write) before every timed call, so
+    the cached keys and values come from HBM."""
+    import torch
+    import shared_prefix_behavior_b200 as R
+    t = R.to_device(inp, dev)
+    cu = np.asarray(inp["cu_seqlens"])
+    L = np.diff(cu)
+    cut = np.maximum(L - n_new, 0)
+    cache = R.KVCache(L, len(t["layers"]), w.d, t["x"].dtype, dev, keep_h=True)
+
+    def part(lo, hi):
+        rows = np.concatenate([np.arange(cu[u] + lo[u], cu[u] + hi[u]) for u in range(len(L))]).astype(np.int64)
+        cu2 = np.zeros(len(L) + 1, dtype=np.int32)
+        cu2[1:] = np.cumsum(hi - lo)
+        ri = torch.from_numpy(rows).to(dev)
+        return t["x"][ri].contiguous(), t["ts"][ri].contiguous(), cu2, inp["ts"][rows]
+
+    xp, tp, cup, tsp = part(np.zeros_like(L), cut)
+    R.encoder_append(xp, tp, cup, t["taus"], t["layers"], t["l_switch"], cache, rope_base=t["rope_base"],
+                     ts_host=tsp)
+    xn, tn, cun, _ = part(cut, L)
+    ws = torch.empty(max(256, R.append_workspace_size(R.REST_BF16 if w.dtype == "bf16" else R.REST_F32, t["taus"],
+                                                      w.d, cun, t["layers"], t["rope_base"])),
+                     dtype=torch.uint8, device=dev)
+    h_out = torch.empty_like(xn)
+
+    def app(check=False):
+        R.encoder_append(xn, tn, cun, t["taus"], t["layers"], t["l_switch"], cache, rope_base=t["rope_base"],
+                         advance=False, h_out=h_out, ws=ws, check=check)
+
+    app(check=True)
+    for _ in range(3):
+        app()
+    torch.cuda.synchronize()
+    n = 20
+    # host time to enqueue one call (the GPU is kept busy by flushes meanwhile)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for i in range(8):
+        flush.fill_(i & 0xff)
+    t_host = time.perf_counter()
+    for _ in range(n):
+        app()
+    host_ms = (time.perf_counter() - t_host) * 1e3 / n
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        flush.fill_(i & 0xff)
+        evs[i][0].record()
+        app()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    ms = sum(x.elapsed_time(y) for x, y in evs) / n
+    # per-kernel split (a separate pass: every launch bracketed by its own events)
+    R.profile_begin()
+    for i in range(n):
+        flush.fill_(i & 0xff)
+        app()
+    stats = R.profile_end()
+    torch.cuda.synchronize()
+    new = int((L - cut).sum())
+    out = {"cached_tokens": int(cut.sum()), "new_tokens": new, "new_per_user": n_new, "ms": ms,
+           "new_tokens_per_s": new / (ms * 1e-3), "full_reencode_ms": full_ms,
+           "speedup_vs_reencode": full_ms / ms, "l2": "flushed before every call (256 MB write)",
+           "launches_per_call": sum(s_["launches"] for s_ in stats) / n, "host_enqueue_ms": host_ms,
+           "kernels_ms_per_call": {s_["name"]: s_["ms"] / n for s_ in sorted(stats, key=lambda x: -x["ms"])}}
+    attn = [s_ for s_ in stats if s_["name"] == "enc_attn"]
+    if attn:
+        # a few new query rows against every cached key: the cached K and V' must cross
+        # HBM once per layer, which bounds the kernel (far below the ridge point)
+        sec = attn[0]["ms"] * 1e-3
+        peaks, src = load_peaks()
+        t_roof = max(attn[0]["flops"] / (float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))) * 1e12),
+                     attn[0]["bytes"] / (float(peaks["hbm_gbs"]) * 1e9))
+        out["attention"] = {"ms": attn[0]["ms"] / n, "tflops": attn[0]["flops"] / sec / 1e12,
+                            "gbs": attn[0]["bytes"] / sec / 1e9, "roofline_frac": t_roof / sec,
+                            "roofline": f"max(FLOPs / sustained bf16 peak, bytes / HBM copy bandwidth) ({src})"}
+    return out
+
+
 # --------------------------------------------------------------------- oracle (CPU baseline / reference arm)
 
 def blas_threads() -> int:
@@ -577,6 +660,8 @@ def main():
     parts = component_timings(args, w, t, H, Y, ws, dev, peaks_for_parts())
     if args.sharing and world == 1:
         parts["sharing"] = sharing_comparison(w, inp, dev, ms_step)
+    if world == 1:
+        parts["append"] = append_comparison(w, inp, dev, parts["encoder_only"]["ms"])
 
     if world > 1:
         dist.barrier()
@@ -629,8 +714,9 @@ def main():
         "encoder_only": parts["encoder_only"],
         "decoder_only": parts["decoder_only"],
     }
-    if "sharing" in parts:
-        out["sharing"] = parts["sharing"]
+    for k in ("sharing", "append"):
+        if k in parts:
+            out[k] = parts[k]
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_budget)
     print(json.dumps(out), flush=True)

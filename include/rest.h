@@ -205,6 +205,62 @@ rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest
                               void* h_out, float* y_out,
                               void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
+/* Append-only encoder cache. The encoder's attention is causal (eqs. 3-5),
+ * its other steps act row by row, and RoTE counts time from a history's first
+ * timestamp (§3.2.2), which appending leaves in place; so the encoder state of
+ * a history's first c tokens does not change when tokens are appended after
+ * them (§3.5 uses the same fact for the prefix a request reads). The cache
+ * keeps, for every layer and cached token, the rotated key R k and the gated
+ * value V' = sigmoid(y W_gv) * (y W_V) that later tokens attend to, and
+ * optionally the token's row of H.
+ *
+ * User u owns rows cu_cap[u] .. cu_cap[u+1]-1 of every cache array; its first
+ * len[u] rows hold positions 0 .. len[u]-1 of its history. The arrays are
+ * caller-owned device memory in the call's dtype, [rows, d] each. Rows that
+ * hold no cached token must hold finite values (allocate the arrays
+ * zero-filled): the attention reads keys in blocks of 128 rows and weights the
+ * rows past a user's last key by zero, and zero times a NaN is NaN.
+ *
+ * With h set, the cache's H rows serve rest_cross_decode directly: pass
+ * {n_users, cu_cap} as its batch and keep every cutoff within len[u]. */
+typedef struct {
+  void* const* k;          /* host [n_layers]: dev [rows, d] arrays, R k of layer l */
+  void* const* v;          /* host [n_layers]: dev [rows, d] arrays, V' of layer l */
+  void* h;                 /* dev [rows, d]: H rows, or NULL */
+  long long rows;          /* rows of each array, < 2^31 */
+  const int32_t* cu_cap;   /* host [n_users+1]: cu_cap[0] == 0, non-decreasing, cu_cap[n_users] <= rows */
+  const int32_t* len;      /* host [n_users]: cached tokens of each user */
+  const int64_t* t_first;  /* host [n_users]: timestamp of the user's first cached token (read when len[u] > 0) */
+  const int64_t* t_last;   /* host [n_users]: timestamp of the user's last cached token (read when len[u] > 0) */
+} rest_kv_cache;
+
+/* Workspace bytes rest_encoder_append needs for these new tokens. */
+rest_status rest_append_workspace_size(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                       const rest_enc_layer* layers, int n_layers, size_t* bytes);
+
+/* Encodes tokens appended to cached histories, computing only their rows:
+ * the result equals rows len[u] .. len[u]+n_u-1 of rest_encoder_attn over
+ * each user's whole history (positions continue after the cached ones and
+ * RoTE time counts from t_first[u]).
+ *   batch: the new tokens, packed: user u's n_u new tokens are rows
+ *          cu_seqlens[u] .. cu_seqlens[u+1]-1 of x and ts
+ *   x:     dev [T_new, d] (dtype of the call)
+ *   ts:    dev [T_new] int64 seconds, non-decreasing within each user and not
+ *          below t_last[u] (a decrease sets *dev_err = REST_ERR_UNSORTED_TIME)
+ *   cache: len[u] + n_u must fit user u's region (else REST_ERR_INVALID_ARG);
+ *          cache->k and cache->v hold n_layers arrays
+ *   h_out: dev [T_new, d] (dtype of the call)  the new rows of H
+ * For every layer the call writes the new tokens' R k and V' into the cache
+ * at rows cu_cap[u] + len[u] + i (and H there too when cache->h is set). It
+ * changes none of the host arrays: afterwards user u has len[u] + n_u cached
+ * tokens, whose first timestamp is t_first[u] (the first new one when len[u]
+ * was 0) and whose last is the last new one. */
+rest_status rest_encoder_append(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                const void* x, const int64_t* ts,
+                                const rest_enc_layer* layers, int n_layers, int l_switch,
+                                const rest_kv_cache* cache, void* h_out,
+                                void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
 /* Decoder block and candidate score ("From Language to Behavior", §3.3.2
  * eq. 8 and Fig. 1 right; the wiring the page leaves open is fixed as: a
  * residual on the query token, a pre-LN feed-forward sublayer whose LN and

@@ -10,6 +10,8 @@ Entry points (same names as the C ABI in include/rest.h):
 * ``encoder_attn``    -- encoder T (§3.2, eqs. 3-6)
 * ``cross_decode``    -- projection-free, token-specific cross decoder C (§3.3, eqs. 7-8)
 * ``rank_request``    -- shared-prefix serving: T once, C for every candidate (§3.5)
+* ``encoder_append``  -- T on tokens appended to cached histories (``KVCache``)
+* ``score_head``      -- decoder block and candidate score (§3.3.2, eq. 8)
 """
 from __future__ import annotations
 
@@ -28,7 +30,8 @@ STATUS = {0: "REST_OK", 1: "REST_ERR_INVALID_ARG", 2: "REST_ERR_UNSORTED_TIME", 
           4: "REST_ERR_CUDA", 5: "REST_ERR_TIMEOUT", 6: "REST_ERR_WORKSPACE", 7: "REST_ERR_NO_DEVICE"}
 EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
            "rest_rank_request", "rest_status_string", "rest_launch_count", "rest_profile_begin",
-           "rest_profile_end", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head")
+           "rest_profile_end", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",
+           "rest_append_workspace_size", "rest_encoder_append")
 STATIC_WS_BYTES = 32 * 1024 * 1024  # REST_STATIC_WS_BYTES
 
 
@@ -67,6 +70,12 @@ class Requests(ctypes.Structure):
                 ("cu_cands", POINTER(c_int32))]
 
 
+class KVCacheStruct(ctypes.Structure):
+    _fields_ = [("k", POINTER(c_void_p)), ("v", POINTER(c_void_p)), ("h", c_void_p), ("rows", c_longlong),
+                ("cu_cap", POINTER(c_int32)), ("len", POINTER(c_int32)), ("t_first", POINTER(c_int64)),
+                ("t_last", POINTER(c_int64))]
+
+
 class KernelStat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char_p), ("launches", c_int), ("ms", c_double), ("flops", c_double),
                 ("bytes", c_double)]
@@ -91,8 +100,13 @@ def _load() -> ctypes.CDLL:
     lib.rest_score_workspace_size.argtypes = [c_int, c_int, c_int, c_longlong, c_int, POINTER(c_size_t)]
     lib.rest_score_head.argtypes = [c_int, c_int, c_int, c_longlong, P, P, POINTER(ScoreParams), P, P, P, c_size_t,
                                     P, P]
+    lib.rest_append_workspace_size.argtypes = [c_int, POINTER(Heads), POINTER(Batch), POINTER(EncLayer), c_int,
+                                               POINTER(c_size_t)]
+    lib.rest_encoder_append.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, POINTER(EncLayer), c_int, c_int,
+                                        POINTER(KVCacheStruct), P, P, c_size_t, P, P]
     for name in ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
-                 "rest_rank_request", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head"):
+                 "rest_rank_request", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",
+                 "rest_append_workspace_size", "rest_encoder_append"):
         getattr(lib, name).restype = c_int
     lib.rest_status_string.argtypes = [c_int]
     lib.rest_status_string.restype = ctypes.c_char_p
@@ -326,6 +340,94 @@ def rank_request(x, ts, cu_seqlens, taus, layers: Sequence[dict], l_switch: int,
     if check:
         check_device_error(err)
     return h_out, y_out
+
+
+class KVCache:
+    """An append-only encoder cache: per layer the rotated keys and gated values
+    of every cached token, and the cached tokens' rows of H, in zero-filled
+    device arrays of ``capacity[u]`` rows per user; plus the host bookkeeping
+    the C ABI reads (cached length, first and last timestamp per user)."""
+
+    def __init__(self, capacity, n_layers: int, d: int, dtype, device, keep_h: bool = True):
+        import torch
+        cap = _i32(capacity)
+        self.n_users = len(cap)
+        self.cu_cap = np.zeros(self.n_users + 1, dtype=np.int32)
+        self.cu_cap[1:] = np.cumsum(cap)
+        self.rows = int(self.cu_cap[-1])
+        shape = (max(1, self.rows), d)
+        self.k = [torch.zeros(shape, dtype=dtype, device=device) for _ in range(n_layers)]
+        self.v = [torch.zeros(shape, dtype=dtype, device=device) for _ in range(n_layers)]
+        self.h = torch.zeros(shape, dtype=dtype, device=device) if keep_h else None
+        self.len = np.zeros(self.n_users, dtype=np.int32)
+        self.t_first = np.zeros(self.n_users, dtype=np.int64)
+        self.t_last = np.zeros(self.n_users, dtype=np.int64)
+
+    def struct(self):
+        """The rest_kv_cache view; the returned tuple keeps its host arrays alive."""
+        kp = (c_void_p * max(1, len(self.k)))(*[t.data_ptr() for t in self.k])
+        vp = (c_void_p * max(1, len(self.v)))(*[t.data_ptr() for t in self.v])
+        st = KVCacheStruct(kp, vp, _ptr(self.h), self.rows, self.cu_cap.ctypes.data_as(POINTER(c_int32)),
+                           self.len.ctypes.data_as(POINTER(c_int32)), self.t_first.ctypes.data_as(POINTER(c_int64)),
+                           self.t_last.ctypes.data_as(POINTER(c_int64)))
+        return st, (kp, vp)
+
+    def advance(self, cu_new, ts_host) -> None:
+        """Record an append of the tokens packed by cu_new with host timestamps ts_host."""
+        cu = _i32(cu_new)
+        ts = np.asarray(ts_host, dtype=np.int64)
+        for u in range(self.n_users):
+            s, e = int(cu[u]), int(cu[u + 1])
+            if e == s:
+                continue
+            if self.len[u] == 0:
+                self.t_first[u] = ts[s]
+            self.t_last[u] = ts[e - 1]
+            self.len[u] += e - s
+
+    def batch(self):
+        """(cu_seqlens, cutoff limit) for decoding against the cached H: the
+        regions' bounds serve as rest_cross_decode's batch."""
+        return self.cu_cap.copy(), self.len.copy()
+
+
+def append_workspace_size(dtype: int, taus, d: int, cu_new, layers: Sequence[dict] = (),
+                          rope_base: float = 10000.0) -> int:
+    h = _Host(taus, d, rope_base, cu_new)
+    arr = _enc_layers(layers)
+    out = c_size_t(0)
+    _check(_lib.rest_append_workspace_size(dtype, ctypes.byref(h.heads), ctypes.byref(h.batch), arr, len(layers),
+                                           ctypes.byref(out)), "rest_append_workspace_size")
+    return out.value
+
+
+def encoder_append(x, ts, cu_new, taus, layers: Sequence[dict], l_switch: int, cache: KVCache,
+                   rope_base: float = 10000.0, ts_host=None, advance: bool = True, h_out=None, ws=None,
+                   stream=None, check=True):
+    """Encoder T on tokens appended to the histories in ``cache``: returns the
+    new rows of H [T_new, d] and writes the new keys, values (and H) into the
+    cache. With ``advance`` the cache's bookkeeping then counts the new tokens
+    (their host timestamps: ``ts_host``, else copied from ``ts``)."""
+    import torch
+    dev, d = x.device, x.shape[1]
+    dt = _dtype_code(x)
+    h = _Host(taus, d, rope_base, cu_new)
+    arr = _enc_layers(layers)
+    if h_out is None:
+        h_out = torch.empty_like(x)
+    if ws is None:
+        ws = _workspace(append_workspace_size(dt, taus, d, cu_new, layers, rope_base), dev)
+    cst, keep = cache.struct()
+    err = _err_word(dev, stream)
+    _check(_lib.rest_encoder_append(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(x), _ptr(ts), arr,
+                                    len(layers), l_switch, ctypes.byref(cst), _ptr(h_out), _ptr(ws), ws.numel(),
+                                    _ptr(err), _stream(stream)), "rest_encoder_append")
+    del keep
+    if check:
+        check_device_error(err)
+    if advance:
+        cache.advance(cu_new, ts.cpu().numpy() if ts_host is None else ts_host)
+    return h_out
 
 
 def launch_count(reset: bool = False) -> int:

@@ -16,9 +16,26 @@ struct TableParams {
   // on the host): idx theta_j mod 2 pi from the 16-bit pieces of idx
   double turn[3][64];
 };
+// Appending to cached histories: per user, the part of its history already in
+// the cache. The call's packed rows cu[u] .. cu[u+1]-1 are the user's new
+// tokens, at positions cached .. cached + n - 1 of its history.
+struct UserAppend {
+  long long t_origin;  // timestamp of the history's first token (RoTE's t_1), when cached > 0
+  long long t_prev;    // timestamp of the last cached token (order check), when cached > 0
+  int cached;          // tokens already cached
+  int key0;            // cache row of position 0
+};
+
+// app (nullable): positions and time origins of appended tokens, as above.
 cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users,
                                   int T, const TableParams& p, int64_t* idx_out, float* cos_out,
-                                  float* sin_out, int32_t* err, cudaStream_t s);
+                                  float* sin_out, int32_t* err, cudaStream_t s,
+                                  const UserAppend* app = nullptr);
+// Copies row i of user u (packed by cu) of src0 / src1 to row
+// app[u].key0 + app[u].cached + (i - cu[u]) of dst0 / dst1; src1, dst1 may be
+// null. row_bytes is a multiple of 16.
+cudaError_t launch_append_rows(const void* src0, void* dst0, const void* src1, void* dst1, const int32_t* cu,
+                               const UserAppend* app, int n_users, long long T, int row_bytes, cudaStream_t s);
 
 // ---------------------------------------------------------------- casts / norms
 // mode 0: y = dt(LN(x))  (pre-LN input of a sublayer)
@@ -96,6 +113,12 @@ struct EncAttnArgs {
   // tensor-core kernel: CTA c runs the work items (tile * n_heads + head)
   // sched[n_cta + 1 + k] for k in [sched[c], sched[c + 1])
   const int* sched; int n_cta;
+  // Appending (app non-null): q, gate and out hold the new rows (packed by cu);
+  // k and v are the cache arrays of key_rows rows, where user u's keys are rows
+  // app[u].key0 .. app[u].key0 + app[u].cached + n_u - 1 and its new row i sits
+  // at position app[u].cached + i.
+  const UserAppend* app;
+  long long key_rows;
 };
 cudaError_t launch_enc_attn_simt(bool bf16, int hd, const EncAttnArgs& a, cudaStream_t s);
 

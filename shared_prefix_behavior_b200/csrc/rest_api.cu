@@ -179,12 +179,16 @@ static std::vector<int> lpt_schedule(const std::vector<long long>& cost) {
   return out;
 }
 
-static std::vector<int> enc_schedule(const rest_batch* b, const std::vector<EncTile>& tiles, int n_heads, int rows) {
+// app (may be empty): the cached positions before each user's rows
+static std::vector<int> enc_schedule(const rest_batch* b, const std::vector<EncTile>& tiles, int n_heads, int rows,
+                                     const std::vector<UserAppend>& app) {
   std::vector<long long> cost;
   for (const EncTile& t : tiles) {
-    const int L = b->cu_seqlens[t.user + 1] - b->cu_seqlens[t.user];
+    const int n = b->cu_seqlens[t.user + 1] - b->cu_seqlens[t.user];
+    const int off = app.empty() ? 0 : app[t.user].cached;
     long long c = 0;
-    for (int r0 = t.q0; r0 < std::min(L, t.q0 + rows); r0 += 128) c += (std::min(L, r0 + 128) + 127) / 128;
+    for (int r0 = t.q0; r0 < std::min(n, t.q0 + rows); r0 += 128)
+      c += (std::min(off + n, off + r0 + 128) + 127) / 128;
     for (int h = 0; h < n_heads; ++h) cost.push_back(c);
   }
   return lpt_schedule(cost);
@@ -202,7 +206,7 @@ static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_he
 // ---------------------------------------------------------------- workspace
 
 struct Layout {
-  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, meta_end;
+  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, app, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
   size_t dq, dg, dout, hlo, part_o, part_ml;
   size_t total;
@@ -211,7 +215,7 @@ struct Layout {
 
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
                           int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split,
-                          size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2) {
+                          size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2, bool append) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -225,6 +229,7 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.enc_sched = take(sizeof(int) * n_enc_sched);
   L.dec_sched = take(sizeof(int) * n_dec_sched);
   L.dec_sched2 = take(sizeof(int) * n_dec_sched2);
+  L.app = take(append ? sizeof(UserAppend) * (size_t)b->n_users : 0);
   L.meta_end = off;
   L.cos_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
   L.sin_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
@@ -255,6 +260,7 @@ struct Plan {
   std::vector<EncTile> enc_tiles;
   std::vector<DecTile> dec_tiles;
   std::vector<int> enc_sched, dec_sched, dec_sched2;  // tensor-core attention: per-CTA item lists
+  std::vector<UserAppend> app;  // appending to a cache: each user's cached prefix
   int n_dec_hlo;  // leading decoder tiles that read H_lo (rank_request, bf16)
   Layout L;
   int32_t* err;
@@ -262,12 +268,42 @@ struct Plan {
   int n_split;  // decoder key splits (tensor-core path)
 };
 
+// The cache of an append: region bounds, cached lengths and their fit, the
+// per-layer arrays. Fills `app` (one entry per user).
+static rest_status check_cache(const rest_kv_cache* c, const rest_batch* b, int n_layers,
+                               std::vector<UserAppend>& app) {
+  app.clear();
+  if (!c || c->rows < 0 || c->rows >= (1LL << 31)) return REST_ERR_INVALID_ARG;
+  if (n_layers > 0 && (!c->k || !c->v)) return REST_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    if (!c->k[l] || !c->v[l] || !aligned16(c->k[l]) || !aligned16(c->v[l])) return REST_ERR_INVALID_ARG;
+  if (c->h && !aligned16(c->h)) return REST_ERR_INVALID_ARG;
+  if (b->n_users == 0) return REST_OK;
+  if (!c->cu_cap || !c->len || c->cu_cap[0] != 0) return REST_ERR_INVALID_ARG;
+  for (int u = 0; u < b->n_users; ++u) {
+    const long long cap = (long long)c->cu_cap[u + 1] - c->cu_cap[u];
+    const long long n = (long long)b->cu_seqlens[u + 1] - b->cu_seqlens[u];
+    if (cap < 0 || c->len[u] < 0 || c->len[u] + n > cap) return REST_ERR_INVALID_ARG;
+    UserAppend a{0, 0, c->len[u], c->cu_cap[u]};
+    if (c->len[u] > 0) {
+      if (!c->t_first || !c->t_last || c->t_last[u] < c->t_first[u]) return REST_ERR_INVALID_ARG;
+      a.t_origin = c->t_first[u];
+      a.t_prev = c->t_last[u];
+    }
+    app.push_back(a);
+  }
+  if (c->cu_cap[b->n_users] > c->rows) return REST_ERR_INVALID_ARG;
+  return REST_OK;
+}
+
 static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const rest_batch* b,
                              const rest_enc_layer* layers, int n_layers, int l_switch, const rest_requests* reqs,
-                             int K, bool encoder_runs) {
+                             int K, bool encoder_runs, const rest_kv_cache* cache = nullptr, bool append = false) {
   rest_status st = check_heads(dt, hs);
   if (st != REST_OK) return st;
   if ((st = check_batch(b, &p.T)) != REST_OK) return st;
+  p.app.clear();
+  if (cache && (st = check_cache(cache, b, n_layers, p.app)) != REST_OK) return st;
   if ((st = check_layers(layers, n_layers, l_switch, &p.max_dff)) != REST_OK) return st;
   p.n_cands = 0;
   if (reqs) {
@@ -300,7 +336,7 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   if (!p.hsplit)
     for (DecTile& t : p.dec_tiles) t.pad = 0;
   if (tile_rows != 128) {  // the tensor-core attention runs: schedule its persistent CTAs
-    if (!p.enc_tiles.empty()) p.enc_sched = enc_schedule(b, p.enc_tiles, hs->n_heads, tile_rows);
+    if (!p.enc_tiles.empty()) p.enc_sched = enc_schedule(b, p.enc_tiles, hs->n_heads, tile_rows, p.app);
     if (!p.dec_tiles.empty()) {  // [tiles that read H_lo | the others], scheduled separately
       std::vector<DecTile> a(p.dec_tiles.begin(), p.dec_tiles.begin() + p.n_dec_hlo);
       std::vector<DecTile> c(p.dec_tiles.begin() + p.n_dec_hlo, p.dec_tiles.end());
@@ -314,7 +350,7 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   }
   p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),
                     (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size(),
-                    p.dec_sched2.size());
+                    p.dec_sched2.size(), append);
   return REST_OK;
 }
 
@@ -402,6 +438,7 @@ static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
     memcpy(host.data() + p.L.dec_sched, p.dec_sched.data(), sizeof(int) * p.dec_sched.size());
   if (!p.dec_sched2.empty())
     memcpy(host.data() + p.L.dec_sched2, p.dec_sched2.data(), sizeof(int) * p.dec_sched2.size());
+  if (!p.app.empty()) memcpy(host.data() + p.L.app, p.app.data(), sizeof(UserAppend) * p.app.size());
   if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) return REST_ERR_CUDA;
   // the status word reports this call only
   if (p.err && cudaMemsetAsync(p.err, 0, sizeof(int32_t), s) != cudaSuccess) return REST_ERR_CUDA;
@@ -466,8 +503,12 @@ static rest_status run_gemm(const Plan& p, const GemmArgs& a, const char* name, 
 
 // ---------------------------------------------------------------- encoder
 
+// With `cache` the rows are tokens appended to cached histories: each layer
+// adds their rotated keys and gated values to the cache and attends to the
+// cached rows and the new ones.
 static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, const rest_enc_layer* layers,
-                               int n_layers, int l_switch, void* h_out, void* ws, int32_t* err, cudaStream_t s) {
+                               int n_layers, int l_switch, void* h_out, void* ws, int32_t* err, cudaStream_t s,
+                               const rest_kv_cache* cache = nullptr) {
   const bool bf = p.dt == REST_BF16;
   const int d = p.hs->d, hd = p.hs->head_dim, H = p.hs->n_heads;
   const long long T = p.T;
@@ -483,17 +524,21 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   float* g = at<float>(ws, L.g);
   void* hid = at<void>(ws, L.hid);
 
-  double causal_pairs = 0;  // sum over users of L(L+1)/2
+  const UserAppend* app = cache ? at<UserAppend>(ws, L.app) : nullptr;
+  double causal_pairs = 0;  // per user: n new rows after `off` cached ones see n off + n(n+1)/2 keys
+  double key_rows = 0;      // keys read per head (cached and new)
   for (int u = 0; u < p.b->n_users; ++u) {
-    double Lu = p.b->cu_seqlens[u + 1] - p.b->cu_seqlens[u];
-    causal_pairs += Lu * (Lu + 1) / 2;
+    const double n = p.b->cu_seqlens[u + 1] - p.b->cu_seqlens[u];
+    const double off = cache ? p.app[u].cached : 0;
+    causal_pairs += n * off + n * (n + 1) / 2;
+    key_rows += n > 0 ? off + n : 0;
   }
   const double attn_flops = 4.0 * d * causal_pairs;  // QK^T and PV over every head
-  const double attn_bytes = Td * (3 * e + 4 + e);
+  const double attn_bytes = Td * (e + 4 + e) + 2.0 * e * key_rows * d;  // Q, gate, out; K and V'
 
   TableParams tp = table_params(p.hs);
   REST_KLAUNCH(s, "rotation_table", 0, 8.0 * T + 4 * Td,
-               launch_rotation_table(ts, cu, p.b->n_users, (int)T, tp, nullptr, cos_t, sin_t, err, s));
+               launch_rotation_table(ts, cu, p.b->n_users, (int)T, tp, nullptr, cos_t, sin_t, err, s, app));
   REST_KLAUNCH(s, "to_f32", 0, Td * (e + 4), launch_to_f32(bf, x, xres, T * d, s));
 
   EncAttnArgs ea;
@@ -504,6 +549,8 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   ea.n_heads = H; ea.d = d;
   ea.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
   ea.rows = T;
+  ea.app = app;
+  ea.key_rows = cache ? cache->rows : T;
 
   // The sublayers in order (attention, then the FFN, per layer), each wrapped
   // by eq. 6: post-LN in the first l_switch layers, pre-LN after. One
@@ -530,8 +577,10 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   };
   // input of the first sublayer: with post-LN it reads x itself, which in bf16
   // is the call's input as it stands
+  // (with no layers H is x)
   const void* a_in = y;
-  if (subs[0].post) {
+  if (subs.empty()) {
+  } else if (subs[0].post) {
     if (bf) a_in = x;
     else if (rest_status st = norm(y, nullptr, nullptr, 2, nullptr, nullptr)) return st;
   } else if (rest_status st = norm(y, subs[0].g, subs[0].b, 0, nullptr, nullptr)) {
@@ -545,6 +594,13 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
       GemmArgs a = gemm(a_in, d, Ly.w_qkvgg, 5LL * d, T, 5 * d, d, EPI_QKVG, q, d);
       a.out1 = k; a.out2 = v; a.out3 = g; a.cos_t = cos_t; a.sin_t = sin_t; a.d = d;
       if (rest_status st = run_gemm(p, a, "gemm_qkvg", s)) return st;
+      if (cache) {  // the new rows' R k and V' join the layer's cache; attention reads keys there
+        REST_KLAUNCH(s, "append_kv", 0, 4.0 * e * Td,
+                     launch_append_rows(k, cache->k[S.layer], v, cache->v[S.layer], cu, app, p.b->n_users, T,
+                                        (int)(d * e), s));
+        ea.k = cache->k[S.layer];
+        ea.v = cache->v[S.layer];
+      }
       if (bf && sm100_attn_supported(hd)) {
         REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_sm100(hd, ea, s, err));
       } else {
@@ -586,6 +642,9 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   } else if (!h_written) {
     if (rest_status st = norm(h_out, nullptr, nullptr, 2, nullptr, nullptr)) return st;
   }
+  if (cache && cache->h)
+    REST_KLAUNCH(s, "append_h", 0, 2.0 * e * Td,
+                 launch_append_rows(h_out, cache->h, nullptr, nullptr, cu, app, p.b->n_users, T, (int)(d * e), s));
   return REST_OK;
 }
 
@@ -798,6 +857,43 @@ rest_status rest_encoder_attn(rest_dtype dt, const rest_heads* heads, const rest
     p.err = dev_err;
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
     return run_encoder(p, x, ts, layers, n_layers, l_switch, h_out, ws, dev_err, s);
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_append_workspace_size(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                       const rest_enc_layer* layers, int n_layers, size_t* bytes) {
+  if (!bytes) return REST_ERR_INVALID_ARG;
+  try {
+    Plan p;
+    rest_status st = make_plan(p, dt, heads, batch, layers, n_layers, n_layers, nullptr, 1, true, nullptr, true);
+    if (st != REST_OK) return st;
+    *bytes = p.L.total;
+    return REST_OK;
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_encoder_append(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, const void* x,
+                                const int64_t* ts, const rest_enc_layer* layers, int n_layers, int l_switch,
+                                const rest_kv_cache* cache, void* h_out, void* ws, size_t ws_bytes,
+                                int32_t* dev_err, void* stream) {
+  try {
+    if (!cache) return REST_ERR_INVALID_ARG;
+    Plan p;
+    rest_status st = make_plan(p, dt, heads, batch, layers, n_layers, l_switch, nullptr, 1, true, cache, true);
+    if (st != REST_OK) return st;
+    if (p.T > 0 && (!x || !ts || !h_out || !aligned16(x) || !aligned16(ts) || !aligned16(h_out)))
+      return REST_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < p.L.total || !aligned16(ws)) return REST_ERR_WORKSPACE;
+    if (p.T == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    return run_encoder(p, x, ts, layers, n_layers, l_switch, h_out, ws, dev_err, s, cache);
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }

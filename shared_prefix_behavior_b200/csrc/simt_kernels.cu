@@ -45,20 +45,29 @@ __device__ __forceinline__ void rotation(long long idx, const TableParams& p, in
 
 // One thread per (token, frequency j), looping over the heads: the user lookup
 // happens once per token, and consecutive threads write consecutive entries.
+// With `app` the rows are tokens appended to cached histories: positions
+// continue after the cached ones and time still counts from the history's
+// first timestamp.
 __global__ void rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu,
                                       int n_users, int T, TableParams p, int64_t* idx_out,
-                                      float* cos_out, float* sin_out, int32_t* err) {
+                                      float* cos_out, float* sin_out, int32_t* err,
+                                      const UserAppend* __restrict__ app) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= (long long)T * p.half) return;
   const int i = (int)(gid / p.half);
   const int j = (int)(gid % p.half);
-  const int s = cu[find_user(cu, n_users, i)];
+  const int u = find_user(cu, n_users, i);
+  const int s = cu[u];
+  const int cached = app ? app[u].cached : 0;
   const long long t = ts[i];
-  if (j == 0 && i > s && ts[i - 1] > t) set_error(err, REST_ERR_UNSORTED_TIME);
-  const long long rel = t - ts[s];  // exact int64
+  if (j == 0) {
+    if (i > s ? ts[i - 1] > t : (cached > 0 && app[u].t_prev > t)) set_error(err, REST_ERR_UNSORTED_TIME);
+  }
+  const long long rel = t - (cached > 0 ? app[u].t_origin : ts[s]);  // exact int64
+  const long long pos = (long long)(i - s) + cached;
   for (int h = 0; h < p.n_heads; ++h) {
     const long long tau = p.tau[h];
-    const long long idx = tau == 0 ? (long long)(i - s) : floor_div(rel, tau);
+    const long long idx = tau == 0 ? pos : floor_div(rel, tau);
     if (idx_out && j == 0) idx_out[(long long)i * p.n_heads + h] = idx;
     if (cos_out) {
       double sv, cv;
@@ -72,13 +81,41 @@ __global__ void rotation_table_kernel(const int64_t* __restrict__ ts, const int3
 
 cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users, int T,
                                     const TableParams& p, int64_t* idx_out, float* cos_out,
-                                    float* sin_out, int32_t* err, cudaStream_t s) {
+                                    float* sin_out, int32_t* err, cudaStream_t s, const UserAppend* app) {
   const long long n = (long long)T * p.half;
   if (n == 0) return cudaSuccess;
   const int threads = 256;
   const long long blocks = (n + threads - 1) / threads;
   rotation_table_kernel<<<(unsigned)blocks, threads, 0, s>>>(ts, cu, n_users, T, p, idx_out, cos_out,
-                                                             sin_out, err);
+                                                             sin_out, err, app);
+  return cudaGetLastError();
+}
+
+// One thread per 16 bytes of a row; rows of a user stay contiguous in the
+// cache, so consecutive threads write consecutive addresses.
+__global__ void append_rows_kernel(const uint4* __restrict__ src0, uint4* __restrict__ dst0,
+                                   const uint4* __restrict__ src1, uint4* __restrict__ dst1,
+                                   const int32_t* __restrict__ cu, const UserAppend* __restrict__ app, int n_users,
+                                   long long T, int row_vecs) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= T * row_vecs) return;
+  const long long i = gid / row_vecs;
+  const int c = (int)(gid % row_vecs);
+  const int u = find_user(cu, n_users, (int)i);
+  const long long dst_row = (long long)app[u].key0 + app[u].cached + (i - cu[u]);
+  dst0[dst_row * row_vecs + c] = src0[gid];
+  if (src1) dst1[dst_row * row_vecs + c] = src1[gid];
+}
+
+cudaError_t launch_append_rows(const void* src0, void* dst0, const void* src1, void* dst1, const int32_t* cu,
+                               const UserAppend* app, int n_users, long long T, int row_bytes, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (row_bytes % 16 != 0) return cudaErrorInvalidValue;
+  const int row_vecs = row_bytes / 16;
+  const long long n = T * row_vecs;
+  const int threads = 256;
+  append_rows_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(
+      (const uint4*)src0, (uint4*)dst0, (const uint4*)src1, (uint4*)dst1, cu, app, n_users, T, row_vecs);
   return cudaGetLastError();
 }
 
@@ -765,21 +802,24 @@ __global__ void __launch_bounds__(ATT_ROWS) enc_attn_simt_kernel(EncAttnArgs a) 
   __shared__ __align__(16) float Vs[ATT_BK][HD];
   EncTile tile = a.tiles[blockIdx.x];
   int h = blockIdx.y;
-  int s = a.cu[tile.user];
-  int L = a.cu[tile.user + 1] - s;
+  int s = a.cu[tile.user];                  // packed row of the user's first query row
+  int n = a.cu[tile.user + 1] - s;          // the user's query rows
+  int off = a.app ? a.app[tile.user].cached : 0;  // position of query row 0 in the history
+  int key0 = a.app ? a.app[tile.user].key0 : s;   // row of the history's first key
   int i = tile.q0 + threadIdx.x;
-  bool valid = i < L;
+  bool valid = i < n;
+  int pos = off + i;
   long long hoff = (long long)h * HD;
   RowState<HD> st;
   load_q<T, HD>(st, (const T*)a.q + (long long)(s + (valid ? i : 0)) * a.d + hoff, a.scale_log2);
-  int kv_end = min(L, tile.q0 + ATT_ROWS);
-  const T* K = (const T*)a.k + (long long)s * a.d + hoff;
-  const T* V = (const T*)a.v + (long long)s * a.d + hoff;
+  int kv_end = min(off + n, off + tile.q0 + ATT_ROWS);
+  const T* K = (const T*)a.k + (long long)key0 * a.d + hoff;
+  const T* V = (const T*)a.v + (long long)key0 * a.d + hoff;
   for (int kb = 0; kb < kv_end; kb += ATT_BK) {
     __syncthreads();
     stage_kv<T, HD, ATT_BK>(Ks, Vs, K + (long long)kb * a.d, V + (long long)kb * a.d, a.d, kv_end - kb);
     __syncthreads();
-    if (valid && kb <= i) row_tile<HD, ATT_BK>(st, Ks, Vs, i - kb + 1);  // causal: key <= i
+    if (valid && kb <= pos) row_tile<HD, ATT_BK>(st, Ks, Vs, pos - kb + 1);  // causal: key <= pos
   }
   if (valid) {
     long long ro = (long long)(s + i) * a.d + hoff;

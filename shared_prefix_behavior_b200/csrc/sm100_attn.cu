@@ -111,8 +111,8 @@ struct AttnItem {
   int key_row0;   // packed row of the item's first key
   int nrow[NT];   // valid query rows of each tile
   int nblk[NT];   // key blocks each tile reads
-  int user_len;   // encoder: the user's history length
-  int q_pos0;     // encoder: position of query row 0 within the user
+  int user_len;   // encoder: keys of the user's history (cached and new rows)
+  int q_pos0;     // encoder: position of query row 0 within the user's history
   int nkeys;      // keys from key_row0 visible to the item (decoder: cutoff minus the split start)
   int split;      // decoder: split index of the partial result
   int h;          // head
@@ -138,16 +138,20 @@ __device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const Dec
     }
   } else {
     const EncTile t = ea.tiles[tile];
-    w.key_row0 = ea.cu[t.user];
-    w.user_len = ea.cu[t.user + 1] - w.key_row0;
-    w.q_pos0 = t.q0;
-    w.q_row0 = w.key_row0 + t.q0;
+    const int s = ea.cu[t.user];
+    const int n = ea.cu[t.user + 1] - s;  // the user's query rows
+    // appending: the query rows follow `cached` positions held in the cache arrays
+    const int off = ea.app ? ea.app[t.user].cached : 0;
+    w.key_row0 = ea.app ? ea.app[t.user].key0 : s;
+    w.user_len = off + n;
+    w.q_pos0 = off + t.q0;
+    w.q_row0 = s + t.q0;
     w.nkeys = 0;
     w.split = 0;
     for (int i = 0; i < NT; ++i) {
       const int r0 = t.q0 + i * ROWS;
-      w.nrow[i] = max(0, min(ROWS, w.user_len - r0));
-      w.nblk[i] = w.nrow[i] > 0 ? (min(w.user_len, r0 + ROWS) + KB - 1) / KB : 0;
+      w.nrow[i] = max(0, min(ROWS, n - r0));
+      w.nblk[i] = w.nrow[i] > 0 ? (min(w.user_len, off + r0 + ROWS) + KB - 1) / KB : 0;
     }
   }
   return w;
@@ -553,9 +557,10 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
     mv = mk;
     if (MODE == 2 && !make_tmap_bf16(&mv, da->h_lo, rows, d, d, HD, ROWS, swz)) return cudaErrorInvalidValue;
   } else {
+    const long long key_rows = ea->app ? ea->key_rows : rows;
     if (!make_tmap_bf16(&mq, ea->q, rows, d, d, HD, ROWS, swz) ||
-        !make_tmap_bf16(&mk, ea->k, rows, d, d, HD, ROWS, swz) ||
-        !make_tmap_bf16(&mv, ea->v, rows, d, d, HD, ROWS, swz))
+        !make_tmap_bf16(&mk, ea->k, key_rows, d, d, HD, ROWS, swz) ||
+        !make_tmap_bf16(&mv, ea->v, key_rows, d, d, HD, ROWS, swz))
       return cudaErrorInvalidValue;
   }
   // at least 120 KB so that exactly one CTA (which takes all 512 TMEM columns) runs per SM

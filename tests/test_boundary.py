@@ -179,3 +179,67 @@ def test_score_head_workspace_and_empty_batch():
 @pytest.mark.skipif(gpu_available(), reason="the no-device status needs a host without a GPU")
 def test_score_head_without_gpu_reports_no_device():
     assert _score_call() == 7
+
+
+# ------------------------------------------------------------ append-only cache
+
+def _append(cu=(0, 4, 6), cap=(16, 8), length=(10, 2), rows=None, t_first=(100, 200), t_last=(150, 250),
+            n_layers=1, kv=FAKE, h=None, x=FAKE, ws_bytes=1 << 40, no_cache=False):
+    t, hs = _heads((0, 0, 1, 64), 64)
+    c, b = _batch(cu)
+    layers = [_layer(64, 192) for _ in range(n_layers)]
+    arr = (R.EncLayer * max(1, n_layers))(*layers)
+    capv = np.asarray(cap, dtype=np.int64)
+    cu_cap = np.zeros(len(capv) + 1, dtype=np.int32)
+    cu_cap[1:] = np.cumsum(capv)
+    ln = np.asarray(length, dtype=np.int32)
+    tf, tl = np.asarray(t_first, dtype=np.int64), np.asarray(t_last, dtype=np.int64)
+    kp = (ctypes.c_void_p * max(1, n_layers))(*([kv] * n_layers))
+    P32, P64 = ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)
+    cache = R.KVCacheStruct(kp, kp, h, int(cu_cap[-1]) if rows is None else rows, cu_cap.ctypes.data_as(P32),
+                            ln.ctypes.data_as(P32), tf.ctypes.data_as(P64), tl.ctypes.data_as(P64))
+    return R.library().rest_encoder_append(R.REST_BF16, ctypes.byref(hs), ctypes.byref(b), x, FAKE, arr, n_layers,
+                                           0, None if no_cache else ctypes.byref(cache), FAKE, FAKE, ws_bytes,
+                                           None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(no_cache=True), INVALID),
+    (dict(length=(13, 2)), INVALID),             # 13 cached + 4 new > 16 rows
+    (dict(length=(10, 7)), INVALID),             # 7 + 2 > 8
+    (dict(length=(-1, 2)), INVALID),
+    (dict(rows=20), INVALID),                    # regions end past the arrays
+    (dict(cap=(16, -2)), INVALID),               # decreasing region bounds
+    (dict(t_first=(200, 200)), INVALID),         # first timestamp after the last
+    (dict(kv=None), INVALID),                    # a layer without cache arrays
+    (dict(kv=FAKE + 8), INVALID),                # misaligned cache array
+    (dict(h=FAKE + 4), INVALID),
+    (dict(x=FAKE + 2), INVALID),
+    (dict(ws_bytes=64), WORKSPACE),
+])
+def test_append_rejects_invalid_arguments(kw, code):
+    assert _append(**kw) == code
+
+
+def test_append_of_no_tokens_is_a_noop_and_workspace_is_sized():
+    assert _append(cu=(0, 0, 0)) == 0
+    w = W.workload(1)
+    small = R.append_workspace_size(R.REST_BF16, w.taus, w.d, [0, 64, 128], [])
+    big = R.append_workspace_size(R.REST_BF16, w.taus, w.d, [0, 4096, 8192], [])
+    assert 0 < small < big
+
+
+@pytest.mark.skipif(gpu_available(), reason="the no-device status needs a host without a GPU")
+def test_append_without_gpu_reports_no_device():
+    assert _append() == NO_DEVICE
+
+
+def test_cache_bookkeeping_counts_appended_tokens():
+    import torch
+    c = R.KVCache([10, 5], n_layers=2, d=64, dtype=torch.float32, device="cpu")
+    assert c.rows == 15 and list(c.cu_cap) == [0, 10, 15] and len(c.k) == 2 and c.h is not None
+    c.advance([0, 3, 3], np.array([7, 9, 9]))
+    assert list(c.len) == [3, 0] and c.t_first[0] == 7 and c.t_last[0] == 9
+    c.advance([0, 1, 3], np.array([12, 40, 41]))
+    assert list(c.len) == [4, 2] and c.t_first[0] == 7 and c.t_last[0] == 12
+    assert c.t_first[1] == 40 and c.t_last[1] == 41
