@@ -379,6 +379,7 @@ struct ProfRec {
   double flops, bytes;
 };
 static thread_local bool g_prof = false;
+bool pdl_enabled() { return !g_prof; }
 static thread_local std::vector<ProfRec>* g_recs = nullptr;
 static thread_local std::vector<cudaEvent_t>* g_event_pool = nullptr;
 

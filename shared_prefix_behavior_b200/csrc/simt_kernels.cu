@@ -52,6 +52,8 @@ __global__ void rotation_table_kernel(const int64_t* __restrict__ ts, const int3
                                       int n_users, int T, TableParams p, int64_t* idx_out,
                                       float* cos_out, float* sin_out, int32_t* err,
                                       const UserAppend* __restrict__ app) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= (long long)T * p.half) return;
   const int i = (int)(gid / p.half);
@@ -86,8 +88,8 @@ cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_us
   if (n == 0) return cudaSuccess;
   const int threads = 256;
   const long long blocks = (n + threads - 1) / threads;
-  rotation_table_kernel<<<(unsigned)blocks, threads, 0, s>>>(ts, cu, n_users, T, p, idx_out, cos_out,
-                                                             sin_out, err, app);
+  if (cudaError_t e_ = launch_k(rotation_table_kernel, (unsigned)blocks, threads, 0, s, ts, cu, n_users, T, p, idx_out, cos_out,
+                                                             sin_out, err, app)) return e_;
   return cudaGetLastError();
 }
 
@@ -97,6 +99,8 @@ __global__ void append_rows_kernel(const uint4* __restrict__ src0, uint4* __rest
                                    const uint4* __restrict__ src1, uint4* __restrict__ dst1,
                                    const int32_t* __restrict__ cu, const UserAppend* __restrict__ app, int n_users,
                                    long long T, int row_vecs) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= T * row_vecs) return;
   const long long i = gid / row_vecs;
@@ -114,8 +118,7 @@ cudaError_t launch_append_rows(const void* src0, void* dst0, const void* src1, v
   const int row_vecs = row_bytes / 16;
   const long long n = T * row_vecs;
   const int threads = 256;
-  append_rows_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(
-      (const uint4*)src0, (uint4*)dst0, (const uint4*)src1, (uint4*)dst1, cu, app, n_users, T, row_vecs);
+  if (cudaError_t e_ = launch_k(append_rows_kernel, (unsigned)((n + threads - 1) / threads), threads, 0, s, (const uint4*)src0, (uint4*)dst0, (const uint4*)src1, (uint4*)dst1, cu, app, n_users, T, row_vecs)) return e_;
   return cudaGetLastError();
 }
 
@@ -205,6 +208,8 @@ template <typename T, int NV>
 __global__ void layernorm_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
                                  const float* __restrict__ b, const float* __restrict__ g2,
                                  const float* __restrict__ b2, int rows, int d, int mode) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   const int lane = threadIdx.x & 31;
   const int n_warps = gridDim.x * (blockDim.x >> 5);
   int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -242,14 +247,14 @@ static cudaError_t layernorm_dispatch(float* x, T* y, const float* g, const floa
   }
   if (blocks > cap) blocks = cap;
   switch (d / 128) {
-    case 1: layernorm_kernel<T, 1><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
-    case 2: layernorm_kernel<T, 2><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
-    case 3: layernorm_kernel<T, 3><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
-    case 4: layernorm_kernel<T, 4><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
-    case 5: layernorm_kernel<T, 5><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
-    case 6: layernorm_kernel<T, 6><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
-    case 7: layernorm_kernel<T, 7><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
-    case 8: layernorm_kernel<T, 8><<<blocks, threads, 0, s>>>(x, y, g, b, g2, b2, rows, d, mode); break;
+    case 1: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 1>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
+    case 2: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 2>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
+    case 3: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 3>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
+    case 4: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 4>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
+    case 5: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 5>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
+    case 6: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 6>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
+    case 7: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 7>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
+    case 8: if (cudaError_t e_ = launch_k(layernorm_kernel<T, 8>, blocks, threads, 0, s, x, y, g, b, g2, b2, rows, d, mode)) return e_; break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -261,6 +266,8 @@ template <typename T>
 __global__ void layernorm_narrow_kernel(float* __restrict__ x, T* __restrict__ y, const float* __restrict__ g,
                                         const float* __restrict__ b, const float* __restrict__ g2,
                                         const float* __restrict__ b2, int rows, int d, int mode) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   constexpr int VMAX = 32;  // d <= 1024
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
@@ -339,10 +346,11 @@ cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, cons
                  : layernorm_dispatch<float>(x, (float*)y, g, b, g2, b2, T, d, mode, s);
   int threads = 256;
   int blocks = (T * 32 + threads - 1) / threads;
-  if (bf16m)
-    layernorm_narrow_kernel<bf16><<<blocks, threads, 0, s>>>(x, (bf16*)y, g, b, g2, b2, T, d, mode);
-  else
-    layernorm_narrow_kernel<float><<<blocks, threads, 0, s>>>(x, (float*)y, g, b, g2, b2, T, d, mode);
+  if (bf16m) {
+    if (cudaError_t e_ = launch_k(layernorm_narrow_kernel<bf16>, blocks, threads, 0, s, x, (bf16*)y, g, b, g2, b2, T, d, mode)) return e_;
+  } else {
+    if (cudaError_t e_ = launch_k(layernorm_narrow_kernel<float>, blocks, threads, 0, s, x, (float*)y, g, b, g2, b2, T, d, mode)) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -357,6 +365,8 @@ template <typename T, int NV>
 __global__ void score_ln_kernel(const T* __restrict__ z, const float* __restrict__ y, float* __restrict__ f,
                                 T* __restrict__ u, T* __restrict__ u_lo, const float* __restrict__ ln_g,
                                 const float* __restrict__ ln_b, long long rows, int d, int K) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   constexpr int VN = NV > 0 ? 4 * NV : 32;  // values per lane
   const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -438,11 +448,11 @@ static cudaError_t score_ln_dispatch(const T* z, const float* y, float* f, T* u,
   const long long blocks = (rows * 32 + threads - 1) / threads;
   const unsigned nb = (unsigned)blocks;
   switch (d % 128 == 0 ? d / 128 : 0) {
-    case 1: score_ln_kernel<T, 1><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
-    case 2: score_ln_kernel<T, 2><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
-    case 4: score_ln_kernel<T, 4><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
-    case 8: score_ln_kernel<T, 8><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
-    default: score_ln_kernel<T, 0><<<nb, threads, 0, s>>>(z, y, f, u, u_lo, ln_g, ln_b, rows, d, K); break;
+    case 1: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 1>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
+    case 2: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 2>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
+    case 4: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 4>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
+    case 8: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 8>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
+    default: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 0>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
   }
   return cudaGetLastError();
 }
@@ -459,6 +469,8 @@ cudaError_t launch_score_ln(bool bf16m, const void* z, const float* y, float* f,
 // score[n] = f[n, 0, :] . w_s + b_s (token 0 is [CLS]); one warp per candidate.
 __global__ void score_readout_kernel(const float* __restrict__ f, const float* __restrict__ w_s, float b_s,
                                      float* __restrict__ score, long long n, int d, int K) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   const long long c = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (c >= n) return;
@@ -475,17 +487,21 @@ cudaError_t launch_score_readout(const float* f, const float* w_s, float b_s, fl
   if (n == 0) return cudaSuccess;
   const int threads = 256;
   const long long blocks = (n * 32 + threads - 1) / threads;
-  score_readout_kernel<<<(unsigned)blocks, threads, 0, s>>>(f, w_s, b_s, score, n, d, K);
+  if (cudaError_t e_ = launch_k(score_readout_kernel, (unsigned)blocks, threads, 0, s, f, w_s, b_s, score, n, d, K)) return e_;
   return cudaGetLastError();
 }
 
 template <typename T>
 __global__ void to_f32_kernel(const T* __restrict__ in, float* __restrict__ out, long long n) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = to_f<T>(in[i]);
 }
 // 8 bf16 values (16 bytes) per thread in, 32 bytes out
 __global__ void bf16_to_f32_x8_kernel(const uint4* __restrict__ in, float4* __restrict__ out, long long n8) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const uint4 u = in[i];
@@ -506,20 +522,22 @@ cudaError_t launch_to_f32(bool bf16m, const void* x_in, float* x_res, long long 
   if (bf16m && n % 8 == 0 && (reinterpret_cast<uintptr_t>(x_in) & 15) == 0 &&
       (reinterpret_cast<uintptr_t>(x_res) & 15) == 0) {
     const long long n8 = n / 8;
-    bf16_to_f32_x8_kernel<<<(unsigned)((n8 + threads - 1) / threads), threads, 0, s>>>(
-        static_cast<const uint4*>(x_in), reinterpret_cast<float4*>(x_res), n8);
+    if (cudaError_t e_ = launch_k(bf16_to_f32_x8_kernel, (unsigned)((n8 + threads - 1) / threads), threads, 0, s, static_cast<const uint4*>(x_in), reinterpret_cast<float4*>(x_res), n8)) return e_;
     return cudaGetLastError();
   }
   long long blocks = (n + threads - 1) / threads;
-  if (bf16m)
-    to_f32_kernel<bf16><<<(unsigned)blocks, threads, 0, s>>>((const bf16*)x_in, x_res, n);
-  else
-    to_f32_kernel<float><<<(unsigned)blocks, threads, 0, s>>>((const float*)x_in, x_res, n);
+  if (bf16m) {
+    if (cudaError_t e_ = launch_k(to_f32_kernel<bf16>, (unsigned)blocks, threads, 0, s, (const bf16*)x_in, x_res, n)) return e_;
+  } else {
+    if (cudaError_t e_ = launch_k(to_f32_kernel<float>, (unsigned)blocks, threads, 0, s, (const float*)x_in, x_res, n)) return e_;
+  }
   return cudaGetLastError();
 }
 
 __global__ void split_bf16_kernel(const float* __restrict__ x, bf16* __restrict__ hi, bf16* __restrict__ lo,
                                   long long n) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) {
     float v = x[i];
@@ -533,7 +551,7 @@ cudaError_t launch_split_bf16(const float* x, void* hi, void* lo, long long n, c
   if (n == 0) return cudaSuccess;
   int threads = 256;
   long long blocks = (n + threads - 1) / threads;
-  split_bf16_kernel<<<(unsigned)blocks, threads, 0, s>>>(x, (bf16*)hi, (bf16*)lo, n);
+  if (cudaError_t e_ = launch_k(split_bf16_kernel, (unsigned)blocks, threads, 0, s, x, (bf16*)hi, (bf16*)lo, n)) return e_;
   return cudaGetLastError();
 }
 
@@ -561,6 +579,8 @@ __device__ __forceinline__ int physical_col(const GemmArgs& a, int n) {
 // TA: type of A; T: the call's dtype (B and the dtype outputs).
 template <typename TA, typename T>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   constexpr int BM = 64, BN = 64, BK = 16;
   __shared__ __align__(16) float As[BK][BM + 4];
   __shared__ __align__(16) float Bs[BK][BN];
@@ -672,12 +692,13 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
 cudaError_t launch_gemm_simt(bool bf16m, const GemmArgs& a, cudaStream_t s) {
   if (a.M == 0 || a.N == 0) return cudaSuccess;
   dim3 grid((a.N + 63) / 64, (a.M + 63) / 64);
-  if (bf16m && a.a_f32)
-    gemm_simt_kernel<float, bf16><<<grid, 256, 0, s>>>(a);
-  else if (bf16m)
-    gemm_simt_kernel<bf16, bf16><<<grid, 256, 0, s>>>(a);
-  else
-    gemm_simt_kernel<float, float><<<grid, 256, 0, s>>>(a);
+  if (bf16m && a.a_f32) {
+    if (cudaError_t e_ = launch_k(gemm_simt_kernel<float, bf16>, grid, 256, 0, s, a)) return e_;
+  } else if (bf16m) {
+    if (cudaError_t e_ = launch_k(gemm_simt_kernel<bf16, bf16>, grid, 256, 0, s, a)) return e_;
+  } else {
+    if (cudaError_t e_ = launch_k(gemm_simt_kernel<float, float>, grid, 256, 0, s, a)) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -798,6 +819,8 @@ constexpr int ATT_BK = 16;     // keys per staged tile
 
 template <typename T, int HD>
 __global__ void __launch_bounds__(ATT_ROWS) enc_attn_simt_kernel(EncAttnArgs a) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   __shared__ __align__(16) float Ks[ATT_BK][HD];
   __shared__ __align__(16) float Vs[ATT_BK][HD];
   EncTile tile = a.tiles[blockIdx.x];
@@ -829,6 +852,8 @@ __global__ void __launch_bounds__(ATT_ROWS) enc_attn_simt_kernel(EncAttnArgs a) 
 
 template <typename T, int HD>
 __global__ void __launch_bounds__(ATT_ROWS) dec_attn_simt_kernel(DecAttnArgs a) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   __shared__ __align__(16) float Ks[ATT_BK][HD];
   __shared__ __align__(16) float Vs[ATT_BK][HD];
   DecTile tile = a.tiles[blockIdx.x];
@@ -858,9 +883,9 @@ template <typename T>
 static cudaError_t enc_dispatch(int hd, const EncAttnArgs& a, cudaStream_t s) {
   dim3 grid(a.n_tiles, a.n_heads);
   switch (hd) {
-    case 16: enc_attn_simt_kernel<T, 16><<<grid, ATT_ROWS, 0, s>>>(a); break;
-    case 32: enc_attn_simt_kernel<T, 32><<<grid, ATT_ROWS, 0, s>>>(a); break;
-    case 64: enc_attn_simt_kernel<T, 64><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    case 16: if (cudaError_t e_ = launch_k(enc_attn_simt_kernel<T, 16>, grid, ATT_ROWS, 0, s, a)) return e_; break;
+    case 32: if (cudaError_t e_ = launch_k(enc_attn_simt_kernel<T, 32>, grid, ATT_ROWS, 0, s, a)) return e_; break;
+    case 64: if (cudaError_t e_ = launch_k(enc_attn_simt_kernel<T, 64>, grid, ATT_ROWS, 0, s, a)) return e_; break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -870,9 +895,9 @@ template <typename T>
 static cudaError_t dec_dispatch(int hd, const DecAttnArgs& a, cudaStream_t s) {
   dim3 grid(a.n_tiles, a.n_heads);
   switch (hd) {
-    case 16: dec_attn_simt_kernel<T, 16><<<grid, ATT_ROWS, 0, s>>>(a); break;
-    case 32: dec_attn_simt_kernel<T, 32><<<grid, ATT_ROWS, 0, s>>>(a); break;
-    case 64: dec_attn_simt_kernel<T, 64><<<grid, ATT_ROWS, 0, s>>>(a); break;
+    case 16: if (cudaError_t e_ = launch_k(dec_attn_simt_kernel<T, 16>, grid, ATT_ROWS, 0, s, a)) return e_; break;
+    case 32: if (cudaError_t e_ = launch_k(dec_attn_simt_kernel<T, 32>, grid, ATT_ROWS, 0, s, a)) return e_; break;
+    case 64: if (cudaError_t e_ = launch_k(dec_attn_simt_kernel<T, 64>, grid, ATT_ROWS, 0, s, a)) return e_; break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -881,6 +906,8 @@ static cudaError_t dec_dispatch(int hd, const DecAttnArgs& a, cudaStream_t s) {
 // Split-key decoder: out = (sum_s 2^(m_s - M) O_s) / (sum_s 2^(m_s - M) l_s) * g,
 // M = max_s m_s; one thread per 4 output columns of a row.
 __global__ void dec_combine_kernel(DecAttnArgs a, int hd) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int cols4 = a.d / 4;
   if (gid >= a.nk_rows * cols4) return;
@@ -917,7 +944,7 @@ cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s) {
   const long long n = a.nk_rows * (a.d / 4);
   if (n == 0) return cudaSuccess;
   const int threads = 256;
-  dec_combine_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, s>>>(a, hd);
+  if (cudaError_t e_ = launch_k(dec_combine_kernel, (unsigned)((n + threads - 1) / threads), threads, 0, s, a, hd)) return e_;
   return cudaGetLastError();
 }
 

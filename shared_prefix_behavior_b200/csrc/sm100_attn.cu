@@ -208,6 +208,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tslot;
+  pdl_wait();  // the previous kernel of the stream has completed: its outputs may be read
+  pdl_release();
 
   if (warp < 4) {
     setmaxnreg_dec72();
@@ -576,7 +578,7 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
   DecAttnArgs d0 = da ? *da : DecAttnArgs{};
   const int n_cta = DEC ? da->n_cta : ea->n_cta;
   if (n_cta <= 0) return cudaErrorInvalidValue;
-  attn_tc_kernel<HD, MODE><<<n_cta, NTHREADS, smem, s>>>(mq, mk, mv, e0, d0, err);
+  if (cudaError_t e_ = launch_k(attn_tc_kernel<HD, MODE>, n_cta, NTHREADS, smem, s, mq, mk, mv, e0, d0, err)) return e_;
   return cudaGetLastError();
 }
 

@@ -358,6 +358,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or complete_tx
   tc_fence_after();
   const uint32_t tmem = tslot;
+  pdl_wait();  // the previous kernel of the stream has completed: its outputs may be read
+  pdl_release();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA producer (both CTAs)
@@ -592,11 +594,13 @@ cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   constexpr int smem = STAGES * STAGE_BYTES + NSLOT * SLOT + 1024;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait()
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -622,6 +626,7 @@ cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   if (grouped(a)) n_tiles_n = a.groups * tiles_per_group(a);
   const int n_tiles = n_tiles_n * ((a.M + 2 * BM - 1) / (2 * BM));
   cfg.gridDim = dim3(2 * (n_tiles < max_pairs ? n_tiles : max_pairs));
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, mp, a, a.K / BK, n_tiles_n, n_tiles, err);
 }
 
