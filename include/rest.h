@@ -71,10 +71,24 @@ typedef struct {
   const int32_t* cu_seqlens;  /* host [n_users+1]; cu_seqlens[0] == 0, non-decreasing */
 } rest_batch;
 
+/* Gates of the attention sublayer. The DGA layer gates the value stream and
+ * the attention output (eqs. 3-4). The other two are the variants of the
+ * page's gated-attention ablation (§4 ablations, "gated attention"): the
+ * output gate alone, and gates on Q, K and V as well as the output, with
+ * q = sigmoid(y W_gq) * (y W_Q) and k = sigmoid(y W_gk) * (y W_K) taken
+ * before the rotation of eq. 5 (so that scores still depend only on the
+ * index difference, eq. 14). */
+typedef enum {
+  REST_GATES_VALUE_OUTPUT = 0, /* w_qkvgg [d, 5d]: W_Q | W_K | W_V | W_gv | W_go */
+  REST_GATES_OUTPUT = 1,       /* w_qkvgg [d, 4d]: W_Q | W_K | W_V | W_go */
+  REST_GATES_QKV_OUTPUT = 2    /* w_qkvgg [d, 7d]: W_Q | W_K | W_V | W_gv | W_go | W_gq | W_gk */
+} rest_gates;
+
 /* One encoder layer (Fig. 1 left): a DGA sublayer and an optional SwiGLU FFN
  * sublayer, each wrapped by SRN (eq. 6). Weights have the dtype of the call. */
 typedef struct {
-  const void* w_qkvgg;   /* dev [d, 5d]: column blocks W_Q | W_K | W_V | W_gv | W_go (eqs. 3-4) */
+  const void* w_qkvgg;   /* dev [d, 5d]: column blocks W_Q | W_K | W_V | W_gv | W_go (eqs. 3-4);
+                            other widths and blocks with the gate variants (rest_gates) */
   const void* w_o;       /* dev [d, d] */
   const void* w_ffn13;   /* dev [d, 2*d_ff]: W_1 | W_3, or NULL for an attention-only layer */
   const void* w_ffn2;    /* dev [d_ff, d] (ignored when w_ffn13 is NULL) */
@@ -85,6 +99,7 @@ typedef struct {
   float alpha_attn;      /* SRN residual scale of each sublayer */
   float alpha_ffn;
   int d_ff;              /* FFN width, a multiple of 64 (0 without FFN) */
+  int gates;             /* a rest_gates value; 0 is the DGA layer */
 } rest_enc_layer;
 
 /* Cross-decoder parameters (§3.3): token-specific W_Q and W_go (eq. 8), a

@@ -72,20 +72,38 @@ def softmax_list(scores):
     return [v / tot for v in e]
 
 
+def weight_blocks(lay, d):
+    """The attention projection's d-wide column blocks by name: W_Q, W_K, W_V,
+    then the gates the layer has (value + output by default; output only;
+    or value, output, Q and K), in that order."""
+    order = {"vo": "q k v gv go", "o": "q k v go", "qkvo": "q k v gv go gq gk"}[lay.get("gates", "vo")].split()
+    W = np.asarray(lay["w_qkvgg"], dtype=np.float64)
+    return {name: W[:, i * d:(i + 1) * d] for i, name in enumerate(order)}
+
+
+def gate_mul(vec, gate_pre):
+    """vec * sigmoid(gate_pre), element by element."""
+    return np.array([vec[c] * sig(gate_pre[c]) for c in range(len(vec))])
+
+
 def dga(yrows, idx, cu_seqlens, lay, H, base):
     d = len(yrows[0])
     hd = d // H
-    W = np.asarray(lay["w_qkvgg"], dtype=np.float64)
-    Wq, Wk, Wv, Wgv, Wgo = (W[:, i * d:(i + 1) * d] for i in range(5))
+    Wb = weight_blocks(lay, d)
     out = []
     for u in range(len(cu_seqlens) - 1):
         s, e = int(cu_seqlens[u]), int(cu_seqlens[u + 1])
-        q = [matvec(yrows[i], Wq) for i in range(s, e)]
-        k = [matvec(yrows[i], Wk) for i in range(s, e)]
-        v = [matvec(yrows[i], Wv) for i in range(s, e)]
-        gv = [matvec(yrows[i], Wgv) for i in range(s, e)]
-        go = [matvec(yrows[i], Wgo) for i in range(s, e)]
-        vg = [np.array([v[i][c] * sig(gv[i][c]) for c in range(d)]) for i in range(e - s)]
+        q = [matvec(yrows[i], Wb["q"]) for i in range(s, e)]
+        k = [matvec(yrows[i], Wb["k"]) for i in range(s, e)]
+        v = [matvec(yrows[i], Wb["v"]) for i in range(s, e)]
+        go = [matvec(yrows[i], Wb["go"]) for i in range(s, e)]
+        if "gq" in Wb:  # Q and K gated before they are rotated
+            q = [gate_mul(q[i], matvec(yrows[s + i], Wb["gq"])) for i in range(e - s)]
+            k = [gate_mul(k[i], matvec(yrows[s + i], Wb["gk"])) for i in range(e - s)]
+        if "gv" in Wb:
+            vg = [gate_mul(v[i], matvec(yrows[s + i], Wb["gv"])) for i in range(e - s)]
+        else:
+            vg = [np.array(v[i]) for i in range(e - s)]
         for n in range(e - s):
             o = np.zeros(d)
             for h in range(H):
@@ -168,8 +186,11 @@ def encoder_stream(inp, cached):
                 post = l <= inp["l_switch"]
                 g, b, a = lay["ln_attn_g"], lay["ln_attn_b"], float(lay["alpha_attn"])
                 y = x if post else ln_row(x, g, b)
-                W = np.asarray(lay["w_qkvgg"], dtype=np.float64)
-                q, k, v, gv, go = (matvec(y, W[:, c * d:(c + 1) * d]) for c in range(5))
+                Wb = weight_blocks(lay, d)
+                q, k, v, go = (matvec(y, Wb[n]) for n in ("q", "k", "v", "go"))
+                if "gq" in Wb:
+                    q, k = gate_mul(q, matvec(y, Wb["gq"])), gate_mul(k, matvec(y, Wb["gk"]))
+                vgt = gate_mul(v, matvec(y, Wb["gv"])) if "gv" in Wb else np.array(v)
                 qr, kr = np.zeros(d), np.zeros(d)
                 for h in range(H):
                     sl = slice(h * hd, (h + 1) * hd)
@@ -177,7 +198,7 @@ def encoder_stream(inp, cached):
                     qr[sl] = R @ q[sl]
                     kr[sl] = R @ k[sl]
                 kc[l - 1].append(kr)
-                vc[l - 1].append(np.array([v[c] * sig(gv[c]) for c in range(d)]))
+                vc[l - 1].append(vgt)
                 o = np.zeros(d)
                 for h in range(H):
                     sl = slice(h * hd, (h + 1) * hd)

@@ -151,6 +151,14 @@ def _f64(a):
     return np.asarray(a, dtype=np.float64)
 
 
+# Column blocks of the attention projection weight for each choice of gates:
+# the DGA layer (value and output gates, eqs. 3-4) and the two variants of the
+# page's gated-attention ablation (output gate alone; Q, K, V and output).
+GATE_BLOCKS = {"vo": ("q", "k", "v", "gv", "go"),
+               "o": ("q", "k", "v", "go"),
+               "qkvo": ("q", "k", "v", "gv", "go", "gq", "gk")}
+
+
 def dga_sublayer(y: np.ndarray, phi: np.ndarray, cu_seqlens: np.ndarray, layer: dict,
                  n_heads: int, gates: bool = True, row_chunk: int = 2048,
                  kv_out: Optional[list] = None) -> np.ndarray:
@@ -159,16 +167,25 @@ def dga_sublayer(y: np.ndarray, phi: np.ndarray, cu_seqlens: np.ndarray, layer: 
     Readings: no biases; the gates are full d x d projections applied
     elementwise; head h owns columns h*d_h..(h+1)*d_h-1; the score scale is
     1/sqrt(d_h) (eq. 7's multi-head form; eq. 3 is written single-head).
-    ``gates=False`` replaces both sigmoids by 1 (test knob). When ``kv_out``
+    ``layer["gates"]`` picks the gates ("vo" when absent, see GATE_BLOCKS);
+    with Q and K gates, the gated projections are what eq. 5 rotates, so the
+    scores keep eq. 14's dependence on the index difference alone.
+    ``gates=False`` replaces every sigmoid by 1 (test knob). When ``kv_out``
     is a list, the rotated keys R k and the gated values V' of every row (the
     operands later queries attend to) are appended to it as a pair.
     """
     T, d = y.shape
     hd = d // n_heads
     W = _f64(layer["w_qkvgg"])
-    P5 = y @ W
-    Q, Kx, V, Gv, Go = (P5[:, i * d:(i + 1) * d] for i in range(5))
-    Vg = V * sigmoid(Gv) if gates else V
+    names = GATE_BLOCKS[layer.get("gates", "vo")]
+    P = y @ W
+    blk = {n: P[:, i * d:(i + 1) * d] for i, n in enumerate(names)}
+    Q, Kx, V = blk["q"], blk["k"], blk["v"]
+    if gates and "gq" in blk:
+        Q = Q * sigmoid(blk["gq"])
+        Kx = Kx * sigmoid(blk["gk"])
+    Vg = V * sigmoid(blk["gv"]) if gates and "gv" in blk else V
+    Go = blk["go"]
     Qr, Kr = rotate(Q, phi), rotate(Kx, phi)
     if kv_out is not None:
         kv_out.append((Kr, Vg))

@@ -26,6 +26,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librest_b200.so")
 
 REST_F32, REST_BF16 = 0, 1
+# attention-sublayer gates (rest_gates): value + output (the DGA layer), output only, Q/K/V + output
+GATES = {"vo": 0, "o": 1, "qkvo": 2}
 STATUS = {0: "REST_OK", 1: "REST_ERR_INVALID_ARG", 2: "REST_ERR_UNSORTED_TIME", 3: "REST_ERR_UNSUPPORTED",
           4: "REST_ERR_CUDA", 5: "REST_ERR_TIMEOUT", 6: "REST_ERR_WORKSPACE", 7: "REST_ERR_NO_DEVICE"}
 EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
@@ -53,7 +55,7 @@ class Batch(ctypes.Structure):
 class EncLayer(ctypes.Structure):
     _fields_ = [("w_qkvgg", c_void_p), ("w_o", c_void_p), ("w_ffn13", c_void_p), ("w_ffn2", c_void_p),
                 ("ln_attn_g", c_void_p), ("ln_attn_b", c_void_p), ("ln_ffn_g", c_void_p), ("ln_ffn_b", c_void_p),
-                ("alpha_attn", c_float), ("alpha_ffn", c_float), ("d_ff", c_int)]
+                ("alpha_attn", c_float), ("alpha_ffn", c_float), ("d_ff", c_int), ("gates", c_int)]
 
 
 class DecParams(ctypes.Structure):
@@ -168,7 +170,7 @@ def _enc_layers(layers: Sequence[dict]):
         arr[i] = EncLayer(_ptr(L["w_qkvgg"]), _ptr(L["w_o"]), _ptr(L["w_ffn13"]) if ffn else None,
                           _ptr(L["w_ffn2"]) if ffn else None, _ptr(L["ln_attn_g"]), _ptr(L["ln_attn_b"]),
                           _ptr(L["ln_ffn_g"]), _ptr(L["ln_ffn_b"]), float(L["alpha_attn"]), float(L["alpha_ffn"]),
-                          int(L["w_ffn13"].shape[1] // 2) if ffn else 0)
+                          int(L["w_ffn13"].shape[1] // 2) if ffn else 0, GATES[L.get("gates", "vo")])
     return arr
 
 
@@ -491,6 +493,7 @@ def to_device(inp: dict, device) -> dict:
         layers.append({
             "w_qkvgg": dev(L["w_qkvgg"]), "w_o": dev(L["w_o"]), "w_ffn13": dev(L["w_ffn13"]),
             "w_ffn2": dev(L["w_ffn2"]), "alpha_attn": L["alpha_attn"], "alpha_ffn": L["alpha_ffn"],
+            "gates": L.get("gates", "vo"),
             **{k: dev(L[k], torch.float32) for k in ("ln_attn_g", "ln_attn_b", "ln_ffn_g", "ln_ffn_b")},
         })
     return {

@@ -70,6 +70,14 @@ enum Epilogue {
   EPI_DECQG = 6     // decoder token-specific projections, all token types in one launch:
                     // q[n, k] = z[n, k] W_Q^(k) -> out0, sigmoid(z[n, k] W_go^(k)) -> out1
 };
+// Gates of the DGA projection (EPI_QKVG), with the column blocks of its weight:
+//   GATES_VO    Q | K | V | Gv | Go             value and output gates (the DGA layer)
+//   GATES_O     Q | K | V | Go                  output gate only
+//   GATES_QKVO  Q | K | V | Gv | Go | Gq | Gk   gates on Q, K, V and the output;
+//               Q and K are gated before the rotation
+enum GateMode { GATES_VO = 0, GATES_O = 1, GATES_QKVO = 2 };
+inline int gate_blocks(int mode) { return mode == GATES_O ? 4 : mode == GATES_QKVO ? 7 : 5; }
+
 struct GemmArgs {
   const void* A; long long lda;   // [M, K], row stride lda elements
   const void* B; long long ldb;   // [K, N] row-major, row stride ldb elements
@@ -89,10 +97,12 @@ struct GemmArgs {
   // groups' weights stacked) and writes output columns [g W, g W + W), W the
   // output width (d_ff, resp. N). 0 or 1: one product.
   int groups;
+  int gate_mode;                  // EPI_QKVG: a GateMode
 };
-// Logical output columns of EPI_QKVG are [Q | K | V,Gv interleaved | Go] and of
-// EPI_SWIGLU [W1,W3 interleaved]: every group of 4 logical columns holds
-// columns (2p, 2p+1) of the first block then of the second.
+// Logical output columns of EPI_QKVG are [Q | K | V,Gv interleaved | Go]
+// (GATES_O: [Q | K | V | Go]; GATES_QKVO: [Q,Gq | K,Gk | V,Gv interleaved | Go])
+// and of EPI_SWIGLU [W1,W3 interleaved]: every group of 4 interleaved logical
+// columns holds columns (2p, 2p+1) of the first block then of the second.
 cudaError_t launch_gemm_simt(bool bf16, const GemmArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention

@@ -59,6 +59,7 @@ static rest_status check_layers(const rest_enc_layer* layers, int n_layers, int 
     if (!aligned16(L.w_qkvgg) || !aligned16(L.w_o) || !aligned16(L.ln_attn_g) || !aligned16(L.ln_attn_b))
       return REST_ERR_INVALID_ARG;
     if (!isfinite(L.alpha_attn) || !isfinite(L.alpha_ffn)) return REST_ERR_INVALID_ARG;
+    if (L.gates != GATES_VO && L.gates != GATES_O && L.gates != GATES_QKVO) return REST_ERR_INVALID_ARG;
     if (L.w_ffn13) {
       if (!L.w_ffn2 || !L.ln_ffn_g || !L.ln_ffn_b || L.d_ff <= 0 || L.d_ff % 64 != 0 || L.d_ff > 16384)
         return REST_ERR_INVALID_ARG;
@@ -592,8 +593,9 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
     const Sub& S = subs[i];
     const rest_enc_layer& Ly = layers[S.layer];
     if (S.attn) {  // DGA sublayer (eqs. 3-5)
-      GemmArgs a = gemm(a_in, d, Ly.w_qkvgg, 5LL * d, T, 5 * d, d, EPI_QKVG, q, d);
-      a.out1 = k; a.out2 = v; a.out3 = g; a.cos_t = cos_t; a.sin_t = sin_t; a.d = d;
+      const int nb = gate_blocks(Ly.gates);  // column blocks of the projection weight
+      GemmArgs a = gemm(a_in, d, Ly.w_qkvgg, (long long)nb * d, T, nb * d, d, EPI_QKVG, q, d);
+      a.out1 = k; a.out2 = v; a.out3 = g; a.cos_t = cos_t; a.sin_t = sin_t; a.d = d; a.gate_mode = Ly.gates;
       if (rest_status st = run_gemm(p, a, "gemm_qkvg", s)) return st;
       if (cache) {  // the new rows' R k and V' join the layer's cache; attention reads keys there
         REST_KLAUNCH(s, "append_kv", 0, 4.0 * e * Td,

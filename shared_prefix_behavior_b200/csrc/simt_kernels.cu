@@ -560,20 +560,35 @@ cudaError_t launch_split_bf16(const float* x, void* hi, void* lo, long long n, c
 // ============================================================================
 
 // Physical column of logical column n for the interleaved epilogues: every
-// group of 4 logical columns is (2p, 2p+1) of block one and (2p, 2p+1) of
-// block two, the blocks `width` columns apart starting at `base`.
-__device__ __forceinline__ int interleave_col(int n, int base, int width) {
-  int r = n - base, p = r >> 2, w = r & 3;
-  return base + (w < 2 ? 2 * p + w : width + 2 * p + w - 2);
+// group of 4 logical columns from `lbase` on is (2p, 2p+1) of the block at
+// physical column `pbase`, then (2p, 2p+1) of the block `width` columns after it.
+__device__ __forceinline__ int interleave_col(int n, int lbase, int pbase, int width) {
+  int r = n - lbase, p = r >> 2, w = r & 3;
+  return pbase + (w < 2 ? 2 * p + w : width + 2 * p + w - 2);
 }
 
 __device__ __forceinline__ int physical_col(const GemmArgs& a, int n) {
+  const int d = a.d;
   if (a.epi == EPI_QKVG) {
-    if (n >= 2 * a.d && n < 4 * a.d) return interleave_col(n, 2 * a.d, a.d);
+    if (a.gate_mode == GATES_O) return n;                       // Q | K | V | Go
+    if (a.gate_mode == GATES_QKVO) {                            // Q,Gq | K,Gk | V,Gv | Go
+      if (n < 2 * d) return interleave_col(n, 0, 0, 5 * d);
+      if (n < 4 * d) return interleave_col(n, 2 * d, d, 5 * d);
+      if (n < 6 * d) return interleave_col(n, 4 * d, 2 * d, d);
+      return n - 2 * d;
+    }
+    if (n >= 2 * d && n < 4 * d) return interleave_col(n, 2 * d, 2 * d, d);  // Q | K | V,Gv | Go
     return n;
   }
-  if (a.epi == EPI_SWIGLU) return interleave_col(n, 0, a.d);
+  if (a.epi == EPI_SWIGLU) return interleave_col(n, 0, 0, a.d);
   return n;
+}
+
+// Rotate the pair (x0, x1) of Q or K at column `col` of row m (eq. 5).
+__device__ __forceinline__ void rotate_pair(const GemmArgs& a, long long m, int col, float x0, float x1, float* out) {
+  const float c = a.cos_t[m * (a.d / 2) + col / 2], s = a.sin_t[m * (a.d / 2) + col / 2];
+  out[0] = x0 * c - x1 * s;
+  out[1] = x0 * s + x1 * c;
 }
 
 // TA: type of A; T: the call's dtype (B and the dtype outputs).
@@ -658,6 +673,30 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
       }
       case EPI_QKVG: {
         int d = a.d;
+        if (a.gate_mode == GATES_QKVO) {
+          if (n < 4 * d) {  // gated Q or K pair (2p, 2p+1), then its rotation (eq. 5)
+            const int blk = n < 2 * d ? 0 : 1, col = ((n - 2 * d * blk) >> 2) * 2;
+            float v[2];
+            rotate_pair(a, m, col, c[0] * sigmoid_f(c[2]), c[1] * sigmoid_f(c[3]), v);
+            store2((T*)(blk == 0 ? a.out0 : a.out1) + ro + col, v[0], v[1]);
+          } else if (n < 6 * d) {  // value gate
+            int col = ((n - 4 * d) >> 2) * 2;
+            store2((T*)a.out2 + ro + col, c[0] * sigmoid_f(c[2]), c[1] * sigmoid_f(c[3]));
+          } else {  // output gate
+            float v[4] = {sigmoid_f(c[0]), sigmoid_f(c[1]), sigmoid_f(c[2]), sigmoid_f(c[3])};
+            store4((float*)a.out3 + ro + (n - 6 * d), v);
+          }
+          break;
+        }
+        if (a.gate_mode == GATES_O && n >= 2 * d) {
+          if (n < 3 * d) {  // V without a gate
+            store4((T*)a.out2 + ro + (n - 2 * d), c);
+          } else {  // output gate
+            float v[4] = {sigmoid_f(c[0]), sigmoid_f(c[1]), sigmoid_f(c[2]), sigmoid_f(c[3])};
+            store4((float*)a.out3 + ro + (n - 3 * d), v);
+          }
+          break;
+        }
         if (n < 2 * d) {  // Q or K: rotate the pairs (eq. 5)
           int col = n < d ? n : n - d;
           const float* ct = a.cos_t + (long long)m * (d / 2) + col / 2;

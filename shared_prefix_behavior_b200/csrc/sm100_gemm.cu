@@ -60,9 +60,9 @@ struct GemmMaps {
 };
 
 // Width (MMA N) of the tiles: 256 columns (128 per CTA of the pair), 128 for
-// the plain bf16 copy. EPI_QKVG tiles: [0, nH) rotated Q and K of head group
-// t (128 columns each), [nH, 2 nH) V and Gv, then Go in 256-column tiles,
-// with nH = d / 128.
+// the plain bf16 copy. EPI_QKVG tiles (DGA gates): [0, nH) rotated Q and K of
+// head group t (128 columns each), [nH, 2 nH) V and Gv, then Go in 256-column
+// tiles, with nH = d / 128; the gate variants are laid out by qkvg_tiles().
 __host__ __device__ __forceinline__ int tile_n(const GemmArgs& a) { return a.epi == EPI_DT ? 128 : 256; }
 // Output columns of a 256-column tile of an fp32 output; the last tile may end past the width.
 __host__ __device__ __forceinline__ int f32_tiles(int width) { return (width + 255) / 256; }
@@ -75,16 +75,44 @@ __host__ __device__ __forceinline__ bool grouped(const GemmArgs& a) {
   return a.groups > 1 && (a.epi == EPI_SWIGLU || a.epi == EPI_RESID || a.epi == EPI_F32);
 }
 
+// N-tiles of the DGA projection by gate mode: rotation tiles [0, rot_end),
+// value tiles [rot_end, val_end), output-gate tiles after. A rotation tile is
+// Q | K of head group t (128 columns each), or with GATES_QKVO X | G_X, X = Q
+// for t < nH and K after; a value tile is V | Gv (128 columns each), or 256
+// columns of V with GATES_O.
+struct QkvgTiles {
+  int nH, rot_end, val_end;
+};
+__host__ __device__ __forceinline__ QkvgTiles qkvg_tiles(const GemmArgs& a) {
+  QkvgTiles q;
+  q.nH = a.d / 128;
+  q.rot_end = a.gate_mode == GATES_QKVO ? 2 * q.nH : q.nH;
+  q.val_end = q.rot_end + (a.gate_mode == GATES_O ? (a.d + 255) / 256 : q.nH);
+  return q;
+}
+// First column of the output-gate block W_go in the projection weight.
+__host__ __device__ __forceinline__ int go_col(const GemmArgs& a) { return (a.gate_mode == GATES_O ? 3 : 4) * a.d; }
+
 // Global column (in the B map that box_map selects) of the 64-column box b
 // that CTA `rank` loads for N-tile t.
 __device__ __forceinline__ int b_box_col(const GemmArgs& a, int t, int rank, int b, bool* second_map) {
   *second_map = false;
   if (a.epi == EPI_QKVG) {
-    const int d = a.d, nH = d / 128;
-    if (t < nH) return (rank ? d : 0) + t * 128 + 64 * b;                   // Q | K
-    if (t < 2 * nH) return (rank ? 3 * d : 2 * d) + (t - nH) * 128 + 64 * b;  // V | Gv
-    *second_map = true;                                                     // Go, through its [K, d] view
-    return (t - 2 * nH) * 256 + 128 * rank + 64 * b;
+    const int d = a.d;
+    const QkvgTiles g = qkvg_tiles(a);
+    if (t < g.rot_end) {
+      if (a.gate_mode == GATES_QKVO) {  // Q | Gq or K | Gk
+        const int k = t >= g.nH ? 1 : 0;
+        return (rank ? (5 + k) * d : k * d) + (t - k * g.nH) * 128 + 64 * b;
+      }
+      return (rank ? d : 0) + t * 128 + 64 * b;  // Q | K
+    }
+    if (t < g.val_end) {
+      if (a.gate_mode == GATES_O) return 2 * d + (t - g.rot_end) * 256 + 128 * rank + 64 * b;  // V
+      return (rank ? 3 * d : 2 * d) + (t - g.rot_end) * 128 + 64 * b;                          // V | Gv
+    }
+    *second_map = true;  // Go, through its [K, d] view
+    return (t - g.val_end) * 256 + 128 * rank + 64 * b;
   }
   if (grouped(a)) t %= tiles_per_group(a);  // the group's rows of B come from the K offset
   if (a.epi == EPI_SWIGLU) {  // W_1 | W_3, each through its own [K, d_ff] view
@@ -173,8 +201,35 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     __syncwarp();
     if (lane == 0) mbar_arrive_cluster(acc_empty_addr);
   };
-  const int nH = a.d / 128;
-  if (a.epi == EPI_QKVG && t < nH) {
+  const QkvgTiles qt = qkvg_tiles(a);
+  if (a.epi == EPI_QKVG && t < qt.rot_end && a.gate_mode == GATES_QKVO) {
+    // X = Q or K of head group t % nH, gated by sigmoid(G_X), then rotated; this warp
+    // takes pairs [32 part, 32 part + 32), and the output takes the bytes of the cos values
+    uint8_t* cb = slot + part * BOX128;
+    const uint8_t* sb = slot + (2 + part) * BOX128;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      tmem_ld32x2(trow + part * 64 + 32 * j, v, trow + 128 + part * 64 + 32 * j, w);  // X and G_X columns
+      if (j == 1) release();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= sigmoid_fast(w[i]);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t off = sw128_off(r, 4 * j + kk);
+        const float4 c = *reinterpret_cast<const float4*>(cb + off);
+        const float4 s = *reinterpret_cast<const float4*>(sb + off);
+        *reinterpret_cast<uint4*>(cb + off) = rotate4(v + 8 * kk, c, s);
+      }
+    }
+    issue();
+    if (lane == 0) {
+      const int k = t >= qt.nH ? 1 : 0;
+      tma_store_2d(&mp.o[k], cb + q * 32 * 128, (t - k * qt.nH) * 128 + 64 * part, y0);
+      bulk_commit();
+    }
+    return;
+  }
+  if (a.epi == EPI_QKVG && t < qt.rot_end) {
     // rotated Q and K of head group t; this warp takes pairs [32 part, 32 part + 32) of both,
     // and the outputs take the bytes of the cos (Q) and sin (K) values they were made from
     uint8_t* cb = slot + part * BOX128;
@@ -202,7 +257,27 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     }
     return;
   }
-  if ((a.epi == EPI_QKVG && t < 2 * nH) || a.epi == EPI_SWIGLU) {
+  if (a.epi == EPI_QKVG && t < qt.val_end && a.gate_mode == GATES_O) {
+    // V without a gate: this warp's 128 accumulator columns as bf16, in two 64-column boxes
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      tmem_ld32(trow + part * 128 + 32 * c, v);
+      if (c == 3) release();
+      if (c == 0) slot_ready();
+      stage_bf16_sw128(slot + (2 * part + (c >> 1)) * BOX128, r, 4 * (c & 1), v);
+    }
+    issue();
+    if (lane == 0) {
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx) {
+        const int x = (t - qt.rot_end) * 256 + 128 * part + 64 * bx;
+        if (x < a.d) tma_store_2d(&mp.o[2], slot + (2 * part + bx) * BOX128 + q * 32 * 128, x, y0);
+      }
+      bulk_commit();
+    }
+    return;
+  }
+  if ((a.epi == EPI_QKVG && t < qt.val_end) || a.epi == EPI_SWIGLU) {
     // V' = sigmoid(Gv) * V (eq. 3) or SiLU(x W_1) * (x W_3): accumulator columns
     // [0, 128) and [128, 256) pair up; this warp makes output columns [64 part, 64 part + 64)
     const bool gate = a.epi == EPI_QKVG;
@@ -229,7 +304,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
       }
     }
     issue();
-    const int tl = gate ? t - nH : grouped(a) ? t % tiles_per_group(a) : t;
+    const int tl = gate ? t - qt.rot_end : grouped(a) ? t % tiles_per_group(a) : t;
     const int gofs = gate || !grouped(a) ? 0 : (t / tiles_per_group(a)) * a.d;
     const int x = tl * 128 + 64 * part;
     if (lane == 0 && x < a.d) {  // the last SwiGLU tile may end past d_ff
@@ -268,7 +343,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
   bool sig = a.epi == EPI_SIGMOID;
   if (a.epi == EPI_QKVG) {
     om = &mp.o[3];
-    x0 = (t - 2 * nH) * 256;
+    x0 = (t - qt.val_end) * 256;
     width = a.d;
     sig = true;
   } else if (a.epi == EPI_DECQG) {  // tile t: group g (q of token k = g, or the gate of token k = g - k_tok), N-tile nt
@@ -335,7 +410,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = (int)cluster_rank();
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-  const int nH = a.d / 128;
+  const QkvgTiles qt = qkvg_tiles(a);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -410,13 +485,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m0 = (tile / n_tiles_n) * 2 * BM + rank * BM;
       const int s = i & 1;
       if (!mbar_wait(&side_empty[s], ((i >> 1) & 1) ^ 1, err, &abort_flag)) break;
-      if (t < nH) {
+      if (t < qt.rot_end) {
+        const int hg = t % qt.nH;  // head group of the tile's columns
         uint8_t* sl = slots + s * SLOT;
         mbar_arrive_expect_tx(&side_full[s], 4 * BOX128);
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
-          tma_load_2d(sl + p * BOX128, &mp.s0, t * 64 + 32 * p, m0, &side_full[s]);
-          tma_load_2d(sl + (2 + p) * BOX128, &mp.s1, t * 64 + 32 * p, m0, &side_full[s]);
+          tma_load_2d(sl + p * BOX128, &mp.s0, hg * 64 + 32 * p, m0, &side_full[s]);
+          tma_load_2d(sl + (2 + p) * BOX128, &mp.s1, hg * 64 + 32 * p, m0, &side_full[s]);
         }
         side_issued = i + 1;
       } else {
@@ -556,7 +632,7 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
       mp.b2 = mp.b;
       // the output-gate block W_go as its own [K, d] view (a ragged last Go tile reads zeros)
       if (ok && a.epi == EPI_QKVG)
-        ok = make_tmap(&mp.b2, false, static_cast<const bf16*>(a.B) + 4LL * a.d, a.K, a.d, a.ldb, 64, BK, 128);
+        ok = make_tmap(&mp.b2, false, static_cast<const bf16*>(a.B) + go_col(a), a.K, a.d, a.ldb, 64, BK, 128);
     }
   }
   if (!ok) return false;
@@ -620,7 +696,7 @@ cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t s, int32_t* err) {
   }
   int n_tiles_n = f32_tiles(a.N);
   if (a.epi == EPI_DT) n_tiles_n = a.N / 128;
-  if (a.epi == EPI_QKVG) n_tiles_n = 2 * (a.d / 128) + f32_tiles(a.d);
+  if (a.epi == EPI_QKVG) n_tiles_n = qkvg_tiles(a).val_end + f32_tiles(a.d);
   if (a.epi == EPI_SWIGLU) n_tiles_n = (a.d + 127) / 128;
   if (a.epi == EPI_DECQG) n_tiles_n = 2 * a.k_tok * f32_tiles(a.N);
   if (grouped(a)) n_tiles_n = a.groups * tiles_per_group(a);
@@ -642,7 +718,8 @@ bool sm100_gemm_supported(const GemmArgs& a) {
   if (a.M <= 0 || a.K % BK != 0 || a.K <= 0) return false;
   if ((a.lda % 8) || (a.ldb % 8) || (a.ldo % 8)) return false;
   switch (a.epi) {
-    case EPI_QKVG: return a.d % 128 == 0 && a.N == 5 * a.d && a.ldb == 5LL * a.d;
+    case EPI_QKVG:
+      return a.d % 128 == 0 && a.N == gate_blocks(a.gate_mode) * a.d && a.ldb == (long long)a.N;
     case EPI_SWIGLU: return a.d % 64 == 0 && a.N == 2 * a.d && a.ldb == 2LL * a.d;
     case EPI_DECQG: return a.N % 128 == 0 && a.ldb == a.N && a.B2 != nullptr && a.k_tok >= 1;
     default: return a.N % 128 == 0 && a.ldb == a.N;

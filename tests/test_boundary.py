@@ -48,8 +48,9 @@ def _batch(cu):
     return cu, R.Batch(len(cu) - 1, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
 
 
-def _layer(d, dff=0):
-    return R.EncLayer(FAKE, FAKE, FAKE if dff else None, FAKE if dff else None, FAKE, FAKE, FAKE, FAKE, 0.1, 0.1, dff)
+def _layer(d, dff=0, gates=0):
+    return R.EncLayer(FAKE, FAKE, FAKE if dff else None, FAKE if dff else None, FAKE, FAKE, FAKE, FAKE, 0.1, 0.1, dff,
+                      gates)
 
 
 def _enc(dt=R.REST_BF16, taus=(0, 0, 1, 64), d=64, cu=(0, 10, 30), layers=None, l_switch=0, x=FAKE, ts=FAKE,
@@ -93,6 +94,7 @@ INVALID, UNSUPPORTED, WORKSPACE, NO_DEVICE = 1, 3, 6, 7
     (dict(x=FAKE + 4), INVALID),                 # misaligned
     (dict(ts=None), INVALID),
     (dict(layers=[_layer(64, 100)]), INVALID),   # d_ff not a multiple of 64
+    (dict(layers=[_layer(64, 192, 3)]), INVALID),  # no such gate variant
     (dict(base=-1.0), INVALID),
     (dict(d=4 * 24, taus=(0, 0, 1, 64)), UNSUPPORTED),  # head_dim 24
     (dict(ws_bytes=1000), WORKSPACE),

@@ -111,6 +111,21 @@ def test_bf16_small_ragged_rank_request(cuda, hd, n_layers, l_switch, ffn):
     assert_parity(y, yr, "bf16", "y")
 
 
+@pytest.mark.parametrize("dtype,hd,d,gates", [("f32", 16, 64, "o"), ("f32", 32, 128, "qkvo"), ("bf16", 32, 128, "o"),
+                                               ("bf16", 32, 256, "o"), ("bf16", 32, 128, "qkvo"),
+                                               ("bf16", 64, 256, "qkvo")])
+def test_gate_variants_small_ragged(cuda, dtype, hd, d, gates):
+    """The gated-attention ablation's variants (output gate only; Q, K, V and
+    output gates) through the whole forward."""
+    w = W.small_workload(dtype, lengths=(300, 129, 1, 64, 255), d=d, n_heads=d // hd, n_layers=2, l_switch=1,
+                         gates=gates, requests=[(0, 300, 20), (1, 129, 7), (2, 1, 3), (4, 200, 11)])
+    inp = W.make_inputs(w, 61, ln_affine=True)
+    H, y = run_rank(inp, cuda)
+    Hr, yr = O.rank_request(inp)
+    assert_parity(H, Hr, dtype, "H")
+    assert_parity(y, yr, dtype, "y")
+
+
 def test_bf16_decoder_with_synthetic_memory(cuda):
     w = W.small_workload("bf16", lengths=(700, 129, 3), d=256, n_heads=8,
                          requests=[(0, 700, 60), (0, 1, 2), (0, 333, 0), (1, 129, 45), (2, 2, 7), (0, 129, 1)])

@@ -318,6 +318,60 @@ def test_union_encoding_equals_encoding_each_prefix_alone():
     assert rel_err(yc, y[3:6]) < 1e-12
 
 
+# ---------------------------------------------- gate variants (ablation flags)
+
+def gate_inputs(gates, seed, n_rope=2, lengths=(7, 5), n_layers=2):
+    w = W.small_workload("f32", lengths=lengths, d=16, n_heads=4, n_rope=n_rope, n_layers=n_layers, l_switch=1,
+                         alpha=0.5, levels=[7, 600, 86400], ncand=3, duplicate_frac=0.2, gates=gates)
+    return W.make_inputs(w, seed, ln_affine=True)
+
+
+def with_blocks(inp, gates, build):
+    """inp with every layer's projection weight replaced by build(blocks of d columns)."""
+    d = inp["x"].shape[1]
+    layers = []
+    for lay in inp["layers"]:
+        W_ = np.asarray(lay["w_qkvgg"], dtype=np.float64)
+        blocks = [W_[:, i * d:(i + 1) * d] for i in range(W_.shape[1] // d)]
+        layers.append(dict(lay, w_qkvgg=np.concatenate(build(blocks), axis=1), gates=gates))
+    return dict(inp, layers=layers)
+
+
+@pytest.mark.parametrize("gates", ["o", "qkvo"])
+def test_gate_variants_match_literal_brute_force(gates):
+    inp = gate_inputs(gates, 24)
+    assert rel_err(O.encoder(inp), brute.encoder(inp)) < 1e-12
+    Hn, kv, _ = O.encoder_append(inp, [3, 2])
+    Hb, kvb = brute.encoder_stream(inp, [3, 2])
+    assert rel_err(Hn, Hb) < 1e-12
+    for (k, v), (kb, vb) in zip(kv, kvb):
+        assert rel_err(k, kb) < 1e-12 and rel_err(v, vb) < 1e-12
+
+
+def test_output_gate_only_is_dga_with_a_constant_half_value_gate():
+    """sigmoid(0) = 1/2 exactly: the DGA layer with W_gv = 0 and W_V doubled has
+    V' = V, which is the layer with the output gate alone."""
+    inp = gate_inputs("o", 25)
+    same = with_blocks(inp, "vo", lambda b: [b[0], b[1], 2.0 * b[2], 0.0 * b[2], b[3]])
+    assert rel_err(O.encoder(inp), O.encoder(same)) < 1e-14
+
+
+def test_qkv_gates_with_zero_gate_weights_halve_q_and_k():
+    """With W_gq = W_gk = 0 the Q and K gates are the constant 1/2: the DGA
+    layer with W_Q and W_K halved."""
+    inp = with_blocks(gate_inputs("qkvo", 26), "qkvo", lambda b: b[:5] + [0.0 * b[5], 0.0 * b[6]])
+    same = with_blocks(inp, "vo", lambda b: [0.5 * b[0], 0.5 * b[1]] + b[2:5])
+    assert rel_err(O.encoder(inp), O.encoder(same)) < 1e-14
+
+
+def test_qkv_gates_keep_scores_relative_in_position():
+    """Q and K are gated before the rotation, so a global shift of every
+    RoPE position leaves the layer's output unchanged (eq. 14); gating after
+    the rotation would not."""
+    inp = gate_inputs("qkvo", 27, n_rope=4, lengths=(30,), n_layers=1)
+    assert rel_err(O.encoder(inp, pos_offset=12345), O.encoder(inp)) < 1e-10
+
+
 # ------------------------------------------------- append-only encoder cache
 
 def truncate(inp, lengths):

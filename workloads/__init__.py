@@ -85,6 +85,7 @@ class Workload:
     rope_base: float = 10000.0
     duplicate_frac: float = 0.0     # share of positions i>=1 copying token i-1
     span_seconds: Optional[int] = None  # rescale each history to this span
+    gates: str = "vo"               # attention gates: "vo" (DGA), "o" or "qkvo" (ablation variants)
 
     @property
     def n_users(self) -> int:
@@ -173,7 +174,7 @@ def small_workload(dtype: str = "bf16", lengths=(300, 129, 64), d: int = 128, n_
                    n_rope: Optional[int] = None, n_layers: int = 2, l_switch: int = 1,
                    requests=None, ncand: int = 20, alpha: float = 0.1, ffn: bool = True,
                    levels=None, K: int = 3, duplicate_frac: float = 0.05,
-                   name: str = "small") -> Workload:
+                   name: str = "small", gates: str = "vo") -> Workload:
     """A small ragged workload for parity tests (several tiles and a ragged tail).
 
     ``requests`` is a list of (user, cutoff, n_candidates); by default every
@@ -188,7 +189,7 @@ def small_workload(dtype: str = "bf16", lengths=(300, 129, 64), d: int = 128, n_
                     head_taus(n_heads, n_rope, levels or SEVEN_LEVELS), n_layers, alpha, alpha,
                     ffn_width(d) if ffn else 0, l_switch,
                     [r[0] for r in requests], [r[1] for r in requests], [r[2] for r in requests],
-                    K=K, duplicate_frac=duplicate_frac)
+                    K=K, duplicate_frac=duplicate_frac, gates=gates)
 
 
 # --------------------------------------------------------------------------
@@ -240,7 +241,8 @@ def make_inputs(w: Workload, seed: int, ln_affine: bool = False) -> dict:
     layers = []
     for _ in range(w.n_layers):
         lay = {
-            "w_qkvgg": _store(rng.standard_normal((d, 5 * d)) * sd, w.dtype),
+            "w_qkvgg": _store(rng.standard_normal((d, {"vo": 5, "o": 4, "qkvo": 7}[w.gates] * d)) * sd, w.dtype),
+            "gates": w.gates,
             "w_o": _store(rng.standard_normal((d, d)) * sd, w.dtype),
             "w_ffn13": _store(rng.standard_normal((d, 2 * w.d_ff)) * sd, w.dtype) if w.d_ff else None,
             "w_ffn2": _store(rng.standard_normal((w.d_ff, d)) * sd, w.dtype) if w.d_ff else None,
