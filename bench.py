@@ -93,6 +93,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ablation", action="store_true",
+                    help="also time the encoder under the gated-attention and RoTE ablation variants")
     ap.add_argument("--sharing", action="store_true",
                     help="also run the no-sharing variant (every candidate re-encodes its own history)")
     return ap.parse_args()
@@ -426,6 +428,54 @@ def append_comparison(w, inp, dev, full_ms, n_new=64):
     return out
 
 
+def ablation_comparison(w, dev, n=20):
+    """The encoder (rest_encoder_attn) of the same workload under the page's
+    ablation variants: the gates of the attention sublayer (value + output,
+    the DGA layer; output only; Q, K, V and output) and RoTE with a single
+    1-second granularity on every time head. Each variant has its own seeded
+    weights; only its cost is compared here (parity is in the tests). FLOPs
+    are the encoder's algorithmic FLOPs, projections included."""
+    import torch
+    import shared_prefix_behavior_b200 as R
+    out = {}
+    base_ms = None
+    for name, wv in (("dga_value_output", w), ("output_gate_only", dataclasses.replace(w, gates="o")),
+                     ("qkv_output_gates", dataclasses.replace(w, gates="qkvo")),
+                     ("rote_single_1s", dataclasses.replace(w, taus=np.where(w.taus > 0, 1, 0).astype(np.int64)))):
+        inp = W.make_inputs(wv, 1000 + 17)
+        t = R.to_device(inp, dev)
+        H = torch.empty_like(t["x"])
+        ws = torch.empty(R.workspace_size(R.REST_BF16 if wv.dtype == "bf16" else R.REST_F32, t["taus"], wv.d,
+                                          t["cu_seqlens"], t["layers"], rope_base=t["rope_base"]),
+                         dtype=torch.uint8, device=dev)
+
+        def enc(check=False):
+            R.encoder_attn(t["x"], t["ts"], t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"],
+                           rope_base=t["rope_base"], h_out=H, ws=ws, check=check)
+
+        enc(check=True)
+        for _ in range(3):
+            enc()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            enc()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / n
+        nb = {"vo": 5, "o": 4, "qkvo": 7}[wv.gates]
+        T, d = wv.total_tokens, wv.d
+        pairs = sum(L * (L + 1) / 2 for L in wv.lengths)
+        flops = wv.n_layers * (2.0 * T * d * nb * d + 2.0 * T * d * d + 6.0 * T * d * wv.d_ff + 4.0 * d * pairs)
+        if base_ms is None:
+            base_ms, base_flops = ms, flops
+        out[name] = {"gates": wv.gates, "taus": [int(x) for x in wv.taus], "ms": ms,
+                     "tokens_per_s": T / (ms * 1e-3), "time_vs_dga": ms / base_ms, "flops": flops,
+                     "flops_vs_dga": flops / base_flops}
+    return out
+
+
 # --------------------------------------------------------------------- oracle (CPU baseline / reference arm)
 
 def blas_threads() -> int:
@@ -662,6 +712,8 @@ def main():
         parts["sharing"] = sharing_comparison(w, inp, dev, ms_step)
     if world == 1:
         parts["append"] = append_comparison(w, inp, dev, parts["encoder_only"]["ms"])
+    if args.ablation and world == 1:
+        parts["ablation"] = ablation_comparison(w, dev)
 
     if world > 1:
         dist.barrier()
@@ -714,7 +766,7 @@ def main():
         "encoder_only": parts["encoder_only"],
         "decoder_only": parts["decoder_only"],
     }
-    for k in ("sharing", "append"):
+    for k in ("sharing", "append", "ablation"):
         if k in parts:
             out[k] = parts[k]
     if world == 1 and not args.no_cpu_baseline:

@@ -201,8 +201,10 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     __syncwarp();
     if (lane == 0) mbar_arrive_cluster(acc_empty_addr);
   };
+  // SIDE holds exactly for the DGA projection (EPI_QKVG): testing it instead of
+  // a.epi keeps each instantiation's code to its own epilogues
   const QkvgTiles qt = qkvg_tiles(a);
-  if (a.epi == EPI_QKVG && t < qt.rot_end && a.gate_mode == GATES_QKVO) {
+  if (SIDE && t < qt.rot_end && a.gate_mode == GATES_QKVO) {
     // X = Q or K of head group t % nH, gated by sigmoid(G_X), then rotated; this warp
     // takes pairs [32 part, 32 part + 32), and the output takes the bytes of the cos values
     uint8_t* cb = slot + part * BOX128;
@@ -229,7 +231,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     }
     return;
   }
-  if (a.epi == EPI_QKVG && t < qt.rot_end) {
+  if (SIDE && t < qt.rot_end) {
     // rotated Q and K of head group t; this warp takes pairs [32 part, 32 part + 32) of both,
     // and the outputs take the bytes of the cos (Q) and sin (K) values they were made from
     uint8_t* cb = slot + part * BOX128;
@@ -257,7 +259,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     }
     return;
   }
-  if (a.epi == EPI_QKVG && t < qt.val_end && a.gate_mode == GATES_O) {
+  if (SIDE && t < qt.val_end && a.gate_mode == GATES_O) {
     // V without a gate: this warp's 128 accumulator columns as bf16, in two 64-column boxes
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -277,11 +279,11 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     }
     return;
   }
-  if ((a.epi == EPI_QKVG && t < qt.val_end) || a.epi == EPI_SWIGLU) {
+  if ((SIDE && t < qt.val_end) || (!SIDE && a.epi == EPI_SWIGLU)) {
     // V' = sigmoid(Gv) * V (eq. 3) or SiLU(x W_1) * (x W_3): accumulator columns
     // [0, 128) and [128, 256) pair up; this warp makes output columns [64 part, 64 part + 64)
-    const bool gate = a.epi == EPI_QKVG;
-    const bool lo = !gate && a.out1 != nullptr;  // SwiGLU output as a bf16 hi + lo pair (out0, out1)
+    const bool gate = SIDE;
+    const bool lo = !SIDE && a.out1 != nullptr;  // SwiGLU output as a bf16 hi + lo pair (out0, out1)
     uint8_t* box = slot + part * BOX128;
     uint8_t* box_lo = slot + (2 + part) * BOX128;
 #pragma unroll
@@ -304,8 +306,8 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
       }
     }
     issue();
-    const int tl = gate ? t - qt.rot_end : grouped(a) ? t % tiles_per_group(a) : t;
-    const int gofs = gate || !grouped(a) ? 0 : (t / tiles_per_group(a)) * a.d;
+    const int tl = SIDE ? t - qt.rot_end : grouped(a) ? t % tiles_per_group(a) : t;
+    const int gofs = SIDE || !grouped(a) ? 0 : (t / tiles_per_group(a)) * a.d;
     const int x = tl * 128 + 64 * part;
     if (lane == 0 && x < a.d) {  // the last SwiGLU tile may end past d_ff
       tma_store_2d(&mp.o[gate ? 2 : 0], box + q * 32 * 128, gofs + x, y0);
@@ -314,7 +316,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     }
     return;
   }
-  if (a.epi == EPI_DT) {  // bf16 copy of the accumulator
+  if (!SIDE && a.epi == EPI_DT) {  // bf16 copy of the accumulator
     uint8_t* box = slot + part * BOX128;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -335,13 +337,13 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
   // plain, sigmoid, the decoder's q / gate, or the residual add
   const CUtensorMap* om = &mp.o[0];
   int x0 = t * 256, width = a.N;
-  if (grouped(a)) {  // group g writes columns [g N, g N + N)
+  if (!SIDE && grouped(a)) {  // group g writes columns [g N, g N + N)
     const int g = t / tiles_per_group(a);
     x0 = g * a.N + (t % tiles_per_group(a)) * 256;
     width = g * a.N + a.N;
   }
-  bool sig = a.epi == EPI_SIGMOID;
-  if (a.epi == EPI_QKVG) {
+  bool sig = !SIDE && a.epi == EPI_SIGMOID;
+  if (SIDE) {
     om = &mp.o[3];
     x0 = (t - qt.val_end) * 256;
     width = a.d;
@@ -353,7 +355,7 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     width = k * a.N + a.N;
     sig = g >= a.k_tok;
   }
-  const bool resid = a.epi == EPI_RESID;
+  const bool resid = !SIDE && a.epi == EPI_RESID;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     tmem_ld32(trow + part * 128 + 32 * c, v);
@@ -664,6 +666,7 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
 
 template <int STAGES, int NSLOT, int SLOT, bool SIDE>
 cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t s, int32_t* err) {
+  if (SIDE != (a.epi == EPI_QKVG)) return cudaErrorInvalidValue;  // the epilogue relies on it
   GemmMaps mp;
   if (!setup_maps(a, mp)) return cudaErrorInvalidValue;
   auto kern = gemm_tc_kernel<STAGES, NSLOT, SLOT, SIDE>;
