@@ -259,6 +259,73 @@ def encoder(inp: dict, gates: bool = True, angle_scale: float = 1.0,
     return x
 
 
+# --------------------------------------------------------------------------
+# §3.5 ULT: the attention core's forward statistics and its backward
+# --------------------------------------------------------------------------
+
+def attention_core(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens: np.ndarray, n_heads: int):
+    """The causal attention core of a DGA sublayer over packed histories:
+    per user and head, O = softmax(q k^T / sqrt(d_h) + M_causal) V, with q, k
+    the rotated queries and keys and V the gated values V' (eq. 3), and
+    lse[i, h] = log sum_{j <= i} exp(q_i . k_j / sqrt(d_h)), the statistic a
+    backward pass reuses. Returns (O [T, d], lse [T, n_heads]).
+
+    ULT (§3.5) encodes the union history of a user's samples once under a
+    prefix-valid causal mask; since a sample ending at row c reads rows < c
+    and every row i sees rows j <= i only, that mask is this causal mask on
+    the union sequence (reading).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, d = q.shape
+    hd = d // n_heads
+    scale = 1.0 / math.sqrt(hd)
+    O = np.zeros((T, d))
+    lse = np.zeros((T, n_heads))
+    for u in range(len(cu_seqlens) - 1):
+        s, e = int(cu_seqlens[u]), int(cu_seqlens[u + 1])
+        if e == s:
+            continue
+        for h in range(n_heads):
+            c = slice(h * hd, (h + 1) * hd)
+            S = (q[s:e, c] @ k[s:e, c].T) * scale
+            S[np.triu_indices(e - s, 1)] = -np.inf
+            m = S.max(axis=1, keepdims=True)
+            lse[s:e, h] = (m + np.log(np.exp(S - m).sum(axis=1, keepdims=True)))[:, 0]
+            O[s:e, c] = softmax_rows(S) @ v[s:e, c]
+    return O, lse
+
+
+def attention_core_backward(q, k, v, cu_seqlens, n_heads, d_o):
+    """Gradients of a scalar loss through attention_core, given dO = dL/dO:
+    with S = q k^T / sqrt(d_h) (causal), P = softmax(S) and O = P V,
+
+        dV = P^T dO,   dP = dO V^T,   dS = P * (dP - rowsum(dP * P)),
+        dq = dS k / sqrt(d_h),   dk = dS^T q / sqrt(d_h),
+
+    per user and head (the chain rule through the row softmax; rowsum(dP * P)
+    equals rowsum(dO * O)). Returns (dq, dk, dv), each [T, d]."""
+    q, k, v, d_o = _f64(q), _f64(k), _f64(v), _f64(d_o)
+    T, d = q.shape
+    hd = d // n_heads
+    scale = 1.0 / math.sqrt(hd)
+    dq, dk, dv = np.zeros((T, d)), np.zeros((T, d)), np.zeros((T, d))
+    for u in range(len(cu_seqlens) - 1):
+        s, e = int(cu_seqlens[u]), int(cu_seqlens[u + 1])
+        if e == s:
+            continue
+        for h in range(n_heads):
+            c = slice(h * hd, (h + 1) * hd)
+            S = (q[s:e, c] @ k[s:e, c].T) * scale
+            S[np.triu_indices(e - s, 1)] = -np.inf
+            P = softmax_rows(S)
+            dv[s:e, c] = P.T @ d_o[s:e, c]
+            dP = d_o[s:e, c] @ v[s:e, c].T
+            dS = P * (dP - (dP * P).sum(axis=1, keepdims=True))
+            dq[s:e, c] = dS @ k[s:e, c] * scale
+            dk[s:e, c] = dS.T @ q[s:e, c] * scale
+    return dq, dk, dv
+
+
 def encoder_append(hist: dict, cached: Sequence[int]):
     """Append-only encoding of the tokens that follow a cached prefix.
 

@@ -372,6 +372,67 @@ def test_qkv_gates_keep_scores_relative_in_position():
     assert rel_err(O.encoder(inp, pos_offset=12345), O.encoder(inp)) < 1e-10
 
 
+# ------------------------------------------------ attention core and its backward (ULT)
+
+def core_inputs(seed, lengths=(5, 3, 1), n_heads=2, hd=4):
+    rng = np.random.default_rng(seed)
+    T, d = sum(lengths), n_heads * hd
+    cu = np.zeros(len(lengths) + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(lengths)
+    q, k, v, d_o = (rng.standard_normal((T, d)) for _ in range(4))
+    return q, k, v, d_o, cu, n_heads
+
+
+def test_attention_core_matches_torch_sdpa_forward_and_autograd():
+    q, k, v, d_o, cu, H = core_inputs(30, lengths=(7, 4))
+    O_, lse = O.attention_core(q, k, v, cu, H)
+    dq, dk, dv = O.attention_core_backward(q, k, v, cu, H, d_o)
+    hd = q.shape[1] // H
+    for u in range(len(cu) - 1):
+        s, e = cu[u], cu[u + 1]
+        for h in range(H):
+            c = slice(h * hd, (h + 1) * hd)
+            tq, tk, tv = (torch.tensor(a[s:e, c], dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+            out = torch.nn.functional.scaled_dot_product_attention(tq[None], tk[None], tv[None], is_causal=True)[0]
+            (out * torch.tensor(d_o[s:e, c])).sum().backward()
+            assert rel_err(O_[s:e, c], out.detach().numpy()) < 1e-13
+            for mine, ref in ((dq, tq), (dk, tk), (dv, tv)):
+                assert rel_err(mine[s:e, c], ref.grad.numpy()) < 1e-12
+            S = (q[s:e, c] @ k[s:e, c].T) / math.sqrt(hd)
+            want = [math.log(sum(math.exp(S[i, j]) for j in range(i + 1))) for i in range(e - s)]
+            assert np.max(np.abs(lse[s:e, h] - np.array(want))) < 1e-12
+
+
+def test_attention_core_backward_matches_finite_differences():
+    q, k, v, d_o, cu, H = core_inputs(31)
+    loss = lambda q_, k_, v_: float((O.attention_core(q_, k_, v_, cu, H)[0] * d_o).sum())
+    grads = O.attention_core_backward(q, k, v, cu, H, d_o)
+    eps = 1e-5
+    for which, g in enumerate(grads):
+        fd = np.zeros_like(q)
+        for i in range(q.shape[0]):
+            for c in range(q.shape[1]):
+                args_p = [q.copy(), k.copy(), v.copy()]
+                args_m = [q.copy(), k.copy(), v.copy()]
+                args_p[which][i, c] += eps
+                args_m[which][i, c] -= eps
+                fd[i, c] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert np.max(np.abs(fd - g)) < 1e-8 * max(1.0, np.max(np.abs(g)))
+
+
+def test_attention_core_backward_closed_forms():
+    """Per user and head: the values' gradients sum to the sum of dO (each
+    softmax row sums to 1); the keys' gradients sum to zero (each row of dS
+    sums to zero); a first row sees one key, so its query gets no gradient."""
+    q, k, v, d_o, cu, H = core_inputs(32, lengths=(9, 6, 1), n_heads=3, hd=4)
+    dq, dk, dv = O.attention_core_backward(q, k, v, cu, H, d_o)
+    for u in range(len(cu) - 1):
+        s, e = cu[u], cu[u + 1]
+        assert np.allclose(dv[s:e].sum(axis=0), d_o[s:e].sum(axis=0), atol=1e-12)
+        assert np.allclose(dk[s:e].sum(axis=0), 0.0, atol=1e-12)
+        assert np.all(dq[s] == 0.0)
+
+
 # ------------------------------------------------- append-only encoder cache
 
 def truncate(inp, lengths):
