@@ -276,6 +276,40 @@ rest_status rest_encoder_append(rest_dtype dt, const rest_heads* heads, const re
                                 const rest_kv_cache* cache, void* h_out,
                                 void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
+/* The causal attention core of a DGA sublayer for training, forward and
+ * backward (ULT, §3.5: the union history of a user's training samples is
+ * encoded once under a prefix-valid causal mask; a sample ending at row c
+ * reads rows < c, and with row i seeing rows j <= i only that mask is the
+ * causal mask on the union sequence). Per user (batch) and head h:
+ *   S = q k^T / sqrt(head_dim) over j <= i,  P = softmax(S),  O = P V,
+ * with q, k the rotated queries and keys and V the gated values V' (eq. 3);
+ * the output gate is not part of it. */
+
+/* Workspace bytes rest_attn_forward and rest_attn_backward need. */
+rest_status rest_attn_workspace_size(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                                     size_t* bytes);
+
+/*   q, k, v: dev [T, d] (dtype of the call)
+ *   o:       dev [T, d] (dtype of the call)  O
+ *   o_lo:    dev [T, d] bf16, or NULL: with REST_BF16, the low part of O
+ *            (O = o + o_lo to about 2^-16 relative), for the backward
+ *   lse:     dev fp32 [T, n_heads]  log sum_{j <= i} exp(S_ij), the statistic the backward reuses */
+rest_status rest_attn_forward(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                              const void* q, const void* k, const void* v, void* o, void* o_lo, float* lse,
+                              void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Gradients of a scalar loss L through the core, from d_o = dL/dO (dev [T, d],
+ * dtype of the call) and the forward's o, o_lo (may be NULL) and lse:
+ *   dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),
+ *   dq = dS k / sqrt(head_dim),  dk = dS^T q / sqrt(head_dim).
+ * rowsum(dO * O) takes O = o + o_lo when o_lo is given: a row with few keys
+ * subtracts nearly equal terms in dS, and O's bf16 rounding alone would show.
+ *   dq, dk, dv: dev fp32 [T, d], overwritten. */
+rest_status rest_attn_backward(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
+                               const void* q, const void* k, const void* v, const void* o, const void* o_lo,
+                               const float* lse, const void* d_o, float* dq, float* dk, float* dv,
+                               void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
 /* Decoder block and candidate score ("From Language to Behavior", §3.3.2
  * eq. 8 and Fig. 1 right; the wiring the page leaves open is fixed as: a
  * residual on the query token, a pre-LN feed-forward sublayer whose LN and

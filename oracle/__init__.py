@@ -7,5 +7,5 @@ the benchmark's CPU-baseline leg. The library under
 from .rest_oracle import (  # noqa: F401
     UnsortedTimestamps, rotation_index, frequencies, rotation_angles, rotate, sigmoid, silu,
     layer_norm, softmax_rows, causal_attention_probs, dga_sublayer, ffn_sublayer, srn,
-    encoder, encoder_append, encoder_rows, attention_core, attention_core_backward, cross_decode, score_head, rank_request,
+    encoder, encoder_append, encoder_rows, attention_core, attention_core_backward, attention_core_dq_rows, cross_decode, score_head, rank_request,
 )

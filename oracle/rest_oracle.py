@@ -326,6 +326,29 @@ def attention_core_backward(q, k, v, cu_seqlens, n_heads, d_o):
     return dq, dk, dv
 
 
+def attention_core_dq_rows(q, k, v, cu_seqlens, n_heads, d_o, rows: Sequence[int]):
+    """Rows of attention_core_backward's dq, each computed on its own: row i
+    needs only its own scores against keys j <= i (same definition), so rows
+    of a 16k-token history can be checked without the L x L matrices."""
+    q, k, v, d_o = _f64(q), _f64(k), _f64(v), _f64(d_o)
+    d = q.shape[1]
+    hd = d // n_heads
+    scale = 1.0 / math.sqrt(hd)
+    cu = np.asarray(cu_seqlens)
+    out = np.zeros((len(rows), d))
+    for n, i in enumerate(rows):
+        s = int(cu[np.searchsorted(cu, i, side="right") - 1])
+        for h in range(n_heads):
+            c = slice(h * hd, (h + 1) * hd)
+            sc = (k[s:i + 1, c] @ q[i, c]) * scale
+            p = np.exp(sc - sc.max())
+            p /= p.sum()
+            dp = v[s:i + 1, c] @ d_o[i, c]
+            ds = p * (dp - (p * dp).sum())
+            out[n, c] = (ds @ k[s:i + 1, c]) * scale
+    return out
+
+
 def encoder_append(hist: dict, cached: Sequence[int]):
     """Append-only encoding of the tokens that follow a cached prefix.
 

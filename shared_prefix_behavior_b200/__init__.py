@@ -33,7 +33,8 @@ STATUS = {0: "REST_OK", 1: "REST_ERR_INVALID_ARG", 2: "REST_ERR_UNSORTED_TIME", 
 EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
            "rest_rank_request", "rest_status_string", "rest_launch_count", "rest_profile_begin",
            "rest_profile_end", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",
-           "rest_append_workspace_size", "rest_encoder_append")
+           "rest_append_workspace_size", "rest_encoder_append", "rest_attn_workspace_size", "rest_attn_forward",
+           "rest_attn_backward")
 STATIC_WS_BYTES = 32 * 1024 * 1024  # REST_STATIC_WS_BYTES
 
 
@@ -106,9 +107,14 @@ def _load() -> ctypes.CDLL:
                                                POINTER(c_size_t)]
     lib.rest_encoder_append.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, POINTER(EncLayer), c_int, c_int,
                                         POINTER(KVCacheStruct), P, P, c_size_t, P, P]
+    lib.rest_attn_workspace_size.argtypes = [c_int, POINTER(Heads), POINTER(Batch), POINTER(c_size_t)]
+    lib.rest_attn_forward.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, P, P, P, P, P, c_size_t, P, P]
+    lib.rest_attn_backward.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, P, P, P, P, P, P, P, P, P,
+                                       c_size_t, P, P]
     for name in ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
                  "rest_rank_request", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",
-                 "rest_append_workspace_size", "rest_encoder_append"):
+                 "rest_append_workspace_size", "rest_encoder_append", "rest_attn_workspace_size",
+                 "rest_attn_forward", "rest_attn_backward"):
         getattr(lib, name).restype = c_int
     lib.rest_status_string.argtypes = [c_int]
     lib.rest_status_string.restype = ctypes.c_char_p
@@ -430,6 +436,61 @@ def encoder_append(x, ts, cu_new, taus, layers: Sequence[dict], l_switch: int, c
     if advance:
         cache.advance(cu_new, ts.cpu().numpy() if ts_host is None else ts_host)
     return h_out
+
+
+def attn_workspace_size(dtype: int, n_heads: int, head_dim: int, cu_seqlens) -> int:
+    h = _Host(np.zeros(n_heads, dtype=np.int64), n_heads * head_dim, 10000.0, cu_seqlens)
+    out = c_size_t(0)
+    _check(_lib.rest_attn_workspace_size(dtype, ctypes.byref(h.heads), ctypes.byref(h.batch), ctypes.byref(out)),
+           "rest_attn_workspace_size")
+    return out.value
+
+
+def attn_forward(q, k, v, cu_seqlens, n_heads: int, o=None, o_lo=None, lse=None, ws=None, stream=None,
+                 check=True):
+    """Causal attention core for training (ULT, §3.5): returns (O [T, d] in
+    q's dtype, O's bf16 low part (bf16 calls; None in fp32), lse [T, n_heads]
+    fp32)."""
+    import torch
+    dev, (T, d) = q.device, q.shape
+    dt = _dtype_code(q)
+    h = _Host(np.zeros(n_heads, dtype=np.int64), d, 10000.0, cu_seqlens)
+    if o is None:
+        o = torch.empty_like(q)
+    if o_lo is None and dt == REST_BF16:
+        o_lo = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((T, n_heads), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(attn_workspace_size(dt, n_heads, d // n_heads, cu_seqlens), dev)
+    err = _err_word(dev, stream)
+    _check(_lib.rest_attn_forward(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(o), _ptr(o_lo), _ptr(lse), _ptr(ws), ws.numel(), _ptr(err),
+                                  _stream(stream)), "rest_attn_forward")
+    if check:
+        check_device_error(err)
+    return o, o_lo, lse
+
+
+def attn_backward(q, k, v, o, o_lo, lse, d_o, cu_seqlens, n_heads: int, dq=None, dk=None, dv=None, ws=None,
+                  stream=None, check=True):
+    """Gradients (dq, dk, dv), fp32 [T, d], of the attention core from dO."""
+    import torch
+    dev, (T, d) = q.device, q.shape
+    dt = _dtype_code(q)
+    h = _Host(np.zeros(n_heads, dtype=np.int64), d, 10000.0, cu_seqlens)
+    dq = torch.empty((T, d), dtype=torch.float32, device=dev) if dq is None else dq
+    dk = torch.empty((T, d), dtype=torch.float32, device=dev) if dk is None else dk
+    dv = torch.empty((T, d), dtype=torch.float32, device=dev) if dv is None else dv
+    if ws is None:
+        ws = _workspace(attn_workspace_size(dt, n_heads, d // n_heads, cu_seqlens), dev)
+    err = _err_word(dev, stream)
+    _check(_lib.rest_attn_backward(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(o), _ptr(o_lo), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk), _ptr(dv),
+                                   _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "rest_attn_backward")
+    if check:
+        check_device_error(err)
+    return dq, dk, dv
 
 
 def launch_count(reset: bool = False) -> int:

@@ -113,8 +113,10 @@ struct EncTile { int user; int q0; };          // q0: first query position withi
 struct DecTile { int row0; int nrows; int key0; int nkeys; int kb0; int kb1; int split; int pad; };
 struct EncAttnArgs {
   const void* q; const void* k; const void* v;  // [T, d] rotated Q, K and gated V'
-  const float* gate;                            // [T, d] sigmoid(Go)
+  const float* gate;                            // [T, d] sigmoid(Go), or null (no output gate)
   void* out;                                    // [T, d] dt(O * gate)
+  void* out_lo;                                 // [T, d] bf16 low part of the output (out + out_lo), or null
+  float* lse;                                   // [T, n_heads] log sum_j exp(q k_j / sqrt(d_h)), or null
   const int32_t* cu;                            // [n_users+1]
   const EncTile* tiles; int n_tiles;
   int n_heads, d;
@@ -131,6 +133,23 @@ struct EncAttnArgs {
   long long key_rows;
 };
 cudaError_t launch_enc_attn_simt(bool bf16, int hd, const EncAttnArgs& a, cudaStream_t s);
+
+// Backward of the causal attention core (training; the forward wrote o and lse
+// with the gate left out): dq, dk, dv from d_o = dL/dO.
+struct AttnBwdArgs {
+  const void* q; const void* k; const void* v; const void* o; const void* d_o;  // [T, d], the call's dtype
+  const void* o_lo;    // [T, d] bf16 low part of o (o + o_lo), or null
+  const float* lse;    // [T, n_heads]
+  float* delta;        // [T, n_heads]: rowsum(dO * O) per head, written by the first kernel
+  float* dq; float* dk; float* dv;  // [T, d] fp32
+  const int32_t* cu;
+  const EncTile* tiles; int n_tiles;  // 128-row tiles of every user (query rows, or key rows)
+  int n_heads, d;
+  float scale_log2;    // log2(e) / sqrt(head_dim)
+  long long rows;
+};
+// part 0: delta; part 1: dq (one thread per query row); part 2: dk and dv (one thread per key row)
+cudaError_t launch_attn_bwd_simt(bool bf16, int hd, int part, const AttnBwdArgs& a, cudaStream_t s);
 
 struct DecAttnArgs {
   const float* q;      // [NK, d] decoder queries (fp32)

@@ -207,16 +207,17 @@ static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_he
 // ---------------------------------------------------------------- workspace
 
 struct Layout {
-  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, app, meta_end;
+  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, app, bwd_tiles, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
-  size_t dq, dg, dout, hlo, part_o, part_ml;
+  size_t dq, dg, dout, hlo, part_o, part_ml, delta;
   size_t total;
-  int n_enc_tiles, n_dec_tiles;
+  int n_enc_tiles, n_dec_tiles, n_bwd_tiles;
 };
 
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
                           int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split,
-                          size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2, bool append) {
+                          size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2, bool append,
+                          int n_bwd_tiles = 0) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -231,6 +232,8 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dec_sched = take(sizeof(int) * n_dec_sched);
   L.dec_sched2 = take(sizeof(int) * n_dec_sched2);
   L.app = take(append ? sizeof(UserAppend) * (size_t)b->n_users : 0);
+  L.n_bwd_tiles = n_bwd_tiles;
+  L.bwd_tiles = take(sizeof(EncTile) * (size_t)n_bwd_tiles);
   L.meta_end = off;
   L.cos_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
   L.sin_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
@@ -248,6 +251,7 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.hlo = take(hsplit ? 2 * (size_t)T * d : 0);
   L.part_o = take(n_split > 1 ? 4 * (size_t)n_split * NK * d : 0);
   L.part_ml = take(n_split > 1 ? 8 * (size_t)n_split * NK * hs->n_heads : 0);
+  L.delta = take(n_bwd_tiles > 0 ? 4 * (size_t)T * hs->n_heads : 0);
   L.total = off;
   return L;
 }
@@ -262,6 +266,7 @@ struct Plan {
   std::vector<DecTile> dec_tiles;
   std::vector<int> enc_sched, dec_sched, dec_sched2;  // tensor-core attention: per-CTA item lists
   std::vector<UserAppend> app;  // appending to a cache: each user's cached prefix
+  std::vector<EncTile> bwd_tiles;  // attention core backward: 128-row tiles of every user
   int n_dec_hlo;  // leading decoder tiles that read H_lo (rank_request, bf16)
   Layout L;
   int32_t* err;
@@ -299,7 +304,8 @@ static rest_status check_cache(const rest_kv_cache* c, const rest_batch* b, int 
 
 static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const rest_batch* b,
                              const rest_enc_layer* layers, int n_layers, int l_switch, const rest_requests* reqs,
-                             int K, bool encoder_runs, const rest_kv_cache* cache = nullptr, bool append = false) {
+                             int K, bool encoder_runs, const rest_kv_cache* cache = nullptr, bool append = false,
+                             bool core = false) {
   rest_status st = check_heads(dt, hs);
   if (st != REST_OK) return st;
   if ((st = check_batch(b, &p.T)) != REST_OK) return st;
@@ -349,9 +355,14 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
       }
     }
   }
-  p.L = make_layout(dt, hs, b, p.T, encoder_runs, p.max_dff, p.NK, (int)p.enc_tiles.size(),
+  // the attention core alone (training): no encoder buffers; the backward's 128-row tiles
+  p.bwd_tiles.clear();
+  if (core)
+    for (int u = 0; u < b->n_users; ++u)
+      for (int r0 = 0; r0 < b->cu_seqlens[u + 1] - b->cu_seqlens[u]; r0 += 128) p.bwd_tiles.push_back(EncTile{u, r0});
+  p.L = make_layout(dt, hs, b, p.T, encoder_runs && !core, p.max_dff, p.NK, (int)p.enc_tiles.size(),
                     (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size(),
-                    p.dec_sched2.size(), append);
+                    p.dec_sched2.size(), append, (int)p.bwd_tiles.size());
   return REST_OK;
 }
 
@@ -441,6 +452,8 @@ static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
   if (!p.dec_sched2.empty())
     memcpy(host.data() + p.L.dec_sched2, p.dec_sched2.data(), sizeof(int) * p.dec_sched2.size());
   if (!p.app.empty()) memcpy(host.data() + p.L.app, p.app.data(), sizeof(UserAppend) * p.app.size());
+  if (!p.bwd_tiles.empty())
+    memcpy(host.data() + p.L.bwd_tiles, p.bwd_tiles.data(), sizeof(EncTile) * p.bwd_tiles.size());
   if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) return REST_ERR_CUDA;
   // the status word reports this call only
   if (p.err && cudaMemsetAsync(p.err, 0, sizeof(int32_t), s) != cudaSuccess) return REST_ERR_CUDA;
@@ -544,6 +557,7 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   REST_KLAUNCH(s, "to_f32", 0, Td * (e + 4), launch_to_f32(bf, x, xres, T * d, s));
 
   EncAttnArgs ea;
+  memset(&ea, 0, sizeof(ea));  // optional outputs (lse, out_lo) stay null
   ea.q = q; ea.k = k; ea.v = v; ea.gate = g; ea.out = o; ea.cu = cu;
   ea.tiles = at<EncTile>(ws, L.enc_tiles); ea.n_tiles = L.n_enc_tiles;
   ea.sched = at<int>(ws, L.enc_sched);
@@ -695,6 +709,7 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   // pair of bf16 arrays (in the same workspace bytes); the CUDA-core one as fp32.
   const bool tc = bf && sm100_attn_supported(hd);
   DecAttnArgs da;
+  memset(&da, 0, sizeof(da));
   da.q = dq; da.g = dg; da.h = h; da.h_lo = h_lo; da.out = dout;
   da.out_lo = tc ? (void*)((bf16*)dout + (size_t)p.NK * d) : nullptr;
   da.tiles = at<DecTile>(ws, L.dec_tiles); da.n_tiles = L.n_dec_tiles;
@@ -897,6 +912,116 @@ rest_status rest_encoder_append(rest_dtype dt, const rest_heads* heads, const re
     p.err = dev_err;
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
     return run_encoder(p, x, ts, layers, n_layers, l_switch, h_out, ws, dev_err, s, cache);
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_attn_workspace_size(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, size_t* bytes) {
+  if (!bytes) return REST_ERR_INVALID_ARG;
+  try {
+    Plan p;
+    rest_status st = make_plan(p, dt, heads, batch, nullptr, 0, 0, nullptr, 1, true, nullptr, false, true);
+    if (st != REST_OK) return st;
+    *bytes = p.L.total;
+    return REST_OK;
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_attn_forward(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, const void* q,
+                              const void* k, const void* v, void* o, void* o_lo, float* lse, void* ws,
+                              size_t ws_bytes, int32_t* dev_err, void* stream) {
+  try {
+    Plan p;
+    rest_status st = make_plan(p, dt, heads, batch, nullptr, 0, 0, nullptr, 1, true, nullptr, false, true);
+    if (st != REST_OK) return st;
+    if (p.T > 0 && (!q || !k || !v || !o || !lse || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+                    !aligned16(o) || !aligned16(lse) || !aligned16(o_lo) || (o_lo && dt != REST_BF16)))
+      return REST_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < p.L.total || !aligned16(ws)) return REST_ERR_WORKSPACE;
+    if (p.T == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    const bool bf = dt == REST_BF16;
+    const int d = heads->d, hd = heads->head_dim, H = heads->n_heads;
+    const size_t e = dt_size(dt);
+    double pairs = 0;
+    for (int u = 0; u < batch->n_users; ++u) {
+      const double L = batch->cu_seqlens[u + 1] - batch->cu_seqlens[u];
+      pairs += L * (L + 1) / 2;
+    }
+    EncAttnArgs ea;
+    memset(&ea, 0, sizeof(ea));
+    ea.q = q; ea.k = k; ea.v = v; ea.gate = nullptr; ea.out = o; ea.out_lo = o_lo; ea.lse = lse;
+    ea.cu = at<int32_t>(ws, p.L.cu);
+    ea.tiles = at<EncTile>(ws, p.L.enc_tiles); ea.n_tiles = p.L.n_enc_tiles;
+    ea.sched = at<int>(ws, p.L.enc_sched);
+    ea.n_cta = p.enc_sched.empty() ? 0 : std::min((int)p.enc_tiles.size() * H, SCHED_CTAS);
+    ea.n_heads = H; ea.d = d;
+    ea.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
+    ea.rows = p.T;
+    ea.key_rows = p.T;
+    const double flops = 4.0 * d * pairs, bytes = (double)p.T * d * ((o_lo ? 5 : 4) * e) + 4.0 * p.T * H;
+    if (bf && sm100_attn_supported(hd)) {
+      REST_KLAUNCH(s, "attn_fwd", flops, bytes, launch_enc_attn_sm100(hd, ea, s, dev_err));
+    } else {
+      REST_KLAUNCH(s, "attn_fwd", flops, bytes, launch_enc_attn_simt(bf, hd, ea, s));
+    }
+    return REST_OK;
+  } catch (...) {
+    return REST_ERR_INVALID_ARG;
+  }
+}
+
+rest_status rest_attn_backward(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, const void* q,
+                               const void* k, const void* v, const void* o, const void* o_lo, const float* lse,
+                               const void* d_o, float* dq, float* dk, float* dv, void* ws, size_t ws_bytes,
+                               int32_t* dev_err, void* stream) {
+  try {
+    Plan p;
+    rest_status st = make_plan(p, dt, heads, batch, nullptr, 0, 0, nullptr, 1, true, nullptr, false, true);
+    if (st != REST_OK) return st;
+    const void* ptrs[] = {q, k, v, o, lse, d_o, dq, dk, dv};
+    if (p.T > 0) {
+      for (const void* ptr : ptrs)
+        if (!ptr || !aligned16(ptr)) return REST_ERR_INVALID_ARG;
+      if (!aligned16(o_lo) || (o_lo && dt != REST_BF16)) return REST_ERR_INVALID_ARG;
+    }
+    if (!ws || ws_bytes < p.L.total || !aligned16(ws)) return REST_ERR_WORKSPACE;
+    if (p.T == 0) return REST_OK;
+    if ((st = check_device()) != REST_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    p.err = dev_err;
+    if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
+    const bool bf = dt == REST_BF16;
+    const int d = heads->d, hd = heads->head_dim, H = heads->n_heads;
+    const size_t e = dt_size(dt);
+    double pairs = 0;
+    for (int u = 0; u < batch->n_users; ++u) {
+      const double L = batch->cu_seqlens[u + 1] - batch->cu_seqlens[u];
+      pairs += L * (L + 1) / 2;
+    }
+    AttnBwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.o = o; a.o_lo = o_lo; a.d_o = d_o; a.lse = lse;
+    a.delta = at<float>(ws, p.L.delta);
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    a.cu = at<int32_t>(ws, p.L.cu);
+    a.tiles = at<EncTile>(ws, p.L.bwd_tiles); a.n_tiles = p.L.n_bwd_tiles;
+    a.n_heads = H; a.d = d;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)hd));
+    a.rows = p.T;
+    // delta = rowsum(dO * O); then dq (S, dP and dS K per visible (query, key, head)) and dk, dv
+    // (S, dP, P^T dO and dS^T q): 6 + 8 d_h-long products, against 5 in one fused pass
+    const double td = (double)p.T * d;
+    REST_KLAUNCH(s, "attn_bwd_delta", 0, td * 2 * e + 4.0 * p.T * H, launch_attn_bwd_simt(bf, hd, 0, a, s));
+    REST_KLAUNCH(s, "attn_bwd_dq", 6.0 * d * pairs, td * (3 * e + 4), launch_attn_bwd_simt(bf, hd, 1, a, s));
+    REST_KLAUNCH(s, "attn_bwd_dkdv", 8.0 * d * pairs, td * (4 * e + 8), launch_attn_bwd_simt(bf, hd, 2, a, s));
+    return REST_OK;
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }

@@ -841,15 +841,23 @@ __device__ __forceinline__ void load_q(RowState<HD>& st, const T* q, float scale
   st.l = 0.f;
 }
 
+// O / l times the output gate (gate null: no gate); with out_lo (bf16 outputs)
+// also the low part, out + out_lo
 template <typename T, int HD>
-__device__ __forceinline__ void store_row(const RowState<HD>& st, const float* gate, T* out) {
+__device__ __forceinline__ void store_row(const RowState<HD>& st, const float* gate, T* out, T* out_lo = nullptr) {
   float inv = 1.0f / st.l;
 #pragma unroll
   for (int c = 0; c < HD; c += 4) {
-    float g[4];
-    load4(gate + c, g);
+    float g[4] = {1.f, 1.f, 1.f, 1.f};
+    if (gate) load4(gate + c, g);
     float v[4] = {st.o[c] * inv * g[0], st.o[c + 1] * inv * g[1], st.o[c + 2] * inv * g[2], st.o[c + 3] * inv * g[3]};
     store4(out + c, v);
+    if (out_lo) {
+      float lo[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lo[i] = v[i] - to_f<T>(from_f<T>(v[i]));
+      store4(out_lo + c, lo);
+    }
   }
 }
 
@@ -885,7 +893,9 @@ __global__ void __launch_bounds__(ATT_ROWS) enc_attn_simt_kernel(EncAttnArgs a) 
   }
   if (valid) {
     long long ro = (long long)(s + i) * a.d + hoff;
-    store_row<T, HD>(st, a.gate + ro, (T*)a.out + ro);
+    store_row<T, HD>(st, a.gate ? a.gate + ro : nullptr, (T*)a.out + ro, a.out_lo ? (T*)a.out_lo + ro : nullptr);
+    // log sum_j exp(score): the running max is kept in the scaled log2 domain
+    if (a.lse) a.lse[(long long)(s + i) * a.n_heads + h] = (st.m + log2f(st.l)) * 0.69314718055994531f;
   }
 }
 
@@ -985,6 +995,185 @@ cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s) {
   const int threads = 256;
   if (cudaError_t e_ = launch_k(dec_combine_kernel, (unsigned)((n + threads - 1) / threads), threads, 0, s, a, hd)) return e_;
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- attention backward
+// delta[i, h] = sum over the head's columns of dO * O (one thread per row and head)
+template <typename T>
+__global__ void attn_bwd_delta_kernel(AttnBwdArgs a, int hd) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= a.rows * a.n_heads) return;
+  const long long i = gid / a.n_heads;
+  const int h = (int)(gid % a.n_heads);
+  const T* o = (const T*)a.o + i * a.d + (long long)h * hd;
+  const T* olo = a.o_lo ? (const T*)a.o_lo + i * a.d + (long long)h * hd : nullptr;
+  const T* g = (const T*)a.d_o + i * a.d + (long long)h * hd;
+  float acc = 0.f;
+  for (int c = 0; c < hd; c += 4) {
+    float ov[4], gv[4];
+    load4(o + c, ov);
+    load4(g + c, gv);
+    if (olo) {  // O = o + o_lo
+      float lv[4];
+      load4(olo + c, lv);
+      for (int e = 0; e < 4; ++e) ov[e] += lv[e];
+    }
+    acc += ov[0] * gv[0] + ov[1] * gv[1] + ov[2] * gv[2] + ov[3] * gv[3];
+  }
+  a.delta[gid] = acc;
+}
+
+// dq: one thread per query row i, over the keys j <= i staged in shared memory:
+// p = exp(s - lse), ds = p (dO_i . v_j - delta_i), dq_i += ds k_j, times 1/sqrt(d_h).
+template <typename T, int HD>
+__global__ void __launch_bounds__(ATT_ROWS) attn_bwd_dq_simt_kernel(AttnBwdArgs a) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  __shared__ __align__(16) float Ks[ATT_BK][HD];
+  __shared__ __align__(16) float Vs[ATT_BK][HD];
+  const EncTile tile = a.tiles[blockIdx.x];
+  const int h = blockIdx.y;
+  const int s = a.cu[tile.user], L = a.cu[tile.user + 1] - s;
+  const int i = tile.q0 + threadIdx.x;
+  const bool valid = i < L;
+  const long long ro = (long long)(s + (valid ? i : 0)) * a.d + (long long)h * HD;
+  float q[HD], go[HD], dq[HD];
+#pragma unroll
+  for (int c = 0; c < HD; c += 4) {
+    load4((const T*)a.q + ro + c, &q[c]);
+    load4((const T*)a.d_o + ro + c, &go[c]);
+  }
+#pragma unroll
+  for (int c = 0; c < HD; ++c) {
+    q[c] *= a.scale_log2;
+    dq[c] = 0.f;
+  }
+  const long long ri = (long long)(s + (valid ? i : 0)) * a.n_heads + h;
+  const float lse2 = a.lse[ri] * 1.4426950408889634f, dlt = a.delta[ri];
+  const int kv_end = min(L, tile.q0 + ATT_ROWS);
+  const T* K = (const T*)a.k + (long long)s * a.d + (long long)h * HD;
+  const T* V = (const T*)a.v + (long long)s * a.d + (long long)h * HD;
+  for (int kb = 0; kb < kv_end; kb += ATT_BK) {
+    __syncthreads();
+    stage_kv<T, HD, ATT_BK>(Ks, Vs, K + (long long)kb * a.d, V + (long long)kb * a.d, a.d, kv_end - kb);
+    __syncthreads();
+    if (!valid || kb > i) continue;
+    const int jmax = min(ATT_BK, i - kb + 1);
+    for (int j = 0; j < jmax; ++j) {
+      float sc = 0.f, dp = 0.f;
+#pragma unroll
+      for (int c = 0; c < HD; ++c) {
+        sc = fmaf(q[c], Ks[j][c], sc);
+        dp = fmaf(go[c], Vs[j][c], dp);
+      }
+      const float ds = exp2f(sc - lse2) * (dp - dlt);
+#pragma unroll
+      for (int c = 0; c < HD; ++c) dq[c] = fmaf(ds, Ks[j][c], dq[c]);
+    }
+  }
+  if (valid) {
+    const float sc = a.scale_log2 * 0.69314718055994531f;  // 1 / sqrt(d_h)
+#pragma unroll
+    for (int c = 0; c < HD; ++c) dq[c] *= sc;
+#pragma unroll
+    for (int c = 0; c < HD; c += 4) store4(a.dq + ro + c, &dq[c]);
+  }
+}
+
+// dk, dv: one thread per key row j, over the queries i >= j staged in shared
+// memory: dv_j += p dO_i, dk_j += p (dO_i . v_j - delta_i) q_i, times 1/sqrt(d_h).
+template <typename T, int HD>
+__global__ void __launch_bounds__(ATT_ROWS) attn_bwd_dkdv_simt_kernel(AttnBwdArgs a) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  __shared__ __align__(16) float Qs[ATT_BK][HD];
+  __shared__ __align__(16) float Gs[ATT_BK][HD];
+  __shared__ float Ls[ATT_BK], Ds[ATT_BK];
+  const EncTile tile = a.tiles[blockIdx.x];
+  const int h = blockIdx.y;
+  const int s = a.cu[tile.user], L = a.cu[tile.user + 1] - s;
+  const int j = tile.q0 + threadIdx.x;
+  const bool valid = j < L;
+  const long long ro = (long long)(s + (valid ? j : 0)) * a.d + (long long)h * HD;
+  float k[HD], v[HD], dk[HD], dv[HD];
+#pragma unroll
+  for (int c = 0; c < HD; c += 4) {
+    load4((const T*)a.k + ro + c, &k[c]);
+    load4((const T*)a.v + ro + c, &v[c]);
+  }
+#pragma unroll
+  for (int c = 0; c < HD; ++c) {
+    k[c] *= a.scale_log2;
+    dk[c] = 0.f;
+    dv[c] = 0.f;
+  }
+  const T* Q = (const T*)a.q + (long long)s * a.d + (long long)h * HD;
+  const T* G = (const T*)a.d_o + (long long)s * a.d + (long long)h * HD;
+  for (int qb = tile.q0; qb < L; qb += ATT_BK) {
+    __syncthreads();
+    stage_kv<T, HD, ATT_BK>(Qs, Gs, Q + (long long)qb * a.d, G + (long long)qb * a.d, a.d, L - qb);
+    if (threadIdx.x < ATT_BK && qb + (int)threadIdx.x < L) {
+      const long long r = (long long)(s + qb + threadIdx.x) * a.n_heads + h;
+      Ls[threadIdx.x] = a.lse[r] * 1.4426950408889634f;
+      Ds[threadIdx.x] = a.delta[r];
+    }
+    __syncthreads();
+    if (!valid) continue;
+    const int imax = min(ATT_BK, L - qb);
+    for (int ii = max(0, j - qb); ii < imax; ++ii) {  // causal: query qb + ii >= j
+      float sc = 0.f, dp = 0.f;
+#pragma unroll
+      for (int c = 0; c < HD; ++c) {
+        sc = fmaf(k[c], Qs[ii][c], sc);
+        dp = fmaf(v[c], Gs[ii][c], dp);
+      }
+      const float p = exp2f(sc - Ls[ii]);
+      const float ds = p * (dp - Ds[ii]);
+#pragma unroll
+      for (int c = 0; c < HD; ++c) {
+        dv[c] = fmaf(p, Gs[ii][c], dv[c]);
+        dk[c] = fmaf(ds, Qs[ii][c], dk[c]);
+      }
+    }
+  }
+  if (valid) {
+    const float sc = a.scale_log2 * 0.69314718055994531f;  // 1 / sqrt(d_h)
+#pragma unroll
+    for (int c = 0; c < HD; ++c) dk[c] *= sc;
+#pragma unroll
+    for (int c = 0; c < HD; c += 4) {
+      store4(a.dk + ro + c, &dk[c]);
+      store4(a.dv + ro + c, &dv[c]);
+    }
+  }
+}
+
+template <typename T, int HD>
+static cudaError_t attn_bwd_part(int part, const AttnBwdArgs& a, cudaStream_t s) {
+  const dim3 grid(a.n_tiles, a.n_heads);
+  if (part == 1) return launch_k(attn_bwd_dq_simt_kernel<T, HD>, grid, ATT_ROWS, 0, s, a);
+  return launch_k(attn_bwd_dkdv_simt_kernel<T, HD>, grid, ATT_ROWS, 0, s, a);
+}
+
+template <typename T>
+static cudaError_t attn_bwd_dispatch(int hd, int part, const AttnBwdArgs& a, cudaStream_t s) {
+  if (part == 0) {
+    const long long n = a.rows * a.n_heads;
+    return launch_k(attn_bwd_delta_kernel<T>, (unsigned)((n + 255) / 256), 256, 0, s, a, hd);
+  }
+  switch (hd) {
+    case 16: return attn_bwd_part<T, 16>(part, a, s);
+    case 32: return attn_bwd_part<T, 32>(part, a, s);
+    case 64: return attn_bwd_part<T, 64>(part, a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_bwd_simt(bool bf16m, int hd, int part, const AttnBwdArgs& a, cudaStream_t s) {
+  if (a.n_tiles == 0) return cudaSuccess;
+  return bf16m ? attn_bwd_dispatch<bf16>(hd, part, a, s) : attn_bwd_dispatch<float>(hd, part, a, s);
 }
 
 cudaError_t launch_enc_attn_simt(bool bf16m, int hd, const EncAttnArgs& a, cudaStream_t s) {

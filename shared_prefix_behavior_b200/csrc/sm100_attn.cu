@@ -473,8 +473,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // at 64 the row would not fit the softmax warps' registers next to O)
       constexpr bool GATE_EARLY = HD <= 32;
       const long long ro = row_g * d + h * HD;
+      const bool has_gate = DEC || ea.gate != nullptr;  // the encoder's gate may be left out (training core)
       float gate_row[GATE_EARLY ? HD : 4];
-      if (GATE_EARLY && valid && !split) {
+      if (GATE_EARLY && valid && !split && has_gate) {
         const float* gate = (DEC ? da.g : ea.gate) + ro;
 #pragma unroll
         for (int c = 0; c < HD; c += 4) load4(gate + c, &gate_row[c]);
@@ -501,12 +502,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         pml[1] = l_run;
       } else if (valid) {
         const float inv = 1.0f / l_run;
+        // log sum_j exp(score) for a backward pass: m_ref is in the scaled log2 domain
+        if (!DEC && ea.lse) ea.lse[row_g * n_heads + h] = (m_ref + log2f(l_run)) * 0.69314718055994531f;
 #pragma unroll
         for (int c0 = 0; c0 < HD; c0 += 32) {  // 32 columns at a time, their gate loads in flight together
           float gh[32];
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
-            if (GATE_EARLY) {
+            if (!has_gate) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) gh[c + i] = 1.f;
+            } else if (GATE_EARLY) {
 #pragma unroll
               for (int i = 0; i < 4; ++i) gh[c + i] = gate_row[(c0 + c + i) % (GATE_EARLY ? HD : 4)];
             } else {
@@ -528,6 +534,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               store4((float*)da.out + ro + cc, v);
             } else {
               store4((bf16*)ea.out + ro + cc, v);
+              if (ea.out_lo) {  // the low part, for a backward pass that needs O beyond bf16
+                float lo[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
+                store4((bf16*)ea.out_lo + ro + cc, lo);
+              }
             }
           }
         }

@@ -245,3 +245,36 @@ def test_cache_bookkeeping_counts_appended_tokens():
     c.advance([0, 1, 3], np.array([12, 40, 41]))
     assert list(c.len) == [4, 2] and c.t_first[0] == 7 and c.t_last[0] == 12
     assert c.t_first[1] == 40 and c.t_last[1] == 41
+
+
+# ------------------------------------------------------------ attention core (training)
+
+def _core(fn="fwd", cu=(0, 10, 30), ptr=FAKE, bad=None, ws_bytes=1 << 40, dt=R.REST_BF16):
+    t, hs = _heads((0, 0, 1, 64), 64)
+    c, b = _batch(cu)
+    lib = R.library()
+    # forward: q k v o o_lo lse; backward: q k v o o_lo lse d_o dq dk dv (o_lo may be NULL, not misaligned)
+    n = 6 if fn == "fwd" else 10
+    args = [ptr] * n
+    if bad is not None:
+        args[bad] = FAKE + 8 if bad % 2 or bad == 4 else None
+    f = lib.rest_attn_forward if fn == "fwd" else lib.rest_attn_backward
+    return f(dt, ctypes.byref(hs), ctypes.byref(b), *args, FAKE, ws_bytes, None, None)
+
+
+@pytest.mark.parametrize("fn,bad", [("fwd", i) for i in range(6)] + [("bwd", i) for i in range(10)])
+def test_attention_core_rejects_missing_or_misaligned_pointers(fn, bad):
+    assert _core(fn, bad=bad) == INVALID
+
+
+def test_attention_core_low_part_only_with_bf16():
+    assert _core("fwd", dt=R.REST_F32) == INVALID  # o_lo given to an fp32 call
+
+
+def test_attention_core_workspace_empty_and_no_device():
+    assert _core("fwd", ws_bytes=16) == WORKSPACE and _core("bwd", ws_bytes=16) == WORKSPACE
+    assert _core("fwd", cu=(0, 0)) == 0 and _core("bwd", cu=(0,)) == 0
+    assert _core("fwd", cu=(0, 5, 3)) == INVALID
+    assert 0 < R.attn_workspace_size(R.REST_BF16, 8, 32, [0, 64]) < R.attn_workspace_size(R.REST_BF16, 8, 32, [0, 4096])
+    if not gpu_available():
+        assert _core("fwd") == NO_DEVICE and _core("bwd") == NO_DEVICE

@@ -433,6 +433,36 @@ def test_attention_core_backward_closed_forms():
         assert np.all(dq[s] == 0.0)
 
 
+def test_row_sampled_dq_equals_full_backward():
+    q, k, v, d_o, cu, H = core_inputs(35, lengths=(13, 6, 1), n_heads=2, hd=8)
+    dq, _, _ = O.attention_core_backward(q, k, v, cu, H, d_o)
+    rows = [0, 1, 12, 13, 18, 19]
+    assert rel_err(O.attention_core_dq_rows(q, k, v, cu, H, d_o, rows), dq[rows]) < 1e-12
+
+
+def test_ult_union_gradient_is_the_sum_of_per_sample_gradients():
+    """ULT (§3.5): a user's samples ending at rows c_1 < c_2 < ... are encoded
+    once as their union history; with the causal mask, a loss that reads each
+    sample's own rows gives, on the union, the sum of the gradients each
+    sample would give encoded alone on its prefix."""
+    q, k, v, _, _, H = core_inputs(33, lengths=(11,), n_heads=2, hd=4)
+    rng = np.random.default_rng(34)
+    cuts = [4, 8, 11]
+    d_os = []
+    for c in cuts:  # sample m's loss reads rows < c_m of the history
+        g = np.zeros_like(q)
+        g[:c] = rng.standard_normal((c, q.shape[1]))
+        d_os.append(g)
+    union = O.attention_core_backward(q, k, v, np.array([0, 11]), H, sum(d_os))
+    alone = [np.zeros_like(q) for _ in range(3)]
+    for c, g in zip(cuts, d_os):
+        parts = O.attention_core_backward(q[:c], k[:c], v[:c], np.array([0, c]), H, g[:c])
+        for acc, p_ in zip(alone, parts):
+            acc[:c] += p_
+    for a, b in zip(union, alone):
+        assert rel_err(a, b) < 1e-12
+
+
 # ------------------------------------------------- append-only encoder cache
 
 def truncate(inp, lengths):
