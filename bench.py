@@ -476,6 +476,62 @@ def ablation_comparison(w, dev, n=20):
     return out
 
 
+def training_comparison(w, inp, dev, n=10):
+    """The attention core a training step runs (ULT, §3.5): rest_attn_forward
+    and rest_attn_backward on the workload's histories (seeded bf16 q, k, V'
+    and dO stand in for a layer's activations), with L2 flushed before every
+    call (a 256 MB write). ULT's comparison: the same core run once per
+    request instead, each request a training sample of its own whose history
+    is its prefix (what encoding the union history once saves)."""
+    import torch
+    import shared_prefix_behavior_b200 as R
+    H, d = w.n_heads, w.d
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    peaks, src = load_peaks()
+    tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + 29)
+
+    def run(cu):
+        T = int(cu[-1])
+        q, k, v, d_o = (torch.randn((T, d), generator=g, device=dev).to(dt) for _ in range(4))
+        ws = torch.empty(R.attn_workspace_size(R.REST_BF16 if dt == torch.bfloat16 else R.REST_F32, H, d // H, cu),
+                         dtype=torch.uint8, device=dev)
+        o, o_lo, lse = R.attn_forward(q, k, v, cu, H, ws=ws)
+        dq, dk, dv = R.attn_backward(q, k, v, o, o_lo, lse, d_o, cu, H, ws=ws)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        for i in range(n):
+            flush.fill_(i & 0xff)
+            ev[i][0].record()
+            R.attn_forward(q, k, v, cu, H, o=o, o_lo=o_lo, lse=lse, ws=ws, check=False)
+            ev[i][1].record()
+            R.attn_backward(q, k, v, o, o_lo, lse, d_o, cu, H, dq=dq, dk=dk, dv=dv, ws=ws, check=False)
+            ev[i][2].record()
+        torch.cuda.synchronize()
+        fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / n
+        bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / n
+        pairs = sum(L * (L + 1) / 2 for L in np.diff(cu))
+        return fwd, bwd, pairs, T
+
+    cu = np.asarray(inp["cu_seqlens"], dtype=np.int32)
+    fwd, bwd, pairs, T = run(cu)
+    f_fwd, f_bwd = 4.0 * d * pairs, 10.0 * d * pairs
+    out = {"tokens": T, "fwd_ms": fwd, "bwd_ms": bwd,
+           "fwd_tflops": f_fwd / fwd / 1e9, "bwd_tflops": f_bwd / bwd / 1e9,
+           "fwd_roofline_frac": f_fwd / fwd / 1e9 / tensor_peak, "bwd_roofline_frac": f_bwd / bwd / 1e9 / tensor_peak,
+           "roofline": f"algorithmic FLOPs (fwd 4 d, bwd 10 d per visible pair) / sustained bf16 peak ({src})",
+           "l2": "flushed before every call (256 MB write)"}
+    # ULT: every request's prefix as a sample of its own, packed into one batch
+    lens = [int(c) for c in inp["req_cutoff"]]
+    cu_s = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    s_fwd, s_bwd, s_pairs, s_T = run(cu_s)
+    out["ult"] = {"samples": len(lens), "union_tokens": T, "per_sample_tokens": s_T,
+                  "per_sample_ms": s_fwd + s_bwd, "union_ms": fwd + bwd,
+                  "speedup_of_union": (s_fwd + s_bwd) / (fwd + bwd), "flop_ratio": s_pairs / pairs}
+    return out
+
+
 # --------------------------------------------------------------------- oracle (CPU baseline / reference arm)
 
 def blas_threads() -> int:
@@ -714,6 +770,8 @@ def main():
         parts["append"] = append_comparison(w, inp, dev, parts["encoder_only"]["ms"])
     if args.ablation and world == 1:
         parts["ablation"] = ablation_comparison(w, dev)
+    if world == 1:
+        parts["training"] = training_comparison(w, inp, dev)
 
     if world > 1:
         dist.barrier()
@@ -766,7 +824,7 @@ def main():
         "encoder_only": parts["encoder_only"],
         "decoder_only": parts["decoder_only"],
     }
-    for k in ("sharing", "append", "ablation"):
+    for k in ("sharing", "append", "ablation", "training"):
         if k in parts:
             out[k] = parts[k]
     if world == 1 and not args.no_cpu_baseline:

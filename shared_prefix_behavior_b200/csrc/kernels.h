@@ -147,6 +147,9 @@ struct AttnBwdArgs {
   int n_heads, d;
   float scale_log2;    // log2(e) / sqrt(head_dim)
   long long rows;
+  // tensor-core kernel: CTA c runs the work items (key tile * n_heads + head)
+  // sched[n_cta + 1 + k] for k in [sched[c], sched[c + 1]); dq starts at zero
+  const int* sched; int n_cta;
 };
 // part 0: delta; part 1: dq (one thread per query row); part 2: dk and dv (one thread per key row)
 cudaError_t launch_attn_bwd_simt(bool bf16, int hd, int part, const AttnBwdArgs& a, cudaStream_t s);

@@ -207,7 +207,7 @@ static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_he
 // ---------------------------------------------------------------- workspace
 
 struct Layout {
-  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, app, bwd_tiles, meta_end;
+  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, app, bwd_tiles, bwd_sched, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
   size_t dq, dg, dout, hlo, part_o, part_ml, delta;
   size_t total;
@@ -217,7 +217,7 @@ struct Layout {
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
                           int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split,
                           size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2, bool append,
-                          int n_bwd_tiles = 0) {
+                          int n_bwd_tiles = 0, size_t n_bwd_sched = 0) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -234,6 +234,7 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.app = take(append ? sizeof(UserAppend) * (size_t)b->n_users : 0);
   L.n_bwd_tiles = n_bwd_tiles;
   L.bwd_tiles = take(sizeof(EncTile) * (size_t)n_bwd_tiles);
+  L.bwd_sched = take(sizeof(int) * n_bwd_sched);
   L.meta_end = off;
   L.cos_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
   L.sin_t = take(enc ? 4 * (size_t)T * d / 2 : 0);
@@ -267,6 +268,7 @@ struct Plan {
   std::vector<int> enc_sched, dec_sched, dec_sched2;  // tensor-core attention: per-CTA item lists
   std::vector<UserAppend> app;  // appending to a cache: each user's cached prefix
   std::vector<EncTile> bwd_tiles;  // attention core backward: 128-row tiles of every user
+  std::vector<int> bwd_sched;      // tensor-core backward: per-CTA lists of (key tile, head) items
   int n_dec_hlo;  // leading decoder tiles that read H_lo (rank_request, bf16)
   Layout L;
   int32_t* err;
@@ -357,12 +359,21 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   }
   // the attention core alone (training): no encoder buffers; the backward's 128-row tiles
   p.bwd_tiles.clear();
-  if (core)
-    for (int u = 0; u < b->n_users; ++u)
-      for (int r0 = 0; r0 < b->cu_seqlens[u + 1] - b->cu_seqlens[u]; r0 += 128) p.bwd_tiles.push_back(EncTile{u, r0});
+  p.bwd_sched.clear();
+  if (core) {
+    std::vector<long long> cost;  // tensor-core backward: a key tile meets the query blocks from its diagonal on
+    for (int u = 0; u < b->n_users; ++u) {
+      const int L = b->cu_seqlens[u + 1] - b->cu_seqlens[u];
+      for (int r0 = 0; r0 < L; r0 += 128) {
+        p.bwd_tiles.push_back(EncTile{u, r0});
+        for (int h = 0; h < hs->n_heads; ++h) cost.push_back((L + 127) / 128 - r0 / 128);
+      }
+    }
+    if (tile_rows != 128 && !cost.empty()) p.bwd_sched = lpt_schedule(cost);
+  }
   p.L = make_layout(dt, hs, b, p.T, encoder_runs && !core, p.max_dff, p.NK, (int)p.enc_tiles.size(),
                     (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size(),
-                    p.dec_sched2.size(), append, (int)p.bwd_tiles.size());
+                    p.dec_sched2.size(), append, (int)p.bwd_tiles.size(), p.bwd_sched.size());
   return REST_OK;
 }
 
@@ -454,6 +465,8 @@ static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
   if (!p.app.empty()) memcpy(host.data() + p.L.app, p.app.data(), sizeof(UserAppend) * p.app.size());
   if (!p.bwd_tiles.empty())
     memcpy(host.data() + p.L.bwd_tiles, p.bwd_tiles.data(), sizeof(EncTile) * p.bwd_tiles.size());
+  if (!p.bwd_sched.empty())
+    memcpy(host.data() + p.L.bwd_sched, p.bwd_sched.data(), sizeof(int) * p.bwd_sched.size());
   if (cudaMemcpyAsync(ws, host.data(), host.size(), cudaMemcpyHostToDevice, s) != cudaSuccess) return REST_ERR_CUDA;
   // the status word reports this call only
   if (p.err && cudaMemsetAsync(p.err, 0, sizeof(int32_t), s) != cudaSuccess) return REST_ERR_CUDA;
@@ -1018,9 +1031,20 @@ rest_status rest_attn_backward(rest_dtype dt, const rest_heads* heads, const res
     // delta = rowsum(dO * O); then dq (S, dP and dS K per visible (query, key, head)) and dk, dv
     // (S, dP, P^T dO and dS^T q): 6 + 8 d_h-long products, against 5 in one fused pass
     const double td = (double)p.T * d;
-    REST_KLAUNCH(s, "attn_bwd_delta", 0, td * 2 * e + 4.0 * p.T * H, launch_attn_bwd_simt(bf, hd, 0, a, s));
-    REST_KLAUNCH(s, "attn_bwd_dq", 6.0 * d * pairs, td * (3 * e + 4), launch_attn_bwd_simt(bf, hd, 1, a, s));
-    REST_KLAUNCH(s, "attn_bwd_dkdv", 8.0 * d * pairs, td * (4 * e + 8), launch_attn_bwd_simt(bf, hd, 2, a, s));
+    REST_KLAUNCH(s, "attn_bwd_delta", 0, td * (o_lo ? 3 : 2) * e + 4.0 * p.T * H,
+                 launch_attn_bwd_simt(bf, hd, 0, a, s));
+    if (bf && sm100_attn_supported(hd) && !p.bwd_sched.empty()) {
+      // one pass: S^T, dP^T, dV, dK, dQ per (key block, query block); dq gathers by atomics
+      if (cudaMemsetAsync(dq, 0, sizeof(float) * (size_t)p.T * d, s) != cudaSuccess) return REST_ERR_CUDA;
+      a.sched = at<int>(ws, p.L.bwd_sched);
+      a.n_cta = std::min((int)p.bwd_tiles.size() * H, SCHED_CTAS);
+      // algorithmic bytes: q, k, v, dO in, dq, dk, dv out (fp32), lse and delta
+      REST_KLAUNCH(s, "attn_bwd", 10.0 * d * pairs, td * (4 * e + 12) + 8.0 * p.T * H,
+                   launch_attn_bwd_sm100(hd, a, s, dev_err));
+    } else {
+      REST_KLAUNCH(s, "attn_bwd_dq", 6.0 * d * pairs, td * (3 * e + 4), launch_attn_bwd_simt(bf, hd, 1, a, s));
+      REST_KLAUNCH(s, "attn_bwd_dkdv", 8.0 * d * pairs, td * (4 * e + 8), launch_attn_bwd_simt(bf, hd, 2, a, s));
+    }
     return REST_OK;
   } catch (...) {
     return REST_ERR_INVALID_ARG;

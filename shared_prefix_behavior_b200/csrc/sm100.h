@@ -24,5 +24,8 @@ bool sm100_attn_supported(int head_dim);
 int sm100_attn_tile_rows();
 cudaError_t launch_enc_attn_sm100(int head_dim, const EncAttnArgs& a, cudaStream_t s, int32_t* err);
 cudaError_t launch_dec_attn_sm100(int head_dim, const DecAttnArgs& a, cudaStream_t s, int32_t* err);
+// Backward of the causal attention core (head_dim 32 or 64): dq (zeroed by the
+// caller, accumulated with atomics), dk and dv.
+cudaError_t launch_attn_bwd_sm100(int head_dim, const AttnBwdArgs& a, cudaStream_t s, int32_t* err);
 
 }  // namespace rest

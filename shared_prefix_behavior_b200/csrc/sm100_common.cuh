@@ -270,6 +270,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, int b_mn) {
          | ((uint32_t)(128 >> 4) << 24); // M / 16
 }
 
+// The same with the majorness of A chosen too (a_mn = 1: A MN-major).
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(int n, int a_mn, int b_mn) {
+  return idesc_bf16(n, b_mn) | ((uint32_t)a_mn << 15);
+}
+
 // Shared-memory matrix descriptor (sm100 layout: version 1 at bit 46).
 // swizzle: 2 = 128B, 4 = 64B, 6 = 32B. Offsets in bytes.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t swizzle) {
