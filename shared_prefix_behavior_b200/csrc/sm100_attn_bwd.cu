@@ -11,14 +11,15 @@
 //          written as bf16 into shared memory by the key-row warpgroup
 //   dV  += P^T dO,  dK += dS^T Q                  (accumulated in TMEM over the item)
 //   dQ   = dS K                                   (the dS^T tile read MN-major)
-// and a query-row warpgroup adds dQ into the fp32 dq with vector atomics.
+// and a query-row warpgroup adds dQ into the fp32 dq with vector reductions.
 //   warp 0       TMA producer (K, V per item; Q, dO per block, two stages)
 //   warp 1       TMEM owner and MMA issuer. Order per block g: dV(g) once P^T(g)
 //                is written, S^T(g+1), then dK(g) and dQ(g) once dS^T(g) is
 //                written, dP^T(g+1): the next block's products run while this
 //                block's dS is computed.
-//   warps 4..7   a thread per key row: P^T, dS^T, and the item's dK, dV rows
-//   warps 8..11  a thread per query row of the block: dQ out of TMEM
+//   warps 4..11  two warpgroups, a thread per key row and half of the block's
+//                queries: P^T, dS^T, and the item's dV (first) or dK (second)
+//   warps 12..15 a thread per query row of the block: dQ out of TMEM
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -31,7 +32,8 @@ namespace {
 using namespace sm100;
 
 constexpr int BR = 128;  // keys per item, queries per block
-constexpr int NTHREADS = 384;
+constexpr int NTHREADS = 512;
+constexpr int NKEY = 256;  // threads of the two key-row warpgroups
 constexpr int PBOX = BR * 128;  // one 64-column box of a [128 x 128] bf16 tile (128-byte swizzle)
 
 template <int HD>
@@ -40,7 +42,8 @@ struct BwdCfg {
   static constexpr int TILE = BR * ROW_BYTES;   // one [128 x head_dim] bf16 tile
   static constexpr int SWZ = HD == 64 ? 2 : 4;  // descriptor swizzle of the head tiles: 128B / 64B
   static constexpr int ATOM = 8 * ROW_BYTES;    // bytes of 8 swizzled rows
-  // shared memory: K | V | Q[2] | dO[2] | P^T | dS^T (each [128 x 128], two boxes)
+  // shared memory: K | V | Q[2] | dO[2] | P^T | dS^T; the last two are [128 x 128] bf16 tiles
+  // kept as two 64-column boxes of 128 rows with 128-byte swizzle (queries 0..63, 64..127)
   static constexpr int K_OFF = 0, V_OFF = TILE, Q_OFF = 2 * TILE, G_OFF = 4 * TILE, P_OFF = 6 * TILE;
   static constexpr int DS_OFF = P_OFF + 2 * PBOX;
   static constexpr int TOTAL = DS_OFF + 2 * PBOX;
@@ -48,16 +51,18 @@ struct BwdCfg {
   static constexpr uint32_t S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 256 + HD, DQ_COL = 256 + 2 * HD;
 };
 
-// byte offset of 16-byte chunk u (0..15) of row r in a [128 x 128] bf16 tile
-// kept as two 64-column boxes with 128-byte swizzle
-__device__ __forceinline__ uint32_t pbox_off(int r, int u) { return (u >> 3) * PBOX + sw128_off(r, u & 7); }
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
-__device__ __forceinline__ void named_sync_128(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void named_sync_keys() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// dst[0..3] += v (fp32 reduction in L2, no value returned)
+__device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
 
 // One work item: keys kb*128 .. of user `user`, head h, against query blocks kb .. nqb-1.
 struct BwdItem {
@@ -114,14 +119,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     mbar_init(&s_full, 1);
     mbar_init(&dp_full, 1);
-    mbar_init(&p_ready, BR);
+    mbar_init(&p_ready, NKEY);
     mbar_init(&p_free, 1);
-    mbar_init(&ds_ready, BR);
+    mbar_init(&ds_ready, NKEY);
     mbar_init(&ds_free, 1);
     mbar_init(&dq_full, 1);
     mbar_init(&dq_empty, BR);
     mbar_init(&acc_full, 1);
-    mbar_init(&acc_empty, BR);
+    mbar_init(&acc_empty, NKEY);
     mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
@@ -135,7 +140,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   pdl_release();
 
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    // 4 x 32 x 64 (control) + 8 x 32 x 168 (key rows) + 4 x 32 x 112 (query rows) = 512 x 128
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;");
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
       int g = 0, kv_issued = 0, q_issued = 0;
@@ -241,130 +247,152 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       volatile int no_abort = 0;
       mbar_wait(&drain, 0, nullptr, &no_abort);
     }
+  } else if (warp < 12) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 168;");
+    // -------------------------------------------------------------- key rows: P^T, dS^T, dK, dV
+    // two warpgroups on the same TMEM lanes: warpgroup hf takes query columns [64 hf, 64 hf + 64)
+    // of every block (box hf of the P^T and dS^T tiles) and, at the item's end, dV (hf 0) or dK (hf 1)
+    const int r = (warp & 3) * 32 + lane;  // the key row (TMEM lane)
+    const int hf = (warp - 4) >> 2, c0 = 64 * hf;
+    const int tid = threadIdx.x - 128;     // 0 .. 255
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    int g = 0, kit = 0;
+    // the lse (log2 domain) and delta of query qb * 128 + tid, loaded one block ahead (tid < 128)
+    auto stats = [&](const BwdItem& w, int qb, float& l2, float& dl) {
+      const int qp = qb * BR + tid;
+      l2 = 0.f;
+      dl = 0.f;
+      if (tid < BR && qp < w.len) {
+        const long long ri = (long long)(w.row0 + qp) * a.n_heads + w.h;
+        l2 = a.lse[ri] * 1.4426950408889634f;
+        dl = a.delta[ri];
+      }
+    };
+    for (int k = k_begin; k < k_end && ok; ++k, ++kit) {
+      const BwdItem w = decode_bwd(a, items[k]);
+      const int kpos = w.kb * BR + r;  // this thread's key position in the history
+      float l2_next, dl_next;
+      stats(w, w.kb, l2_next, dl_next);
+      for (int i = 0; i < w.n; ++i, ++g) {
+        const int qb = w.kb + i, b = g & 1;
+        if (tid < BR) {
+          lse_s[b][tid] = l2_next;
+          dlt_s[b][tid] = dl_next;
+        }
+        if (i + 1 < w.n) stats(w, qb + 1, l2_next, dl_next);
+        named_sync_keys();
+        if (!mbar_wait(&s_full, g & 1, err, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        // this half's query column c is visible when kpos <= qb*128 + c0 + c < len
+        const int first = kpos - qb * BR - c0, lim = (kpos < w.len ? w.len - qb * BR : 0) - c0;
+        const bool open = first <= 0 && lim >= 64;  // no masked column in this half
+        float p[64];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float sv[32];
+          tmem_ld32(tmem + lane_off + C::S_COL + c0 + 32 * c, sv);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(&lse_s[b][c0 + 32 * c + e]);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const int col = 32 * c + e + t;
+              const float pv = exp2_approx(fmaf(sv[e + t], sl2, -lv[t]));
+              p[col] = (open || (col >= first && col < lim)) ? pv : 0.f;
+            }
+          }
+        }
+        // P^T(g) into shared memory once dV(g-1) has read P^T(g-1)
+        if (g >= 1 && !mbar_wait(&p_free, (g - 1) & 1, err, &abort_flag)) { ok = false; break; }
+        uint8_t* pt = smem + C::P_OFF + hf * PBOX;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(pt + sw128_off(r, u)) =
+              make_uint4(pack_bf16x2(p[8 * u], p[8 * u + 1]), pack_bf16x2(p[8 * u + 2], p[8 * u + 3]),
+                         pack_bf16x2(p[8 * u + 4], p[8 * u + 5]), pack_bf16x2(p[8 * u + 6], p[8 * u + 7]));
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&p_ready);
+        // dS^T(g) = P^T (dP^T - delta), once dK(g-1), dQ(g-1) have read dS^T(g-1)
+        if (!mbar_wait(&dp_full, g & 1, err, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (g >= 1 && !mbar_wait(&ds_free, (g - 1) & 1, err, &abort_flag)) { ok = false; break; }
+        uint8_t* dst = smem + C::DS_OFF + hf * PBOX;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float dp[32];
+          tmem_ld32(tmem + lane_off + C::DP_COL + c0 + 32 * c, dp);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(&dlt_s[b][c0 + 32 * c + e]);
+            dp[e] = p[32 * c + e] * (dp[e] - d4.x);
+            dp[e + 1] = p[32 * c + e + 1] * (dp[e + 1] - d4.y);
+            dp[e + 2] = p[32 * c + e + 2] * (dp[e + 2] - d4.z);
+            dp[e + 3] = p[32 * c + e + 3] * (dp[e + 3] - d4.w);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(dst + sw128_off(r, 4 * c + u)) =
+                make_uint4(pack_bf16x2(dp[8 * u], dp[8 * u + 1]), pack_bf16x2(dp[8 * u + 2], dp[8 * u + 3]),
+                           pack_bf16x2(dp[8 * u + 4], dp[8 * u + 5]), pack_bf16x2(dp[8 * u + 6], dp[8 * u + 7]));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(&ds_ready);
+      }
+      if (!ok) break;
+      // the item's dV (warpgroup 0) or dK (warpgroup 1) rows
+      if (!mbar_wait(&acc_full, kit & 1, err, &abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t col = hf ? C::DK_COL : C::DV_COL;
+      const float mul = hf ? sl2 * 0.69314718055994531f : 1.f;  // dK carries 1 / sqrt(head_dim)
+      float* out = (hf ? a.dk : a.dv) + (long long)(w.row0 + kpos) * a.d + w.h * HD;
+      float acc[HD];
+#pragma unroll
+      for (int cc = 0; cc < HD; cc += 32) {
+        float t[32];
+        tmem_ld32(tmem + lane_off + col + cc, t);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[cc + e] = t[e] * mul;
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty);  // the accumulators may be started over
+      if (kpos < w.len) {
+#pragma unroll
+        for (int c = 0; c < HD; c += 4) store4(out + c, &acc[c]);
+      }
+    }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
-    const int r = (warp & 3) * 32 + lane;  // TMEM lane: a key row (warps 4..7) or a query row (8..11)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 112;");
+    // -------------------------------------------------------------- query rows: dQ += dS K
+    const int r = (warp & 3) * 32 + lane;  // the query row of the block (TMEM lane)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float scale = a.scale_log2 * 0.69314718055994531f;  // 1 / sqrt(head_dim)
     bool ok = true;
-    int g = 0, kit = 0;
-    if (warp < 8) {
-      // -------------------------------------------------------------- key rows: P^T, dS^T, dK, dV
-      for (int k = k_begin; k < k_end && ok; ++k, ++kit) {
-        const BwdItem w = decode_bwd(a, items[k]);
-        const int kpos = w.kb * BR + r;  // this thread's key position in the history
-        for (int i = 0; i < w.n; ++i, ++g) {
-          const int qb = w.kb + i, b = g & 1;
-          {  // the block's lse (log2 domain) and delta, one query per thread
-            const int qp = qb * BR + r;
-            float l2 = 0.f, dl = 0.f;
-            if (qp < w.len) {
-              const long long ri = (long long)(w.row0 + qp) * a.n_heads + w.h;
-              l2 = a.lse[ri] * 1.4426950408889634f;
-              dl = a.delta[ri];
-            }
-            lse_s[b][r] = l2;
-            dlt_s[b][r] = dl;
-          }
-          named_sync_128(1);
-          if (!mbar_wait(&s_full, g & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          // P^T row: query column c of this block is visible when kpos <= qb*128 + c < len
-          const int first = kpos - qb * BR, lim = kpos < w.len ? w.len - qb * BR : 0;
-          float p[BR];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float sv[32];
-            tmem_ld32(tmem + lane_off + C::S_COL + 32 * c, sv);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int col = 32 * c + e;
-              const float pv = exp2_approx(sv[e] * a.scale_log2 - lse_s[b][col]);
-              p[col] = (col >= first && col < lim) ? pv : 0.f;
-            }
-          }
-          // P^T(g) into shared memory once dV(g-1) has read P^T(g-1)
-          if (g >= 1 && !mbar_wait(&p_free, (g - 1) & 1, err, &abort_flag)) { ok = false; break; }
-          uint8_t* pt = smem + C::P_OFF;
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            *reinterpret_cast<uint4*>(pt + pbox_off(r, u)) =
-                make_uint4(pack_bf16x2(p[8 * u], p[8 * u + 1]), pack_bf16x2(p[8 * u + 2], p[8 * u + 3]),
-                           pack_bf16x2(p[8 * u + 4], p[8 * u + 5]), pack_bf16x2(p[8 * u + 6], p[8 * u + 7]));
-          fence_async_smem();
-          tc_fence_before();
-          mbar_arrive(&p_ready);
-          // dS^T(g) = P^T (dP^T - delta), once dK(g-1), dQ(g-1) have read dS^T(g-1)
-          if (!mbar_wait(&dp_full, g & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          if (g >= 1 && !mbar_wait(&ds_free, (g - 1) & 1, err, &abort_flag)) { ok = false; break; }
-          uint8_t* dst = smem + C::DS_OFF;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float dp[32];
-            tmem_ld32(tmem + lane_off + C::DP_COL + 32 * c, dp);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) dp[e] = p[32 * c + e] * (dp[e] - dlt_s[b][32 * c + e]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              *reinterpret_cast<uint4*>(dst + pbox_off(r, 4 * c + u)) =
-                  make_uint4(pack_bf16x2(dp[8 * u], dp[8 * u + 1]), pack_bf16x2(dp[8 * u + 2], dp[8 * u + 3]),
-                             pack_bf16x2(dp[8 * u + 4], dp[8 * u + 5]), pack_bf16x2(dp[8 * u + 6], dp[8 * u + 7]));
-          }
-          fence_async_smem();
-          tc_fence_before();
-          mbar_arrive(&ds_ready);
-        }
-        if (!ok) break;
-        // the item's dK and dV rows
-        if (!mbar_wait(&acc_full, kit & 1, err, &abort_flag)) { ok = false; break; }
+    int g = 0;
+    for (int k = k_begin; k < k_end && ok; ++k) {
+      const BwdItem w = decode_bwd(a, items[k]);
+      for (int i = 0; i < w.n; ++i, ++g) {
+        const int qpos = (w.kb + i) * BR + r;
+        if (!mbar_wait(&dq_full, g & 1, err, &abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float dvr[HD], dkr[HD];
+        float v[HD];
 #pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += 32) {
-          float t0[32], t1[32];
-          tmem_ld32x2(tmem + lane_off + C::DV_COL + c0, t0, tmem + lane_off + C::DK_COL + c0, t1);
+        for (int cc = 0; cc < HD; cc += 32) {
+          float t[32];
+          tmem_ld32(tmem + lane_off + C::DQ_COL + cc, t);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            dvr[c0 + e] = t0[e];
-            dkr[c0 + e] = t1[e] * scale;
-          }
+          for (int e = 0; e < 32; ++e) v[cc + e] = t[e] * scale;
         }
         tc_fence_before();
-        mbar_arrive(&acc_empty);
-        if (kpos < w.len) {
-          const long long ro = (long long)(w.row0 + kpos) * a.d + w.h * HD;
+        mbar_arrive(&dq_empty);
+        if (qpos < w.len) {
+          float* dst = a.dq + (long long)(w.row0 + qpos) * a.d + w.h * HD;
 #pragma unroll
-          for (int c = 0; c < HD; c += 4) {
-            store4(a.dv + ro + c, &dvr[c]);
-            store4(a.dk + ro + c, &dkr[c]);
-          }
-        }
-      }
-    } else {
-      // -------------------------------------------------------------- query rows: dQ += dS K
-      for (int k = k_begin; k < k_end && ok; ++k) {
-        const BwdItem w = decode_bwd(a, items[k]);
-        for (int i = 0; i < w.n; ++i, ++g) {
-          const int qpos = (w.kb + i) * BR + r;
-          if (!mbar_wait(&dq_full, g & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          float v[HD];
-#pragma unroll
-          for (int c0 = 0; c0 < HD; c0 += 32) {
-            float t[32];
-            tmem_ld32(tmem + lane_off + C::DQ_COL + c0, t);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[c0 + e] = t[e] * scale;
-          }
-          tc_fence_before();
-          mbar_arrive(&dq_empty);
-          if (qpos < w.len) {
-            float* dst = a.dq + (long long)(w.row0 + qpos) * a.d + w.h * HD;
-#pragma unroll
-            for (int c = 0; c < HD; c += 4)
-              atomicAdd(reinterpret_cast<float4*>(dst + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
-          }
+          for (int c = 0; c < HD; c += 4) red_add4(dst + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
         }
       }
     }
