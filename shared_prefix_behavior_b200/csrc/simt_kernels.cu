@@ -534,8 +534,31 @@ cudaError_t launch_to_f32(bool bf16m, const void* x_in, float* x_res, long long 
   return cudaGetLastError();
 }
 
-__global__ void split_bf16_kernel(const float* __restrict__ x, bf16* __restrict__ hi, bf16* __restrict__ lo,
-                                  long long n) {
+// 8 values per thread: two 16-byte loads, a 16-byte store of each part
+__global__ void split_bf16_kernel(const float4* __restrict__ x, uint4* __restrict__ hi, uint4* __restrict__ lo,
+                                  long long n8) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = x[2 * i], b = x[2 * i + 1];
+  const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+    const float2 hf = __bfloat1622float2(h2);
+    const __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * k] - hf.x, v[2 * k + 1] - hf.y);
+    h[k] = *reinterpret_cast<const uint32_t*>(&h2);
+    l[k] = *reinterpret_cast<const uint32_t*>(&l2);
+  }
+  hi[i] = make_uint4(h[0], h[1], h[2], h[3]);
+  lo[i] = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// one value per thread, for sizes or addresses the vector form does not take
+__global__ void split_bf16_scalar_kernel(const float* __restrict__ x, bf16* __restrict__ hi, bf16* __restrict__ lo,
+                                         long long n) {
   pdl_wait();  // the previous kernel of the stream has completed
   pdl_release();
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -549,10 +572,16 @@ __global__ void split_bf16_kernel(const float* __restrict__ x, bf16* __restrict_
 
 cudaError_t launch_split_bf16(const float* x, void* hi, void* lo, long long n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  int threads = 256;
-  long long blocks = (n + threads - 1) / threads;
-  if (cudaError_t e_ = launch_k(split_bf16_kernel, (unsigned)blocks, threads, 0, s, x, (bf16*)hi, (bf16*)lo, n)) return e_;
-  return cudaGetLastError();
+  const int threads = 256;
+  const bool vec = n % 8 == 0 && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(hi) |
+                                   reinterpret_cast<uintptr_t>(lo)) & 15) == 0;
+  if (vec) {
+    const long long n8 = n / 8;
+    return launch_k(split_bf16_kernel, (unsigned)((n8 + threads - 1) / threads), threads, 0, s,
+                    reinterpret_cast<const float4*>(x), static_cast<uint4*>(hi), static_cast<uint4*>(lo), n8);
+  }
+  const long long blocks = (n + threads - 1) / threads;
+  return launch_k(split_bf16_scalar_kernel, (unsigned)blocks, threads, 0, s, x, (bf16*)hi, (bf16*)lo, n);
 }
 
 // ============================================================================
