@@ -344,6 +344,14 @@ rest_status rest_score_head(rest_dtype dt, int d, int K, long long n_cands, cons
                             const rest_score_params* sp, float* f_out, float* score_out,
                             void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
+/* Failure-detection self-test (no GPU fault): launches n_ctas (1..1024) CTAs
+ * whose threads wait, with the bounded wait every library kernel uses, on a
+ * barrier that nothing completes. CTA 0 gives up after limit_cycles SM clock
+ * cycles (1e6 .. 4e9) and writes REST_ERR_TIMEOUT to *dev_err (dev, required);
+ * the other CTAs give up as soon as they see it. After synchronizing, the
+ * word holds REST_ERR_TIMEOUT and the context is usable. */
+rest_status rest_selftest_wait_timeout(int n_ctas, long long limit_cycles, int32_t* dev_err, void* stream);
+
 /* Static description of a status code. */
 const char* rest_status_string(rest_status s);
 

@@ -34,7 +34,7 @@ EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "r
            "rest_rank_request", "rest_status_string", "rest_launch_count", "rest_profile_begin",
            "rest_profile_end", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",
            "rest_append_workspace_size", "rest_encoder_append", "rest_attn_workspace_size", "rest_attn_forward",
-           "rest_attn_backward")
+           "rest_attn_backward", "rest_selftest_wait_timeout")
 STATIC_WS_BYTES = 32 * 1024 * 1024  # REST_STATIC_WS_BYTES
 
 
@@ -111,7 +111,9 @@ def _load() -> ctypes.CDLL:
     lib.rest_attn_forward.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, P, P, P, P, P, c_size_t, P, P]
     lib.rest_attn_backward.argtypes = [c_int, POINTER(Heads), POINTER(Batch), P, P, P, P, P, P, P, P, P, P, P,
                                        c_size_t, P, P]
-    for name in ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
+    lib.rest_selftest_wait_timeout.argtypes = [c_int, c_longlong, P, P]
+    for name in ("rest_selftest_wait_timeout", "rest_workspace_size", "rest_rotation_table", "rest_encoder_attn",
+                 "rest_cross_decode",
                  "rest_rank_request", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",
                  "rest_append_workspace_size", "rest_encoder_append", "rest_attn_workspace_size",
                  "rest_attn_forward", "rest_attn_backward"):
@@ -491,6 +493,16 @@ def attn_backward(q, k, v, o, o_lo, lse, d_o, cu_seqlens, n_heads: int, dq=None,
     if check:
         check_device_error(err)
     return dq, dk, dv
+
+
+def selftest_wait_timeout(device, n_ctas: int = 148, limit_cycles: int = 20_000_000, stream=None) -> int:
+    """Runs the failure-detection self-test and returns the status word it left
+    (REST_ERR_TIMEOUT, 5, when detection works)."""
+    import torch
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(_lib.rest_selftest_wait_timeout(n_ctas, limit_cycles, _ptr(err), _stream(stream)),
+           "rest_selftest_wait_timeout")
+    return int(err.item())
 
 
 def launch_count(reset: bool = False) -> int:

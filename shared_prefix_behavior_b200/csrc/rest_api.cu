@@ -930,6 +930,17 @@ rest_status rest_encoder_append(rest_dtype dt, const rest_heads* heads, const re
   }
 }
 
+rest_status rest_selftest_wait_timeout(int n_ctas, long long limit_cycles, int32_t* dev_err, void* stream) {
+  if (n_ctas < 1 || n_ctas > 1024 || limit_cycles < 1000000LL || limit_cycles > 4000000000LL || !dev_err)
+    return REST_ERR_INVALID_ARG;
+  rest_status st = check_device();
+  if (st != REST_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(dev_err, 0, sizeof(int32_t), s) != cudaSuccess) return REST_ERR_CUDA;
+  REST_KLAUNCH(s, "selftest_wait_timeout", 0, 0, launch_wait_timeout(n_ctas, limit_cycles, dev_err, s));
+  return REST_OK;
+}
+
 rest_status rest_attn_workspace_size(rest_dtype dt, const rest_heads* heads, const rest_batch* batch, size_t* bytes) {
   if (!bytes) return REST_ERR_INVALID_ARG;
   try {

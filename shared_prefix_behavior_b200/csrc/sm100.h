@@ -28,4 +28,8 @@ cudaError_t launch_dec_attn_sm100(int head_dim, const DecAttnArgs& a, cudaStream
 // caller, accumulated with atomics), dk and dv.
 cudaError_t launch_attn_bwd_sm100(int head_dim, const AttnBwdArgs& a, cudaStream_t s, int32_t* err);
 
+// Failure-detection self-test: n_ctas CTAs wait on a barrier nothing completes;
+// CTA 0 gives up after limit_cycles and sets REST_ERR_TIMEOUT, the others on seeing it.
+cudaError_t launch_wait_timeout(int n_ctas, long long limit_cycles, int32_t* err, cudaStream_t s);
+
 }  // namespace rest

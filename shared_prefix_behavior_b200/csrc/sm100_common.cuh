@@ -51,7 +51,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // The abort flag, the global error word and the clock are looked at only
 // every 128 unsuccessful polls, so that a phase that completes is seen at the
 // next poll rather than after a round trip to global memory.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort,
+                                              long long limit_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t n = 1;; ++n) {
@@ -62,12 +63,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
       *abort = 1;
       return false;
     }
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit_cycles) {
       set_error(err, REST_ERR_TIMEOUT);
       *abort = 1;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err, volatile int* abort) {
+  return mbar_wait_for(bar, parity, err, abort, kWaitCycles);
 }
 
 // ------------------------------------------------------------------ TMA

@@ -278,3 +278,13 @@ def test_attention_core_workspace_empty_and_no_device():
     assert 0 < R.attn_workspace_size(R.REST_BF16, 8, 32, [0, 64]) < R.attn_workspace_size(R.REST_BF16, 8, 32, [0, 4096])
     if not gpu_available():
         assert _core("fwd") == NO_DEVICE and _core("bwd") == NO_DEVICE
+
+
+def test_selftest_rejects_invalid_arguments():
+    lib = R.library()
+    assert lib.rest_selftest_wait_timeout(0, 10**7, FAKE, None) == INVALID       # no CTA
+    assert lib.rest_selftest_wait_timeout(2000, 10**7, FAKE, None) == INVALID    # too many
+    assert lib.rest_selftest_wait_timeout(4, 10, FAKE, None) == INVALID          # limit too short
+    assert lib.rest_selftest_wait_timeout(4, 10**7, None, None) == INVALID       # no status word
+    if not gpu_available():
+        assert lib.rest_selftest_wait_timeout(4, 10**7, FAKE, None) == NO_DEVICE
