@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <mutex>
 #include <new>
+#include <queue>
 #include <vector>
 
 #include "common.cuh"
@@ -180,6 +181,57 @@ static std::vector<int> lpt_schedule(const std::vector<long long>& cost) {
   return out;
 }
 
+// Longest finishing time of the longest-first assignment of `cost` to n_cta CTAs.
+static long long lpt_makespan(std::vector<long long> cost, int n_cta) {
+  std::sort(cost.begin(), cost.end(), std::greater<long long>());
+  std::priority_queue<long long, std::vector<long long>, std::greater<long long>> load;
+  for (int c = 0; c < n_cta; ++c) load.push(0);
+  long long most = 0;
+  for (long long c : cost) {
+    const long long l = load.top() + c;
+    load.pop();
+    load.push(l);
+    most = std::max(most, l);
+  }
+  return most;
+}
+
+// Key splits of the decoder when its work items alone would leave SMs idle: the
+// count (1..8, at least about 4 key blocks per split) whose longest-first schedule
+// finishes first, counting an item as its key blocks times its query tiles plus a
+// fixed cost in the same unit (q staging, pipeline fill, the output). The fixed
+// cost, 7 blocks, fits the kernel's measured times at two split counts on two
+// workloads (8 x 4096 and 2 x 16384 keys); a split count wins only when it is at
+// least 5% shorter than every smaller one, since each split also writes a
+// partial output that the combine reads back.
+constexpr long long DEC_ITEM_COST = 7;
+static int choose_dec_split(const rest_batch* b, const rest_requests* r, int K, int rows, int n_heads) {
+  std::vector<DecTile> t;
+  build_dec_tiles(b, r, K, rows, 1, t);
+  if (t.empty()) return 1;
+  const long long base = (long long)t.size() * n_heads;
+  if (base >= TARGET_CTAS) return 1;
+  long long blocks = 0;
+  for (const DecTile& x : t) blocks += x.kb1 - x.kb0;
+  const long long most = std::min(8LL, std::max(1LL, blocks / (long long)t.size() / 4));
+  int best = 1;
+  long long best_t = -1;
+  for (int ns = 1; ns <= most; ++ns) {
+    build_dec_tiles(b, r, K, rows, ns, t);
+    std::vector<long long> cost;
+    for (const DecTile& x : t) {
+      const long long c = (long long)(x.kb1 - x.kb0) * ((x.nrows + 127) / 128) + DEC_ITEM_COST;
+      for (int h = 0; h < n_heads; ++h) cost.push_back(c);
+    }
+    const long long m = lpt_makespan(cost, SCHED_CTAS);
+    if (best_t < 0 || m * 20 < best_t * 19) {
+      best = ns;
+      best_t = m;
+    }
+  }
+  return best;
+}
+
 // app (may be empty): the cached positions before each user's rows
 static std::vector<int> enc_schedule(const rest_batch* b, const std::vector<EncTile>& tiles, int n_heads, int rows,
                                      const std::vector<UserAppend>& app) {
@@ -326,16 +378,7 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   if (encoder_runs) build_enc_tiles(b, tile_rows, p.enc_tiles);
   // split the decoder's keys when its work items alone would leave SMs idle
   p.n_split = 1;
-  if (reqs && tile_rows != 128) {
-    build_dec_tiles(b, reqs, K, tile_rows, 1, p.dec_tiles);
-    long long base = (long long)p.dec_tiles.size() * hs->n_heads, blocks = 0;
-    for (const DecTile& t : p.dec_tiles) blocks += t.kb1 - t.kb0;
-    if (base > 0 && base < TARGET_CTAS) {
-      long long want = (TARGET_CTAS + base - 1) / base;
-      long long most = std::max(1LL, blocks / (long long)p.dec_tiles.size() / 4);  // >= ~4 blocks per split
-      p.n_split = (int)std::min<long long>(8, std::min(want, most));
-    }
-  }
+  if (reqs && tile_rows != 128) p.n_split = choose_dec_split(b, reqs, K, tile_rows, hs->n_heads);
   build_dec_tiles(b, reqs, K, tile_rows, p.n_split, p.dec_tiles);
   // encoder followed by the decoder in bf16: the decoder reads H as hi + lo
   p.n_dec_hlo = 0;
