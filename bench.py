@@ -295,6 +295,32 @@ def component_timings(args, w, t, H, Y, ws, dev, peaks):
     return {"encoder_only": enc_part, "decoder_only": dec_part}
 
 
+def no_sharing_inputs(inp: dict, users, max_cands=None):
+    """The candidates of the given users without the shared prefix: each one a
+    user of its own whose history is its request's prefix (at most max_cands
+    of them). Returns (inputs, the source rows of the re-encoded tokens)."""
+    cu = np.asarray(inp["cu_seqlens"])
+    ru, rc, cc = (np.asarray(inp[k]) for k in ("req_user", "req_cutoff", "cu_cands"))
+    rows, z_rows, lens = [], [], []
+    for r in range(len(ru)):
+        if ru[r] not in users:
+            continue
+        s0 = int(cu[ru[r]])
+        for c in range(int(cc[r]), int(cc[r + 1])):
+            if max_cands is not None and len(lens) >= max_cands:
+                break
+            rows.append(np.arange(s0, s0 + int(rc[r])))
+            z_rows.append(c)
+            lens.append(int(rc[r]))
+    rows = np.concatenate(rows)
+    n = len(lens)
+    ns = dict(inp, x=inp["x"][rows], ts=inp["ts"][rows],
+              cu_seqlens=np.concatenate([[0], np.cumsum(lens)]).astype(np.int32),
+              req_user=np.arange(n, dtype=np.int32), req_cutoff=np.asarray(lens, dtype=np.int32),
+              cu_cands=np.arange(n + 1, dtype=np.int32), z=inp["z"][np.asarray(z_rows)])
+    return ns, rows
+
+
 def sharing_comparison(w, inp, dev, ms_shared):
     """The same candidates without the shared prefix: every candidate becomes a
     user of its own whose history is its request's prefix, encoded and decoded
@@ -311,21 +337,8 @@ def sharing_comparison(w, inp, dev, ms_shared):
             break
         users.append(u)
         tok += need
-    rows, ts_rows, z_rows, lens = [], [], [], []
-    for r in range(len(ru)):
-        if ru[r] not in users:
-            continue
-        s0 = int(cu[ru[r]])
-        for c in range(int(cc[r]), int(cc[r + 1])):
-            rows.append(np.arange(s0, s0 + int(rc[r])))
-            z_rows.append(c)
-            lens.append(int(rc[r]))
-    rows = np.concatenate(rows)
-    n = len(lens)
-    ns = dict(inp, x=inp["x"][rows], ts=inp["ts"][rows],
-              cu_seqlens=np.concatenate([[0], np.cumsum(lens)]).astype(np.int32),
-              req_user=np.arange(n, dtype=np.int32), req_cutoff=np.asarray(lens, dtype=np.int32),
-              cu_cands=np.arange(n + 1, dtype=np.int32), z=inp["z"][np.asarray(z_rows)])
+    ns, rows = no_sharing_inputs(inp, users)
+    n = len(ns["req_user"])
     t = R.to_device(ns, dev)
     args_rank = (t["x"], t["ts"], t["cu_seqlens"], t["taus"], t["layers"], t["l_switch"], t["reqs"], t["z"],
                  t["dec"], t["rope_base"])
@@ -563,9 +576,31 @@ def cpu_baseline(w: W.Workload, inp: dict, budget_s: float) -> dict:
         users.append(u)
         if t_tot >= budget_s:
             break
-    return {"value": c_tot / t_tot, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{len(users)} of {w.n_users} users of {w.name} (encoder + all their candidates), "
-                      f"fp64 numpy, {t_tot:.1f} s", "encoder_tokens_per_s": tok_tot / t_tot}
+    out = {"value": c_tot / t_tot, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+           "sample": f"{len(users)} of {w.n_users} users of {w.name} (encoder + all their candidates), "
+                     f"fp64 numpy, {t_tot:.1f} s", "encoder_tokens_per_s": tok_tot / t_tot}
+    # the oracle without the shared prefix: candidates of user 0, each re-encoding
+    # its request's prefix, one at a time until a quarter of the budget is spent
+    # (prefixes of at most 2048 tokens: longer ones take one candidate past it)
+    from oracle import rest_oracle as O
+    own = [r for r in range(len(inp["req_user"])) if int(inp["req_user"][r]) == 0]
+    if max(int(inp["req_cutoff"][r]) for r in own) > 2048:
+        out["no_sharing"] = {"skipped": "user 0 has a prefix longer than 2048 tokens"}
+        return out
+    ns, _ = no_sharing_inputs(inp, [0], max_cands=16)
+    t_alone, n_alone = 0.0, 0
+    while t_alone < budget_s / 4 and n_alone < len(ns["req_user"]):
+        one = W.subset_users(ns, [n_alone])
+        t0 = time.perf_counter()
+        O.rank_request(one)
+        t_alone += time.perf_counter() - t0
+        n_alone += 1
+    shared = t_tot / c_tot
+    out["no_sharing"] = {"candidates": n_alone, "s_per_candidate_alone": t_alone / n_alone,
+                         "s_per_candidate_shared": shared, "speedup_of_sharing": t_alone / n_alone / shared,
+                         "sample": f"the first {n_alone} candidates of user 0, each encoding its request's "
+                                   f"prefix alone, fp64 numpy, {t_alone:.1f} s"}
+    return out
 
 
 def run_reference(args, rank: int):
