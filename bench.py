@@ -53,11 +53,11 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (91120640, "attn", "cefea56c5f2c23d0",
+    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89436416, "attn", "b1642b8d5af3c5df",
                                                 "profiles/attn_tc_kernel_bf16-32x1024-d256.md"),
-    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (256857856, "attn", "cefea56c5f2c23d0",
+    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (256394496, "attn", "b1642b8d5af3c5df",
                                                     "profiles/attn_tc_kernel_bf16-8x4096-d512.md"),
-    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (286871296, "attn", "cefea56c5f2c23d0",
+    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (283005184, "attn", "b1642b8d5af3c5df",
                                                    "profiles/attn_tc_kernel_bf16-2x16384-d512.md"),
 }
 
