@@ -43,53 +43,74 @@ __device__ __forceinline__ void rotation(long long idx, const TableParams& p, in
   sincospi(2.0 * tr, sv, cv);
 }
 
-// One thread per (token, frequency j), looping over the heads: the user lookup
-// happens once per token, and consecutive threads write consecutive entries.
-// With `app` the rows are tokens appended to cached histories: positions
-// continue after the cached ones and time still counts from the history's
-// first timestamp.
-__global__ void rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu,
-                                      int n_users, int T, TableParams p, int64_t* idx_out,
-                                      float* cos_out, float* sin_out, int32_t* err,
-                                      const UserAppend* __restrict__ app) {
+// A block takes TB = min(256 / half, 128) consecutive tokens. Its first threads find
+// each token's user and, per (token, head), the rotation index (one exact
+// integer division per time head, shared by all the head's frequencies);
+// then one thread per (token, frequency j) loops over the heads, so that
+// consecutive threads write consecutive table entries. With `app` the rows
+// are tokens appended to cached histories: positions continue after the
+// cached ones and time still counts from the history's first timestamp.
+constexpr int ROT_THREADS = 256;
+constexpr int ROT_MAX_HEADS = 32;  // TableParams::tau
+constexpr int ROT_TB_MAX = 128;    // tokens per block
+
+__host__ __device__ __forceinline__ int rot_tokens_per_block(int half) {
+  return ROT_THREADS / half < ROT_TB_MAX ? ROT_THREADS / half : ROT_TB_MAX;
+}
+
+__global__ void __launch_bounds__(ROT_THREADS)
+    rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu, int n_users, int T,
+                          TableParams p, int64_t* idx_out, float* cos_out, float* sin_out, int32_t* err,
+                          const UserAppend* __restrict__ app) {
+  __shared__ long long s_idx[ROT_TB_MAX][ROT_MAX_HEADS];
+  __shared__ long long s_rel[ROT_TB_MAX], s_pos[ROT_TB_MAX];
   pdl_wait();  // the previous kernel of the stream has completed
   pdl_release();
-  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= (long long)T * p.half) return;
-  const int i = (int)(gid / p.half);
-  const int j = (int)(gid % p.half);
-  const int u = find_user(cu, n_users, i);
-  const int s = cu[u];
-  const int cached = app ? app[u].cached : 0;
-  const long long t = ts[i];
-  if (j == 0) {
+  const int TB = rot_tokens_per_block(p.half);
+  const int i0 = blockIdx.x * TB;
+  const int nt = min(TB, T - i0);
+  const int H = p.n_heads;
+  for (int k = threadIdx.x; k < nt; k += blockDim.x) {  // per token: user, time since its first token, position
+    const int i = i0 + k;
+    const int u = find_user(cu, n_users, i);
+    const int s = cu[u];
+    const int cached = app ? app[u].cached : 0;
+    const long long t = ts[i];
     if (i > s ? ts[i - 1] > t : (cached > 0 && app[u].t_prev > t)) set_error(err, REST_ERR_UNSORTED_TIME);
+    s_rel[k] = t - (cached > 0 ? app[u].t_origin : ts[s]);  // exact int64
+    s_pos[k] = (long long)(i - s) + cached;
   }
-  const long long rel = t - (cached > 0 ? app[u].t_origin : ts[s]);  // exact int64
-  const long long pos = (long long)(i - s) + cached;
-  for (int h = 0; h < p.n_heads; ++h) {
+  __syncthreads();
+  for (int k = threadIdx.x; k < nt * H; k += blockDim.x) {  // per (token, head): the rotation index
+    const int tk = k / H, h = k % H;
     const long long tau = p.tau[h];
-    const long long idx = tau == 0 ? pos : floor_div(rel, tau);
-    if (idx_out && j == 0) idx_out[(long long)i * p.n_heads + h] = idx;
-    if (cos_out) {
-      double sv, cv;
-      rotation(idx, p, j, &sv, &cv);
-      const long long o = ((long long)i * p.n_heads + h) * p.half + j;
-      cos_out[o] = (float)cv;
-      sin_out[o] = (float)sv;
-    }
+    const long long idx = tau == 0 ? s_pos[tk] : floor_div(s_rel[tk], tau);
+    s_idx[tk][h] = idx;
+    if (idx_out) idx_out[(long long)(i0 + tk) * H + h] = idx;
+  }
+  __syncthreads();
+  if (!cos_out) return;
+  const int tk = threadIdx.x / p.half, j = threadIdx.x % p.half;
+  if (tk >= nt) return;
+  const long long i = i0 + tk;
+  for (int h = 0; h < H; ++h) {
+    double sv, cv;
+    rotation(s_idx[tk][h], p, j, &sv, &cv);
+    const long long o = (i * H + h) * p.half + j;
+    cos_out[o] = (float)cv;
+    sin_out[o] = (float)sv;
   }
 }
 
 cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users, int T,
                                     const TableParams& p, int64_t* idx_out, float* cos_out,
                                     float* sin_out, int32_t* err, cudaStream_t s, const UserAppend* app) {
-  const long long n = (long long)T * p.half;
-  if (n == 0) return cudaSuccess;
-  const int threads = 256;
-  const long long blocks = (n + threads - 1) / threads;
-  if (cudaError_t e_ = launch_k(rotation_table_kernel, (unsigned)blocks, threads, 0, s, ts, cu, n_users, T, p, idx_out, cos_out,
-                                                             sin_out, err, app)) return e_;
+  if (T == 0) return cudaSuccess;
+  if (p.half < 1 || p.half > 64 || p.n_heads < 1 || p.n_heads > ROT_MAX_HEADS) return cudaErrorInvalidValue;
+  const int tb = rot_tokens_per_block(p.half);
+  const long long blocks = ((long long)T + tb - 1) / tb;
+  if (cudaError_t e_ = launch_k(rotation_table_kernel, (unsigned)blocks, ROT_THREADS, 0, s, ts, cu, n_users, T, p,
+                                idx_out, cos_out, sin_out, err, app)) return e_;
   return cudaGetLastError();
 }
 
