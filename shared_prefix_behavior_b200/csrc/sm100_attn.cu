@@ -46,6 +46,7 @@ constexpr int ROWS = 128;  // query rows per tile
 constexpr int NT = 2;      // tiles per CTA
 constexpr int KB = 128;    // keys per block
 constexpr int NTHREADS = 384;
+constexpr int ITEM_CACHE = 64;  // work items per CTA decoded into shared memory up front
 constexpr float RESCALE_LOG2 = 8.0f;  // rescale O when the row max grows by more than 2^8
 
 template <int HD>
@@ -192,6 +193,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // exponentials of its n-th key block (two barriers per pair so that a warp one
   // or two blocks ahead never completes the phase its partner still waits for)
   __shared__ uint64_t xe[NT][4][2];
+  __shared__ AttnItem s_items[HD <= 32 ? ITEM_CACHE : 1];
   __shared__ uint32_t tslot;
   __shared__ volatile int abort_flag;
 
@@ -231,6 +233,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = tslot;
   pdl_wait();  // the previous kernel of the stream has completed: its outputs may be read
   pdl_release();
+  // head_dim 32: the CTA's first ITEM_CACHE work items, decoded once by warp 3
+  // (a lane per item, so their chains of dependent loads overlap) for every
+  // role to read from shared memory; later items are decoded where they are
+  // used. Items there are short (a few key blocks), and each role's decode, three
+  // dependent global loads, was about 5 % of an item. head_dim 64 decodes in
+  // place: its items are long, and the table cost registers in its softmax.
+  constexpr bool CACHE_ITEMS = HD <= 32;
+  const int k_first = sched[blockIdx.x];
+  if (CACHE_ITEMS && warp == 3) {
+    const int n = min(sched[blockIdx.x + 1] - k_first, ITEM_CACHE);
+    for (int i = lane; i < n; i += 32) s_items[i] = decode_item<DEC>(ea, da, items[k_first + i]);
+  }
+  __syncthreads();
+  auto item_at = [&](int k) -> AttnItem {
+    return CACHE_ITEMS && k - k_first < ITEM_CACHE ? s_items[k - k_first] : decode_item<DEC>(ea, da, items[k]);
+  };
 
   if (warp < 4) {
     setmaxnreg_dec72();
@@ -239,7 +257,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int g = 0, issued = 0, qn[NT] = {0, 0};
       bool ok = true;
       for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-        const AttnItem w = decode_item<DEC>(ea, da, items[k]);
+        const AttnItem w = item_at(k);
         if (!DEC) {
           for (int t = 0; t < NT && ok; ++t) {
             if (w.nblk[t] == 0) continue;
@@ -290,7 +308,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int g = 0, cb = 0, qn = 0;
         bool ok = true;
         for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-          const AttnItem w = decode_item<DEC>(ea, da, items[k]);
+          const AttnItem w = item_at(k);
           const int nblk_all = max(w.nblk[0], w.nblk[1]);
           const int nb = w.nblk[t];
           if (nb > 0) ok = mbar_wait(&q_full[t], qn & 1, err, &abort_flag);
@@ -372,7 +390,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int g = 0, cb[NT] = {0, 0}, qn[NT] = {0, 0};
         bool ok = true;
         for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-          const AttnItem w = decode_item<DEC>(ea, da, items[k]);
+          const AttnItem w = item_at(k);
           const int nblk_all = max(w.nblk[0], w.nblk[1]);
           for (int t = 0; t < NT && ok; ++t)
             if (w.nblk[t] > 0) ok = mbar_wait(&q_full[t], qn[t] & 1, err, &abort_flag);
@@ -485,7 +503,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int cb = 0, qn = 0, cbo = 0;  // cbo: the other tile's key blocks in earlier items
     bool ok = true;
     for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-      const AttnItem w = decode_item<DEC>(ea, da, items[k]);
+      const AttnItem w = item_at(k);
       const int nb = w.nblk[t];
       const bool valid = r < w.nrow[t];
       const long long row_g = (long long)(w.q_row0 + t * ROWS + r);
