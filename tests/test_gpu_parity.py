@@ -138,7 +138,7 @@ def test_bf16_decoder_with_synthetic_memory(cuda):
 @pytest.mark.parametrize("hd", [32, 64])
 def test_bf16_decoder_split_keys(cuda, hd):
     """Few query rows against long prefixes: the tensor-core decoder splits the
-    keys across CTAs (one split of the 300-key request is empty) and combines
+    keys across CTAs (the 1-key request's first split is empty) and combines
     the partial results."""
     w = W.small_workload("bf16", lengths=(2000, 300), d=4 * hd, n_heads=4,
                          requests=[(0, 2000, 20), (1, 300, 7), (0, 1, 3), (0, 1500, 2)])
@@ -148,8 +148,11 @@ def test_bf16_decoder_split_keys(cuda, hd):
     assert_parity(y, oracle_decode(inp, Hm), "bf16", "y")
 
 
-def test_bf16_rank_request_split_keys(cuda):
-    w = W.small_workload("bf16", lengths=(1800, 300), d=128, n_heads=4, n_layers=1, l_switch=0,
+@pytest.mark.parametrize("hd", [32, 64])
+def test_bf16_rank_request_split_keys(cuda, hd):
+    """The split decoder after an encoder in the same call: prefixes under 1024
+    keys also read H_lo (the third operand pair of the tensor-core decoder)."""
+    w = W.small_workload("bf16", lengths=(1800, 300), d=4 * hd, n_heads=4, n_layers=1, l_switch=0,
                          requests=[(0, 1800, 12), (1, 300, 5), (0, 400, 3)])
     inp = W.make_inputs(w, 48)
     H, y = run_rank(inp, cuda)
