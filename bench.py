@@ -53,11 +53,11 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89436416, "attn", "b1642b8d5af3c5df",
+    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89037824, "attn", "f6f2ff69b36ea278",
                                                 "profiles/attn_tc_kernel_bf16-32x1024-d256.md"),
-    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (256394496, "attn", "b1642b8d5af3c5df",
+    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (255269888, "attn", "f6f2ff69b36ea278",
                                                     "profiles/attn_tc_kernel_bf16-8x4096-d512.md"),
-    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (283005184, "attn", "b1642b8d5af3c5df",
+    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (297228032, "attn", "f6f2ff69b36ea278",
                                                    "profiles/attn_tc_kernel_bf16-2x16384-d512.md"),
 }
 
