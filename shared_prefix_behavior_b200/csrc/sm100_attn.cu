@@ -79,7 +79,10 @@ struct SmemLayout {
   static constexpr int KV = (MODE >= 1 ? 2 : 1) * NT * Cfg<HD>::TILE_BYTES;
   // a stage holds K and V' (encoder), H (decoder), or H_hi and H_lo
   static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
-  static constexpr int TOTAL = KV + STAGES * STAGE;
+  // encoder: per softmax warp, its 32 output rows in bf16 (rows padded by 16 bytes)
+  static constexpr int STG_ROW = HD * 2 + 16;
+  static constexpr int STG = KV + STAGES * STAGE;
+  static constexpr int TOTAL = STG + (MODE == 0 ? 8 * 32 * STG_ROW : 0);
 };
 
 // Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
@@ -668,7 +671,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&o_empty[t]);  // O_t may now be overwritten by the next item
-      if (valid && split) {  // partial result of this key range, combined later
+      if (!DEC && ea.out_lo == nullptr) {
+        // The output rows through shared memory: each lane writes its row's bf16
+        // values into the warp's staging rows, then the warp stores them 16 bytes a
+        // lane, HD / 8 lanes to a row, so that a store instruction writes whole
+        // sectors of a few rows instead of 8 bytes of each of 32 rows.
+        const float inv = valid ? 1.0f / l_run : 0.f;
+        if (valid && ea.lse) ea.lse[row_g * n_heads + h] = (m_ref + log2f(l_run)) * 0.69314718055994531f;
+        uint8_t* stg = smem + L::STG + (warp - 4) * 32 * L::STG_ROW;
+#pragma unroll
+        for (int c0 = 0; c0 < HD; c0 += 8) {
+          float gh[8];
+          if (!has_gate || !valid) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) gh[i] = 1.f;
+          } else if (GATE_EARLY) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) gh[i] = gate_row[(c0 + i) % (GATE_EARLY ? HD : 4)];
+          } else {
+            load4(ea.gate + ro + c0, gh);
+            load4(ea.gate + ro + c0 + 4, gh + 4);
+          }
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[c0 + 2 * i] * inv * gh[2 * i], o[c0 + 2 * i + 1] * inv * gh[2 * i + 1]);
+            pk[i] = *reinterpret_cast<uint32_t*>(&t2);
+          }
+          *reinterpret_cast<uint4*>(stg + lane * L::STG_ROW + c0 * 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        __syncwarp();
+        constexpr int CPR = HD / 8;  // 16-byte chunks of a row
+#pragma unroll
+        for (int rr = 0; rr < 32; rr += 32 / CPR) {
+          const int r = rr + lane / CPR, ch = lane % CPR;
+          const int tr = q4 * 32 + r;  // row within the tile
+          if (tr < w.nrow[t]) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * L::STG_ROW + ch * 16);
+            *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(ea.out) + (long long)(w.q_row0 + t * ROWS + tr) * d +
+                                      h * HD + ch * 8) = val;
+          }
+        }
+        __syncwarp();  // the staging rows are free for the next item
+      } else if (valid && split) {  // partial result of this key range, combined later
         float* po = da.part_o + ((long long)w.split * da.nk_rows + row_g) * d + h * HD;
 #pragma unroll
         for (int c = 0; c < HD; c += 4) store4(po + c, &o[c]);
