@@ -57,11 +57,11 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89037824, "attn", "f6f2ff69b36ea278",
+    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89945344, "attn", "4d3f95c2bf757856",
                                                 "profiles/attn_tc_kernel_bf16-32x1024-d256.md"),
-    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (255269888, "attn", "f6f2ff69b36ea278",
+    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (261767168, "attn", "4d3f95c2bf757856",
                                                     "profiles/attn_tc_kernel_bf16-8x4096-d512.md"),
-    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (297228032, "attn", "f6f2ff69b36ea278",
+    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (287949568, "attn", "4d3f95c2bf757856",
                                                    "profiles/attn_tc_kernel_bf16-2x16384-d512.md"),
 }
 
