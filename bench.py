@@ -26,6 +26,7 @@ import dataclasses
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -57,20 +58,25 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89945344, "attn", "4d3f95c2bf757856",
+    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89945344, "attn", "f517c71877da86dc",
                                                 "profiles/attn_tc_kernel_bf16-32x1024-d256.md"),
-    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (261767168, "attn", "4d3f95c2bf757856",
+    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (261767168, "attn", "f517c71877da86dc",
                                                     "profiles/attn_tc_kernel_bf16-8x4096-d512.md"),
-    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (287949568, "attn", "4d3f95c2bf757856",
+    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (287949568, "attn", "f517c71877da86dc",
                                                    "profiles/attn_tc_kernel_bf16-2x16384-d512.md"),
 }
 
 
 def source_digest(kind: str) -> str:
+    """Digest of the kernel's code: its sources with comments and blank space
+    removed, so that a comment edit keeps a capture's figures."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kind]:
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

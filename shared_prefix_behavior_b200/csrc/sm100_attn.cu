@@ -15,6 +15,8 @@
 //                into the tile's head_dim-column accumulator. head_dim 32: one
 //                thread issues for both tiles in lockstep; head_dim 64: warp 1
 //                issues for tile 0 and warp 2 for tile 1.
+//   warp 3       head_dim 32: decodes the CTA's work items into a shared-memory
+//                table at the start (a lane per item).
 //   warps 4..7   softmax of tile 0, warps 8..11 of tile 1: a thread owns a
 //                query row; it reads its row of S from TMEM, masks, keeps the
 //                running max, exponentiates in base 2, and writes P (bf16
@@ -25,7 +27,8 @@
 //                max (values up to 2^8, exact in fp32 accumulation). At
 //                head_dim 64 the two tiles' warps of a lane quarter, which
 //                share a sub-partition's special-function unit, take turns at
-//                the exponentials block by block.
+//                the exponentials block by block. The encoder's output rows go
+//                out through a per-warp staging area in shared memory.
 // The decoder's query comes in fp32 and is staged as a hi + lo pair of bf16
 // tiles (S = q_hi H^T + q_lo H^T); when the encoder ran in the same call the
 // decoder also reads H_lo (H = H_hi + H_lo): S adds q_hi H_lo^T, O adds P H_lo.
