@@ -106,7 +106,10 @@ struct GemmArgs {
 cudaError_t launch_gemm_simt(bool bf16, const GemmArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
-struct EncTile { int user; int q0; };          // q0: first query position within the user
+// Encoder work item: query positions [q0, q0 + rows) of a user. With kb1 > 0
+// (appending, keys split across CTAs) it covers only the 128-key blocks
+// [kb0, kb1) of the user's keys and writes partial results as split `split`.
+struct EncTile { int user; int q0; int kb0; int kb1; int split; };
 // Decoder work item: query rows [row0, row0 + nrows) against the first nkeys
 // rows of H starting at key0; it covers the 128-key blocks [kb0, kb1) and, when
 // the launch splits keys, writes partial results as split number `split`.
@@ -131,8 +134,14 @@ struct EncAttnArgs {
   // at position app[u].cached + i.
   const UserAppend* app;
   long long key_rows;
+  // Keys split across CTAs (tensor-core kernel, appending): per split the
+  // unnormalised fp32 output [n_split, rows, d] and its reference max m (log2
+  // domain) and sum l [n_split, rows, n_heads, 2]; launch_enc_combine merges
+  // them, normalises, applies the gate and writes out.
+  float* part_o; float* part_ml; int n_split;
 };
 cudaError_t launch_enc_attn_simt(bool bf16, int hd, const EncAttnArgs& a, cudaStream_t s);
+cudaError_t launch_enc_combine(int hd, const EncAttnArgs& a, cudaStream_t s);
 
 // Backward of the causal attention core (training; the forward wrote o and lse
 // with the gate left out): dq, dk, dv from d_o = dL/dO.

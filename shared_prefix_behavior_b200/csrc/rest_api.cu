@@ -232,19 +232,83 @@ static int choose_dec_split(const rest_batch* b, const rest_requests* r, int K, 
   return best;
 }
 
-// app (may be empty): the cached positions before each user's rows
+// Key blocks an encoder item reads, summed over its 128-row query tiles (each
+// reads every key up to its last row; with split keys only blocks [kb0, kb1)).
+// app (may be empty): the cached positions before each user's rows.
+static long long enc_item_cost(const rest_batch* b, const std::vector<UserAppend>& app, const EncTile& t, int rows) {
+  const int n = b->cu_seqlens[t.user + 1] - b->cu_seqlens[t.user];
+  const int off = app.empty() ? 0 : app[t.user].cached;
+  long long c = 0;
+  for (int r0 = t.q0; r0 < std::min(n, t.q0 + rows); r0 += 128) {
+    int nb = (std::min(off + n, off + r0 + 128) + 127) / 128;
+    if (t.kb1 > 0) nb = std::max(0, std::min(nb, t.kb1) - t.kb0);
+    c += nb;
+  }
+  return c;
+}
+
 static std::vector<int> enc_schedule(const rest_batch* b, const std::vector<EncTile>& tiles, int n_heads, int rows,
                                      const std::vector<UserAppend>& app) {
   std::vector<long long> cost;
   for (const EncTile& t : tiles) {
-    const int n = b->cu_seqlens[t.user + 1] - b->cu_seqlens[t.user];
-    const int off = app.empty() ? 0 : app[t.user].cached;
-    long long c = 0;
-    for (int r0 = t.q0; r0 < std::min(n, t.q0 + rows); r0 += 128)
-      c += (std::min(off + n, off + r0 + 128) + 127) / 128;
+    const long long c = enc_item_cost(b, app, t, rows);
     for (int h = 0; h < n_heads; ++h) cost.push_back(c);
   }
   return lpt_schedule(cost);
+}
+
+constexpr int MAX_ENC_SPLIT = 16;
+// Appending on the tensor-core path: when the items alone would leave SMs idle
+// (a few users' new rows against long cached prefixes), every tile's key blocks
+// are split over n_split items whose partial results a combine kernel merges.
+// The count is chosen as the decoder's is (longest-first makespan with the same
+// per-item cost; a larger count must win by 5 %), among the counts where every
+// split has at least two blocks and begins at or before the tile's first query
+// position, so that each query row sees at least one key in every split.
+static void split_enc_tiles(const rest_batch* b, const std::vector<UserAppend>& app, int rows, int n_heads,
+                            std::vector<EncTile>& tiles, int* n_split) {
+  *n_split = 1;
+  if (app.empty() || tiles.empty() || (long long)tiles.size() * n_heads >= TARGET_CTAS) return;
+  auto blocks_all = [&](const EncTile& t) {  // key blocks of the item's last query row
+    const int n = b->cu_seqlens[t.user + 1] - b->cu_seqlens[t.user], off = app[t.user].cached;
+    return (std::min(off + n, off + t.q0 + rows) + 127) / 128;
+  };
+  auto split_of = [&](int ns) {
+    std::vector<EncTile> out;
+    for (const EncTile& t : tiles) {
+      const int nb = blocks_all(t);
+      for (int sp = 0; sp < ns; ++sp)
+        out.push_back(EncTile{t.user, t.q0, (int)((long long)nb * sp / ns), (int)((long long)nb * (sp + 1) / ns), sp});
+    }
+    return out;
+  };
+  auto makespan = [&](const std::vector<EncTile>& ts) {
+    std::vector<long long> cost;
+    for (const EncTile& t : ts) {
+      const long long c = enc_item_cost(b, app, t, rows) + DEC_ITEM_COST;
+      for (int h = 0; h < n_heads; ++h) cost.push_back(c);
+    }
+    return lpt_makespan(cost, SCHED_CTAS);
+  };
+  int best = 1;
+  long long best_t = makespan(tiles);
+  for (int ns = 2; ns <= MAX_ENC_SPLIT; ++ns) {
+    bool ok = true;
+    for (const EncTile& t : tiles) {
+      const int nb = blocks_all(t), first = app[t.user].cached + t.q0;
+      if (nb / ns < 2 || (long long)nb * (ns - 1) / ns * 128 > first) ok = false;
+    }
+    if (!ok) continue;
+    const long long m = makespan(split_of(ns));
+    if (m * 20 < best_t * 19) {
+      best = ns;
+      best_t = m;
+    }
+  }
+  if (best > 1) {
+    tiles = split_of(best);
+    *n_split = best;
+  }
 }
 
 static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_heads) {
@@ -269,7 +333,7 @@ struct Layout {
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
                           int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split,
                           size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2, bool append,
-                          int n_bwd_tiles = 0, size_t n_bwd_sched = 0) {
+                          int n_bwd_tiles = 0, size_t n_bwd_sched = 0, int n_split_enc = 1) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
   const size_t d = (size_t)hs->d;
@@ -302,8 +366,11 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dg = take(4 * (size_t)NK * d);
   L.dout = take(4 * (size_t)NK * d);
   L.hlo = take(hsplit ? 2 * (size_t)T * d : 0);
-  L.part_o = take(n_split > 1 ? 4 * (size_t)n_split * NK * d : 0);
-  L.part_ml = take(n_split > 1 ? 8 * (size_t)n_split * NK * hs->n_heads : 0);
+  // split partial results: the decoder's [n_split, NK] or the appending encoder's [n_split_enc, T] rows
+  const size_t part_rows = std::max(n_split > 1 ? (size_t)n_split * NK : 0,
+                                    n_split_enc > 1 ? (size_t)n_split_enc * T : 0);
+  L.part_o = take(4 * part_rows * d);
+  L.part_ml = take(8 * part_rows * hs->n_heads);
   L.delta = take(n_bwd_tiles > 0 ? 4 * (size_t)T * hs->n_heads : 0);
   L.total = off;
   return L;
@@ -325,7 +392,8 @@ struct Plan {
   Layout L;
   int32_t* err;
   bool hsplit;
-  int n_split;  // decoder key splits (tensor-core path)
+  int n_split;      // decoder key splits (tensor-core path)
+  int n_split_enc;  // encoder key splits when appending (tensor-core path)
 };
 
 // The cache of an append: region bounds, cached lengths and their fit, the
@@ -376,6 +444,19 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   if (p.T * (long long)hs->d >= (1LL << 40) || p.NK >= (1LL << 31)) return REST_ERR_UNSUPPORTED;
   const int tile_rows = attn_tile_rows(dt, hs->head_dim);
   if (encoder_runs) build_enc_tiles(b, tile_rows, p.enc_tiles);
+  p.n_split_enc = 1;
+  if (encoder_runs && append && tile_rows != 128) {
+    if (cache) {
+      split_enc_tiles(b, p.app, tile_rows, hs->n_heads, p.enc_tiles, &p.n_split_enc);
+    } else if ((long long)p.enc_tiles.size() * hs->n_heads < TARGET_CTAS) {
+      // the workspace query (no cache yet): room for the most splits a call can take
+      std::vector<EncTile> most;
+      for (const EncTile& t : p.enc_tiles)
+        for (int sp = 0; sp < MAX_ENC_SPLIT; ++sp) most.push_back(EncTile{t.user, t.q0, 0, 1, sp});
+      p.enc_tiles.swap(most);
+      p.n_split_enc = MAX_ENC_SPLIT;
+    }
+  }
   // split the decoder's keys when its work items alone would leave SMs idle
   p.n_split = 1;
   if (reqs && tile_rows != 128) p.n_split = choose_dec_split(b, reqs, K, tile_rows, hs->n_heads);
@@ -416,7 +497,7 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   }
   p.L = make_layout(dt, hs, b, p.T, encoder_runs && !core, p.max_dff, p.NK, (int)p.enc_tiles.size(),
                     (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size(),
-                    p.dec_sched2.size(), append, (int)p.bwd_tiles.size(), p.bwd_sched.size());
+                    p.dec_sched2.size(), append, (int)p.bwd_tiles.size(), p.bwd_sched.size(), p.n_split_enc);
   return REST_OK;
 }
 
@@ -623,6 +704,11 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   ea.rows = T;
   ea.app = app;
   ea.key_rows = cache ? cache->rows : T;
+  ea.n_split = p.n_split_enc;
+  if (p.n_split_enc > 1) {
+    ea.part_o = at<float>(ws, L.part_o);
+    ea.part_ml = at<float>(ws, L.part_ml);
+  }
 
   // The sublayers in order (attention, then the FFN, per layer), each wrapped
   // by eq. 6: post-LN in the first l_switch layers, pre-LN after. One
@@ -676,6 +762,9 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
       }
       if (bf && sm100_attn_supported(hd)) {
         REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_sm100(hd, ea, s, err));
+        if (p.n_split_enc > 1)
+          REST_KLAUNCH(s, "enc_combine", 0, Td * (4.0 * (p.n_split_enc + 1) + e),
+                       launch_enc_combine(hd, ea, s));
       } else {
         REST_KLAUNCH(s, "enc_attn", attn_flops, attn_bytes, launch_enc_attn_simt(bf, hd, ea, s));
       }

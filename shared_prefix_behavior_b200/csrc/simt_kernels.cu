@@ -1047,6 +1047,45 @@ cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Split-key encoder (appending): out = dt((sum_s 2^(m_s - M) O_s) / (sum_s 2^(m_s - M) l_s) * gate),
+// M = max_s m_s; one thread per 4 output columns of a row. Every split of a
+// valid row holds at least one visible key, so M is finite.
+__global__ void enc_combine_kernel(EncAttnArgs a, int hd) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int cols4 = a.d / 4;
+  if (gid >= a.rows * cols4) return;
+  const long long row = gid / cols4;
+  const int c = (int)(gid % cols4) * 4;
+  const int h = c / hd;
+  float M = -INFINITY;
+  for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, a.part_ml[((s * a.rows + row) * a.n_heads + h) * 2]);
+  float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < a.n_split; ++s) {
+    const float* ml = a.part_ml + ((s * a.rows + row) * a.n_heads + h) * 2;
+    if (ml[0] == -INFINITY) continue;  // a split with no keys
+    const float w = exp2f(ml[0] - M);
+    L = fmaf(w, ml[1], L);
+    float v[4];
+    load4(a.part_o + (s * a.rows + row) * a.d + c, v);
+    for (int i = 0; i < 4; ++i) o[i] = fmaf(w, v[i], o[i]);
+  }
+  float g[4] = {1.f, 1.f, 1.f, 1.f};
+  if (a.gate) load4(a.gate + row * a.d + c, g);
+  const float inv = 1.0f / L;
+  float r[4] = {o[0] * inv * g[0], o[1] * inv * g[1], o[2] * inv * g[2], o[3] * inv * g[3]};
+  store4((bf16*)a.out + row * a.d + c, r);
+}
+
+cudaError_t launch_enc_combine(int hd, const EncAttnArgs& a, cudaStream_t s) {
+  const long long n = a.rows * (a.d / 4);
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  if (cudaError_t e_ = launch_k(enc_combine_kernel, (unsigned)((n + threads - 1) / threads), threads, 0, s, a, hd)) return e_;
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- attention backward
 // delta[i, h] = sum over the head's columns of dO * O (one thread per row and head)
 template <typename T>

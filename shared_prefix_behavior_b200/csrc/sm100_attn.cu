@@ -125,7 +125,8 @@ struct AttnItem {
   int user_len;   // encoder: keys of the user's history (cached and new rows)
   int q_pos0;     // encoder: position of query row 0 within the user's history
   int nkeys;      // keys from key_row0 visible to the item (decoder: cutoff minus the split start)
-  int split;      // decoder: split index of the partial result
+  int key_off;    // encoder with split keys: position of key_row0 within the user's keys
+  int split;      // split index of the partial result
   int h;          // head
 };
 
@@ -143,6 +144,7 @@ __device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const Dec
     w.user_len = 0;
     w.q_pos0 = 0;
     w.split = t.split;
+    w.key_off = 0;
     for (int i = 0; i < NT; ++i) {
       w.nrow[i] = max(0, min(ROWS, t.nrows - i * ROWS));
       w.nblk[i] = w.nrow[i] > 0 ? t.kb1 - t.kb0 : 0;
@@ -158,11 +160,15 @@ __device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const Dec
     w.q_pos0 = off + t.q0;
     w.q_row0 = s + t.q0;
     w.nkeys = 0;
-    w.split = 0;
+    w.split = t.split;
+    // split keys: blocks [kb0, kb1) of the user's keys only
+    const int kb0 = t.kb1 > 0 ? t.kb0 : 0, kb1 = t.kb1 > 0 ? t.kb1 : (1 << 30);
+    w.key_off = kb0 * KB;
+    w.key_row0 += w.key_off;
     for (int i = 0; i < NT; ++i) {
       const int r0 = t.q0 + i * ROWS;
       w.nrow[i] = max(0, min(ROWS, n - r0));
-      w.nblk[i] = w.nrow[i] > 0 ? (min(w.user_len, off + r0 + ROWS) + KB - 1) / KB : 0;
+      w.nblk[i] = w.nrow[i] > 0 ? max(0, min((min(w.user_len, off + r0 + ROWS) + KB - 1) / KB, kb1) - kb0) : 0;
     }
   }
   return w;
@@ -505,7 +511,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tS = tmem + lane_off + s_col(t);
     const uint32_t tO = tmem + lane_off + o_col<HD>(t);
     const uint32_t tP = tmem + lane_off + p_col<HD>(t);
-    const bool split = DEC && da.n_split > 1;
+    const bool split = DEC ? da.n_split > 1 : ea.n_split > 1;
+    float* const part_o = DEC ? da.part_o : ea.part_o;       // split: partial results
+    float* const part_ml = DEC ? da.part_ml : ea.part_ml;
+    const long long part_rows = DEC ? da.nk_rows : ea.rows;
     int cb = 0, qn = 0, cbo = 0;  // cbo: the other tile's key blocks in earlier items
     bool ok = true;
     for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
@@ -516,11 +525,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int h = w.h;
       if (nb == 0) {
         if (split && valid) {  // an empty key range: a partial that carries no weight
-          float* po = da.part_o + ((long long)w.split * da.nk_rows + row_g) * d + h * HD;
+          float* po = part_o + ((long long)w.split * part_rows + row_g) * d + h * HD;
           const float z4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < HD; c += 4) store4(po + c, z4);
-          float* pml = da.part_ml + (((long long)w.split * da.nk_rows + row_g) * n_heads + h) * 2;
+          float* pml = part_ml + (((long long)w.split * part_rows + row_g) * n_heads + h) * 2;
           pml[0] = -INFINITY;
           pml[1] = 0.f;
         }
@@ -556,7 +565,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&q_full[t]);
       }
       // visible keys: index < row_lim - 128 j (the causal bound and the user end / cutoff)
-      const int row_lim = DEC ? w.nkeys : min(w.q_pos0 + t * ROWS + r + 1, w.user_len);
+      const int row_lim = DEC ? w.nkeys : min(w.q_pos0 + t * ROWS + r + 1, w.user_len) - w.key_off;
       float m_ref = -INFINITY;  // reference max (scaled, log2 domain) of P and O
       float l_run = 0.f;        // sum of exponentials relative to m_ref
       for (int j = 0; j < nb; ++j) {
@@ -674,7 +683,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&o_empty[t]);  // O_t may now be overwritten by the next item
-      if (!DEC && ea.out_lo == nullptr) {
+      if (!DEC && !split && ea.out_lo == nullptr) {
         // The output rows through shared memory: each lane writes its row's bf16
         // values into the warp's staging rows, then the warp stores them 16 bytes a
         // lane, HD / 8 lanes to a row, so that a store instruction writes whole
@@ -717,10 +726,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         __syncwarp();  // the staging rows are free for the next item
       } else if (valid && split) {  // partial result of this key range, combined later
-        float* po = da.part_o + ((long long)w.split * da.nk_rows + row_g) * d + h * HD;
+        float* po = part_o + ((long long)w.split * part_rows + row_g) * d + h * HD;
 #pragma unroll
         for (int c = 0; c < HD; c += 4) store4(po + c, &o[c]);
-        float* pml = da.part_ml + (((long long)w.split * da.nk_rows + row_g) * n_heads + h) * 2;
+        float* pml = part_ml + (((long long)w.split * part_rows + row_g) * n_heads + h) * 2;
         pml[0] = m_ref;
         pml[1] = l_run;
       } else if (valid) {
