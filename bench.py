@@ -58,11 +58,11 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (89945344, "attn", "f517c71877da86dc",
+    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (90079744, "attn", "233aab49b12b7c9e",
                                                 "profiles/attn_tc_kernel_bf16-32x1024-d256.md"),
-    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (261767168, "attn", "f517c71877da86dc",
+    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (271378176, "attn", "233aab49b12b7c9e",
                                                     "profiles/attn_tc_kernel_bf16-8x4096-d512.md"),
-    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (287949568, "attn", "f517c71877da86dc",
+    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (296346368, "attn", "233aab49b12b7c9e",
                                                    "profiles/attn_tc_kernel_bf16-2x16384-d512.md"),
 }
 

@@ -33,7 +33,8 @@
 // tiles (S = q_hi H^T + q_lo H^T); when the encoder ran in the same call the
 // decoder also reads H_lo (H = H_hi + H_lo): S adds q_hi H_lo^T, O adds P H_lo.
 //
-// MODE 0: encoder; 1: decoder over H; 2: decoder over H_hi + H_lo.
+// MODE 0: encoder; 1: decoder over H; 2: decoder over H_hi + H_lo; 3: encoder
+// over a range of key blocks (appending with split keys), writing partials.
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -79,7 +80,7 @@ struct SmemLayout {
   static constexpr int STAGES = MODE == 2 ? 2 : 3;
   static constexpr int Q = 0;
   static constexpr int QLO = NT * Cfg<HD>::TILE_BYTES;
-  static constexpr int KV = (MODE >= 1 ? 2 : 1) * NT * Cfg<HD>::TILE_BYTES;
+  static constexpr int KV = (MODE == 1 || MODE == 2 ? 2 : 1) * NT * Cfg<HD>::TILE_BYTES;
   // a stage holds K and V' (encoder), H (decoder), or H_hi and H_lo
   static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
   // encoder: per softmax warp, its 32 output rows in bf16 (rows padded by 16 bytes)
@@ -130,7 +131,7 @@ struct AttnItem {
   int h;          // head
 };
 
-template <bool DEC>
+template <bool DEC, bool SPLITK>
 __device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const DecAttnArgs& da, int item) {
   AttnItem w;
   const int n_heads = DEC ? da.n_heads : ea.n_heads;
@@ -160,15 +161,16 @@ __device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const Dec
     w.q_pos0 = off + t.q0;
     w.q_row0 = s + t.q0;
     w.nkeys = 0;
-    w.split = t.split;
+    w.split = SPLITK ? t.split : 0;
     // split keys: blocks [kb0, kb1) of the user's keys only
-    const int kb0 = t.kb1 > 0 ? t.kb0 : 0, kb1 = t.kb1 > 0 ? t.kb1 : (1 << 30);
+    const int kb0 = SPLITK ? t.kb0 : 0;
     w.key_off = kb0 * KB;
     w.key_row0 += w.key_off;
     for (int i = 0; i < NT; ++i) {
       const int r0 = t.q0 + i * ROWS;
       w.nrow[i] = max(0, min(ROWS, n - r0));
-      w.nblk[i] = w.nrow[i] > 0 ? max(0, min((min(w.user_len, off + r0 + ROWS) + KB - 1) / KB, kb1) - kb0) : 0;
+      const int nb = (min(w.user_len, off + r0 + ROWS) + KB - 1) / KB;
+      w.nblk[i] = w.nrow[i] > 0 ? (SPLITK ? max(0, min(nb, t.kb1) - kb0) : nb) : 0;
     }
   }
   return w;
@@ -183,7 +185,7 @@ template <int HD, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, EncAttnArgs ea, DecAttnArgs da, int32_t* err) {
-  constexpr bool DEC = MODE >= 1, HLO = MODE == 2;
+  constexpr bool DEC = MODE == 1 || MODE == 2, HLO = MODE == 2, ESPLIT = MODE == 3;
   // head_dim 64: one MMA-issuing thread per tile, and the two tiles' softmax warps
   // take turns at the exponentials (see the softmax). head_dim 32: one thread
   // issues both tiles' MMAs in lockstep. At 64 the single issuer was the longest
@@ -255,11 +257,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int k_first = sched[blockIdx.x];
   if (CACHE_ITEMS && warp == 3) {
     const int n = min(sched[blockIdx.x + 1] - k_first, ITEM_CACHE);
-    for (int i = lane; i < n; i += 32) s_items[i] = decode_item<DEC>(ea, da, items[k_first + i]);
+    for (int i = lane; i < n; i += 32) s_items[i] = decode_item<DEC, ESPLIT>(ea, da, items[k_first + i]);
   }
   __syncthreads();
   auto item_at = [&](int k) -> AttnItem {
-    return CACHE_ITEMS && k - k_first < ITEM_CACHE ? s_items[k - k_first] : decode_item<DEC>(ea, da, items[k]);
+    return CACHE_ITEMS && k - k_first < ITEM_CACHE ? s_items[k - k_first] : decode_item<DEC, ESPLIT>(ea, da, items[k]);
   };
 
   if (warp < 4) {
@@ -511,7 +513,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tS = tmem + lane_off + s_col(t);
     const uint32_t tO = tmem + lane_off + o_col<HD>(t);
     const uint32_t tP = tmem + lane_off + p_col<HD>(t);
-    const bool split = DEC ? da.n_split > 1 : ea.n_split > 1;
+    const bool split = DEC ? da.n_split > 1 : ESPLIT;
     float* const part_o = DEC ? da.part_o : ea.part_o;       // split: partial results
     float* const part_ml = DEC ? da.part_ml : ea.part_ml;
     const long long part_rows = DEC ? da.nk_rows : ea.rows;
@@ -565,7 +567,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&q_full[t]);
       }
       // visible keys: index < row_lim - 128 j (the causal bound and the user end / cutoff)
-      const int row_lim = DEC ? w.nkeys : min(w.q_pos0 + t * ROWS + r + 1, w.user_len) - w.key_off;
+      const int row_lim = DEC ? w.nkeys : min(w.q_pos0 + t * ROWS + r + 1, w.user_len) - (ESPLIT ? w.key_off : 0);
       float m_ref = -INFINITY;  // reference max (scaled, log2 domain) of P and O
       float l_run = 0.f;        // sum of exponentials relative to m_ref
       for (int j = 0; j < nb; ++j) {
@@ -791,7 +793,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 template <int HD, int MODE>
 cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream_t s, int32_t* err) {
-  constexpr bool DEC = MODE >= 1;
+  constexpr bool DEC = MODE == 1 || MODE == 2;
   const int swz = HD == 64 ? 128 : 64;
   CUtensorMap mq, mk, mv;
   const int n_tiles = DEC ? da->n_tiles : ea->n_tiles;
@@ -833,6 +835,8 @@ bool sm100_attn_supported(int head_dim) { return head_dim == 32 || head_dim == 6
 int sm100_attn_tile_rows() { return NT * ROWS; }
 
 cudaError_t launch_enc_attn_sm100(int hd, const EncAttnArgs& a, cudaStream_t s, int32_t* err) {
+  if (a.n_split > 1)  // appending with split keys: partial results for launch_enc_combine
+    return hd == 64 ? launch_attn<64, 3>(&a, nullptr, s, err) : launch_attn<32, 3>(&a, nullptr, s, err);
   return hd == 64 ? launch_attn<64, 0>(&a, nullptr, s, err) : launch_attn<32, 0>(&a, nullptr, s, err);
 }
 
