@@ -257,7 +257,7 @@ static std::vector<int> enc_schedule(const rest_batch* b, const std::vector<EncT
   return lpt_schedule(cost);
 }
 
-constexpr int MAX_ENC_SPLIT = 16;
+constexpr int MAX_ENC_SPLIT = 8;  // also bounds the workspace an append query reserves
 // Appending on the tensor-core path: when the items alone would leave SMs idle
 // (a few users' new rows against long cached prefixes), every tile's key blocks
 // are split over n_split items whose partial results a combine kernel merges.
