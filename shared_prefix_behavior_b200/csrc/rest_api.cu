@@ -204,7 +204,7 @@ static long long lpt_makespan(std::vector<long long> cost, int n_cta) {
 // workloads (8 x 4096 and 2 x 16384 keys); a split count wins only when it is at
 // least 5% shorter than every smaller one, since each split also writes a
 // partial output that the combine reads back.
-constexpr long long DEC_ITEM_COST = 7;
+constexpr long long ITEM_COST_BLOCKS = 7;
 static int choose_dec_split(const rest_batch* b, const rest_requests* r, int K, int rows, int n_heads) {
   std::vector<DecTile> t;
   build_dec_tiles(b, r, K, rows, 1, t);
@@ -220,7 +220,7 @@ static int choose_dec_split(const rest_batch* b, const rest_requests* r, int K, 
     build_dec_tiles(b, r, K, rows, ns, t);
     std::vector<long long> cost;
     for (const DecTile& x : t) {
-      const long long c = (long long)(x.kb1 - x.kb0) * ((x.nrows + 127) / 128) + DEC_ITEM_COST;
+      const long long c = (long long)(x.kb1 - x.kb0) * ((x.nrows + 127) / 128) + ITEM_COST_BLOCKS;
       for (int h = 0; h < n_heads; ++h) cost.push_back(c);
     }
     const long long m = lpt_makespan(cost, SCHED_CTAS);
@@ -285,7 +285,7 @@ static void split_enc_tiles(const rest_batch* b, const std::vector<UserAppend>& 
   auto makespan = [&](const std::vector<EncTile>& ts) {
     std::vector<long long> cost;
     for (const EncTile& t : ts) {
-      const long long c = enc_item_cost(b, app, t, rows) + DEC_ITEM_COST;
+      const long long c = enc_item_cost(b, app, t, rows) + ITEM_COST_BLOCKS;
       for (int h = 0; h < n_heads; ++h) cost.push_back(c);
     }
     return lpt_makespan(cost, SCHED_CTAS);
