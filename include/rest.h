@@ -180,6 +180,10 @@ rest_status rest_cross_decode(rest_dtype dt, const rest_heads* heads, const rest
 /* Size in bytes of the scratch array that rest_cross_decode_static_ws uses. */
 #define REST_STATIC_WS_BYTES (32u * 1024u * 1024u)
 
+/* REST_STATIC_WS_BYTES as the library was built with it (for bindings that
+ * cannot read this header). */
+size_t rest_static_ws_bytes(void);
+
 /* rest_cross_decode without a workspace argument. The paper has no
  * counterpart to this entry point; it exists for callers that cannot
  * allocate device memory themselves. Examples: a plain-C host program
@@ -189,17 +193,22 @@ rest_status rest_cross_decode(rest_dtype dt, const rest_heads* heads, const rest
  *
  * The decoder's scratch (index/tile lists and the per-row q, g and o
  * buffers) lives in one REST_STATIC_WS_BYTES array in the library's device
- * image instead. Every GPU that loads the library holds this array until the
- * process exits. The caller still passes inputs and outputs exactly as for
+ * image instead. The caller still passes inputs and outputs exactly as for
  * rest_cross_decode, with the same meaning, and the same results.
+ *   - The CUDA runtime loads the library's device image, and with it the
+ *     array, on a device's first call of this entry point (lazy module
+ *     loading). From then on that GPU holds the array until the process
+ *     exits. A call with no candidates (n_req = 0, or no candidates in any
+ *     request) loads it too and does nothing else: make one such call per
+ *     device, with that device current, before handing device memory to an
+ *     arena and before any CUDA stream capture.
+ *   - Every call looks up the array's address in the current device's
+ *     context, so `stream` must belong to the current device.
  *   - A batch whose scratch would exceed the array returns
  *     REST_ERR_WORKSPACE; rest_workspace_size() with n_layers = 0 tells the
  *     bytes a batch needs.
  *   - This entry point calls no cudaMalloc, cudaFree or other allocating
  *     routine.
- *   - The first call on a device looks up the array's device address
- *     (once per device, with that device current). Make that first call
- *     before any CUDA stream capture.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Nothing in it needs to start at zero. Calls whose work overlaps on the
  *     GPU (different streams, or different host threads without ordering)

@@ -34,8 +34,7 @@ EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "r
            "rest_rank_request", "rest_status_string", "rest_launch_count", "rest_profile_begin",
            "rest_profile_end", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",
            "rest_append_workspace_size", "rest_encoder_append", "rest_attn_workspace_size", "rest_attn_forward",
-           "rest_attn_backward", "rest_selftest_wait_timeout")
-STATIC_WS_BYTES = 32 * 1024 * 1024  # REST_STATIC_WS_BYTES
+           "rest_attn_backward", "rest_selftest_wait_timeout", "rest_static_ws_bytes")
 
 
 class RestError(RuntimeError):
@@ -126,10 +125,14 @@ def _load() -> ctypes.CDLL:
     lib.rest_profile_begin.restype = None
     lib.rest_profile_end.argtypes = [POINTER(KernelStat), c_int]
     lib.rest_profile_end.restype = c_int
+    lib.rest_static_ws_bytes.argtypes = []
+    lib.rest_static_ws_bytes.restype = c_size_t
     return lib
 
 
 _lib = _load()
+# the scratch array of rest_cross_decode_static_ws, as the library was built
+STATIC_WS_BYTES = int(_lib.rest_static_ws_bytes())
 
 
 def library() -> ctypes.CDLL:
@@ -302,15 +305,16 @@ def cross_decode(hmem, cu_seqlens, taus, reqs, z, dec: dict, rope_base: float = 
 
 
 def cross_decode_static_ws(hmem, cu_seqlens, taus, reqs, z, dec: dict, rope_base: float = 10000.0, y_out=None,
-                           stream=None, check=True):
+                           stream=None, check=True, err=None):
     """``cross_decode`` for callers that cannot allocate device memory.
 
     The decoder's scratch lives in the library's own fixed device array of
     STATIC_WS_BYTES bytes instead of a caller workspace; batches that need
     more raise RestError(REST_ERR_WORKSPACE). Calls share that array, so
-    calls that overlap on the GPU race; order them on one stream. (This
-    wrapper itself allocates y_out and the status word with torch when they
-    are not given; a caller that cannot allocate passes its own.)
+    calls that overlap on the GPU race; order them on one stream. A device's
+    first call loads the array (one with no candidates does only that).
+    (This wrapper itself allocates y_out and the status word with torch when
+    they are not given; a caller that cannot allocate passes its own.)
     """
     import torch
     dev, d = hmem.device, hmem.shape[1]
@@ -319,7 +323,8 @@ def cross_decode_static_ws(hmem, cu_seqlens, taus, reqs, z, dec: dict, rope_base
     dp = _dec(dec)
     if y_out is None:
         y_out = torch.empty(z.shape, dtype=torch.float32, device=dev)
-    err = _err_word(dev, stream)
+    if err is None:
+        err = _err_word(dev, stream)
     _check(_lib.rest_cross_decode_static_ws(dt, ctypes.byref(h.heads), ctypes.byref(h.batch), _ptr(hmem),
                                             ctypes.byref(h.reqs), _ptr(z), ctypes.byref(dp), _ptr(y_out), _ptr(err),
                                             _stream(stream)), "rest_cross_decode_static_ws")

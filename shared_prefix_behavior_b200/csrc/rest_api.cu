@@ -6,7 +6,6 @@
 #include <string.h>
 
 #include <algorithm>
-#include <mutex>
 #include <new>
 #include <queue>
 #include <vector>
@@ -1365,32 +1364,25 @@ namespace rest {
 
 static __device__ __align__(256) unsigned char g_static_ws[REST_STATIC_WS_BYTES];
 
-static std::mutex g_static_ws_mu;
-static void* g_static_ws_ptr[64];
-
-// Device address of g_static_ws on the current device, looked up once per
-// device (host code may not use the symbol itself as an address).
+// Device address of g_static_ws in the current device's context. Host code may
+// not use the symbol itself as an address. The lookup runs on every call: once
+// the library's device image is loaded it costs little, and it also loads that
+// image (with the array) on a device's first call, since the CUDA runtime loads
+// modules lazily. An address cached across calls would go stale if the context
+// were destroyed and re-created (cudaDeviceReset loads the image again).
 static rest_status static_ws_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) {
     cudaGetLastError();
-    return REST_ERR_NO_DEVICE;
+    return REST_ERR_CUDA;
   }
-  if (dev < 0 || dev >= 64) return REST_ERR_NO_DEVICE;
-  std::lock_guard<std::mutex> lock(g_static_ws_mu);
-  if (!g_static_ws_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return REST_ERR_CUDA;
-    }
-    g_static_ws_ptr[dev] = p;
-  }
-  *out = g_static_ws_ptr[dev];
+  *out = p;
   return REST_OK;
 }
 
 }  // namespace rest
+
+extern "C" size_t rest_static_ws_bytes(void) { return (size_t)REST_STATIC_WS_BYTES; }
 
 extern "C" rest_status rest_cross_decode_static_ws(rest_dtype dt, const rest_heads* heads, const rest_batch* batch,
                                                    const void* h, const rest_requests* reqs, const void* z,
@@ -1405,10 +1397,12 @@ extern "C" rest_status rest_cross_decode_static_ws(rest_dtype dt, const rest_hea
     if (p.NK > 0 && (!h || !z || !y_out || !aligned16(h) || !aligned16(z) || !aligned16(y_out)))
       return REST_ERR_INVALID_ARG;
     if (p.L.total > (size_t)REST_STATIC_WS_BYTES) return REST_ERR_WORKSPACE;  // batch too large for the array
-    if (p.NK == 0) return REST_OK;
     if ((st = check_device()) != REST_OK) return st;
+    // Before the empty-batch return, so that a call with no candidates loads the
+    // array on this device: the warm-up call that reserves it up front.
     void* ws = nullptr;
     if ((st = static_ws_address(&ws)) != REST_OK) return st;
+    if (p.NK == 0) return REST_OK;
     cudaStream_t s = (cudaStream_t)stream;
     p.err = dev_err;
     // Nothing in the scratch needs to start at zero: the index/tile lists are

@@ -29,6 +29,13 @@ def test_library_exports_every_declared_symbol():
     assert set(R.EXPORTS) <= set(names)
 
 
+def test_static_ws_size_matches_the_header():
+    src = open(os.path.join(ROOT, "include", "rest.h")).read()
+    m = re.search(r"#define REST_STATIC_WS_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", src)
+    assert m, "REST_STATIC_WS_BYTES not found in rest.h"
+    assert R.STATIC_WS_BYTES == int(m.group(1)) * int(m.group(2)) * int(m.group(3))
+
+
 def test_status_strings():
     for code in range(8):
         assert R.library().rest_status_string(code)

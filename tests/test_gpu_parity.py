@@ -239,6 +239,48 @@ def test_full_workload_single_layer_sampled_rows(cuda, cfg):
     assert_parity(H[rows], O.encoder_rows(inp, rows), "bf16", "H rows")
 
 
+def _end_to_end_users(w, cfg):
+    """Users whose whole forward the oracle runs: on the 16k workload one of
+    its two users; on the ragged one the shortest user, the first user whose
+    every request is under 1024 keys (the decoder reads H_hi + H_lo there),
+    the first user with requests on both sides of 1024 keys, and the first
+    user of 4096-6144 tokens (H_hi alone)."""
+    if cfg == 3:
+        return [0]
+    L = np.asarray(w.lengths)
+    ru, rc = np.asarray(w.req_user), np.asarray(w.req_cutoff)
+    short = [u for u in range(w.n_users) if (rc[ru == u] < 1024).all()]
+    mixed = [u for u in range(w.n_users) if (rc[ru == u] < 1024).any() and (rc[ru == u] >= 1024).any()]
+    long_ = [u for u in range(w.n_users) if 4096 <= L[u] <= 6144]
+    return sorted({int(np.argmin(L)), short[0], mixed[0], long_[0]})
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_full_workload_single_layer_end_to_end(cuda, cfg):
+    """The one-layer workloads at full size through rank_request, y included:
+    the GPU runs the whole batch; the oracle encodes the sampled users in full
+    and scores every candidate of their requests. This checks the product's
+    decoder on real encoder output, where requests under 1024 keys read H as
+    H_hi + H_lo and longer ones H_hi alone (each request is also held to the
+    bar on its own). The passage: scoring with a request's prefix of the
+    union history equals scoring that prefix alone (§3.5)."""
+    w = W.workload(cfg)
+    inp = W.make_inputs(w, 1000 + cfg)
+    H, y = run_rank(inp, cuda)
+    users = _end_to_end_users(w, cfg)
+    sub = subset_users(inp, users)
+    Hr, yr = O.rank_request(sub)
+    assert_parity(H[sub["_rows"]], Hr, "bf16", "H")
+    yg = y[sub["_cand_rows"]]
+    assert_parity(yg, yr, "bf16", "y")
+    cc = sub["cu_cands"]
+    for r in range(len(sub["req_user"])):
+        if cc[r + 1] > cc[r]:
+            assert_parity(yg[cc[r]:cc[r + 1]], yr[cc[r]:cc[r + 1]], "bf16",
+                          f"request {r} (cutoff {int(sub['req_cutoff'][r])})")
+
+
 @pytest.mark.parametrize("cfg,n_req", [(3, 2), (4, 6)])
 def test_full_workload_decoder_sampled_requests(cuda, cfg, n_req):
     """The decoder over the full workload's requests with a synthetic memory;
