@@ -9,20 +9,24 @@
 //                128-key block. Decoder: H (and H_lo) per block; one H tile
 //                is both the keys (K-major operand of S = q H^T) and the
 //                values (N-major operand of O = P H).
-//   warp 1       TMEM owner and MMA issuer. Per block j and tile t: S_t(j) =
-//                Q_t K_j^T into the tile's 128-column TMEM buffer (as soon as
-//                the softmax has read S_t(j-1)), then O_t += P_t(j-1) V_{j-1}
-//                into the tile's head_dim-column accumulator. head_dim 32: one
-//                thread issues for both tiles in lockstep; head_dim 64: warp 1
-//                issues for tile 0 and warp 2 for tile 1.
-//   warp 3       head_dim 32: decodes the CTA's work items into a shared-memory
-//                table at the start (a lane per item).
+//   warp 1       TMEM owner and S issuer: S_t(j) = Q_t K_j^T for both tiles into
+//                each tile's 128-column TMEM buffer, as soon as the tile's
+//                softmax has read S_t(j-1).
+//   warps 2, 3   P V issuers of tiles 0 and 1: O_t += P_t(j) V_j into the
+//                tile's head_dim-column accumulator once P_t(j) is written. A
+//                warp issues one tcgen05.mma about every hundred cycles whatever
+//                its size (measured), so the products are spread over three
+//                issuing warps, each running whole with one elected lane.
+//   warp 3       head_dim 32: first decodes the CTA's work items into a
+//                shared-memory table (a lane per item).
 //   warps 4..7   softmax of tile 0, warps 8..11 of tile 1: a thread owns a
 //                query row; it reads its row of S from TMEM, masks, keeps the
 //                running max, exponentiates in base 2, and writes P (bf16
 //                pairs) back to the tile's P columns of TMEM, from where the
-//                P V MMA takes its A operand. O stays in TMEM: when a row's max grows by more than
-//                2^8 the thread rescales its O row in TMEM (after the previous
+//                P V MMA takes its A operand; the exponentials are computed
+//                before the wait for the previous P V, which only their store
+//                needs. O stays in TMEM: when a row's max grows by more than
+//                2^8 the warp rescales its O rows in TMEM (after the previous
 //                P V has completed); otherwise P is taken relative to the old
 //                max (values up to 2^8, exact in fp32 accumulation). At
 //                head_dim 64 the two tiles' warps of a lane quarter, which
@@ -186,12 +190,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, EncAttnArgs ea, DecAttnArgs da, int32_t* err) {
   constexpr bool DEC = MODE == 1 || MODE == 2, HLO = MODE == 2, ESPLIT = MODE == 3;
-  // head_dim 64: one MMA-issuing thread per tile, and the two tiles' softmax warps
-  // take turns at the exponentials (see the softmax). head_dim 32: one thread
-  // issues both tiles' MMAs in lockstep. At 64 the single issuer was the longest
-  // chain of a block (a tcgen05.mma costs its thread about a hundred cycles, 24 of
-  // them per block pair); at 32, with fewer MMAs per block and short items, the
-  // per-tile issuers measured slower.
+  // head_dim 64: the two tiles' softmax warps of a lane quarter take turns at the
+  // exponentials block by block (see the softmax); at 32 they do not.
   constexpr bool TURNS = HD >= 64;
   using C = Cfg<HD>;
   using L = SmemLayout<HD, MODE>;
@@ -229,9 +229,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], TURNS ? NT : 1);  // one arrival per MMA issuer
+      mbar_init(&kv_empty[s], 1 + NT);  // one arrival per MMA-issuing warp
     }
-    mbar_init(&drain, TURNS ? NT : 1);
+    mbar_init(&drain, 1 + NT);
     for (int t = 0; t < NT; ++t)
       for (int q = 0; q < 4; ++q) {
         mbar_init(&xe[t][q][0], 1);
@@ -266,6 +266,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp < 4) {
     setmaxnreg_dec72();
+    // Warp 0, lane 0 loads (the other lanes of warp 0 have no role and wait at
+    // the end); warp 1 issues S; warps 2 and 3 issue P V. The issuing warps run
+    // whole: their elect.sync needs every lane.
     if (warp == 0 && lane == 0) {
       // -------------------------------------------------------- TMA producer
       int g = 0, issued = 0, qn[NT] = {0, 0};
@@ -300,207 +303,122 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
           mbar_wait(&kv_full[i % STAGES], (i / STAGES) & 1, nullptr, &no_abort);
       }
-    } else if (TURNS ? ((warp == 1 || warp == 2) && lane == 0) : (warp == 1 && lane == 0)) {
-      if constexpr (TURNS) {
-        // -------------------------------------------------------- MMA issuers
-        // One thread per query tile (warp 1: tile 0, warp 2: tile 1) issues that
-        // tile's S = Q K^T and O += P V. A tcgen05.mma costs its issuing thread about
-        // a hundred cycles whatever its size, so a single issuer for both tiles was
-        // the longest chain of the block. The K/V stage of a block is released when
-        // both issuers have committed it (kv_empty counts two arrivals); a tile with
-        // fewer blocks in the item still waits for each remaining block to land
-        // before releasing it, so neither issuer can arrive for a later use of a
-        // stage before the earlier use has completed.
-        const int t = warp - 1;
-        constexpr uint32_t idS = idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
-        constexpr uint32_t idO = idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
-        // S(j) as soon as the softmax has loaded S(j-1) into registers (s_free), so
-        // the next scores are computed while it exponentiates, then P(j-1) V.
-        const uint32_t tS = tmem + s_col(t), tO = tmem + o_col<HD>(t), tP = tmem + p_col<HD>(t);
-        const uint64_t qd = smem_desc(smem_u32(smem + L::Q + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
-        const uint64_t qld = smem_desc(smem_u32(smem + L::QLO + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
-        int g = 0, cb = 0, qn = 0;
-        bool ok = true;
-        for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-          const AttnItem w = item_at(k);
-          const int nblk_all = max(w.nblk[0], w.nblk[1]);
-          const int nb = w.nblk[t];
-          if (nb > 0) ok = mbar_wait(&q_full[t], qn & 1, err, &abort_flag);
-          tc_fence_after();
-          // Descriptors are built once per operand tile and stepped along K: a K step of
-          // 16 elements is 32 bytes, 2 in the descriptor's 16-byte address field.
-          for (int j = 0; ok && j <= nb; ++j) {
-            const int st = (g + j) % STAGES;
-            if (j < nb) {
-              if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
-              tc_fence_after();
-            }
-            if (j >= 1) {  // the S buffer is free again
-              if (!mbar_wait(&s_free[t], (cb + j - 1) & 1, err, &abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            if (j < nb) {  // S(j) = Q K_j^T, overwriting the tile's S buffer
-              const uint64_t kd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE), 16, C::ATOM, C::SWZ);
-  #pragma unroll
-              for (int kk = 0; kk < HD / 16; ++kk) mma_bf16_nc(tS, qd + 2 * kk, kd + 2 * kk, idS, kk != 0);
-              if (DEC) {  // + q_lo . H^T
-  #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) mma_bf16_nc(tS, qld + 2 * kk, kd + 2 * kk, idS, 1);
-              }
-              if (HLO) {  // + q_hi . H_lo^T
-  #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                  mma_bf16_nc(tS, qd + 2 * kk, kd + (C::TILE_BYTES >> 4) + 2 * kk, idS, 1);
-              }
-              if (j == nb - 1) mma_commit(&q_empty[t]);  // the item's last read of Q_t
-              mma_commit(&s_full[t]);
-            }
-            if (j >= 1) {  // O += P(j-1) V_{j-1}
-              const int i = j - 1, sti = (g + i) % STAGES;
-              if (!mbar_wait(&p_full[t], (cb + i) & 1, err, &abort_flag)) { ok = false; break; }
-              tc_fence_after();
-              if (i == 0 && qn >= 1) {  // the previous item's O_t has been read out
-                if (!mbar_wait(&o_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
-                tc_fence_after();
-              }
-              const uint64_t vd = smem_desc(smem_u32(smem + L::KV + sti * L::STAGE + (DEC ? 0 : C::TILE_BYTES)),
-                                            64 * KB * 2, C::ATOM, C::SWZ);
-              constexpr uint32_t V_STEP = (2 * C::ATOM) >> 4;  // 16 keys of V: two 8-row atoms
-              // A = P_t from TMEM, 8 columns per K step of 16
-  #pragma unroll
-              for (int kk = 0; kk < KB / 16; ++kk)
-                mma_bf16_ts_nc(tO, tP + kk * 8, vd + V_STEP * kk, idO, (i | kk) != 0);
-              if (HLO) {  // + P H_lo
-  #pragma unroll
-                for (int kk = 0; kk < KB / 16; ++kk)
-                  mma_bf16_ts_nc(tO, tP + kk * 8, vd + (C::TILE_BYTES >> 4) + V_STEP * kk, idO, 1);
-              }
-              mma_commit(&p_free[t]);
-              mma_commit(&kv_empty[sti]);  // this tile is done with block j-1
-            }
-          }
-          // the item's blocks this tile has no rows for: released once each has landed
-          for (int j = nb; ok && j < nblk_all; ++j) {
-            const int st = (g + j) % STAGES;
-            if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
-            mbar_arrive(&kv_empty[st]);
-          }
-          g += nblk_all;
-          if (nb > 0) {
-            cb += nb;
-            ++qn;
-          }
-        }
-        mma_commit(&drain);
-        volatile int no_abort = 0;
-        mbar_wait(&drain, 0, nullptr, &no_abort);
-      } else {
-        // -------------------------------------------------------- MMA issuer
-        constexpr uint32_t idS = idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
-        constexpr uint32_t idO = idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
-        int g = 0, cb[NT] = {0, 0}, qn[NT] = {0, 0};
-        bool ok = true;
-        for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-          const AttnItem w = item_at(k);
-          const int nblk_all = max(w.nblk[0], w.nblk[1]);
-          for (int t = 0; t < NT && ok; ++t)
-            if (w.nblk[t] > 0) ok = mbar_wait(&q_full[t], qn[t] & 1, err, &abort_flag);
-          tc_fence_after();
-          for (int j = 0; ok && j <= nblk_all; ++j) {
-            const int st = (g + j) % STAGES;
-            if (j < nblk_all) {
-              if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
-              tc_fence_after();
-            }
-            // S_t(j) = Q_t K_j^T, overwriting the tile's S buffer
-            auto issue_s = [&](int t) {
-              const uint32_t k_base = smem_u32(smem + L::KV + st * L::STAGE);
-              const uint32_t q_base = smem_u32(smem + L::Q + t * C::TILE_BYTES);
-              const uint32_t tS = tmem + s_col(t);
-  #pragma unroll
-              for (int k = 0; k < HD / 16; ++k)
-                mma_bf16(tS, smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ),
-                         smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, k != 0);
-              if (DEC) {  // + q_lo . H^T
-                const uint32_t qlo_base = smem_u32(smem + L::QLO + t * C::TILE_BYTES);
-  #pragma unroll
-                for (int k = 0; k < HD / 16; ++k)
-                  mma_bf16(tS, smem_desc(qlo_base + k * 32, 16, C::ATOM, C::SWZ),
-                           smem_desc(k_base + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
-              }
-              if (HLO) {  // + q_hi . H_lo^T
-  #pragma unroll
-                for (int k = 0; k < HD / 16; ++k)
-                  mma_bf16(tS, smem_desc(q_base + k * 32, 16, C::ATOM, C::SWZ),
-                           smem_desc(k_base + C::TILE_BYTES + k * 32, 16, C::ATOM, C::SWZ), idS, 1);
-              }
-              if (j == w.nblk[t] - 1) mma_commit(&q_empty[t]);  // the item's last read of Q_t
-              mma_commit(&s_full[t]);
-            };
-            // O_t += P_t(j-1) V_{j-1}; P_t(j-1) is written
-            auto issue_pv = [&](int t) -> bool {
-              const int i = j - 1, sti = (g + i) % STAGES;
-              if (i == 0 && qn[t] >= 1 &&  // the previous item's O_t has been read out
-                  !mbar_wait(&o_empty[t], (qn[t] - 1) & 1, err, &abort_flag))
-                return false;
-              tc_fence_after();
-              const uint32_t tP = tmem + p_col<HD>(t);  // A = P_t from TMEM, 8 columns per K step of 16
-              const uint32_t v_base = smem_u32(smem + L::KV + sti * L::STAGE + (DEC ? 0 : C::TILE_BYTES));
-              const uint32_t tO = tmem + o_col<HD>(t);
-  #pragma unroll
-              for (int k = 0; k < KB / 16; ++k)
-                mma_bf16_ts(tO, tP + k * 8, smem_desc(v_base + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO,
-                            (i | k) != 0);
-              if (HLO) {  // + P H_lo
-  #pragma unroll
-                for (int k = 0; k < KB / 16; ++k)
-                  mma_bf16_ts(tO, tP + k * 8,
-                              smem_desc(v_base + C::TILE_BYTES + k * 2 * C::ATOM, 64 * KB * 2, C::ATOM, C::SWZ), idO,
-                              1);
-              }
-              mma_commit(&p_free[t]);
-              return true;
-            };
-            // Both tiles' S(j) as soon as each softmax has loaded S(j-1) into registers
-            // (s_free), so the next scores are computed while it exponentiates, then the
-            // P V products (-3% attention time on 1k-token histories against issuing S(j)
-            // once P(j-1) is written).
-            constexpr bool EARLY_S = true;
-            for (int t = 0; t < NT; ++t) {
-              const bool prev = j >= 1 && j - 1 < w.nblk[t];
-              if (prev) {
-                if (!mbar_wait(EARLY_S ? &s_free[t] : &p_full[t], (cb[t] + j - 1) & 1, err, &abort_flag)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-              }
-              if (j < w.nblk[t]) issue_s(t);
-              if (!EARLY_S && prev && !issue_pv(t)) { ok = false; break; }
-            }
-            if (EARLY_S)
-              for (int t = 0; t < NT && ok; ++t) {
-                if (!(j >= 1 && j - 1 < w.nblk[t])) continue;
-                if (!mbar_wait(&p_full[t], (cb[t] + j - 1) & 1, err, &abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                if (!issue_pv(t)) { ok = false; break; }
-              }
-            if (j >= 1 && ok) mma_commit(&kv_empty[(g + j - 1) % STAGES]);  // block j-1 fully consumed
-          }
-          g += nblk_all;
-          for (int t = 0; t < NT; ++t)
-            if (w.nblk[t] > 0) {
-              cb[t] += w.nblk[t];
-              ++qn[t];
-            }
-        }
-        mma_commit(&drain);
-        volatile int no_abort = 0;
-        mbar_wait(&drain, 0, nullptr, &no_abort);
+    } else if (warp == 1) {
+      // -------------------------------------------------------- S issuer
+      // S_t(j) = Q_t K_j^T for both tiles, each into its tile's S buffer as soon
+      // as the tile's softmax has loaded the previous S into registers (s_free),
+      // so the next scores are ready while it exponentiates. The whole warp runs
+      // the loop and one elected lane issues: a warp issues one tcgen05.mma about
+      // every hundred cycles whatever its size, so the S and the P V products of
+      // the two tiles are spread over three issuing warps.
+      constexpr uint32_t idS = idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
+      uint64_t qd[NT], qld[NT];
+      for (int t = 0; t < NT; ++t) {
+        qd[t] = smem_desc(smem_u32(smem + L::Q + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
+        qld[t] = smem_desc(smem_u32(smem + L::QLO + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
       }
+      int g = 0, ns[NT] = {0, 0}, qn[NT] = {0, 0};  // ns: S blocks issued per tile in earlier items
+      bool ok = true;
+      for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
+        const AttnItem w = item_at(k);
+        const int nblk_all = max(w.nblk[0], w.nblk[1]);
+        for (int t = 0; t < NT && ok; ++t)
+          if (w.nblk[t] > 0) ok = mbar_wait(&q_full[t], qn[t] & 1, err, &abort_flag);
+        tc_fence_after();
+        for (int j = 0; ok && j < nblk_all; ++j) {
+          const int st = (g + j) % STAGES;
+          if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          // Descriptors step along K: 16 elements are 32 bytes, 2 in the 16-byte address field.
+          const uint64_t kd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE), 16, C::ATOM, C::SWZ);
+          for (int t = 0; t < NT; ++t) {
+            if (j >= w.nblk[t]) continue;
+            const int n = ns[t] + j;  // the tile's S block number
+            if (n >= 1) {             // S_t(n - 1) has been read: the buffer is free
+              if (!mbar_wait(&s_free[t], (n - 1) & 1, err, &abort_flag)) { ok = false; break; }
+              tc_fence_after();
+            }
+            const uint32_t tS = tmem + s_col(t);
+  #pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk) mma_bf16_e(tS, qd[t] + 2 * kk, kd + 2 * kk, idS, kk != 0);
+            if (DEC) {  // + q_lo . H^T
+  #pragma unroll
+              for (int kk = 0; kk < HD / 16; ++kk) mma_bf16_e(tS, qld[t] + 2 * kk, kd + 2 * kk, idS, 1);
+            }
+            if (HLO) {  // + q_hi . H_lo^T
+  #pragma unroll
+              for (int kk = 0; kk < HD / 16; ++kk)
+                mma_bf16_e(tS, qd[t] + 2 * kk, kd + (C::TILE_BYTES >> 4) + 2 * kk, idS, 1);
+            }
+            if (j == w.nblk[t] - 1) mma_commit_e(&q_empty[t]);  // the item's last read of Q_t
+            mma_commit_e(&s_full[t]);
+          }
+          if (ok) mma_commit_e(&kv_empty[st]);  // this block's keys have been read
+        }
+        g += nblk_all;
+        for (int t = 0; t < NT; ++t)
+          if (w.nblk[t] > 0) {
+            ns[t] += w.nblk[t];
+            ++qn[t];
+          }
+      }
+      mma_commit_e(&drain);
+      volatile int no_abort = 0;
+      mbar_wait(&drain, 0, nullptr, &no_abort);
+    } else if (warp >= 2) {
+      // -------------------------------------------------------- P V issuers
+      // Warp 2 for tile 0, warp 3 for tile 1: O_t += P_t(j) V_j once the softmax
+      // has written P_t(j) into TMEM (p_full). A block's K/V stage is released when
+      // the S issuer and both P V issuers have committed it (kv_empty counts three
+      // arrivals); a tile with fewer blocks in the item still waits for each
+      // remaining block to land before releasing it, so no issuer can arrive for a
+      // later use of a stage before the earlier use has completed.
+      const int t = warp - 2;
+      constexpr uint32_t idO = idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
+      constexpr uint32_t V_STEP = (2 * C::ATOM) >> 4;  // 16 keys of V: two 8-row atoms
+      const uint32_t tO = tmem + o_col<HD>(t), tP = tmem + p_col<HD>(t);
+      int g = 0, cb = 0, qn = 0;
+      bool ok = true;
+      for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
+        const AttnItem w = item_at(k);
+        const int nblk_all = max(w.nblk[0], w.nblk[1]);
+        const int nb = w.nblk[t];
+        for (int j = 0; ok && j < nblk_all; ++j) {
+          const int st = (g + j) % STAGES;
+          if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+          if (j >= nb) {  // a block this tile has no rows for
+            if (lane == 0) mbar_arrive(&kv_empty[st]);
+            continue;
+          }
+          if (!mbar_wait(&p_full[t], (cb + j) & 1, err, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          if (j == 0 && qn >= 1) {  // the previous item's O_t has been read out
+            if (!mbar_wait(&o_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const uint64_t vd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE + (DEC ? 0 : C::TILE_BYTES)),
+                                        64 * KB * 2, C::ATOM, C::SWZ);
+          // A = P_t from TMEM, 8 columns per K step of 16
+  #pragma unroll
+          for (int kk = 0; kk < KB / 16; ++kk)
+            mma_bf16_ts_e(tO, tP + kk * 8, vd + V_STEP * kk, idO, (j | kk) != 0);
+          if (HLO) {  // + P H_lo
+  #pragma unroll
+            for (int kk = 0; kk < KB / 16; ++kk)
+              mma_bf16_ts_e(tO, tP + kk * 8, vd + (C::TILE_BYTES >> 4) + V_STEP * kk, idO, 1);
+          }
+          mma_commit_e(&p_free[t]);
+          mma_commit_e(&kv_empty[st]);  // this tile is done with block j
+        }
+        g += nblk_all;
+        if (nb > 0) {
+          cb += nb;
+          ++qn;
+        }
+      }
+      mma_commit_e(&drain);
+      volatile int no_abort = 0;
+      mbar_wait(&drain, 0, nullptr, &no_abort);
     }
   } else {
     setmaxnreg_inc216();
@@ -603,15 +521,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
         const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-        // P_t replaces the previous block's: wait until its O += P V has completed
-        if (gj >= 1) {
-          if (!mbar_wait(&p_free[t], (gj - 1) & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-        }
+        // P_t replaces the previous block's P once that block's O += P V has
+        // completed (p_free). The wait comes after the exponentials, which need
+        // only the reference max, unless the O row must be rescaled first.
+        bool pv_done = gj == 0;
         if (j == 0) {
           m_ref = m_blk;
-        } else if (m_blk > m_ref + RESCALE_LOG2) {  // rescale the O row and l to the new max
-          const float f = exp2_approx(m_ref - m_blk);
+        } else if (__any_sync(0xffffffffu, m_blk > m_ref + RESCALE_LOG2)) {
+          // Some row's max grew by more than 2^8: the warp rescales its O rows and
+          // sums to their new maxima (a factor of 1 for the rows whose max did not
+          // grow). Warp-wide, since the TMEM loads and stores are warp-collective.
+          if (!mbar_wait(&p_free[t], (gj - 1) & 1, err, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          pv_done = true;
+          const float m_new = fmaxf(m_ref, m_blk);
+          const float f = exp2_approx(m_ref - m_new);
 #pragma unroll
           for (int c0 = 0; c0 < HD; c0 += 32) {
             float o[32];
@@ -621,7 +545,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_st32(tO + c0, o);
           }
           l_run *= f;
-          m_ref = m_blk;
+          m_ref = m_new;
         }
         // The two tiles' warps of a lane quarter share an SM sub-partition and its
         // special-function unit: they take turns at the exponentials, block by block
@@ -636,25 +560,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m_ref, -m_ref);
-        // P as bf16 pairs (keys 2c, 2c+1 in column c) into the tile's P columns of TMEM
+        // P as bf16 pairs (keys 2c, 2c+1 in column c), stored into the tile's P
+        // columns of TMEM once the previous P V has completed
+        uint32_t pk[64];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int e = 64 * half + 2 * c;
-            const float2 x = ffma2(make_float2(s[e], s[e + 1]), scale2, neg_m2);
-            const float p0 = exp2_approx(x.x), p1 = exp2_approx(x.y);
-            sum2[c & 1] = fadd2(sum2[c & 1], make_float2(p0, p1));
-            __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
-            pk[c] = *reinterpret_cast<uint32_t*>(&t2);
-          }
-          tmem_st32_async(tP + 32 * half, pk);
+        for (int c = 0; c < 64; ++c) {
+          const int e = 2 * c;
+          const float2 x = ffma2(make_float2(s[e], s[e + 1]), scale2, neg_m2);
+          const float p0 = exp2_approx(x.x), p1 = exp2_approx(x.y);
+          sum2[c & 1] = fadd2(sum2[c & 1], make_float2(p0, p1));
+          __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
+          pk[c] = *reinterpret_cast<uint32_t*>(&t2);
         }
         if (TURNS) {
           __syncwarp();
           if (lane == 0) mbar_arrive(&xe[t][q4][(cb + j) & 1]);
         }
+        if (!pv_done) {
+          if (!mbar_wait(&p_free[t], (gj - 1) & 1, err, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+        }
+        tmem_st32_async(tP, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+        tmem_st32_async(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
         l_run += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
         tmem_wait_st();
         tc_fence_before();

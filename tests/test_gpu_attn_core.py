@@ -53,6 +53,23 @@ def test_attention_core_small_ragged(cuda, dtype, hd):
         assert_parity(got, ref, dtype, name)
 
 
+@pytest.mark.parametrize("hd", [32, 64])
+def test_attention_core_row_max_growth(cuda, hd):
+    """Keys that grow with their position (x (1 + position // 128)): every
+    causal row's running max rises block by block past the kernel's 2^8
+    threshold, so the forward rescales the accumulated output in TMEM."""
+    (q, k, v, _), cu, H = core_case("bf16", hd, (700, 300), 74)
+    for u in range(len(cu) - 1):
+        pos = np.arange(cu[u + 1] - cu[u])
+        k[cu[u]:cu[u + 1]] = W.round_bf16(k[cu[u]:cu[u + 1]] * (1 + pos // 128)[:, None])
+    tq, tk, tv = to_dev([q, k, v], "bf16", cuda)
+    o, o_lo, lse = R.attn_forward(tq, tk, tv, cu, H)
+    torch.cuda.synchronize()
+    O_ref, lse_ref = O.attention_core(q, k, v, cu, H)
+    assert_parity((o.float() + o_lo.float()).cpu().numpy(), O_ref, "bf16", "O")
+    assert np.max(np.abs(lse.cpu().numpy() - lse_ref)) <= 1e-3 * np.max(np.abs(lse_ref))
+
+
 def test_ult_union_gradients_equal_per_sample_sums_on_gpu(cuda):
     """Samples of one user ending at rows 100, 257 and 400, encoded once as
     their union (one call) and each alone on its prefix (three calls)."""

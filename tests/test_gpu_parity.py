@@ -148,6 +148,31 @@ def test_bf16_decoder_split_keys(cuda, hd):
     assert_parity(y, oracle_decode(inp, Hm), "bf16", "y")
 
 
+def _growing_memory(w, inp, seed):
+    """A synthetic memory whose rows grow with their position in the user's
+    history (x (1 + position // 128)): each 128-key block scores well above the
+    ones before it."""
+    Hm = W.make_memory(w, seed).astype(np.float64)
+    cu = inp["cu_seqlens"]
+    for u in range(len(cu) - 1):
+        pos = np.arange(cu[u + 1] - cu[u])
+        Hm[cu[u]:cu[u + 1]] *= (1 + pos // 128)[:, None]
+    return W.round_bf16(Hm)
+
+
+@pytest.mark.parametrize("hd", [32, 64])
+def test_bf16_decoder_row_max_growth(cuda, hd):
+    """Keys whose scores grow block by block: a row's running max rises by more
+    than the kernel's 2^8 threshold several times, so it rescales the row's
+    accumulated output in TMEM (the online softmax's correction)."""
+    w = W.small_workload("bf16", lengths=(1000, 300), d=4 * hd, n_heads=4,
+                         requests=[(0, 1000, 40), (1, 300, 9), (0, 600, 3)])
+    inp = W.make_inputs(w, 49)
+    Hm = _growing_memory(w, inp, 49)
+    y = run_decoder(inp, Hm, cuda)
+    assert_parity(y, oracle_decode(inp, Hm), "bf16", "y")
+
+
 @pytest.mark.parametrize("hd", [32, 64])
 def test_bf16_rank_request_split_keys(cuda, hd):
     """The split decoder after an encoder in the same call: prefixes under 1024
