@@ -87,11 +87,29 @@ struct SmemLayout {
   static constexpr int KV = (MODE == 1 || MODE == 2 ? 2 : 1) * NT * Cfg<HD>::TILE_BYTES;
   // a stage holds K and V' (encoder), H (decoder), or H_hi and H_lo
   static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
-  // encoder: per softmax warp, its 32 output rows in bf16 (rows padded by 16 bytes)
-  static constexpr int STG_ROW = HD * 2 + 16;
+  // per softmax warp, its 32 output rows in bf16 (rows padded by 16 bytes): the
+  // encoder's O, or the decoder's o * g as its hi and lo halves side by side
+  static constexpr bool DEC = MODE == 1 || MODE == 2;
+  static constexpr int STG_ROW = (DEC ? 2 : 1) * HD * 2 + 16;
   static constexpr int STG = KV + STAGES * STAGE;
-  static constexpr int TOTAL = STG + (MODE == 0 ? 8 * 32 * STG_ROW : 0);
+  static constexpr bool STAGED_OUT = MODE == 0 || (DEC && HD <= 32);
+  // head_dim 32: every softmax thread's fp32 rows fetched ahead by cp.async, the
+  // item's output gate row (and, decoding, the next item's query row), rows
+  // padded by 16 bytes: [gate rows of 256 threads | query rows of 256 threads]
+  static constexpr bool PREFETCH = HD <= 32 && MODE != 3;
+  static constexpr int PF_ROW = HD * 4 + 16;
+  static constexpr int PF = STG + (STAGED_OUT ? 8 * 32 * STG_ROW : 0);
+  static constexpr int TOTAL = PF + (PREFETCH ? (DEC ? 2 : 1) * 256 * PF_ROW : 0);
 };
+
+// Asynchronous 16-byte copies global -> shared memory (no TMA): a thread
+// fetches its own rows ahead of their use and waits for its own groups.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
@@ -436,6 +454,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float* const part_ml = DEC ? da.part_ml : ea.part_ml;
     const long long part_rows = DEC ? da.nk_rows : ea.rows;
     int cb = 0, qn = 0, cbo = 0;  // cbo: the other tile's key blocks in earlier items
+    // head_dim 32: this thread's fetched-ahead rows (see SmemLayout::PREFETCH)
+    const int tid = threadIdx.x - 128;
+    uint8_t* const pf_gate = smem + L::PF + tid * L::PF_ROW;
+    uint8_t* const pf_q = smem + L::PF + (256 + tid) * L::PF_ROW;
+    // the query row of item k for this thread (row 0 of the tile for rows past its end)
+    auto q_src = [&](const AttnItem& x) {
+      return da.q + (long long)(x.q_row0 + t * ROWS + (r < x.nrow[t] ? r : 0)) * d + x.h * HD;
+    };
+    auto fetch_row = [&](uint8_t* dst, const float* src) {
+#pragma unroll
+      for (int u = 0; u < HD / 4; ++u) cp_async16(dst + 16 * u, src + 4 * u);
+    };
+    int q_fetched = -1;  // the item whose query row is (being) fetched into pf_q
     bool ok = true;
     for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
       const AttnItem w = item_at(k);
@@ -453,12 +484,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           pml[0] = -INFINITY;
           pml[1] = 0.f;
         }
+        if (L::PREFETCH) cp_async_wait<0>();  // a query row fetched for this item lands before pf_q is reused
         cbo += w.nblk[1 - t];
         continue;
       }
       if (DEC) {  // stage q (fp32) as hi + lo bf16 tiles in the swizzled K-major layout
         if (qn >= 1 && !mbar_wait(&q_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
-        const float* qrow = da.q + (long long)(w.q_row0 + t * ROWS + (valid ? r : 0)) * d + h * HD;
+        const float* qrow = q_src(w);
+        if (L::PREFETCH) {  // this item's row was fetched during the previous one, else now
+          if (q_fetched != k) {
+            fetch_row(pf_q, qrow);
+            cp_async_commit();
+          }
+          cp_async_wait<0>();
+          qrow = reinterpret_cast<const float*>(pf_q);
+        }
         uint8_t* qh = smem + L::Q + t * C::TILE_BYTES;
         uint8_t* ql = smem + L::QLO + t * C::TILE_BYTES;
 #pragma unroll
@@ -483,6 +523,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         fence_async_smem();
         mbar_arrive(&q_full[t]);
+      }
+      const long long ro = row_g * d + h * HD;
+      const bool has_gate = DEC || ea.gate != nullptr;  // the encoder's gate may be left out (training core)
+      if (L::PREFETCH) {
+        // this item's output gate row (in flight through the item's key blocks), then,
+        // decoding, the next item's query row (once this item's is staged above)
+        if (valid && !split && has_gate) fetch_row(pf_gate, (DEC ? da.g : ea.gate) + ro);
+        cp_async_commit();
+        if (DEC && k + 1 < sched[blockIdx.x + 1]) {
+          const AttnItem nx = item_at(k + 1);
+          if (nx.nrow[t] > 0) {
+            fetch_row(pf_q, q_src(nx));
+            q_fetched = k + 1;
+          }
+        }
+        cp_async_commit();
       }
       // visible keys: index < row_lim - 128 j (the causal bound and the user end / cutoff)
       const int row_lim = DEC ? w.nkeys : min(w.q_pos0 + t * ROWS + r + 1, w.user_len) - (ESPLIT ? w.key_off : 0);
@@ -588,16 +644,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
-      // the output gate of this row, loaded while the last P V completes (head_dim 32;
-      // at 64 the row would not fit the softmax warps' registers next to O)
-      constexpr bool GATE_EARLY = HD <= 32;
-      const long long ro = row_g * d + h * HD;
-      const bool has_gate = DEC || ea.gate != nullptr;  // the encoder's gate may be left out (training core)
-      float gate_row[GATE_EARLY ? HD : 4];
-      if (GATE_EARLY && valid && !split && has_gate) {
-        const float* gate = (DEC ? da.g : ea.gate) + ro;
+      // the output gate of this row: fetched ahead into shared memory (head_dim 32;
+      // the group of this item's gate is the older of the two in flight), or
+      // loaded here (64: the row would not fit the softmax warps' registers next to O)
+      constexpr bool GATE_ROW = L::PREFETCH;
+      float gate_row[GATE_ROW ? HD : 4];
+      if (GATE_ROW && valid && !split && has_gate) {
+        cp_async_wait<1>();
 #pragma unroll
-        for (int c = 0; c < HD; c += 4) load4(gate + c, &gate_row[c]);
+        for (int c = 0; c < HD; c += 4) load4(reinterpret_cast<const float*>(pf_gate) + c, &gate_row[c]);
       }
       if (!mbar_wait(&p_free[t], (cb + nb - 1) & 1, err, &abort_flag)) { ok = false; break; }  // the last P V
       tc_fence_after();
@@ -612,13 +667,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&o_empty[t]);  // O_t may now be overwritten by the next item
-      if (!DEC && !split && ea.out_lo == nullptr) {
+      if (L::STAGED_OUT && !split && (DEC ? da.out_lo != nullptr : ea.out_lo == nullptr)) {
         // The output rows through shared memory: each lane writes its row's bf16
-        // values into the warp's staging rows, then the warp stores them 16 bytes a
-        // lane, HD / 8 lanes to a row, so that a store instruction writes whole
-        // sectors of a few rows instead of 8 bytes of each of 32 rows.
+        // values (decoding: o * g as hi and lo halves) into the warp's staging
+        // rows, then the warp stores them 16 bytes a lane, HD / 8 lanes to a row,
+        // so that a store instruction writes whole sectors of a few rows instead
+        // of 8 bytes of each of 32 rows.
         const float inv = valid ? 1.0f / l_run : 0.f;
-        if (valid && ea.lse) ea.lse[row_g * n_heads + h] = (m_ref + log2f(l_run)) * 0.69314718055994531f;
+        if (!DEC && valid && ea.lse) ea.lse[row_g * n_heads + h] = (m_ref + log2f(l_run)) * 0.69314718055994531f;
         uint8_t* stg = smem + L::STG + (warp - 4) * 32 * L::STG_ROW;
 #pragma unroll
         for (int c0 = 0; c0 < HD; c0 += 8) {
@@ -626,31 +682,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!has_gate || !valid) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) gh[i] = 1.f;
-          } else if (GATE_EARLY) {
+          } else if (GATE_ROW) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) gh[i] = gate_row[(c0 + i) % (GATE_EARLY ? HD : 4)];
+            for (int i = 0; i < 8; ++i) gh[i] = gate_row[(c0 + i) % (GATE_ROW ? HD : 4)];
           } else {
-            load4(ea.gate + ro + c0, gh);
-            load4(ea.gate + ro + c0 + 4, gh + 4);
+            load4((DEC ? da.g : ea.gate) + ro + c0, gh);
+            load4((DEC ? da.g : ea.gate) + ro + c0 + 4, gh + 4);
           }
-          uint32_t pk[4];
+          uint32_t pk[4], pl[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 t2 = __floats2bfloat162_rn(o[c0 + 2 * i] * inv * gh[2 * i], o[c0 + 2 * i + 1] * inv * gh[2 * i + 1]);
+            const float v0 = o[c0 + 2 * i] * inv * gh[2 * i], v1 = o[c0 + 2 * i + 1] * inv * gh[2 * i + 1];
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(v0, v1);
             pk[i] = *reinterpret_cast<uint32_t*>(&t2);
+            if (DEC) {  // the low part: v - bf16(v)
+              const float2 hf = __bfloat1622float2(t2);
+              __nv_bfloat162 l2 = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+              pl[i] = *reinterpret_cast<uint32_t*>(&l2);
+            }
           }
           *reinterpret_cast<uint4*>(stg + lane * L::STG_ROW + c0 * 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          if (DEC)
+            *reinterpret_cast<uint4*>(stg + lane * L::STG_ROW + HD * 2 + c0 * 2) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
         }
         __syncwarp();
-        constexpr int CPR = HD / 8;  // 16-byte chunks of a row
+        constexpr int CPR = HD / 8;  // 16-byte chunks of a row (of each half)
 #pragma unroll
-        for (int rr = 0; rr < 32; rr += 32 / CPR) {
-          const int r = rr + lane / CPR, ch = lane % CPR;
-          const int tr = q4 * 32 + r;  // row within the tile
-          if (tr < w.nrow[t]) {
-            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * L::STG_ROW + ch * 16);
-            *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(ea.out) + (long long)(w.q_row0 + t * ROWS + tr) * d +
-                                      h * HD + ch * 8) = val;
+        for (int half = 0; half < (DEC ? 2 : 1); ++half) {
+          bf16* const dst = reinterpret_cast<bf16*>(half ? da.out_lo : DEC ? da.out : ea.out);
+#pragma unroll
+          for (int rr = 0; rr < 32; rr += 32 / CPR) {
+            const int r = rr + lane / CPR, ch = lane % CPR;
+            const int tr = q4 * 32 + r;  // row within the tile
+            if (tr < w.nrow[t]) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + r * L::STG_ROW + half * HD * 2 + ch * 16);
+              *reinterpret_cast<uint4*>(dst + (long long)(w.q_row0 + t * ROWS + tr) * d + h * HD + ch * 8) = val;
+            }
           }
         }
         __syncwarp();  // the staging rows are free for the next item
@@ -673,9 +740,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!has_gate) {
 #pragma unroll
               for (int i = 0; i < 4; ++i) gh[c + i] = 1.f;
-            } else if (GATE_EARLY) {
+            } else if (GATE_ROW) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) gh[c + i] = gate_row[(c0 + c + i) % (GATE_EARLY ? HD : 4)];
+              for (int i = 0; i < 4; ++i) gh[c + i] = gate_row[(c0 + c + i) % (GATE_ROW ? HD : 4)];
             } else {
               load4((DEC ? da.g : ea.gate) + ro + c0 + c, &gh[c]);
             }
@@ -709,6 +776,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       cbo += w.nblk[1 - t];
       ++qn;
     }
+    if (L::PREFETCH) cp_async_wait<0>();  // no copy into shared memory outlives the loop
   }
   tc_fence_before();
   __syncthreads();
