@@ -48,7 +48,9 @@ typedef enum {
   REST_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, copy, device query) */
   REST_ERR_TIMEOUT = 5,       /* (device) a bounded wait inside a kernel ran out */
   REST_ERR_WORKSPACE = 6,     /* ws is NULL or smaller than rest_workspace_size() */
-  REST_ERR_NO_DEVICE = 7      /* no CUDA device of compute capability 10.0 is current */
+  REST_ERR_NO_DEVICE = 7,     /* no CUDA device of compute capability 10.0 is current */
+  REST_ERR_RANGE = 8          /* (device) a decoder query or memory value is beyond the fp16 range
+                                 (|v| > 65504) that the bf16 tensor-core decoder computes in */
 } rest_status;
 
 typedef enum { REST_F32 = 0, REST_BF16 = 1 } rest_dtype;

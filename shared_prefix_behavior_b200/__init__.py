@@ -29,7 +29,8 @@ REST_F32, REST_BF16 = 0, 1
 # attention-sublayer gates (rest_gates): value + output (the DGA layer), output only, Q/K/V + output
 GATES = {"vo": 0, "o": 1, "qkvo": 2}
 STATUS = {0: "REST_OK", 1: "REST_ERR_INVALID_ARG", 2: "REST_ERR_UNSORTED_TIME", 3: "REST_ERR_UNSUPPORTED",
-          4: "REST_ERR_CUDA", 5: "REST_ERR_TIMEOUT", 6: "REST_ERR_WORKSPACE", 7: "REST_ERR_NO_DEVICE"}
+          4: "REST_ERR_CUDA", 5: "REST_ERR_TIMEOUT", 6: "REST_ERR_WORKSPACE", 7: "REST_ERR_NO_DEVICE",
+          8: "REST_ERR_RANGE"}
 EXPORTS = ("rest_workspace_size", "rest_rotation_table", "rest_encoder_attn", "rest_cross_decode",
            "rest_rank_request", "rest_status_string", "rest_launch_count", "rest_profile_begin",
            "rest_profile_end", "rest_cross_decode_static_ws", "rest_score_workspace_size", "rest_score_head",

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -31,6 +32,22 @@ __device__ __forceinline__ float exp2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// Largest finite fp16 value: the tensor-core decoder multiplies in fp16, and a
+// query or memory value beyond it is reported (REST_ERR_RANGE).
+constexpr float FP16_MAX = 65504.0f;
+
+// Two floats as an f16x2 pair (round to nearest even), low half first.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// false for a value the fp16 products cannot take (beyond FP16_MAX, or NaN)
+__device__ __forceinline__ bool fits_f16(float v) { return fabsf(v) <= FP16_MAX; }
 
 // Record the first device-side error in the caller's status word.
 __device__ __forceinline__ void set_error(int32_t* err, int code) {

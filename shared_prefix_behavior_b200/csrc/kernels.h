@@ -57,6 +57,12 @@ cudaError_t launch_score_readout(const float* f, const float* w_s, float b_s, fl
 cudaError_t launch_to_f32(bool bf16, const void* x_in, float* x_res, long long n, cudaStream_t s);
 // hi = bf16(x), lo = bf16(x - hi): x as an unevaluated sum of two bf16 numbers
 cudaError_t launch_split_bf16(const float* x, void* hi, void* lo, long long n, cudaStream_t s);
+// hb = bf16(x) and h16 = fp16(x) (the memory of the tensor-core decoder); a
+// value beyond fp16's range sets REST_ERR_RANGE in err. n a multiple of 8,
+// pointers 16-byte aligned.
+cudaError_t launch_split_h16(const float* x, void* hb, void* h16, long long n, int32_t* err, cudaStream_t s);
+// dst = fp16(src) for a bf16 src, with the same range check
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, long long n, int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- GEMM
 enum Epilogue {
@@ -166,8 +172,8 @@ cudaError_t launch_attn_bwd_simt(bool bf16, int hd, int part, const AttnBwdArgs&
 struct DecAttnArgs {
   const float* q;      // [NK, d] decoder queries (fp32)
   const float* g;      // [NK, d] sigmoid output gate
-  const void* h;       // [T, d] encoder memory: keys and values
-  const void* h_lo;    // [T, d] bf16 low part of H (H = h + h_lo), or null
+  const void* h;       // [T, d] encoder memory: keys and values (the tensor-core decoder: fp16)
+  const void* h_lo;    // [T, d] bf16 low part of H (H = h + h_lo), or null (CUDA-core decoder)
   void* out;           // [NK, d] o * g: fp32, or its bf16 high part when out_lo is set
   void* out_lo;        // [NK, d] bf16 low part of o * g, or null
   const DecTile* tiles; int n_tiles;

@@ -113,11 +113,12 @@ static void build_enc_tiles(const rest_batch* b, int rows, std::vector<EncTile>&
 }
 
 constexpr int KEY_BLOCK = 128;   // keys per block of the attention kernels
-// In rank_request the decoder reads H_lo (H = H_hi + H_lo) only for requests
-// with fewer keys than this: H's bf16 rounding reaches y through per-key
-// perturbations that the attention average shrinks about as 1/sqrt(keys), so
-// long prefixes do not need the extra MMA passes, while a cutoff of 1 key
-// passes H's rounding straight into y.
+// In rank_request the CUDA-core decoder (fp32 arithmetic) reads H_lo (H =
+// H_hi + H_lo) for requests with fewer keys than this: H's bf16 rounding reaches
+// y through per-key perturbations that the attention average shrinks about as
+// 1/sqrt(keys), while a cutoff of 1 key passes H's rounding straight into y.
+// (The tensor-core decoder reads H in fp16, 8 times finer than bf16, for every
+// request.)
 constexpr int HLO_MAX_CUTOFF = 1024;
 constexpr int TARGET_CTAS = 296;  // two waves of the B200's 148 SMs
 
@@ -322,16 +323,16 @@ static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_he
 // ---------------------------------------------------------------- workspace
 
 struct Layout {
-  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, dec_sched2, app, bwd_tiles, bwd_sched, meta_end;
+  size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, app, bwd_tiles, bwd_sched, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
-  size_t dq, dg, dout, hlo, part_o, part_ml, delta;
+  size_t dq, dg, dout, hx, part_o, part_ml, delta;
   size_t total;
   int n_enc_tiles, n_dec_tiles, n_bwd_tiles;
 };
 
 static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch* b, long long T, bool enc,
-                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hsplit, int n_split,
-                          size_t n_enc_sched, size_t n_dec_sched, size_t n_dec_sched2, bool append,
+                          int max_dff, long long NK, int n_enc_tiles, int n_dec_tiles, bool hx, int n_split,
+                          size_t n_enc_sched, size_t n_dec_sched, bool append,
                           int n_bwd_tiles = 0, size_t n_bwd_sched = 0, int n_split_enc = 1) {
   Layout L;
   const size_t A = 256, e = dt_size(dt);
@@ -345,7 +346,6 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dec_tiles = take(sizeof(DecTile) * (size_t)n_dec_tiles);
   L.enc_sched = take(sizeof(int) * n_enc_sched);
   L.dec_sched = take(sizeof(int) * n_dec_sched);
-  L.dec_sched2 = take(sizeof(int) * n_dec_sched2);
   L.app = take(append ? sizeof(UserAppend) * (size_t)b->n_users : 0);
   L.n_bwd_tiles = n_bwd_tiles;
   L.bwd_tiles = take(sizeof(EncTile) * (size_t)n_bwd_tiles);
@@ -364,7 +364,8 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dq = take(4 * (size_t)NK * d);
   L.dg = take(4 * (size_t)NK * d);
   L.dout = take(4 * (size_t)NK * d);
-  L.hlo = take(hsplit ? 2 * (size_t)T * d : 0);
+  // H_lo for the CUDA-core decoder, or the fp16 H of the tensor-core decoder
+  L.hx = take(hx ? 2 * (size_t)T * d : 0);
   // split partial results: the decoder's [n_split, NK] or the appending encoder's [n_split_enc, T] rows
   const size_t part_rows = std::max(n_split > 1 ? (size_t)n_split * NK : 0,
                                     n_split_enc > 1 ? (size_t)n_split_enc * T : 0);
@@ -383,14 +384,15 @@ struct Plan {
   int max_dff, K;
   std::vector<EncTile> enc_tiles;
   std::vector<DecTile> dec_tiles;
-  std::vector<int> enc_sched, dec_sched, dec_sched2;  // tensor-core attention: per-CTA item lists
+  std::vector<int> enc_sched, dec_sched;  // tensor-core attention: per-CTA item lists
   std::vector<UserAppend> app;  // appending to a cache: each user's cached prefix
   std::vector<EncTile> bwd_tiles;  // attention core backward: 128-row tiles of every user
   std::vector<int> bwd_sched;      // tensor-core backward: per-CTA lists of (key tile, head) items
-  int n_dec_hlo;  // leading decoder tiles that read H_lo (rank_request, bf16)
+  int n_dec_hlo;  // decoder tiles that read H_lo (CUDA-core decoder in rank_request, bf16)
   Layout L;
   int32_t* err;
-  bool hsplit;
+  bool hsplit;    // the CUDA-core decoder reads H as H_hi + H_lo (the workspace's hx)
+  bool h16;       // the tensor-core decoder: it reads H in fp16 (the workspace's hx)
   int n_split;      // decoder key splits (tensor-core path)
   int n_split_enc;  // encoder key splits when appending (tensor-core path)
 };
@@ -438,7 +440,8 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
     if ((st = check_requests(reqs, b, &p.n_cands)) != REST_OK) return st;
     if (K < 1 || K > 8) return REST_ERR_INVALID_ARG;
   }
-  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false; p.n_split = 1; p.n_dec_hlo = 0;
+  p.dt = dt; p.hs = hs; p.b = b; p.K = K; p.err = nullptr; p.hsplit = false; p.h16 = false; p.n_split = 1;
+  p.n_dec_hlo = 0;
   p.NK = p.n_cands * (reqs ? K : 0);
   if (p.T * (long long)hs->d >= (1LL << 40) || p.NK >= (1LL << 31)) return REST_ERR_UNSUPPORTED;
   const int tile_rows = attn_tile_rows(dt, hs->head_dim);
@@ -460,25 +463,19 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
   p.n_split = 1;
   if (reqs && tile_rows != 128) p.n_split = choose_dec_split(b, reqs, K, tile_rows, hs->n_heads);
   build_dec_tiles(b, reqs, K, tile_rows, p.n_split, p.dec_tiles);
-  // encoder followed by the decoder in bf16: the decoder reads H as hi + lo
+  // The tensor-core decoder multiplies in fp16: it reads an fp16 copy of H that
+  // the encoder's last launch writes beside H (rank_request) or that is converted
+  // from the caller's bf16 H (cross_decode). The CUDA-core decoder after an
+  // encoder in bf16 reads H as hi + lo for short prefixes.
+  p.h16 = reqs != nullptr && tile_rows != 128 && p.NK > 0;
   p.n_dec_hlo = 0;
-  if (encoder_runs && reqs != nullptr && dt == REST_BF16)
+  if (!p.h16 && encoder_runs && reqs != nullptr && dt == REST_BF16)
     for (const DecTile& t : p.dec_tiles) p.n_dec_hlo += t.pad;
   p.hsplit = p.n_dec_hlo > 0;
-  if (!p.hsplit)
-    for (DecTile& t : p.dec_tiles) t.pad = 0;
+  for (DecTile& t : p.dec_tiles) t.pad = 0;
   if (tile_rows != 128) {  // the tensor-core attention runs: schedule its persistent CTAs
     if (!p.enc_tiles.empty()) p.enc_sched = enc_schedule(b, p.enc_tiles, hs->n_heads, tile_rows, p.app);
-    if (!p.dec_tiles.empty()) {  // [tiles that read H_lo | the others], scheduled separately
-      std::vector<DecTile> a(p.dec_tiles.begin(), p.dec_tiles.begin() + p.n_dec_hlo);
-      std::vector<DecTile> c(p.dec_tiles.begin() + p.n_dec_hlo, p.dec_tiles.end());
-      if (a.empty()) {
-        p.dec_sched = dec_schedule(c, hs->n_heads);
-      } else {
-        p.dec_sched = dec_schedule(a, hs->n_heads);
-        if (!c.empty()) p.dec_sched2 = dec_schedule(c, hs->n_heads);
-      }
-    }
+    if (!p.dec_tiles.empty()) p.dec_sched = dec_schedule(p.dec_tiles, hs->n_heads);
   }
   // the attention core alone (training): no encoder buffers; the backward's 128-row tiles
   p.bwd_tiles.clear();
@@ -495,8 +492,8 @@ static rest_status make_plan(Plan& p, rest_dtype dt, const rest_heads* hs, const
     if (tile_rows != 128 && !cost.empty()) p.bwd_sched = lpt_schedule(cost);
   }
   p.L = make_layout(dt, hs, b, p.T, encoder_runs && !core, p.max_dff, p.NK, (int)p.enc_tiles.size(),
-                    (int)p.dec_tiles.size(), p.hsplit, p.n_split, p.enc_sched.size(), p.dec_sched.size(),
-                    p.dec_sched2.size(), append, (int)p.bwd_tiles.size(), p.bwd_sched.size(), p.n_split_enc);
+                    (int)p.dec_tiles.size(), p.hsplit || p.h16, p.n_split, p.enc_sched.size(), p.dec_sched.size(),
+                    append, (int)p.bwd_tiles.size(), p.bwd_sched.size(), p.n_split_enc);
   return REST_OK;
 }
 
@@ -583,8 +580,6 @@ static rest_status upload_meta(const Plan& p, void* ws, cudaStream_t s) {
     memcpy(host.data() + p.L.enc_sched, p.enc_sched.data(), sizeof(int) * p.enc_sched.size());
   if (!p.dec_sched.empty())
     memcpy(host.data() + p.L.dec_sched, p.dec_sched.data(), sizeof(int) * p.dec_sched.size());
-  if (!p.dec_sched2.empty())
-    memcpy(host.data() + p.L.dec_sched2, p.dec_sched2.data(), sizeof(int) * p.dec_sched2.size());
   if (!p.app.empty()) memcpy(host.data() + p.L.app, p.app.data(), sizeof(UserAppend) * p.app.size());
   if (!p.bwd_tiles.empty())
     memcpy(host.data() + p.L.bwd_tiles, p.bwd_tiles.data(), sizeof(EncTile) * p.bwd_tiles.size());
@@ -787,7 +782,7 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
       else if (S.post) st = norm(y, S.g, S.b, 4, N.g, N.b);                     // x = LN(x), y = LN'(x)
       else st = norm(y, N.g, N.b, 0, nullptr, nullptr);                         // y = LN'(x)
     } else if (S.post) {
-      if (p.hsplit) {
+      if (p.hsplit || p.h16) {
         st = norm(nullptr, S.g, S.b, 3, nullptr, nullptr);  // x = LN(x)
       } else {
         st = norm(h_out, S.g, S.b, 1, nullptr, nullptr);    // x = LN(x), H = x
@@ -797,9 +792,12 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
     if (st != REST_OK) return st;
   }
   // H: the residual stream after the last layer, in the call's dtype (no final norm).
-  // When the decoder follows in bf16 it also gets H's low part: H = h_out + h_lo.
-  if (p.hsplit) {
-    REST_KLAUNCH(s, "split_h", 0, Td * 8, launch_split_bf16(xres, h_out, at<void>(ws, L.hlo), T * d, s));
+  // When the tensor-core decoder follows, also H in fp16 (what it multiplies in);
+  // when the CUDA-core decoder follows in bf16, H's low part: H = h_out + h_lo.
+  if (p.h16) {
+    REST_KLAUNCH(s, "split_h", 0, Td * 8, launch_split_h16(xres, h_out, at<void>(ws, L.hx), T * d, err, s));
+  } else if (p.hsplit) {
+    REST_KLAUNCH(s, "split_h", 0, Td * 8, launch_split_bf16(xres, h_out, at<void>(ws, L.hx), T * d, s));
   } else if (!h_written) {
     if (rest_status st = norm(h_out, nullptr, nullptr, 2, nullptr, nullptr)) return st;
   }
@@ -811,7 +809,10 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
 
 // ---------------------------------------------------------------- decoder
 
-static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const void* h, const void* h_lo,
+// h: the caller's H (the call's dtype). from_encoder: the encoder ran in the
+// same call and left the workspace's hx as the decoder needs it (the fp16 H of
+// the tensor-core decoder, or H_lo of the CUDA-core one).
+static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const void* h, bool from_encoder,
                                const void* z, const rest_dec_params* dec, float* y_out, void* ws, int32_t* err,
                                cudaStream_t s) {
   const bool bf = p.dt == REST_BF16;
@@ -840,6 +841,15 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
              dg + (size_t)kk * d, (long long)K * d);
     if (rest_status st = run_gemm(p, a, "gemm_dec_g", s)) return st;
   }
+  // The tensor-core decoder multiplies in fp16 (H, q and P): its H is the fp16
+  // copy in the workspace, converted here unless the encoder wrote it.
+  const bool tc = bf && sm100_attn_supported(hd);
+  const void* h_lo = !tc && from_encoder && p.hsplit ? at<void>(ws, L.hx) : nullptr;
+  if (tc) {
+    if (!from_encoder)
+      REST_KLAUNCH(s, "h_to_f16", 0, 4.0 * p.T * d, launch_bf16_to_f16(h, at<void>(ws, L.hx), p.T * d, err, s));
+    h = at<void>(ws, L.hx);
+  }
   // every H prefix is read once per request; each candidate row reads q, g and writes o
   double flops = 0, hbytes = 0;
   for (int r = 0; r < reqs->n_req; ++r) {
@@ -851,7 +861,6 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   const double bytes = hbytes + (double)p.NK * d * 12;
   // The tensor-core decoder hands o * g to the output projection as a hi + lo
   // pair of bf16 arrays (in the same workspace bytes); the CUDA-core one as fp32.
-  const bool tc = bf && sm100_attn_supported(hd);
   DecAttnArgs da;
   memset(&da, 0, sizeof(da));
   da.q = dq; da.g = dg; da.h = h; da.h_lo = h_lo; da.out = dout;
@@ -865,29 +874,10 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   da.nk_rows = p.NK;
   da.part_o = at<float>(ws, L.part_o);
   da.part_ml = at<float>(ws, L.part_ml);
-  if (bf && sm100_attn_supported(hd)) {
-    // tiles that read H_lo (short cutoffs, within rank_request) and the others
-    const int n_hlo = h_lo ? p.n_dec_hlo : 0;
-    const int n_rest = L.n_dec_tiles - n_hlo;
-    const int H = p.hs->n_heads;
-    if (n_hlo > 0) {
-      DecAttnArgs a1 = da;
-      a1.n_tiles = n_hlo;
-      a1.sched = at<int>(ws, L.dec_sched);
-      a1.n_cta = std::min(n_hlo * H, SCHED_CTAS);
-      REST_KLAUNCH(s, "dec_attn", flops * n_hlo / L.n_dec_tiles, bytes * n_hlo / L.n_dec_tiles,
-                   launch_dec_attn_sm100(hd, a1, s, err));
-    }
-    if (n_rest > 0) {
-      DecAttnArgs a2 = da;
-      a2.h_lo = nullptr;
-      a2.tiles = da.tiles + n_hlo;
-      a2.n_tiles = n_rest;
-      a2.sched = at<int>(ws, n_hlo > 0 ? L.dec_sched2 : L.dec_sched);
-      a2.n_cta = std::min(n_rest * H, SCHED_CTAS);
-      REST_KLAUNCH(s, "dec_attn", flops * n_rest / L.n_dec_tiles, bytes * n_rest / L.n_dec_tiles,
-                   launch_dec_attn_sm100(hd, a2, s, err));
-    }
+  if (tc) {
+    da.sched = at<int>(ws, L.dec_sched);
+    da.n_cta = std::min(L.n_dec_tiles * p.hs->n_heads, SCHED_CTAS);
+    if (L.n_dec_tiles > 0) REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_sm100(hd, da, s, err));
     if (p.n_split > 1)
       REST_KLAUNCH(s, "dec_combine", 0, (double)p.NK * d * 4 * (p.n_split + 2),
                    launch_dec_combine(hd, da, s));
@@ -919,6 +909,7 @@ const char* rest_status_string(rest_status s) {
     case REST_ERR_TIMEOUT: return "bounded device wait ran out";
     case REST_ERR_WORKSPACE: return "workspace missing or too small";
     case REST_ERR_NO_DEVICE: return "no sm_100 CUDA device is current";
+    case REST_ERR_RANGE: return "decoder value beyond the fp16 range";
   }
   return "unknown status";
 }
@@ -1210,7 +1201,7 @@ rest_status rest_cross_decode(rest_dtype dt, const rest_heads* heads, const rest
     cudaStream_t s = (cudaStream_t)stream;
     p.err = dev_err;
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
-    return run_decoder(p, reqs, h, nullptr, z, dec, y_out, ws, dev_err, s);
+    return run_decoder(p, reqs, h, false, z, dec, y_out, ws, dev_err, s);
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }
@@ -1237,7 +1228,7 @@ rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
     if ((st = run_encoder(p, x, ts, layers, n_layers, l_switch, h_out, ws, dev_err, s)) != REST_OK) return st;
     if (p.NK == 0) return REST_OK;
-    return run_decoder(p, reqs, h_out, p.hsplit ? at<void>(ws, p.L.hlo) : nullptr, z, dec, y_out, ws, dev_err, s);
+    return run_decoder(p, reqs, h_out, true, z, dec, y_out, ws, dev_err, s);
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }
@@ -1408,7 +1399,7 @@ extern "C" rest_status rest_cross_decode_static_ws(rest_dtype dt, const rest_hea
     // Nothing in the scratch needs to start at zero: the index/tile lists are
     // uploaded and q, g, o are written in full before they are read.
     if ((st = upload_meta(p, ws, s)) != REST_OK) return st;
-    return run_decoder(p, reqs, h, nullptr, z, dec, y_out, ws, dev_err, s);
+    return run_decoder(p, reqs, h, false, z, dec, y_out, ws, dev_err, s);
   } catch (...) {
     return REST_ERR_INVALID_ARG;
   }

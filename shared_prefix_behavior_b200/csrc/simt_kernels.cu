@@ -605,6 +605,73 @@ cudaError_t launch_split_bf16(const float* x, void* hi, void* lo, long long n, c
   return launch_k(split_bf16_scalar_kernel, (unsigned)blocks, threads, 0, s, x, (bf16*)hi, (bf16*)lo, n);
 }
 
+// H for the tensor-core decoder, which multiplies in fp16: from the fp32
+// residual stream, H in bf16 (the call's output) and an fp16 copy, 8 values per
+// thread; a value beyond fp16's range sets REST_ERR_RANGE.
+__global__ void split_h16_kernel(const float4* __restrict__ x, uint4* __restrict__ hb, uint4* __restrict__ h16,
+                                 long long n8, int32_t* err) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = x[2 * i], b = x[2 * i + 1];
+  const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t hh[4], hf[4];
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    hh[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
+    hf[k] = pack_f16x2(v[2 * k], v[2 * k + 1]);
+    ok = ok && fits_f16(v[2 * k]) && fits_f16(v[2 * k + 1]);
+  }
+  hb[i] = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+  h16[i] = make_uint4(hf[0], hf[1], hf[2], hf[3]);
+  if (!ok) set_error(err, REST_ERR_RANGE);
+}
+
+// The caller's bf16 H as fp16 for the tensor-core decoder, 8 values per thread
+// (exact within fp16's range; a value beyond it sets REST_ERR_RANGE).
+__global__ void bf16_to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long long n8,
+                                   int32_t* err) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 w4 = src[i];
+  const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+  uint32_t hf[4];
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xffff0000u);
+    hf[k] = pack_f16x2(lo, hi);
+    ok = ok && fits_f16(lo) && fits_f16(hi);
+  }
+  dst[i] = make_uint4(hf[0], hf[1], hf[2], hf[3]);
+  if (!ok) set_error(err, REST_ERR_RANGE);
+}
+
+cudaError_t launch_split_h16(const float* x, void* hb, void* h16, long long n, int32_t* err, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8 != 0 || ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(hb) |
+                      reinterpret_cast<uintptr_t>(h16)) & 15) != 0)
+    return cudaErrorInvalidValue;  // d is a multiple of 32 and the buffers 16-byte aligned
+  const int threads = 256;
+  const long long n8 = n / 8;
+  return launch_k(split_h16_kernel, (unsigned)((n8 + threads - 1) / threads), threads, 0, s,
+                  reinterpret_cast<const float4*>(x), static_cast<uint4*>(hb), static_cast<uint4*>(h16), n8, err);
+}
+
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, long long n, int32_t* err, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8 != 0 || ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) != 0)
+    return cudaErrorInvalidValue;
+  const int threads = 256;
+  const long long n8 = n / 8;
+  return launch_k(bf16_to_f16_kernel, (unsigned)((n8 + threads - 1) / threads), threads, 0, s,
+                  static_cast<const uint4*>(src), static_cast<uint4*>(dst), n8, err);
+}
+
 // ============================================================================
 // Tiled GEMM with the fused epilogues
 // ============================================================================

@@ -9,14 +9,14 @@
 //                128-key block. Decoder: H (and H_lo) per block; one H tile
 //                is both the keys (K-major operand of S = q H^T) and the
 //                values (N-major operand of O = P H).
-//   warp 1       TMEM owner and S issuer: S_t(j) = Q_t K_j^T for both tiles into
-//                each tile's 128-column TMEM buffer, as soon as the tile's
-//                softmax has read S_t(j-1).
-//   warps 2, 3   P V issuers of tiles 0 and 1: O_t += P_t(j) V_j into the
-//                tile's head_dim-column accumulator once P_t(j) is written. A
-//                warp issues one tcgen05.mma about every hundred cycles whatever
-//                its size (measured), so the products are spread over three
-//                issuing warps, each running whole with one elected lane.
+//   warps 1, 2   MMA issuers of tiles 0 and 1 (warp 1 also owns TMEM): per
+//                block j, S_t(j) = Q_t K_j^T into the tile's 128-column TMEM
+//                buffer as soon as its softmax has read S_t(j-1), then
+//                O_t += P_t(j-1) V_{j-1} into the tile's head_dim-column
+//                accumulator once P_t(j-1) is written. A warp issues one
+//                tcgen05.mma about every hundred cycles whatever its size
+//                (measured), so each tile has its own issuing warp, running
+//                whole with one elected lane.
 //   warp 3       head_dim 32: first decodes the CTA's work items into a
 //                shared-memory table (a lane per item).
 //   warps 4..7   softmax of tile 0, warps 8..11 of tile 1: a thread owns a
@@ -33,12 +33,14 @@
 //                share a sub-partition's special-function unit, take turns at
 //                the exponentials block by block. The encoder's output rows go
 //                out through a per-warp staging area in shared memory.
-// The decoder's query comes in fp32 and is staged as a hi + lo pair of bf16
-// tiles (S = q_hi H^T + q_lo H^T); when the encoder ran in the same call the
-// decoder also reads H_lo (H = H_hi + H_lo): S adds q_hi H_lo^T, O adds P H_lo.
+// The decoder multiplies in fp16 (kind::f16 with fp16 operands, fp32
+// accumulation): H comes as an fp16 copy, the fp32 query is staged in fp16
+// (scaled by log2(e) / sqrt(head_dim) first, so S is in the base-2 domain), and
+// P is written as fp16 pairs. fp16's 11-bit significand rounds q, H and P 8
+// times finer than bf16; a query value beyond fp16's range sets REST_ERR_RANGE.
 //
-// MODE 0: encoder; 1: decoder over H; 2: decoder over H_hi + H_lo; 3: encoder
-// over a range of key blocks (appending with split keys), writing partials.
+// MODE 0: encoder; 1: decoder; 3: encoder over a range of key blocks
+// (appending with split keys), writing partials.
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
@@ -80,16 +82,15 @@ __device__ __forceinline__ uint32_t swz_off(int r, int u) {
 
 template <int HD, int MODE>
 struct SmemLayout {
-  // [Q_0 | Q_1 | (decoder) Qlo_0 | Qlo_1 | KV stages], 1024-aligned blocks
-  static constexpr int STAGES = MODE == 2 ? 2 : 3;
+  // [Q_0 | Q_1 | KV stages], 1024-aligned blocks
+  static constexpr int STAGES = 3;
   static constexpr int Q = 0;
-  static constexpr int QLO = NT * Cfg<HD>::TILE_BYTES;
-  static constexpr int KV = (MODE == 1 || MODE == 2 ? 2 : 1) * NT * Cfg<HD>::TILE_BYTES;
-  // a stage holds K and V' (encoder), H (decoder), or H_hi and H_lo
+  static constexpr int KV = NT * Cfg<HD>::TILE_BYTES;
+  // a stage holds K and V' (encoder) or H (decoder)
   static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
   // per softmax warp, its 32 output rows in bf16 (rows padded by 16 bytes): the
   // encoder's O, or the decoder's o * g as its hi and lo halves side by side
-  static constexpr bool DEC = MODE == 1 || MODE == 2;
+  static constexpr bool DEC = MODE == 1;
   static constexpr int STG_ROW = (DEC ? 2 : 1) * HD * 2 + 16;
   static constexpr int STG = KV + STAGES * STAGE;
   static constexpr bool STAGED_OUT = MODE == 0 || (DEC && HD <= 32);
@@ -207,7 +208,7 @@ template <int HD, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, EncAttnArgs ea, DecAttnArgs da, int32_t* err) {
-  constexpr bool DEC = MODE == 1 || MODE == 2, HLO = MODE == 2, ESPLIT = MODE == 3;
+  constexpr bool DEC = MODE == 1, ESPLIT = MODE == 3;
   // head_dim 64: the two tiles' softmax warps of a lane quarter take turns at the
   // exponentials block by block (see the softmax); at 32 they do not.
   constexpr bool TURNS = HD >= 64;
@@ -247,9 +248,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1 + NT);  // one arrival per MMA-issuing warp
+      mbar_init(&kv_empty[s], NT);  // one arrival per MMA-issuing warp
     }
-    mbar_init(&drain, 1 + NT);
+    mbar_init(&drain, NT);
     for (int t = 0; t < NT; ++t)
       for (int q = 0; q < 4; ++q) {
         mbar_init(&xe[t][q][0], 1);
@@ -285,8 +286,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp < 4) {
     setmaxnreg_dec72();
     // Warp 0, lane 0 loads (the other lanes of warp 0 have no role and wait at
-    // the end); warp 1 issues S; warps 2 and 3 issue P V. The issuing warps run
-    // whole: their elect.sync needs every lane.
+    // the end); warps 1 and 2 issue the MMAs of tiles 0 and 1 (warp 3 has no
+    // role after the item table). The issuing warps run whole: their
+    // elect.sync needs every lane.
     if (warp == 0 && lane == 0) {
       // -------------------------------------------------------- TMA producer
       int g = 0, issued = 0, qn[NT] = {0, 0};
@@ -321,112 +323,70 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
           mbar_wait(&kv_full[i % STAGES], (i / STAGES) & 1, nullptr, &no_abort);
       }
-    } else if (warp == 1) {
-      // -------------------------------------------------------- S issuer
-      // S_t(j) = Q_t K_j^T for both tiles, each into its tile's S buffer as soon
-      // as the tile's softmax has loaded the previous S into registers (s_free),
-      // so the next scores are ready while it exponentiates. The whole warp runs
-      // the loop and one elected lane issues: a warp issues one tcgen05.mma about
-      // every hundred cycles whatever its size, so the S and the P V products of
-      // the two tiles are spread over three issuing warps.
-      constexpr uint32_t idS = idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
-      uint64_t qd[NT], qld[NT];
-      for (int t = 0; t < NT; ++t) {
-        qd[t] = smem_desc(smem_u32(smem + L::Q + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
-        qld[t] = smem_desc(smem_u32(smem + L::QLO + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
-      }
-      int g = 0, ns[NT] = {0, 0}, qn[NT] = {0, 0};  // ns: S blocks issued per tile in earlier items
-      bool ok = true;
-      for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-        const AttnItem w = item_at(k);
-        const int nblk_all = max(w.nblk[0], w.nblk[1]);
-        for (int t = 0; t < NT && ok; ++t)
-          if (w.nblk[t] > 0) ok = mbar_wait(&q_full[t], qn[t] & 1, err, &abort_flag);
-        tc_fence_after();
-        for (int j = 0; ok && j < nblk_all; ++j) {
-          const int st = (g + j) % STAGES;
-          if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          // Descriptors step along K: 16 elements are 32 bytes, 2 in the 16-byte address field.
-          const uint64_t kd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE), 16, C::ATOM, C::SWZ);
-          for (int t = 0; t < NT; ++t) {
-            if (j >= w.nblk[t]) continue;
-            const int n = ns[t] + j;  // the tile's S block number
-            if (n >= 1) {             // S_t(n - 1) has been read: the buffer is free
-              if (!mbar_wait(&s_free[t], (n - 1) & 1, err, &abort_flag)) { ok = false; break; }
-              tc_fence_after();
-            }
-            const uint32_t tS = tmem + s_col(t);
-  #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk) mma_bf16_e(tS, qd[t] + 2 * kk, kd + 2 * kk, idS, kk != 0);
-            if (DEC) {  // + q_lo . H^T
-  #pragma unroll
-              for (int kk = 0; kk < HD / 16; ++kk) mma_bf16_e(tS, qld[t] + 2 * kk, kd + 2 * kk, idS, 1);
-            }
-            if (HLO) {  // + q_hi . H_lo^T
-  #pragma unroll
-              for (int kk = 0; kk < HD / 16; ++kk)
-                mma_bf16_e(tS, qd[t] + 2 * kk, kd + (C::TILE_BYTES >> 4) + 2 * kk, idS, 1);
-            }
-            if (j == w.nblk[t] - 1) mma_commit_e(&q_empty[t]);  // the item's last read of Q_t
-            mma_commit_e(&s_full[t]);
-          }
-          if (ok) mma_commit_e(&kv_empty[st]);  // this block's keys have been read
-        }
-        g += nblk_all;
-        for (int t = 0; t < NT; ++t)
-          if (w.nblk[t] > 0) {
-            ns[t] += w.nblk[t];
-            ++qn[t];
-          }
-      }
-      mma_commit_e(&drain);
-      volatile int no_abort = 0;
-      mbar_wait(&drain, 0, nullptr, &no_abort);
-    } else if (warp >= 2) {
-      // -------------------------------------------------------- P V issuers
-      // Warp 2 for tile 0, warp 3 for tile 1: O_t += P_t(j) V_j once the softmax
-      // has written P_t(j) into TMEM (p_full). A block's K/V stage is released when
-      // the S issuer and both P V issuers have committed it (kv_empty counts three
-      // arrivals); a tile with fewer blocks in the item still waits for each
-      // remaining block to land before releasing it, so no issuer can arrive for a
-      // later use of a stage before the earlier use has completed.
-      const int t = warp - 2;
-      constexpr uint32_t idO = idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
+    } else if (warp == 1 || warp == 2) {
+      // -------------------------------------------------------- MMA issuers
+      // Warp 1 for tile 0, warp 2 for tile 1: S_t(j) = Q_t K_j^T into the tile's S
+      // buffer as soon as its softmax has loaded S_t(j-1) (s_free), then
+      // O_t += P_t(j-1) V_{j-1} once P_t(j-1) is written (p_full). A warp issues one
+      // tcgen05.mma about every hundred cycles whatever its size (measured), so
+      // each tile has its own issuing warp, which also keeps one tile's softmax
+      // from waiting on the other's. The whole warp runs the loop and one elected
+      // lane issues. A block's K/V stage is released when both issuers have
+      // committed it (kv_empty counts two arrivals); a tile with fewer blocks in
+      // the item still waits for each remaining block to land before releasing
+      // it, so neither issuer can arrive for a later use of a stage before the
+      // earlier use has completed.
+      const int t = warp - 1;
+      // the decoder's operands are fp16, the encoder's bf16
+      constexpr uint32_t idS = DEC ? idesc_f16(KB, 0) : idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
+      constexpr uint32_t idO = DEC ? idesc_f16(HD, 1) : idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
       constexpr uint32_t V_STEP = (2 * C::ATOM) >> 4;  // 16 keys of V: two 8-row atoms
-      const uint32_t tO = tmem + o_col<HD>(t), tP = tmem + p_col<HD>(t);
+      const uint32_t tS = tmem + s_col(t), tO = tmem + o_col<HD>(t), tP = tmem + p_col<HD>(t);
+      // Descriptors step along K: 16 elements are 32 bytes, 2 in the 16-byte address field.
+      const uint64_t qd = smem_desc(smem_u32(smem + L::Q + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
       int g = 0, cb = 0, qn = 0;
       bool ok = true;
       for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
         const AttnItem w = item_at(k);
         const int nblk_all = max(w.nblk[0], w.nblk[1]);
         const int nb = w.nblk[t];
-        for (int j = 0; ok && j < nblk_all; ++j) {
-          const int st = (g + j) % STAGES;
-          if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
-          if (j >= nb) {  // a block this tile has no rows for
-            if (lane == 0) mbar_arrive(&kv_empty[st]);
-            continue;
-          }
-          if (!mbar_wait(&p_full[t], (cb + j) & 1, err, &abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          if (j == 0 && qn >= 1) {  // the previous item's O_t has been read out
-            if (!mbar_wait(&o_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
+        if (nb > 0) ok = mbar_wait(&q_full[t], qn & 1, err, &abort_flag);
+        tc_fence_after();
+        for (int j = 0; ok && j <= nb; ++j) {
+          if (j < nb) {  // S(j), overwriting the tile's S buffer
+            const int st = (g + j) % STAGES;
+            if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+            if (cb + j >= 1 && !mbar_wait(&s_free[t], (cb + j - 1) & 1, err, &abort_flag)) { ok = false; break; }
             tc_fence_after();
-          }
-          const uint64_t vd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE + (DEC ? 0 : C::TILE_BYTES)),
-                                        64 * KB * 2, C::ATOM, C::SWZ);
-          // A = P_t from TMEM, 8 columns per K step of 16
+            const uint64_t kd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE), 16, C::ATOM, C::SWZ);
   #pragma unroll
-          for (int kk = 0; kk < KB / 16; ++kk)
-            mma_bf16_ts_e(tO, tP + kk * 8, vd + V_STEP * kk, idO, (j | kk) != 0);
-          if (HLO) {  // + P H_lo
+            for (int kk = 0; kk < HD / 16; ++kk) mma_bf16_e(tS, qd + 2 * kk, kd + 2 * kk, idS, kk != 0);
+            if (j == nb - 1) mma_commit_e(&q_empty[t]);  // the item's last read of Q_t
+            mma_commit_e(&s_full[t]);
+          }
+          if (j >= 1) {  // O += P(j-1) V_{j-1}
+            const int i = j - 1, st = (g + i) % STAGES;
+            if (!mbar_wait(&p_full[t], (cb + i) & 1, err, &abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (i == 0 && qn >= 1) {  // the previous item's O_t has been read out
+              if (!mbar_wait(&o_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
+              tc_fence_after();
+            }
+            const uint64_t vd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE + (DEC ? 0 : C::TILE_BYTES)),
+                                          64 * KB * 2, C::ATOM, C::SWZ);
+            // A = P_t from TMEM, 8 columns per K step of 16
   #pragma unroll
             for (int kk = 0; kk < KB / 16; ++kk)
-              mma_bf16_ts_e(tO, tP + kk * 8, vd + (C::TILE_BYTES >> 4) + V_STEP * kk, idO, 1);
+              mma_bf16_ts_e(tO, tP + kk * 8, vd + V_STEP * kk, idO, (i | kk) != 0);
+            mma_commit_e(&p_free[t]);
+            mma_commit_e(&kv_empty[st]);  // this tile is done with block i (its S and its P V)
           }
-          mma_commit_e(&p_free[t]);
-          mma_commit_e(&kv_empty[st]);  // this tile is done with block j
+        }
+        // the item's blocks this tile has no rows for: released once each has landed
+        for (int j = nb; ok && j < nblk_all; ++j) {
+          const int st = (g + j) % STAGES;
+          if (!mbar_wait(&kv_full[st], ((g + j) / STAGES) & 1, err, &abort_flag)) { ok = false; break; }
+          if (lane == 0) mbar_arrive(&kv_empty[st]);
         }
         g += nblk_all;
         if (nb > 0) {
@@ -445,7 +405,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q4 = warp & 3;                     // TMEM lane quarter
     const int r = q4 * 32 + lane;                // row within the tile
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const float sl2 = DEC ? da.scale_log2 : ea.scale_log2;
+    // the decoder's scores arrive in the base-2 domain (its query is staged pre-scaled)
+    const float sl2 = DEC ? 1.0f : ea.scale_log2;
     const uint32_t tS = tmem + lane_off + s_col(t);
     const uint32_t tO = tmem + lane_off + o_col<HD>(t);
     const uint32_t tP = tmem + lane_off + p_col<HD>(t);
@@ -488,7 +449,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         cbo += w.nblk[1 - t];
         continue;
       }
-      if (DEC) {  // stage q (fp32) as hi + lo bf16 tiles in the swizzled K-major layout
+      if (DEC) {  // stage q (fp32) in fp16, scaled to the base-2 domain, in the swizzled K-major layout
         if (qn >= 1 && !mbar_wait(&q_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
         const float* qrow = q_src(w);
         if (L::PREFETCH) {  // this item's row was fetched during the previous one, else now
@@ -500,7 +461,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           qrow = reinterpret_cast<const float*>(pf_q);
         }
         uint8_t* qh = smem + L::Q + t * C::TILE_BYTES;
-        uint8_t* ql = smem + L::QLO + t * C::TILE_BYTES;
+        const float qs = da.scale_log2;
+        bool in_range = true;
 #pragma unroll
         for (int u = 0; u < HD / 8; ++u) {
           float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -508,19 +470,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             load4(qrow + 8 * u, v);
             load4(qrow + 8 * u + 4, v + 4);
           }
-          uint32_t hi[4], lo[4];
+          uint32_t hf[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-            float2 hf = __bfloat1622float2(h2);
-            __nv_bfloat162 l2 = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
-            hi[e] = *reinterpret_cast<uint32_t*>(&h2);
-            lo[e] = *reinterpret_cast<uint32_t*>(&l2);
+            const float a = v[2 * e] * qs, b = v[2 * e + 1] * qs;
+            in_range = in_range && fits_f16(a) && fits_f16(b);
+            hf[e] = pack_f16x2(a, b);
           }
-          const uint32_t off = swz_off<HD>(r, u);
-          *reinterpret_cast<uint4*>(qh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(ql + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(qh + swz_off<HD>(r, u)) = make_uint4(hf[0], hf[1], hf[2], hf[3]);
         }
+        if (!in_range) set_error(err, REST_ERR_RANGE);
         fence_async_smem();
         mbar_arrive(&q_full[t]);
       }
@@ -616,8 +575,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m_ref, -m_ref);
-        // P as bf16 pairs (keys 2c, 2c+1 in column c), stored into the tile's P
-        // columns of TMEM once the previous P V has completed
+        // P as bf16 (decoder: fp16) pairs, keys 2c, 2c+1 in column c, stored into the
+        // tile's P columns of TMEM once the previous P V has completed
         uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -625,8 +584,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float2 x = ffma2(make_float2(s[e], s[e + 1]), scale2, neg_m2);
           const float p0 = exp2_approx(x.x), p1 = exp2_approx(x.y);
           sum2[c & 1] = fadd2(sum2[c & 1], make_float2(p0, p1));
-          __nv_bfloat162 t2 = __floats2bfloat162_rn(p0, p1);
-          pk[c] = *reinterpret_cast<uint32_t*>(&t2);
+          pk[c] = DEC ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
         }
         if (TURNS) {
           __syncwarp();
@@ -788,18 +746,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 template <int HD, int MODE>
 cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream_t s, int32_t* err) {
-  constexpr bool DEC = MODE == 1 || MODE == 2;
+  constexpr bool DEC = MODE == 1;
   const int swz = HD == 64 ? 128 : 64;
   CUtensorMap mq, mk, mv;
   const int n_tiles = DEC ? da->n_tiles : ea->n_tiles;
   const int d = DEC ? da->d : ea->d;
   if (n_tiles == 0) return cudaSuccess;
   const long long rows = DEC ? da->key_rows : ea->rows;
-  if (DEC) {
+  if (DEC) {  // fp16 H, moved as 2-byte elements like bf16
     if (!make_tmap_bf16(&mk, da->h, rows, d, d, HD, ROWS, swz)) return cudaErrorInvalidValue;
     mq = mk;
     mv = mk;
-    if (MODE == 2 && !make_tmap_bf16(&mv, da->h_lo, rows, d, d, HD, ROWS, swz)) return cudaErrorInvalidValue;
   } else {
     const long long key_rows = ea->app ? ea->key_rows : rows;
     if (!make_tmap_bf16(&mq, ea->q, rows, d, d, HD, ROWS, swz) ||
@@ -836,7 +793,6 @@ cudaError_t launch_enc_attn_sm100(int hd, const EncAttnArgs& a, cudaStream_t s, 
 }
 
 cudaError_t launch_dec_attn_sm100(int hd, const DecAttnArgs& a, cudaStream_t s, int32_t* err) {
-  if (a.h_lo) return hd == 64 ? launch_attn<64, 2>(nullptr, &a, s, err) : launch_attn<32, 2>(nullptr, &a, s, err);
   return hd == 64 ? launch_attn<64, 1>(nullptr, &a, s, err) : launch_attn<32, 1>(nullptr, &a, s, err);
 }
 

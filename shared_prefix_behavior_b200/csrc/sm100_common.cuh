@@ -274,6 +274,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, int b_mn) {
          | ((uint32_t)(128 >> 4) << 24); // M / 16
 }
 
+// The same for fp16 A and B (formats 0): kind::f16 takes both operands in one type.
+__host__ __device__ constexpr uint32_t idesc_f16(int n, int b_mn) {
+  return idesc_bf16(n, b_mn) & ~((7u << 7) | (7u << 10));
+}
+
 // The same with the majorness of A chosen too (a_mn = 1: A MN-major).
 __host__ __device__ constexpr uint32_t idesc_bf16_ab(int n, int a_mn, int b_mn) {
   return idesc_bf16(n, b_mn) | ((uint32_t)a_mn << 15);

@@ -37,7 +37,7 @@ def test_static_ws_size_matches_the_header():
 
 
 def test_status_strings():
-    for code in range(8):
+    for code in range(9):
         assert R.library().rest_status_string(code)
     assert R.library().rest_status_string(0) == b"ok"
 

@@ -173,10 +173,23 @@ def test_bf16_decoder_row_max_growth(cuda, hd):
     assert_parity(y, oracle_decode(inp, Hm), "bf16", "y")
 
 
+def test_decoder_reports_values_beyond_fp16(cuda):
+    """The tensor-core decoder multiplies in fp16: a memory value that bf16
+    holds but fp16 does not (1e5 > 65504) is reported on the device status
+    word as REST_ERR_RANGE instead of turning the scores into infinities."""
+    w = W.small_workload("bf16", lengths=(300,), d=128, n_heads=4, requests=[(0, 300, 5)])
+    inp = W.make_inputs(w, 50)
+    Hm = W.make_memory(w, 50)
+    Hm[17, 5] = 1.0e5
+    with pytest.raises(R.RestError) as e:
+        run_decoder(inp, Hm, cuda)
+    assert e.value.status == 8
+
+
 @pytest.mark.parametrize("hd", [32, 64])
 def test_bf16_rank_request_split_keys(cuda, hd):
-    """The split decoder after an encoder in the same call: prefixes under 1024
-    keys also read H_lo (the third operand pair of the tensor-core decoder)."""
+    """The split decoder after an encoder in the same call, reading the fp16
+    copy of H that the encoder's last launch writes beside H."""
     w = W.small_workload("bf16", lengths=(1800, 300), d=4 * hd, n_heads=4, n_layers=1, l_switch=0,
                          requests=[(0, 1800, 12), (1, 300, 5), (0, 400, 3)])
     inp = W.make_inputs(w, 48)
