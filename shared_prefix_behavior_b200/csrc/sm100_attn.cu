@@ -131,6 +131,31 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+// 2^x for two values on the FMA and integer pipes instead of the special-function
+// unit. x = n + f with n the nearest integer (adding 1.5 * 2^23 leaves n in the
+// low bits of the sum) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial
+// fitted here for least maximum relative error on that interval (Remez
+// exchange: 7.5e-5, below the bf16 or fp16 rounding P gets), times 2^n built in
+// the exponent field. x is first raised to -127, where 2^n's bits are those of
+// +0: a masked score (minus infinity) gives an exact 0, as the special-function
+// unit does, and so does anything below 2^-127.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261113f, c3 = 0.05517167f;
+  x = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(f, make_float2(c3, c3), make_float2(c2, c2));
+  p = ffma2(p, f, make_float2(c1, c1));
+  p = ffma2(p, f, make_float2(c0, c0));
+  // t's bits are 0x4B400000 + n, which shifted by 23 leave n << 23 (mod 2^32):
+  // 2^n's bits are (n + 127) << 23, zero for n = -127
+  const float2 e2 = make_float2(__uint_as_float((__float_as_uint(t.x) << 23) + (127u << 23)),
+                                __uint_as_float((__float_as_uint(t.y) << 23) + (127u << 23)));
+  return make_float2(p.x * e2.x, p.y * e2.y);
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -578,13 +603,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // P as bf16 (decoder: fp16) pairs, keys 2c, 2c+1 in column c, stored into the
         // tile's P columns of TMEM once the previous P V has completed
         uint32_t pk[64];
+        // head_dim 32: the pairs c with bit c % 8 of POLY_PAIRS set (one in eight)
+        // are exponentiated on the FMA pipe, so the two tiles' warps, which
+        // exponentiate at the same time, queue less on the special-function unit
+        // (measured: one pair in eight -2.5 % decoder attention on the ragged
+        // workload; two or three in eight were slower than none).
+        // The choice follows the key's column alone, so a score gets the same P
+        // whatever rows share its warp (appending equals re-encoding bit for bit).
+        constexpr unsigned POLY_PAIRS = HD <= 32 ? 0x80u : 0u;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int e = 2 * c;
           const float2 x = ffma2(make_float2(s[e], s[e + 1]), scale2, neg_m2);
-          const float p0 = exp2_approx(x.x), p1 = exp2_approx(x.y);
-          sum2[c & 1] = fadd2(sum2[c & 1], make_float2(p0, p1));
-          pk[c] = DEC ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+          const float2 p = (POLY_PAIRS >> (c & 7)) & 1u ? exp2_fma2(x)
+                                                         : make_float2(exp2_approx(x.x), exp2_approx(x.y));
+          sum2[c & 1] = fadd2(sum2[c & 1], p);
+          pk[c] = DEC ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
         }
         if (TURNS) {
           __syncwarp();
