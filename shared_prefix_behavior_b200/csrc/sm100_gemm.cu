@@ -506,8 +506,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int j = (side_issued > 2 ? side_issued - 2 : 0); j < side_issued; ++j)
         mbar_wait(&side_full[j & 1], (j >> 1) & 1, nullptr, &no_abort);
     }
-  } else if (warp == 1 && lane == 0 && rank == 0) {
+  } else if (warp == 1 && rank == 0) {
     // ------------------------------------------------ MMA issuer (rank 0 only)
+    // The whole warp runs the loop and one elected lane issues: a lone lane of a
+    // diverged warp took about 160 cycles per N = 256 pair MMA, a whole warp about
+    // 127, against about 128 of tensor work per SM (measured).
     int it = 0, i = 0;
     bool ok = true;
     for (int tile = pair; tile < n_tiles && ok; tile += n_pairs, ++i) {
@@ -529,13 +532,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
           // B: N-major, 128B swizzle; 8-row K groups 1024 B apart, 64-column boxes 8 KB apart
           const uint64_t bd = smem_desc(b_base + k * 2048, BOX_B_BYTES, 1024, 2);
-          mma_bf16_pair(acc, ad, bd, idesc, (kb | k) != 0);
+          mma_bf16_pair_e(acc, ad, bd, idesc, (kb | k) != 0);
         }
-        mma_commit_pair(&empty[s]);
+        mma_commit_pair_e(&empty[s]);
       }
-      if (ok) mma_commit_pair(&acc_full[b]);
+      if (ok) mma_commit_pair_e(&acc_full[b]);
     }
-    mma_commit_pair(&drain);
+    mma_commit_pair_e(&drain);
     volatile int no_abort = 0;
     mbar_wait(&drain, 0, nullptr, &no_abort);
   } else if (warp >= 2 && warp < 10) {
