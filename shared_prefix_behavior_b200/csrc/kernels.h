@@ -47,9 +47,11 @@ cudaError_t launch_layernorm(bool bf16, float* x, void* y, const float* g, const
                              int mode, cudaStream_t s, const float* g2 = nullptr, const float* b2 = nullptr);
 // Decoder block input: a = z + y (fp32, into f) and u = dt(LN_k(a)) with the
 // parameters of token type k = row % K (ln_g, ln_b are [K, d]); in bf16 with
-// u_lo also the low part, u_lo = bf16(LN_k(a) - u). One warp per row.
+// u_lo also the low part, u_lo = bf16(LN_k(a) - u); with u16, u in fp16 instead
+// (a value beyond fp16's range sets REST_ERR_RANGE in err). One warp per row.
 cudaError_t launch_score_ln(bool bf16, const void* z, const float* y, float* f, void* u, void* u_lo,
-                            const float* ln_g, const float* ln_b, long long rows, int d, int K, cudaStream_t s);
+                            const float* ln_g, const float* ln_b, long long rows, int d, int K, cudaStream_t s,
+                            bool u16 = false, int32_t* err = nullptr);
 // score[n] = f[n, 0, :] . w_s + b_s; one warp per candidate.
 cudaError_t launch_score_readout(const float* f, const float* w_s, float b_s, float* score, long long n, int d, int K,
                                  cudaStream_t s);
@@ -104,6 +106,9 @@ struct GemmArgs {
   // output width (d_ff, resp. N). 0 or 1: one product.
   int groups;
   int gate_mode;                  // EPI_QKVG: a GateMode
+  // A and B are fp16 (kind::f16 with fp16 operands); EPI_SWIGLU then writes out0
+  // in fp16, and a value beyond fp16's range sets REST_ERR_RANGE
+  int f16;
 };
 // Logical output columns of EPI_QKVG are [Q | K | V,Gv interleaved | Go]
 // (GATES_O: [Q | K | V | Go]; GATES_QKVO: [Q,Gq | K,Gk | V,Gv interleaved | Go])

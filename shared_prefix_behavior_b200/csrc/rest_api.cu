@@ -632,6 +632,7 @@ static double gemm_out_bytes(const GemmArgs& a, size_t e) {
 
 static rest_status run_gemm(const Plan& p, const GemmArgs& a, const char* name, cudaStream_t s) {
   const bool bf = p.dt == REST_BF16;
+  if (a.f16 && !(bf && sm100_gemm_supported(a))) return REST_ERR_UNSUPPORTED;  // fp16 products: tensor cores only
   const size_t e = dt_size(p.dt);
   const double groups = a.epi == EPI_DECQG ? 2.0 * a.k_tok : a.groups > 1 ? (double)a.groups : 1.0;
   const double flops = 2.0 * a.M * a.N * a.K * groups;
@@ -1236,12 +1237,17 @@ rest_status rest_rank_request(rest_dtype dt, const rest_heads* heads, const rest
 
 // ---------------------------------------------------------------- decoder block and score
 
-// Workspace of the score head: the LN output u and the SwiGLU hidden state,
-// each with a low part in bf16 (u = u + u_lo, hid = hid + hid_lo feed the
-// tensor-core products at fp32-level precision: the block has no residual
-// scale to damp their rounding).
+// Workspace of the score head: the LN output u and the SwiGLU hidden state.
+// The block has no residual scale to damp their rounding, so they do not enter
+// its products as plain bf16. In bf16 with d a multiple of 128 and d_ff of 64
+// (the tensor-core GEMMs' shapes) the products run in fp16 (kind::f16 with fp16
+// operands): u and the hidden state in fp16, 8 times finer than bf16, and fp16
+// copies of the token-specific weights made each call (exact within fp16's
+// range). Otherwise (bf16) u = u + u_lo and hid = hid + hid_lo, each with a bf16
+// low part, feed two passes of the products at fp32-level precision.
 struct ScoreLayout {
-  size_t u, u_lo, hid, hid_lo, total;
+  size_t u, u_lo, hid, hid_lo, w13, w2, total;
+  bool f16;
 };
 
 static rest_status score_layout(rest_dtype dt, int d, int K, long long n, int d_ff, ScoreLayout* L) {
@@ -1250,12 +1256,15 @@ static rest_status score_layout(rest_dtype dt, int d, int K, long long n, int d_
     return REST_ERR_INVALID_ARG;
   const size_t e = dt_size(dt), rows = (size_t)n * K;
   const size_t ub = align_up(rows * d * e, 256), hb = align_up(rows * (size_t)d_ff * e, 256);
-  const bool lo = dt == REST_BF16;
+  L->f16 = dt == REST_BF16 && d % 128 == 0 && d_ff % 64 == 0;
+  const bool lo = dt == REST_BF16 && !L->f16;
   L->u = 0;
   L->u_lo = ub;
   L->hid = L->u_lo + (lo ? ub : 0);
   L->hid_lo = L->hid + hb;
-  L->total = L->hid_lo + (lo ? hb : 0);
+  L->w13 = L->hid_lo + (lo ? hb : 0);
+  L->w2 = L->w13 + (L->f16 ? align_up((size_t)K * d * 2 * d_ff * 2, 256) : 0);
+  L->total = L->w2 + (L->f16 ? align_up((size_t)K * d_ff * d * 2, 256) : 0);
   if (L->total == 0) L->total = 256;
   return REST_OK;
 }
@@ -1289,25 +1298,37 @@ rest_status rest_score_head(rest_dtype dt, int d, int K, long long n_cands, cons
     p.dt = dt;
     p.err = dev_err;
     const bool bf = dt == REST_BF16;
+    const bool f16 = SL.f16;  // the products in fp16
     const size_t e = dt_size(dt);
     const long long rows = n_cands * K;
     const int dff = sp->d_ff;
     char* u = at<char>(ws, SL.u);
-    char* u_lo = bf ? at<char>(ws, SL.u_lo) : nullptr;
+    char* u_lo = bf && !f16 ? at<char>(ws, SL.u_lo) : nullptr;
     char* hid = at<char>(ws, SL.hid);
-    char* hid_lo = bf ? at<char>(ws, SL.hid_lo) : nullptr;
+    char* hid_lo = bf && !f16 ? at<char>(ws, SL.hid_lo) : nullptr;
+    const void* w13 = sp->w_ffn13;
+    const void* w2 = sp->w_ffn2;
+    if (f16) {  // fp16 copies of the token-specific weights
+      w13 = at<void>(ws, SL.w13);
+      w2 = at<void>(ws, SL.w2);
+      REST_KLAUNCH(s, "score_w_f16", 0, 4.0 * K * d * 2 * dff,
+                   launch_bf16_to_f16(sp->w_ffn13, at<void>(ws, SL.w13), (long long)K * d * 2 * dff, dev_err, s));
+      REST_KLAUNCH(s, "score_w_f16", 0, 4.0 * K * dff * d,
+                   launch_bf16_to_f16(sp->w_ffn2, at<void>(ws, SL.w2), (long long)K * dff * d, dev_err, s));
+    }
     // a = z + y (the query token's residual, fp32 in f_out) and u = LN_k(a)
-    REST_KLAUNCH(s, "score_ln", 0, (double)rows * d * (e + 4 + 4 + 2 * e),
-                 launch_score_ln(bf, z, y, f_out, u, u_lo, sp->ln_g, sp->ln_b, rows, d, K, s));
+    REST_KLAUNCH(s, "score_ln", 0, (double)rows * d * (e + 4 + 4 + (f16 ? 2 : 2 * e)),
+                 launch_score_ln(bf, z, y, f_out, u, u_lo, sp->ln_g, sp->ln_b, rows, d, K, s, f16, dev_err));
     // token type k: columns [k d, k d + d) of u and f_out and [k d_ff, k d_ff + d_ff) of the
     // hidden state (rows n K + k of the [n K, d] views), with that type's weights (eq. 8). The
     // tensor-core GEMM takes all token types in one grouped launch; otherwise one launch each.
     auto ffn13 = [&](int k) {
       GemmArgs a = gemm(u + e * (size_t)k * d, (long long)K * d,
-                        (const char*)sp->w_ffn13 + e * (size_t)k * d * 2 * dff, 2LL * dff, n_cands, 2 * dff, d,
+                        (const char*)w13 + e * (size_t)k * d * 2 * dff, 2LL * dff, n_cands, 2 * dff, d,
                         EPI_SWIGLU, hid + e * (size_t)k * dff, (long long)K * dff);
       a.d = dff;
-      if (bf) {
+      a.f16 = f16;
+      if (bf && !f16) {
         a.A2 = u_lo + e * (size_t)k * d;
         a.out1 = hid_lo + e * (size_t)k * dff;
       }
@@ -1315,10 +1336,11 @@ rest_status rest_score_head(rest_dtype dt, int d, int K, long long n_cands, cons
     };
     auto ffn2 = [&](int k) {
       GemmArgs a = gemm(hid + e * (size_t)k * dff, (long long)K * dff,
-                        (const char*)sp->w_ffn2 + e * (size_t)k * dff * d, d, n_cands, d, dff, EPI_RESID,
+                        (const char*)w2 + e * (size_t)k * dff * d, d, n_cands, d, dff, EPI_RESID,
                         f_out + (size_t)k * d, (long long)K * d);
       a.alpha = 1.0f;
-      if (bf) a.A2 = hid_lo + e * (size_t)k * dff;
+      a.f16 = f16;
+      if (bf && !f16) a.A2 = hid_lo + e * (size_t)k * dff;
       return a;
     };
     for (int stage = 0; stage < 2; ++stage) {

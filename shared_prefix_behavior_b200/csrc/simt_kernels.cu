@@ -379,13 +379,14 @@ cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, cons
 // Decoder block and candidate score (ReST §3.3.2 eq. 8, Fig. 1 right)
 // ============================================================================
 
-// a = z + y into f; u = dt(LN_k(a)) with token type k = row % K. One warp per
-// row; lane holds columns 128 i + 4 lane .. + 3 (d a multiple of 128, NV = d / 128)
-// or, for other widths, columns lane, lane + 32, ... (NV = 0).
-template <typename T, int NV>
+// a = z + y into f; u = dt(LN_k(a)) with token type k = row % K (U16: u in
+// fp16, for an fp16 product; a value beyond fp16's range sets REST_ERR_RANGE).
+// One warp per row; lane holds columns 128 i + 4 lane .. + 3 (d a multiple of
+// 128, NV = d / 128) or, for other widths, columns lane, lane + 32, ... (NV = 0).
+template <typename T, int NV, bool U16 = false>
 __global__ void score_ln_kernel(const T* __restrict__ z, const float* __restrict__ y, float* __restrict__ f,
                                 T* __restrict__ u, T* __restrict__ u_lo, const float* __restrict__ ln_g,
-                                const float* __restrict__ ln_b, long long rows, int d, int K) {
+                                const float* __restrict__ ln_b, long long rows, int d, int K, int32_t* err) {
   pdl_wait();  // the previous kernel of the stream has completed
   pdl_release();
   constexpr int VN = NV > 0 ? 4 * NV : 32;  // values per lane
@@ -432,7 +433,24 @@ __global__ void score_ln_kernel(const T* __restrict__ z, const float* __restrict
   const float rstd = 1.0f / sqrtf(sq / d + 1e-5f);
   const float* g = ln_g + (long long)k * d;
   const float* b = ln_b + (long long)k * d;
-  if (NV > 0) {
+  if (NV > 0 && U16) {
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 128 * i + 4 * lane;
+      float gg[4], bb[4], n[4];
+      load4(g + c, gg);
+      load4(b + c, bb);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        n[e] = (v[4 * i + e] - mean) * rstd * gg[e] + bb[e];
+        ok = ok && fits_f16(n[e]);
+      }
+      *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(u) + o + c) =
+          make_uint2(pack_f16x2(n[0], n[1]), pack_f16x2(n[2], n[3]));
+    }
+    if (!ok) set_error(err, REST_ERR_RANGE);
+  } else if (NV > 0) {
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = 128 * i + 4 * lane;
@@ -462,29 +480,34 @@ __global__ void score_ln_kernel(const T* __restrict__ z, const float* __restrict
   }
 }
 
-template <typename T>
+template <typename T, bool U16 = false>
 static cudaError_t score_ln_dispatch(const T* z, const float* y, float* f, T* u, T* u_lo, const float* ln_g,
-                                    const float* ln_b, long long rows, int d, int K, cudaStream_t s) {
+                                    const float* ln_b, long long rows, int d, int K, cudaStream_t s, int32_t* err) {
   const int threads = 256;
   const long long blocks = (rows * 32 + threads - 1) / threads;
   const unsigned nb = (unsigned)blocks;
   switch (d % 128 == 0 ? d / 128 : 0) {
-    case 1: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 1>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
-    case 2: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 2>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
-    case 4: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 4>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
-    case 8: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 8>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
-    default: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 0>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K)) return e_; break;
+    case 1: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 1, U16>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K, err)) return e_; break;
+    case 2: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 2, U16>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K, err)) return e_; break;
+    case 4: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 4, U16>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K, err)) return e_; break;
+    case 8: if (cudaError_t e_ = launch_k(score_ln_kernel<T, 8, U16>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K, err)) return e_; break;
+    default:
+      if (U16) return cudaErrorInvalidValue;  // the fp16 output takes d a multiple of 128
+      if (cudaError_t e_ = launch_k(score_ln_kernel<T, 0>, nb, threads, 0, s, z, y, f, u, u_lo, ln_g, ln_b, rows, d, K, err)) return e_; break;
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_score_ln(bool bf16m, const void* z, const float* y, float* f, void* u, void* u_lo,
-                            const float* ln_g, const float* ln_b, long long rows, int d, int K, cudaStream_t s) {
+                            const float* ln_g, const float* ln_b, long long rows, int d, int K, cudaStream_t s,
+                            bool u16, int32_t* err) {
   if (rows == 0) return cudaSuccess;
   if (d > 1024 || K < 1) return cudaErrorInvalidValue;
+  if (bf16m && u16)
+    return score_ln_dispatch<bf16, true>((const bf16*)z, y, f, (bf16*)u, nullptr, ln_g, ln_b, rows, d, K, s, err);
   if (bf16m)
-    return score_ln_dispatch<bf16>((const bf16*)z, y, f, (bf16*)u, (bf16*)u_lo, ln_g, ln_b, rows, d, K, s);
-  return score_ln_dispatch<float>((const float*)z, y, f, (float*)u, nullptr, ln_g, ln_b, rows, d, K, s);
+    return score_ln_dispatch<bf16>((const bf16*)z, y, f, (bf16*)u, (bf16*)u_lo, ln_g, ln_b, rows, d, K, s, err);
+  return score_ln_dispatch<float>((const float*)z, y, f, (float*)u, nullptr, ln_g, ln_b, rows, d, K, s, err);
 }
 
 // score[n] = f[n, 0, :] . w_s + b_s (token 0 is [CLS]); one warp per candidate.

@@ -379,6 +379,10 @@ __device__ __forceinline__ void mma_commit_e(uint64_t* bar) {
 __host__ __device__ constexpr uint32_t idesc_bf16_pair(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
+// The same for fp16 A and B.
+__host__ __device__ constexpr uint32_t idesc_f16_pair(int n) {
+  return idesc_bf16_pair(n) & ~((7u << 7) | (7u << 10));
+}
 __device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                               uint32_t accumulate) {
   asm volatile(

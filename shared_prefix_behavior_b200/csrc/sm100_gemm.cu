@@ -162,6 +162,24 @@ __device__ __forceinline__ void stage_bf16_sw128(uint8_t* box, int r, int k0, co
   }
 }
 
+// 32 values as fp16 into half (chunks k0..k0+3) of a 128-byte row of a
+// 128B-swizzled box; false if one is beyond fp16's range
+__device__ __forceinline__ bool stage_f16_sw128(uint8_t* box, int r, int k0, const float (&v)[32]) {
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint4 u;
+    u.x = pack_f16x2(v[8 * k], v[8 * k + 1]);
+    u.y = pack_f16x2(v[8 * k + 2], v[8 * k + 3]);
+    u.z = pack_f16x2(v[8 * k + 4], v[8 * k + 5]);
+    u.w = pack_f16x2(v[8 * k + 6], v[8 * k + 7]);
+    *reinterpret_cast<uint4*>(box + sw128_off(r, k0 + k)) = u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ok = ok && fits_f16(v[8 * k + i]);
+  }
+  return ok;
+}
+
 // Q and K columns of four rotation pairs (ReST eq. 5): outputs 8 bf16 each.
 __device__ __forceinline__ uint4 rotate4(const float* p, float4 c, float4 s) {
   uint4 u;
@@ -181,7 +199,7 @@ __device__ __forceinline__ uint4 rotate4(const float* p, float4 c, float4 s) {
 // the previous tile have left the slot.
 template <bool SIDE, int NSLOT>
 __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, uint32_t trow, uint8_t* slot, int t,
-                                         int m0, int q, int lane, int part, uint32_t acc_empty_addr) {
+                                         int m0, int q, int lane, int part, uint32_t acc_empty_addr, int32_t* err) {
   const int r = q * 32 + lane;
   const int y0 = m0 + q * 32;
   float v[32], w[32];
@@ -298,7 +316,11 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
         for (int i = 0; i < 32; ++i) v[i] = v[i] * sigmoid_fast(v[i]) * w[i];
       }
       if (j == 0) slot_ready();
-      stage_bf16_sw128(box, r, 4 * j, v);
+      if (!SIDE && a.f16) {  // the hidden state for an fp16 product
+        if (!stage_f16_sw128(box, r, 4 * j, v)) set_error(err, REST_ERR_RANGE);
+      } else {
+        stage_bf16_sw128(box, r, 4 * j, v);
+      }
       if (lo) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) w[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
@@ -514,7 +536,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int it = 0, i = 0;
     bool ok = true;
     for (int tile = pair; tile < n_tiles && ok; tile += n_pairs, ++i) {
-      const uint32_t idesc = idesc_bf16_pair(tile_n(a));
+      const uint32_t idesc = a.f16 ? idesc_f16_pair(tile_n(a)) : idesc_bf16_pair(tile_n(a));
       const int b = i & 1;
       // both CTAs' epilogues have drained this accumulator (tile i-2)
       if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, err, &abort_flag)) { ok = false; break; }
@@ -563,7 +585,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&acc_full[b], (i >> 1) & 1, err, &abort_flag)) break;
       tc_fence_after();
       epilogue<SIDE, NSLOT>(a, mp, tmem + b * ACC_COLS + lane_off, slots + (i % NSLOT) * SLOT, t, m0, q, lane, part,
-                            acc_empty0[b]);
+                            acc_empty0[b], err);
     }
     if (lane == 0) bulk_wait<0>();  // every store has completed before the CTA's shared memory goes away
   }
@@ -721,6 +743,7 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long 
 
 bool sm100_gemm_supported(const GemmArgs& a) {
   if (a.a_f32) return false;
+  if (a.f16 && (a.A2 || a.out1 || (a.epi != EPI_SWIGLU && a.epi != EPI_RESID))) return false;
   if (a.M <= 0 || a.K % BK != 0 || a.K <= 0) return false;
   if ((a.lda % 8) || (a.ldb % 8) || (a.ldo % 8)) return false;
   switch (a.epi) {
