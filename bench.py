@@ -60,12 +60,10 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("enc_attn", "bf16-32x1024-d256-4L-N128"): (90079744, "attn", "233aab49b12b7c9e",
-                                                "profiles/attn_tc_kernel_bf16-32x1024-d256.md"),
-    ("enc_attn", "bf16-8x4096-d512-2L-N256-dup5"): (271378176, "attn", "233aab49b12b7c9e",
-                                                    "profiles/attn_tc_kernel_bf16-8x4096-d512.md"),
-    ("enc_attn", "bf16-2x16384-d512-1L-N512-1y"): (296346368, "attn", "233aab49b12b7c9e",
-                                                   "profiles/attn_tc_kernel_bf16-2x16384-d512.md"),
+    ("dec_attn", "bf16-ragged64-d256"): (935722240, "attn", "044212b94c5e3b4b",
+                                         "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
+    ("enc_attn", "bf16-ragged64-d256"): (984920320, "attn", "044212b94c5e3b4b",
+                                         "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
 }
 
 
@@ -109,6 +107,9 @@ def parse():
                     help="also time the encoder under the gated-attention and RoTE ablation variants")
     ap.add_argument("--sharing", action="store_true",
                     help="also run the no-sharing variant (every candidate re-encodes its own history)")
+    ap.add_argument("--core-only", action="store_true",
+                    help="the step, its per-kernel pass, e2e and the two halves alone; no append, training or "
+                         "CPU baseline (for profiler runs)")
     return ap.parse_args()
 
 
@@ -854,11 +855,11 @@ def main():
     parts = component_timings(args, w, t, H, Y, ws, dev, peaks_for_parts())
     if args.sharing and world == 1:
         parts["sharing"] = sharing_comparison(w, inp, dev, ms_step)
-    if world == 1:
+    if world == 1 and not args.core_only:
         parts["append"] = append_comparison(w, inp, dev, parts["encoder_only"]["ms"])
     if args.ablation and world == 1:
         parts["ablation"] = ablation_comparison(w, dev)
-    if world == 1:
+    if world == 1 and not args.core_only:
         parts["training"] = training_comparison(w, inp, dev)
 
     if world > 1:
@@ -936,7 +937,7 @@ def main():
     for k in ("sharing", "append", "ablation", "training"):
         if k in parts:
             out[k] = parts[k]
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.core_only:
         out["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_budget)
     print(json.dumps(out), flush=True)
 
