@@ -109,6 +109,10 @@ struct GemmArgs {
   // A and B are fp16 (kind::f16 with fp16 operands); EPI_SWIGLU then writes out0
   // in fp16, and a value beyond fp16's range sets REST_ERR_RANGE
   int f16;
+  // EPI_DECQG (bf16 A and B): q * alpha and sigmoid(g) written in fp16 (for the
+  // tensor-core decoder's fp16 products; a value beyond fp16's range sets
+  // REST_ERR_RANGE)
+  int out16;
 };
 // Logical output columns of EPI_QKVG are [Q | K | V,Gv interleaved | Go]
 // (GATES_O: [Q | K | V | Go]; GATES_QKVO: [Q,Gq | K,Gk | V,Gv interleaved | Go])
@@ -175,19 +179,22 @@ struct AttnBwdArgs {
 cudaError_t launch_attn_bwd_simt(bool bf16, int hd, int part, const AttnBwdArgs& a, cudaStream_t s);
 
 struct DecAttnArgs {
-  const float* q;      // [NK, d] decoder queries (fp32)
-  const float* g;      // [NK, d] sigmoid output gate
+  const float* q;      // [NK, d] decoder queries (fp32; CUDA-core decoder)
+  const float* g;      // [NK, d] sigmoid output gate (fp32; CUDA-core decoder)
+  // the tensor-core decoder's query rows, scaled by log2(e) / sqrt(head_dim), and
+  // output gate, [NK, d] fp16 each
+  const void* q16; const void* g16;
   const void* h;       // [T, d] encoder memory: keys and values (the tensor-core decoder: fp16)
   const void* h_lo;    // [T, d] bf16 low part of H (H = h + h_lo), or null (CUDA-core decoder)
-  void* out;           // [NK, d] o * g: fp32, or its bf16 high part when out_lo is set
-  void* out_lo;        // [NK, d] bf16 low part of o * g, or null
+  void* out;           // [NK, d] o * g: fp32 (CUDA-core decoder) or fp16 (tensor-core decoder)
+  void* out_lo;        // unused (null)
   const DecTile* tiles; int n_tiles;
   int n_heads, d;
   float scale_log2;
   long long key_rows;  // T, rows of h
   // split keys (n_split > 1): per split, the unnormalized O [NK, d] and the
   // reference max m (log2 domain) and sum l [NK, n_heads, 2]; combined by
-  // launch_dec_combine into out.
+  // launch_dec_combine into out (tensor-core decoder: fp16, with the fp16 gate).
   int n_split;
   long long nk_rows;   // NK
   float* part_o;

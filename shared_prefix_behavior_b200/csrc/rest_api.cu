@@ -325,7 +325,7 @@ static std::vector<int> dec_schedule(const std::vector<DecTile>& tiles, int n_he
 struct Layout {
   size_t cu, enc_tiles, dec_tiles, enc_sched, dec_sched, app, bwd_tiles, bwd_sched, meta_end;
   size_t cos_t, sin_t, xres, y, q, k, v, g, o, hid;
-  size_t dq, dg, dout, hx, part_o, part_ml, delta;
+  size_t dq, dg, dout, hx, wo16, part_o, part_ml, delta;
   size_t total;
   int n_enc_tiles, n_dec_tiles, n_bwd_tiles;
 };
@@ -364,8 +364,10 @@ static Layout make_layout(rest_dtype dt, const rest_heads* hs, const rest_batch*
   L.dq = take(4 * (size_t)NK * d);
   L.dg = take(4 * (size_t)NK * d);
   L.dout = take(4 * (size_t)NK * d);
-  // H_lo for the CUDA-core decoder, or the fp16 H of the tensor-core decoder
+  // H_lo for the CUDA-core decoder, or the fp16 H of the tensor-core decoder and
+  // its fp16 copy of W_o
   L.hx = take(hx ? 2 * (size_t)T * d : 0);
+  L.wo16 = take(hx ? 2 * d * d : 0);
   // split partial results: the decoder's [n_split, NK] or the appending encoder's [n_split_enc, T] rows
   const size_t part_rows = std::max(n_split > 1 ? (size_t)n_split * NK : 0,
                                     n_split_enc > 1 ? (size_t)n_split_enc * T : 0);
@@ -625,7 +627,7 @@ static double gemm_out_bytes(const GemmArgs& a, size_t e) {
     case EPI_RESID: return 8 * MN;
     case EPI_QKVG: return (double)a.M * a.d * (3 * e + 4) + 4.0 * a.M * a.d;  // + cos/sin reads
     case EPI_SWIGLU: return e * MN / 2;
-    case EPI_DECQG: return 8.0 * a.k_tok * MN;  // q and g, fp32, for every token type
+    case EPI_DECQG: return (a.out16 ? 4.0 : 8.0) * a.k_tok * MN;  // q and g (fp16 or fp32), every token type
   }
   return 0;
 }
@@ -824,14 +826,23 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   float* dg = at<float>(ws, L.dg);
   float* dout = at<float>(ws, L.dout);
   const long long N = p.n_cands;
+  const bool tc = bf && sm100_attn_supported(hd);
   // token-specific projections (eq. 8): rows n*K + k use W_Q^(k), W_go^(k);
-  // the tensor-core GEMM does all token types and both weights in one launch
+  // the tensor-core GEMM does all token types and both weights in one launch. For
+  // the tensor-core decoder it writes q, already scaled by log2(e) / sqrt(d_h),
+  // and the gate in fp16 (in the fp32 buffers' bytes).
   GemmArgs qg = gemm(z, (long long)K * d, dec->w_q, d, N, d, d, EPI_DECQG, dq, (long long)K * d);
   qg.out1 = dg;
   qg.B2 = dec->w_go;
   qg.k_tok = K;
+  if (tc) {
+    qg.out16 = 1;
+    qg.alpha = (float)(1.4426950408889634 / sqrt((double)hd));
+  }
   if (bf && sm100_gemm_supported(qg)) {
     if (rest_status st = run_gemm(p, qg, "gemm_dec_qg", s)) return st;
+  } else if (tc) {
+    return REST_ERR_UNSUPPORTED;  // the fp16 queries come from the tensor-core projection only
   } else
   for (int kk = 0; kk < K; ++kk) {
     const char* zk = (const char*)z + e * (size_t)kk * d;
@@ -844,7 +855,6 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   }
   // The tensor-core decoder multiplies in fp16 (H, q and P): its H is the fp16
   // copy in the workspace, converted here unless the encoder wrote it.
-  const bool tc = bf && sm100_attn_supported(hd);
   const void* h_lo = !tc && from_encoder && p.hsplit ? at<void>(ws, L.hx) : nullptr;
   if (tc) {
     if (!from_encoder)
@@ -859,13 +869,14 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
     flops += 4.0 * d * rows * reqs->req_cutoff[r];
     hbytes += (double)e * reqs->req_cutoff[r] * d * (h_lo ? 2 : 1);
   }
-  const double bytes = hbytes + (double)p.NK * d * 12;
-  // The tensor-core decoder hands o * g to the output projection as a hi + lo
-  // pair of bf16 arrays (in the same workspace bytes); the CUDA-core one as fp32.
+  // q and g in, o * g out: fp16 each for the tensor-core decoder, fp32 for the CUDA-core one
+  const double bytes = hbytes + (double)p.NK * d * (tc ? 6 : 12);
+  // The tensor-core decoder hands o * g to the output projection in fp16, the
+  // CUDA-core one in fp32.
   DecAttnArgs da;
   memset(&da, 0, sizeof(da));
   da.q = dq; da.g = dg; da.h = h; da.h_lo = h_lo; da.out = dout;
-  da.out_lo = tc ? (void*)((bf16*)dout + (size_t)p.NK * d) : nullptr;
+  da.q16 = dq; da.g16 = dg;
   da.tiles = at<DecTile>(ws, L.dec_tiles); da.n_tiles = L.n_dec_tiles;
 
   da.n_heads = p.hs->n_heads; da.d = d;
@@ -885,9 +896,16 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
   } else {
     REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_simt(bf, hd, da, s));
   }
-  GemmArgs a = gemm(dout, d, dec->w_o, d, p.NK, d, d, EPI_F32, y_out, d);
+  // y = (o * g) W_o: one fp16 product for the tensor-core decoder (W_o copied to
+  // fp16 per call), fp32 A otherwise
+  const void* wo = dec->w_o;
+  if (tc) {
+    REST_KLAUNCH(s, "w_o_f16", 0, 4.0 * d * d, launch_bf16_to_f16(dec->w_o, at<void>(ws, L.wo16), (long long)d * d, err, s));
+    wo = at<void>(ws, L.wo16);
+  }
+  GemmArgs a = gemm(dout, d, wo, d, p.NK, d, d, EPI_F32, y_out, d);
   if (tc)
-    a.A2 = da.out_lo;
+    a.f16 = 1;
   else
     a.a_f32 = 1;
   if (rest_status st = run_gemm(p, a, "gemm_dec_out", s)) return st;

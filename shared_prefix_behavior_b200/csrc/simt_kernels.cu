@@ -1092,8 +1092,9 @@ static cudaError_t dec_dispatch(int hd, const DecAttnArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// Split-key decoder: out = (sum_s 2^(m_s - M) O_s) / (sum_s 2^(m_s - M) l_s) * g,
-// M = max_s m_s; one thread per 4 output columns of a row.
+// Split-key decoder (after the tensor-core decoder): out = (sum_s 2^(m_s - M) O_s)
+// / (sum_s 2^(m_s - M) l_s) * g in fp16, g the fp16 gate, M = max_s m_s; one
+// thread per 4 output columns of a row.
 __global__ void dec_combine_kernel(DecAttnArgs a, int hd) {
   pdl_wait();  // the previous kernel of the stream has completed
   pdl_release();
@@ -1115,18 +1116,12 @@ __global__ void dec_combine_kernel(DecAttnArgs a, int hd) {
     load4(a.part_o + (s * a.nk_rows + row) * a.d + c, v);
     for (int i = 0; i < 4; ++i) o[i] = fmaf(w, v[i], o[i]);
   }
+  // the tensor-core decoder's gate and o * g are fp16
   float g[4];
-  load4(a.g + row * a.d + c, g);
+  load4_f16(static_cast<const __half*>(a.g16) + row * a.d + c, g);
   const float inv = 1.0f / L;
-  float r[4] = {o[0] * inv * g[0], o[1] * inv * g[1], o[2] * inv * g[2], o[3] * inv * g[3]};
-  if (a.out_lo) {  // as a hi + lo pair of bf16 values
-    float lo[4];
-    for (int i = 0; i < 4; ++i) lo[i] = r[i] - __bfloat162float(__float2bfloat16_rn(r[i]));
-    store4((bf16*)a.out + row * a.d + c, r);
-    store4((bf16*)a.out_lo + row * a.d + c, lo);
-  } else {
-    store4((float*)a.out + row * a.d + c, r);
-  }
+  *reinterpret_cast<uint2*>(static_cast<__half*>(a.out) + row * a.d + c) =
+      make_uint2(pack_f16x2(o[0] * inv * g[0], o[1] * inv * g[1]), pack_f16x2(o[2] * inv * g[2], o[3] * inv * g[3]));
 }
 
 cudaError_t launch_dec_combine(int hd, const DecAttnArgs& a, cudaStream_t s) {

@@ -88,19 +88,18 @@ struct SmemLayout {
   static constexpr int KV = NT * Cfg<HD>::TILE_BYTES;
   // a stage holds K and V' (encoder) or H (decoder)
   static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
-  // per softmax warp, its 32 output rows in bf16 (rows padded by 16 bytes): the
-  // encoder's O, or the decoder's o * g as its hi and lo halves side by side
+  // per softmax warp, its 32 output rows in 2-byte values (rows padded by 16
+  // bytes): the encoder's O (bf16) or the decoder's o * g (fp16)
   static constexpr bool DEC = MODE == 1;
-  static constexpr int STG_ROW = (DEC ? 2 : 1) * HD * 2 + 16;
+  static constexpr int STG_ROW = HD * 2 + 16;
   static constexpr int STG = KV + STAGES * STAGE;
   static constexpr bool STAGED_OUT = MODE == 0 || (DEC && HD <= 32);
-  // head_dim 32: every softmax thread's fp32 rows fetched ahead by cp.async, the
-  // item's output gate row (and, decoding, the next item's query row), rows
-  // padded by 16 bytes: [gate rows of 256 threads | query rows of 256 threads]
+  // head_dim 32: every softmax thread's output-gate row (fp32; decoding fp16)
+  // fetched ahead by cp.async, rows padded by 16 bytes
   static constexpr bool PREFETCH = HD <= 32 && MODE != 3;
-  static constexpr int PF_ROW = HD * 4 + 16;
+  static constexpr int PF_ROW = HD * (DEC ? 2 : 4) + 16;
   static constexpr int PF = STG + (STAGED_OUT ? 8 * 32 * STG_ROW : 0);
-  static constexpr int TOTAL = PF + (PREFETCH ? (DEC ? 2 : 1) * 256 * PF_ROW : 0);
+  static constexpr int TOTAL = PF + (PREFETCH ? 256 * PF_ROW : 0);
 };
 
 // Asynchronous 16-byte copies global -> shared memory (no TMA): a thread
@@ -263,7 +262,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < NT; ++t) {
-      mbar_init(&q_full[t], DEC ? 128 : 1);
+      mbar_init(&q_full[t], 1);
       mbar_init(&q_empty[t], 1);
       mbar_init(&s_full[t], 1);
       mbar_init(&s_free[t], 128);
@@ -320,14 +319,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool ok = true;
       for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
         const AttnItem w = item_at(k);
-        if (!DEC) {
-          for (int t = 0; t < NT && ok; ++t) {
-            if (w.nblk[t] == 0) continue;
-            if (qn[t] >= 1 && !mbar_wait(&q_empty[t], (qn[t] - 1) & 1, err, &abort_flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
-            tma_load_2d(smem + L::Q + t * C::TILE_BYTES, &tmQ, w.h * HD, w.q_row0 + t * ROWS, &q_full[t]);
-            ++qn[t];
-          }
+        // the query tiles (decoding: fp16, scaled to the base-2 domain by the projection)
+        for (int t = 0; t < NT && ok; ++t) {
+          if (w.nblk[t] == 0) continue;
+          if (qn[t] >= 1 && !mbar_wait(&q_empty[t], (qn[t] - 1) & 1, err, &abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
+          tma_load_2d(smem + L::Q + t * C::TILE_BYTES, &tmQ, w.h * HD, w.q_row0 + t * ROWS, &q_full[t]);
+          ++qn[t];
         }
         const int nblk_all = max(w.nblk[0], w.nblk[1]);
         for (int j = 0; j < nblk_all && ok; ++j, ++g) {
@@ -342,8 +340,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (!ok) {  // let the copies in flight land before the CTA exits
         volatile int no_abort = 0;
-        if (!DEC)
-          for (int t = 0; t < NT; ++t)
+        for (int t = 0; t < NT; ++t)
             if (qn[t] >= 1) mbar_wait(&q_full[t], (qn[t] - 1) & 1, nullptr, &no_abort);
         for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
           mbar_wait(&kv_full[i % STAGES], (i / STAGES) & 1, nullptr, &no_abort);
@@ -440,19 +437,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float* const part_ml = DEC ? da.part_ml : ea.part_ml;
     const long long part_rows = DEC ? da.nk_rows : ea.rows;
     int cb = 0, qn = 0, cbo = 0;  // cbo: the other tile's key blocks in earlier items
-    // head_dim 32: this thread's fetched-ahead rows (see SmemLayout::PREFETCH)
+    // head_dim 32: this thread's output-gate row, fetched ahead (see SmemLayout::PREFETCH)
     const int tid = threadIdx.x - 128;
     uint8_t* const pf_gate = smem + L::PF + tid * L::PF_ROW;
-    uint8_t* const pf_q = smem + L::PF + (256 + tid) * L::PF_ROW;
-    // the query row of item k for this thread (row 0 of the tile for rows past its end)
-    auto q_src = [&](const AttnItem& x) {
-      return da.q + (long long)(x.q_row0 + t * ROWS + (r < x.nrow[t] ? r : 0)) * d + x.h * HD;
-    };
-    auto fetch_row = [&](uint8_t* dst, const float* src) {
-#pragma unroll
-      for (int u = 0; u < HD / 4; ++u) cp_async16(dst + 16 * u, src + 4 * u);
-    };
-    int q_fetched = -1;  // the item whose query row is (being) fetched into pf_q
+    constexpr int GATE_ES = DEC ? 2 : 4;  // the gate's element size: fp16 decoding, fp32 encoding
     bool ok = true;
     for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
       const AttnItem w = item_at(k);
@@ -470,57 +458,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           pml[0] = -INFINITY;
           pml[1] = 0.f;
         }
-        if (L::PREFETCH) cp_async_wait<0>();  // a query row fetched for this item lands before pf_q is reused
         cbo += w.nblk[1 - t];
         continue;
       }
-      if (DEC) {  // stage q (fp32) in fp16, scaled to the base-2 domain, in the swizzled K-major layout
-        if (qn >= 1 && !mbar_wait(&q_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
-        const float* qrow = q_src(w);
-        if (L::PREFETCH) {  // this item's row was fetched during the previous one, else now
-          if (q_fetched != k) {
-            fetch_row(pf_q, qrow);
-            cp_async_commit();
-          }
-          cp_async_wait<0>();
-          qrow = reinterpret_cast<const float*>(pf_q);
-        }
-        uint8_t* qh = smem + L::Q + t * C::TILE_BYTES;
-        const float qs = da.scale_log2;
-        bool in_range = true;
-#pragma unroll
-        for (int u = 0; u < HD / 8; ++u) {
-          float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-          if (valid) {
-            load4(qrow + 8 * u, v);
-            load4(qrow + 8 * u + 4, v + 4);
-          }
-          uint32_t hf[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = v[2 * e] * qs, b = v[2 * e + 1] * qs;
-            in_range = in_range && fits_f16(a) && fits_f16(b);
-            hf[e] = pack_f16x2(a, b);
-          }
-          *reinterpret_cast<uint4*>(qh + swz_off<HD>(r, u)) = make_uint4(hf[0], hf[1], hf[2], hf[3]);
-        }
-        if (!in_range) set_error(err, REST_ERR_RANGE);
-        fence_async_smem();
-        mbar_arrive(&q_full[t]);
-      }
       const long long ro = row_g * d + h * HD;
       const bool has_gate = DEC || ea.gate != nullptr;  // the encoder's gate may be left out (training core)
-      if (L::PREFETCH) {
-        // this item's output gate row (in flight through the item's key blocks), then,
-        // decoding, the next item's query row (once this item's is staged above)
-        if (valid && !split && has_gate) fetch_row(pf_gate, (DEC ? da.g : ea.gate) + ro);
-        cp_async_commit();
-        if (DEC && k + 1 < sched[blockIdx.x + 1]) {
-          const AttnItem nx = item_at(k + 1);
-          if (nx.nrow[t] > 0) {
-            fetch_row(pf_q, q_src(nx));
-            q_fetched = k + 1;
-          }
+      const uint8_t* const gate_src = DEC ? static_cast<const uint8_t*>(da.g16) : reinterpret_cast<const uint8_t*>(ea.gate);
+      if (L::PREFETCH) {  // this item's output gate row, in flight through the item's key blocks
+        if (valid && !split && has_gate) {
+#pragma unroll
+          for (int u = 0; u < HD * GATE_ES / 16; ++u) cp_async16(pf_gate + 16 * u, gate_src + ro * GATE_ES + 16 * u);
         }
         cp_async_commit();
       }
@@ -636,15 +583,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&p_full[t]);
       }
       if (!ok) break;
-      // the output gate of this row: fetched ahead into shared memory (head_dim 32;
-      // the group of this item's gate is the older of the two in flight), or
-      // loaded here (64: the row would not fit the softmax warps' registers next to O)
+      // the output gate of this row: fetched ahead into shared memory (head_dim 32),
+      // or loaded here (64: the row would not fit the softmax warps' registers next to O)
       constexpr bool GATE_ROW = L::PREFETCH;
       float gate_row[GATE_ROW ? HD : 4];
       if (GATE_ROW && valid && !split && has_gate) {
-        cp_async_wait<1>();
+        cp_async_wait<0>();
+        if (DEC) {
 #pragma unroll
-        for (int c = 0; c < HD; c += 4) load4(reinterpret_cast<const float*>(pf_gate) + c, &gate_row[c]);
+          for (int c = 0; c < HD; c += 8) load8_f16(reinterpret_cast<const __half*>(pf_gate) + c, &gate_row[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < HD; c += 4) load4(reinterpret_cast<const float*>(pf_gate) + c, &gate_row[c]);
+        }
       }
       if (!mbar_wait(&p_free[t], (cb + nb - 1) & 1, err, &abort_flag)) { ok = false; break; }  // the last P V
       tc_fence_after();
@@ -659,12 +610,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(&o_empty[t]);  // O_t may now be overwritten by the next item
-      if (L::STAGED_OUT && !split && (DEC ? da.out_lo != nullptr : ea.out_lo == nullptr)) {
-        // The output rows through shared memory: each lane writes its row's bf16
-        // values (decoding: o * g as hi and lo halves) into the warp's staging
-        // rows, then the warp stores them 16 bytes a lane, HD / 8 lanes to a row,
-        // so that a store instruction writes whole sectors of a few rows instead
-        // of 8 bytes of each of 32 rows.
+      if (L::STAGED_OUT && !split && (DEC || ea.out_lo == nullptr)) {
+        // The output rows through shared memory: each lane writes its row's 2-byte
+        // values (the encoder's O * gate in bf16, the decoder's o * g in fp16) into the
+        // warp's staging rows, then the warp stores them 16 bytes a lane, HD / 8 lanes
+        // to a row, so that a store instruction writes whole sectors of a few rows
+        // instead of 8 bytes of each of 32 rows.
         const float inv = valid ? 1.0f / l_run : 0.f;
         if (!DEC && valid && ea.lse) ea.lse[row_g * n_heads + h] = (m_ref + log2f(l_run)) * 0.69314718055994531f;
         uint8_t* stg = smem + L::STG + (warp - 4) * 32 * L::STG_ROW;
@@ -677,39 +628,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           } else if (GATE_ROW) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) gh[i] = gate_row[(c0 + i) % (GATE_ROW ? HD : 4)];
+          } else if (DEC) {
+            load8_f16(static_cast<const __half*>(da.g16) + ro + c0, gh);
           } else {
-            load4((DEC ? da.g : ea.gate) + ro + c0, gh);
-            load4((DEC ? da.g : ea.gate) + ro + c0 + 4, gh + 4);
+            load4(ea.gate + ro + c0, gh);
+            load4(ea.gate + ro + c0 + 4, gh + 4);
           }
-          uint32_t pk[4], pl[4];
+          uint32_t pk[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float v0 = o[c0 + 2 * i] * inv * gh[2 * i], v1 = o[c0 + 2 * i + 1] * inv * gh[2 * i + 1];
-            __nv_bfloat162 t2 = __floats2bfloat162_rn(v0, v1);
-            pk[i] = *reinterpret_cast<uint32_t*>(&t2);
-            if (DEC) {  // the low part: v - bf16(v)
-              const float2 hf = __bfloat1622float2(t2);
-              __nv_bfloat162 l2 = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
-              pl[i] = *reinterpret_cast<uint32_t*>(&l2);
-            }
+            pk[i] = DEC ? pack_f16x2(v0, v1) : pack_bf16x2(v0, v1);
           }
           *reinterpret_cast<uint4*>(stg + lane * L::STG_ROW + c0 * 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          if (DEC)
-            *reinterpret_cast<uint4*>(stg + lane * L::STG_ROW + HD * 2 + c0 * 2) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
         }
         __syncwarp();
-        constexpr int CPR = HD / 8;  // 16-byte chunks of a row (of each half)
+        constexpr int CPR = HD / 8;  // 16-byte chunks of a row
+        uint8_t* const dst = static_cast<uint8_t*>(DEC ? da.out : ea.out);
 #pragma unroll
-        for (int half = 0; half < (DEC ? 2 : 1); ++half) {
-          bf16* const dst = reinterpret_cast<bf16*>(half ? da.out_lo : DEC ? da.out : ea.out);
-#pragma unroll
-          for (int rr = 0; rr < 32; rr += 32 / CPR) {
-            const int r = rr + lane / CPR, ch = lane % CPR;
-            const int tr = q4 * 32 + r;  // row within the tile
-            if (tr < w.nrow[t]) {
-              const uint4 val = *reinterpret_cast<const uint4*>(stg + r * L::STG_ROW + half * HD * 2 + ch * 16);
-              *reinterpret_cast<uint4*>(dst + (long long)(w.q_row0 + t * ROWS + tr) * d + h * HD + ch * 8) = val;
-            }
+        for (int rr = 0; rr < 32; rr += 32 / CPR) {
+          const int r = rr + lane / CPR, ch = lane % CPR;
+          const int tr = q4 * 32 + r;  // row within the tile
+          if (tr < w.nrow[t]) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * L::STG_ROW + ch * 16);
+            *reinterpret_cast<uint4*>(dst + ((long long)(w.q_row0 + t * ROWS + tr) * d + h * HD + ch * 8) * 2) = val;
           }
         }
         __syncwarp();  // the staging rows are free for the next item
@@ -735,8 +677,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             } else if (GATE_ROW) {
 #pragma unroll
               for (int i = 0; i < 4; ++i) gh[c + i] = gate_row[(c0 + c + i) % (GATE_ROW ? HD : 4)];
+            } else if (DEC) {
+              load4_f16(static_cast<const __half*>(da.g16) + ro + c0 + c, &gh[c]);
             } else {
-              load4((DEC ? da.g : ea.gate) + ro + c0 + c, &gh[c]);
+              load4(ea.gate + ro + c0 + c, &gh[c]);
             }
           }
 #pragma unroll
@@ -744,14 +688,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int cc = c0 + c;
             float v[4] = {o[cc] * inv * gh[c], o[cc + 1] * inv * gh[c + 1], o[cc + 2] * inv * gh[c + 2],
                           o[cc + 3] * inv * gh[c + 3]};
-            if (DEC && da.out_lo) {  // o * g as a hi + lo pair of bf16 values
-              float lo[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) lo[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
-              store4((bf16*)da.out + ro + cc, v);
-              store4((bf16*)da.out_lo + ro + cc, lo);
-            } else if (DEC) {
-              store4((float*)da.out + ro + cc, v);
+            if (DEC) {  // o * g in fp16 for the output projection's fp16 product
+              *reinterpret_cast<uint2*>(static_cast<__half*>(da.out) + ro + cc) =
+                  make_uint2(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]));
             } else {
               store4((bf16*)ea.out + ro + cc, v);
               if (ea.out_lo) {  // the low part, for a backward pass that needs O beyond bf16
@@ -787,9 +726,10 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
   const int d = DEC ? da->d : ea->d;
   if (n_tiles == 0) return cudaSuccess;
   const long long rows = DEC ? da->key_rows : ea->rows;
-  if (DEC) {  // fp16 H, moved as 2-byte elements like bf16
-    if (!make_tmap_bf16(&mk, da->h, rows, d, d, HD, ROWS, swz)) return cudaErrorInvalidValue;
-    mq = mk;
+  if (DEC) {  // fp16 H and queries, moved as 2-byte elements like bf16
+    if (!make_tmap_bf16(&mk, da->h, rows, d, d, HD, ROWS, swz) ||
+        !make_tmap_bf16(&mq, da->q16, da->nk_rows, d, d, HD, ROWS, swz))
+      return cudaErrorInvalidValue;
     mv = mk;
   } else {
     const long long key_rows = ea->app ? ea->key_rows : rows;

@@ -354,6 +354,39 @@ __device__ __forceinline__ void epilogue(const GemmArgs& a, const GemmMaps& mp, 
     }
     return;
   }
+  if (!SIDE && a.epi == EPI_DECQG && a.out16) {
+    // the decoder's q (scaled by alpha) and sigmoid gate in fp16: this warp's 128
+    // columns of the 256-column tile as two 64-column fp16 boxes
+    const int per = f32_tiles(a.N), g = t / per, nt = t % per, k = g % a.k_tok;
+    const bool gate = g >= a.k_tok;
+    const int x0 = k * a.N + nt * 256, width = k * a.N + a.N;
+    bool in_range = true;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      tmem_ld32(trow + part * 128 + 32 * c, v);
+      if (c == 3) release();
+      if (gate) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = sigmoid_fast(v[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= a.alpha;
+      }
+      if (c == 0) slot_ready();
+      in_range = stage_f16_sw128(slot + (2 * part + (c >> 1)) * BOX128, r, 4 * (c & 1), v) && in_range;
+    }
+    if (!in_range) set_error(err, REST_ERR_RANGE);
+    issue();
+    if (lane == 0) {
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx) {
+        const int x = x0 + part * 128 + 64 * bx;
+        if (x < width) tma_store_2d(&mp.o[gate ? 1 : 0], slot + (2 * part + bx) * BOX128 + q * 32 * 128, x, y0);
+      }
+      bulk_commit();
+    }
+    return;
+  }
   // fp32 outputs (256-column tiles, this warp's 128 columns in four 32-column
   // chunks through two staging boxes): the output gate sigmoid(Go) (eq. 4),
   // plain, sigmoid, the decoder's q / gate, or the residual add
@@ -681,6 +714,9 @@ bool setup_maps(const GemmArgs& a, GemmMaps& mp) {
     case EPI_DT: return make_tmap(&mp.o[0], false, a.out0, a.M, a.N, a.ldo, 64, 32, 128);
     case EPI_DECQG: {
       const long long w = (long long)a.k_tok * a.N;
+      if (a.out16)  // fp16 q and gate, 64-column boxes
+        return make_tmap(&mp.o[0], false, a.out0, a.M, w, a.ldo, 64, 32, 128) &&
+               make_tmap(&mp.o[1], false, a.out1, a.M, w, a.ldo, 64, 32, 128);
       return make_tmap(&mp.o[0], true, a.out0, a.M, w, a.ldo, 32, 32, 128) &&
              make_tmap(&mp.o[1], true, a.out1, a.M, w, a.ldo, 32, 32, 128);
     }
@@ -743,7 +779,8 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long 
 
 bool sm100_gemm_supported(const GemmArgs& a) {
   if (a.a_f32) return false;
-  if (a.f16 && (a.A2 || a.out1 || (a.epi != EPI_SWIGLU && a.epi != EPI_RESID))) return false;
+  if (a.f16 && (a.A2 || a.out1 || (a.epi != EPI_SWIGLU && a.epi != EPI_RESID && a.epi != EPI_F32))) return false;
+  if (a.out16 && (a.f16 || a.epi != EPI_DECQG)) return false;
   if (a.M <= 0 || a.K % BK != 0 || a.K <= 0) return false;
   if ((a.lda % 8) || (a.ldb % 8) || (a.ldo % 8)) return false;
   switch (a.epi) {
