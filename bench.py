@@ -60,9 +60,9 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("dec_attn", "bf16-ragged64-d256"): (935722240, "attn", "044212b94c5e3b4b",
+    ("dec_attn", "bf16-ragged64-d256"): (519736064, "attn", "8828a32718c8a6a1",
                                          "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
-    ("enc_attn", "bf16-ragged64-d256"): (984920320, "attn", "044212b94c5e3b4b",
+    ("enc_attn", "bf16-ragged64-d256"): (994301440, "attn", "8828a32718c8a6a1",
                                          "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
 }
 

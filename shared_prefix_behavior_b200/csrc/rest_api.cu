@@ -869,8 +869,10 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
     flops += 4.0 * d * rows * reqs->req_cutoff[r];
     hbytes += (double)e * reqs->req_cutoff[r] * d * (h_lo ? 2 : 1);
   }
-  // q and g in, o * g out: fp16 each for the tensor-core decoder, fp32 for the CUDA-core one
-  const double bytes = hbytes + (double)p.NK * d * (tc ? 6 : 12);
+  // q and g in, o * g out: fp16 each for the tensor-core decoder, fp32 for the
+  // CUDA-core one; with split keys the tensor-core decoder reads q and writes
+  // one fp32 partial o per split, and the combine reads g
+  const double bytes = hbytes + (double)p.NK * d * (!tc ? 12 : p.n_split > 1 ? 2 + 4.0 * p.n_split : 6);
   // The tensor-core decoder hands o * g to the output projection in fp16, the
   // CUDA-core one in fp32.
   DecAttnArgs da;
@@ -891,7 +893,7 @@ static rest_status run_decoder(const Plan& p, const rest_requests* reqs, const v
     da.n_cta = std::min(L.n_dec_tiles * p.hs->n_heads, SCHED_CTAS);
     if (L.n_dec_tiles > 0) REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_sm100(hd, da, s, err));
     if (p.n_split > 1)
-      REST_KLAUNCH(s, "dec_combine", 0, (double)p.NK * d * 4 * (p.n_split + 2),
+      REST_KLAUNCH(s, "dec_combine", 0, (double)p.NK * d * (4.0 * p.n_split + 4),
                    launch_dec_combine(hd, da, s));
   } else {
     REST_KLAUNCH(s, "dec_attn", flops, bytes, launch_dec_attn_simt(bf, hd, da, s));
