@@ -627,9 +627,12 @@ def cpu_baseline(w: W.Workload, inp: dict, budget_s: float) -> dict:
         users.append(u)
         if t_tot >= budget_s:
             break
+    short = all(w.lengths[u] <= ORACLE_MAX_LEN for u in users)
+    rule = (f"skipping users of more than {ORACLE_MAX_LEN} tokens" if short
+            else f"no user has {ORACLE_MAX_LEN} tokens or fewer")
     out = {"value": c_tot / t_tot, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-           "sample": f"{len(users)} of {w.n_users} users of {w.name} in order, skipping users of more than "
-                     f"{ORACLE_MAX_LEN} tokens (encoder + all their candidates), fp64 numpy, {t_tot:.1f} s",
+           "sample": f"{len(users)} of {w.n_users} users of {w.name} in order, {rule} "
+                     f"(encoder + all their candidates), fp64 numpy, {t_tot:.1f} s",
            "encoder_tokens_per_s": tok_tot / t_tot}
     # the oracle without the shared prefix: candidates of user 0, each re-encoding
     # its request's prefix, one at a time until a quarter of the budget is spent

@@ -6,9 +6,9 @@
 // every staged key block (so each K/V (or H) tile crosses to shared memory
 // once per 256 query rows), with one softmax warpgroup per tile:
 //   warp 0       TMA producer. Encoder: Q tiles once, then K and V' per
-//                128-key block. Decoder: H (and H_lo) per block; one H tile
-//                is both the keys (K-major operand of S = q H^T) and the
-//                values (N-major operand of O = P H).
+//                128-key block. Decoder: the fp16 q tiles, then H per block;
+//                one H tile is both the keys (K-major operand of S = q H^T)
+//                and the values (N-major operand of O = P H).
 //   warps 1, 2   MMA issuers of tiles 0 and 1 (warp 1 also owns TMEM): per
 //                block j, S_t(j) = Q_t K_j^T into the tile's 128-column TMEM
 //                buffer as soon as its softmax has read S_t(j-1), then
@@ -34,10 +34,11 @@
 //                the exponentials block by block. The encoder's output rows go
 //                out through a per-warp staging area in shared memory.
 // The decoder multiplies in fp16 (kind::f16 with fp16 operands, fp32
-// accumulation): H comes as an fp16 copy, the fp32 query is staged in fp16
-// (scaled by log2(e) / sqrt(head_dim) first, so S is in the base-2 domain), and
-// P is written as fp16 pairs. fp16's 11-bit significand rounds q, H and P 8
-// times finer than bf16; a query value beyond fp16's range sets REST_ERR_RANGE.
+// accumulation): H comes as an fp16 copy, the query as the fp16 rows the
+// projection wrote (scaled by log2(e) / sqrt(head_dim) there, so S is in the
+// base-2 domain), and P is written as fp16 pairs; o * g goes out in fp16.
+// fp16's 11-bit significand rounds q, H and P 8 times finer than bf16; the
+// producers of H and q report values beyond fp16's range (REST_ERR_RANGE).
 //
 // MODE 0: encoder; 1: decoder; 3: encoder over a range of key blocks
 // (appending with split keys), writing partials.

@@ -1,5 +1,6 @@
 // tcgen05 GEMM for sm_100a with the fused epilogues of the ReST encoder and
-// decoder (bf16 operands, fp32 accumulation in TMEM).
+// decoder (bf16 operands, or fp16 for the decoder's output projection and the
+// score head; fp32 accumulation in TMEM).
 //
 // CTA pairs (clusters of two CTAs on two SMs) walk tiles of 256 rows of C =
 // A . B; each pair tile is one M=256 tcgen05 MMA chain issued by rank 0, with

@@ -280,9 +280,9 @@ def test_full_workload_single_layer_sampled_rows(cuda, cfg):
 def _end_to_end_users(w, cfg):
     """Users whose whole forward the oracle runs: on the 16k workload one of
     its two users; on the ragged one the shortest user, the first user whose
-    every request is under 1024 keys (the decoder reads H_hi + H_lo there),
-    the first user with requests on both sides of 1024 keys, and the first
-    user of 4096-6144 tokens (H_hi alone)."""
+    every request is under 1024 keys (short prefixes average H's fp16
+    rounding least), the first user with requests on both sides of 1024
+    keys, and the first user of 4096-6144 tokens."""
     if cfg == 3:
         return [0]
     L = np.asarray(w.lengths)
@@ -299,10 +299,11 @@ def test_full_workload_single_layer_end_to_end(cuda, cfg):
     """The one-layer workloads at full size through rank_request, y included:
     the GPU runs the whole batch; the oracle encodes the sampled users in full
     and scores every candidate of their requests. This checks the product's
-    decoder on real encoder output, where requests under 1024 keys read H as
-    H_hi + H_lo and longer ones H_hi alone (each request is also held to the
-    bar on its own). The passage: scoring with a request's prefix of the
-    union history equals scoring that prefix alone (§3.5)."""
+    decoder on real encoder output: the fp16 copy of H that the encoder
+    writes from its fp32 residual stream, at every cutoff length (each
+    request is also held to the bar on its own). The passage: scoring with a
+    request's prefix of the union history equals scoring that prefix alone
+    (§3.5)."""
     w = W.workload(cfg)
     inp = W.make_inputs(w, 1000 + cfg)
     H, y = run_rank(inp, cuda)
