@@ -99,7 +99,7 @@ static rest_status check_dec(const rest_dec_params* dec) {
 // Query rows per work item: 128 for the CUDA-core attention, the
 // tensor-core kernel's own size (two 128-row tiles) otherwise.
 static int attn_tile_rows(rest_dtype dt, int head_dim) {
-  return (dt == REST_BF16 && sm100_attn_supported(head_dim)) ? sm100_attn_tile_rows() : 128;
+  return (dt == REST_BF16 && sm100_attn_supported(head_dim)) ? sm100_attn_tile_rows(head_dim) : 128;
 }
 
 static void build_enc_tiles(const rest_batch* b, int rows, std::vector<EncTile>& t) {

@@ -21,7 +21,7 @@ cudaError_t launch_gemm_sm100(const GemmArgs& a, cudaStream_t s, int32_t* err);
 // True when the tensor-core attention kernels handle this head_dim.
 bool sm100_attn_supported(int head_dim);
 // Query rows per work item of the tensor-core attention kernels.
-int sm100_attn_tile_rows();
+int sm100_attn_tile_rows(int head_dim);
 cudaError_t launch_enc_attn_sm100(int head_dim, const EncAttnArgs& a, cudaStream_t s, int32_t* err);
 cudaError_t launch_dec_attn_sm100(int head_dim, const DecAttnArgs& a, cudaStream_t s, int32_t* err);
 // Backward of the causal attention core (head_dim 32 or 64): dq (zeroed by the

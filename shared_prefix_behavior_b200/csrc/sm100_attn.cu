@@ -54,25 +54,47 @@ namespace {
 using namespace sm100;
 
 constexpr int ROWS = 128;  // query rows per tile
-constexpr int NT = 2;      // tiles per CTA
-constexpr int KB = 128;    // keys per block
-constexpr int NTHREADS = 384;
+constexpr int HKB = 128;   // keys per block in the host's work items (their kb0, kb1)
+constexpr int MAXNT = 3;   // most tiles per work item
 constexpr int ITEM_CACHE = 64;  // work items per CTA decoded into shared memory up front
 constexpr float RESCALE_LOG2 = 8.0f;  // rescale O when the row max grows by more than 2^8
+
+// The shape of a CTA by head size. head_dim 64: two query tiles, 128-key blocks,
+// 384 threads. head_dim 32: three query tiles and 64-key blocks (S, P and O of a
+// tile then take 64 + 32 + 32 TMEM columns, 384 for the three), 512 threads, so
+// that three softmax warps share each SM sub-partition's special-function unit
+// where two did.
+template <int HD>
+struct Geo {
+  static constexpr int NT = HD <= 32 ? 3 : 2;     // query tiles per work item
+  static constexpr int KB = HD <= 32 ? 64 : 128;  // keys per block
+  static constexpr int NTHREADS = 128 * (NT + 1);
+  // registers per thread after setmaxnreg: warps 0-3, then the softmax warpgroups
+  // (4 x 32 x REG_CTRL + NT x 128 x REG_SOFT stays within the 65,536 of the SM)
+  static constexpr int REG_CTRL = HD <= 32 ? 56 : 72;
+  static constexpr int REG_SOFT = HD <= 32 ? 152 : 216;
+  static_assert(4 * 32 * REG_CTRL + NT * 128 * REG_SOFT <= 65536, "register split");
+  static_assert(NT <= MAXNT && HKB % KB == 0, "tile shape");
+};
 
 template <int HD>
 struct Cfg {
   static constexpr int ROW_BYTES = HD * 2;             // one bf16 row of a head slice
-  static constexpr int TILE_BYTES = ROWS * ROW_BYTES;  // 128 rows
+  static constexpr int TILE_BYTES = ROWS * ROW_BYTES;  // a query tile: 128 rows
+  static constexpr int KV_TILE_BYTES = Geo<HD>::KB * ROW_BYTES;  // a key block
   static constexpr int SWZ = HD == 64 ? 2 : 4;         // descriptor code: 128B / 64B swizzle
   static constexpr int ATOM = 8 * ROW_BYTES;           // bytes of 8 swizzled rows
 };
-// TMEM columns: S_0 | S_1 | O_0 | O_1 | P_0 | P_1 (P: 128 bf16 keys packed in 64 columns)
-__device__ __forceinline__ uint32_t s_col(int t) { return (uint32_t)(t * 128); }
+// TMEM columns: S_0 .. S_{NT-1} (KB each) | O_0 .. (HD each) | P_0 .. (KB bf16
+// keys packed in KB / 2 columns each)
 template <int HD>
-__device__ __forceinline__ uint32_t o_col(int t) { return (uint32_t)(256 + t * HD); }
+__device__ __forceinline__ uint32_t s_col(int t) { return (uint32_t)(t * Geo<HD>::KB); }
 template <int HD>
-__device__ __forceinline__ uint32_t p_col(int t) { return (uint32_t)(256 + NT * HD + t * 64); }
+__device__ __forceinline__ uint32_t o_col(int t) { return (uint32_t)(Geo<HD>::NT * Geo<HD>::KB + t * HD); }
+template <int HD>
+__device__ __forceinline__ uint32_t p_col(int t) {
+  return (uint32_t)(Geo<HD>::NT * (Geo<HD>::KB + HD) + t * (Geo<HD>::KB / 2));
+}
 
 // byte offset of 16-byte chunk u of row r in a swizzled [128 x HD] bf16 tile
 template <int HD>
@@ -83,12 +105,12 @@ __device__ __forceinline__ uint32_t swz_off(int r, int u) {
 
 template <int HD, int MODE>
 struct SmemLayout {
-  // [Q_0 | Q_1 | KV stages], 1024-aligned blocks
-  static constexpr int STAGES = 3;
+  // [Q_0 .. Q_{NT-1} | KV stages], 1024-aligned blocks
+  static constexpr int STAGES = HD <= 32 ? 6 : 3;
   static constexpr int Q = 0;
-  static constexpr int KV = NT * Cfg<HD>::TILE_BYTES;
+  static constexpr int KV = Geo<HD>::NT * Cfg<HD>::TILE_BYTES;
   // a stage holds K and V' (encoder) or H (decoder)
-  static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::TILE_BYTES;
+  static constexpr int STAGE = (MODE == 1 ? 1 : 2) * Cfg<HD>::KV_TILE_BYTES;
   // per softmax warp, its 32 output rows in 2-byte values (rows padded by 16
   // bytes): the encoder's O (bf16) or the decoder's o * g (fp16)
   static constexpr bool DEC = MODE == 1;
@@ -99,8 +121,9 @@ struct SmemLayout {
   // fetched ahead by cp.async, rows padded by 16 bytes
   static constexpr bool PREFETCH = HD <= 32 && MODE != 3;
   static constexpr int PF_ROW = HD * (DEC ? 2 : 4) + 16;
-  static constexpr int PF = STG + (STAGED_OUT ? 8 * 32 * STG_ROW : 0);
-  static constexpr int TOTAL = PF + (PREFETCH ? 256 * PF_ROW : 0);
+  static constexpr int PF = STG + (STAGED_OUT ? Geo<HD>::NT * 4 * 32 * STG_ROW : 0);
+  static constexpr int TOTAL = PF + (PREFETCH ? Geo<HD>::NT * ROWS * PF_ROW : 0);
+  static_assert(KV % 1024 == 0 && STAGE % 1024 == 0, "1024-aligned tiles");
 };
 
 // Asynchronous 16-byte copies global -> shared memory (no TMA): a thread
@@ -162,15 +185,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-__device__ __forceinline__ void setmaxnreg_dec72() { asm volatile("setmaxnreg.dec.sync.aligned.u32 72;"); }
-__device__ __forceinline__ void setmaxnreg_inc216() { asm volatile("setmaxnreg.inc.sync.aligned.u32 216;"); }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 
-// One work item: 256 query rows (two 128-row tiles) of one head.
+// One work item: NT x 128 query rows (NT 128-row tiles) of one head.
+template <int NT>
 struct AttnItem {
   int q_row0;     // packed row of query row 0 of tile 0
   int key_row0;   // packed row of the item's first key
   int nrow[NT];   // valid query rows of each tile
-  int nblk[NT];   // key blocks each tile reads
+  int nblk[NT];   // key blocks (of the kernel's KB keys) each tile reads
   int user_len;   // encoder: keys of the user's history (cached and new rows)
   int q_pos0;     // encoder: position of query row 0 within the user's history
   int nkeys;      // keys from key_row0 visible to the item (decoder: cutoff minus the split start)
@@ -179,24 +205,30 @@ struct AttnItem {
   int h;          // head
 };
 
-template <bool DEC, bool SPLITK>
-__device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const DecAttnArgs& da, int item) {
-  AttnItem w;
+// The host's items count keys in blocks of HKB (128); the kernel walks them in
+// blocks of KB (64 at head_dim 32, 128 at 64).
+template <int HD, bool DEC, bool SPLITK>
+__device__ __forceinline__ AttnItem<Geo<HD>::NT> decode_item(const EncAttnArgs& ea, const DecAttnArgs& da, int item) {
+  constexpr int NT = Geo<HD>::NT, KB = Geo<HD>::KB;
+  AttnItem<NT> w;
   const int n_heads = DEC ? da.n_heads : ea.n_heads;
   const int tile = item / n_heads;
   w.h = item % n_heads;
   if (DEC) {
     const DecTile t = da.tiles[tile];
     w.q_row0 = t.row0;
-    w.key_row0 = t.key0 + t.kb0 * KB;  // this item's keys: blocks kb0 .. kb1-1
-    w.nkeys = t.nkeys - t.kb0 * KB;
+    w.key_row0 = t.key0 + t.kb0 * HKB;  // this item's keys: host blocks kb0 .. kb1-1
+    w.nkeys = t.nkeys - t.kb0 * HKB;
     w.user_len = 0;
     w.q_pos0 = 0;
     w.split = t.split;
     w.key_off = 0;
+    // key blocks of the item's range (with KB = HKB, its host blocks)
+    const int nk = min(t.nkeys, t.kb1 * HKB) - t.kb0 * HKB;
+    const int nbk = KB == HKB ? t.kb1 - t.kb0 : nk > 0 ? (nk + KB - 1) / KB : 0;
     for (int i = 0; i < NT; ++i) {
       w.nrow[i] = max(0, min(ROWS, t.nrows - i * ROWS));
-      w.nblk[i] = w.nrow[i] > 0 ? t.kb1 - t.kb0 : 0;
+      w.nblk[i] = w.nrow[i] > 0 ? nbk : 0;
     }
   } else {
     const EncTile t = ea.tiles[tile];
@@ -210,18 +242,27 @@ __device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const Dec
     w.q_row0 = s + t.q0;
     w.nkeys = 0;
     w.split = SPLITK ? t.split : 0;
-    // split keys: blocks [kb0, kb1) of the user's keys only
-    const int kb0 = SPLITK ? t.kb0 : 0;
+    // split keys: host blocks [kb0, kb1) of the user's keys only
+    const int kb0 = SPLITK ? t.kb0 * (HKB / KB) : 0;
     w.key_off = kb0 * KB;
     w.key_row0 += w.key_off;
     for (int i = 0; i < NT; ++i) {
       const int r0 = t.q0 + i * ROWS;
       w.nrow[i] = max(0, min(ROWS, n - r0));
       const int nb = (min(w.user_len, off + r0 + ROWS) + KB - 1) / KB;
-      w.nblk[i] = w.nrow[i] > 0 ? (SPLITK ? max(0, min(nb, t.kb1) - kb0) : nb) : 0;
+      w.nblk[i] = w.nrow[i] > 0 ? (SPLITK ? max(0, min(nb, t.kb1 * (HKB / KB)) - kb0) : nb) : 0;
     }
   }
   return w;
+}
+
+// key blocks of the item's longest tile (the blocks the producer loads)
+template <int NT>
+__device__ __forceinline__ int max_blocks(const AttnItem<NT>& w) {
+  int m = 0;
+#pragma unroll
+  for (int i = 0; i < NT; ++i) m = max(m, w.nblk[i]);
+  return m;
 }
 
 // Persistent: one CTA per SM walks its own list of work items (a
@@ -230,10 +271,11 @@ __device__ __forceinline__ AttnItem decode_item(const EncAttnArgs& ea, const Dec
 // across items; every role keeps, per tile, the count of key blocks (cb) and of
 // items with work (qn) processed so far, from which all barrier parities follow.
 template <int HD, int MODE>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(Geo<HD>::NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, EncAttnArgs ea, DecAttnArgs da, int32_t* err) {
   constexpr bool DEC = MODE == 1, ESPLIT = MODE == 3;
+  constexpr int NT = Geo<HD>::NT, KB = Geo<HD>::KB;
   // head_dim 64: the two tiles' softmax warps of a lane quarter take turns at the
   // exponentials block by block (see the softmax); at 32 they do not.
   constexpr bool TURNS = HD >= 64;
@@ -251,7 +293,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // exponentials of its n-th key block (two barriers per pair so that a warp one
   // or two blocks ahead never completes the phase its partner still waits for)
   __shared__ uint64_t xe[NT][4][2];
-  __shared__ AttnItem s_items[HD <= 32 ? ITEM_CACHE : 1];
+  __shared__ AttnItem<NT> s_items[HD <= 32 ? ITEM_CACHE : 1];
   __shared__ uint32_t tslot;
   __shared__ volatile int abort_flag;
 
@@ -301,25 +343,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int k_first = sched[blockIdx.x];
   if (CACHE_ITEMS && warp == 3) {
     const int n = min(sched[blockIdx.x + 1] - k_first, ITEM_CACHE);
-    for (int i = lane; i < n; i += 32) s_items[i] = decode_item<DEC, ESPLIT>(ea, da, items[k_first + i]);
+    for (int i = lane; i < n; i += 32) s_items[i] = decode_item<HD, DEC, ESPLIT>(ea, da, items[k_first + i]);
   }
   __syncthreads();
-  auto item_at = [&](int k) -> AttnItem {
-    return CACHE_ITEMS && k - k_first < ITEM_CACHE ? s_items[k - k_first] : decode_item<DEC, ESPLIT>(ea, da, items[k]);
+  auto item_at = [&](int k) -> AttnItem<NT> {
+    return CACHE_ITEMS && k - k_first < ITEM_CACHE ? s_items[k - k_first]
+                                                   : decode_item<HD, DEC, ESPLIT>(ea, da, items[k]);
   };
 
   if (warp < 4) {
-    setmaxnreg_dec72();
+    setmaxnreg_dec<Geo<HD>::REG_CTRL>();
     // Warp 0, lane 0 loads (the other lanes of warp 0 have no role and wait at
-    // the end); warps 1 and 2 issue the MMAs of tiles 0 and 1 (warp 3 has no
-    // role after the item table). The issuing warps run whole: their
-    // elect.sync needs every lane.
+    // the end); warps 1 .. NT issue the MMAs of tiles 0 .. NT-1 (with two tiles,
+    // warp 3 has no role after the item table). The issuing warps run whole:
+    // their elect.sync needs every lane.
     if (warp == 0 && lane == 0) {
       // -------------------------------------------------------- TMA producer
-      int g = 0, issued = 0, qn[NT] = {0, 0};
+      int g = 0, issued = 0, qn[NT] = {};
       bool ok = true;
       for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-        const AttnItem w = item_at(k);
+        const AttnItem<NT> w = item_at(k);
         // the query tiles (decoding: fp16, scaled to the base-2 domain by the projection)
         for (int t = 0; t < NT && ok; ++t) {
           if (w.nblk[t] == 0) continue;
@@ -328,14 +371,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_2d(smem + L::Q + t * C::TILE_BYTES, &tmQ, w.h * HD, w.q_row0 + t * ROWS, &q_full[t]);
           ++qn[t];
         }
-        const int nblk_all = max(w.nblk[0], w.nblk[1]);
+        const int nblk_all = max_blocks<NT>(w);
         for (int j = 0; j < nblk_all && ok; ++j, ++g) {
           const int st = g % STAGES;
           if (!mbar_wait(&kv_empty[st], ((g / STAGES) & 1) ^ 1, err, &abort_flag)) { ok = false; break; }
           uint8_t* base = smem + L::KV + st * L::STAGE;
           mbar_arrive_expect_tx(&kv_full[st], L::STAGE);
           tma_load_2d(base, &tmK, w.h * HD, w.key_row0 + j * KB, &kv_full[st]);
-          if (MODE != 1) tma_load_2d(base + C::TILE_BYTES, &tmV, w.h * HD, w.key_row0 + j * KB, &kv_full[st]);
+          if (MODE != 1) tma_load_2d(base + C::KV_TILE_BYTES, &tmV, w.h * HD, w.key_row0 + j * KB, &kv_full[st]);
           issued = g + 1;
         }
       }
@@ -346,32 +389,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
           mbar_wait(&kv_full[i % STAGES], (i / STAGES) & 1, nullptr, &no_abort);
       }
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp >= 1 && warp <= NT) {
       // -------------------------------------------------------- MMA issuers
-      // Warp 1 for tile 0, warp 2 for tile 1: S_t(j) = Q_t K_j^T into the tile's S
+      // Warp 1 + t for tile t: S_t(j) = Q_t K_j^T into the tile's S
       // buffer as soon as its softmax has loaded S_t(j-1) (s_free), then
       // O_t += P_t(j-1) V_{j-1} once P_t(j-1) is written (p_full). A warp issues one
       // tcgen05.mma about every hundred cycles whatever its size (measured), so
       // each tile has its own issuing warp, which also keeps one tile's softmax
       // from waiting on the other's. The whole warp runs the loop and one elected
-      // lane issues. A block's K/V stage is released when both issuers have
-      // committed it (kv_empty counts two arrivals); a tile with fewer blocks in
+      // lane issues. A block's K/V stage is released when every issuer has
+      // committed it (kv_empty counts NT arrivals); a tile with fewer blocks in
       // the item still waits for each remaining block to land before releasing
       // it, so neither issuer can arrive for a later use of a stage before the
       // earlier use has completed.
       const int t = warp - 1;
       // the decoder's operands are fp16, the encoder's bf16
-      constexpr uint32_t idS = DEC ? idesc_f16(KB, 0) : idesc_bf16(KB, 0);  // N = 128 keys, B (keys) K-major
+      constexpr uint32_t idS = DEC ? idesc_f16(KB, 0) : idesc_bf16(KB, 0);  // N = KB keys, B (keys) K-major
       constexpr uint32_t idO = DEC ? idesc_f16(HD, 1) : idesc_bf16(HD, 1);  // N = head_dim, B (values) N-major
       constexpr uint32_t V_STEP = (2 * C::ATOM) >> 4;  // 16 keys of V: two 8-row atoms
-      const uint32_t tS = tmem + s_col(t), tO = tmem + o_col<HD>(t), tP = tmem + p_col<HD>(t);
+      const uint32_t tS = tmem + s_col<HD>(t), tO = tmem + o_col<HD>(t), tP = tmem + p_col<HD>(t);
       // Descriptors step along K: 16 elements are 32 bytes, 2 in the 16-byte address field.
       const uint64_t qd = smem_desc(smem_u32(smem + L::Q + t * C::TILE_BYTES), 16, C::ATOM, C::SWZ);
       int g = 0, cb = 0, qn = 0;
       bool ok = true;
       for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-        const AttnItem w = item_at(k);
-        const int nblk_all = max(w.nblk[0], w.nblk[1]);
+        const AttnItem<NT> w = item_at(k);
+        const int nblk_all = max_blocks<NT>(w);
         const int nb = w.nblk[t];
         if (nb > 0) ok = mbar_wait(&q_full[t], qn & 1, err, &abort_flag);
         tc_fence_after();
@@ -395,7 +438,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               if (!mbar_wait(&o_empty[t], (qn - 1) & 1, err, &abort_flag)) { ok = false; break; }
               tc_fence_after();
             }
-            const uint64_t vd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE + (DEC ? 0 : C::TILE_BYTES)),
+            const uint64_t vd = smem_desc(smem_u32(smem + L::KV + st * L::STAGE + (DEC ? 0 : C::KV_TILE_BYTES)),
                                           64 * KB * 2, C::ATOM, C::SWZ);
             // A = P_t from TMEM, 8 columns per K step of 16
   #pragma unroll
@@ -422,7 +465,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_wait(&drain, 0, nullptr, &no_abort);
     }
   } else {
-    setmaxnreg_inc216();
+    setmaxnreg_inc<Geo<HD>::REG_SOFT>();
     // -------------------------------------------------------------- softmax
     const int t = (warp - 4) >> 2;               // tile of this warpgroup
     const int q4 = warp & 3;                     // TMEM lane quarter
@@ -430,7 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     // the decoder's scores arrive in the base-2 domain (its query is staged pre-scaled)
     const float sl2 = DEC ? 1.0f : ea.scale_log2;
-    const uint32_t tS = tmem + lane_off + s_col(t);
+    const uint32_t tS = tmem + lane_off + s_col<HD>(t);
     const uint32_t tO = tmem + lane_off + o_col<HD>(t);
     const uint32_t tP = tmem + lane_off + p_col<HD>(t);
     const bool split = DEC ? da.n_split > 1 : ESPLIT;
@@ -444,7 +487,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr int GATE_ES = DEC ? 2 : 4;  // the gate's element size: fp16 decoding, fp32 encoding
     bool ok = true;
     for (int k = sched[blockIdx.x]; k < sched[blockIdx.x + 1] && ok; ++k) {
-      const AttnItem w = item_at(k);
+      const AttnItem<NT> w = item_at(k);
       const int nb = w.nblk[t];
       const bool valid = r < w.nrow[t];
       const long long row_g = (long long)(w.q_row0 + t * ROWS + r);
@@ -459,7 +502,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           pml[0] = -INFINITY;
           pml[1] = 0.f;
         }
-        cbo += w.nblk[1 - t];
+        if constexpr (TURNS) cbo += w.nblk[1 - t];
         continue;
       }
       const long long ro = row_g * d + h * HD;
@@ -472,7 +515,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         cp_async_commit();
       }
-      // visible keys: index < row_lim - 128 j (the causal bound and the user end / cutoff)
+      // visible keys: index < row_lim - KB j (the causal bound and the user end / cutoff)
       const int row_lim = DEC ? w.nkeys : min(w.q_pos0 + t * ROWS + r + 1, w.user_len) - (ESPLIT ? w.key_off : 0);
       float m_ref = -INFINITY;  // reference max (scaled, log2 domain) of P and O
       float l_run = 0.f;        // sum of exponentials relative to m_ref
@@ -482,14 +525,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         float s[KB];
         {
-          uint32_t raw[4][32];
+          uint32_t raw[KB / 32][32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, raw[c]);
+          for (int c = 0; c < KB / 32; ++c) tmem_ld32_async(tS + 32 * c, raw[c]);
           tmem_wait_ld();
           tc_fence_before();
           mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next block's scores
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < KB / 32; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[c][i]);
         }
@@ -539,7 +582,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // special-function unit: they take turns at the exponentials, block by block
         // (tile 0's block j, tile 1's block j, tile 0's block j + 1, ...), so each
         // one's loads, maxima and waits overlap the other's exponentials.
-        if (TURNS) {
+        if constexpr (TURNS) {
           const int oj = t == 0 ? j - 1 : j;  // the other tile's block that goes first
           if (oj >= 0 && oj < w.nblk[1 - t]) {
             const int n = cbo + oj;
@@ -550,7 +593,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m_ref, -m_ref);
         // P as bf16 (decoder: fp16) pairs, keys 2c, 2c+1 in column c, stored into the
         // tile's P columns of TMEM once the previous P V has completed
-        uint32_t pk[64];
+        uint32_t pk[KB / 2];
         // head_dim 32: the pairs c with bit c % 8 of POLY_PAIRS set (one in eight)
         // are exponentiated on the FMA pipe, so the two tiles' warps, which
         // exponentiate at the same time, queue less on the special-function unit
@@ -560,7 +603,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // whatever rows share its warp (appending equals re-encoding bit for bit).
         constexpr unsigned POLY_PAIRS = HD <= 32 ? 0x80u : 0u;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < KB / 2; ++c) {
           const int e = 2 * c;
           const float2 x = ffma2(make_float2(s[e], s[e + 1]), scale2, neg_m2);
           const float2 p = (POLY_PAIRS >> (c & 7)) & 1u ? exp2_fma2(x)
@@ -568,7 +611,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           sum2[c & 1] = fadd2(sum2[c & 1], p);
           pk[c] = DEC ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
         }
-        if (TURNS) {
+        if constexpr (TURNS) {
           __syncwarp();
           if (lane == 0) mbar_arrive(&xe[t][q4][(cb + j) & 1]);
         }
@@ -576,8 +619,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait(&p_free[t], (gj - 1) & 1, err, &abort_flag)) { ok = false; break; }
           tc_fence_after();
         }
-        tmem_st32_async(tP, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32_async(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+#pragma unroll
+        for (int u = 0; u < KB / 64; ++u)
+          tmem_st32_async(tP + 32 * u, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * u]));
         l_run += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
         tmem_wait_st();
         tc_fence_before();
@@ -705,7 +749,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       cb += nb;
-      cbo += w.nblk[1 - t];
+      if constexpr (TURNS) cbo += w.nblk[1 - t];
       ++qn;
     }
     if (L::PREFETCH) cp_async_wait<0>();  // no copy into shared memory outlives the loop
@@ -721,6 +765,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 template <int HD, int MODE>
 cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream_t s, int32_t* err) {
   constexpr bool DEC = MODE == 1;
+  constexpr int KB = Geo<HD>::KB;
   const int swz = HD == 64 ? 128 : 64;
   CUtensorMap mq, mk, mv;
   const int n_tiles = DEC ? da->n_tiles : ea->n_tiles;
@@ -728,15 +773,15 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
   if (n_tiles == 0) return cudaSuccess;
   const long long rows = DEC ? da->key_rows : ea->rows;
   if (DEC) {  // fp16 H and queries, moved as 2-byte elements like bf16
-    if (!make_tmap_bf16(&mk, da->h, rows, d, d, HD, ROWS, swz) ||
+    if (!make_tmap_bf16(&mk, da->h, rows, d, d, HD, KB, swz) ||
         !make_tmap_bf16(&mq, da->q16, da->nk_rows, d, d, HD, ROWS, swz))
       return cudaErrorInvalidValue;
     mv = mk;
   } else {
     const long long key_rows = ea->app ? ea->key_rows : rows;
     if (!make_tmap_bf16(&mq, ea->q, rows, d, d, HD, ROWS, swz) ||
-        !make_tmap_bf16(&mk, ea->k, key_rows, d, d, HD, ROWS, swz) ||
-        !make_tmap_bf16(&mv, ea->v, key_rows, d, d, HD, ROWS, swz))
+        !make_tmap_bf16(&mk, ea->k, key_rows, d, d, HD, KB, swz) ||
+        !make_tmap_bf16(&mv, ea->v, key_rows, d, d, HD, KB, swz))
       return cudaErrorInvalidValue;
   }
   // at least 120 KB so that exactly one CTA (which takes all 512 TMEM columns) runs per SM
@@ -752,14 +797,15 @@ cudaError_t launch_attn(const EncAttnArgs* ea, const DecAttnArgs* da, cudaStream
   DecAttnArgs d0 = da ? *da : DecAttnArgs{};
   const int n_cta = DEC ? da->n_cta : ea->n_cta;
   if (n_cta <= 0) return cudaErrorInvalidValue;
-  if (cudaError_t e_ = launch_k(attn_tc_kernel<HD, MODE>, n_cta, NTHREADS, smem, s, mq, mk, mv, e0, d0, err)) return e_;
+  if (cudaError_t e_ = launch_k(attn_tc_kernel<HD, MODE>, n_cta, Geo<HD>::NTHREADS, smem, s, mq, mk, mv, e0, d0, err))
+    return e_;
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool sm100_attn_supported(int head_dim) { return head_dim == 32 || head_dim == 64; }
-int sm100_attn_tile_rows() { return NT * ROWS; }
+int sm100_attn_tile_rows(int head_dim) { return (head_dim <= 32 ? Geo<32>::NT : Geo<64>::NT) * ROWS; }
 
 cudaError_t launch_enc_attn_sm100(int hd, const EncAttnArgs& a, cudaStream_t s, int32_t* err) {
   if (a.n_split > 1)  // appending with split keys: partial results for launch_enc_combine

@@ -27,7 +27,7 @@ def test_digest_ignores_comments_and_blank_space_but_not_code(tmp_path, monkeypa
     text = f.read_text()
     f.write_text("// a new comment line\n/* and a block\n   comment */\n" + text.replace("\n", "\n\n", 3))
     assert bench.source_digest("attn") == base
-    f.write_text(text.replace("constexpr int KB = 128;", "constexpr int KB = 64;", 1))
+    f.write_text(text + "\nconstexpr int an_extra_constant = 64;\n")
     assert bench.source_digest("attn") != base
 
 
