@@ -33,14 +33,24 @@ __device__ __forceinline__ long long floor_div(long long rel, long long tau) {
   return q;
 }
 
-// sin and cos of idx * theta_j: the angle in turns is reduced modulo 1 from the
-// three 16-bit pieces of idx and the host's fractional turns of 2^(16 k) theta_j,
-// so the library routine only ever sees an argument in [-1, 1] half-turns.
-__device__ __forceinline__ void rotation(long long idx, const TableParams& p, int j, double* sv, double* cv) {
+// sin and cos of idx * theta_j: the angle in turns is reduced modulo 1 in fp64
+// from the three 16-bit pieces of idx and the host's fractional turns of
+// 2^(16 k) theta_j. The reduced turns r (|r| <= 1/2) split into an fp32 part
+// r_hi and a remainder r_lo (|r_lo| <= 2^-25); the library's fp32 sincospi of
+// 2 r_hi (exact) is corrected to first order in the remaining angle
+// d = 2 pi r_lo (|d| < 2e-7 rad, so the dropped d^2 / 2 term is below 2e-14):
+// sin(a + d) ~ sin a + d cos a, cos(a + d) ~ cos a - d sin a. The result is the
+// fp32 table value within about 1.5 ulp, without fp64 transcendental work.
+__device__ __forceinline__ void rotation(long long idx, const TableParams& p, int j, float* sv, float* cv) {
   const double h2 = (double)(idx >> 32), h1 = (double)((idx >> 16) & 0xffff), h0 = (double)(idx & 0xffff);
   double tr = fma(h2, p.turn[2][j], fma(h1, p.turn[1][j], h0 * p.turn[0][j]));
   tr -= rint(tr);
-  sincospi(2.0 * tr, sv, cv);
+  const float hi = (float)tr;
+  const float d = 6.28318530717958648f * (float)(tr - (double)hi);
+  float sa, ca;
+  sincospif(2.0f * hi, &sa, &ca);
+  *sv = fmaf(d, ca, sa);
+  *cv = fmaf(-d, sa, ca);
 }
 
 // A block takes TB = min(256 / half, 128) consecutive tokens. Its first threads find
@@ -94,11 +104,11 @@ __global__ void __launch_bounds__(ROT_THREADS)
   if (tk >= nt) return;
   const long long i = i0 + tk;
   for (int h = 0; h < H; ++h) {
-    double sv, cv;
+    float sv, cv;
     rotation(s_idx[tk][h], p, j, &sv, &cv);
     const long long o = (i * H + h) * p.half + j;
-    cos_out[o] = (float)cv;
-    sin_out[o] = (float)sv;
+    cos_out[o] = cv;
+    sin_out[o] = sv;
   }
 }
 
