@@ -594,14 +594,14 @@ __global__ void __launch_bounds__(Geo<HD>::NTHREADS, 1)
         // P as bf16 (decoder: fp16) pairs, keys 2c, 2c+1 in column c, stored into the
         // tile's P columns of TMEM once the previous P V has completed
         uint32_t pk[KB / 2];
-        // head_dim 32: the pairs c with bit c % 8 of POLY_PAIRS set (two in eight)
-        // are exponentiated on the FMA pipe, so the tiles' warps, which
-        // exponentiate at the same time, queue less on the special-function unit
-        // (measured on the ragged workload, decoder attention: none 1.45 ms, one
-        // pair in eight 1.39, two 1.36; the encoder's is the same at one or two).
+        // The pairs c with bit c % 8 of POLY_PAIRS set (two in eight) are
+        // exponentiated on the FMA pipe, so the softmax warps queue less on the
+        // special-function unit (measured, decoder attention: head_dim 32 on the
+        // ragged workload, none 1.45 ms, one pair in eight 1.39, two 1.36; head_dim
+        // 64 at 16k, none 0.155, one 0.152, two 0.151, three 0.161, four 0.166).
         // The choice follows the key's column alone, so a score gets the same P
         // whatever rows share its warp (appending equals re-encoding bit for bit).
-        constexpr unsigned POLY_PAIRS = HD <= 32 ? 0x88u : 0u;
+        constexpr unsigned POLY_PAIRS = 0x88u;
 #pragma unroll
         for (int c = 0; c < KB / 2; ++c) {
           const int e = 2 * c;
