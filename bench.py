@@ -60,9 +60,9 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("dec_attn", "bf16-ragged64-d256"): (522401536, "attn", "173dd506c35de6be",
+    ("dec_attn", "bf16-ragged64-d256"): (524781568, "attn", "28d4235658bed2db",
                                          "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
-    ("enc_attn", "bf16-ragged64-d256"): (905059840, "attn", "173dd506c35de6be",
+    ("enc_attn", "bf16-ragged64-d256"): (941727488, "attn", "28d4235658bed2db",
                                          "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
 }
 
