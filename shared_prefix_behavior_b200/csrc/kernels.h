@@ -38,6 +38,13 @@ cudaError_t launch_append_rows(const void* src0, void* dst0, const void* src1, v
                                const UserAppend* app, int n_users, long long T, int row_bytes, cudaStream_t s);
 
 // ---------------------------------------------------------------- casts / norms
+// The encoder's first launch, bf16 with d a multiple of 128 (up to 1024): the
+// rotation table (as launch_rotation_table, without idx_out), x_res = fp32(x),
+// and with y non-null y = bf16(LN(x)) with g, b (a pre-LN first sublayer's input).
+cudaError_t launch_table_cast_ln(const int64_t* ts, const int32_t* cu, int n_users, int T, const TableParams& p,
+                                 float* cos_out, float* sin_out, int32_t* err, const UserAppend* app,
+                                 const void* x, float* xres, void* y, const float* g, const float* b, int d,
+                                 cudaStream_t s);
 // mode 0: y = dt(LN(x))  (pre-LN input of a sublayer)
 // mode 1: x = LN(x); y = dt(x)  (post-LN after the residual add)
 // mode 2: y = dt(x)  (post-LN sublayer input, no norm)

@@ -686,9 +686,6 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   const double attn_bytes = Td * (e + 4 + e) + 2.0 * e * key_rows * d;  // Q, gate, out; K and V'
 
   TableParams tp = table_params(p.hs);
-  REST_KLAUNCH(s, "rotation_table", 0, 8.0 * T + 4 * Td,
-               launch_rotation_table(ts, cu, p.b->n_users, (int)T, tp, nullptr, cos_t, sin_t, err, s, app));
-  REST_KLAUNCH(s, "to_f32", 0, Td * (e + 4), launch_to_f32(bf, x, xres, T * d, s));
 
   EncAttnArgs ea;
   memset(&ea, 0, sizeof(ea));  // optional outputs (lse, out_lo) stay null
@@ -730,6 +727,21 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
     REST_KLAUNCH(s, "layernorm", 0, bytes, launch_layernorm(bf, xres, out, g, b, (int)T, d, mode, s, g2, b2));
     return REST_OK;
   };
+  // The rotation table, x into the fp32 residual stream and (pre-LN) the first
+  // sublayer's input: in bf16 one launch, whose table blocks (arithmetic-bound)
+  // and row blocks (HBM-bound) share the SMs; otherwise three.
+  const bool fuse_first = bf && d % 128 == 0 && d <= 1024;
+  const bool pre0 = !subs.empty() && !subs[0].post;
+  if (fuse_first) {
+    REST_KLAUNCH(s, "table_cast_ln", 0, 8.0 * T + 4 * Td + Td * (e + 4) + (pre0 ? Td * e : 0),
+                 launch_table_cast_ln(ts, cu, p.b->n_users, (int)T, tp, cos_t, sin_t, err, app, x, xres,
+                                      pre0 ? y : nullptr, pre0 ? subs[0].g : nullptr, pre0 ? subs[0].b : nullptr,
+                                      d, s));
+  } else {
+    REST_KLAUNCH(s, "rotation_table", 0, 8.0 * T + 4 * Td,
+                 launch_rotation_table(ts, cu, p.b->n_users, (int)T, tp, nullptr, cos_t, sin_t, err, s, app));
+    REST_KLAUNCH(s, "to_f32", 0, Td * (e + 4), launch_to_f32(bf, x, xres, T * d, s));
+  }
   // input of the first sublayer: with post-LN it reads x itself, which in bf16
   // is the call's input as it stands
   // (with no layers H is x)
@@ -738,8 +750,8 @@ static rest_status run_encoder(const Plan& p, const void* x, const int64_t* ts, 
   } else if (subs[0].post) {
     if (bf) a_in = x;
     else if (rest_status st = norm(y, nullptr, nullptr, 2, nullptr, nullptr)) return st;
-  } else if (rest_status st = norm(y, subs[0].g, subs[0].b, 0, nullptr, nullptr)) {
-    return st;
+  } else if (!fuse_first) {
+    if (rest_status st = norm(y, subs[0].g, subs[0].b, 0, nullptr, nullptr)) return st;
   }
   bool h_written = false;
   for (size_t i = 0; i < subs.size(); ++i) {

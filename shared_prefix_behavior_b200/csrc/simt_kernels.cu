@@ -62,22 +62,21 @@ __device__ __forceinline__ void rotation(long long idx, const TableParams& p, in
 // cached ones and time still counts from the history's first timestamp.
 constexpr int ROT_THREADS = 256;
 constexpr int ROT_MAX_HEADS = 32;  // TableParams::tau
-constexpr int ROT_TB_MAX = 128;    // tokens per block
+constexpr int ROT_TB_MAX = 32;     // tokens per block (256 / half from head_dim 16 on)
 
 __host__ __device__ __forceinline__ int rot_tokens_per_block(int half) {
   return ROT_THREADS / half < ROT_TB_MAX ? ROT_THREADS / half : ROT_TB_MAX;
 }
 
-__global__ void __launch_bounds__(ROT_THREADS)
-    rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu, int n_users, int T,
-                          TableParams p, int64_t* idx_out, float* cos_out, float* sin_out, int32_t* err,
-                          const UserAppend* __restrict__ app) {
+// The table's block `blk` (all threads of a block of ROT_THREADS take part).
+__device__ __forceinline__ void rotation_table_block(int blk, const int64_t* __restrict__ ts,
+                                                     const int32_t* __restrict__ cu, int n_users, int T,
+                                                     const TableParams& p, int64_t* idx_out, float* cos_out,
+                                                     float* sin_out, int32_t* err, const UserAppend* __restrict__ app) {
   __shared__ long long s_idx[ROT_TB_MAX][ROT_MAX_HEADS];
   __shared__ long long s_rel[ROT_TB_MAX], s_pos[ROT_TB_MAX];
-  pdl_wait();  // the previous kernel of the stream has completed
-  pdl_release();
   const int TB = rot_tokens_per_block(p.half);
-  const int i0 = blockIdx.x * TB;
+  const int i0 = blk * TB;
   const int nt = min(TB, T - i0);
   const int H = p.n_heads;
   for (int k = threadIdx.x; k < nt; k += blockDim.x) {  // per token: user, time since its first token, position
@@ -110,6 +109,15 @@ __global__ void __launch_bounds__(ROT_THREADS)
     cos_out[o] = cv;
     sin_out[o] = sv;
   }
+}
+
+__global__ void __launch_bounds__(ROT_THREADS)
+    rotation_table_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu, int n_users, int T,
+                          TableParams p, int64_t* idx_out, float* cos_out, float* sin_out, int32_t* err,
+                          const UserAppend* __restrict__ app) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  rotation_table_block(blockIdx.x, ts, cu, n_users, T, p, idx_out, cos_out, sin_out, err, app);
 }
 
 cudaError_t launch_rotation_table(const int64_t* ts, const int32_t* cu, int n_users, int T,
@@ -382,6 +390,89 @@ cudaError_t launch_layernorm(bool bf16m, float* x, void* y, const float* g, cons
   } else {
     if (cudaError_t e_ = launch_k(layernorm_narrow_kernel<float>, blocks, threads, 0, s, x, (float*)y, g, b, g2, b2, T, d, mode)) return e_;
   }
+  return cudaGetLastError();
+}
+
+// The encoder's first launch: the rotation table (blocks n_cast ..) and, in blocks
+// 0 .. n_cast - 1, the bf16 input into the fp32 residual stream with, for a
+// pre-LN first sublayer, that sublayer's input y = bf16(LN(x)). The table is
+// bound by its arithmetic and the rows by HBM, so the two kinds of block share
+// the SMs: the row blocks, few and grid-striding, take two of each SM's block
+// slots and the table's blocks the rest. A row's arithmetic is the LayerNorm
+// kernel's (mode 0) on the same values, bf16 -> fp32 being exact.
+template <int NV>
+__global__ void __launch_bounds__(ROT_THREADS)
+    table_cast_ln_kernel(const int64_t* __restrict__ ts, const int32_t* __restrict__ cu, int n_users, int T,
+                         TableParams p, float* cos_out, float* sin_out, int32_t* err,
+                         const UserAppend* __restrict__ app, const bf16* __restrict__ x, float* __restrict__ xres,
+                         bf16* __restrict__ y, const float* __restrict__ g, const float* __restrict__ b, int d,
+                         int n_cast) {
+  pdl_wait();  // the previous kernel of the stream has completed
+  pdl_release();
+  if ((int)blockIdx.x >= n_cast) {
+    rotation_table_block(blockIdx.x - n_cast, ts, cu, n_users, T, p, nullptr, cos_out, sin_out, err, app);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int n_warps = n_cast * (blockDim.x >> 5);
+  int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  float v[NV][4], nx[NV][4];
+  if (row < T) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) load4(x + (long long)row * d + 128 * k + 4 * lane, v[k]);
+  }
+  for (; row < T; row += n_warps) {  // the next row's loads in flight during this row's work
+    const int next = row + n_warps;
+    if (next < T) {
+#pragma unroll
+      for (int k = 0; k < NV; ++k) load4(x + (long long)next * d + 128 * k + 4 * lane, nx[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) store4(xres + (long long)row * d + 128 * k + 4 * lane, v[k]);
+    if (y) ln_row<bf16, NV>(nullptr, y + (long long)row * d, g, b, nullptr, nullptr, d, 0, lane, v);
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = nx[k][i];
+  }
+}
+
+cudaError_t launch_table_cast_ln(const int64_t* ts, const int32_t* cu, int n_users, int T, const TableParams& p,
+                                 float* cos_out, float* sin_out, int32_t* err, const UserAppend* app,
+                                 const void* x, float* xres, void* y, const float* g, const float* b, int d,
+                                 cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (p.half < 1 || p.half > 64 || p.n_heads < 1 || p.n_heads > ROT_MAX_HEADS) return cudaErrorInvalidValue;
+  if (d % 128 != 0 || d > 1024 || (y && (!g || !b))) return cudaErrorInvalidValue;
+  if (((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 7) != 0 ||
+      (reinterpret_cast<uintptr_t>(xres) & 15) != 0)
+    return cudaErrorInvalidValue;
+  static int n_sm = 0;
+  if (n_sm == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0)
+      n_sm = 148;
+  }
+  const long long rot_blocks = ((long long)T + rot_tokens_per_block(p.half) - 1) / rot_tokens_per_block(p.half);
+  const long long row_blocks = ((long long)T * 32 + ROT_THREADS - 1) / ROT_THREADS;
+  const int n_cast = (int)(row_blocks < 2LL * n_sm ? row_blocks : 2LL * n_sm);
+  const unsigned grid = (unsigned)(n_cast + rot_blocks);
+  const bf16* xb = static_cast<const bf16*>(x);
+  bf16* yb = static_cast<bf16*>(y);
+  cudaError_t e_ = cudaSuccess;
+  switch (d / 128) {
+    case 1: e_ = launch_k(table_cast_ln_kernel<1>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    case 2: e_ = launch_k(table_cast_ln_kernel<2>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    case 3: e_ = launch_k(table_cast_ln_kernel<3>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    case 4: e_ = launch_k(table_cast_ln_kernel<4>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    case 5: e_ = launch_k(table_cast_ln_kernel<5>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    case 6: e_ = launch_k(table_cast_ln_kernel<6>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    case 7: e_ = launch_k(table_cast_ln_kernel<7>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    case 8: e_ = launch_k(table_cast_ln_kernel<8>, grid, ROT_THREADS, 0, s, ts, cu, n_users, T, p, cos_out, sin_out, err, app, xb, xres, yb, g, b, d, n_cast); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e_ != cudaSuccess) return e_;
   return cudaGetLastError();
 }
 
