@@ -60,9 +60,9 @@ KERNEL_SOURCES = {
     "gemm": ("sm100_gemm.cu", "sm100_common.cuh", "common.cuh", "kernels.h"),
 }
 TRAFFIC = {  # (kernel, workload): (bytes per launch, sources, digest, summary)
-    ("dec_attn", "bf16-ragged64-d256"): (524781568, "attn", "28d4235658bed2db",
+    ("dec_attn", "bf16-ragged64-d256"): (522458880, "attn", "6fdb154546b94f5a",
                                          "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
-    ("enc_attn", "bf16-ragged64-d256"): (941727488, "attn", "28d4235658bed2db",
+    ("enc_attn", "bf16-ragged64-d256"): (905321472, "attn", "6fdb154546b94f5a",
                                          "profiles/attn_tc_kernel_bf16-ragged64-d256.md"),
 }
 
