@@ -621,7 +621,15 @@ __global__ void score_readout_kernel(const float* __restrict__ f, const float* _
   if (c >= n) return;
   const float* row = f + c * K * d;
   float acc = 0.f;
-  for (int i = lane; i < d; i += 32) acc = fmaf(row[i], w_s[i], acc);
+  if ((d & 127) == 0 && ((reinterpret_cast<uintptr_t>(f) | reinterpret_cast<uintptr_t>(w_s)) & 15) == 0) {
+    // 16 bytes a lane: a row's loads are in flight together
+    for (int i = 4 * lane; i < d; i += 128) {
+      const float4 a = *reinterpret_cast<const float4*>(row + i), w = *reinterpret_cast<const float4*>(w_s + i);
+      acc = fmaf(a.x, w.x, fmaf(a.y, w.y, fmaf(a.z, w.z, fmaf(a.w, w.w, acc))));
+    }
+  } else {
+    for (int i = lane; i < d; i += 32) acc = fmaf(row[i], w_s[i], acc);
+  }
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
   if (lane == 0) score[c] = acc + b_s;
