@@ -2,37 +2,40 @@
 // Attention of the ReST encoder (§3.2.1 eqs. 3-4) and the shared-prefix,
 // projection-free cross attention of the decoder (§3.3.1 eq. 7, §3.5).
 //
-// One CTA owns 256 query rows of one head as two 128-row tiles that share
-// every staged key block (so each K/V (or H) tile crosses to shared memory
-// once per 256 query rows), with one softmax warpgroup per tile:
-//   warp 0       TMA producer. Encoder: Q tiles once, then K and V' per
-//                128-key block. Decoder: the fp16 q tiles, then H per block;
-//                one H tile is both the keys (K-major operand of S = q H^T)
-//                and the values (N-major operand of O = P H).
-//   warps 1, 2   MMA issuers of tiles 0 and 1 (warp 1 also owns TMEM): per
-//                block j, S_t(j) = Q_t K_j^T into the tile's 128-column TMEM
-//                buffer as soon as its softmax has read S_t(j-1), then
+// One CTA owns NT x 128 query rows of one head as NT 128-row tiles that share
+// every staged key block (so each K/V (or H) block crosses to shared memory
+// once per NT x 128 query rows), with one softmax warpgroup per tile. NT = 2
+// with 128-key blocks at head_dim 64, NT = 3 with 64-key blocks at head_dim 32
+// (see Geo):
+//   warp 0       TMA producer. Encoder: Q tiles once, then K and V' per key
+//                block. Decoder: the fp16 q tiles, then H per block; one H
+//                tile is both the keys (K-major operand of S = q H^T) and the
+//                values (N-major operand of O = P H).
+//   warps 1..NT  MMA issuers of tiles 0..NT-1 (warp 1 also owns TMEM): per
+//                block j, S_t(j) = Q_t K_j^T into the tile's TMEM S buffer as
+//                soon as its softmax has read S_t(j-1), then
 //                O_t += P_t(j-1) V_{j-1} into the tile's head_dim-column
 //                accumulator once P_t(j-1) is written. A warp issues one
 //                tcgen05.mma about every hundred cycles whatever its size
 //                (measured), so each tile has its own issuing warp, running
 //                whole with one elected lane.
 //   warp 3       head_dim 32: first decodes the CTA's work items into a
-//                shared-memory table (a lane per item).
-//   warps 4..7   softmax of tile 0, warps 8..11 of tile 1: a thread owns a
-//                query row; it reads its row of S from TMEM, masks, keeps the
-//                running max, exponentiates in base 2, and writes P (bf16
-//                pairs) back to the tile's P columns of TMEM, from where the
-//                P V MMA takes its A operand; the exponentials are computed
-//                before the wait for the previous P V, which only their store
-//                needs. O stays in TMEM: when a row's max grows by more than
-//                2^8 the warp rescales its O rows in TMEM (after the previous
-//                P V has completed); otherwise P is taken relative to the old
-//                max (values up to 2^8, exact in fp32 accumulation). At
-//                head_dim 64 the two tiles' warps of a lane quarter, which
-//                share a sub-partition's special-function unit, take turns at
-//                the exponentials block by block. The encoder's output rows go
-//                out through a per-warp staging area in shared memory.
+//                shared-memory table (a lane per item), then issues tile 2.
+//   warps 4..    softmax, four warps per tile (warps 4..7 tile 0, 8..11 tile 1,
+//                12..15 tile 2): a thread owns a query row; it reads its row
+//                of S from TMEM, masks, keeps the running max, exponentiates in
+//                base 2, and writes P (bf16 pairs) back to the tile's P columns
+//                of TMEM, from where the P V MMA takes its A operand; the
+//                exponentials are computed before the wait for the previous
+//                P V, which only their store needs. O stays in TMEM: when a
+//                row's max grows by more than 2^8 the warp rescales its O rows
+//                in TMEM (after the previous P V has completed); otherwise P is
+//                taken relative to the old max (values up to 2^8, exact in fp32
+//                accumulation). At head_dim 64 the two tiles' warps of a lane
+//                quarter, which share a sub-partition's special-function unit,
+//                take turns at the exponentials block by block. The encoder's
+//                output rows go out through a per-warp staging area in shared
+//                memory.
 // The decoder multiplies in fp16 (kind::f16 with fp16 operands, fp32
 // accumulation): H comes as an fp16 copy, the query as the fp16 rows the
 // projection wrote (scaled by log2(e) / sqrt(head_dim) there, so S is in the
