@@ -97,7 +97,8 @@ static rest_status check_dec(const rest_dec_params* dec) {
 // ---------------------------------------------------------------- work lists
 
 // Query rows per work item: 128 for the CUDA-core attention, the
-// tensor-core kernel's own size (two 128-row tiles) otherwise.
+// tensor-core kernel's own size otherwise (three 128-row tiles at head_dim 32,
+// two at 64).
 static int attn_tile_rows(rest_dtype dt, int head_dim) {
   return (dt == REST_BF16 && sm100_attn_supported(head_dim)) ? sm100_attn_tile_rows(head_dim) : 128;
 }
